@@ -1,0 +1,32 @@
+"""CPU oracle for MHA2MLA conversion and latent-cache decode — TEST INFRASTRUCTURE ONLY.
+
+Plain float64 numpy (LAPACK SVD, BLAS matmul as library steps), written from the
+method's definitions and sharing no code with the CUDA path.  Only ``tests/``,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+it; the product library never calls it and has no CPU fallback.
+
+Every function cites the passage it follows.  Page short names:
+  NOTES  = "MHA2MLA: Towards Economical Inference by Enabling DeepSeek's Multi-Head
+           Latent Attention in Any Transformer-based LLMs" (paper notes, ACL 2025);
+           sections 方法详解/整体框架 (overall framework), 关键设计 (key designs:
+           contribution-aware partial-RoPE removal; joint SVD low-rank approximation
+           (SVDjoint); compatibility with KV-cache quantization), 实验关键数据 (tables).
+  ABSTRACT = arXiv record "Towards Economical Inference: Enabling DeepSeek's Multi-Head
+           Latent Attention in Any Transformer-based LLMs", abstract.
+  SUMMARY = "What is MHA2MLA" product page, §Technical principles.
+  README = GitHub README "MHA2MLA", §Fine-Tuning (strategy tables), §LongBench
+           Evaluation (quantized cache).
+
+Pinning status (see tests/test_oracle_pins.py):
+  pair_scores, select_pairs, split_dims, svd_joint, krope_weights, rotate, append,
+  decode_unabsorbed, decode_absorbed, mha_textbook_* — pinned by closed forms,
+  brute force, invariants and hand-derived fixtures.
+  quant_int4_g32 / dequant_int4_g32 — the scheme itself is a reading (the pages
+  name 4-bit quantization of the latent but not its encoding); the oracle's
+  implementation of that reading is pinned by its error bound, exact round trips and
+  hand-derived codes.
+  cache_bytes_per_token — pinned by the pages' printed reduction figures under a
+  stated reading of the unstated configuration.
+"""
+
+from .mha2mla import *  # noqa: F401,F403
