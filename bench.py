@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark of one MHA2MLA decode step over the latent KV cache.
+
+A step is the serving-loop decode step for one batch: `mla_append` writes each
+sequence's new token (latent c_kv + rotated RoPE key dims) at position L_b-1, then
+`mla_decode` attends each sequence's new query over its L_b cached tokens (query
+absorption, split-K latent attention, split merge + W_uv).  Metric: cached tokens per
+second, sum_b L_b / step time.  Pair selection and SVDjoint run once at conversion
+and are timed separately (`conversion_s`).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+        python bench.py --impl reference ...   (the float64 CPU oracle, timed on host cores)
+Multi-GPU (torchrun, one process per GPU): every rank runs an independent replica of
+the workload (the path has no cross-sequence exchange); value = tokens of all ranks /
+max-over-ranks time.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode cached tokens/s (batch×ctx per step) and % of B200 HBM peak"
+UNIT = "cached tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama2_7b_bf16")
+    ap.add_argument("--kernel", type=int, default=0, help="decode kernel: 0 auto, 1 CUDA-core, 2 tcgen05")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    return ap.parse_args()
+
+
+def workload(name):
+    from workloads import get
+    try:
+        return get(int(name))
+    except ValueError:
+        return get(name)
+
+
+def wl_config(wl, lens):
+    return {"workload": wl.name, "batch": wl.batch,
+            "ctx": wl.ctx if wl.ctx is not None else f"ragged U[{wl.ctx_range[0]},{wl.ctx_range[1]}]",
+            "cached_tokens_per_step": int(np.sum(lens)), "hidden": wl.hidden, "heads": wl.n_heads,
+            "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "r_pairs": wl.r_pairs, "d_c": wl.d_c,
+            "latent_cache": "int4 g32 + fp16 scales" if wl.cache == "int4_g32" else wl.dtype,
+            "step": "mla_append(B new tokens) + mla_decode(B queries)"}
+
+
+# ------------------------------------------------------------------ oracle (CPU) timing
+def oracle_decode_sample(wl, n_tokens, rounds, seconds_cap=None):
+    """Time the float64 oracle's decode (unabsorbed form) of sequence 0's query over its
+    first n_tokens cached tokens (all heads).  Weights come from the oracle's own
+    conversion of a reduced-hidden copy of the layer: the decode cost does not depend on
+    the hidden size (it reads the cache, W_uk and W_uv only)."""
+    import oracle as O
+    from workloads import generate as gen
+    small = wl.with_(hidden=min(wl.hidden, 512), t_cal=256)
+    w = gen.layer_weights(small)
+    qc, kc = gen.calib_activations(small, w)
+    conv = O.convert(w, qc, kc, small, cast=lambda a: gen.cast(a, small.dtype))
+    theta = O.rope_theta(wl.head_dim, wl.rope_base)
+    x = gen.context_tokens(small, 0, n_tokens)
+    c, kr = O.append(x, np.arange(n_tokens), conv["W_dkv"], conv["W_krope"], conv["pair_idx"], theta)
+    kr = gen.cast(kr, wl.dtype)
+    if wl.cache == "int4_g32":
+        codes, scales = O.quant_int4_g32(c)
+    else:
+        c = gen.cast(c, wl.dtype)
+    q = gen.decode_queries(small, w)[0]
+    times = []
+    t_start = time.perf_counter()
+    for _ in range(rounds):
+        t0 = time.perf_counter()
+        cc = O.dequant_int4_g32(codes, scales) if wl.cache == "int4_g32" else c
+        O.decode_unabsorbed(q, cc, kr, conv["W_uk"], conv["W_uv"], conv["pair_idx"], theta)
+        times.append(time.perf_counter() - t0)
+        if seconds_cap and time.perf_counter() - t_start > seconds_cap:
+            break
+    return times
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(int(i.get("num_threads", 1)) for i in threadpool_info()) or os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = workload(args.workload)
+    from workloads import generate as gen
+    lens = gen.seq_lens(wl)
+    # size each step so the whole warmup+steps run stays within about two minutes
+    probe_tokens = min(int(lens[0]), 512)
+    t = statistics.median(oracle_decode_sample(wl, probe_tokens, 3))
+    per_tok = t / probe_tokens
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n_tok = int(max(16, min(int(lens[0]), budget / per_tok)))
+    times = oracle_decode_sample(wl, n_tok, args.warmup + args.steps)
+    timed = times[args.warmup:] or times
+    step_s = statistics.mean(timed)
+    value = n_tok / step_s
+    sample = (f"oracle decode (float64, unabsorbed) of sequence 0's query over its first {n_tok} "
+              f"cached tokens, all {wl.n_heads} heads, per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": len(timed), "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded generators)", "config": wl_config(wl, lens),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU helpers
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peak_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s pool figure)"
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+
+    from mha_mla_latent_b200 import build
+    build.build()
+    import mha_mla_latent_b200 as mla
+    from mha_mla_latent_b200.cache import LatentCache, workspace
+    from mha_mla_latent_b200.convert import convert_layer, plan_from_converted
+    from workloads import generate as gen
+
+    wl = workload(args.workload)
+    dev = torch.device("cuda", local)
+    dt = gen.torch_dtype(wl.dtype)
+    cfg = mla.config_from_workload(wl)
+    lens = gen.seq_lens(wl)
+    B = wl.batch
+
+    # ---- conversion (once): GPU pair selection + device SVD
+    t0 = time.perf_counter()
+    w = gen.layer_weights(wl)
+    q_cal, k_cal = gen.calib_activations(wl, w)
+    conv = convert_layer(cfg, gen.to_torch(w["W_k"], wl.dtype, dev), gen.to_torch(w["W_v"], wl.dtype, dev),
+                         gen.to_torch(q_cal, wl.dtype, dev), gen.to_torch(k_cal, wl.dtype, dev))
+    plan = plan_from_converted(cfg, conv)
+    if args.kernel:
+        mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, args.kernel)
+    torch.cuda.synchronize()
+    conversion_s = time.perf_counter() - t0
+
+    # ---- caches: enough replicas that consecutive steps never hit L2 from the previous one
+    per_tok = mla.mla_cache_bytes_per_token(cfg)
+    cache_bytes = int(np.sum(lens)) * per_tok
+    n_rep = max(1, -(-2 * L2_BYTES // cache_bytes))
+    T_cap = int(lens.max())
+    caches = [LatentCache(cfg, B, T_cap, dev) for _ in range(n_rep)]
+    x_dec = gen.decode_tokens(wl)
+    t0 = time.perf_counter()
+    chunk = 16384
+    for b in range(B):
+        L = int(lens[b])
+        ctx = gen.context_tokens(wl, b, L - 1)
+        for s in range(0, L - 1, chunk):
+            e = min(L - 1, s + chunk)
+            xt = gen.to_torch(ctx[s:e], wl.dtype, dev)
+            mla.mla_append(plan, xt, torch.full((e - s,), b, dtype=torch.int32, device=dev),
+                           torch.arange(s, e, dtype=torch.int32, device=dev), caches[0].struct)
+    torch.cuda.synchronize()
+    for c in caches[1:]:
+        c.c_kv.copy_(caches[0].c_kv)
+        if c.c_scales is not None:
+            c.c_scales.copy_(caches[0].c_scales)
+        if c.k_rope is not None:
+            c.k_rope.copy_(caches[0].k_rope)
+    prefill_s = time.perf_counter() - t0
+    assert mla.mla_device_error(plan) == 0
+
+    # ---- step inputs
+    xd = gen.to_torch(x_dec, wl.dtype, dev)
+    q = gen.to_torch(gen.decode_queries(wl, w), wl.dtype, dev)
+    seq_idx = torch.arange(B, dtype=torch.int32, device=dev)
+    pos = torch.tensor(lens - 1, dtype=torch.int32, device=dev)
+    seq_lens = torch.tensor(lens, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    ws = workspace(plan, B, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        c = caches[i % n_rep].struct
+        mla.mla_append(plan, xd, seq_idx, pos, c, stream=stream)
+        mla.mla_decode(plan, c, seq_lens, q, out, ws, stream=stream)
+
+    launches_per_step = 4   # append, absorb(+schedule), split-K attention, combine(+W_uv)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, dominant-kernel events recorded on the launching stream
+    import ctypes
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ev:
+        a.record(stream); b.record(stream)
+    handles = [(ctypes.c_void_p * 2)(a.cuda_event, b.cuda_event) for a, b in ev]
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    sampler = ClockSampler(vis.split(",")[local] if vis else local)
+    sampler.start()
+    # keep the GPU under the same load for ~1.5 s before the timed region so that the
+    # 100 ms clock samples cover the timed region and its steady state
+    t_soak = time.perf_counter()
+    i = 0
+    while time.perf_counter() - t_soak < 1.5:
+        step(i)
+        i += 1
+        if i % 64 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    start.record(stream)
+    for i in range(K):
+        mla.mla_plan_set_option(plan, mla.MLA_OPT_PROFILE_EVENTS, ctypes.addressof(handles[i]))
+        step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    mla.mla_plan_set_option(plan, mla.MLA_OPT_PROFILE_EVENTS, 0)
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    kern_ms = [a.elapsed_time(b) for a, b in ev]
+    kern_avg_ms = statistics.mean(kern_ms)
+    t_local = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
+    total_ms = float(t_local.item())
+    ms_per_step = total_ms / K
+    tokens = int(np.sum(lens))
+    value = tokens * world / (ms_per_step * 1e-3)
+
+    # ---- decode-only timing (same inputs, no append) for the whole-decode roofline
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nd = min(K, 1000)
+    s2.record(stream)
+    for i in range(nd):
+        mla.mla_decode(plan, caches[i % n_rep].struct, seq_lens, q, out, ws, stream=stream)
+    e2.record(stream)
+    torch.cuda.synchronize()
+    decode_ms = s2.elapsed_time(e2) / nd
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside
+    xh = xd.cpu().pin_memory()
+    qh = q.cpu().pin_memory()
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    E = args.e2e_steps
+    torch.cuda.synchronize()
+    s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s3.record(stream)
+    for i in range(E):
+        xd.copy_(xh, non_blocking=True)
+        q.copy_(qh, non_blocking=True)
+        step(i)
+        oh.copy_(out, non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([s3.elapsed_time(e3) / E], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = tokens * world / (float(e2e_ms.item()) * 1e-3)
+    h2d = xd.numel() * xd.element_size() + q.numel() * q.element_size()
+    d2h = out.numel() * out.element_size()
+
+    # ---- roofline of the dominant kernel (split-K attention over the cache)
+    peak, peak_src = measured_peak_hbm()
+    kern_bytes = cache_bytes                      # algorithmic: every cached byte read once
+    achieved = kern_bytes / (kern_avg_ms * 1e-3) / 1e9
+    wuk = wl.n_kv_heads * wl.d_c * (wl.head_dim - 2 * wl.r_pairs) * (2 if wl.dtype == "bf16" else 4)
+    wuv = wl.n_kv_heads * wl.d_c * wl.head_dim * (2 if wl.dtype == "bf16" else 4)
+    decode_frac = (cache_bytes + wuk + wuv) / (decode_ms * 1e-3) / 1e9 / peak
+    kernel_name = "tcgen05 split-K latent attention" if args.kernel == 2 else "split-K latent attention"
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype if wl.cache != "int4_g32" else "bf16 (int4 latent cache)",
+        "data": "synthetic (seeded generators; random-init layer of the named shape)",
+        "config": dict(wl_config(wl, lens), parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                       l2=f"{n_rep} cache replicas rotated per step ({n_rep * cache_bytes / 2**20:.0f} MiB > 2x L2)"),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": kernel_name,
+                     "bytes_per_launch": kern_bytes, "avg_launch_ms": kern_avg_ms, "peak_source": peak_src},
+        "decode_only_ms": decode_ms, "decode_roofline_frac": decode_frac,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+        "conversion_s": conversion_s, "prefill_s": prefill_s,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_tok = int(min(lens[0], 4096))
+        times = oracle_decode_sample(wl, n_tok, 50, seconds_cap=20.0)
+        cpu_val = n_tok / statistics.median(times)
+        line["cpu_baseline"] = {"value": cpu_val, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                                "sample": f"float64 oracle decode of one query (all {wl.n_heads} heads) over "
+                                          f"{n_tok} cached tokens, median of {len(times)} runs"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    plan.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

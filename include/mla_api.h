@@ -1,0 +1,184 @@
+/*
+ * mla_api.h — C ABI of the MHA2MLA latent-cache decode library (B200, sm_100a).
+ *
+ * The method (paper notes "MHA2MLA: Towards Economical Inference by Enabling
+ * DeepSeek's Multi-Head Latent Attention in Any Transformer-based LLMs", ACL 2025,
+ * §方法详解/整体框架 and §关键设计) converts an MHA layer in two steps: partial-RoPE
+ * keeps, per head, the r frequency pairs with the largest 2-norm contribution, and
+ * a joint SVD of the NoPE key and value projections gives one shared latent
+ * c_kv = x W_dkv with per-head up-projections W_uk, W_uv.  Decoding then caches
+ * only c_kv and the kept RoPE key dims.
+ *
+ * Conventions (all entry points):
+ *   - Notation: d hidden, H query heads, n_kv KV heads (G = H/n_kv, head h uses KV
+ *     head g = h / G), d_h head dim, r kept pairs per KV head, R = n_kv*2r,
+ *     d_c latent width.  Pair k is the dims (2k, 2k+1); theta_k = base^(-2k/d_h);
+ *     positions are 0-based.
+ *   - Arrays are dense row-major (C order).  "dtype" means the config's dtype:
+ *     MLA_F32 = IEEE float32, MLA_BF16 = bfloat16 (uint16 storage).
+ *   - Pointers documented "device" must be device memory of the current device and
+ *     16-byte aligned; "host" pointers are ordinary host memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Work is enqueued on it; calls return before it completes.
+ *   - Every call validates its arguments first and returns a status without
+ *     launching anything when they are bad.  MLA_ERR_CUDA reports a failed CUDA
+ *     call (including an earlier asynchronous error surfacing at launch).
+ *     Device-side conditions (a sequence length beyond the cache capacity, a
+ *     pipeline wait that exceeded its bound) are recorded in the plan's device
+ *     error word and read with mla_device_error().
+ *   - The library never allocates device memory inside mla_append or mla_decode;
+ *     the caller owns inputs, outputs, the cache and the workspace.  A plan owns
+ *     its packed weight copies.  Calls on one plan are not thread-safe.
+ */
+#ifndef MLA_API_H
+#define MLA_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,          /* null pointer, non-positive or inconsistent size */
+  MLA_ERR_UNSUPPORTED = 2,          /* valid shape/dtype combination this build does not run */
+  MLA_ERR_ALIGNMENT = 3,            /* a device pointer is not 16-byte aligned */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes < mla_decode_workspace_bytes() */
+  MLA_ERR_CUDA = 5,                 /* a CUDA runtime/driver call failed */
+  MLA_ERR_DEVICE = 6                /* a kernel recorded an error (see mla_device_error) */
+} mla_status_t;
+
+typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype_t;
+
+/* Latent cache encoding.  MLA_CACHE_SAME stores c_kv in the config dtype.
+ * MLA_CACHE_INT4_G32 stores it per token in groups of 32 elements: one fp16
+ * scale s = fp16(absmax/7) per group and 4-bit two's-complement codes
+ * clamp(round_half_even(c/s), -7, 7) (codes 0 when s == 0), element 2i in the low
+ * nibble of byte i; value = code*s.  (Notes §关键设计: 4-bit quantisation stacks on
+ * the latent; the group layout is this library's choice.)  RoPE dims stay in dtype. */
+typedef enum { MLA_CACHE_SAME = 0, MLA_CACHE_INT4_G32 = 1 } mla_cache_kind_t;
+
+typedef struct {
+  int32_t hidden;       /* d */
+  int32_t n_heads;      /* H, multiple of n_kv_heads */
+  int32_t n_kv_heads;   /* n_kv */
+  int32_t head_dim;     /* d_h, even */
+  int32_t r_pairs;      /* r, 0 <= r <= d_h/2 */
+  int32_t d_c;          /* latent width (multiple of 32 for the int4 cache) */
+  double rope_base;     /* RoPE base (10000 for the Llama/SmolLM shapes) */
+  int32_t dtype;        /* mla_dtype_t */
+  int32_t cache_kind;   /* mla_cache_kind_t (int4 requires dtype MLA_BF16) */
+} mla_config_t;
+
+/* Caller-owned cache, device memory, capacity T_cap tokens per sequence.
+ *   c_kv     SAME: [B][T_cap][d_c] dtype;  INT4: [B][T_cap][d_c/2] uint8 codes
+ *   c_scales INT4: [B][T_cap][d_c/32] fp16;  SAME: must be NULL
+ *   k_rope   [B][T_cap][n_kv][2r] dtype (may be NULL when r == 0)          */
+typedef struct {
+  void* c_kv;
+  void* c_scales;
+  void* k_rope;
+  int32_t B;
+  int32_t T_cap;
+} mla_cache_t;
+
+typedef struct mla_plan mla_plan_t;   /* opaque, created by mla_plan_create */
+
+/* Options for mla_plan_set_option. */
+enum {
+  MLA_OPT_DECODE_KERNEL = 1,  /* 0 auto, 1 CUDA-core split-K kernel, 2 tcgen05 kernel */
+  MLA_OPT_DECODE_SPLITS = 2,  /* 0 auto (SM count based); n > 0: split the context
+                                 tiles into n contiguous worker ranges */
+  MLA_OPT_PROFILE_EVENTS = 3  /* value: address of a host array of two cudaEvent_t; each
+                                 mla_decode records [0] just before and [1] just after its
+                                 split-K attention kernel on the call's stream (0 = off).
+                                 The array must stay valid while the option is set. */
+};
+
+MLA_API const char* mla_status_string(mla_status_t s);
+MLA_API const char* mla_version(void);
+
+/* Bytes cached per token per layer for this config (c_kv, scales, RoPE dims).
+ * Notes §关键设计 (SVDjoint; KV-cache quantisation).  Returns 0 for an invalid config. */
+MLA_API size_t mla_cache_bytes_per_token(const mla_config_t* cfg);
+
+/* 2-norm contribution scores and head-wise top-r pair selection.
+ * Notes §关键设计, contribution-aware partial-RoPE removal: the contribution of pair k
+ * is bounded by ||q^[2k,2k+1]||*||k^[2k,2k+1]||; it is averaged over the T calibration
+ * tokens and over the G query heads of each KV head, then the r largest pairs are kept
+ * (equal scores: lower k first).  Accumulation is float32 in a fixed order.
+ *   q_cal    device [T][H][d_h] dtype, unrotated calibration queries
+ *   k_cal    device [T][n_kv][d_h] dtype, unrotated calibration keys
+ *   pair_idx device out [n_kv][r] int32, ascending within each KV head
+ *   contrib  device out [n_kv][d_h/2] float32 scores, or NULL               */
+MLA_API mla_status_t mla_select_pairs(const mla_config_t* cfg, const void* q_cal, const void* k_cal,
+                              int32_t T, int32_t* pair_idx, float* contrib, void* stream);
+
+/* Build a plan: validate the config and copy/pack the converted weights into
+ * plan-owned device memory.  All weight pointers are HOST memory in the config dtype.
+ *   W_dkv    [d][d_c]            joint-SVD down-projection (U_trunc)
+ *   W_k      [d][n_kv*d_h]       original key projection; the plan keeps the columns
+ *                                of the selected pairs (the RoPE key dims)
+ *   pair_idx [n_kv][r] int32     selected pairs, ascending, each in [0, d_h/2)
+ *   W_uk     [n_kv][d_c][d_h-2r] NoPE key up-projection (rows of Sigma V^T)
+ *   W_uv     [n_kv][d_c][d_h]    value up-projection
+ * Notes §关键设计 (SVDjoint): W_dkv = U_trunc, Sigma V^T split per head.
+ * On success *out receives the plan; release it with mla_plan_destroy. */
+MLA_API mla_status_t mla_plan_create(const mla_config_t* cfg, const void* W_dkv, const void* W_k,
+                             const int32_t* pair_idx, const void* W_uk, const void* W_uv,
+                             mla_plan_t** out);
+MLA_API void mla_plan_destroy(mla_plan_t* plan);
+MLA_API mla_status_t mla_plan_set_option(mla_plan_t* plan, int32_t option, int64_t value);
+
+/* Append N tokens to the cache.  For token n: c = x[n] W_dkv (float32 accumulation),
+ * the RoPE key dims x[n] W_k[:, kept pairs of g] are rotated at position pos[n]
+ * (angle computed in float64), c is stored in the cache encoding, and both are written
+ * at (seq_idx[n], pos[n]).  Notes §关键设计 (SVDjoint: c_kv = x W_dkv; partial-RoPE).
+ *   x       device [N][d] dtype
+ *   seq_idx device [N] int32 in [0, B);  pos device [N] int32 in [0, T_cap)
+ * Tokens with an out-of-range seq_idx/pos are skipped and flag the device error word.
+ * Distinct tokens must target distinct (seq, pos) slots. */
+MLA_API mla_status_t mla_append(const mla_plan_t* plan, const void* x, const int32_t* seq_idx,
+                        const int32_t* pos, int32_t N, const mla_cache_t* cache, void* stream);
+
+/* Device workspace mla_decode needs for a batch of B sequences (bytes, 256-aligned). */
+MLA_API size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B);
+
+/* One decode step: attention of each sequence's new query over its cached tokens
+ * [0, seq_lens[b]).  The query sits at position seq_lens[b]-1 (append it first).
+ * Steps: split q into NoPE and kept-RoPE dims; rotate the RoPE part; absorb W_uk into
+ * the NoPE part (q_lat = q_nope W_uk^T) so it scores against c_kv directly; add the
+ * RoPE score; scale 1/sqrt(d_h); split-K online softmax over the context; accumulate
+ * the probability-weighted latent; merge the splits; apply W_uv per head.
+ * Notes §关键设计 (the RoPE part cannot join the matrix merge and is computed apart).
+ *   seq_lens device [B] int32 (0 <= L <= T_cap; L == 0 gives a zero output row)
+ *   q        device [B][H][d_h] dtype, unrotated, original dim order
+ *   out      device [B][H][d_h] dtype, per-head attention output (before W_o)
+ *   workspace device, >= mla_decode_workspace_bytes(plan, B) bytes              */
+MLA_API mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
+                        const void* q, int32_t B, void* out, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/* Synchronise the device, read and clear the plan's device error word.
+ * *code receives 0 (none) or a bitwise OR of MLA_DEVERR_* values.
+ * Returns MLA_OK, or MLA_ERR_CUDA when the synchronisation itself failed. */
+enum {
+  MLA_DEVERR_SEQ_LEN = 1,     /* a seq_lens entry was < 0 or > T_cap (treated as 0) */
+  MLA_DEVERR_APPEND_SLOT = 2, /* an append token had seq_idx/pos out of range (skipped) */
+  MLA_DEVERR_TIMEOUT = 4      /* a pipeline wait exceeded its bound (output invalid) */
+};
+MLA_API mla_status_t mla_device_error(mla_plan_t* plan, int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_API_H */

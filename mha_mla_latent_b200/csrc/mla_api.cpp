@@ -1,0 +1,237 @@
+// Host side of the C ABI: argument validation, plan construction (weight packing),
+// workspace layout and kernel launches.  See include/mla_api.h for the contract.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <new>
+#include <vector>
+
+#include "mla_internal.h"
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+size_t elem_bytes(const mla_config_t& c) { return c.dtype == MLA_F32 ? 4 : 2; }
+
+mla_status_t validate_config(const mla_config_t* c) {
+  if (!c) return MLA_ERR_INVALID_ARG;
+  if (c->hidden <= 0 || c->n_heads <= 0 || c->n_kv_heads <= 0 || c->head_dim <= 0 || c->d_c <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (c->n_heads % c->n_kv_heads != 0 || c->head_dim % 2 != 0) return MLA_ERR_INVALID_ARG;
+  if (c->r_pairs < 0 || 2 * c->r_pairs > c->head_dim) return MLA_ERR_INVALID_ARG;
+  if (!(c->rope_base > 1.0)) return MLA_ERR_INVALID_ARG;
+  if (c->dtype != MLA_F32 && c->dtype != MLA_BF16) return MLA_ERR_INVALID_ARG;
+  if (c->cache_kind != MLA_CACHE_SAME && c->cache_kind != MLA_CACHE_INT4_G32) return MLA_ERR_INVALID_ARG;
+  if (c->cache_kind == MLA_CACHE_INT4_G32 && (c->dtype != MLA_BF16 || c->d_c % 32 != 0))
+    return MLA_ERR_UNSUPPORTED;
+  // limits of the kernels in this build
+  if (c->head_dim > 256 || c->d_c > 1024 || c->n_heads > 256) return MLA_ERR_UNSUPPORTED;
+  if (c->d_c % 2 != 0) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+mla_status_t validate_cache(const mla_config_t& cfg, const mla_cache_t* c) {
+  if (!c || !c->c_kv || c->B <= 0 || c->T_cap <= 0) return MLA_ERR_INVALID_ARG;
+  bool int4 = cfg.cache_kind == MLA_CACHE_INT4_G32;
+  if (int4 && !c->c_scales) return MLA_ERR_INVALID_ARG;
+  if (!int4 && c->c_scales) return MLA_ERR_INVALID_ARG;
+  if (cfg.r_pairs > 0 && !c->k_rope) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(c->c_kv) || (c->c_scales && !aligned16(c->c_scales)) ||
+      (c->k_rope && !aligned16(c->k_rope)))
+    return MLA_ERR_ALIGNMENT;
+  return MLA_OK;
+}
+
+mla_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+bool dev_alloc_copy(void** dst, const void* src, size_t bytes) {
+  if (cudaMalloc(dst, bytes) != cudaSuccess) { *dst = nullptr; return false; }
+  return cudaMemcpy(*dst, src, bytes, cudaMemcpyHostToDevice) == cudaSuccess;
+}
+
+void free_plan(mla_plan* p) {
+  if (!p) return;
+  void* bufs[] = {p->W_app, p->W_ukT, p->W_uv, p->nope_idx, p->rope_pair, p->theta, p->err};
+  for (void* b : bufs)
+    if (b) cudaFree(b);
+  delete p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(mla_status_t s) {
+  switch (s) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_INVALID_ARG: return "invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MLA_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case MLA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MLA_ERR_CUDA: return "CUDA error";
+    case MLA_ERR_DEVICE: return "device-side error recorded";
+  }
+  return "unknown status";
+}
+
+const char* mla_version(void) { return "mla_b200 0.1 (sm_100a)"; }
+
+size_t mla_cache_bytes_per_token(const mla_config_t* cfg) {
+  if (validate_config(cfg) == MLA_ERR_INVALID_ARG) return 0;
+  size_t eb = elem_bytes(*cfg);
+  size_t rope = (size_t)cfg->n_kv_heads * 2 * cfg->r_pairs * eb;
+  if (cfg->cache_kind == MLA_CACHE_INT4_G32) return (size_t)cfg->d_c / 2 + 2 * ((size_t)cfg->d_c / 32) + rope;
+  return (size_t)cfg->d_c * eb + rope;
+}
+
+mla_status_t mla_select_pairs(const mla_config_t* cfg, const void* q_cal, const void* k_cal,
+                              int32_t T, int32_t* pair_idx, float* contrib, void* stream) {
+  mla_status_t st = validate_config(cfg);
+  if (st != MLA_OK) return st;
+  if (!q_cal || !k_cal || !pair_idx || T <= 0) return MLA_ERR_INVALID_ARG;
+  if (cfg->head_dim / 2 > 128) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(q_cal) || !aligned16(k_cal)) return MLA_ERR_ALIGNMENT;
+  return cuda_status(mla_launch_select_pairs(*cfg, q_cal, k_cal, T, pair_idx, contrib,
+                                             (cudaStream_t)stream));
+}
+
+mla_status_t mla_plan_create(const mla_config_t* cfg, const void* W_dkv, const void* W_k,
+                             const int32_t* pair_idx, const void* W_uk, const void* W_uv,
+                             mla_plan_t** out) {
+  if (!out) return MLA_ERR_INVALID_ARG;
+  *out = nullptr;
+  mla_status_t st = validate_config(cfg);
+  if (st != MLA_OK) return st;
+  const int d = cfg->hidden, nkv = cfg->n_kv_heads, dh = cfg->head_dim, r = cfg->r_pairs;
+  const int dc = cfg->d_c;
+  if (!W_dkv || !W_uv || (dh - 2 * r > 0 && !W_uk) || (r > 0 && (!W_k || !pair_idx)))
+    return MLA_ERR_INVALID_ARG;
+  for (int g = 0; g < nkv; ++g)
+    for (int j = 0; j < r; ++j) {
+      int k = pair_idx[g * r + j];
+      if (k < 0 || k >= dh / 2) return MLA_ERR_INVALID_ARG;
+      if (j > 0 && k <= pair_idx[g * r + j - 1]) return MLA_ERR_INVALID_ARG;  // strictly ascending
+    }
+  mla_plan* p = new (std::nothrow) mla_plan();
+  if (!p) return MLA_ERR_CUDA;
+  p->cfg = *cfg;
+  p->R = nkv * 2 * r;
+  p->dn = dh - 2 * r;
+  p->ncols = dc + p->R;
+  if (cudaGetDevice(&p->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess) {
+    free_plan(p);
+    return MLA_ERR_CUDA;
+  }
+  const size_t eb = elem_bytes(*cfg);
+  // [W_dkv | W_krope]: column block of the selected pairs of each KV head, ascending.
+  std::vector<unsigned char> app((size_t)d * p->ncols * eb);
+  for (int i = 0; i < d; ++i) {
+    memcpy(&app[((size_t)i * p->ncols) * eb], (const unsigned char*)W_dkv + (size_t)i * dc * eb, dc * eb);
+    for (int g = 0; g < nkv; ++g)
+      for (int j = 0; j < r; ++j)
+        for (int e = 0; e < 2; ++e) {
+          int src_col = g * dh + 2 * pair_idx[g * r + j] + e;
+          int dst_col = dc + g * 2 * r + 2 * j + e;
+          memcpy(&app[((size_t)i * p->ncols + dst_col) * eb],
+                 (const unsigned char*)W_k + ((size_t)i * nkv * dh + src_col) * eb, eb);
+        }
+  }
+  // W_uk transposed per head: [g][j][c]
+  std::vector<unsigned char> ukT((size_t)nkv * std::max(p->dn, 1) * dc * eb, 0);
+  for (int g = 0; g < nkv; ++g)
+    for (int c = 0; c < dc; ++c)
+      for (int j = 0; j < p->dn; ++j)
+        memcpy(&ukT[(((size_t)g * p->dn + j) * dc + c) * eb],
+               (const unsigned char*)W_uk + (((size_t)g * dc + c) * p->dn + j) * eb, eb);
+  std::vector<int32_t> nope((size_t)nkv * std::max(p->dn, 1), 0), rp((size_t)nkv * std::max(r, 1), 0);
+  for (int g = 0; g < nkv; ++g) {
+    std::vector<char> kept(dh / 2, 0);
+    for (int j = 0; j < r; ++j) { kept[pair_idx[g * r + j]] = 1; rp[g * r + j] = pair_idx[g * r + j]; }
+    int n = 0;
+    for (int i = 0; i < dh; ++i)
+      if (!kept[i / 2]) nope[(size_t)g * p->dn + (n++)] = i;
+  }
+  std::vector<double> theta(dh / 2);
+  for (int k = 0; k < dh / 2; ++k) theta[k] = pow(cfg->rope_base, -2.0 * k / dh);
+
+  bool ok = dev_alloc_copy(&p->W_app, app.data(), app.size()) &&
+            dev_alloc_copy(&p->W_ukT, ukT.data(), ukT.size()) &&
+            dev_alloc_copy(&p->W_uv, W_uv, (size_t)nkv * dc * dh * eb) &&
+            dev_alloc_copy((void**)&p->nope_idx, nope.data(), nope.size() * sizeof(int32_t)) &&
+            dev_alloc_copy((void**)&p->rope_pair, rp.data(), rp.size() * sizeof(int32_t)) &&
+            dev_alloc_copy((void**)&p->theta, theta.data(), theta.size() * sizeof(double)) &&
+            cudaMalloc((void**)&p->err, sizeof(int32_t)) == cudaSuccess &&
+            cudaMemset(p->err, 0, sizeof(int32_t)) == cudaSuccess;
+  if (!ok) {
+    free_plan(p);
+    return MLA_ERR_CUDA;
+  }
+  *out = p;
+  return MLA_OK;
+}
+
+void mla_plan_destroy(mla_plan_t* plan) { free_plan(plan); }
+
+mla_status_t mla_plan_set_option(mla_plan_t* plan, int32_t option, int64_t value) {
+  if (!plan) return MLA_ERR_INVALID_ARG;
+  switch (option) {
+    case MLA_OPT_DECODE_KERNEL:
+      if (value < 0 || value > 2) return MLA_ERR_INVALID_ARG;
+      plan->opt_kernel = (int)value;
+      return MLA_OK;
+    case MLA_OPT_DECODE_SPLITS:
+      if (value < 0 || value > (1 << 20)) return MLA_ERR_INVALID_ARG;
+      plan->opt_splits = (int)value;
+      return MLA_OK;
+    case MLA_OPT_PROFILE_EVENTS:
+      plan->opt_events = (const void* const*)(uintptr_t)value;
+      return MLA_OK;
+  }
+  return MLA_ERR_INVALID_ARG;
+}
+
+mla_status_t mla_append(const mla_plan_t* plan, const void* x, const int32_t* seq_idx,
+                        const int32_t* pos, int32_t N, const mla_cache_t* cache, void* stream) {
+  if (!plan || !x || !seq_idx || !pos || N <= 0) return MLA_ERR_INVALID_ARG;
+  mla_status_t st = validate_cache(plan->cfg, cache);
+  if (st != MLA_OK) return st;
+  if (!aligned16(x) || ((uintptr_t)seq_idx & 3) || ((uintptr_t)pos & 3)) return MLA_ERR_ALIGNMENT;
+  return cuda_status(mla_launch_append(*plan, x, seq_idx, pos, N, *cache, (cudaStream_t)stream));
+}
+
+size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B) {
+  if (!plan || B <= 0) return 0;
+  return mla_decode_layout(*plan, B).total;
+}
+
+mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
+                        const void* q, int32_t B, void* out, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  if (!plan || !seq_lens || !q || !out || !workspace || B <= 0) return MLA_ERR_INVALID_ARG;
+  mla_status_t st = validate_cache(plan->cfg, cache);
+  if (st != MLA_OK) return st;
+  if (B > cache->B) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace) || ((uintptr_t)seq_lens & 3))
+    return MLA_ERR_ALIGNMENT;
+  if ((size_t)plan->cfg.n_heads * plan->cfg.d_c > 8192) return MLA_ERR_UNSUPPORTED;
+  DecodeLayout L = mla_decode_layout(*plan, B);
+  if (ws_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  return cuda_status(mla_launch_decode(*plan, *cache, seq_lens, q, B, out, workspace, L,
+                                       (cudaStream_t)stream));
+}
+
+mla_status_t mla_device_error(mla_plan_t* plan, int32_t* code) {
+  if (!plan || !code) return MLA_ERR_INVALID_ARG;
+  *code = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaMemcpy(code, plan->err, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (cudaMemset(plan->err, 0, sizeof(int32_t)) != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,65 @@
+// Internal declarations shared by the host API (mla_api.cpp) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mla_api.h"
+
+struct mla_plan {
+  mla_config_t cfg;
+  int device = 0;
+  int num_sms = 0;
+  int R = 0;       // n_kv * 2r   (RoPE key dims per token)
+  int dn = 0;      // d_h - 2r    (NoPE dims per head)
+  int ncols = 0;   // d_c + R     (columns of the packed append weight)
+  // plan-owned device memory
+  void* W_app = nullptr;       // [d][ncols] dtype: [W_dkv | W_krope]
+  void* W_ukT = nullptr;       // [n_kv][dn][d_c] dtype (W_uk transposed per head)
+  void* W_uv = nullptr;        // [n_kv][d_c][d_h] dtype
+  int32_t* nope_idx = nullptr;   // [n_kv][dn]  NoPE dims, ascending
+  int32_t* rope_pair = nullptr;  // [n_kv][r]   kept pair indices, ascending
+  double* theta = nullptr;       // [d_h/2]     RoPE frequencies
+  int32_t* err = nullptr;        // device error word (MLA_DEVERR_* bits)
+  // options
+  int opt_kernel = 0;
+  int opt_splits = 0;
+  const void* const* opt_events = nullptr;  // cudaEvent_t[2] or null
+};
+
+// Decode workspace layout (byte offsets from the workspace base).
+struct DecodeLayout {
+  int kernel = 1;          // 1 CUDA-core, 2 tcgen05
+  int tile = 32;           // tokens per schedule tile
+  int G = 0;               // workers (CTAs of the split-K kernel)
+  int P = 0;               // max pieces = B + G
+  int K = 0;               // tcgen05 query row width (d_c + R)
+  size_t off_seq_tile0, off_seq_ntiles, off_seq_ne, off_seq_first, off_seq_np;
+  size_t off_worker_first, off_piece_b, off_piece_t0, off_piece_t1;
+  size_t off_qlat, off_qrope, off_opart, off_mlpart;
+  size_t total = 0;
+};
+
+// Schedule view passed to kernels (pointers into the workspace).
+struct Sched {
+  int32_t* seq_tile0;     // [B]  first global tile of sequence b
+  int32_t* seq_ntiles;    // [B]
+  int32_t* seq_ne;        // [B+1] number of non-empty sequences before b
+  int32_t* seq_first;     // [B]  first piece of b
+  int32_t* seq_np;        // [B]  pieces of b
+  int32_t* worker_first;  // [G+1]
+  int32_t* piece_b;       // [P]
+  int32_t* piece_t0;      // [P] token begin within sequence
+  int32_t* piece_t1;      // [P] token end (exclusive)
+};
+
+DecodeLayout mla_decode_layout(const mla_plan& p, int B);
+Sched mla_sched_view(const DecodeLayout& L, void* ws, int B);
+
+cudaError_t mla_launch_select_pairs(const mla_config_t& cfg, const void* q, const void* k, int T,
+                                    int32_t* pair_idx, float* contrib, cudaStream_t s);
+cudaError_t mla_launch_append(const mla_plan& p, const void* x, const int32_t* seq_idx,
+                              const int32_t* pos, int N, const mla_cache_t& c, cudaStream_t s);
+cudaError_t mla_launch_decode(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens,
+                              const void* q, int B, void* out, void* ws, const DecodeLayout& L,
+                              cudaStream_t s);

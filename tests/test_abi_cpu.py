@@ -1,0 +1,95 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared entry point,
+and rejects bad arguments with the documented status before touching the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "mla_api.h")
+
+
+@pytest.fixture(scope="module")
+def mla():
+    from mha_mla_latent_b200 import build
+    build.build()
+    import mha_mla_latent_b200._lib as lib
+    return lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MLA_API\s+[\w\s\*]+?\b(mla_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("mla_select_pairs", "mla_plan_create", "mla_append", "mla_decode",
+              "mla_decode_workspace_bytes", "mla_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(mla):
+    so = ctypes.CDLL(mla.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(so, name), name
+    assert set(declared_functions()) == set(mla.EXPORTED)
+
+
+def test_status_strings_and_version(mla):
+    assert "sm_100a" in mla.mla_version()
+    for s in range(7):
+        assert mla.mla_status_string(s)
+
+
+def test_cache_bytes_per_token_matches_oracle_accounting(mla):
+    import oracle as O
+    from workloads import WORKLOADS
+    for w in WORKLOADS:
+        cfg = mla.config_from_workload(w)
+        ref = O.cache_bytes_per_token(w.n_kv_heads, w.r_pairs, w.d_c, 4 if w.dtype == "f32" else 2,
+                                      int4=w.cache == "int4_g32")
+        assert mla.mla_cache_bytes_per_token(cfg) == ref, w.name
+
+
+def test_invalid_configs_rejected(mla):
+    ok = mla.make_config(512, 8, 4, 64, 4, 64)
+    out = ctypes.c_void_p()
+    bad = [
+        mla.make_config(512, 9, 4, 64, 4, 64),       # H not a multiple of n_kv
+        mla.make_config(512, 8, 4, 63, 4, 64),       # odd head dim
+        mla.make_config(512, 8, 4, 64, 40, 64),      # r > d_h/2
+        mla.make_config(0, 8, 4, 64, 4, 64),
+    ]
+    for cfg in bad:
+        st = mla._lib.mla_plan_create(ctypes.byref(cfg), None, None, None, None, None, ctypes.byref(out))
+        assert st == mla.MLA_ERR_INVALID_ARG
+    f32_int4 = mla.make_config(512, 8, 4, 64, 4, 64, dtype="f32", cache="int4_g32")
+    st = mla._lib.mla_plan_create(ctypes.byref(f32_int4), None, None, None, None, None, ctypes.byref(out))
+    assert st == mla.MLA_ERR_UNSUPPORTED
+    # null weights with a valid config
+    st = mla._lib.mla_plan_create(ctypes.byref(ok), None, None, None, None, None, ctypes.byref(out))
+    assert st == mla.MLA_ERR_INVALID_ARG
+    assert mla._lib.mla_plan_create(ctypes.byref(ok), None, None, None, None, None, None) == mla.MLA_ERR_INVALID_ARG
+
+
+def test_pair_selection_validation(mla):
+    cfg = mla.make_config(512, 8, 4, 64, 4, 64)
+    sp = mla._lib.mla_select_pairs
+    assert sp(ctypes.byref(cfg), None, 4096, 16, 8192, None, None) == mla.MLA_ERR_INVALID_ARG
+    assert sp(ctypes.byref(cfg), 4096, 4096, 0, 8192, None, None) == mla.MLA_ERR_INVALID_ARG
+    assert sp(ctypes.byref(cfg), 4097, 4096, 16, 8192, None, None) == mla.MLA_ERR_ALIGNMENT
+
+
+def test_append_and_decode_need_a_plan(mla):
+    cache = mla.MlaCache(4096, None, 8192, 2, 16)
+    assert mla._lib.mla_append(None, 4096, 4096, 4096, 1, ctypes.byref(cache), None) == mla.MLA_ERR_INVALID_ARG
+    assert mla._lib.mla_decode(None, ctypes.byref(cache), 4096, 4096, 1, 4096, 4096, 1 << 20, None) \
+        == mla.MLA_ERR_INVALID_ARG
+    assert mla._lib.mla_decode_workspace_bytes(None, 4) == 0
+    assert mla._lib.mla_plan_set_option(None, 1, 0) == mla.MLA_ERR_INVALID_ARG
+    code = ctypes.c_int32()
+    assert mla._lib.mla_device_error(None, ctypes.byref(code)) == mla.MLA_ERR_INVALID_ARG

@@ -1,0 +1,201 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle.
+
+Tolerances: pair indices bit-exact; fp32 rel-L2 <= 1e-5; bf16/int4 rel-L2 <= 1e-2 and
+max-abs <= 3e-2 (decode outputs and appended cache).  int4 codes are bit-exact when
+the latent the kernel quantises is exact (one-hot tokens).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from tests.helpers import OracleCase, assert_close, plan_inputs, upload_oracle_cache
+from workloads import PARITY_WORKLOADS, generate as gen
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import mha_mla_latent_b200 as mla
+    from mha_mla_latent_b200.cache import LatentCache, workspace
+
+IDS = [w.name for w in PARITY_WORKLOADS]
+_CASES = {}
+
+
+def case_for(wl):
+    if wl.name not in _CASES:
+        _CASES[wl.name] = OracleCase(wl)
+    return _CASES[wl.name]
+
+
+def make_plan(case, kernel=0, splits=0):
+    cfg = mla.config_from_workload(case.wl)
+    plan = mla.mla_plan_create(cfg, **plan_inputs(case))
+    if kernel:
+        mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, kernel)
+    if splits:
+        mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_SPLITS, splits)
+    return cfg, plan
+
+
+def run_decode(case, plan, cfg, cache=None, lens=None):
+    wl = case.wl
+    dev = "cuda"
+    lens = case.lens if lens is None else lens
+    T_cap = max(1, int(max(lens)))
+    if cache is None:
+        cache = LatentCache(cfg, wl.batch, T_cap, dev)
+        upload_oracle_cache(case, cache, T_cap)
+    seq = torch.tensor(np.asarray(lens), dtype=torch.int32, device=dev)
+    q = gen.to_torch(case.q, wl.dtype, dev)
+    out = torch.empty_like(q)
+    ws = workspace(plan, wl.batch, dev)
+    mla.mla_decode(plan, cache.struct, seq, q, out, ws)
+    torch.cuda.synchronize()
+    return out.double().cpu().numpy()
+
+
+# --------------------------------------------------------------------------- a9
+@pytest.mark.parametrize("wl", PARITY_WORKLOADS, ids=IDS)
+def test_select_pairs_bit_exact(wl):
+    case = case_for(wl)
+    cfg = mla.config_from_workload(wl)
+    q = gen.to_torch(case.q_cal, wl.dtype, "cuda")
+    k = gen.to_torch(case.k_cal, wl.dtype, "cuda")
+    from mha_mla_latent_b200.convert import select_pairs
+    pair_idx, contrib = select_pairs(cfg, q, k)
+    torch.cuda.synchronize()
+    ref = case.conv["contrib"]
+    # the seed must not be near-tied at the r-th/(r+1)-th boundary for a bit-exact claim
+    srt = -np.sort(-ref, axis=1)
+    gap = (srt[:, wl.r_pairs - 1] - srt[:, wl.r_pairs]) / srt[:, wl.r_pairs - 1]
+    assert np.all(gap > 1e-4), f"near-tied seed: min relative gap {gap.min():.2e}"
+    assert pair_idx.cpu().numpy().tolist() == case.conv["pair_idx"].tolist()
+    np.testing.assert_allclose(contrib.cpu().numpy(), ref, rtol=2e-5)
+
+
+# --------------------------------------------------------------------------- a0
+@pytest.mark.parametrize("wl", PARITY_WORKLOADS, ids=IDS)
+def test_append_parity(wl):
+    case = case_for(wl)
+    cfg, plan = make_plan(case)
+    T_cap = int(max(case.lens))
+    cache = LatentCache(cfg, wl.batch, max(T_cap, 1), "cuda")
+    xs, sidx, pos = [], [], []
+    for b in case.seqs:
+        x = case.tokens(b)
+        xs.append(x)
+        sidx += [b] * x.shape[0]
+        pos += list(range(x.shape[0]))
+    x = gen.to_torch(np.concatenate(xs), wl.dtype, "cuda")
+    mla.mla_append(plan, x, torch.tensor(sidx, dtype=torch.int32, device="cuda"),
+                   torch.tensor(pos, dtype=torch.int32, device="cuda"), cache.struct)
+    assert mla.mla_device_error(plan) == 0
+    for b in case.seqs:
+        L = int(case.lens[b])
+        if L == 0:
+            continue
+        cc = case.cache[b]
+        kr = cache.k_rope[b, :L].double().cpu().numpy()
+        assert_close(kr, cc["kr_exact"], wl.dtype, f"k_rope seq {b}")
+        if wl.cache == "int4_g32":
+            codes = O.unpack_int4(cache.c_kv[b, :L].cpu().numpy())
+            scales = cache.c_scales[b, :L].cpu().numpy()
+            deq = O.dequant_int4_g32(codes, scales)
+            assert_close(deq, cc["c"], wl.dtype, f"int4 latent seq {b}")
+            # codes differ only where the float32 latents straddle a rounding boundary
+            assert np.mean(codes != cc["codes"]) < 1e-3
+        else:
+            c = cache.c_kv[b, :L].double().cpu().numpy()
+            assert_close(c, cc["c_exact"], wl.dtype, f"latent seq {b}")
+
+
+def test_append_int4_codes_bit_exact_on_exact_latents():
+    """One-hot tokens make c = a row of W_dkv exactly; codes and scales must match bit for bit."""
+    wl = PARITY_WORKLOADS[4]
+    case = case_for(wl)
+    cfg, plan = make_plan(case)
+    n = 64
+    x = np.zeros((n, wl.hidden))
+    rows = np.arange(n) * 7 % wl.hidden
+    x[np.arange(n), rows] = 1.0
+    cache = LatentCache(cfg, 1, n, "cuda")
+    mla.mla_append(plan, gen.to_torch(x, wl.dtype, "cuda"), torch.zeros(n, dtype=torch.int32, device="cuda"),
+                   torch.arange(n, dtype=torch.int32, device="cuda"), cache.struct)
+    torch.cuda.synchronize()
+    c = case.conv["W_dkv"][rows]
+    codes_ref, scales_ref = O.quant_int4_g32(c)
+    np.testing.assert_array_equal(cache.c_kv[0].cpu().numpy(), O.pack_int4(codes_ref))
+    np.testing.assert_array_equal(cache.c_scales[0].cpu().numpy().view(np.uint16), scales_ref.view(np.uint16))
+
+
+# --------------------------------------------------------------------------- a1-a8
+@pytest.mark.parametrize("kernel", [0, 1])
+@pytest.mark.parametrize("wl", PARITY_WORKLOADS, ids=IDS)
+def test_decode_parity(wl, kernel):
+    case = case_for(wl)
+    cfg, plan = make_plan(case, kernel=kernel)
+    got = run_decode(case, plan, cfg)
+    assert mla.mla_device_error(plan) == 0
+    for b in case.seqs:
+        assert_close(got[b], case.reference(b), wl.dtype, f"decode seq {b} (L={case.lens[b]})")
+
+
+@pytest.mark.parametrize("wl", PARITY_WORKLOADS[2:4], ids=IDS[2:4])
+def test_decode_split_invariance(wl):
+    case = case_for(wl)
+    outs = []
+    for splits in (1, 2, 7, 0):
+        cfg, plan = make_plan(case, splits=splits)
+        outs.append(run_decode(case, plan, cfg))
+    for o in outs[1:]:
+        np.testing.assert_allclose(o, outs[0], rtol=0, atol=2e-2 if wl.dtype == "bf16" else 1e-6)
+
+
+def test_decode_empty_and_overlong_sequences():
+    wl = PARITY_WORKLOADS[2]
+    case = case_for(wl)
+    cfg, plan = make_plan(case)
+    lens = np.array(case.lens)
+    T_cap = int(lens.max())
+    cache = LatentCache(cfg, wl.batch, T_cap, "cuda")
+    upload_oracle_cache(case, cache, T_cap)
+    bad = lens.copy()
+    bad[1] = 0            # empty sequence -> zero row, no error
+    got = run_decode(case, plan, cfg, cache=cache, lens=bad)
+    assert mla.mla_device_error(plan) == 0
+    assert np.all(got[1] == 0)
+    assert_close(got[0], case.reference(0), wl.dtype, "seq 0 beside an empty sequence")
+    bad[2] = T_cap + 5    # beyond capacity -> flagged, treated as empty
+    got = run_decode(case, plan, cfg, cache=cache, lens=bad)
+    assert mla.mla_device_error(plan) & mla.MLA_DEVERR_SEQ_LEN
+    assert np.all(got[2] == 0)
+
+
+# --------------------------------------------------------------------------- end to end
+@pytest.mark.parametrize("wl", PARITY_WORKLOADS, ids=IDS)
+def test_end_to_end_conversion_append_decode(wl):
+    """Product conversion (GPU pair selection + device SVD) -> GPU append -> GPU decode,
+    against the oracle's own conversion, append and decode from the same raw layer."""
+    case = case_for(wl)
+    from mha_mla_latent_b200.convert import convert_layer, plan_from_converted
+    cfg = mla.config_from_workload(wl)
+    conv = convert_layer(cfg, gen.to_torch(case.w["W_k"], wl.dtype, "cuda"),
+                         gen.to_torch(case.w["W_v"], wl.dtype, "cuda"),
+                         gen.to_torch(case.q_cal, wl.dtype, "cuda"), gen.to_torch(case.k_cal, wl.dtype, "cuda"))
+    assert conv["pair_idx"].numpy().tolist() == case.conv["pair_idx"].tolist()
+    plan = plan_from_converted(cfg, conv)
+    T_cap = max(1, int(max(case.lens)))
+    cache = LatentCache(cfg, wl.batch, T_cap, "cuda")
+    for b in case.seqs:
+        x = case.tokens(b)
+        if x.shape[0] == 0:
+            continue
+        mla.mla_append(plan, gen.to_torch(x, wl.dtype, "cuda"),
+                       torch.full((x.shape[0],), b, dtype=torch.int32, device="cuda"),
+                       torch.arange(x.shape[0], dtype=torch.int32, device="cuda"), cache.struct)
+    got = run_decode(case, plan, cfg, cache=cache)
+    assert mla.mla_device_error(plan) == 0
+    for b in case.seqs:
+        assert_close(got[b], case.reference(b), wl.dtype, f"end-to-end seq {b}")
