@@ -36,6 +36,33 @@ def assert_close(got, ref, dtype: str, what: str = ""):
     return rl
 
 
+def bf16_ulp(x):
+    """Spacing of bfloat16 numbers at |x| (8 significand bits)."""
+    ax = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(ax, 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+def assert_stored_close(got, exact, dtype: str, what: str = ""):
+    """Cache entries are stored in the config dtype, so they are compared with the exact
+    float64 value within one unit in the last place of that dtype (the kernel rounds a
+    float32 sum once; when the sum sits next to a rounding midpoint it may land on the
+    other neighbour), plus the rel-L2 bound.  A fixed 3e-2 absolute bound is below the
+    bf16 spacing for |x| >= 8, so it cannot apply to stored values."""
+    got = np.asarray(got, dtype=np.float64)
+    exact = np.asarray(exact, dtype=np.float64)
+    assert got.shape == exact.shape and np.all(np.isfinite(got)), what
+    rl = rel_l2(got, exact)
+    if dtype == "f32":
+        assert rl <= TOL_F32_REL, f"{what}: rel-L2 {rl:.3e}"
+        return rl
+    err = np.abs(got - exact)
+    bound = bf16_ulp(exact) + 1e-6
+    worst = float(np.max(err / bound)) if err.size else 0.0
+    assert rl <= TOL_BF16_REL and worst <= 1.0, f"{what}: rel-L2 {rl:.3e}, worst error {worst:.2f} ulp"
+    return rl
+
+
 class OracleCase:
     """Oracle conversion, cache and reference outputs for one workload (float64)."""
 

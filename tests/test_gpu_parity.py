@@ -1,8 +1,9 @@
 """GPU parity: the CUDA path through the C ABI against the float64 oracle.
 
-Tolerances: pair indices bit-exact; fp32 rel-L2 <= 1e-5; bf16/int4 rel-L2 <= 1e-2 and
-max-abs <= 3e-2 (decode outputs and appended cache).  int4 codes are bit-exact when
-the latent the kernel quantises is exact (one-hot tokens).
+Tolerances: pair indices bit-exact; fp32 rel-L2 <= 1e-5; bf16/int4 decode outputs
+rel-L2 <= 1e-2 and max-abs <= 3e-2.  Appended cache entries (stored in the config
+dtype) are within one storage ulp of the exact value and rel-L2 <= 1e-2.  int4 codes
+are bit-exact when the latent the kernel quantises is exact (one-hot tokens).
 """
 
 import numpy as np
@@ -10,7 +11,7 @@ import pytest
 import torch
 
 import oracle as O
-from tests.helpers import OracleCase, assert_close, plan_inputs, upload_oracle_cache
+from tests.helpers import OracleCase, assert_close, assert_stored_close, plan_inputs, upload_oracle_cache
 from workloads import PARITY_WORKLOADS, generate as gen
 
 pytestmark = pytest.mark.gpu
@@ -98,7 +99,7 @@ def test_append_parity(wl):
             continue
         cc = case.cache[b]
         kr = cache.k_rope[b, :L].double().cpu().numpy()
-        assert_close(kr, cc["kr_exact"], wl.dtype, f"k_rope seq {b}")
+        assert_stored_close(kr, cc["kr_exact"], wl.dtype, f"k_rope seq {b}")
         if wl.cache == "int4_g32":
             codes = O.unpack_int4(cache.c_kv[b, :L].cpu().numpy())
             scales = cache.c_scales[b, :L].cpu().numpy()
@@ -108,7 +109,7 @@ def test_append_parity(wl):
             assert np.mean(codes != cc["codes"]) < 1e-3
         else:
             c = cache.c_kv[b, :L].double().cpu().numpy()
-            assert_close(c, cc["c_exact"], wl.dtype, f"latent seq {b}")
+            assert_stored_close(c, cc["c_exact"], wl.dtype, f"latent seq {b}")
 
 
 def test_append_int4_codes_bit_exact_on_exact_latents():
@@ -131,12 +132,18 @@ def test_append_int4_codes_bit_exact_on_exact_latents():
 
 
 # --------------------------------------------------------------------------- a1-a8
-@pytest.mark.parametrize("kernel", [0, 1])
+@pytest.mark.parametrize("kernel", [0, 1, 2])
 @pytest.mark.parametrize("wl", PARITY_WORKLOADS, ids=IDS)
 def test_decode_parity(wl, kernel):
+    """kernel 0: the plan's choice; 1: CUDA-core split-K; 2: tcgen05 (bf16, 32 heads)."""
     case = case_for(wl)
     cfg, plan = make_plan(case, kernel=kernel)
-    got = run_decode(case, plan, cfg)
+    try:
+        got = run_decode(case, plan, cfg)
+    except mla.MlaError as e:
+        if kernel == 2 and e.status == mla.MLA_ERR_UNSUPPORTED:
+            pytest.skip("shape outside the tensor-core kernel (fp32 or H != 32)")
+        raise
     assert mla.mla_device_error(plan) == 0
     for b in case.seqs:
         assert_close(got[b], case.reference(b), wl.dtype, f"decode seq {b} (L={case.lens[b]})")
