@@ -88,6 +88,7 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
     float acc[kAbsMaxRows];
 #pragma unroll
     for (int i = 0; i < kAbsMaxRows; ++i) acc[i] = 0.f;
+#pragma unroll 8
     for (int j = 0; j < a.dn; ++j) {
       float w = to_f32(W[(size_t)j * a.d_c + c]);
 #pragma unroll
@@ -236,35 +237,67 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   const int nb = min(a.bchunk, a.B - b0);
   const int rows = nb * G;
   extern __shared__ float sm[];
-  float* s_o = sm;                 // [rows][d_c]
-  float* s_w = s_o + rows * a.d_c; // scratch: per (row) weights are recomputed per element
-  (void)s_w;
-  // Merge: O_lat = sum_j 2^(m_j - M) O_j / sum_j 2^(m_j - M) l_j.
-  for (int i = threadIdx.x; i < rows * a.d_c; i += blockDim.x) {
-    int row = i / a.d_c, c = i % a.d_c;
-    int b = b0 + row / G, h = g * G + row % G;
-    int first = a.sched.seq_first[b], np = a.sched.seq_np[b];
+  float* s_o = sm;                    // [rows][d_c]
+  float* s_M = s_o + rows * a.d_c;    // [rows] merged running max
+  float* s_inv = s_M + rows;          // [rows] 1 / merged sum
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+  // per (b, h): M = max_j m_j, 1 / sum_j 2^(m_j - M) l_j   (one warp per row)
+  for (int row = warp; row < rows; row += nwarp) {
+    const int b = b0 + row / G, h = g * G + row % G;
+    const int first = a.sched.seq_first[b], np = a.sched.seq_np[b];
     float M = -INFINITY;
-    for (int j = 0; j < np; ++j) M = fmaxf(M, a.mlpart[((size_t)(first + j) * a.H + h) * 2]);
-    float num = 0.f, den = 0.f;
-    for (int j = 0; j < np; ++j) {
+    for (int j = lane; j < np; j += 32) M = fmaxf(M, a.mlpart[((size_t)(first + j) * a.H + h) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float den = 0.f;
+    for (int j = lane; j < np; j += 32) {
       const float* ml = a.mlpart + ((size_t)(first + j) * a.H + h) * 2;
-      float wgt = exp2f(ml[0] - M);
-      den += wgt * ml[1];
-      num += wgt * a.opart[((size_t)(first + j) * a.H + h) * a.d_c + c];
+      den += exp2f(ml[0] - M) * ml[1];
     }
-    s_o[i] = (np > 0 && den > 0.f) ? num / den : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (lane == 0) {
+      s_M[row] = M;
+      s_inv[row] = (np > 0 && den > 0.f) ? 1.f / den : 0.f;
+    }
   }
   __syncthreads();
-  // o[row][d] = sum_c O_lat[row][c] W_uv[g][c][d]
+  // merged latent O_lat[row][c]
+  for (int i = threadIdx.x; i < rows * a.d_c; i += blockDim.x) {
+    const int row = i / a.d_c, c = i % a.d_c;
+    const int b = b0 + row / G, h = g * G + row % G;
+    const int first = a.sched.seq_first[b], np = a.sched.seq_np[b];
+    const float M = s_M[row];
+    float num = 0.f;
+    for (int j = 0; j < np; ++j) {
+      const size_t pj = (size_t)(first + j) * a.H + h;
+      num += exp2f(a.mlpart[pj * 2] - M) * a.opart[pj * a.d_c + c];
+    }
+    s_o[i] = num * s_inv[row];
+  }
+  __syncthreads();
+  // o[row][d] = sum_c O_lat[row][c] W_uv[g][c][d]; each thread owns one d for a set of rows
   const T* W = (const T*)a.W_uv + (size_t)g * a.d_c * a.dh;
-  for (int i = threadIdx.x; i < rows * a.dh; i += blockDim.x) {
-    int row = i / a.dh, d = i % a.dh;
-    float acc = 0.f;
-    const float* o = s_o + row * a.d_c;
-    for (int c = 0; c < a.d_c; ++c) acc += o[c] * to_f32(W[(size_t)c * a.dh + d]);
-    int b = b0 + row / G, h = g * G + row % G;
-    ((T*)a.out)[((size_t)b * a.H + h) * a.dh + d] = from_f32<T>(acc);
+  constexpr int kRows = 8;
+  for (int i = threadIdx.x; i < a.dh * ((rows + kRows - 1) / kRows); i += blockDim.x) {
+    const int d = i % a.dh, r0 = (i / a.dh) * kRows;
+    float acc[kRows];
+#pragma unroll
+    for (int k = 0; k < kRows; ++k) acc[k] = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < a.d_c; ++c) {
+      const float wv = to_f32(W[(size_t)c * a.dh + d]);
+#pragma unroll
+      for (int k = 0; k < kRows; ++k)
+        if (r0 + k < rows) acc[k] += s_o[(r0 + k) * a.d_c + c] * wv;
+    }
+#pragma unroll
+    for (int k = 0; k < kRows; ++k) {
+      const int row = r0 + k;
+      if (row >= rows) break;
+      const int b = b0 + row / G, h = g * G + row % G;
+      ((T*)a.out)[((size_t)b * a.H + h) * a.dh + d] = from_f32<T>(acc[k]);
+    }
   }
 }
 
@@ -312,7 +345,11 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
     if (e != cudaSuccess) return e;
     if (p.opt_events) cudaEventRecord((cudaEvent_t)p.opt_events[1], s);
   } else {
-    return cudaErrorNotSupported;
+    if (p.opt_events) cudaEventRecord((cudaEvent_t)p.opt_events[0], s);
+    e = mla_launch_decode_tc(p, c, B, sched, base + L.off_qlat, (float*)(base + L.off_opart),
+                             (float*)(base + L.off_mlpart), L.G, s);
+    if (e != cudaSuccess) return e;
+    if (p.opt_events) cudaEventRecord((cudaEvent_t)p.opt_events[1], s);
   }
   // 3. merge the splits and apply W_uv
   CombineArgs ca;
@@ -321,7 +358,7 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
   ca.sched = sched; ca.W_uv = p.W_uv; ca.out = out;
   ca.bchunk = max(1, 8 / G);
   int cchunks = (B + ca.bchunk - 1) / ca.bchunk;
-  size_t smem_c = (size_t)ca.bchunk * G * cfg.d_c * sizeof(float);
+  size_t smem_c = (size_t)ca.bchunk * G * (cfg.d_c + 2) * sizeof(float);
   combine_kernel<T><<<cfg.n_kv_heads * cchunks, 256, smem_c, s>>>(ca);
   return cudaGetLastError();
 }
@@ -330,12 +367,12 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-DecodeLayout mla_decode_layout(const mla_plan& p, int B) {
+DecodeLayout mla_decode_layout(const mla_plan& p, int B, int kernel) {
   const mla_config_t& cfg = p.cfg;
   DecodeLayout L;
-  L.kernel = 1;
-  L.tile = mla::kSimtTile;
-  L.G = p.opt_splits > 0 ? p.opt_splits : 2 * p.num_sms;
+  L.kernel = kernel;
+  L.tile = kernel == 2 ? 64 : mla::kSimtTile;
+  L.G = p.opt_splits > 0 ? p.opt_splits : (kernel == 2 ? p.num_sms : 2 * p.num_sms);
   L.P = B + L.G;
   L.K = cfg.d_c + p.R;
   const int H = cfg.n_heads;

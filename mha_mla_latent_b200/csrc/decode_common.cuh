@@ -12,17 +12,43 @@
 
 namespace mla {
 
+// Block-wide exclusive scan of one int per thread (blockDim.x a multiple of 32, <= 1024).
+// Returns the exclusive prefix; *total receives the block sum.  Uses s_warp[32].
+__device__ inline int block_exscan(int v, int* total, int* s_warp) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int wv = lane < nw ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, wv, o);
+      if (lane >= o) wv += y;
+    }
+    s_warp[lane] = wv;  // inclusive warp totals
+  }
+  __syncthreads();
+  const int base = wid > 0 ? s_warp[wid - 1] : 0;
+  *total = s_warp[nw - 1];
+  __syncthreads();
+  return base + x - v;
+}
+
 // Single-block schedule builder.  Must be run by one whole CTA.
 __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int B, int T_cap,
                                       int tile, int G, Sched s, int32_t* err) {
-  __shared__ int32_t s_carry[2];
-  __shared__ int32_t s_tot;
+  __shared__ int s_warp[32];
   const int tid = threadIdx.x, nt = blockDim.x;
-  // 1. tiles per sequence and exclusive prefix sums (tiles and non-empty count).
-  if (tid == 0) { s_carry[0] = 0; s_carry[1] = 0; }
-  __syncthreads();
+  // 1. tiles per sequence; exclusive prefix sums of tiles and of non-empty sequences
+  int carry_t = 0, carry_ne = 0;
   for (int base = 0; base < B; base += nt) {
-    int b = base + tid;
+    const int b = base + tid;
     int nti = 0;
     if (b < B) {
       int L = seq_lens[b];
@@ -32,48 +58,48 @@ __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int 
       s.seq_np[b] = 0;
       s.seq_first[b] = 0;
     }
-    // serial scan by thread 0 over this chunk (B is small compared to the decode work)
-    __syncthreads();
-    if (tid == 0) {
-      int c0 = s_carry[0], c1 = s_carry[1];
-      for (int i = base; i < min(B, base + nt); ++i) {
-        s.seq_tile0[i] = c0;
-        s.seq_ne[i] = c1;
-        c0 += s.seq_ntiles[i];
-        c1 += s.seq_ntiles[i] > 0 ? 1 : 0;
-      }
-      s_carry[0] = c0; s_carry[1] = c1;
+    int tot_t, tot_ne;
+    const int ex_t = block_exscan(nti, &tot_t, s_warp);
+    const int ex_ne = block_exscan(nti > 0 ? 1 : 0, &tot_ne, s_warp);
+    if (b < B) {
+      s.seq_tile0[b] = carry_t + ex_t;
+      s.seq_ne[b] = carry_ne + ex_ne;
     }
-    __syncthreads();
+    carry_t += tot_t;
+    carry_ne += tot_ne;
   }
-  if (tid == 0) { s_tot = s_carry[0]; s.seq_ne[B] = s_carry[1]; }
+  if (tid == 0) s.seq_ne[B] = carry_ne;
   __syncthreads();
-  const long long T = s_tot;
+  const long long T = carry_t;
 
-  // sequence containing global tile t (t < T): last b with seq_tile0[b] <= t
+  // sequence containing global tile t (t < T): last b with seq_tile0[b] <= t; it is
+  // non-empty because empty sequences share their start with the next sequence
   auto seq_of = [&](long long t) {
-    int lo = 0, hi = B;  // first b with tile0 > t, in [0, B]
+    int lo = 0, hi = B;
     while (lo < hi) {
       int mid = (lo + hi) >> 1;
       if (s.seq_tile0[mid] > t) hi = mid; else lo = mid + 1;
     }
     return lo - 1;
   };
-  // 2. pieces per worker, 3. serial exclusive scan into worker_first.
-  for (int i = tid; i < G; i += nt) {
-    long long c0 = (long long)i * T / G, c1 = (long long)(i + 1) * T / G;
+  // 2./3. pieces per worker and their exclusive prefix (worker_first)
+  int carry_p = 0;
+  for (int base = 0; base < G; base += nt) {
+    const int i = base + tid;
     int np = 0;
-    if (c0 < c1) {
-      int b0 = seq_of(c0), b1 = seq_of(c1 - 1);
-      np = s.seq_ne[b1 + 1] - s.seq_ne[b0];
+    if (i < G) {
+      long long c0 = (long long)i * T / G, c1 = (long long)(i + 1) * T / G;
+      if (c0 < c1) {
+        int b0 = seq_of(c0), b1 = seq_of(c1 - 1);
+        np = s.seq_ne[b1 + 1] - s.seq_ne[b0];
+      }
     }
-    s.worker_first[i + 1] = np;
+    int tot;
+    const int ex = block_exscan(np, &tot, s_warp);
+    if (i < G) s.worker_first[i] = carry_p + ex;
+    carry_p += tot;
   }
-  __syncthreads();
-  if (tid == 0) {
-    s.worker_first[0] = 0;
-    for (int i = 0; i < G; ++i) s.worker_first[i + 1] += s.worker_first[i];
-  }
+  if (tid == 0) s.worker_first[G] = carry_p;
   __syncthreads();
   // 4. write pieces
   for (int i = tid; i < G; i += nt) {
@@ -98,7 +124,7 @@ __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int 
   }
   __syncthreads();
   // 5. per-sequence piece ranges (pieces are ordered by global tile, hence by sequence)
-  const int P = s.worker_first[G];
+  const int P = carry_p;
   for (int p = tid; p < P; p += nt) {
     int b = s.piece_b[p];
     if (p == 0 || s.piece_b[p - 1] != b) s.seq_first[b] = p;

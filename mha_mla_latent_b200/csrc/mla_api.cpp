@@ -205,7 +205,9 @@ mla_status_t mla_append(const mla_plan_t* plan, const void* x, const int32_t* se
 
 size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B) {
   if (!plan || B <= 0) return 0;
-  return mla_decode_layout(*plan, B).total;
+  size_t n = mla_decode_layout(*plan, B, 1).total;
+  if (mla_tc_capable(*plan)) n = std::max(n, mla_decode_layout(*plan, B, 2).total);
+  return n;
 }
 
 mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
@@ -217,8 +219,11 @@ mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache, const 
   if (B > cache->B) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace) || ((uintptr_t)seq_lens & 3))
     return MLA_ERR_ALIGNMENT;
-  if ((size_t)plan->cfg.n_heads * plan->cfg.d_c > 8192) return MLA_ERR_UNSUPPORTED;
-  DecodeLayout L = mla_decode_layout(*plan, B);
+  int kernel = 1;
+  if (plan->opt_kernel != 1 && mla_tc_supported(*plan, *cache)) kernel = 2;
+  if (plan->opt_kernel == 2 && kernel != 2) return MLA_ERR_UNSUPPORTED;
+  if (kernel == 1 && (size_t)plan->cfg.n_heads * plan->cfg.d_c > 8192) return MLA_ERR_UNSUPPORTED;
+  DecodeLayout L = mla_decode_layout(*plan, B, kernel);
   if (ws_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
   return cuda_status(mla_launch_decode(*plan, *cache, seq_lens, q, B, out, workspace, L,
                                        (cudaStream_t)stream));

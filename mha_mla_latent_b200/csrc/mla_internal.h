@@ -53,7 +53,11 @@ struct Sched {
   int32_t* piece_t1;      // [P] token end (exclusive)
 };
 
-DecodeLayout mla_decode_layout(const mla_plan& p, int B);
+DecodeLayout mla_decode_layout(const mla_plan& p, int B, int kernel);
+bool mla_tc_supported(const mla_plan& p, const mla_cache_t& c);
+bool mla_tc_capable(const mla_plan& p);   // shape/dtype allow the tensor-core kernel
+cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, int B, const Sched& sched,
+                                 const void* qcat, float* opart, float* mlpart, int G, cudaStream_t s);
 Sched mla_sched_view(const DecodeLayout& L, void* ws, int B);
 
 cudaError_t mla_launch_select_pairs(const mla_config_t& cfg, const void* q, const void* k, int T,
