@@ -310,6 +310,9 @@ def run_ours(args):
     torch.cuda.synchronize()
     clocks = sampler.stop()
     mla.mla_plan_set_option(plan, mla.MLA_OPT_PROFILE_EVENTS, 0)
+    dev_err = mla.mla_device_error(plan)
+    if dev_err:
+        raise RuntimeError(f"device error word {dev_err} after the timed region: result invalid")
     if world > 1:
         dist.barrier()
     total_ms = start.elapsed_time(end)
