@@ -167,6 +167,32 @@ MLA_API mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache
                         const void* q, int32_t B, void* out, void* workspace, size_t ws_bytes,
                         void* stream);
 
+/* Size of the static scratch array behind mla_decode_noalloc (bytes, per device). */
+#define MLA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* mla_decode without any device allocation, by the caller or by the library.
+ * The paper has no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory when they decode: a server whose memory pool is carved up
+ * once at start-up, a real-time loop that must not call the allocator (an allocation
+ * can synchronise the device and has no bounded latency), or a host program that only
+ * links this C ABI and has no allocator of its own.  Arguments, outputs and results are
+ * those of mla_decode, minus the workspace: the workspace is a static device array of
+ * MLA_NOALLOC_SCRATCH_BYTES compiled into the library, present on every GPU that loads
+ * the library until the process exits.
+ *   - Returns MLA_ERR_WORKSPACE_TOO_SMALL when the batch needs more workspace than the
+ *     array holds (mla_decode_workspace_bytes(plan, B) tells how much a batch needs).
+ *   - The first call on a device looks up the array's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - The plan must belong to the current device (MLA_ERR_INVALID_ARG otherwise).
+ *   - All calls share the one array and each leaves its contents behind.  Nothing in
+ *     it needs clearing: every call writes each part of the workspace before reading it.
+ *     Calls whose work overlaps on the GPU (different streams, or different plans on
+ *     concurrent streams) race on the array; serialise them, e.g. on one stream.
+ *   - It calls no cudaMalloc/cudaFree or other allocating routine. */
+MLA_API mla_status_t mla_decode_noalloc(const mla_plan_t* plan, const mla_cache_t* cache,
+                                        const int32_t* seq_lens, const void* q, int32_t B, void* out,
+                                        void* stream);
+
 /* Synchronise the device, read and clear the plan's device error word.
  * *code receives 0 (none) or a bitwise OR of MLA_DEVERR_* values.
  * Returns MLA_OK, or MLA_ERR_CUDA when the synchronisation itself failed. */

@@ -24,8 +24,9 @@ MLA_DEVERR_SEQ_LEN, MLA_DEVERR_APPEND_SLOT, MLA_DEVERR_TIMEOUT = 1, 2, 4
 EXPORTED = (
     "mla_status_string", "mla_version", "mla_cache_bytes_per_token", "mla_select_pairs",
     "mla_plan_create", "mla_plan_destroy", "mla_plan_set_option", "mla_append",
-    "mla_decode_workspace_bytes", "mla_decode", "mla_device_error",
+    "mla_decode_workspace_bytes", "mla_decode", "mla_device_error", "mla_decode_noalloc",
 )
+MLA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class MlaConfig(ctypes.Structure):
@@ -65,6 +66,7 @@ def _load():
         "mla_decode_workspace_bytes": (sz, [vp, i32]),
         "mla_decode": (i32, [vp, cachep, vp, vp, i32, vp, vp, sz, vp]),
         "mla_device_error": (i32, [vp, ctypes.POINTER(i32)]),
+        "mla_decode_noalloc": (i32, [vp, cachep, vp, vp, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -191,6 +193,15 @@ def mla_decode(plan: Plan, cache: MlaCache, seq_lens, q, out, workspace, stream=
                          _ptr(out), _ptr(workspace), ws_bytes, _stream(stream))
     if check:
         _check(st, "mla_decode")
+    return st
+
+
+def mla_decode_noalloc(plan: Plan, cache: MlaCache, seq_lens, q, out, stream=None, check=True):
+    """mla_decode with the library's static scratch array as workspace (no allocation)."""
+    st = _lib.mla_decode_noalloc(plan.handle, ctypes.byref(cache), _ptr(seq_lens), _ptr(q), int(q.shape[0]),
+                                 _ptr(out), _stream(stream))
+    if check:
+        _check(st, "mla_decode_noalloc")
     return st
 
 

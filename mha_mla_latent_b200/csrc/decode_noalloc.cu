@@ -1,0 +1,69 @@
+// mla_decode_noalloc: the decode step with its workspace in a static device array.
+//
+// Some callers cannot allocate device memory at decode time: a serving process whose
+// memory pool is carved up once at start-up, a real-time loop that must not call the
+// allocator (cudaMalloc can synchronise the device and take unbounded time), or a host
+// program that drives this library through its C ABI alone and has no allocator of its
+// own.  For them this entry point needs no workspace argument: it uses a fixed scratch
+// array compiled into the library (kNoAllocScratchBytes on every GPU that loads the
+// library, held until the process exits).  Everything else matches mla_decode.
+#include <mutex>
+
+#include "mla_internal.h"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;   // 16 MiB
+static_assert(kNoAllocScratchBytes == (size_t)MLA_NOALLOC_SCRATCH_BYTES, "header and library disagree");
+
+// The scratch array.  In host code its name is only a stand-in symbol, never a device
+// address: the device address is obtained per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_once[kMaxDevices];
+void* g_scratch[kMaxDevices];
+cudaError_t g_scratch_err[kMaxDevices];
+
+// Runs once per device, with that device current.
+void resolve_scratch(int dev) {
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  g_scratch_err[dev] = e;
+  g_scratch[dev] = e == cudaSuccess ? p : nullptr;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace
+
+extern "C" mla_status_t mla_decode_noalloc(const mla_plan_t* plan, const mla_cache_t* cache,
+                                           const int32_t* seq_lens, const void* q, int32_t B, void* out,
+                                           void* stream) {
+  if (!plan || !cache || !seq_lens || !q || !out || B <= 0) return MLA_ERR_INVALID_ARG;
+  const mla_config_t& cfg = plan->cfg;
+  const bool int4 = cfg.cache_kind == MLA_CACHE_INT4_G32;
+  if (!cache->c_kv || cache->B <= 0 || cache->T_cap <= 0 || B > cache->B) return MLA_ERR_INVALID_ARG;
+  if (int4 != (cache->c_scales != nullptr)) return MLA_ERR_INVALID_ARG;
+  if (cfg.r_pairs > 0 && !cache->k_rope) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(cache->c_kv) || (cache->c_scales && !aligned16(cache->c_scales)) ||
+      (cache->k_rope && !aligned16(cache->k_rope)) || !aligned16(q) || !aligned16(out) ||
+      ((uintptr_t)seq_lens & 3))
+    return MLA_ERR_ALIGNMENT;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev != plan->device) return MLA_ERR_INVALID_ARG;   // the plan's weights live on its device
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  std::call_once(g_once[dev], resolve_scratch, dev);
+  if (g_scratch_err[dev] != cudaSuccess || !g_scratch[dev]) return MLA_ERR_CUDA;
+
+  int kernel = 1;
+  if (plan->opt_kernel != 1 && mla_tc_supported(*plan, *cache)) kernel = 2;
+  if (plan->opt_kernel == 2 && kernel != 2) return MLA_ERR_UNSUPPORTED;
+  if (kernel == 1 && (size_t)cfg.n_heads * cfg.d_c > 8192) return MLA_ERR_UNSUPPORTED;
+  const DecodeLayout L = mla_decode_layout(*plan, B, kernel);
+  if (L.total > kNoAllocScratchBytes) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  const cudaError_t e =
+      mla_launch_decode(*plan, *cache, seq_lens, q, B, out, g_scratch[dev], L, (cudaStream_t)stream);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
