@@ -223,8 +223,6 @@ def run_ours(args):
     conv = convert_layer(cfg, gen.to_torch(w["W_k"], wl.dtype, dev), gen.to_torch(w["W_v"], wl.dtype, dev),
                          gen.to_torch(q_cal, wl.dtype, dev), gen.to_torch(k_cal, wl.dtype, dev))
     plan = plan_from_converted(cfg, conv)
-    if args.kernel:
-        mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, args.kernel)
     torch.cuda.synchronize()
     conversion_s = time.perf_counter() - t0
 
@@ -264,6 +262,16 @@ def run_ours(args):
     out = torch.empty_like(q)
     ws = workspace(plan, B, dev)
     stream = torch.cuda.current_stream(dev)
+
+    # which split-K kernel runs: the tcgen05 kernel where the shape allows it
+    kernel_used = args.kernel
+    if kernel_used == 0:
+        mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, 2)
+        st = mla.mla_decode(plan, caches[0].struct, seq_lens, q, out, ws, stream=stream, check=False)
+        kernel_used = 2 if st == mla.MLA_OK else 1
+    mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, kernel_used)
+    torch.cuda.synchronize()
+    assert mla.mla_device_error(plan) == 0
 
     def step(i):
         c = caches[i % n_rep].struct
@@ -366,7 +374,8 @@ def run_ours(args):
     wuk = wl.n_kv_heads * wl.d_c * (wl.head_dim - 2 * wl.r_pairs) * (2 if wl.dtype == "bf16" else 4)
     wuv = wl.n_kv_heads * wl.d_c * wl.head_dim * (2 if wl.dtype == "bf16" else 4)
     decode_frac = (cache_bytes + wuk + wuv) / (decode_ms * 1e-3) / 1e9 / peak
-    kernel_name = "tcgen05 split-K latent attention" if args.kernel == 2 else "split-K latent attention"
+    kernel_name = ("tcgen05 split-K latent attention (decode_tc_kernel)" if kernel_used == 2
+                   else "CUDA-core split-K latent attention (decode_simt_kernel)")
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,

@@ -81,7 +81,10 @@ typedef struct {
 /* Caller-owned cache, device memory, capacity T_cap tokens per sequence.
  *   c_kv     SAME: [B][T_cap][d_c] dtype;  INT4: [B][T_cap][d_c/2] uint8 codes
  *   c_scales INT4: [B][T_cap][d_c/32] fp16;  SAME: must be NULL
- *   k_rope   [B][T_cap][n_kv][2r] dtype (may be NULL when r == 0)          */
+ *   k_rope   [B][ceil(T_cap/32)][n_kv][32][2r] dtype (may be NULL when r == 0): the kept
+ *            RoPE key dims in blocks of 32 tokens, KV-head-major inside a block, so the
+ *            2r dims of one KV head for 32 consecutive tokens are contiguous; element
+ *            (b, t, g, j) sits at ((b*ceil(T_cap/32) + t/32)*n_kv + g)*32*2r + (t%32)*2r + j */
 typedef struct {
   void* c_kv;
   void* c_scales;

@@ -12,7 +12,7 @@ import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "lib", "libmla_b200.so")
+LIB_PATH = os.environ.get("MLA_B200_LIB", os.path.join(_PKG, "lib", "libmla_b200.so"))
 
 MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_ALIGNMENT = 0, 1, 2, 3
 MLA_ERR_WORKSPACE_TOO_SMALL, MLA_ERR_CUDA, MLA_ERR_DEVICE = 4, 5, 6
@@ -149,7 +149,8 @@ class Plan:
 
     def close(self):
         if getattr(self, "handle", None):
-            _lib.mla_plan_destroy(self.handle)
+            if _lib is not None:   # module globals may already be gone at interpreter exit
+                _lib.mla_plan_destroy(self.handle)
             self.handle = None
 
 

@@ -22,9 +22,24 @@ class LatentCache:
             self.c_kv = torch.zeros(B, T_cap, cfg.d_c, dtype=dt, device=device)
             self.c_scales = None
         R = cfg.n_kv_heads * 2 * cfg.r_pairs
-        self.k_rope = torch.zeros(B, T_cap, cfg.n_kv_heads, 2 * cfg.r_pairs, dtype=dt, device=device) \
-            if R > 0 else None
+        # blocked layout [B][ceil(T_cap/32)][n_kv][32][2r] (see mla_cache_t)
+        self.k_rope = torch.zeros(B, (T_cap + 31) // 32, cfg.n_kv_heads, 32, 2 * cfg.r_pairs, dtype=dt,
+                                  device=device) if R > 0 else None
         self.struct = _lib.cache_struct(self.c_kv, self.c_scales, self.k_rope, B, T_cap)
+
+    def _kr_index(self, t0: int, t1: int):
+        t = torch.arange(t0, t1, device=self.k_rope.device)
+        return t // 32, t % 32
+
+    def k_rope_tokens(self, b: int, t0: int, t1: int) -> torch.Tensor:
+        """RoPE key dims of tokens [t0, t1) of sequence b, as [t1-t0][n_kv][2r] (a copy)."""
+        blk, row = self._kr_index(t0, t1)
+        return self.k_rope[b].permute(0, 2, 1, 3)[blk, row]
+
+    def set_k_rope_tokens(self, b: int, t0: int, values: torch.Tensor) -> None:
+        """Write [n][n_kv][2r] RoPE key dims as tokens [t0, t0+n) of sequence b."""
+        blk, row = self._kr_index(t0, t0 + values.shape[0])
+        self.k_rope[b].permute(0, 2, 1, 3)[blk, row] = values.to(self.k_rope.dtype)
 
     def nbytes_used(self, seq_lens) -> int:
         per_tok = _lib.mla_cache_bytes_per_token(self.cfg)

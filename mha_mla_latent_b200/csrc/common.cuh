@@ -7,6 +7,35 @@
 
 #include "mla_internal.h"
 
+#ifdef MLA_TC_TRACE
+// Development builds only (-DMLA_TC_TRACE): each CTA's start and end %globaltimer stamps,
+// per kernel id, in a translation-unit-local array with an exported reader.
+#define MLA_KSPAN_DEFINE(name)                                                                  \
+  static __device__ unsigned long long g_kspan[8 * 1024 * 2];                                   \
+  extern "C" __attribute__((visibility("default"))) int mla_kspan_read_##name(unsigned long long* h) { \
+    return cudaMemcpyFromSymbol(h, g_kspan, sizeof(g_kspan)) == cudaSuccess ? 8 * 1024 * 2 : -1;  \
+  }
+#define MLA_KSPAN(k)                                                                            \
+  struct KSpanT {                                                                               \
+    unsigned long long t0;                                                                      \
+    __device__ static unsigned long long now() {                                                \
+      unsigned long long t;                                                                     \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));                                     \
+      return t;                                                                                 \
+    }                                                                                           \
+    __device__ ~KSpanT() {                                                                      \
+      const int blk = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);           \
+      if (threadIdx.x == 0 && blk < 1024) {                                                     \
+        g_kspan[((k) * 1024 + blk) * 2] = t0;                                                   \
+        g_kspan[((k) * 1024 + blk) * 2 + 1] = now();                                            \
+      }                                                                                         \
+    }                                                                                           \
+  } kspan_{KSpanT::now()}
+#else
+#define MLA_KSPAN_DEFINE(name)
+#define MLA_KSPAN(k) do { } while (0)
+#endif
+
 namespace mla {
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
@@ -24,6 +53,10 @@ template <> __device__ __forceinline__ float from_f64<float>(double v) { return 
 template <> __device__ __forceinline__ __nv_bfloat16 from_f64<__nv_bfloat16>(double v) {
   return __double2bfloat16(v);  // single round-to-nearest-even from double
 }
+
+// Read-only global load (non-coherent path): tells the compiler the source cannot alias
+// shared memory, so loads are not serialised behind shared-memory stores.
+template <typename T> __device__ __forceinline__ float ldg_f32(const T* p) { return to_f32(__ldg(p)); }
 
 __device__ __forceinline__ void raise_error(int32_t* err, int32_t bit) {
   if (err) atomicOr(err, bit);

@@ -7,7 +7,11 @@
 // scores the NoPE part directly against c_kv; the probability-weighted latent is taken
 // through W_uv after the softmax sum.  Scores are kept in log2 units (the query is
 // pre-scaled by log2(e)/sqrt(d_h)) so the softmax uses exp2.
+#include <algorithm>
+
 #include "decode_common.cuh"
+
+MLA_KSPAN_DEFINE(decode)
 
 namespace mla {
 
@@ -28,79 +32,157 @@ struct AbsorbArgs {
   Sched sched;
   int tile, G;
   int32_t* err;
+  int smem_ints;              // dynamic shared memory of the CTA, in ints
+  int vec_ok;                 // W_uk rows and q rows allow 16-byte loads
 };
 
-constexpr int kAbsMaxRows = 16;   // (b, h) rows per CTA
+constexpr int kAbsRows = 16;   // (b, h) rows per CTA
+constexpr int kAbsCols = 64;   // latent columns per CTA
 
+// grid: n_kv * (column chunks) * (row chunks) CTAs, plus one CTA that builds the schedule.
+// Each CTA stages its slice of W_uk[g] (all NoPE dims x 64 latent columns) and the NoPE
+// query dims of its rows in shared memory, then each thread accumulates 4 rows of one
+// latent column.
 template <typename T>
 __global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
-  const int nchunks = (a.B + a.bchunk - 1) / a.bchunk;
-  if (blockIdx.x == a.n_kv * nchunks) {  // the last CTA builds the split-K schedule
-    build_schedule(a.seq_lens, a.B, a.T_cap, a.tile, a.G, a.sched, a.err);
+  MLA_KSPAN(0);
+  const int G = a.H / a.n_kv;
+  const int rows_total = a.B * G;
+  const int n_rc = (rows_total + kAbsRows - 1) / kAbsRows;
+  const int n_cc = (a.d_c + kAbsCols - 1) / kAbsCols;
+  if (blockIdx.x == a.n_kv * n_cc * n_rc) {  // the last CTA builds the split-K schedule
+    extern __shared__ float sm_sched[];
+    build_schedule(a.seq_lens, a.B, a.T_cap, a.tile, a.G, a.sched, a.err, reinterpret_cast<int32_t*>(sm_sched),
+                   a.smem_ints);
     return;
   }
-  const int g = blockIdx.x % a.n_kv, chunk = blockIdx.x / a.n_kv;
-  const int G = a.H / a.n_kv;
-  const int b0 = chunk * a.bchunk;
-  const int nb = min(a.bchunk, a.B - b0);
-  const int rows = nb * G;
+  const int g = blockIdx.x % a.n_kv;
+  const int cc = (blockIdx.x / a.n_kv) % n_cc;
+  const int rc = blockIdx.x / (a.n_kv * n_cc);
+  const int row0 = rc * kAbsRows;
+  const int rows = min(kAbsRows, rows_total - row0);
   extern __shared__ float sm[];
-  float* qn = sm;                           // [rows][dn]
+  float* s_w = sm;                          // [dn][kAbsCols]
+  float* s_q = s_w + a.dn * kAbsCols;       // [kAbsRows][dn]
   const float scale = kLog2e * rsqrtf((float)a.dh);
   const T* q = (const T*)a.q;
-  for (int i = threadIdx.x; i < rows * a.dn; i += blockDim.x) {
-    int row = i / a.dn, j = i % a.dn;
-    int b = b0 + row / G, h = g * G + row % G;
-    qn[i] = to_f32(q[((size_t)b * a.H + h) * a.dh + a.nope_idx[g * a.dn + j]]);
-  }
-  // RoPE part: rotate the kept pairs at position L-1 (angle in double), scale.
-  for (int i = threadIdx.x; i < rows * a.r; i += blockDim.x) {
-    int row = i / a.r, j = i % a.r;
-    int b = b0 + row / G, h = g * G + row % G;
-    int L = a.seq_lens[b];
-    int p = (L >= 1 && L <= a.T_cap) ? L - 1 : 0;
-    int k = a.rope_pair[g * a.r + j];
-    const T* qp = q + ((size_t)b * a.H + h) * a.dh + 2 * k;
-    double x0 = to_f32(qp[0]), x1 = to_f32(qp[1]);
-    double sn, cs;
-    sincos((double)p * a.theta[k], &sn, &cs);
-    float o0 = (float)((x0 * cs - x1 * sn) * (double)scale);
-    float o1 = (float)((x0 * sn + x1 * cs) * (double)scale);
-    size_t bh = (size_t)b * a.H + h;
-    if (a.qrope) { a.qrope[bh * 2 * a.r + 2 * j] = o0; a.qrope[bh * 2 * a.r + 2 * j + 1] = o1; }
-    if (a.qcat) {
-      a.qcat[bh * a.K + a.d_c + g * 2 * a.r + 2 * j] = __float2bfloat16_rn(o0);
-      a.qcat[bh * a.K + a.d_c + g * 2 * a.r + 2 * j + 1] = __float2bfloat16_rn(o1);
+  const T* W = (const T*)a.W_ukT + (size_t)g * a.dn * a.d_c;
+  const int c0 = cc * kAbsCols;
+  float* s_qraw = s_q + kAbsRows * a.dn;    // [kAbsRows][dh]
+  // all loads of the CTA are issued before any is used (one memory round trip)
+  constexpr int VEC = 16 / sizeof(T);
+  const bool vec = a.vec_ok && (c0 + kAbsCols <= a.d_c);
+  if (vec) {
+    constexpr int kMaxW = 8;                 // dn <= 256: dn * 64 / VEC / 256 <= 8 (bf16)
+    const int nw = a.dn * (kAbsCols / VEC);
+    uint4 wr[kMaxW];
+#pragma unroll
+    for (int k = 0; k < kMaxW; ++k) {
+      const int v = threadIdx.x + 256 * k;
+      if (v < nw) {
+        const int j = v / (kAbsCols / VEC), part = v % (kAbsCols / VEC);
+        wr[k] = __ldg(reinterpret_cast<const uint4*>(W + (size_t)j * a.d_c + c0 + part * VEC));
+      }
     }
-  }
-  if (a.qcat) {  // zero the other KV heads' RoPE slots of the concatenated query row
-    for (int i = threadIdx.x; i < rows * a.R; i += blockDim.x) {
-      int row = i / a.R, j = i % a.R;
-      if (j / (2 * a.r) == g) continue;
-      size_t bh = (size_t)(b0 + row / G) * a.H + g * G + row % G;
-      a.qcat[bh * a.K + a.d_c + j] = __float2bfloat16_rn(0.f);
+    const int nq = rows * (a.dh / VEC);
+    uint4 qr[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int v = threadIdx.x + 256 * k;
+      if (v < nq) {
+        const int r = v / (a.dh / VEC), part = v % (a.dh / VEC);
+        const int row = row0 + r, b = row / G, h = g * G + row % G;
+        qr[k] = __ldg(reinterpret_cast<const uint4*>(q + ((size_t)b * a.H + h) * a.dh + part * VEC));
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxW; ++k) {
+      const int v = threadIdx.x + 256 * k;
+      if (v < nw) {
+        const int j = v / (kAbsCols / VEC), part = v % (kAbsCols / VEC);
+        const T* e = reinterpret_cast<const T*>(&wr[k]);
+#pragma unroll
+        for (int t = 0; t < VEC; ++t) s_w[j * kAbsCols + part * VEC + t] = to_f32(e[t]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int v = threadIdx.x + 256 * k;
+      if (v < nq) {
+        const int r = v / (a.dh / VEC), part = v % (a.dh / VEC);
+        const T* e = reinterpret_cast<const T*>(&qr[k]);
+#pragma unroll
+        for (int t = 0; t < VEC; ++t) s_qraw[r * a.dh + part * VEC + t] = to_f32(e[t]);
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < a.dn * kAbsCols; i += blockDim.x) {
+      const int j = i / kAbsCols, cl = i % kAbsCols;
+      s_w[i] = (c0 + cl < a.d_c) ? ldg_f32(W + (size_t)j * a.d_c + c0 + cl) : 0.f;
+    }
+    for (int i = threadIdx.x; i < rows * a.dh; i += blockDim.x) {
+      const int r = i / a.dh, e = i % a.dh;
+      const int row = row0 + r, b = row / G, h = g * G + row % G;
+      s_qraw[i] = ldg_f32(q + ((size_t)b * a.H + h) * a.dh + e);
     }
   }
   __syncthreads();
-  // Latent part: q_lat[row][c] = scale * sum_j qn[row][j] * W_uk[g][c][j].
-  const T* W = (const T*)a.W_ukT + (size_t)g * a.dn * a.d_c;
-  for (int c = threadIdx.x; c < a.d_c; c += blockDim.x) {
-    float acc[kAbsMaxRows];
-#pragma unroll
-    for (int i = 0; i < kAbsMaxRows; ++i) acc[i] = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < a.dn; ++j) {
-      float w = to_f32(W[(size_t)j * a.d_c + c]);
-#pragma unroll
-      for (int i = 0; i < kAbsMaxRows; ++i)
-        if (i < rows) acc[i] += qn[i * a.dn + j] * w;
+  for (int i = threadIdx.x; i < rows * a.dn; i += blockDim.x) {
+    const int r = i / a.dn, j = i % a.dn;
+    s_q[i] = s_qraw[r * a.dh + __ldg(a.nope_idx + g * a.dn + j)];
+  }
+  if (cc == 0) {
+    // RoPE part: rotate the kept pairs at position L-1 (angle in double), scale.
+    for (int i = threadIdx.x; i < rows * a.r; i += blockDim.x) {
+      const int r = i / a.r, j = i % a.r;
+      const int row = row0 + r, b = row / G, h = g * G + row % G;
+      const int L = a.seq_lens[b];
+      const int p = (L >= 1 && L <= a.T_cap) ? L - 1 : 0;
+      const int k = a.rope_pair[g * a.r + j];
+      const double x0 = s_qraw[r * a.dh + 2 * k], x1 = s_qraw[r * a.dh + 2 * k + 1];
+      double sn, cs;
+      sincos((double)p * a.theta[k], &sn, &cs);
+      const float o0 = (float)((x0 * cs - x1 * sn) * (double)scale);
+      const float o1 = (float)((x0 * sn + x1 * cs) * (double)scale);
+      const size_t bh = (size_t)b * a.H + h;
+      if (a.qrope) { a.qrope[bh * 2 * a.r + 2 * j] = o0; a.qrope[bh * 2 * a.r + 2 * j + 1] = o1; }
+      if (a.qcat && a.K > a.d_c) {
+        a.qcat[bh * a.K + a.d_c + g * 2 * a.r + 2 * j] = __float2bfloat16_rn(o0);
+        a.qcat[bh * a.K + a.d_c + g * 2 * a.r + 2 * j + 1] = __float2bfloat16_rn(o1);
+      }
     }
+    if (a.qcat && a.K > a.d_c) {  // zero the other KV heads' RoPE slots of a concatenated row
+      for (int i = threadIdx.x; i < rows * a.R; i += blockDim.x) {
+        const int r = i / a.R, j = i % a.R;
+        if (j / (2 * a.r) == g) continue;
+        const int row = row0 + r;
+        const size_t bh = (size_t)(row / G) * a.H + g * G + row % G;
+        a.qcat[bh * a.K + a.d_c + j] = __float2bfloat16_rn(0.f);
+      }
+    }
+  }
+  __syncthreads();
+  // q_lat[row][c] = scale * sum_j q_nope[row][j] * W_uk[g][c][j]
+  const int cl = threadIdx.x % kAbsCols, rg = threadIdx.x / kAbsCols;  // 4 row groups
+  const int c = c0 + cl;
+  float acc[kAbsRows / 4];
 #pragma unroll
-    for (int i = 0; i < kAbsMaxRows; ++i) {
-      if (i >= rows) break;
-      size_t bh = (size_t)(b0 + i / G) * a.H + g * G + i % G;
-      if (a.qlat) a.qlat[bh * a.d_c + c] = acc[i] * scale;
-      if (a.qcat) a.qcat[bh * a.K + c] = __float2bfloat16_rn(acc[i] * scale);
+  for (int k = 0; k < kAbsRows / 4; ++k) acc[k] = 0.f;
+#pragma unroll 4
+  for (int j = 0; j < a.dn; ++j) {
+    const float wv = s_w[j * kAbsCols + cl];
+#pragma unroll
+    for (int k = 0; k < kAbsRows / 4; ++k) acc[k] += s_q[(rg * (kAbsRows / 4) + k) * a.dn + j] * wv;
+  }
+  if (c < a.d_c) {
+#pragma unroll
+    for (int k = 0; k < kAbsRows / 4; ++k) {
+      const int r = rg * (kAbsRows / 4) + k;
+      if (r >= rows) break;
+      const int row = row0 + r;
+      const size_t bh = (size_t)(row / G) * a.H + g * G + row % G;
+      if (a.qlat) a.qlat[bh * a.d_c + c] = acc[k] * scale;
+      if (a.qcat) a.qcat[bh * a.K + c] = __float2bfloat16_rn(acc[k] * scale);
     }
   }
 }
@@ -111,8 +193,9 @@ struct DecodeArgs {
   int B, H, n_kv, r, d_c, R;
   const float* qlat;
   const float* qrope;
-  float* opart;     // [P][H][d_c]
-  float* mlpart;    // [P][H][2]
+  float* opart;     // [H][P][d_c]
+  float* mlpart;    // [H][P][2]
+  int P;            // piece capacity
   Sched sched;
 };
 
@@ -121,6 +204,7 @@ constexpr int kSimtMaxE = 32;   // H*d_c / 256 owned accumulators per thread
 
 template <typename T, bool INT4>
 __global__ void __launch_bounds__(256) decode_simt_kernel(DecodeArgs a) {
+  MLA_KSPAN(1);
   const int H = a.H, dc = a.d_c, R = a.R, r2 = 2 * a.r;
   const int G = H / a.n_kv;
   extern __shared__ float sm[];
@@ -163,7 +247,8 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(DecodeArgs a) {
       }
       for (int i = tid; i < n * R; i += 256) {
         int tt = i / R, j = i % R;
-        s_kr[tt * (R + 1) + j] = to_f32(((const T*)a.cache.k_rope)[(slot0 + tt) * R + j]);
+        s_kr[tt * (R + 1) + j] =
+            to_f32(((const T*)a.cache.k_rope)[mla_kr_offset(b, t + tt, j / r2, j % r2, a.cache.T_cap, a.n_kv, r2)]);
       }
       __syncthreads();
       for (int i = tid; i < n * H; i += 256) {
@@ -208,11 +293,11 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(DecodeArgs a) {
     for (int e = 0; e < kSimtMaxE; ++e) {
       if (e >= nE) break;
       int idx = tid + 256 * e;
-      if (idx < H * dc) a.opart[(size_t)pc * H * dc + idx] = O[e];
+      if (idx < H * dc) a.opart[((size_t)(idx / dc) * a.P + pc) * dc + idx % dc] = O[e];
     }
     if (tid < H) {
-      a.mlpart[((size_t)pc * H + tid) * 2] = s_m[tid];
-      a.mlpart[((size_t)pc * H + tid) * 2 + 1] = s_l[tid];
+      a.mlpart[((size_t)tid * a.P + pc) * 2] = s_m[tid];
+      a.mlpart[((size_t)tid * a.P + pc) * 2 + 1] = s_l[tid];
     }
     __syncthreads();
   }
@@ -227,70 +312,111 @@ struct CombineArgs {
   const void* W_uv;   // [n_kv][d_c][dh]
   void* out;          // [B][H][dh]
   int bchunk;
+  int max_pieces;     // upper bound on pieces per sequence (G + 1)
+  int P;              // piece capacity of the partial arrays [H][P]
 };
 
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  MLA_KSPAN(2);
   const int g = blockIdx.x % a.n_kv, chunk = blockIdx.x / a.n_kv;
   const int G = a.H / a.n_kv;
   const int b0 = chunk * a.bchunk;
   const int nb = min(a.bchunk, a.B - b0);
   const int rows = nb * G;
   extern __shared__ float sm[];
-  float* s_o = sm;                    // [rows][d_c]
-  float* s_M = s_o + rows * a.d_c;    // [rows] merged running max
-  float* s_inv = s_M + rows;          // [rows] 1 / merged sum
+  float* s_o = sm;                      // [rows][d_c] merged latent
+  float* s_wt = s_o + rows * a.d_c;     // [rows][max_pieces] merge weights
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
-  // per (b, h): M = max_j m_j, 1 / sum_j 2^(m_j - M) l_j   (one warp per row)
+  // 1. per (b, h): merge weights 2^(m_j - M) / sum_j 2^(m_j - M) l_j of its pieces
+  //    (one warp per row; lanes stride over the pieces)
   for (int row = warp; row < rows; row += nwarp) {
     const int b = b0 + row / G, h = g * G + row % G;
     const int first = a.sched.seq_first[b], np = a.sched.seq_np[b];
     float M = -INFINITY;
-    for (int j = lane; j < np; j += 32) M = fmaxf(M, a.mlpart[((size_t)(first + j) * a.H + h) * 2]);
+    for (int j = lane; j < np; j += 32) M = fmaxf(M, __ldg(a.mlpart + ((size_t)h * a.P + first + j) * 2));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float den = 0.f;
     for (int j = lane; j < np; j += 32) {
-      const float* ml = a.mlpart + ((size_t)(first + j) * a.H + h) * 2;
-      den += exp2f(ml[0] - M) * ml[1];
+      const float* ml = a.mlpart + ((size_t)h * a.P + first + j) * 2;
+      const float wj = exp2f(__ldg(ml) - M);
+      s_wt[row * a.max_pieces + j] = wj;
+      den += wj * __ldg(ml + 1);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if (lane == 0) {
-      s_M[row] = M;
-      s_inv[row] = (np > 0 && den > 0.f) ? 1.f / den : 0.f;
-    }
+    const float inv = (np > 0 && den > 0.f) ? 1.f / den : 0.f;
+    __syncwarp();
+    for (int j = lane; j < np; j += 32) s_wt[row * a.max_pieces + j] *= inv;
   }
   __syncthreads();
-  // merged latent O_lat[row][c]
-  for (int i = threadIdx.x; i < rows * a.d_c; i += blockDim.x) {
-    const int row = i / a.d_c, c = i % a.d_c;
+  // 2. merged latent: each item is (row, 4 consecutive c); all pieces' loads issued together
+  const int c4n = a.d_c / 4;
+  for (int it = threadIdx.x; it < rows * c4n; it += blockDim.x) {
+    const int row = it / c4n, c4 = it % c4n;
     const int b = b0 + row / G, h = g * G + row % G;
     const int first = a.sched.seq_first[b], np = a.sched.seq_np[b];
-    const float M = s_M[row];
-    float num = 0.f;
-    for (int j = 0; j < np; ++j) {
-      const size_t pj = (size_t)(first + j) * a.H + h;
-      num += exp2f(a.mlpart[pj * 2] - M) * a.opart[pj * a.d_c + c];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < np; j0 += 8) {
+      float4 o[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (j0 + k < np)
+          o[k] = __ldg(reinterpret_cast<const float4*>(a.opart + ((size_t)h * a.P + first + j0 + k) * a.d_c) + c4);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (j0 + k < np) {
+          const float wgt = s_wt[row * a.max_pieces + j0 + k];
+          acc.x += wgt * o[k].x; acc.y += wgt * o[k].y; acc.z += wgt * o[k].z; acc.w += wgt * o[k].w;
+        }
     }
-    s_o[i] = num * s_inv[row];
+    *reinterpret_cast<float4*>(&s_o[row * a.d_c + c4 * 4]) = acc;
   }
   __syncthreads();
-  // o[row][d] = sum_c O_lat[row][c] W_uv[g][c][d]; each thread owns one d for a set of rows
+  // 3. o[row][d] = sum_c O_lat[row][c] W_uv[g][c][d], W_uv[g] staged in chunks of 64 latent
+  //    rows (one 16-byte load per thread and chunk row group, all issued before use)
   const T* W = (const T*)a.W_uv + (size_t)g * a.d_c * a.dh;
-  constexpr int kRows = 8;
-  for (int i = threadIdx.x; i < a.dh * ((rows + kRows - 1) / kRows); i += blockDim.x) {
-    const int d = i % a.dh, r0 = (i / a.dh) * kRows;
-    float acc[kRows];
+  float* s_w = s_wt + rows * a.max_pieces;   // [kWc][dh]
+  constexpr int kRows = 8, kWc = 64;
+  constexpr int VEC = 16 / sizeof(T);
+  const int n_items = a.dh * ((rows + kRows - 1) / kRows);
+  const int item = threadIdx.x;
+  const int d = item % a.dh, r0 = (item / a.dh) * kRows;
+  float acc[kRows];
 #pragma unroll
-    for (int k = 0; k < kRows; ++k) acc[k] = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < a.d_c; ++c) {
-      const float wv = to_f32(W[(size_t)c * a.dh + d]);
+  for (int k = 0; k < kRows; ++k) acc[k] = 0.f;
+  for (int cb = 0; cb < a.d_c; cb += kWc) {
+    const int nc = min(kWc, a.d_c - cb);
+    const int nvec = nc * a.dh / VEC;
+    uint4 wr[8];
 #pragma unroll
-      for (int k = 0; k < kRows; ++k)
-        if (r0 + k < rows) acc[k] += s_o[(r0 + k) * a.d_c + c] * wv;
+    for (int k = 0; k < 8; ++k) {
+      const int v = threadIdx.x + 256 * k;
+      if (v < nvec) wr[k] = __ldg(reinterpret_cast<const uint4*>(W + (size_t)cb * a.dh) + v);
     }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int v = threadIdx.x + 256 * k;
+      if (v < nvec) {
+        const T* e = reinterpret_cast<const T*>(&wr[k]);
+#pragma unroll
+        for (int t = 0; t < VEC; ++t) s_w[v * VEC + t] = to_f32(e[t]);
+      }
+    }
+    __syncthreads();
+    if (item < n_items) {
+#pragma unroll 4
+      for (int c = 0; c < nc; ++c) {
+        const float wv = s_w[c * a.dh + d];
+#pragma unroll
+        for (int k = 0; k < kRows; ++k)
+          if (r0 + k < rows) acc[k] += s_o[(r0 + k) * a.d_c + cb + c] * wv;
+      }
+    }
+    __syncthreads();
+  }
+  if (item < n_items) {
 #pragma unroll
     for (int k = 0; k < kRows; ++k) {
       const int row = r0 + k;
@@ -316,15 +442,24 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
   aa.dn = p.dn; aa.R = p.R; aa.W_ukT = p.W_ukT; aa.nope_idx = p.nope_idx;
   aa.rope_pair = p.rope_pair; aa.theta = p.theta;
   aa.qlat = L.kernel == 1 ? (float*)(base + L.off_qlat) : nullptr;
-  aa.qrope = L.kernel == 1 ? (float*)(base + L.off_qrope) : nullptr;
+  aa.qrope = (float*)(base + L.off_qrope);
   aa.qcat = L.kernel == 2 ? (__nv_bfloat16*)(base + L.off_qlat) : nullptr;
-  aa.K = L.K;
-  aa.bchunk = max(1, kAbsMaxRows / G);
+  aa.K = cfg.d_c;
+  aa.bchunk = 0;
   aa.sched = sched; aa.tile = L.tile; aa.G = L.G; aa.err = p.err;
-  int nchunks = (B + aa.bchunk - 1) / aa.bchunk;
-  size_t smem_abs = (size_t)aa.bchunk * G * p.dn * sizeof(float);
-  absorb_kernel<T><<<cfg.n_kv_heads * nchunks + 1, 256, smem_abs, s>>>(aa);
-  cudaError_t e = cudaGetLastError();
+  const int n_rc = (B * G + kAbsRows - 1) / kAbsRows, n_cc = (cfg.d_c + kAbsCols - 1) / kAbsCols;
+  const size_t smem_abs = std::max((size_t)(p.dn * kAbsCols + kAbsRows * p.dn + kAbsRows * cfg.head_dim) * sizeof(float),
+                                    (size_t)(4 * B + 1) * sizeof(int32_t));
+  {
+    const int vecn = 16 / (int)sizeof(T);  // elements per 16-byte load
+    aa.vec_ok = ((uintptr_t)q % 16 == 0) && cfg.d_c % vecn == 0 && cfg.head_dim % vecn == 0 &&
+                p.dn * (kAbsCols / vecn) <= 256 * 8 && kAbsRows * (cfg.head_dim / vecn) <= 256 * 2;
+  }
+  aa.smem_ints = (int)(smem_abs / sizeof(int32_t));
+  cudaError_t e = cudaFuncSetAttribute(absorb_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_abs);
+  if (e != cudaSuccess) return e;
+  absorb_kernel<T><<<cfg.n_kv_heads * n_cc * n_rc + 1, 256, smem_abs, s>>>(aa);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // 2. split-K attention over the latent cache
   if (L.kernel == 1) {
@@ -332,6 +467,7 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
     da.cache = c; da.B = B; da.H = H; da.n_kv = cfg.n_kv_heads; da.r = cfg.r_pairs;
     da.d_c = cfg.d_c; da.R = p.R; da.qlat = aa.qlat; da.qrope = aa.qrope;
     da.opart = (float*)(base + L.off_opart); da.mlpart = (float*)(base + L.off_mlpart);
+    da.P = L.P;
     da.sched = sched;
     size_t smem = sizeof(float) * ((size_t)H * cfg.d_c + H * 2 * cfg.r_pairs +
                                    kSimtTile * (cfg.d_c + 1) + kSimtTile * (p.R + 1) +
@@ -339,26 +475,30 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
     e = cudaFuncSetAttribute(decode_simt_kernel<T, INT4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    if (p.opt_events) cudaEventRecord((cudaEvent_t)p.opt_events[0], s);
+    if ((e = mla_profile_event(p, 0, s)) != cudaSuccess) return e;
     decode_simt_kernel<T, INT4><<<L.G, 256, smem, s>>>(da);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    if (p.opt_events) cudaEventRecord((cudaEvent_t)p.opt_events[1], s);
+    if ((e = mla_profile_event(p, 1, s)) != cudaSuccess) return e;
   } else {
-    if (p.opt_events) cudaEventRecord((cudaEvent_t)p.opt_events[0], s);
-    e = mla_launch_decode_tc(p, c, B, sched, base + L.off_qlat, (float*)(base + L.off_opart),
-                             (float*)(base + L.off_mlpart), L.G, s);
+    e = mla_launch_decode_tc(p, c, B, sched, base + L.off_qlat, (const float*)(base + L.off_qrope),
+                             (float*)(base + L.off_opart), (float*)(base + L.off_mlpart), L.P, L.G, s);
     if (e != cudaSuccess) return e;
-    if (p.opt_events) cudaEventRecord((cudaEvent_t)p.opt_events[1], s);
   }
   // 3. merge the splits and apply W_uv
   CombineArgs ca;
   ca.B = B; ca.H = H; ca.n_kv = cfg.n_kv_heads; ca.d_c = cfg.d_c; ca.dh = cfg.head_dim;
   ca.opart = (const float*)(base + L.off_opart); ca.mlpart = (const float*)(base + L.off_mlpart);
-  ca.sched = sched; ca.W_uv = p.W_uv; ca.out = out;
-  ca.bchunk = max(1, 8 / G);
-  int cchunks = (B + ca.bchunk - 1) / ca.bchunk;
-  size_t smem_c = (size_t)ca.bchunk * G * (cfg.d_c + 2) * sizeof(float);
+  ca.sched = sched; ca.W_uv = p.W_uv; ca.out = out; ca.P = L.P;
+  // rows (b, h) per CTA: at most 8 per thread and 256 / d_h row groups
+  const int rows_cta = std::max(G, (8 * std::max(1, 256 / cfg.head_dim)) / G * G);
+  ca.bchunk = std::max(1, rows_cta / G);
+  const int cchunks = (B + ca.bchunk - 1) / ca.bchunk;
+  ca.max_pieces = L.G + 1;
+  const size_t smem_c =
+      ((size_t)ca.bchunk * G * (cfg.d_c + ca.max_pieces) + 64 * (size_t)cfg.head_dim) * sizeof(float);
+  e = cudaFuncSetAttribute(combine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
+  if (e != cudaSuccess) return e;
   combine_kernel<T><<<cfg.n_kv_heads * cchunks, 256, smem_c, s>>>(ca);
   return cudaGetLastError();
 }
@@ -371,7 +511,7 @@ DecodeLayout mla_decode_layout(const mla_plan& p, int B, int kernel) {
   const mla_config_t& cfg = p.cfg;
   DecodeLayout L;
   L.kernel = kernel;
-  L.tile = kernel == 2 ? 64 : mla::kSimtTile;
+  L.tile = kernel == 2 ? 128 : mla::kSimtTile;
   L.G = p.opt_splits > 0 ? p.opt_splits : (kernel == 2 ? p.num_sms : 2 * p.num_sms);
   L.P = B + L.G;
   L.K = cfg.d_c + p.R;
@@ -387,13 +527,11 @@ DecodeLayout mla_decode_layout(const mla_plan& p, int B, int kernel) {
   L.off_piece_b = take(sizeof(int32_t) * L.P);
   L.off_piece_t0 = take(sizeof(int32_t) * L.P);
   L.off_piece_t1 = take(sizeof(int32_t) * L.P);
-  if (L.kernel == 1) {
-    L.off_qlat = take(sizeof(float) * (size_t)B * H * cfg.d_c);
-    L.off_qrope = take(sizeof(float) * (size_t)B * H * 2 * cfg.r_pairs + 4);
-  } else {
-    L.off_qlat = take(sizeof(uint16_t) * (size_t)B * H * L.K);
-    L.off_qrope = L.off_qlat;
-  }
+  if (L.kernel == 1)
+    L.off_qlat = take(sizeof(float) * (size_t)B * H * cfg.d_c);          // f32 absorbed query
+  else
+    L.off_qlat = take(sizeof(uint16_t) * (size_t)B * H * cfg.d_c);       // bf16 absorbed query
+  L.off_qrope = take(sizeof(float) * (size_t)B * H * 2 * cfg.r_pairs + 4);
   L.off_opart = take(sizeof(float) * (size_t)L.P * H * cfg.d_c);
   L.off_mlpart = take(sizeof(float) * (size_t)L.P * H * 2);
   L.total = o;

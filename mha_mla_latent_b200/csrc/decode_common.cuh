@@ -40,21 +40,32 @@ __device__ inline int block_exscan(int v, int* total, int* s_warp) {
   return base + x - v;
 }
 
-// Single-block schedule builder.  Must be run by one whole CTA.
+// Single-block schedule builder.  Must be run by one whole CTA.  `scratch` (shared memory,
+// `scratch_ints` ints) holds the per-sequence arrays when they fit, so the searches below
+// run on shared memory; otherwise they live in the workspace.
 __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int B, int T_cap,
-                                      int tile, int G, Sched s, int32_t* err) {
+                                      int tile, int G, Sched s, int32_t* err, int32_t* scratch,
+                                      int scratch_ints) {
   __shared__ int s_warp[32];
   const int tid = threadIdx.x, nt = blockDim.x;
+  int32_t* seq_len = nullptr;  // validated lengths, when there is room to keep them
+  if (scratch && 4 * B + 1 <= scratch_ints) {
+    s.seq_tile0 = scratch;
+    s.seq_ntiles = scratch + B;
+    s.seq_ne = scratch + 2 * B;
+    seq_len = scratch + 3 * B + 1;
+  }
   // 1. tiles per sequence; exclusive prefix sums of tiles and of non-empty sequences
   int carry_t = 0, carry_ne = 0;
   for (int base = 0; base < B; base += nt) {
     const int b = base + tid;
     int nti = 0;
     if (b < B) {
-      int L = seq_lens[b];
+      int L = __ldg(seq_lens + b);
       if (L < 0 || L > T_cap) { raise_error(err, MLA_DEVERR_SEQ_LEN); L = 0; }
       nti = (L + tile - 1) / tile;
       s.seq_ntiles[b] = nti;
+      if (seq_len) seq_len[b] = L;
       s.seq_np[b] = 0;
       s.seq_first[b] = 0;
     }
@@ -111,7 +122,7 @@ __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int 
     while (t < c1) {
       long long e = (long long)s.seq_tile0[b] + s.seq_ntiles[b];
       if (e > c1) e = c1;
-      int L = seq_lens[b];
+      int L = seq_len ? seq_len[b] : __ldg(seq_lens + b);
       if (L < 0 || L > T_cap) L = 0;
       s.piece_b[pidx] = b;
       s.piece_t0[pidx] = (int)((t - s.seq_tile0[b]) * tile);

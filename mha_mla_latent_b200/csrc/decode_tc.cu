@@ -2,26 +2,31 @@
 //
 // Paper notes "MHA2MLA" (ACL 2025), §关键设计: all heads score against the one shared
 // latent c_kv (W_uk absorbed into the query), the kept RoPE dims add a separate score
-// term, and the value side is the probability-weighted latent taken through W_uv.
-// Because every head reads the same c_kv row, the per-tile work is a real dense
-// contraction: for a tile of 64 cached tokens
-//     S[t][h]  = sum_k [C | KR][t][k] * Q'[h][k]          (MMA1, tokens on M, heads on N)
-//     O[d][h] += sum_t C[t][d] * P[t][h]                  (MMA2, latent dims on M)
-// where Q' is the absorbed query row [q_lat | block-diagonal q_rope] (bf16, pre-scaled
-// by log2(e)/sqrt(d_h)), so the RoPE score is folded into MMA1 as K = d_c + n_kv*2r.
-// MMA2 reuses the C tile already in shared memory as an MN-major A operand.
+// term that cannot join the matrix merge, and the value side is the probability-weighted
+// latent taken through W_uv.  Because every head reads the same c_kv row, the per-tile
+// work is a real dense contraction.  For a tile of 128 cached tokens of one sequence:
+//     S[t][h]   = sum_c C[t][c] * Qlat[h][c]            MMA1  M = 128 tokens, N = 32 heads
+//     S[t][h]  += sum_j KR[t][g(h)][j] * Qrope[h][j]    CUDA cores (fp32), from the KR tile
+//     O^T[h][d] += sum_t P^T[h][t] * C[t][d]            MMA2  M = 64 (32 heads + pad), N = d_c
+// MMA2 reuses the C tile already in shared memory as an MN-major B operand, so each
+// cached byte is read from HBM once.  A tcgen05.mma costs about the same issue time
+// whatever its shape, so the orientations maximise work per instruction: per 128
+// tokens d_c/16 + 8 instructions (24 at d_c = 256).
 //
 // One persistent CTA per SM walks its contiguous range of tiles (split-K schedule).
 // Warp roles:
-//   warp 0      TMA producer: Q' per piece; C and KR tiles into two rings of stages
-//               (int4 cache: codes + scales into a raw ring instead of C)
+//   warp 0      TMA producer: Q_lat per piece; C and KR tiles into two rings of stages
+//               (int4 cache: codes + scales into a raw ring instead of C); L2 prefetch of
+//               the tiles after the rings
 //   warp 1      TMEM owner and single-thread MMA issuer; MMA1(n+1) is issued before
 //               MMA2(n) so the tensor pipe works while the softmax of tile n finishes
-//   warps 2-5   softmax: one TMEM lane (token) per thread, 32 heads per thread; online
-//               softmax in log2 units with lazy rescaling (the running max is raised only
-//               when a score exceeds it by more than 2^8, then O in TMEM is rescaled);
-//               writes P (bf16) for MMA2; per-piece epilogue writes the partial (m, l, O)
-//   warps 6-9   (int4 cache) dequantise codes*scale into the bf16 C stage
+//   warps 2-9   softmax: one token per thread (TMEM lane), 16 heads per thread (two warps
+//               per lane quarter); adds the
+//               RoPE score, online softmax in log2 units with lazy rescaling (the running
+//               max is raised only when a score exceeds it by more than 2^8, then the O
+//               rows are rescaled in TMEM), writes P^T (bf16) for MMA2, and per piece the
+//               partial (m, l, O) for the split merge
+//   warps 10-11 (int4 cache) dequantise codes*scale into the bf16 C stage
 // Every wait is bounded (about 1 s); a timeout sets MLA_DEVERR_TIMEOUT, all roles stop,
 // in-flight copies and MMAs are drained and TMEM is released before the CTA exits.
 #include <cuda.h>
@@ -34,64 +39,71 @@ namespace tc {
 
 using namespace sm100;
 
-constexpr int kTile = 64;        // tokens per tile (MMA1 M)
-constexpr int kH = 32;           // heads handled by this kernel (MMA N)
-constexpr float kTau = 8.0f;     // lazy-rescale threshold, log2 units
-constexpr uint32_t kBox = 8192;  // 64 rows x 128 B TMA box
-constexpr uint32_t kQBox = 4096; // 32 rows x 128 B
-constexpr uint32_t kPBytes = kTile * kH * 2;
+constexpr int kTile = 128;          // tokens per tile
+constexpr int kH = 32;              // heads handled by this kernel
+constexpr int kHh = 16;             // heads per softmax warp (two warps per TMEM lane quarter)
+constexpr int kSoftWarps = 8;
+constexpr float kTau = 8.0f;        // lazy-rescale threshold, log2 units
+constexpr uint32_t kBox = 16384;    // TMA box: 128 rows x 128 B (C, KR)
+constexpr uint32_t kQBox = 4096;    // Q_lat box: 32 rows x 128 B
+constexpr uint32_t kPtAtom = 8192;  // P^T: 64 rows x 128 B per 64-token atom
+constexpr uint32_t kPtBytes = 2 * kPtAtom;
 
 struct TcArgs {
-  int B, H, d_c, R, K, T_cap;
+  int B, H, d_c, R, r2, T_cap, P;
   Sched sched;
-  float* opart;
-  float* mlpart;
+  float* opart;           // [H][P][d_c]
+  float* mlpart;          // [H][P][2]
+  const float* qrope;     // [B][H][2r] rotated, scaled RoPE query part
   const __half* scales;   // int4: [B*T_cap][d_c/32]
+  const uint8_t* kr_base;
+  uint32_t c_row, kr_row;
   int32_t* err;
-  int NC, NK, NRAW;       // ring depths
-  uint32_t off_c, off_kr, off_q, off_p, off_raw, off_bar, off_misc;  // from the 1024-aligned base
+  int NC, NRAW, NP, NO;  // ring depths; P^T and O buffers
+  uint32_t off_c, off_q, off_p, off_raw, off_qr, off_bar, off_misc;
+  uint32_t off_kr;        // RoPE key stage: one tile, 4 blocks of [n_kv][32][2r]
 };
 
-// barrier indices inside the barrier block
 struct Bars {
   uint32_t base;
-  int NC, NK, NRAW;
+  int NC, NRAW, NP, NO;
   __device__ uint32_t at(int i) const { return base + 8u * (uint32_t)i; }
   __device__ uint32_t c_full(int s) const { return at(s); }
   __device__ uint32_t c_empty(int s) const { return at(NC + s); }
-  __device__ uint32_t kr_full(int s) const { return at(2 * NC + s); }
-  __device__ uint32_t kr_empty(int s) const { return at(2 * NC + NK + s); }
-  __device__ uint32_t raw_full(int s) const { return at(2 * NC + 2 * NK + s); }
-  __device__ uint32_t raw_empty(int s) const { return at(2 * NC + 2 * NK + NRAW + s); }
-  __device__ int fixed() const { return 2 * NC + 2 * NK + 2 * NRAW; }
-  __device__ uint32_t q_full() const { return at(fixed() + 0); }
-  __device__ uint32_t q_empty() const { return at(fixed() + 1); }
-  __device__ uint32_t s_full(int i) const { return at(fixed() + 2 + i); }
-  __device__ uint32_t s_empty(int i) const { return at(fixed() + 4 + i); }
-  __device__ uint32_t p_full(int i) const { return at(fixed() + 6 + i); }
-  __device__ uint32_t p_empty(int i) const { return at(fixed() + 8 + i); }
-  __device__ uint32_t o_full(int i) const { return at(fixed() + 10 + i); }
-  __device__ uint32_t o_empty(int i) const { return at(fixed() + 12 + i); }
-  __device__ uint32_t grp(int i) const { return at(fixed() + 14 + i); }  // softmax-group syncs
-  __device__ uint32_t mma_done() const { return at(fixed() + 16); }
-  __device__ int count() const { return fixed() + 17; }
+  __device__ uint32_t raw_full(int s) const { return at(2 * NC + s); }
+  __device__ uint32_t raw_empty(int s) const { return at(2 * NC + NRAW + s); }
+  __device__ int o1() const { return 2 * NC + 2 * NRAW; }
+  __device__ uint32_t p_full(int i) const { return at(o1() + i); }
+  __device__ uint32_t p_empty(int i) const { return at(o1() + 2 + i); }
+  __device__ uint32_t o_full(int i) const { return at(o1() + 4 + i); }
+  __device__ uint32_t o_empty(int i) const { return at(o1() + 6 + i); }
+  __device__ uint32_t s_full(int i) const { return at(o1() + 8 + i); }
+  __device__ uint32_t s_empty(int i) const { return at(o1() + 10 + i); }
+  __device__ uint32_t q_full() const { return at(o1() + 12); }
+  __device__ uint32_t q_empty() const { return at(o1() + 13); }
+  __device__ uint32_t grp(int i) const { return at(o1() + 14 + i); }
+  __device__ uint32_t mma_done() const { return at(o1() + 16); }
+  __device__ uint32_t kr_full() const { return at(o1() + 17); }
 };
+constexpr int kFixedBars = 18;
 
 struct Misc {  // small shared scratch
   uint32_t tmem_base;
   int abort_flag;
-  int vote[2][4];
+  int vote[2][kSoftWarps];
   float red_max[2][4][kH];
-  float red_sum[4][kH];
-  float mt[4][kH];
+  float red_l[4][kH];
+  float mt[kSoftWarps][kHh];
+  int kr_released;   // softmax warps done with the RoPE key stage (the 8th issues the next copy)
+  int kr_issued;     // RoPE key copies issued
 };
 
 // Per-worker iteration over (piece, tile) in schedule order.
 struct TileIter {
   const Sched* s;
-  int pc, pc_end;     // current piece, end
-  int b, t0, t1;      // piece
-  int t;              // current tile start (token)
+  int pc, pc_end;
+  int b, t0, t1;
+  int t;
   __device__ void init(const Sched* sc, int w) {
     s = sc;
     pc = sc->worker_first[w];
@@ -111,10 +123,37 @@ struct TileIter {
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 __device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Maximum over the warp (sm_100 warp-wide float reduction).
+__device__ __forceinline__ float warp_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// Reduction over the 32 lanes of each of 16 values (15 + 1 shuffles): lanes i and i ^ 16
+// end with the result for element (i & 15).
+template <bool kMax>
+__device__ __forceinline__ float transpose_reduce16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int off = 8; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int k = 0; k < off; ++k) {
+      float send = upper ? v[k] : v[k + off];
+      float keep = upper ? v[k + off] : v[k];
+      float recv = __shfl_xor_sync(0xffffffffu, send, off);
+      v[k] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  const float other = __shfl_xor_sync(0xffffffffu, v[0], 16);
+  return kMax ? fmaxf(v[0], other) : v[0] + other;
 }
 
 // lane i ends with the reduction over the warp of element i (31 shuffles)
@@ -134,54 +173,74 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[kH], int lane) {
   return v[0];
 }
 
-template <bool INT4>
-__global__ void __launch_bounds__(INT4 ? 320 : 192, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_kr,
-                 const __grid_constant__ CUtensorMap tm_q, TcArgs a) {
+#ifdef MLA_TC_TRACE
+// Timeline instrumentation for development builds only (-DMLA_TC_TRACE): %globaltimer
+// stamps per (CTA, event, tile) for the first kTraceCtas CTAs.
+constexpr int kTraceCtas = 4, kTraceEv = 40, kTraceTiles = 64;
+__device__ unsigned long long g_trace[kTraceCtas * kTraceEv * kTraceTiles];
+__device__ unsigned long long g_cta_span[1024 * 2];
+#define MLA_TRACE(ev, n)                                                                          \
+  do {                                                                                            \
+    if (blockIdx.x < kTraceCtas && (n) < kTraceTiles)                                             \
+      g_trace[(blockIdx.x * kTraceEv + (ev)) * kTraceTiles + (n)] = globaltimer();                \
+  } while (0)
+#else
+#define MLA_TRACE(ev, n) do { } while (0)
+#endif
+
+template <bool INT4, int R2>
+__global__ void __launch_bounds__(384, 1)
+decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
+                 const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (sbase_u32 - smem_u32(smem_raw));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int dc = a.d_c, R = a.R, K = a.K;
-  const int n_cbox = dc / 64, n_krbox = R / 64, n_qbox = K / 64;
-  const uint32_t c_stage = (uint32_t)n_cbox * kBox, kr_stage = (uint32_t)n_krbox * kBox;
+#ifdef MLA_TC_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 1024) g_cta_span[2 * blockIdx.x] = globaltimer();
+#endif
+  const int dc = a.d_c, R = a.R;
+  const int n_cbox = dc / 64;
+  const uint32_t c_stage = (uint32_t)n_cbox * kBox;
   const uint32_t raw_codes = (uint32_t)kTile * (dc / 2), raw_stage = raw_codes + (uint32_t)kTile * (dc / 16);
-  const int nchunk = dc >= 128 ? dc / 128 : 1;      // MMA2 M-chunks (M = 128, or one M = 64)
-  const int m2 = dc >= 128 ? 128 : 64;
-  const uint32_t S_COL = 0, O_COL = 2 * kH, O_STRIDE = (uint32_t)nchunk * kH;
-  Bars bars{sbase_u32 + a.off_bar, a.NC, a.NK, a.NRAW};
+  const uint32_t S_COL = 0, O_COL = 2 * kH;
+  Bars bars{sbase_u32 + a.off_bar, a.NC, a.NRAW, a.NP, a.NO};
   Misc* misc = reinterpret_cast<Misc*>(sbase + a.off_misc);
   volatile int* abort_flag = &misc->abort_flag;
+  float* qr_s = reinterpret_cast<float*>(sbase + a.off_qr);   // [32][2r]
+  // Q_lat boxes 0 and 1 live in the padding rows (32..63) of P^T buffer 0: MMA2 reads those
+  // rows only into output rows that are never used; further boxes follow at off_q
+  auto qbox = [&](int kb) -> uint32_t {
+    return sbase_u32 + (kb < 2 ? a.off_p + 4096u + kPtAtom * kb : a.off_q + kQBox * (kb - 2));
+  };
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     misc->abort_flag = 0;
-    for (int s = 0; s < a.NC; ++s) {
-      mbar_init(bars.c_full(s), INT4 ? 4 : 1);
-      mbar_init(bars.c_empty(s), 1);
-    }
-    for (int s = 0; s < a.NK; ++s) { mbar_init(bars.kr_full(s), 1); mbar_init(bars.kr_empty(s), 1); }
-    for (int s = 0; s < a.NRAW; ++s) { mbar_init(bars.raw_full(s), 1); mbar_init(bars.raw_empty(s), 4); }
-    mbar_init(bars.q_full(), 1);
-    mbar_init(bars.q_empty(), 1);
+    for (int s = 0; s < a.NC; ++s) { mbar_init(bars.c_full(s), INT4 ? 2 : 1); mbar_init(bars.c_empty(s), 1); }
+    for (int s = 0; s < a.NRAW; ++s) { mbar_init(bars.raw_full(s), 1); mbar_init(bars.raw_empty(s), 2); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bars.s_full(i), 1);
-      mbar_init(bars.s_empty(i), 4);
-      mbar_init(bars.p_full(i), 4);
+      mbar_init(bars.p_full(i), kSoftWarps);
       mbar_init(bars.p_empty(i), 1);
       mbar_init(bars.o_full(i), 1);
-      mbar_init(bars.o_empty(i), 4);
-      mbar_init(bars.grp(i), 4);
+      mbar_init(bars.o_empty(i), kSoftWarps);
+      mbar_init(bars.s_full(i), 1);
+      mbar_init(bars.s_empty(i), kSoftWarps);
+      mbar_init(bars.grp(i), kSoftWarps);
     }
+    mbar_init(bars.q_full(), 1);
+    mbar_init(bars.q_empty(), 1);
     mbar_init(bars.mma_done(), 1);
+    mbar_init(bars.kr_full(), 1);
+    misc->kr_released = 0;
+    misc->kr_issued = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_c);
-    tma_prefetch_desc(&tm_kr);
     tma_prefetch_desc(&tm_q);
   }
-  const uint32_t tmem_cols = (O_COL + 2 * O_STRIDE) <= 128 ? 128u : 256u;
+  const uint32_t tmem_cols = (O_COL + a.NO * dc) <= 256 ? 256u : 512u;
   if (warp == 1) {
     tmem_alloc(smem_u32(&misc->tmem_base), tmem_cols);
     tmem_relinquish();
@@ -191,374 +250,478 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = misc->tmem_base;
   const int w = blockIdx.x;
+  if (threadIdx.x == 0) MLA_TRACE(7, 0);
 
-  if (warp == 0) {
-    // ============================================================ TMA producer
-    if (lane == 0) {
-      TileIter it;
-      it.init(&a.sched, w);
-      int n = 0, u = 0;
-      int last_c = -1, last_kr = -1, last_raw = -1;
-      int q_loads = 0;
-      bool ok = true;
-      while (ok && it.valid()) {
-        if (it.first_of_piece()) {
-          if (u > 0) ok = mbar_wait(bars.q_empty(), (u - 1) & 1, abort_flag);
-          if (!ok) break;
-          mbar_expect_tx(bars.q_full(), (uint32_t)n_qbox * kQBox);
-          for (int kb = 0; kb < n_qbox; ++kb)
-            tma_load_2d(sbase_u32 + a.off_q + kb * kQBox, &tm_q, bars.q_full(), kb * 64, it.b * a.H);
-          ++q_loads;
+  // register split: the control warpgroup (producer, MMA issuer, int4 dequant) gives up
+  // registers to the two softmax warpgroups: 128 * 56 + 256 * 224 = 384 * 168 at launch
+  if (warp < 4) {
+    setmaxnreg_dec<56>();
+    if (warp == 0) {
+      // ============================================================ TMA producer
+      if (lane == 0) {
+        TileIter it;
+        it.init(&a.sched, w);
+        int n = 0, u = 0, q_loads = 0;
+        int last_c = -1, last_raw = -1;
+        bool ok = true;
+        while (ok && it.valid()) {
+          if (it.first_of_piece()) {
+            if (u > 0) ok = mbar_wait(bars.q_empty(), (u - 1) & 1, abort_flag);
+            if (!ok) break;
+            mbar_expect_tx(bars.q_full(), (uint32_t)n_cbox * kQBox);
+            for (int kb = 0; kb < n_cbox; ++kb)
+              tma_load_2d(qbox(kb), &tm_q, bars.q_full(), kb * 64, it.b * a.H);
+            ++q_loads;
+          }
+          const int row = it.b * a.T_cap + it.t;
+          MLA_TRACE(0, n);
+          if (!INT4) {
+            const int cs = n % a.NC;
+            if (n >= a.NC) ok = mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag);
+            if (!ok) break;
+            mbar_expect_tx(bars.c_full(cs), c_stage);
+            for (int cb = 0; cb < n_cbox; ++cb)
+              tma_load_2d(sbase_u32 + a.off_c + cs * c_stage + cb * kBox, &tm_c, bars.c_full(cs), cb * 64, row);
+            last_c = n;
+          } else {
+            const int rs = n % a.NRAW;
+            if (n >= a.NRAW) ok = mbar_wait(bars.raw_empty(rs), ((n / a.NRAW) - 1) & 1, abort_flag);
+            if (!ok) break;
+            const int nvalid = min(kTile, it.t1 - it.t);
+            const uint32_t sbytes = (uint32_t)((((nvalid + 1) & ~1) * (dc / 16) + 15) & ~15);
+            mbar_expect_tx(bars.raw_full(rs), raw_codes + sbytes);
+            tma_load_2d(sbase_u32 + a.off_raw + rs * raw_stage, &tm_c, bars.raw_full(rs), 0, row);
+            bulk_load(sbase_u32 + a.off_raw + rs * raw_stage + raw_codes, a.scales + (size_t)row * (dc / 32), sbytes,
+                      bars.raw_full(rs));
+            last_raw = n;
+          }
+          MLA_TRACE(1, n);
+          if (it.last_of_piece()) ++u;
+          it.next();
+          ++n;
         }
-        const int row = it.b * a.T_cap + it.t;
-        const int ks = n % a.NK;
-        if (n >= a.NK) ok = mbar_wait(bars.kr_empty(ks), ((n / a.NK) - 1) & 1, abort_flag);
-        if (!ok) break;
-        mbar_expect_tx(bars.kr_full(ks), kr_stage);
-        for (int rb = 0; rb < n_krbox; ++rb)
-          tma_load_2d(sbase_u32 + a.off_kr + ks * kr_stage + rb * kBox, &tm_kr, bars.kr_full(ks), rb * 64, row);
-        last_kr = n;
+        // drain: every issued copy must land before the CTA can exit
+        volatile int never = 0;
+        if (q_loads > 0) mbar_wait(bars.q_full(), (q_loads - 1) & 1, &never);
         if (!INT4) {
-          const int cs = n % a.NC;
-          if (n >= a.NC) ok = mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag);
-          if (!ok) break;
-          mbar_expect_tx(bars.c_full(cs), c_stage);
-          for (int cb = 0; cb < n_cbox; ++cb)
-            tma_load_2d(sbase_u32 + a.off_c + cs * c_stage + cb * kBox, &tm_c, bars.c_full(cs), cb * 64, row);
-          last_c = n;
+          for (int s = 0; s < a.NC; ++s) {
+            const int k = last_c - ((last_c - s) % a.NC + a.NC) % a.NC;
+            if (last_c >= 0 && k >= 0) mbar_wait(bars.c_full(s), (k / a.NC) & 1, &never);
+          }
         } else {
-          const int rs = n % a.NRAW;
-          if (n >= a.NRAW) ok = mbar_wait(bars.raw_empty(rs), ((n / a.NRAW) - 1) & 1, abort_flag);
-          if (!ok) break;
-          const int nvalid = min(kTile, it.t1 - it.t);
-          const uint32_t sbytes = (uint32_t)((((nvalid + 1) & ~1) * (dc / 16) + 15) & ~15);
-          mbar_expect_tx(bars.raw_full(rs), raw_codes + sbytes);
-          tma_load_2d(sbase_u32 + a.off_raw + rs * raw_stage, &tm_c, bars.raw_full(rs), 0, row);
-          bulk_load(sbase_u32 + a.off_raw + rs * raw_stage + raw_codes, a.scales + (size_t)row * (dc / 32), sbytes,
-                    bars.raw_full(rs));
-          last_raw = n;
-        }
-        if (it.last_of_piece()) ++u;
-        it.next();
-        ++n;
-      }
-      // drain: every issued copy must land before the CTA can exit
-      volatile int never = 0;
-      if (q_loads > 0) mbar_wait(bars.q_full(), (q_loads - 1) & 1, &never);
-      for (int s = 0; s < a.NK; ++s) {
-        int k = last_kr - ((last_kr - s) % a.NK + a.NK) % a.NK;  // last issue into slot s
-        if (last_kr >= 0 && k >= 0) mbar_wait(bars.kr_full(s), (k / a.NK) & 1, &never);
-      }
-      if (!INT4) {
-        for (int s = 0; s < a.NC; ++s) {
-          int k = last_c - ((last_c - s) % a.NC + a.NC) % a.NC;
-          if (last_c >= 0 && k >= 0) mbar_wait(bars.c_full(s), (k / a.NC) & 1, &never);
-        }
-      } else {
-        for (int s = 0; s < a.NRAW; ++s) {
-          int k = last_raw - ((last_raw - s) % a.NRAW + a.NRAW) % a.NRAW;
-          if (last_raw >= 0 && k >= 0) mbar_wait(bars.raw_full(s), (k / a.NRAW) & 1, &never);
+          for (int s = 0; s < a.NRAW; ++s) {
+            const int k = last_raw - ((last_raw - s) % a.NRAW + a.NRAW) % a.NRAW;
+            if (last_raw >= 0 && k >= 0) mbar_wait(bars.raw_full(s), (k / a.NRAW) & 1, &never);
+          }
         }
       }
-    }
-  } else if (warp == 1) {
-    // ============================================================ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc1 = idesc_bf16_f32(kTile, kH, false, false);
-      const uint32_t idesc2 = idesc_bf16_f32(m2, kH, true, true);
-      TileIter it;
-      it.init(&a.sched, w);
-      int n = 0, u = 0;
-      bool ok = true;
-      // state of the tile whose MMA2 is pending
-      int pend_n = -1, pend_u = 0;
-      bool pend_first = false, pend_last = false;
-      auto do_mma2 = [&](int pn, int pu, bool first, bool last) -> bool {
-        const int pb = pn & 1, cs = pn % a.NC, ob = pu & 1;
-        if (!mbar_wait(bars.p_full(pb), (pn >> 1) & 1, abort_flag)) return false;
-        if (first && pu >= 2)
-          if (!mbar_wait(bars.o_empty(ob), ((pu >> 1) - 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t c0 = sbase_u32 + a.off_c + cs * c_stage;
-        const uint32_t p0 = sbase_u32 + a.off_p + pb * kPBytes;
-        for (int mc = 0; mc < nchunk; ++mc) {
-          const uint32_t d = tmem + O_COL + ob * O_STRIDE + mc * kH;
-#pragma unroll
+    } else if (warp == 1) {
+      // ============================================================ MMA issuer
+      if (lane == 0) {
+        const uint32_t idesc1 = idesc_bf16_f32(kTile, kH, false, false);  // S[t][h]
+        const uint32_t idesc2 = idesc_bf16_f32(64, dc, false, true);      // O^T[h][d]
+        TileIter it;
+        it.init(&a.sched, w);
+        int n = 0, u = 0;
+        bool ok = true;
+        int pend_n = -1, pend_u = 0;
+        bool pend_first = false, pend_last = false;
+        auto do_mma2 = [&](int pn, int pu, bool first, bool last) -> bool {
+          const int pb = pn % a.NP, cs = pn % a.NC, ob = pu % a.NO;
+          if (!mbar_wait(bars.p_full(pb), (pn / a.NP) & 1, abort_flag)) return false;
+          if (first && pu >= a.NO)
+            if (!mbar_wait(bars.o_empty(ob), ((pu / a.NO) - 1) & 1, abort_flag)) return false;
+          MLA_TRACE(4, pn);
+          tc_fence_after();
+          const uint32_t c0 = sbase_u32 + a.off_c + cs * c_stage;
+          const uint32_t p0 = sbase_u32 + a.off_p + pb * kPtBytes;
+          const uint32_t d = tmem + O_COL + ob * dc;
+  #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk) {
-            uint64_t ad = smem_desc(c0 + mc * 2 * kBox + kk * 2048, kBox, 1024, kLayoutSW128);
-            uint64_t bd = smem_desc(p0 + kk * 256, 128, 1024, kLayoutNone);
+            const uint64_t ad = smem_desc(p0 + (kk >> 2) * kPtAtom + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+            const uint64_t bd = smem_desc(c0 + kk * 2048, kBox, 1024, kLayoutSW128);
             tc_mma_bf16(d, ad, bd, idesc2, (first && kk == 0) ? 0u : 1u);
           }
-        }
-        tc_commit(bars.p_empty(pb));
-        tc_commit(bars.c_empty(cs));
-        if (last) tc_commit(bars.o_full(ob));
-        return true;
-      };
-      while (ok && it.valid()) {
-        const int sb = n & 1, cs = n % a.NC, ks = n % a.NK;
-        if (n >= 2) ok = mbar_wait(bars.s_empty(sb), ((n >> 1) - 1) & 1, abort_flag);
-        if (ok && it.first_of_piece()) ok = mbar_wait(bars.q_full(), u & 1, abort_flag);
-        if (ok) ok = mbar_wait(bars.kr_full(ks), (n / a.NK) & 1, abort_flag);
-        if (ok) ok = mbar_wait(bars.c_full(cs), (n / a.NC) & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        {  // MMA1: S = [C | KR] Q'^T
-          const uint32_t d = tmem + S_COL + sb * kH;
-          const uint32_t c0 = sbase_u32 + a.off_c + cs * c_stage;
-          const uint32_t k0 = sbase_u32 + a.off_kr + ks * kr_stage;
-          const uint32_t q0 = sbase_u32 + a.off_q;
-          for (int kk = 0; kk < dc / 16; ++kk) {
-            uint64_t ad = smem_desc(c0 + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-            uint64_t bd = smem_desc(q0 + (kk >> 2) * kQBox + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-            tc_mma_bf16(d, ad, bd, idesc1, kk > 0 ? 1u : 0u);
+          tc_commit(bars.p_empty(pb));
+          tc_commit(bars.c_empty(cs));
+          if (last) tc_commit(bars.o_full(ob));
+          return true;
+        };
+        while (ok && it.valid()) {
+          const int sb = n & 1, cs = n % a.NC;
+          const bool first = it.first_of_piece();
+          // MMA1(n) needs its S buffer free, the piece's Q_lat and the latent tile; MMA2 of the
+          // pending tile needs its P^T.  Whichever is ready first goes first, so a pending tile
+          // releases its latent stage (and the next copy can start) as early as possible.
+          {
+            const uint64_t t_start = globaltimer();
+            while (true) {
+              if (pend_n >= 0 && mbar_test(bars.p_full(pend_n % a.NP), (pend_n / a.NP) & 1)) {
+                ok = do_mma2(pend_n, pend_u, pend_first, pend_last);
+                pend_n = -1;
+                if (!ok) break;
+                continue;
+              }
+              if ((n < 2 || mbar_test(bars.s_empty(sb), ((n >> 1) - 1) & 1)) &&
+                  (!first || mbar_test(bars.q_full(), u & 1)) && mbar_test(bars.c_full(cs), (n / a.NC) & 1))
+                break;
+              if (*abort_flag || globaltimer() - t_start > kWaitLimitNs) {
+                *abort_flag = 1;
+                ok = false;
+                break;
+              }
+            }
           }
-          for (int kk = 0; kk < R / 16; ++kk) {
-            uint64_t ad = smem_desc(k0 + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-            uint64_t bd = smem_desc(q0 + (n_cbox + (kk >> 2)) * kQBox + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-            tc_mma_bf16(d, ad, bd, idesc1, 1u);
-          }
-          tc_commit(bars.s_full(sb));
-          tc_commit(bars.kr_empty(ks));
-          if (it.last_of_piece()) tc_commit(bars.q_empty());
-        }
-        if (pend_n >= 0) {
-          ok = do_mma2(pend_n, pend_u, pend_first, pend_last);
           if (!ok) break;
+          MLA_TRACE(2, n);
+          tc_fence_after();
+          {  // MMA1: S = C Q_lat^T
+            const uint32_t d = tmem + S_COL + sb * kH;
+            const uint32_t c0 = sbase_u32 + a.off_c + cs * c_stage;
+            for (int kk = 0; kk < dc / 16; ++kk) {
+              const uint64_t ad = smem_desc(c0 + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+              const uint64_t bd = smem_desc(qbox(kk >> 2) + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+              tc_mma_bf16(d, ad, bd, idesc1, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bars.s_full(sb));
+            if (it.last_of_piece()) tc_commit(bars.q_empty());
+            MLA_TRACE(3, n);
+          }
+          if (pend_n >= 0) {   // one pending tile at most: MMA2(n-1) before tile n waits
+            ok = do_mma2(pend_n, pend_u, pend_first, pend_last);
+            if (!ok) break;
+          }
+          pend_n = n; pend_u = u; pend_first = first; pend_last = it.last_of_piece();
+          if (it.last_of_piece()) ++u;
+          it.next();
+          ++n;
         }
-        pend_n = n; pend_u = u; pend_first = it.first_of_piece(); pend_last = it.last_of_piece();
-        if (it.last_of_piece()) ++u;
+        if (ok && pend_n >= 0) do_mma2(pend_n, pend_u, pend_first, pend_last);
+        // drain: all issued MMAs complete before TMEM is released
+        tc_commit(bars.mma_done());
+        volatile int never = 0;
+        mbar_wait(bars.mma_done(), 0, &never);
+      }
+    } else if (INT4 && warp >= 2) {
+      // ============================================================ int4 dequantisation
+      const int tid_dq = threadIdx.x - 64;   // 0..63: token rows tid_dq, tid_dq + 64
+      TileIter it;
+      it.init(&a.sched, w);
+      int n = 0;
+      bool ok = true;
+      while (ok && it.valid()) {
+        const int rs = n % a.NRAW, cs = n % a.NC;
+        ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_full(rs), (n / a.NRAW) & 1, abort_flag));
+        if (ok && n >= a.NC)
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag));
+        if (!ok) break;
+        const int nvalid = min(kTile, it.t1 - it.t);
+        const uint8_t* raw = sbase + a.off_raw + rs * raw_stage;
+        for (int rr = 0; rr < 2; ++rr) {
+          const int tok = tid_dq + 64 * rr;
+          uint8_t* C = sbase + a.off_c + cs * c_stage + tok * 128;
+          if (tok < nvalid) {
+            const __half* sc = reinterpret_cast<const __half*>(raw + raw_codes) + tok * (dc / 32);
+            for (int half = 0; half < dc / 64; ++half) {
+              const uint4 c0 = *reinterpret_cast<const uint4*>(raw + tok * (dc / 2) + half * 32);
+              const uint4 c1 = *reinterpret_cast<const uint4*>(raw + tok * (dc / 2) + half * 32 + 16);
+              const float s0 = __half2float(sc[half * 2]), s1 = __half2float(sc[half * 2 + 1]);
+              const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  #pragma unroll
+              for (int ch = 0; ch < 8; ++ch) {           // 8 latent values per 16-byte chunk
+                const uint32_t wd = words[ch];
+                const float s = ch < 4 ? s0 : s1;
+                uint32_t o[4];
+  #pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const uint32_t byte = (wd >> (8 * j)) & 0xFFu;
+                  o[j] = pack_bf16x2((float)nib_to_int(byte & 15u) * s, (float)nib_to_int(byte >> 4) * s);
+                }
+                *reinterpret_cast<uint4*>(C + half * kBox + ((ch ^ (tok & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
+              }
+            }
+          } else {
+            for (int half = 0; half < dc / 64; ++half)
+  #pragma unroll
+              for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(C + half * kBox + ch * 16) = make_uint4(0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bars.raw_empty(rs));
+          mbar_arrive(bars.c_full(cs));
+        }
         it.next();
         ++n;
       }
-      if (ok && pend_n >= 0) do_mma2(pend_n, pend_u, pend_first, pend_last);
-      // drain: all issued MMAs complete before TMEM is released
-      tc_commit(bars.mma_done());
-      volatile int never = 0;
-      mbar_wait(bars.mma_done(), 0, &never);
     }
-  } else if (warp < 6) {
+  } else {
+    setmaxnreg_inc<224>();
     // ============================================================ softmax + epilogue
-    const int q = warp & 3;            // TMEM lane quarter of this warp
-    const int row = 16 * q + lane;     // token row within the tile (M = 64 layout), lane < 16
+    // eight warps: two per TMEM lane quarter (tokens 32q .. 32q+31), each one head half
+    const int q = warp & 3;
+    const int sw = warp - 4;             // softmax warp 0..7
+    const int hh = sw >> 2;              // heads 16hh .. 16hh+15
+    const int tr = 32 * q + lane;        // this thread's token row in the tile
     TileIter it;
     it.init(&a.sched, w);
     int n = 0, u = 0, gphase0 = 0, gphase1 = 0;
     bool ok = true;
-    float m[kH], l[kH];
+    float m[kHh], l[kHh];
     auto wwait = [&](uint32_t bar, int parity) -> bool {  // warp-uniform outcome
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
-    auto grp_sync = [&](int i) -> bool {  // all 4 softmax warps, bounded
+    auto grp_sync = [&](int i) -> bool {  // all softmax warps, bounded
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.grp(i));
-      int& ph = i ? gphase1 : gphase0;
-      bool r = wwait(bars.grp(i), ph & 1);
-      ++ph;
-      return r;
+      const int ph = i ? gphase1++ : gphase0++;
+      return wwait(bars.grp(i), ph & 1);
     };
+    const int G = kH / (R / R2);         // query heads per KV head
+    // RoPE keys: in the blocked cache layout a tile's keys (4 blocks of [n_kv][32][2r]) are
+    // one contiguous range, brought into the shared stage by a single bulk copy.  Each warp
+    // moves its part (block q, the KV heads of its 16 heads: lane t reads token t, so the
+    // reads are conflict-free) into registers as soon as the copy lands and releases the
+    // stage; the eighth warp to release it issues the copy of the tile after.  The
+    // registers hold tile n+1's keys while tile n is processed, so the copy of tile n+2
+    // has a whole tile period to land.
+    const int n_kv = R / R2;
+    const uint32_t kr_blk = (uint32_t)n_kv * 32u * R2 * 2u;   // bytes per 32-token block
+    uint4 kr[kHh];
+    auto issue_kr = [&](const TileIter& ti) {   // one thread
+      if (!ti.valid()) return;
+      const int nblk = min(4, (ti.t1 - ti.t + 31) / 32);
+      const uint8_t* src = a.kr_base + mla_kr_offset(ti.b, ti.t, 0, 0, a.T_cap, n_kv, R2) * 2;
+      fence_proxy_async_smem();
+      mbar_expect_tx(bars.kr_full(), nblk * kr_blk);
+      bulk_load(sbase_u32 + a.off_kr, src, nblk * kr_blk, bars.kr_full());
+      misc->kr_issued += 1;
+    };
+    auto fetch_kr = [&](int k, const TileIter& ti_after) -> bool {   // tile k's keys -> kr
+      if (!wwait(bars.kr_full(), k & 1)) return false;
+      const uint8_t* blk = sbase + a.off_kr + q * kr_blk + lane * 16;
+#pragma unroll
+      for (int h = 0; h < kHh; ++h)
+        kr[h] = *reinterpret_cast<const uint4*>(blk + (size_t)((kHh * hh + h) / G) * 32 * 16);
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        if (atomicAdd(&misc->kr_released, 1) % kSoftWarps == kSoftWarps - 1) issue_kr(ti_after);
+      }
+      return true;
+    };
+    if (it.valid()) {   // a worker with no tiles issues and waits for nothing
+      if (sw == 0 && lane == 0) issue_kr(it);
+      TileIter nx = it;
+      nx.next();
+      ok = fetch_kr(0, nx);
+    }
     while (ok && it.valid()) {
       const int pc = it.pc;
       const bool first = it.first_of_piece();
       if (first) {
+        // the previous piece's RoPE queries are no longer read: load this piece's
+        ok = grp_sync(1);
+        if (!ok) break;
+        for (int i = threadIdx.x - 128; i < kH * R2; i += 32 * kSoftWarps)
+          qr_s[i] = __ldg(a.qrope + (size_t)it.b * kH * R2 + i);
+        ok = grp_sync(1);
+        if (!ok) break;
 #pragma unroll
-        for (int h = 0; h < kH; ++h) { m[h] = -INFINITY; l[h] = 0.f; }
+        for (int h = 0; h < kHh; ++h) { m[h] = -INFINITY; l[h] = 0.f; }
       }
-      const int sb = n & 1, pb = n & 1, ob = u & 1;
+      const int sb = n & 1, pb = n % a.NP, ob = u % a.NO;
       const int nvalid = min(kTile, it.t1 - it.t);
-      const bool valid = lane < 16 && row < nvalid;
+      const bool valid = tr < nvalid;
       ok = wwait(bars.s_full(sb), (n >> 1) & 1);
       if (!ok) break;
+      if (warp == 4 && lane == 0) MLA_TRACE(5, n);
       tc_fence_after();
-      float v[kH];
+      float v[kHh];
       {
-        uint32_t raw[32];
-        tmem_ld32(taddr(tmem, 32 * q, S_COL + sb * kH), raw);
+        uint32_t raw[16];
+        tmem_ld16(taddr(tmem, 32 * q, S_COL + sb * kH + kHh * hh), raw);
         tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < kH; ++h) v[h] = valid ? u2f(raw[h]) : -INFINITY;
+        for (int h = 0; h < kHh; ++h) v[h] = u2f(raw[h]);
       }
+      if (lane == 0) MLA_TRACE(16 + sw, n);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.s_empty(sb));
+      // RoPE score: head 16hh + h against the 2r dims of its KV head
+#pragma unroll
+      for (int h = 0; h < kHh; ++h) {
+        const int H = kHh * hh + h;
+        const uint4 kw = kr[h];
+        const float4 qa = *reinterpret_cast<const float4*>(qr_s + H * R2);
+        const float4 qb = *reinterpret_cast<const float4*>(qr_s + H * R2 + 4);
+        v[h] += qa.x * bf16lo(kw.x) + qa.y * bf16hi(kw.x) + qa.z * bf16lo(kw.y) + qa.w * bf16hi(kw.y) +
+                qb.x * bf16lo(kw.z) + qb.y * bf16hi(kw.z) + qb.z * bf16lo(kw.w) + qb.w * bf16hi(kw.w);
+      }
+      if (lane == 0) MLA_TRACE(24 + sw, n);
+      {
+        TileIter nx = it;
+        nx.next();
+        if (nx.valid()) {
+          TileIter nx2 = nx;
+          nx2.next();
+          ok = fetch_kr(n + 1, nx2);
+          if (!ok) break;
+        }
+      }
+      if (warp == 4 && lane == 0) MLA_TRACE(10, n);
+      if (!valid) {
+#pragma unroll
+        for (int h = 0; h < kHh; ++h) v[h] = -INFINITY;
+      }
       // does any score exceed its head's running max by more than tau?
       bool need = false;
       if (valid) {
 #pragma unroll
-        for (int h = 0; h < kH; ++h) need |= (v[h] - m[h] > kTau);
+        for (int h = 0; h < kHh; ++h) need |= (v[h] - m[h] > kTau);
       }
       need = __any_sync(0xffffffffu, need);
-      if (lane == 0) misc->vote[n & 1][q] = need ? 1 : 0;
+      if (lane == 0) MLA_TRACE(32 + sw, n);
+      if (lane == 0) misc->vote[n & 1][sw] = need ? 1 : 0;
       ok = grp_sync(0);
       if (!ok) break;
-      const bool need_all = misc->vote[n & 1][0] | misc->vote[n & 1][1] | misc->vote[n & 1][2] | misc->vote[n & 1][3];
-      if (need_all) {
-        float t[kH];
+      bool need_all = false;
 #pragma unroll
-        for (int h = 0; h < kH; ++h) t[h] = v[h];
-        const float wmax = transpose_reduce<true>(t, lane);
-        misc->red_max[n & 1][q][lane] = wmax;
+      for (int i = 0; i < kSoftWarps; ++i) need_all |= misc->vote[n & 1][i] != 0;
+      if (warp == 4 && lane == 0) MLA_TRACE(11, n);
+      if (need_all) {
+        // exact tile max per head: over the 32 tokens of the warp, then over the 4 quarters
+        float wmax = -INFINITY;   // lane h ends with head 16hh + h
+#pragma unroll
+        for (int h = 0; h < kHh; ++h) {
+          const float r = warp_max(v[h]);
+          wmax = (lane == h) ? r : wmax;
+        }
+        if (lane < 16) misc->red_max[n & 1][q][kHh * hh + lane] = wmax;
         ok = grp_sync(1);
         if (!ok) break;
-        float mt = fmaxf(fmaxf(misc->red_max[n & 1][0][lane], misc->red_max[n & 1][1][lane]),
-                         fmaxf(misc->red_max[n & 1][2][lane], misc->red_max[n & 1][3][lane]));
-        misc->mt[q][lane] = mt;
+        if (lane < 16) {
+          const int H = kHh * hh + lane;
+          misc->mt[sw][lane] = fmaxf(fmaxf(misc->red_max[n & 1][0][H], misc->red_max[n & 1][1][H]),
+                                     fmaxf(misc->red_max[n & 1][2][H], misc->red_max[n & 1][3][H]));
+        }
         __syncwarp();
-        float alpha[kH];
         bool any_scale = false;
+        float my_alpha = 1.f;   // the factor of head 16hh + lane (lanes < 16)
 #pragma unroll
-        for (int h = 0; h < kH; ++h) {
-          const float mn = fmaxf(m[h], misc->mt[q][h]);
-          alpha[h] = exp2f(m[h] - mn);   // m = -inf on a piece's first tile -> 0
+        for (int h = 0; h < kHh; ++h) {
+          const float mn = fmaxf(m[h], misc->mt[sw][h]);
+          const float al = exp2f(m[h] - mn);   // m = -inf on a piece's first tile -> 0
           any_scale |= (mn != m[h]);
           m[h] = mn;
-          l[h] *= alpha[h];
+          l[h] *= al;
+          if (h == lane) my_alpha = al;
         }
-        if (!first && any_scale) {
-          // O holds tiles < n of this piece: wait for MMA2(n-1), rescale the columns
+        if (!first && any_scale && q < 2 && hh == q) {
+          // O^T rows of heads 16q .. 16q+15 (lanes 0-15 of quarter q) hold the tiles before
+          // this one: wait for MMA2(n-1), rescale them in TMEM
           const int pn = n - 1;
-          ok = wwait(bars.p_empty(pn & 1), (pn >> 1) & 1);
-          if (!ok) break;
+          if (!wwait(bars.p_empty(pn % a.NP), (pn / a.NP) & 1)) { ok = false; break; }
           tc_fence_after();
-          for (int mc = 0; mc < nchunk; ++mc) {
-            const uint32_t ta = taddr(tmem, 32 * q, O_COL + ob * O_STRIDE + mc * kH);
-            uint32_t o[32];
-            tmem_ld32(ta, o);
+          for (int cc = 0; cc < dc / 16; ++cc) {
+            const uint32_t ta = taddr(tmem, 32 * q, O_COL + ob * dc + 16 * cc);
+            uint32_t o[16];
+            tmem_ld16(ta, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int h = 0; h < kH; ++h) o[h] = f2u(u2f(o[h]) * alpha[h]);
-            tmem_st32(ta, o);
+            for (int k = 0; k < 16; ++k) o[k] = f2u(u2f(o[k]) * my_alpha);
+            tmem_st16(ta, o);
           }
           tmem_wait_st();
         }
       }
-      // probabilities for this tile
-      uint32_t pk[kH / 2];
+      if (warp == 4 && lane == 0) MLA_TRACE(12, n);
+      // probabilities of this tile, P^T for MMA2 (row h, column = token, bf16)
+      float pr[kHh];
 #pragma unroll
-      for (int h = 0; h < kH; h += 2) {
-        const float p0 = valid ? exp2f(v[h] - m[h]) : 0.f;
-        const float p1 = valid ? exp2f(v[h + 1] - m[h + 1]) : 0.f;
-        l[h] += p0;
-        l[h + 1] += p1;
-        pk[h / 2] = pack_bf16x2(p0, p1);
+      for (int h = 0; h < kHh; ++h) {
+        pr[h] = valid ? exp2f(v[h] - m[h]) : 0.f;
+        l[h] += pr[h];
       }
-      if (n >= 2) {
-        ok = wwait(bars.p_empty(pb), ((n - 2) >> 1) & 1);
+      if (warp == 4 && lane == 0) MLA_TRACE(13, n);
+      if (n >= a.NP) {
+        ok = wwait(bars.p_empty(pb), ((n / a.NP) - 1) & 1);
         if (!ok) break;
       }
-      if (lane < 16) {
-        // P as the MN-major (heads contiguous) B operand, no swizzle: core matrices of
-        // 8 heads x 8 tokens; head block at 1024 B, token block at 128 B.
-        uint8_t* P = sbase + a.off_p + pb * kPBytes + (row >> 3) * 128 + (row & 7) * 16;
+      if (warp == 4 && lane == 0) MLA_TRACE(14, n);
+      {
+        uint8_t* Pt = sbase + a.off_p + pb * kPtBytes + (tr >> 6) * kPtAtom + (tr & 7) * 2;
+        const int c8 = (tr & 63) >> 3;
 #pragma unroll
-        for (int hb = 0; hb < 4; ++hb)
-          *reinterpret_cast<uint4*>(P + hb * 1024) =
-              make_uint4(pk[4 * hb], pk[4 * hb + 1], pk[4 * hb + 2], pk[4 * hb + 3]);
-        if (!INT4 && row >= nvalid) {
-          // rows past the sequence end: clear the latent row so MMA2 never multiplies
-          // stale cache contents (0 * NaN would poison O)
-          uint8_t* C = sbase + a.off_c + (n % a.NC) * c_stage + row * 128;
-          for (int cb = 0; cb < n_cbox; ++cb)
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(C + cb * kBox + ch * 16) = make_uint4(0, 0, 0, 0);
+        for (int h = 0; h < kHh; ++h) {
+          const int H = kHh * hh + h;
+          *reinterpret_cast<__nv_bfloat16*>(Pt + H * 128 + ((c8 ^ (H & 7)) << 4)) = __float2bfloat16_rn(pr[h]);
         }
+      }
+      if (!INT4 && !valid) {
+        // rows past the sequence end: clear this token's latent row (both warps of the
+        // quarter take half the boxes) so MMA2 never multiplies stale cache contents
+        uint8_t* C = sbase + a.off_c + (n % a.NC) * c_stage + tr * 128;
+        for (int cb = hh; cb < n_cbox; cb += 2)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(C + cb * kBox + ch * 16) = make_uint4(0, 0, 0, 0);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.p_full(pb));
+      if (warp == 4 && lane == 0) MLA_TRACE(6, n);
 
       if (it.last_of_piece()) {
         // ---------------- piece epilogue: partial (m, l, O) for the split merge
-        float t[kH];
-#pragma unroll
-        for (int h = 0; h < kH; ++h) t[h] = (lane < 16) ? l[h] : 0.f;
-        const float lsum = transpose_reduce<false>(t, lane);
-        misc->red_sum[q][lane] = lsum;
+        const float lsum = transpose_reduce16<false>(l, lane);   // l is reset by the next piece
+        if (lane < 16) misc->red_l[q][kHh * hh + lane] = lsum;
         ok = grp_sync(1);
         if (!ok) break;
-        if (q == 0) {
-          const float L = misc->red_sum[0][lane] + misc->red_sum[1][lane] + misc->red_sum[2][lane] +
-                          misc->red_sum[3][lane];
+        if (q == 0 && lane < 16) {
+          const int H = kHh * hh + lane;
+          const float L = misc->red_l[0][H] + misc->red_l[1][H] + misc->red_l[2][H] + misc->red_l[3][H];
           float mh = m[0];
 #pragma unroll
-          for (int h = 1; h < kH; ++h) mh = (lane == h) ? m[h] : mh;
-          a.mlpart[((size_t)pc * kH + lane) * 2] = mh;
-          a.mlpart[((size_t)pc * kH + lane) * 2 + 1] = L;
+          for (int h = 1; h < kHh; ++h) mh = (lane == h) ? m[h] : mh;
+          a.mlpart[((size_t)H * a.P + pc) * 2] = mh;
+          a.mlpart[((size_t)H * a.P + pc) * 2 + 1] = L;
         }
-        ok = wwait(bars.o_full(ob), (u >> 1) & 1);
+        ok = wwait(bars.o_full(ob), (u / a.NO) & 1);
         if (!ok) break;
         tc_fence_after();
-        for (int mc = 0; mc < nchunk; ++mc) {
-          uint32_t o[32];
-          tmem_ld32(taddr(tmem, 32 * q, O_COL + ob * O_STRIDE + mc * kH), o);
-          tmem_wait_ld();
-          int d;
-          bool dv;
-          if (m2 == 128) { d = mc * 128 + 32 * q + lane; dv = true; }
-          else { d = 16 * q + lane; dv = lane < 16; }
-          if (dv) {
-            float* dst = a.opart + (size_t)pc * kH * dc + d;
+        if (q < 2) {
+          // O^T rows (M = 64 layout): head 16q + lane in lane `lane` (< 16) of quarter q; the
+          // two warps of the quarter take alternate 16-column chunks
+          const int H = 16 * q + lane;
+          float* dst = a.opart + ((size_t)H * a.P + pc) * dc;
+          for (int cc = hh; cc < dc / 16; cc += 2) {
+            uint32_t o[16];
+            tmem_ld16(taddr(tmem, 32 * q, O_COL + ob * dc + 16 * cc), o);
+            tmem_wait_ld();
+            if (lane < 16) {
 #pragma unroll
-            for (int h = 0; h < kH; ++h) dst[(size_t)h * dc] = u2f(o[h]);
+              for (int k = 0; k < 16; k += 4)
+                *reinterpret_cast<float4*>(dst + 16 * cc + k) = make_float4(u2f(o[k]), u2f(o[k + 1]), u2f(o[k + 2]),
+                                                                            u2f(o[k + 3]));
+            }
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.o_empty(ob));
+        if (warp == 4 && lane == 0) MLA_TRACE(9, u);
         ++u;
       }
       it.next();
       ++n;
     }
-  } else if (INT4) {
-    // ============================================================ int4 dequantisation
-    const int dw = warp - 6;
-    const int tok = dw * 16 + (lane & 15);
-    const int half = lane >> 4;                 // which 64-wide box of the 128-wide latent
-    TileIter it;
-    it.init(&a.sched, w);
-    int n = 0;
-    bool ok = true;
-    while (ok && it.valid()) {
-      const int rs = n % a.NRAW, cs = n % a.NC;
-      ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_full(rs), (n / a.NRAW) & 1, abort_flag));
-      if (ok && n >= a.NC)
-        ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag));
-      if (!ok) break;
-      const int nvalid = min(kTile, it.t1 - it.t);
-      const uint8_t* raw = sbase + a.off_raw + rs * raw_stage;
-      uint8_t* C = sbase + a.off_c + cs * c_stage + half * kBox + tok * 128;
-      if (tok < nvalid) {
-        const uint4 c0 = *reinterpret_cast<const uint4*>(raw + tok * (dc / 2) + half * 32);
-        const uint4 c1 = *reinterpret_cast<const uint4*>(raw + tok * (dc / 2) + half * 32 + 16);
-        const __half* sc = reinterpret_cast<const __half*>(raw + raw_codes) + tok * (dc / 32) + half * 2;
-        const float s0 = __half2float(sc[0]), s1 = __half2float(sc[1]);
-        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {           // 8 latent values per 16-byte chunk
-          const uint32_t wd = words[ch];
-          const float s = ch < 4 ? s0 : s1;
-          uint32_t o[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t byte = (wd >> (8 * j)) & 0xFFu;
-            o[j] = pack_bf16x2((float)nib_to_int(byte & 15u) * s, (float)nib_to_int(byte >> 4) * s);
-          }
-          *reinterpret_cast<uint4*>(C + ((ch ^ (tok & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-      } else {
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(C + ch * 16) = make_uint4(0, 0, 0, 0);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bars.raw_empty(rs));
-        mbar_arrive(bars.c_full(cs));
-      }
-      it.next();
-      ++n;
+    // no RoPE key copy may still be landing when the CTA exits
+    if (sw == 0 && lane == 0 && misc->kr_issued > 0) {
+      volatile int never = 0;
+      mbar_wait(bars.kr_full(), (misc->kr_issued - 1) & 1, &never);
     }
   }
 
@@ -571,6 +734,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
     tmem_dealloc(tmem, tmem_cols);
   }
   if (threadIdx.x == 0 && misc->abort_flag) raise_error(a.err, MLA_DEVERR_TIMEOUT);
+  if (threadIdx.x == 0) MLA_TRACE(8, 0);
+#ifdef MLA_TC_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 1024) g_cta_span[2 * blockIdx.x + 1] = globaltimer();
+#endif
 }
 
 // ------------------------------------------------------------------ host side
@@ -603,38 +770,44 @@ static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base
 }
 
 struct TcLayout {
-  int NC, NK, NRAW;
-  uint32_t off_c, off_kr, off_q, off_p, off_raw, off_bar, off_misc, total;
+  int NC, NRAW, NP, NO;
+  uint32_t off_c, off_q, off_p, off_raw, off_qr, off_kr, off_bar, off_misc, total;
 };
 
-static TcLayout tc_layout(int dc, int R, int K, bool int4) {
-  const uint32_t budget = 232448 - 1024;  // max dynamic smem per block minus alignment slack
-  const uint32_t c_stage = (uint32_t)(dc / 64) * kBox, kr_stage = (uint32_t)(R / 64) * kBox;
+static TcLayout tc_layout(int dc, int R, int r2, bool int4) {
+  const uint32_t budget = 232448 - 1024;   // max dynamic smem per block minus alignment slack
+  const uint32_t c_stage = (uint32_t)(dc / 64) * kBox;
   const uint32_t raw_stage = (uint32_t)kTile * (dc / 2) + (uint32_t)kTile * (dc / 16);
-  const uint32_t q_bytes = (uint32_t)(K / 64) * kQBox;
-  TcLayout L{};
-  auto size = [&](int nc, int nk, int nraw) {
-    uint32_t s = nc * c_stage + nk * kr_stage + q_bytes + 2 * kPBytes;
+  const uint32_t q_bytes = (uint32_t)(dc / 64 > 2 ? dc / 64 - 2 : 0) * kQBox;  // boxes 0-1 sit in P^T padding
+  const uint32_t qr_bytes = (uint32_t)kH * r2 * 4;
+  const uint32_t kr_bytes = (uint32_t)kTile * R * 2;
+  auto size = [&](int nc, int nraw, int np) {
+    uint32_t s = nc * c_stage + q_bytes + np * kPtBytes + kr_bytes;
     s += int4 ? ((nraw * raw_stage + 1023) & ~1023u) : 0;
-    s += 8 * (2 * nc + 2 * nk + 2 * nraw + 17) + sizeof(Misc) + 64;
+    s += qr_bytes + 8 * (2 * nc + 2 * nraw + kFixedBars) + sizeof(Misc) + 64;
     return s;
   };
-  int nc = 2, nk = 2, nraw = int4 ? 2 : 0;
-  for (int it = 0; it < 12; ++it) {  // grow the rings while they fit, KR first (largest stream)
+  int nc = 2, np = 1, nraw = int4 ? 2 : 0;
+  for (int it = 0; it < 16; ++it) {  // deepen the rings while they fit (latent stages first)
     bool grew = false;
-    if (nk < 6 && size(nc, nk + 1, nraw) <= budget) { ++nk; grew = true; }
-    if (int4 && nraw < 6 && size(nc, nk, nraw + 1) <= budget) { ++nraw; grew = true; }
-    if (nc < 6 && size(nc + 1, nk, nraw) <= budget) { ++nc; grew = true; }
+    if (nc < 6 && size(nc + 1, nraw, np) <= budget) { ++nc; grew = true; }
+    if (np < 2 && size(nc, nraw, np + 1) <= budget) { ++np; grew = true; }
+    if (int4 && nraw < 4 && size(nc, nraw + 1, np) <= budget) { ++nraw; grew = true; }
     if (!grew) break;
   }
-  L.NC = nc; L.NK = nk; L.NRAW = nraw;
+  TcLayout L{};
+  L.NC = nc; L.NRAW = nraw; L.NP = np;
+  L.NO = (2 * kH + 2 * dc) <= 512 ? 2 : 1;
   uint32_t o = 0;
   L.off_c = o; o += nc * c_stage;
-  L.off_kr = o; o += nk * kr_stage;
+  L.off_p = o; o += np * kPtBytes;
   L.off_q = o; o += q_bytes;
-  L.off_p = o; o += 2 * kPBytes;
   L.off_raw = o; o += int4 ? ((nraw * raw_stage + 1023) & ~1023u) : 0;
-  L.off_bar = o; o += 8 * (2 * nc + 2 * nk + 2 * nraw + 17);
+  L.off_qr = o; o += qr_bytes;
+  o = (o + 127) & ~127u;
+  L.off_kr = o; o += kr_bytes;
+  o = (o + 15) & ~15u;
+  L.off_bar = o; o += 8 * (2 * nc + 2 * nraw + kFixedBars);
   o = (o + 15) & ~15u;
   L.off_misc = o; o += sizeof(Misc);
   L.total = o + 1024;
@@ -644,14 +817,16 @@ static TcLayout tc_layout(int dc, int R, int K, bool int4) {
 }  // namespace tc
 }  // namespace mla
 
-// Shapes the tensor-core kernel covers: bf16, 32 heads, d_c in {64, 128, 256}, RoPE
-// width a multiple of 64; the int4 cache with d_c = 128.
+// Shapes the tensor-core kernel covers: bf16, 32 query heads, d_c in {64, 128, 256}, r = 4
+// kept pairs per KV head (RoPE width a multiple of 64); the int4 cache with d_c = 128.
 bool mla_tc_capable(const mla_plan& p) {
   const mla_config_t& cfg = p.cfg;
   if (cfg.dtype != MLA_BF16 || cfg.n_heads != mla::tc::kH) return false;
-  if (cfg.d_c % 64 != 0 || cfg.d_c > 256 || p.R % 64 != 0 || p.R == 0) return false;
+  if (cfg.d_c % 64 != 0 || cfg.d_c > 256) return false;
+  if (p.R == 0 || p.R % 64 != 0 || 2 * cfg.r_pairs != 8) return false;   // 2r = 8 (r = 4) build
   if (cfg.cache_kind == MLA_CACHE_INT4_G32 && cfg.d_c != 128) return false;
-  return true;
+  const mla::tc::TcLayout L = mla::tc::tc_layout(cfg.d_c, p.R, 2 * cfg.r_pairs, cfg.cache_kind == MLA_CACHE_INT4_G32);
+  return L.total <= 232448;
 }
 
 // The int4 scale rows are fetched with 1-D bulk copies, which need an even capacity.
@@ -662,12 +837,13 @@ bool mla_tc_supported(const mla_plan& p, const mla_cache_t& c) {
 }
 
 cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, int B, const Sched& sched,
-                                 const void* qcat, float* opart, float* mlpart, int G, cudaStream_t s) {
+                                 const void* qlat, const float* qrope, float* opart, float* mlpart, int P, int G,
+                                 cudaStream_t s) {
   using namespace mla::tc;
   const mla_config_t& cfg = p.cfg;
   const bool int4 = cfg.cache_kind == MLA_CACHE_INT4_G32;
-  const int dc = cfg.d_c, R = p.R, K = dc + R;
-  CUtensorMap tm_c, tm_kr, tm_q;
+  const int dc = cfg.d_c, R = p.R;
+  CUtensorMap tm_c, tm_q;
   const uint64_t rows = (uint64_t)c.B * c.T_cap;
   bool ok = true;
   if (int4)
@@ -676,22 +852,44 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, int B,
   else
     ok &= make_map_2d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.c_kv, dc, rows, (uint64_t)dc * 2, 64, kTile,
                       CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map_2d(&tm_kr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.k_rope, R, rows, (uint64_t)R * 2, 64, kTile,
-                    CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qcat, K, (uint64_t)B * kH, (uint64_t)K * 2, 64, kH,
+  ok &= make_map_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qlat, dc, (uint64_t)B * kH, (uint64_t)dc * 2, 64, kH,
                     CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
-  TcLayout L = tc_layout(dc, R, K, int4);
+  const TcLayout L = tc_layout(dc, R, 2 * cfg.r_pairs, int4);
   TcArgs a;
-  a.B = B; a.H = kH; a.d_c = dc; a.R = R; a.K = K; a.T_cap = c.T_cap;
-  a.sched = sched; a.opart = opart; a.mlpart = mlpart;
+  a.B = B; a.H = kH; a.d_c = dc; a.R = R; a.r2 = 2 * cfg.r_pairs; a.T_cap = c.T_cap; a.P = P;
+  a.sched = sched; a.opart = opart; a.mlpart = mlpart; a.qrope = qrope;
   a.scales = (const __half*)c.c_scales; a.err = p.err;
-  a.NC = L.NC; a.NK = L.NK; a.NRAW = L.NRAW;
-  a.off_c = L.off_c; a.off_kr = L.off_kr; a.off_q = L.off_q; a.off_p = L.off_p; a.off_raw = L.off_raw;
-  a.off_bar = L.off_bar; a.off_misc = L.off_misc;
-  auto kern = int4 ? decode_tc_kernel<true> : decode_tc_kernel<false>;
+  a.kr_base = (const uint8_t*)c.k_rope;
+  a.c_row = int4 ? (uint32_t)dc / 2 : (uint32_t)dc * 2;
+  a.kr_row = (uint32_t)R * 2;
+  a.NC = L.NC; a.NRAW = L.NRAW; a.NP = L.NP; a.NO = L.NO;
+  a.off_c = L.off_c; a.off_q = L.off_q; a.off_p = L.off_p; a.off_raw = L.off_raw;
+  a.off_qr = L.off_qr; a.off_kr = L.off_kr; a.off_bar = L.off_bar; a.off_misc = L.off_misc;
+  // the RoPE width per KV head is a compile-time constant so the score loop fully unrolls
+  // and the per-head registers never move to local memory
+  auto kern = int4 ? decode_tc_kernel<true, 8> : decode_tc_kernel<false, 8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
-  kern<<<G, int4 ? 320 : 192, L.total, s>>>(tm_c, tm_kr, tm_q, a);
-  return cudaGetLastError();
+  // the optional profiling events bracket the launch alone, after all host-side set-up
+  if ((e = mla_profile_event(p, 0, s)) != cudaSuccess) return e;
+  kern<<<G, 384, L.total, s>>>(tm_c, tm_q, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if ((e = mla_profile_event(p, 1, s)) != cudaSuccess) return e;
+  return cudaSuccess;
 }
+
+#ifdef MLA_TC_TRACE
+extern "C" __attribute__((visibility("default"))) int mla_tc_trace_read(unsigned long long* host, int n) {
+  const int total = mla::tc::kTraceCtas * mla::tc::kTraceEv * mla::tc::kTraceTiles;
+  if (n < total) return -1;
+  if (cudaMemcpyFromSymbol(host, mla::tc::g_trace, sizeof(unsigned long long) * total) != cudaSuccess) return -2;
+  return total;
+}
+extern "C" __attribute__((visibility("default"))) int mla_tc_span_read(unsigned long long* host, int n) {
+  if (n < 2048) return -1;
+  if (cudaMemcpyFromSymbol(host, mla::tc::g_cta_span, sizeof(unsigned long long) * 2048) != cudaSuccess) return -2;
+  return 2048;
+}
+#endif

@@ -6,6 +6,13 @@
 
 #include "mla_api.h"
 
+// Element offset of RoPE key dim j of KV head g, token t of sequence b, in the blocked
+// k_rope layout [B][ceil(T_cap/32)][n_kv][32][2r].
+inline __host__ __device__ size_t mla_kr_offset(int b, int t, int g, int j, int T_cap, int n_kv, int r2) {
+  const size_t blocks = (size_t)(T_cap + 31) / 32;
+  return (((size_t)b * blocks + (size_t)(t >> 5)) * n_kv + g) * 32u * r2 + (size_t)(t & 31) * r2 + j;
+}
+
 struct mla_plan {
   mla_config_t cfg;
   int device = 0;
@@ -26,6 +33,19 @@ struct mla_plan {
   int opt_splits = 0;
   const void* const* opt_events = nullptr;  // cudaEvent_t[2] or null
 };
+
+// Records profiling event i (0 before, 1 after the split-K kernel) when the option is set.
+// Under stream capture the record becomes an external event node of the graph, so the
+// event still marks each replay.  A failed record is returned, never left pending.
+inline cudaError_t mla_profile_event(const mla_plan& p, int i, cudaStream_t s) {
+  if (!p.opt_events) return cudaSuccess;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(s, &cs);
+  if (e != cudaSuccess) return e;
+  return cudaEventRecordWithFlags((cudaEvent_t)p.opt_events[i], s,
+                                  cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal
+                                                                      : cudaEventRecordDefault);
+}
 
 // Decode workspace layout (byte offsets from the workspace base).
 struct DecodeLayout {
@@ -57,7 +77,8 @@ DecodeLayout mla_decode_layout(const mla_plan& p, int B, int kernel);
 bool mla_tc_supported(const mla_plan& p, const mla_cache_t& c);
 bool mla_tc_capable(const mla_plan& p);   // shape/dtype allow the tensor-core kernel
 cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, int B, const Sched& sched,
-                                 const void* qcat, float* opart, float* mlpart, int G, cudaStream_t s);
+                                 const void* qlat, const float* qrope, float* opart, float* mlpart, int P, int G,
+                                 cudaStream_t s);
 Sched mla_sched_view(const DecodeLayout& L, void* ws, int B);
 
 cudaError_t mla_launch_select_pairs(const mla_config_t& cfg, const void* q, const void* k, int T,

@@ -132,7 +132,7 @@ def upload_oracle_cache(case: OracleCase, cache, T_cap):
         else:
             cache.c_kv[b, :L] = gen.to_torch(cc["c"], wl.dtype, cache.c_kv.device)
         if cache.k_rope is not None:
-            cache.k_rope[b, :L] = gen.to_torch(cc["kr"], wl.dtype, cache.k_rope.device)
+            cache.set_k_rope_tokens(b, 0, gen.to_torch(cc["kr"], wl.dtype, cache.k_rope.device))
 
 
 def plan_inputs(case: OracleCase):

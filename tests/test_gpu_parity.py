@@ -98,7 +98,7 @@ def test_append_parity(wl):
         if L == 0:
             continue
         cc = case.cache[b]
-        kr = cache.k_rope[b, :L].double().cpu().numpy()
+        kr = cache.k_rope_tokens(b, 0, L).double().cpu().numpy()
         assert_stored_close(kr, cc["kr_exact"], wl.dtype, f"k_rope seq {b}")
         if wl.cache == "int4_g32":
             codes = O.unpack_int4(cache.c_kv[b, :L].cpu().numpy())
@@ -110,6 +110,32 @@ def test_append_parity(wl):
         else:
             c = cache.c_kv[b, :L].double().cpu().numpy()
             assert_stored_close(c, cc["c_exact"], wl.dtype, f"latent seq {b}")
+
+
+@pytest.mark.parametrize("wl", PARITY_WORKLOADS, ids=IDS)
+def test_append_decode_step_batch(wl):
+    """The decode-step shape: one new token per sequence (N = B) appended at L_b - 1."""
+    case = case_for(wl)
+    cfg, plan = make_plan(case)
+    T_cap = max(1, int(max(case.lens)))
+    cache = LatentCache(cfg, wl.batch, T_cap, "cuda")
+    seqs = [b for b in case.seqs if case.lens[b] > 0]
+    x = np.stack([case.x_dec[b] for b in seqs])
+    mla.mla_append(plan, gen.to_torch(x, wl.dtype, "cuda"), torch.tensor(seqs, dtype=torch.int32, device="cuda"),
+                   torch.tensor([int(case.lens[b]) - 1 for b in seqs], dtype=torch.int32, device="cuda"),
+                   cache.struct)
+    assert mla.mla_device_error(plan) == 0
+    for b in seqs:
+        p_ = int(case.lens[b]) - 1
+        cc = case.cache[b]
+        assert_stored_close(cache.k_rope_tokens(b, p_, p_ + 1)[0].double().cpu().numpy(), cc["kr_exact"][p_],
+                            wl.dtype, f"kr {b}")
+        if wl.cache == "int4_g32":
+            codes = O.unpack_int4(cache.c_kv[b, p_:p_ + 1].cpu().numpy())
+            deq = O.dequant_int4_g32(codes, cache.c_scales[b, p_:p_ + 1].cpu().numpy())
+            assert_close(deq[0], cc["c"][p_], wl.dtype, f"int4 latent {b}")
+        else:
+            assert_stored_close(cache.c_kv[b, p_].double().cpu().numpy(), cc["c_exact"][p_], wl.dtype, f"c {b}")
 
 
 def test_append_int4_codes_bit_exact_on_exact_latents():
@@ -138,12 +164,12 @@ def test_decode_parity(wl, kernel):
     """kernel 0: the plan's choice; 1: CUDA-core split-K; 2: tcgen05 (bf16, 32 heads)."""
     case = case_for(wl)
     cfg, plan = make_plan(case, kernel=kernel)
-    try:
-        got = run_decode(case, plan, cfg)
-    except mla.MlaError as e:
-        if kernel == 2 and e.status == mla.MLA_ERR_UNSUPPORTED:
-            pytest.skip("shape outside the tensor-core kernel (fp32 or H != 32)")
-        raise
+    if kernel == 2 and (wl.dtype == "f32" or wl.n_heads != 32):
+        with pytest.raises(mla.MlaError) as ei:
+            run_decode(case, plan, cfg)
+        assert ei.value.status == mla.MLA_ERR_UNSUPPORTED
+        pytest.skip("shape outside the tensor-core kernel (fp32 or H != 32)")
+    got = run_decode(case, plan, cfg)
     assert mla.mla_device_error(plan) == 0
     for b in case.seqs:
         assert_close(got[b], case.reference(b), wl.dtype, f"decode seq {b} (L={case.lens[b]})")
