@@ -72,7 +72,7 @@ typedef struct {
   int32_t n_kv_heads;   /* n_kv */
   int32_t head_dim;     /* d_h, even */
   int32_t r_pairs;      /* r, 0 <= r <= d_h/2 */
-  int32_t d_c;          /* latent width (multiple of 32 for the int4 cache) */
+  int32_t d_c;          /* latent width, multiple of 4 (of 32 for the int4 cache) */
   double rope_base;     /* RoPE base (10000 for the Llama/SmolLM shapes) */
   int32_t dtype;        /* mla_dtype_t */
   int32_t cache_kind;   /* mla_cache_kind_t (int4 requires dtype MLA_BF16) */
@@ -100,10 +100,14 @@ enum {
   MLA_OPT_DECODE_KERNEL = 1,  /* 0 auto, 1 CUDA-core split-K kernel, 2 tcgen05 kernel */
   MLA_OPT_DECODE_SPLITS = 2,  /* 0 auto (SM count based); n > 0: split the context
                                  tiles into n contiguous worker ranges */
-  MLA_OPT_PROFILE_EVENTS = 3  /* value: address of a host array of two cudaEvent_t; each
+  MLA_OPT_PROFILE_EVENTS = 3, /* value: address of a host array of two cudaEvent_t; each
                                  mla_decode records [0] just before and [1] just after its
                                  split-K attention kernel on the call's stream (0 = off).
                                  The array must stay valid while the option is set. */
+  MLA_OPT_OVERLAP_LAUNCH = 4  /* 1 (default): launch the kernels of mla_append / mla_decode
+                                 with programmatic stream serialization, so each one's
+                                 independent prologue (weight loads, set-up) overlaps the
+                                 tail of the kernel before it; 0: plain stream order */
 };
 
 MLA_API const char* mla_status_string(mla_status_t s);

@@ -12,7 +12,11 @@
 // (deterministic), which then runs the epilogue.
 #include <cooperative_groups.h>
 
+#include <algorithm>
+
 #include "common.cuh"
+#include "sm100.cuh"
+#include "warp_mma.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -140,6 +144,8 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
     __syncthreads();
   }
 
+  pdl_wait();   // the cache may still be read by the kernel before this one
+  pdl_trigger();
   // Partial tile to shared memory; cluster reduction when the hidden dim is split.
 #pragma unroll
   for (int i = 0; i < 2; ++i)
@@ -169,120 +175,111 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   append_epilogue<T, INT4, kAppTokens, kAppCols>(a, &red[0][0], tok0, col0);
 }
 
-// Decode-step append (few tokens): a CTA computes 32 tokens x 32 packed columns over one
-// eighth of the hidden dim.  It loads its whole x and W slices up front (16-byte vector
-// loads, all in flight together), accumulates 4x4 register tiles in four hidden-dim
-// groups, and the eight CTAs of the cluster sum their tiles over distributed shared
-// memory (fixed rank order) before rank 0 runs the epilogue.
-constexpr int kSmTok = 32, kSmCols = 32, kSmSplit = 8;
+// Decode-step append (few tokens).  The product out[N][ncols] = x W_app is split into
+// 32-token x 32-column tiles and kAppSplit slices of the hidden dim, one CTA each.  A CTA
+// stages its x and W slices in one batch of loads, its eight warps each take an eighth of
+// the slice with 8 x 4 register tiles, and the warps' tiles are summed in shared memory.
+// The slice's partial tile goes to the plan's scratch; the last CTA of a tile to finish
+// (ticket counter) sums the kAppSplit partials in slice order (deterministic) and runs the
+// epilogue, whose per-token and per-column inputs every CTA prefetched at its start.
+constexpr int kSmTok = 32, kSmCols = 32, kAppSplit = 8;
 
+struct AppendSmallArgs {
+  AppendArgs a;
+  float* part;        // [kAppSplit][tiles][32 * 32] partial tiles
+  int32_t* ticket;    // [tiles] arrival counters (the last CTA resets its counter)
+};
+
+// Second half of the decode-step append, after the eight warps' 32 x 32 tiles of this hidden-dim
+// slice are in red[8][32 * 32]: sum them into the slice's partial, and let the last CTA of the
+// tile sum the partials in slice order and write the cache (latent, RoPE keys rotated at the
+// token's position, int4 codes).
 template <typename T, bool INT4>
-__global__ void __launch_bounds__(256) append_small_kernel(AppendArgs a) {
-  MLA_KSPAN(0);
-  extern __shared__ __align__(16) float smf[];
-  const int ks = a.kslice;                       // multiple of 32
-  float* xs = smf;                               // [ks][kSmTok]   (k-major)
-  float* ws = xs + ks * kSmTok;                  // [ks][kSmCols]
-  float* red = ws + ks * kSmCols;                // [4][kSmTok][kSmCols]
-  const int tid = threadIdx.x;
-  const int col0 = blockIdx.x * kSmCols, tok0 = blockIdx.y * kSmTok;
-  const int rank = blockIdx.z;
-  const int k_begin = rank * ks, k_end = min(a.d, k_begin + ks);
-  const T* x = (const T*)a.x;
-  const T* W = (const T*)a.W;
-  constexpr int VEC = 16 / sizeof(T);
-  // x slice [32 tokens][ks] and W slice [ks][32 columns]: batches of eight 16-byte loads per
-  // thread are all issued before any is stored, so each batch costs one memory round trip.
-  // x: consecutive threads take consecutive tokens so the transposed stores do not collide.
-  const int nxv = kSmTok * (ks / VEC), nwv = ks * (kSmCols / VEC);
-  for (int base = 0; base < nxv + nwv; base += 8 * 256) {
-    uint4 r[8];
+__device__ __forceinline__ void append_small_finish(const AppendSmallArgs& sa, float* red, const int* s_sq,
+                                                    const int* s_pos, const double* s_theta, int* s_last,
+                                                    int tok0, int col0, int tile, int ntile, int split) {
+  const AppendArgs& a = sa.a;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // the scratch and the cache may still be in use by the kernels before this one
+  pdl_wait();
+  pdl_trigger();
+  float* my_part = sa.part + ((size_t)split * ntile + tile) * (kSmTok * kSmCols);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int v = base + tid + 256 * k;
-      r[k] = make_uint4(0, 0, 0, 0);
-      if (v < nxv) {
-        const int t = v % kSmTok, ch = v / kSmTok;
-        const int n = tok0 + t, kd = k_begin + ch * VEC;
-        if (n < a.N && kd + VEC <= k_end && a.vec_ok)
-          r[k] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * a.d + kd));
-      } else if (v < nxv + nwv) {
-        const int vw = v - nxv;
-        const int kk = vw / (kSmCols / VEC), part = vw % (kSmCols / VEC);
-        const int kd = k_begin + kk, col = col0 + part * VEC;
-        if (kd < k_end && col + VEC <= a.ncols && a.vec_ok)
-          r[k] = __ldg(reinterpret_cast<const uint4*>(W + (size_t)kd * a.ncols + col));
+  for (int e = 0; e < 4; ++e) {
+    const int o = tid + 256 * e;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[w * kSmTok * kSmCols + o];
+    my_part[o] = v;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int prev = atomicAdd(sa.ticket + tile, 1);
+    *s_last = prev == kAppSplit - 1;
+    if (*s_last) sa.ticket[tile] = 0;   // ready for the next call
+  }
+  __syncthreads();
+  if (!*s_last) return;
+  __threadfence();
+  // ---- last CTA of the tile: sum the partials in slice order, then the epilogue
+  float* tileb = red;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int o = tid + 256 * e;
+    float v = 0.f;
+    for (int sp = 0; sp < kAppSplit; ++sp) v += __ldcg(sa.part + ((size_t)sp * ntile + tile) * (kSmTok * kSmCols) + o);
+    tileb[o] = v;
+  }
+  __syncthreads();
+  const mla_cache_t& c = a.cache;
+  const int n_kv = a.R / max(2 * a.r, 1);
+  for (int i = tid; i < kSmTok * (kSmCols / 2); i += 256) {
+    const int t = i / (kSmCols / 2), cp = i % (kSmCols / 2);
+    const int n = tok0 + t, col = col0 + 2 * cp;
+    if (n >= a.N || col >= a.ncols) continue;
+    const int sq = s_sq[t], p = s_pos[t];
+    if (sq < 0 || sq >= c.B || p < 0 || p >= c.T_cap) {
+      if (col == 0) raise_error(a.err, MLA_DEVERR_APPEND_SLOT);
+      continue;
+    }
+    const float v0 = tileb[t * kSmCols + 2 * cp], v1 = tileb[t * kSmCols + 2 * cp + 1];
+    if (col < a.d_c) {
+      if (!INT4) {
+        T* dst = (T*)c.c_kv + ((size_t)sq * c.T_cap + p) * a.d_c + col;
+        dst[0] = from_f32<T>(v0);
+        dst[1] = from_f32<T>(v1);
       }
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int v = base + tid + 256 * k;
-      float f[VEC];
-      const T* e = reinterpret_cast<const T*>(&r[k]);
-      if (v < nxv) {
-        const int t = v % kSmTok, ch = v / kSmTok;
-        const int n = tok0 + t, kd = k_begin + ch * VEC;
-        const bool whole = n < a.N && kd + VEC <= k_end && a.vec_ok;
-#pragma unroll
-        for (int q = 0; q < VEC; ++q)
-          f[q] = whole ? to_f32(e[q]) : ((n < a.N && kd + q < k_end) ? ldg_f32(x + (size_t)n * a.d + kd + q) : 0.f);
-#pragma unroll
-        for (int q = 0; q < VEC; ++q) xs[(ch * VEC + q) * kSmTok + t] = f[q];
-      } else if (v < nxv + nwv) {
-        const int vw = v - nxv;
-        const int kk = vw / (kSmCols / VEC), part = vw % (kSmCols / VEC);
-        const int kd = k_begin + kk, col = col0 + part * VEC;
-        const bool whole = kd < k_end && col + VEC <= a.ncols && a.vec_ok;
-#pragma unroll
-        for (int q = 0; q < VEC; ++q)
-          f[q] = whole ? to_f32(e[q])
-                       : ((kd < k_end && col + q < a.ncols) ? ldg_f32(W + (size_t)kd * a.ncols + col + q) : 0.f);
-#pragma unroll
-        for (int q = 0; q < VEC; ++q) ws[kk * kSmCols + part * VEC + q] = f[q];
-      }
+    } else {
+      const int rc = col - a.d_c;
+      double sn, cs;
+      sincos((double)p * s_theta[cp], &sn, &cs);
+      T* dst = (T*)c.k_rope + mla_kr_offset(sq, p, rc / (2 * a.r), rc % (2 * a.r), c.T_cap, n_kv, 2 * a.r);
+      dst[0] = from_f64<T>((double)v0 * cs - (double)v1 * sn);
+      dst[1] = from_f64<T>((double)v0 * sn + (double)v1 * cs);
     }
   }
-  __syncthreads();
-  // 4 hidden-dim groups x (8 token quads x 8 column quads)
-  const int kg = tid / 64, tt = (tid % 64) / 8, cc = tid % 8;
-  float acc[4][4] = {};
-  const int kq = ks / 4;
-#pragma unroll 4
-  for (int kk = kg * kq; kk < (kg + 1) * kq; ++kk) {
-    const float4 xv = *reinterpret_cast<const float4*>(&xs[kk * kSmTok + tt * 4]);
-    const float4 wv = *reinterpret_cast<const float4*>(&ws[kk * kSmCols + cc * 4]);
-    const float xa[4] = {xv.x, xv.y, xv.z, xv.w}, wa[4] = {wv.x, wv.y, wv.z, wv.w};
+  if (INT4 && col0 < a.d_c) {
+    // one warp per token: the tile's 32 latent columns are one quantisation group
+    for (int t = warp; t < kSmTok; t += 8) {
+      const int n = tok0 + t;
+      const int sq = s_sq[t], p = s_pos[t];
+      if (n >= a.N || sq < 0 || sq >= c.B || p < 0 || p >= c.T_cap) continue;
+      const size_t slot = (size_t)sq * c.T_cap + p;
+      const float v = tileb[t * kSmCols + lane];
+      float am = fabsf(v);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] += xa[i] * wa[j];
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) red[(kg * kSmTok + tt * 4 + i) * kSmCols + cc * 4 + j] = acc[i][j];
-  __syncthreads();
-  float* tile = red;   // group sums into group 0's slot
-  for (int i = tid; i < kSmTok * kSmCols; i += 256)
-    tile[i] = red[i] + red[kSmTok * kSmCols + i] + red[2 * kSmTok * kSmCols + i] + red[3 * kSmTok * kSmCols + i];
-  cg::cluster_group cluster = cg::this_cluster();
-  cluster.sync();
-  float fin[kSmTok * kSmCols / 256];
-  if (rank == 0) {
-#pragma unroll
-    for (int e = 0; e < kSmTok * kSmCols / 256; ++e) fin[e] = tile[tid + 256 * e];
-    for (int rr = 1; rr < (int)gridDim.z; ++rr) {
-      const float* remote = cluster.map_shared_rank(tile, rr);
-#pragma unroll
-      for (int e = 0; e < kSmTok * kSmCols / 256; ++e) fin[e] += remote[tid + 256 * e];
+      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      const __half sh = __float2half_rn(__fdiv_rn(am, 7.0f));
+      const float sc = __half2float(sh);
+      int code = 0;
+      if (sc > 0.f) code = max(-7, min(7, (int)rintf(__fdiv_rn(v, sc))));
+      const uint32_t nib = (uint32_t)code & 15u;
+      const uint32_t hi = __shfl_down_sync(0xffffffffu, nib, 1);
+      if ((lane & 1) == 0) ((uint8_t*)c.c_kv)[slot * (a.d_c / 2) + (col0 + lane) / 2] = (uint8_t)(nib | (hi << 4));
+      if (lane == 0) ((__half*)c.c_scales)[slot * (a.d_c / 32) + col0 / 32] = sh;
     }
   }
-  cluster.sync();  // remote tiles stay alive until rank 0 has read them
-  if (rank != 0) return;
-#pragma unroll
-  for (int e = 0; e < kSmTok * kSmCols / 256; ++e) tile[tid + 256 * e] = fin[e];
-  __syncthreads();
-  append_epilogue<T, INT4, kSmTok, kSmCols>(a, tile, tok0, col0);
 }
 
 template <typename T, bool INT4>
@@ -303,23 +300,240 @@ cudaError_t launch_append_t(const AppendArgs& args, int ksplit, cudaStream_t s) 
 }
 
 template <typename T, bool INT4>
-cudaError_t launch_append_small_t(const AppendArgs& args, cudaStream_t s) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((args.ncols + kSmCols - 1) / kSmCols, (args.N + kSmTok - 1) / kSmTok, kSmSplit);
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = sizeof(float) * ((size_t)args.kslice * (kSmTok + kSmCols) + 4 * kSmTok * kSmCols);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = kSmSplit;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaFuncSetAttribute(append_small_kernel<T, INT4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)cfg.dynamicSmemBytes);
+__global__ void __launch_bounds__(256) append_small_kernel(AppendSmallArgs sa) {
+  MLA_KSPAN(0);
+  const AppendArgs& a = sa.a;
+  extern __shared__ __align__(16) float smf[];
+  const int ks = a.kslice;                       // multiple of 64
+  float* xs = smf;                               // [ks][kSmTok]   (k-major)
+  float* ws = xs + ks * kSmTok;                  // [ks][kSmCols]
+  float* red = xs;                               // [8][kSmTok * kSmCols], after the product
+  __shared__ int s_sq[kSmTok], s_pos[kSmTok];
+  __shared__ double s_theta[kSmCols / 2];
+  __shared__ int s_last;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int col0 = blockIdx.x * kSmCols, tok0 = blockIdx.y * kSmTok;
+  const int split = blockIdx.z;
+  const int tile = blockIdx.y * gridDim.x + blockIdx.x, ntile = gridDim.x * gridDim.y;
+  const int k_begin = split * ks, k_end = min(a.d, k_begin + ks);
+  const T* x = (const T*)a.x;
+  const T* W = (const T*)a.W;
+  constexpr int VEC = 16 / sizeof(T);
+  // ---- epilogue inputs (token slots, rotation frequencies), prefetched
+  if (tid < kSmTok) {
+    const int n = tok0 + tid;
+    s_sq[tid] = n < a.N ? __ldg(a.seq_idx + n) : -1;
+    s_pos[tid] = n < a.N ? __ldg(a.pos + n) : -1;
+  } else if (tid < kSmTok + kSmCols / 2) {
+    const int cp = tid - kSmTok, col = col0 + 2 * cp;
+    double th = 0.0;
+    if (col >= a.d_c && col < a.ncols) {
+      const int rc = col - a.d_c, g = rc / (2 * a.r), j = (rc % (2 * a.r)) / 2;
+      th = __ldg(a.theta + __ldg(a.rope_pair + g * a.r + j));
+    }
+    s_theta[cp] = th;
+  }
+  // ---- x slice -> xs[k][t] and W slice -> ws[k][c]: 8 loads per thread in flight
+  {
+    const int nxv = kSmTok * (ks / VEC), nwv = ks * (kSmCols / VEC);
+    for (int base = 0; base < nxv + nwv; base += 8 * 256) {
+      uint4 r[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int v = base + tid + 256 * k;
+        r[k] = make_uint4(0, 0, 0, 0);
+        if (v < nxv) {
+          const int t = v % kSmTok, ch = v / kSmTok;
+          const int n = tok0 + t, kd = k_begin + ch * VEC;
+          if (n < a.N && kd + VEC <= k_end && a.vec_ok)
+            r[k] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * a.d + kd));
+        } else if (v < nxv + nwv) {
+          const int vw = v - nxv;
+          const int kk = vw / (kSmCols / VEC), part = vw % (kSmCols / VEC);
+          const int kd = k_begin + kk, col = col0 + part * VEC;
+          if (kd < k_end && col + VEC <= a.ncols && a.vec_ok)
+            r[k] = __ldg(reinterpret_cast<const uint4*>(W + (size_t)kd * a.ncols + col));
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int v = base + tid + 256 * k;
+        float f[VEC];
+        const T* e = reinterpret_cast<const T*>(&r[k]);
+        if (v < nxv) {
+          const int t = v % kSmTok, ch = v / kSmTok;
+          const int n = tok0 + t, kd = k_begin + ch * VEC;
+          const bool whole = n < a.N && kd + VEC <= k_end && a.vec_ok;
+#pragma unroll
+          for (int q = 0; q < VEC; ++q)
+            f[q] = whole ? to_f32(e[q]) : ((n < a.N && kd + q < k_end) ? ldg_f32(x + (size_t)n * a.d + kd + q) : 0.f);
+#pragma unroll
+          for (int q = 0; q < VEC; ++q) xs[(ch * VEC + q) * kSmTok + t] = f[q];
+        } else if (v < nxv + nwv) {
+          const int vw = v - nxv;
+          const int kk = vw / (kSmCols / VEC), part = vw % (kSmCols / VEC);
+          const int kd = k_begin + kk, col = col0 + part * VEC;
+          const bool whole = kd < k_end && col + VEC <= a.ncols && a.vec_ok;
+#pragma unroll
+          for (int q = 0; q < VEC; ++q)
+            f[q] = whole ? to_f32(e[q])
+                         : ((kd < k_end && col + q < a.ncols) ? ldg_f32(W + (size_t)kd * a.ncols + col + q) : 0.f);
+#pragma unroll
+          for (int q = 0; q < VEC; ++q) ws[kk * kSmCols + part * VEC + q] = f[q];
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // ---- product: warp w takes hidden dims [w ks/8, (w+1) ks/8); lane -> 8 tokens x 4 columns
+  const int tg = lane >> 3, cg = lane & 7;
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  const int kw = ks / 8;
+#pragma unroll 4
+  for (int kk = warp * kw; kk < (warp + 1) * kw; ++kk) {
+    const float4 x0 = *reinterpret_cast<const float4*>(&xs[kk * kSmTok + 8 * tg]);
+    const float4 x1 = *reinterpret_cast<const float4*>(&xs[kk * kSmTok + 8 * tg + 4]);
+    const float4 wv = *reinterpret_cast<const float4*>(&ws[kk * kSmCols + 4 * cg]);
+    const float xa[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w}, wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += xa[i] * wa[j];
+  }
+  __syncthreads();   // xs is reused for the warps' tiles
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    *reinterpret_cast<float4*>(&red[warp * kSmTok * kSmCols + (8 * tg + i) * kSmCols + 4 * cg]) =
+        make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+  __syncthreads();
+  append_small_finish<T, INT4>(sa, red, s_sq, s_pos, s_theta, &s_last, tok0, col0, tile, ntile, split);
+}
+
+// bf16 form of the decode-step append: the slice product runs on the tensor cores as
+// m16n8k16 warp MMAs from bf16 tiles staged with cp.async (x [32][ks], W [ks][32], rows
+// padded by 16 bytes so the ldmatrix reads are conflict-free); warp w takes hidden dims
+// [w ks/8, (w+1) ks/8) for the whole 32 x 32 tile.
+template <bool INT4>
+__global__ void __launch_bounds__(256) append_small_mma_kernel(AppendSmallArgs sa) {
+  MLA_KSPAN(2);
+  using bf16 = __nv_bfloat16;
+  const AppendArgs& a = sa.a;
+  extern __shared__ __align__(16) uint8_t sm8[];
+  const int ks = a.kslice;                       // multiple of 128
+  const int XLD = ks + 8;
+  constexpr int WLD = kSmCols + 8;
+  bf16* xs = reinterpret_cast<bf16*>(sm8);       // [kSmTok][XLD]
+  bf16* wsm = xs + kSmTok * XLD;                 // [ks][WLD]
+  float* red = reinterpret_cast<float*>(sm8);    // [8][kSmTok * kSmCols], after the product
+  __shared__ int s_sq[kSmTok], s_pos[kSmTok];
+  __shared__ double s_theta[kSmCols / 2];
+  __shared__ int s_last;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int col0 = blockIdx.x * kSmCols, tok0 = blockIdx.y * kSmTok;
+  const int split = blockIdx.z;
+  const int tile = blockIdx.y * gridDim.x + blockIdx.x, ntile = gridDim.x * gridDim.y;
+  const int k_begin = split * ks, k_end = min(a.d, k_begin + ks);
+  const bf16* x = (const bf16*)a.x;
+  const bf16* W = (const bf16*)a.W;
+  if (tid < kSmTok) {
+    const int n = tok0 + tid;
+    s_sq[tid] = n < a.N ? __ldg(a.seq_idx + n) : -1;
+    s_pos[tid] = n < a.N ? __ldg(a.pos + n) : -1;
+  } else if (tid < kSmTok + kSmCols / 2) {
+    const int cp = tid - kSmTok, col = col0 + 2 * cp;
+    double th = 0.0;
+    if (col >= a.d_c && col < a.ncols) {
+      const int rc = col - a.d_c, g = rc / (2 * a.r), j = (rc % (2 * a.r)) / 2;
+      th = __ldg(a.theta + __ldg(a.rope_pair + g * a.r + j));
+    }
+    s_theta[cp] = th;
+  }
+  // ---- stage: 16-byte asynchronous copies, all in flight together (missing rows and
+  // columns are zero-filled)
+  {
+    const int nxv = kSmTok * (ks / 8), nwv = ks * (kSmCols / 8);
+    for (int v = tid; v < nxv + nwv; v += 256) {
+      if (v < nxv) {
+        const int t = v / (ks / 8), ch = v % (ks / 8);
+        const int n = tok0 + t, kd = k_begin + ch * 8;
+        const bool ok = n < a.N && kd + 8 <= k_end;
+        sm100::cp_async16(wmma16::smem_addr(xs + t * XLD + ch * 8), ok ? (const void*)(x + (size_t)n * a.d + kd) : a.x,
+                          ok ? 16u : 0u);
+      } else {
+        const int vw = v - nxv;
+        const int kk = vw / (kSmCols / 8), part = vw % (kSmCols / 8);
+        const int kd = k_begin + kk, col = col0 + part * 8;
+        const bool ok = kd < k_end && col + 8 <= a.ncols;
+        sm100::cp_async16(wmma16::smem_addr(wsm + kk * WLD + part * 8),
+                          ok ? (const void*)(W + (size_t)kd * a.ncols + col) : a.W, ok ? 16u : 0u);
+      }
+    }
+    sm100::cp_async_commit();
+    sm100::cp_async_wait_all();
+  }
+  __syncthreads();
+  float acc[2][4][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+  const int kw = ks / 8;
+  for (int k0 = warp * kw; k0 < (warp + 1) * kw; k0 += 16) {
+    uint32_t a0[4], a1[4], b0[4], b1[4];
+    wmma16::load_a(a0, xs, XLD, 0, k0, lane);
+    wmma16::load_a(a1, xs, XLD, 16, k0, lane);
+    wmma16::load_b2(b0, wsm, WLD, k0, 0, lane);
+    wmma16::load_b2(b1, wsm, WLD, k0, 16, lane);
+    wmma16::mma_16816(acc[0][0], a0, b0[0], b0[1]);
+    wmma16::mma_16816(acc[0][1], a0, b0[2], b0[3]);
+    wmma16::mma_16816(acc[0][2], a0, b1[0], b1[1]);
+    wmma16::mma_16816(acc[0][3], a0, b1[2], b1[3]);
+    wmma16::mma_16816(acc[1][0], a1, b0[0], b0[1]);
+    wmma16::mma_16816(acc[1][1], a1, b0[2], b0[3]);
+    wmma16::mma_16816(acc[1][2], a1, b1[0], b1[1]);
+    wmma16::mma_16816(acc[1][3], a1, b1[2], b1[3]);
+  }
+  __syncthreads();   // the staging area is reused for the warps' tiles
+  float* my = red + warp * kSmTok * kSmCols;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int row = 16 * i + (lane >> 2), col = 8 * j + 2 * (lane & 3);
+      *reinterpret_cast<float2*>(my + row * kSmCols + col) = make_float2(acc[i][j][0], acc[i][j][1]);
+      *reinterpret_cast<float2*>(my + (row + 8) * kSmCols + col) = make_float2(acc[i][j][2], acc[i][j][3]);
+    }
+  __syncthreads();
+  append_small_finish<bf16, INT4>(sa, red, s_sq, s_pos, s_theta, &s_last, tok0, col0, tile, ntile, split);
+}
+
+template <bool INT4>
+cudaError_t launch_append_small_mma(const AppendSmallArgs& sa, cudaStream_t s, bool pdl) {
+  const AppendArgs& a = sa.a;
+  dim3 grid((a.ncols + kSmCols - 1) / kSmCols, (a.N + kSmTok - 1) / kSmTok, kAppSplit);
+  const size_t smem = std::max<size_t>(sizeof(__nv_bfloat16) * ((size_t)kSmTok * (a.kslice + 8) +
+                                                                (size_t)a.kslice * (kSmCols + 8)),
+                                       sizeof(float) * 8 * kSmTok * kSmCols);
+  cudaError_t e = cudaFuncSetAttribute(append_small_mma_kernel<INT4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&cfg, append_small_kernel<T, INT4>, args);
+  return mla_launch_kernel(append_small_mma_kernel<INT4>, grid, dim3(256), smem, s, pdl, sa);
+}
+
+template <typename T, bool INT4>
+cudaError_t launch_append_small_t(const AppendSmallArgs& sa, size_t smem, cudaStream_t s, bool pdl) {
+  const AppendArgs& a = sa.a;
+  dim3 grid((a.ncols + kSmCols - 1) / kSmCols, (a.N + kSmTok - 1) / kSmTok, kAppSplit);
+  cudaError_t e = cudaFuncSetAttribute(append_small_kernel<T, INT4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  return mla_launch_kernel(append_small_kernel<T, INT4>, grid, dim3(256), smem, s, pdl, sa);
 }
 
 }  // namespace mla
@@ -335,15 +549,32 @@ cudaError_t mla_launch_append(const mla_plan& p, const void* x, const int32_t* s
   const size_t eb = cfg.dtype == MLA_BF16 ? 2 : 4;
   a.vec_ok = ((uintptr_t)x % 16 == 0) && ((size_t)cfg.hidden * eb) % 16 == 0 && ((size_t)p.ncols * eb) % 16 == 0;
   const bool int4 = cfg.cache_kind == MLA_CACHE_INT4_G32;
-  if (N <= 4 * kSmTok) {
-    // decode-step size: split the hidden dim over an 8-CTA cluster, 32-column tiles
-    int ks = (cfg.hidden + kSmSplit - 1) / kSmSplit;
-    a.kslice = (ks + 31) / 32 * 32;
-    if (sizeof(float) * ((size_t)a.kslice * (kSmTok + kSmCols) + 4 * kSmTok * kSmCols) <= 200 * 1024) {
+  if (N <= kAppMaxSmallTokens && p.app_part && p.app_ticket && cfg.dtype == MLA_BF16 && a.vec_ok) {
+    int ks = (cfg.hidden + kAppSplit - 1) / kAppSplit;
+    a.kslice = (ks + 127) / 128 * 128;
+    if ((size_t)a.kslice * (kSmTok + kSmCols + 16) * 2 <= 200 * 1024) {
+      AppendSmallArgs sa;
+      sa.a = a;
+      sa.part = p.app_part;
+      sa.ticket = p.app_ticket;
+      return int4 ? launch_append_small_mma<true>(sa, s, p.opt_pdl) : launch_append_small_mma<false>(sa, s, p.opt_pdl);
+    }
+  }
+  if (N <= kAppMaxSmallTokens && p.app_part && p.app_ticket) {
+    // decode-step size: kAppSplit slices of the hidden dim, 32 x 32 tiles
+    int ks = (cfg.hidden + kAppSplit - 1) / kAppSplit;
+    a.kslice = (ks + 63) / 64 * 64;
+    // x and W slices, later reused for the eight warps' 32 x 32 tiles
+    const size_t smem = sizeof(float) * std::max<size_t>((size_t)a.kslice * (kSmTok + kSmCols), 8 * kSmTok * kSmCols);
+    if (smem <= 200 * 1024) {
+      AppendSmallArgs sa;
+      sa.a = a;
+      sa.part = p.app_part;
+      sa.ticket = p.app_ticket;
       if (cfg.dtype == MLA_BF16)
-        return int4 ? launch_append_small_t<__nv_bfloat16, true>(a, s)
-                    : launch_append_small_t<__nv_bfloat16, false>(a, s);
-      return launch_append_small_t<float, false>(a, s);
+        return int4 ? launch_append_small_t<__nv_bfloat16, true>(sa, smem, s, p.opt_pdl)
+                    : launch_append_small_t<__nv_bfloat16, false>(sa, smem, s, p.opt_pdl);
+      return launch_append_small_t<float, false>(sa, smem, s, p.opt_pdl);
     }
   }
   // Split the hidden dim over a cluster when there are too few (token, column) tiles

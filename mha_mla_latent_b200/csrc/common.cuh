@@ -58,6 +58,61 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f64<__nv_bfloat16>(dou
 // shared memory, so loads are not serialised behind shared-memory stores.
 template <typename T> __device__ __forceinline__ float ldg_f32(const T* p) { return to_f32(__ldg(p)); }
 
+// Stages a tile of `rows` x `cols` elements of T into shared memory as float
+// (dst[r * dst_ld + c]), row r starting at row_ptr(r).  Each thread issues a batch of up to
+// 8 loads before it uses any (16-byte vectors when `vec`: every row start 16-byte aligned
+// and cols a multiple of 16 / sizeof(T)), so a batch costs one memory round trip.
+template <typename T, typename RowPtr>
+__device__ __forceinline__ void stage_rows_f32(float* dst, int dst_ld, int rows, int cols, bool vec, RowPtr row_ptr) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  if (vec) {
+    constexpr int VEC = 16 / sizeof(T);
+    const int vpr = cols / VEC, nv = rows * vpr;
+    for (int base = 0; base < nv; base += 8 * nt) {
+      uint4 r[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int v = base + tid + k * nt;
+        if (v < nv) r[k] = __ldg(reinterpret_cast<const uint4*>(row_ptr(v / vpr) + (v % vpr) * VEC));
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int v = base + tid + k * nt;
+        if (v < nv) {
+          const T* e = reinterpret_cast<const T*>(&r[k]);
+          float* d = dst + (v / vpr) * dst_ld + (v % vpr) * VEC;
+#pragma unroll
+          for (int t = 0; t < VEC; ++t) d[t] = to_f32(e[t]);
+        }
+      }
+    }
+  } else {
+    const int n = rows * cols;
+    for (int base = 0; base < n; base += 8 * nt) {
+      float f[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = base + tid + k * nt;
+        f[k] = i < n ? to_f32(__ldg(row_ptr(i / cols) + i % cols)) : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = base + tid + k * nt;
+        if (i < n) dst[(i / cols) * dst_ld + i % cols] = f[k];
+      }
+    }
+  }
+}
+
+// Programmatic dependent launch.  pdl_wait() returns once the preceding kernel in the
+// stream has completed and its writes are visible (at once when the launch carries no
+// programmatic dependency); pdl_trigger() lets the next kernel start launching.  Every
+// kernel of the library waits before its first global write and before reading anything
+// an earlier kernel produced, and triggers only after that wait, so completion stays
+// ordered along the stream.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void raise_error(int32_t* err, int32_t bit) {
   if (err) atomicOr(err, bit);
 }

@@ -10,6 +10,10 @@
 #include <algorithm>
 
 #include "decode_common.cuh"
+#include "sm100.cuh"
+#include "warp_mma.cuh"
+
+#include <type_traits>
 
 MLA_KSPAN_DEFINE(decode)
 
@@ -19,170 +23,126 @@ namespace mla {
 struct AbsorbArgs {
   const void* q;              // [B][H][d_h]
   const int32_t* seq_lens;
-  int B, T_cap, H, n_kv, dh, r, d_c, dn, R;
+  int B, T_cap, H, n_kv, dh, r, d_c, dn;
   const void* W_ukT;          // [n_kv][dn][d_c]
   const int32_t* nope_idx;    // [n_kv][dn]
   const int32_t* rope_pair;   // [n_kv][r]
   const double* theta;
-  float* qlat;                // f32 [B][H][d_c]        (CUDA-core kernel)
+  float* qlat;                // f32 [B][H][d_c]        (CUDA-core kernel), or null
+  __nv_bfloat16* qlat16;      // bf16 [B][H][d_c]       (tcgen05 kernel), or null
   float* qrope;               // f32 [B][H][2r]
-  __nv_bfloat16* qcat;        // bf16 [B][H][K]         (tcgen05 kernel), or null
-  int K;
-  int bchunk;                 // sequences per CTA
   Sched sched;
   int tile, G;
   int32_t* err;
-  int smem_ints;              // dynamic shared memory of the CTA, in ints
-  int vec_ok;                 // W_uk rows and q rows allow 16-byte loads
+  int sched_ints;             // shared memory of the schedule CTA, in ints
+  int vec_ok;                 // q and W_uk^T rows allow 16-byte loads
 };
 
-constexpr int kAbsRows = 16;   // (b, h) rows per CTA
-constexpr int kAbsCols = 64;   // latent columns per CTA
+constexpr int kAbsRows = 8;    // (b, h) rows per CTA: one per warp in the product
+constexpr int kAbsCols = 64;   // latent columns per CTA: two per lane
 
-// grid: n_kv * (column chunks) * (row chunks) CTAs, plus one CTA that builds the schedule.
-// Each CTA stages its slice of W_uk[g] (all NoPE dims x 64 latent columns) and the NoPE
-// query dims of its rows in shared memory, then each thread accumulates 4 rows of one
-// latent column.
+// grid: n_kv * (row blocks) * (column chunks) CTAs, plus one CTA that builds the split-K
+// schedule.  A CTA reads everything it needs (its W_uk^T slice, its query rows, the NoPE
+// index table, and for the first column chunk the RoPE tables and positions) in one batch
+// of loads, then q_lat[row][c] = scale * sum_j q[row][nope_j] * W_uk^T[g][j][c] with warp r
+// owning row r and lane l columns 2l, 2l+1 of the chunk.
 template <typename T>
 __global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
   MLA_KSPAN(0);
+  extern __shared__ __align__(16) float sm[];
   const int G = a.H / a.n_kv;
   const int rows_total = a.B * G;
-  const int n_rc = (rows_total + kAbsRows - 1) / kAbsRows;
+  const int n_rb = (rows_total + kAbsRows - 1) / kAbsRows;
   const int n_cc = (a.d_c + kAbsCols - 1) / kAbsCols;
-  if (blockIdx.x == a.n_kv * n_cc * n_rc) {  // the last CTA builds the split-K schedule
-    extern __shared__ float sm_sched[];
-    build_schedule(a.seq_lens, a.B, a.T_cap, a.tile, a.G, a.sched, a.err, reinterpret_cast<int32_t*>(sm_sched),
-                   a.smem_ints);
+  if (blockIdx.x == a.n_kv * n_rb * n_cc) {  // the last CTA builds the split-K schedule
+    pdl_wait();
+    pdl_trigger();
+    build_schedule(a.seq_lens, a.B, a.T_cap, a.tile, a.G, a.sched, a.err, reinterpret_cast<int32_t*>(sm),
+                   a.sched_ints);
     return;
   }
   const int g = blockIdx.x % a.n_kv;
-  const int cc = (blockIdx.x / a.n_kv) % n_cc;
-  const int rc = blockIdx.x / (a.n_kv * n_cc);
-  const int row0 = rc * kAbsRows;
-  const int rows = min(kAbsRows, rows_total - row0);
-  extern __shared__ float sm[];
-  float* s_w = sm;                          // [dn][kAbsCols]
-  float* s_q = s_w + a.dn * kAbsCols;       // [kAbsRows][dn]
-  const float scale = kLog2e * rsqrtf((float)a.dh);
+  const int rb = (blockIdx.x / a.n_kv) % n_rb;
+  const int cc = blockIdx.x / (a.n_kv * n_rb);
+  const int row0 = rb * kAbsRows, c0 = cc * kAbsCols;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int dn = a.dn, dh = a.dh, dnp = (dn + 3) & ~3;
+  float* s_w = sm;                              // [dn][kAbsCols]
+  float* s_q = s_w + dn * kAbsCols;             // [kAbsRows][dh] raw query rows
+  float* s_qn = s_q + kAbsRows * dh;            // [kAbsRows][dnp] NoPE dims, gathered
+  int* s_idx = reinterpret_cast<int*>(s_qn + kAbsRows * dnp);   // [dn]
   const T* q = (const T*)a.q;
-  const T* W = (const T*)a.W_ukT + (size_t)g * a.dn * a.d_c;
-  const int c0 = cc * kAbsCols;
-  float* s_qraw = s_q + kAbsRows * a.dn;    // [kAbsRows][dh]
-  // all loads of the CTA are issued before any is used (one memory round trip)
-  constexpr int VEC = 16 / sizeof(T);
-  const bool vec = a.vec_ok && (c0 + kAbsCols <= a.d_c);
-  if (vec) {
-    constexpr int kMaxW = 8;                 // dn <= 256: dn * 64 / VEC / 256 <= 8 (bf16)
-    const int nw = a.dn * (kAbsCols / VEC);
-    uint4 wr[kMaxW];
-#pragma unroll
-    for (int k = 0; k < kMaxW; ++k) {
-      const int v = threadIdx.x + 256 * k;
-      if (v < nw) {
-        const int j = v / (kAbsCols / VEC), part = v % (kAbsCols / VEC);
-        wr[k] = __ldg(reinterpret_cast<const uint4*>(W + (size_t)j * a.d_c + c0 + part * VEC));
-      }
-    }
-    const int nq = rows * (a.dh / VEC);
-    uint4 qr[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int v = threadIdx.x + 256 * k;
-      if (v < nq) {
-        const int r = v / (a.dh / VEC), part = v % (a.dh / VEC);
-        const int row = row0 + r, b = row / G, h = g * G + row % G;
-        qr[k] = __ldg(reinterpret_cast<const uint4*>(q + ((size_t)b * a.H + h) * a.dh + part * VEC));
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < kMaxW; ++k) {
-      const int v = threadIdx.x + 256 * k;
-      if (v < nw) {
-        const int j = v / (kAbsCols / VEC), part = v % (kAbsCols / VEC);
-        const T* e = reinterpret_cast<const T*>(&wr[k]);
-#pragma unroll
-        for (int t = 0; t < VEC; ++t) s_w[j * kAbsCols + part * VEC + t] = to_f32(e[t]);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int v = threadIdx.x + 256 * k;
-      if (v < nq) {
-        const int r = v / (a.dh / VEC), part = v % (a.dh / VEC);
-        const T* e = reinterpret_cast<const T*>(&qr[k]);
-#pragma unroll
-        for (int t = 0; t < VEC; ++t) s_qraw[r * a.dh + part * VEC + t] = to_f32(e[t]);
-      }
-    }
-  } else {
-    for (int i = threadIdx.x; i < a.dn * kAbsCols; i += blockDim.x) {
-      const int j = i / kAbsCols, cl = i % kAbsCols;
-      s_w[i] = (c0 + cl < a.d_c) ? ldg_f32(W + (size_t)j * a.d_c + c0 + cl) : 0.f;
-    }
-    for (int i = threadIdx.x; i < rows * a.dh; i += blockDim.x) {
-      const int r = i / a.dh, e = i % a.dh;
-      const int row = row0 + r, b = row / G, h = g * G + row % G;
-      s_qraw[i] = ldg_f32(q + ((size_t)b * a.H + h) * a.dh + e);
-    }
+  const T* W = (const T*)a.W_ukT + (size_t)g * dn * a.d_c;
+  // ---- loads: W slice, query rows, NoPE indices (inputs and plan tables only)
+  const int ncol = min(kAbsCols, a.d_c - c0);
+  if (ncol < kAbsCols)
+    for (int i = tid; i < dn * kAbsCols; i += 256) s_w[i] = 0.f;   // columns past d_c
+  stage_rows_f32<T>(s_w, kAbsCols, dn, ncol, a.vec_ok && ncol == kAbsCols,
+                    [&](int j) { return W + (size_t)j * a.d_c + c0; });
+  const int nrow = min(kAbsRows, rows_total - row0);
+  stage_rows_f32<T>(s_q, dh, nrow, dh, a.vec_ok, [&](int r) {
+    const int row = row0 + r;
+    return q + ((size_t)(row / G) * a.H + g * G + row % G) * dh;
+  });
+  for (int j = tid; j < dn; j += 256) s_idx[j] = __ldg(a.nope_idx + g * dn + j);
+  // RoPE query part (first column chunk): rotate the kept pairs at position L-1 (angle in
+  // double), scale.  Positions and frequencies are loaded in the same batch.
+  const float scale = kLog2e * rsqrtf((float)dh);
+  const int nrope = (cc == 0) ? kAbsRows * a.r : 0;
+  int rp_pos = 0, rp_k = 0;
+  double rp_th = 0.0;
+  const bool rope_item = tid < nrope && row0 + tid / max(a.r, 1) < rows_total;
+  if (rope_item) {
+    const int r = tid / a.r, row = row0 + r;
+    rp_k = __ldg(a.rope_pair + g * a.r + tid % a.r);
+    rp_th = __ldg(a.theta + rp_k);
+    rp_pos = __ldg(a.seq_lens + row / G);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < rows * a.dn; i += blockDim.x) {
-    const int r = i / a.dn, j = i % a.dn;
-    s_q[i] = s_qraw[r * a.dh + __ldg(a.nope_idx + g * a.dn + j)];
-  }
-  if (cc == 0) {
-    // RoPE part: rotate the kept pairs at position L-1 (angle in double), scale.
-    for (int i = threadIdx.x; i < rows * a.r; i += blockDim.x) {
-      const int r = i / a.r, j = i % a.r;
-      const int row = row0 + r, b = row / G, h = g * G + row % G;
-      const int L = a.seq_lens[b];
-      const int p = (L >= 1 && L <= a.T_cap) ? L - 1 : 0;
-      const int k = a.rope_pair[g * a.r + j];
-      const double x0 = s_qraw[r * a.dh + 2 * k], x1 = s_qraw[r * a.dh + 2 * k + 1];
-      double sn, cs;
-      sincos((double)p * a.theta[k], &sn, &cs);
-      const float o0 = (float)((x0 * cs - x1 * sn) * (double)scale);
-      const float o1 = (float)((x0 * sn + x1 * cs) * (double)scale);
-      const size_t bh = (size_t)b * a.H + h;
-      if (a.qrope) { a.qrope[bh * 2 * a.r + 2 * j] = o0; a.qrope[bh * 2 * a.r + 2 * j + 1] = o1; }
-      if (a.qcat && a.K > a.d_c) {
-        a.qcat[bh * a.K + a.d_c + g * 2 * a.r + 2 * j] = __float2bfloat16_rn(o0);
-        a.qcat[bh * a.K + a.d_c + g * 2 * a.r + 2 * j + 1] = __float2bfloat16_rn(o1);
-      }
-    }
-    if (a.qcat && a.K > a.d_c) {  // zero the other KV heads' RoPE slots of a concatenated row
-      for (int i = threadIdx.x; i < rows * a.R; i += blockDim.x) {
-        const int r = i / a.R, j = i % a.R;
-        if (j / (2 * a.r) == g) continue;
-        const int row = row0 + r;
-        const size_t bh = (size_t)(row / G) * a.H + g * G + row % G;
-        a.qcat[bh * a.K + a.d_c + j] = __float2bfloat16_rn(0.f);
-      }
-    }
+  for (int i = tid; i < kAbsRows * dn; i += 256) s_qn[(i / dn) * dnp + i % dn] = s_q[(i / dn) * dh + s_idx[i % dn]];
+  // outputs are read by the attention kernel of the previous call until it has finished
+  pdl_wait();
+  pdl_trigger();
+  if (rope_item) {
+    const int r = tid / a.r, j = tid % a.r, row = row0 + r;
+    const int b = row / G, h = g * G + row % G;
+    const int p = (rp_pos >= 1 && rp_pos <= a.T_cap) ? rp_pos - 1 : 0;
+    const double x0 = s_q[r * dh + 2 * rp_k], x1 = s_q[r * dh + 2 * rp_k + 1];
+    double sn, cs;
+    sincos((double)p * rp_th, &sn, &cs);
+    const size_t o = ((size_t)b * a.H + h) * 2 * a.r + 2 * j;
+    a.qrope[o] = (float)((x0 * cs - x1 * sn) * (double)scale);
+    a.qrope[o + 1] = (float)((x0 * sn + x1 * cs) * (double)scale);
   }
   __syncthreads();
-  // q_lat[row][c] = scale * sum_j q_nope[row][j] * W_uk[g][c][j]
-  const int cl = threadIdx.x % kAbsCols, rg = threadIdx.x / kAbsCols;  // 4 row groups
-  const int c = c0 + cl;
-  float acc[kAbsRows / 4];
-#pragma unroll
-  for (int k = 0; k < kAbsRows / 4; ++k) acc[k] = 0.f;
-#pragma unroll 4
-  for (int j = 0; j < a.dn; ++j) {
-    const float wv = s_w[j * kAbsCols + cl];
-#pragma unroll
-    for (int k = 0; k < kAbsRows / 4; ++k) acc[k] += s_q[(rg * (kAbsRows / 4) + k) * a.dn + j] * wv;
+  // ---- product: warp r -> row r, lane l -> columns 2l, 2l+1 of the chunk
+  const int r = warp, row = row0 + r, c = c0 + 2 * lane;
+  const float* qn = s_qn + r * dnp;
+  float acc0 = 0.f, acc1 = 0.f;
+  int j = 0;
+  for (; j + 4 <= dn; j += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(qn + j);
+    const float2 w0 = *reinterpret_cast<const float2*>(s_w + (j + 0) * kAbsCols + 2 * lane);
+    const float2 w1 = *reinterpret_cast<const float2*>(s_w + (j + 1) * kAbsCols + 2 * lane);
+    const float2 w2 = *reinterpret_cast<const float2*>(s_w + (j + 2) * kAbsCols + 2 * lane);
+    const float2 w3 = *reinterpret_cast<const float2*>(s_w + (j + 3) * kAbsCols + 2 * lane);
+    acc0 += x.x * w0.x + x.y * w1.x + x.z * w2.x + x.w * w3.x;
+    acc1 += x.x * w0.y + x.y * w1.y + x.z * w2.y + x.w * w3.y;
   }
-  if (c < a.d_c) {
-#pragma unroll
-    for (int k = 0; k < kAbsRows / 4; ++k) {
-      const int r = rg * (kAbsRows / 4) + k;
-      if (r >= rows) break;
-      const int row = row0 + r;
-      const size_t bh = (size_t)(row / G) * a.H + g * G + row % G;
-      if (a.qlat) a.qlat[bh * a.d_c + c] = acc[k] * scale;
-      if (a.qcat) a.qcat[bh * a.K + c] = __float2bfloat16_rn(acc[k] * scale);
+  for (; j < dn; ++j) {
+    const float2 w = *reinterpret_cast<const float2*>(s_w + j * kAbsCols + 2 * lane);
+    acc0 += qn[j] * w.x;
+    acc1 += qn[j] * w.y;
+  }
+  if (row < rows_total && c < a.d_c) {
+    const size_t o = ((size_t)(row / G) * a.H + g * G + row % G) * a.d_c + c;
+    if (a.qlat) {
+      a.qlat[o] = acc0 * scale;
+      if (c + 1 < a.d_c) a.qlat[o + 1] = acc1 * scale;
+    }
+    if (a.qlat16) {
+      a.qlat16[o] = __float2bfloat16_rn(acc0 * scale);
+      if (c + 1 < a.d_c) a.qlat16[o + 1] = __float2bfloat16_rn(acc1 * scale);
     }
   }
 }
@@ -219,6 +179,8 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(DecodeArgs a) {
   const int tid = threadIdx.x;
   const int nE = (H * dc + 255) / 256;
   const int w = blockIdx.x;
+  pdl_wait();   // schedule and absorbed queries
+  pdl_trigger();
   for (int pc = a.sched.worker_first[w]; pc < a.sched.worker_first[w + 1]; ++pc) {
     const int b = a.sched.piece_b[pc];
     const int t0 = a.sched.piece_t0[pc], t1 = a.sched.piece_t1[pc];
@@ -311,119 +273,170 @@ struct CombineArgs {
   Sched sched;
   const void* W_uv;   // [n_kv][d_c][dh]
   void* out;          // [B][H][dh]
-  int bchunk;
-  int max_pieces;     // upper bound on pieces per sequence (G + 1)
   int P;              // piece capacity of the partial arrays [H][P]
+  int ncols;          // output columns per CTA: 64, or 32 when the latent is wide
+  int vec_ok;         // W_uv rows allow 16-byte loads
 };
 
+constexpr int kCmbRows = 8;    // (b, h) rows per CTA, one warp each
+
+// grid: n_kv * (row blocks) * (output column chunks).  Before the dependency wait the CTA
+// stages its W_uv[g] column chunk; after it, warp r merges the pieces of row r,
+//     O_lat = sum_j 2^(m_j - M) O_j / sum_j 2^(m_j - M) l_j,
+// into shared memory (all of a batch of pieces' loads in flight together), and then
+// out[row][d] = sum_c O_lat[row][c] W_uv[g][c][d] with lane l on columns 2l, 2l+1.
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   MLA_KSPAN(2);
-  const int g = blockIdx.x % a.n_kv, chunk = blockIdx.x / a.n_kv;
+  extern __shared__ __align__(16) float sm[];
   const int G = a.H / a.n_kv;
-  const int b0 = chunk * a.bchunk;
-  const int nb = min(a.bchunk, a.B - b0);
-  const int rows = nb * G;
-  extern __shared__ float sm[];
-  float* s_o = sm;                      // [rows][d_c] merged latent
-  float* s_wt = s_o + rows * a.d_c;     // [rows][max_pieces] merge weights
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
-  // 1. per (b, h): merge weights 2^(m_j - M) / sum_j 2^(m_j - M) l_j of its pieces
-  //    (one warp per row; lanes stride over the pieces)
-  for (int row = warp; row < rows; row += nwarp) {
-    const int b = b0 + row / G, h = g * G + row % G;
-    const int first = a.sched.seq_first[b], np = a.sched.seq_np[b];
-    float M = -INFINITY;
-    for (int j = lane; j < np; j += 32) M = fmaxf(M, __ldg(a.mlpart + ((size_t)h * a.P + first + j) * 2));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float den = 0.f;
-    for (int j = lane; j < np; j += 32) {
-      const float* ml = a.mlpart + ((size_t)h * a.P + first + j) * 2;
-      const float wj = exp2f(__ldg(ml) - M);
-      s_wt[row * a.max_pieces + j] = wj;
-      den += wj * __ldg(ml + 1);
+  const int rows_total = a.B * G;
+  const int n_rb = (rows_total + kCmbRows - 1) / kCmbRows;
+  const int g = blockIdx.x % a.n_kv;
+  const int rb = (blockIdx.x / a.n_kv) % n_rb;
+  const int dcb = blockIdx.x / (a.n_kv * n_rb);
+  const int NCOL = a.ncols;
+  const int row0 = rb * kCmbRows, d0 = dcb * NCOL;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int dc = a.d_c;
+  // bf16 with whole 16-byte rows: the output product runs as warp MMAs on bf16 tiles
+  const bool mma = std::is_same<T, __nv_bfloat16>::value && a.vec_ok && NCOL == 64 && d0 + 64 <= a.dh;
+  constexpr int WLD = 64 + 8;            // bf16 W tile row stride (conflict-free ldmatrix)
+  const int ALD = dc + 8;                // bf16 A tile row stride
+  float* s_w = sm;                       // f32 [d_c][NCOL], or bf16 [d_c][WLD] for the MMA form
+  float* s_o = s_w + dc * NCOL;          // [kCmbRows][d_c]
+  __nv_bfloat16* s_a = reinterpret_cast<__nv_bfloat16*>(s_o + kCmbRows * dc);   // [16][ALD]
+  const T* W = (const T*)a.W_uv + (size_t)g * dc * a.dh;
+  const int ncol = min(NCOL, a.dh - d0);
+  if (mma) {
+    __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(s_w);
+    for (int v = tid; v < dc * 8; v += 256) {
+      const int c = v >> 3, part = v & 7;
+      sm100::cp_async16(wmma16::smem_addr(wt + c * WLD + part * 8), W + (size_t)c * a.dh + d0 + part * 8, 16u);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    const float inv = (np > 0 && den > 0.f) ? 1.f / den : 0.f;
-    __syncwarp();
-    for (int j = lane; j < np; j += 32) s_wt[row * a.max_pieces + j] *= inv;
+    sm100::cp_async_commit();
+  } else {
+    if (ncol < NCOL)
+      for (int i = tid; i < dc * NCOL; i += 256) s_w[i] = 0.f;   // columns past d_h
+    stage_rows_f32<T>(s_w, NCOL, dc, ncol, a.vec_ok && ncol == NCOL, [&](int c) { return W + (size_t)c * a.dh + d0; });
   }
-  __syncthreads();
-  // 2. merged latent: each item is (row, 4 consecutive c); all pieces' loads issued together
-  const int c4n = a.d_c / 4;
-  for (int it = threadIdx.x; it < rows * c4n; it += blockDim.x) {
-    const int row = it / c4n, c4 = it % c4n;
-    const int b = b0 + row / G, h = g * G + row % G;
-    const int first = a.sched.seq_first[b], np = a.sched.seq_np[b];
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < np; j0 += 8) {
-      float4 o[8];
+  pdl_wait();   // the partials of the attention kernel
+  pdl_trigger();
+  {
+    const int r = warp, row = row0 + r;
+    float* o = s_o + r * dc;
+    if (row < rows_total) {
+      const int b = row / G, h = g * G + row % G;
+      const int first = __ldg(a.sched.seq_first + b), np = __ldg(a.sched.seq_np + b);
+      const float* ml = a.mlpart + ((size_t)h * a.P + first) * 2;
+      const float* op = a.opart + ((size_t)h * a.P + first) * dc;
+      // pieces j = lane (+32k): running max and sum; the first 8 pieces' latent rows are
+      // loaded in the same round trip (they do not depend on the weights)
+      const int nc4 = dc / 4;
+      float4 v0[8], v1[8];   // columns lane and lane + 32 (float4 units) of pieces 0..7
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        if (j0 + k < np)
-          o[k] = __ldg(reinterpret_cast<const float4*>(a.opart + ((size_t)h * a.P + first + j0 + k) * a.d_c) + c4);
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        if (j0 + k < np) {
-          const float wgt = s_wt[row * a.max_pieces + j0 + k];
-          acc.x += wgt * o[k].x; acc.y += wgt * o[k].y; acc.z += wgt * o[k].z; acc.w += wgt * o[k].w;
+      for (int k = 0; k < 8; ++k) {
+        if (k < np) {
+          if (lane < nc4) v0[k] = __ldg(reinterpret_cast<const float4*>(op + (size_t)k * dc) + lane);
+          if (lane + 32 < nc4) v1[k] = __ldg(reinterpret_cast<const float4*>(op + (size_t)k * dc) + lane + 32);
         }
+      }
+      float mj = -INFINITY, lj = 0.f;
+      if (lane < np) { mj = __ldg(ml + 2 * lane); lj = __ldg(ml + 2 * lane + 1); }
+      float M = mj;
+      for (int j = lane + 32; j < np; j += 32) M = fmaxf(M, __ldg(ml + 2 * j));
+#pragma unroll
+      for (int s = 16; s > 0; s >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, s));
+      const float wl = lane < np ? exp2f(mj - M) : 0.f;   // weight of piece `lane`
+      float den = wl * lj;
+      for (int j = lane + 32; j < np; j += 32) den += exp2f(__ldg(ml + 2 * j) - M) * __ldg(ml + 2 * j + 1);
+#pragma unroll
+      for (int s = 16; s > 0; s >>= 1) den += __shfl_xor_sync(0xffffffffu, den, s);
+      const float inv = (np > 0 && den > 0.f) ? 1.f / den : 0.f;
+      float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k < np) {
+          const float w = __shfl_sync(0xffffffffu, wl, k);
+          a0.x += w * v0[k].x; a0.y += w * v0[k].y; a0.z += w * v0[k].z; a0.w += w * v0[k].w;
+          a1.x += w * v1[k].x; a1.y += w * v1[k].y; a1.z += w * v1[k].z; a1.w += w * v1[k].w;
+        }
+      }
+      for (int j = 8; j < np; ++j) {   // more than 8 pieces: one at a time
+        const float w = j < 32 ? __shfl_sync(0xffffffffu, wl, j) : exp2f(__ldg(ml + 2 * j) - M);
+        if (lane < nc4) {
+          const float4 x = __ldg(reinterpret_cast<const float4*>(op + (size_t)j * dc) + lane);
+          a0.x += w * x.x; a0.y += w * x.y; a0.z += w * x.z; a0.w += w * x.w;
+        }
+        if (lane + 32 < nc4) {
+          const float4 x = __ldg(reinterpret_cast<const float4*>(op + (size_t)j * dc) + lane + 32);
+          a1.x += w * x.x; a1.y += w * x.y; a1.z += w * x.z; a1.w += w * x.w;
+        }
+      }
+      if (lane < nc4) *reinterpret_cast<float4*>(o + 4 * lane) = make_float4(a0.x * inv, a0.y * inv, a0.z * inv, a0.w * inv);
+      if (lane + 32 < nc4)
+        *reinterpret_cast<float4*>(o + 4 * lane + 128) = make_float4(a1.x * inv, a1.y * inv, a1.z * inv, a1.w * inv);
+      for (int c4 = lane + 64; c4 < nc4; c4 += 32) {   // latents wider than 256
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < np; ++j) {
+          const float w = j < 32 ? __shfl_sync(0xffffffffu, wl, j) : exp2f(__ldg(ml + 2 * j) - M);
+          const float4 x = __ldg(reinterpret_cast<const float4*>(op + (size_t)j * dc) + c4);
+          acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
+        }
+        *reinterpret_cast<float4*>(o + 4 * c4) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      }
+    } else {
+      for (int c = lane; c < dc; c += 32) o[c] = 0.f;
     }
-    *reinterpret_cast<float4*>(&s_o[row * a.d_c + c4 * 4]) = acc;
+  }
+  if (mma) {
+    // A = merged rows as bf16 (rows 8..15 zero), B = W_uv chunk; warps 0-3 take 16 columns each
+    __syncthreads();   // every warp's merged row is in s_o
+    for (int i = tid; i < 16 * dc; i += 256) {
+      const int r = i / dc, c = i % dc;
+      s_a[r * ALD + c] = __float2bfloat16_rn(r < kCmbRows ? s_o[r * dc + c] : 0.f);
+    }
+    sm100::cp_async_wait_all();
+    __syncthreads();
+    if (warp >= 4) return;
+    const __nv_bfloat16* wt = reinterpret_cast<const __nv_bfloat16*>(s_w);
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int k0 = 0; k0 < dc; k0 += 16) {
+      uint32_t af[4], bf[4];
+      wmma16::load_a(af, s_a, ALD, 0, k0, lane);
+      wmma16::load_b2(bf, wt, WLD, k0, 16 * warp, lane);
+      wmma16::mma_16816(acc[0], af, bf[0], bf[1]);
+      wmma16::mma_16816(acc[1], af, bf[2], bf[3]);
+    }
+    const int r = lane >> 2, row = row0 + r;
+    if (row < rows_total) {
+      T* out = (T*)a.out + ((size_t)(row / G) * a.H + g * G + row % G) * a.dh + d0 + 16 * warp + 2 * (lane & 3);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(acc[j][0], acc[j][1]);
+        *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(out) + 8 * j) = v;
+      }
+    }
+    return;
   }
   __syncthreads();
-  // 3. o[row][d] = sum_c O_lat[row][c] W_uv[g][c][d], W_uv[g] staged in chunks of 64 latent
-  //    rows (one 16-byte load per thread and chunk row group, all issued before use)
-  const T* W = (const T*)a.W_uv + (size_t)g * a.d_c * a.dh;
-  float* s_w = s_wt + rows * a.max_pieces;   // [kWc][dh]
-  constexpr int kRows = 8, kWc = 64;
-  constexpr int VEC = 16 / sizeof(T);
-  const int n_items = a.dh * ((rows + kRows - 1) / kRows);
-  const int item = threadIdx.x;
-  const int d = item % a.dh, r0 = (item / a.dh) * kRows;
-  float acc[kRows];
-#pragma unroll
-  for (int k = 0; k < kRows; ++k) acc[k] = 0.f;
-  for (int cb = 0; cb < a.d_c; cb += kWc) {
-    const int nc = min(kWc, a.d_c - cb);
-    const int nvec = nc * a.dh / VEC;
-    uint4 wr[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int v = threadIdx.x + 256 * k;
-      if (v < nvec) wr[k] = __ldg(reinterpret_cast<const uint4*>(W + (size_t)cb * a.dh) + v);
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int v = threadIdx.x + 256 * k;
-      if (v < nvec) {
-        const T* e = reinterpret_cast<const T*>(&wr[k]);
-#pragma unroll
-        for (int t = 0; t < VEC; ++t) s_w[v * VEC + t] = to_f32(e[t]);
-      }
-    }
-    __syncthreads();
-    if (item < n_items) {
-#pragma unroll 4
-      for (int c = 0; c < nc; ++c) {
-        const float wv = s_w[c * a.dh + d];
-#pragma unroll
-        for (int k = 0; k < kRows; ++k)
-          if (r0 + k < rows) acc[k] += s_o[(r0 + k) * a.d_c + cb + c] * wv;
-      }
-    }
-    __syncthreads();
+  const int r = warp, row = row0 + r, d = d0 + 2 * lane;
+  if (2 * lane >= NCOL) return;
+  const float* o = s_o + r * dc;
+  float acc0 = 0.f, acc1 = 0.f;
+  for (int c = 0; c < dc; c += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(o + c);
+    const float2 w0 = *reinterpret_cast<const float2*>(s_w + (c + 0) * NCOL + 2 * lane);
+    const float2 w1 = *reinterpret_cast<const float2*>(s_w + (c + 1) * NCOL + 2 * lane);
+    const float2 w2 = *reinterpret_cast<const float2*>(s_w + (c + 2) * NCOL + 2 * lane);
+    const float2 w3 = *reinterpret_cast<const float2*>(s_w + (c + 3) * NCOL + 2 * lane);
+    acc0 += x.x * w0.x + x.y * w1.x + x.z * w2.x + x.w * w3.x;
+    acc1 += x.x * w0.y + x.y * w1.y + x.z * w2.y + x.w * w3.y;
   }
-  if (item < n_items) {
-#pragma unroll
-    for (int k = 0; k < kRows; ++k) {
-      const int row = r0 + k;
-      if (row >= rows) break;
-      const int b = b0 + row / G, h = g * G + row % G;
-      ((T*)a.out)[((size_t)b * a.H + h) * a.dh + d] = from_f32<T>(acc[k]);
-    }
+  if (row < rows_total && d < a.dh) {
+    T* out = (T*)a.out + ((size_t)(row / G) * a.H + g * G + row % G) * a.dh + d;
+    out[0] = from_f32<T>(acc0);
+    if (d + 1 < a.dh) out[1] = from_f32<T>(acc1);
   }
 }
 
@@ -439,27 +452,28 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
   AbsorbArgs aa;
   aa.q = q; aa.seq_lens = seq_lens; aa.B = B; aa.T_cap = c.T_cap; aa.H = H;
   aa.n_kv = cfg.n_kv_heads; aa.dh = cfg.head_dim; aa.r = cfg.r_pairs; aa.d_c = cfg.d_c;
-  aa.dn = p.dn; aa.R = p.R; aa.W_ukT = p.W_ukT; aa.nope_idx = p.nope_idx;
+  aa.dn = p.dn; aa.W_ukT = p.W_ukT; aa.nope_idx = p.nope_idx;
   aa.rope_pair = p.rope_pair; aa.theta = p.theta;
   aa.qlat = L.kernel == 1 ? (float*)(base + L.off_qlat) : nullptr;
+  aa.qlat16 = L.kernel == 2 ? (__nv_bfloat16*)(base + L.off_qlat) : nullptr;
   aa.qrope = (float*)(base + L.off_qrope);
-  aa.qcat = L.kernel == 2 ? (__nv_bfloat16*)(base + L.off_qlat) : nullptr;
-  aa.K = cfg.d_c;
-  aa.bchunk = 0;
   aa.sched = sched; aa.tile = L.tile; aa.G = L.G; aa.err = p.err;
-  const int n_rc = (B * G + kAbsRows - 1) / kAbsRows, n_cc = (cfg.d_c + kAbsCols - 1) / kAbsCols;
-  const size_t smem_abs = std::max((size_t)(p.dn * kAbsCols + kAbsRows * p.dn + kAbsRows * cfg.head_dim) * sizeof(float),
-                                    (size_t)(4 * B + 1) * sizeof(int32_t));
   {
-    const int vecn = 16 / (int)sizeof(T);  // elements per 16-byte load
-    aa.vec_ok = ((uintptr_t)q % 16 == 0) && cfg.d_c % vecn == 0 && cfg.head_dim % vecn == 0 &&
-                p.dn * (kAbsCols / vecn) <= 256 * 8 && kAbsRows * (cfg.head_dim / vecn) <= 256 * 2;
+    const int vecn = 16 / (int)sizeof(T);   // elements per 16-byte load
+    aa.vec_ok = ((uintptr_t)q % 16 == 0) && cfg.d_c % vecn == 0 && cfg.head_dim % vecn == 0;
   }
-  aa.smem_ints = (int)(smem_abs / sizeof(int32_t));
+  const int n_rb = (B * G + kAbsRows - 1) / kAbsRows, n_cc = (cfg.d_c + kAbsCols - 1) / kAbsCols;
+  const int dnp = (p.dn + 3) & ~3;
+  const size_t smem_work = sizeof(float) * ((size_t)p.dn * kAbsCols + (size_t)kAbsRows * cfg.head_dim +
+                                            (size_t)kAbsRows * dnp + p.dn);
+  const size_t sched_ints = (size_t)9 * B + 4 * L.G + 2;
+  const size_t smem_abs = std::min<size_t>(std::max(smem_work, sched_ints * sizeof(int32_t)),
+                                           std::max<size_t>(smem_work, 160 * 1024));
+  aa.sched_ints = (int)(smem_abs / sizeof(int32_t));
   cudaError_t e = cudaFuncSetAttribute(absorb_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_abs);
   if (e != cudaSuccess) return e;
-  absorb_kernel<T><<<cfg.n_kv_heads * n_cc * n_rc + 1, 256, smem_abs, s>>>(aa);
-  e = cudaGetLastError();
+  e = mla_launch_kernel(absorb_kernel<T>, dim3(cfg.n_kv_heads * n_rb * n_cc + 1), dim3(256), smem_abs, s, p.opt_pdl,
+                        aa);
   if (e != cudaSuccess) return e;
   // 2. split-K attention over the latent cache
   if (L.kernel == 1) {
@@ -476,8 +490,7 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
                              (int)smem);
     if (e != cudaSuccess) return e;
     if ((e = mla_profile_event(p, 0, s)) != cudaSuccess) return e;
-    decode_simt_kernel<T, INT4><<<L.G, 256, smem, s>>>(da);
-    e = cudaGetLastError();
+    e = mla_launch_kernel(decode_simt_kernel<T, INT4>, dim3(L.G), dim3(256), smem, s, p.opt_pdl, da);
     if (e != cudaSuccess) return e;
     if ((e = mla_profile_event(p, 1, s)) != cudaSuccess) return e;
   } else {
@@ -490,17 +503,15 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
   ca.B = B; ca.H = H; ca.n_kv = cfg.n_kv_heads; ca.d_c = cfg.d_c; ca.dh = cfg.head_dim;
   ca.opart = (const float*)(base + L.off_opart); ca.mlpart = (const float*)(base + L.off_mlpart);
   ca.sched = sched; ca.W_uv = p.W_uv; ca.out = out; ca.P = L.P;
-  // rows (b, h) per CTA: at most 8 per thread and 256 / d_h row groups
-  const int rows_cta = std::max(G, (8 * std::max(1, 256 / cfg.head_dim)) / G * G);
-  ca.bchunk = std::max(1, rows_cta / G);
-  const int cchunks = (B + ca.bchunk - 1) / ca.bchunk;
-  ca.max_pieces = L.G + 1;
-  const size_t smem_c =
-      ((size_t)ca.bchunk * G * (cfg.d_c + ca.max_pieces) + 64 * (size_t)cfg.head_dim) * sizeof(float);
+  ca.ncols = (size_t)cfg.d_c * (64 + kCmbRows) * sizeof(float) <= 160 * 1024 ? 64 : 32;
+  ca.vec_ok = cfg.head_dim % (16 / (int)sizeof(T)) == 0;
+  const size_t smem_c = (size_t)cfg.d_c * (ca.ncols + kCmbRows) * sizeof(float) +
+                        (size_t)16 * (cfg.d_c + 8) * sizeof(__nv_bfloat16);   // + the MMA form's A tile
+  const int n_rbc = (B * G + kCmbRows - 1) / kCmbRows, n_dc = (cfg.head_dim + ca.ncols - 1) / ca.ncols;
   e = cudaFuncSetAttribute(combine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
   if (e != cudaSuccess) return e;
-  combine_kernel<T><<<cfg.n_kv_heads * cchunks, 256, smem_c, s>>>(ca);
-  return cudaGetLastError();
+  return mla_launch_kernel(combine_kernel<T>, dim3(cfg.n_kv_heads * n_rbc * n_dc), dim3(256), smem_c, s, p.opt_pdl,
+                           ca);
 }
 
 }  // namespace mla

@@ -40,20 +40,31 @@ __device__ inline int block_exscan(int v, int* total, int* s_warp) {
   return base + x - v;
 }
 
-// Single-block schedule builder.  Must be run by one whole CTA.  `scratch` (shared memory,
-// `scratch_ints` ints) holds the per-sequence arrays when they fit, so the searches below
-// run on shared memory; otherwise they live in the workspace.
+// Single-block schedule builder.  Must be run by one whole CTA.  When `scratch` (shared
+// memory, `scratch_ints` ints) can hold all of it, the schedule is built there and copied out
+// once at the end, so no step waits on a global-memory round trip; otherwise it is built in
+// the workspace directly.
 __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int B, int T_cap,
-                                      int tile, int G, Sched s, int32_t* err, int32_t* scratch,
+                                      int tile, int G, Sched out, int32_t* err, int32_t* scratch,
                                       int scratch_ints) {
   __shared__ int s_warp[32];
   const int tid = threadIdx.x, nt = blockDim.x;
-  int32_t* seq_len = nullptr;  // validated lengths, when there is room to keep them
-  if (scratch && 4 * B + 1 <= scratch_ints) {
-    s.seq_tile0 = scratch;
-    s.seq_ntiles = scratch + B;
-    s.seq_ne = scratch + 2 * B;
-    seq_len = scratch + 3 * B + 1;
+  const int Pcap = B + G;
+  const bool local = scratch && (long long)9 * B + 4 * G + 2 <= scratch_ints;
+  Sched s = out;
+  int32_t* seq_len = nullptr;
+  if (local) {
+    int32_t* q = scratch;
+    s.seq_tile0 = q; q += B;
+    s.seq_ntiles = q; q += B;
+    s.seq_ne = q; q += B + 1;
+    s.seq_first = q; q += B;
+    s.seq_np = q; q += B;
+    s.worker_first = q; q += G + 1;
+    s.piece_b = q; q += Pcap;
+    s.piece_t0 = q; q += Pcap;
+    s.piece_t1 = q; q += Pcap;
+    seq_len = q;  // [B]
   }
   // 1. tiles per sequence; exclusive prefix sums of tiles and of non-empty sequences
   int carry_t = 0, carry_ne = 0;
@@ -140,6 +151,22 @@ __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int 
     int b = s.piece_b[p];
     if (p == 0 || s.piece_b[p - 1] != b) s.seq_first[b] = p;
     atomicAdd(&s.seq_np[b], 1);
+  }
+  if (local) {   // copy the schedule out (coalesced)
+    __syncthreads();
+    for (int i = tid; i < B; i += nt) {
+      out.seq_tile0[i] = s.seq_tile0[i];
+      out.seq_ntiles[i] = s.seq_ntiles[i];
+      out.seq_first[i] = s.seq_first[i];
+      out.seq_np[i] = s.seq_np[i];
+    }
+    for (int i = tid; i <= B; i += nt) out.seq_ne[i] = s.seq_ne[i];
+    for (int i = tid; i <= G; i += nt) out.worker_first[i] = s.worker_first[i];
+    for (int i = tid; i < P; i += nt) {
+      out.piece_b[i] = s.piece_b[i];
+      out.piece_t0[i] = s.piece_t0[i];
+      out.piece_t1[i] = s.piece_t1[i];
+    }
   }
 }
 

@@ -248,6 +248,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the schedule, absorbed queries and the cache come from earlier kernels
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tmem = misc->tmem_base;
   const int w = blockIdx.x;
   if (threadIdx.x == 0) MLA_TRACE(7, 0);
@@ -873,8 +876,7 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, int B,
   if (e != cudaSuccess) return e;
   // the optional profiling events bracket the launch alone, after all host-side set-up
   if ((e = mla_profile_event(p, 0, s)) != cudaSuccess) return e;
-  kern<<<G, 384, L.total, s>>>(tm_c, tm_q, a);
-  e = cudaGetLastError();
+  e = mla_launch_kernel(kern, dim3(G), dim3(384), L.total, s, p.opt_pdl, tm_c, tm_q, a);
   if (e != cudaSuccess) return e;
   if ((e = mla_profile_event(p, 1, s)) != cudaSuccess) return e;
   return cudaSuccess;

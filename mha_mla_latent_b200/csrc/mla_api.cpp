@@ -29,7 +29,7 @@ mla_status_t validate_config(const mla_config_t* c) {
     return MLA_ERR_UNSUPPORTED;
   // limits of the kernels in this build
   if (c->head_dim > 256 || c->d_c > 1024 || c->n_heads > 256) return MLA_ERR_UNSUPPORTED;
-  if (c->d_c % 2 != 0) return MLA_ERR_UNSUPPORTED;
+  if (c->d_c % 4 != 0) return MLA_ERR_UNSUPPORTED;   // float4 rows in the split merge
   return MLA_OK;
 }
 
@@ -54,7 +54,8 @@ bool dev_alloc_copy(void** dst, const void* src, size_t bytes) {
 
 void free_plan(mla_plan* p) {
   if (!p) return;
-  void* bufs[] = {p->W_app, p->W_ukT, p->W_uv, p->nope_idx, p->rope_pair, p->theta, p->err};
+  void* bufs[] = {p->W_app, p->W_ukT, p->W_uv, p->nope_idx, p->rope_pair, p->theta, p->err, p->app_part,
+                  p->app_ticket};
   for (void* b : bufs)
     if (b) cudaFree(b);
   delete p;
@@ -166,6 +167,11 @@ mla_status_t mla_plan_create(const mla_config_t* cfg, const void* W_dkv, const v
             dev_alloc_copy((void**)&p->theta, theta.data(), theta.size() * sizeof(double)) &&
             cudaMalloc((void**)&p->err, sizeof(int32_t)) == cudaSuccess &&
             cudaMemset(p->err, 0, sizeof(int32_t)) == cudaSuccess;
+  // decode-step append scratch: 8 hidden-dim slices x (tiles of 32 tokens x 32 columns)
+  const size_t app_tiles = (size_t)((p->ncols + 31) / 32) * ((kAppMaxSmallTokens + 31) / 32);
+  ok = ok && cudaMalloc((void**)&p->app_part, app_tiles * 8 * 32 * 32 * sizeof(float)) == cudaSuccess &&
+       cudaMalloc((void**)&p->app_ticket, app_tiles * sizeof(int32_t)) == cudaSuccess &&
+       cudaMemset(p->app_ticket, 0, app_tiles * sizeof(int32_t)) == cudaSuccess;
   if (!ok) {
     free_plan(p);
     return MLA_ERR_CUDA;
@@ -189,6 +195,10 @@ mla_status_t mla_plan_set_option(mla_plan_t* plan, int32_t option, int64_t value
       return MLA_OK;
     case MLA_OPT_PROFILE_EVENTS:
       plan->opt_events = (const void* const*)(uintptr_t)value;
+      return MLA_OK;
+    case MLA_OPT_OVERLAP_LAUNCH:
+      if (value < 0 || value > 1) return MLA_ERR_INVALID_ARG;
+      plan->opt_pdl = (int)value;
       return MLA_OK;
   }
   return MLA_ERR_INVALID_ARG;

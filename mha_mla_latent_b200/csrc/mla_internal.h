@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "mla_api.h"
 
 // Element offset of RoPE key dim j of KV head g, token t of sequence b, in the blocked
@@ -12,6 +14,9 @@ inline __host__ __device__ size_t mla_kr_offset(int b, int t, int g, int j, int 
   const size_t blocks = (size_t)(T_cap + 31) / 32;
   return (((size_t)b * blocks + (size_t)(t >> 5)) * n_kv + g) * 32u * r2 + (size_t)(t & 31) * r2 + j;
 }
+
+// Largest token count the decode-step append path takes (its scratch is sized for it).
+constexpr int kAppMaxSmallTokens = 128;
 
 struct mla_plan {
   mla_config_t cfg;
@@ -28,11 +33,32 @@ struct mla_plan {
   int32_t* rope_pair = nullptr;  // [n_kv][r]   kept pair indices, ascending
   double* theta = nullptr;       // [d_h/2]     RoPE frequencies
   int32_t* err = nullptr;        // device error word (MLA_DEVERR_* bits)
+  float* app_part = nullptr;     // decode-step append: partial tiles [8][tiles][32*32]
+  int32_t* app_ticket = nullptr; // decode-step append: per-tile arrival counters (zeroed)
   // options
   int opt_kernel = 0;
   int opt_splits = 0;
   const void* const* opt_events = nullptr;  // cudaEvent_t[2] or null
+  int opt_pdl = 1;                            // programmatic dependent launch
 };
+
+// Launches a kernel, with programmatic stream serialization when `pdl` is set (the kernel
+// then orders itself after its predecessor with griddepcontrol.wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t mla_launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                     bool pdl, Args&&... args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&lc, kern, std::forward<Args>(args)...);
+}
 
 // Records profiling event i (0 before, 1 after the split-K kernel) when the option is set.
 // Under stream capture the record becomes an external event node of the graph, so the
