@@ -153,7 +153,7 @@ struct DecodeArgs {
   int B, H, n_kv, r, d_c, R;
   const float* qlat;
   const float* qrope;
-  float* opart;     // [H][P][d_c]
+  float* opart;     // [P][H][d_c]
   float* mlpart;    // [H][P][2]
   int P;            // piece capacity
   Sched sched;
@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(DecodeArgs a) {
     for (int e = 0; e < kSimtMaxE; ++e) {
       if (e >= nE) break;
       int idx = tid + 256 * e;
-      if (idx < H * dc) a.opart[((size_t)(idx / dc) * a.P + pc) * dc + idx % dc] = O[e];
+      if (idx < H * dc) a.opart[((size_t)pc * H + idx / dc) * dc + idx % dc] = O[e];
     }
     if (tid < H) {
       a.mlpart[((size_t)tid * a.P + pc) * 2] = s_m[tid];
@@ -329,7 +329,8 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
       const int b = row / G, h = g * G + row % G;
       const int first = __ldg(a.sched.seq_first + b), np = __ldg(a.sched.seq_np + b);
       const float* ml = a.mlpart + ((size_t)h * a.P + first) * 2;
-      const float* op = a.opart + ((size_t)h * a.P + first) * dc;
+      const float* op = a.opart + ((size_t)first * a.H + h) * dc;   // piece j at op + j * H * d_c
+      const size_t ps = (size_t)a.H * dc;
       // pieces j = lane (+32k): running max and sum; the first 8 pieces' latent rows are
       // loaded in the same round trip (they do not depend on the weights)
       const int nc4 = dc / 4;
@@ -337,8 +338,8 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         if (k < np) {
-          if (lane < nc4) v0[k] = __ldg(reinterpret_cast<const float4*>(op + (size_t)k * dc) + lane);
-          if (lane + 32 < nc4) v1[k] = __ldg(reinterpret_cast<const float4*>(op + (size_t)k * dc) + lane + 32);
+          if (lane < nc4) v0[k] = __ldg(reinterpret_cast<const float4*>(op + (size_t)k * ps) + lane);
+          if (lane + 32 < nc4) v1[k] = __ldg(reinterpret_cast<const float4*>(op + (size_t)k * ps) + lane + 32);
         }
       }
       float mj = -INFINITY, lj = 0.f;
@@ -365,11 +366,11 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
       for (int j = 8; j < np; ++j) {   // more than 8 pieces: one at a time
         const float w = j < 32 ? __shfl_sync(0xffffffffu, wl, j) : exp2f(__ldg(ml + 2 * j) - M);
         if (lane < nc4) {
-          const float4 x = __ldg(reinterpret_cast<const float4*>(op + (size_t)j * dc) + lane);
+          const float4 x = __ldg(reinterpret_cast<const float4*>(op + (size_t)j * ps) + lane);
           a0.x += w * x.x; a0.y += w * x.y; a0.z += w * x.z; a0.w += w * x.w;
         }
         if (lane + 32 < nc4) {
-          const float4 x = __ldg(reinterpret_cast<const float4*>(op + (size_t)j * dc) + lane + 32);
+          const float4 x = __ldg(reinterpret_cast<const float4*>(op + (size_t)j * ps) + lane + 32);
           a1.x += w * x.x; a1.y += w * x.y; a1.z += w * x.z; a1.w += w * x.w;
         }
       }
@@ -380,7 +381,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < np; ++j) {
           const float w = j < 32 ? __shfl_sync(0xffffffffu, wl, j) : exp2f(__ldg(ml + 2 * j) - M);
-          const float4 x = __ldg(reinterpret_cast<const float4*>(op + (size_t)j * dc) + c4);
+          const float4 x = __ldg(reinterpret_cast<const float4*>(op + (size_t)j * ps) + c4);
           acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
         }
         *reinterpret_cast<float4*>(o + 4 * c4) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);

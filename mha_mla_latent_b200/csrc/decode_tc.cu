@@ -52,7 +52,7 @@ constexpr uint32_t kPtBytes = 2 * kPtAtom;
 struct TcArgs {
   int B, H, d_c, R, r2, T_cap, P;
   Sched sched;
-  float* opart;           // [H][P][d_c]
+  float* opart;           // [P][H][d_c]
   float* mlpart;          // [H][P][2]
   const float* qrope;     // [B][H][2r] rotated, scaled RoPE query part
   const __half* scales;   // int4: [B*T_cap][d_c/32]
@@ -90,10 +90,8 @@ constexpr int kFixedBars = 18;
 struct Misc {  // small shared scratch
   uint32_t tmem_base;
   int abort_flag;
-  int vote[2][kSoftWarps];
-  float red_max[2][4][kH];
-  float red_l[4][kH];
-  float mt[kSoftWarps][kHh];
+  alignas(16) float red_max[2][4][kH];   // per tile parity, quarter, head: the warp's max score
+  alignas(16) float red_l[4][kH];          // (read as float4)
   int kr_released;   // softmax warps done with the RoPE key stage (the 8th issues the next copy)
   int kr_issued;     // RoPE key copies issued
 };
@@ -176,13 +174,17 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[kH], int lane) {
 #ifdef MLA_TC_TRACE
 // Timeline instrumentation for development builds only (-DMLA_TC_TRACE): %globaltimer
 // stamps per (CTA, event, tile) for the first kTraceCtas CTAs.
-constexpr int kTraceCtas = 4, kTraceEv = 40, kTraceTiles = 64;
+constexpr int kTraceCtas = 4, kTraceEv = 48, kTraceTiles = 64;
 __device__ unsigned long long g_trace[kTraceCtas * kTraceEv * kTraceTiles];
 __device__ unsigned long long g_cta_span[1024 * 2];
+__device__ __forceinline__ int trace_slot() {   // CTAs 0, 1 and two that straddle sequences
+  return blockIdx.x < 2 ? (int)blockIdx.x : blockIdx.x == 23 ? 2 : blockIdx.x == 60 ? 3 : -1;
+}
 #define MLA_TRACE(ev, n)                                                                          \
   do {                                                                                            \
-    if (blockIdx.x < kTraceCtas && (n) < kTraceTiles)                                             \
-      g_trace[(blockIdx.x * kTraceEv + (ev)) * kTraceTiles + (n)] = globaltimer();                \
+    const int ts_ = trace_slot();                                                                 \
+    if (ts_ >= 0 && (n) < kTraceTiles)                                                            \
+      g_trace[(ts_ * kTraceEv + (ev)) * kTraceTiles + (n)] = globaltimer();                       \
   } while (0)
 #else
 #define MLA_TRACE(ev, n) do { } while (0)
@@ -498,7 +500,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
       const uint8_t* src = a.kr_base + mla_kr_offset(ti.b, ti.t, 0, 0, a.T_cap, n_kv, R2) * 2;
       fence_proxy_async_smem();
       mbar_expect_tx(bars.kr_full(), nblk * kr_blk);
-      bulk_load(sbase_u32 + a.off_kr, src, nblk * kr_blk, bars.kr_full());
+      for (int k = 0; k < nblk; ++k)   // one copy per 32-token block: they proceed in parallel
+        bulk_load(sbase_u32 + a.off_kr + k * kr_blk, src + (size_t)k * kr_blk, kr_blk, bars.kr_full());
       misc->kr_issued += 1;
     };
     auto fetch_kr = [&](int k, const TileIter& ti_after) -> bool {   // tile k's keys -> kr
@@ -515,25 +518,23 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
       return true;
     };
     if (it.valid()) {   // a worker with no tiles issues and waits for nothing
+      for (int i = threadIdx.x - 128; i < kH * R2; i += 32 * kSoftWarps)
+        qr_s[i] = __ldg(a.qrope + (size_t)it.b * kH * R2 + i);
       if (sw == 0 && lane == 0) issue_kr(it);
       TileIter nx = it;
       nx.next();
       ok = fetch_kr(0, nx);
+      if (ok) ok = grp_sync(1);   // the first piece's RoPE queries are in place
     }
     while (ok && it.valid()) {
       const int pc = it.pc;
       const bool first = it.first_of_piece();
-      if (first) {
-        // the previous piece's RoPE queries are no longer read: load this piece's
-        ok = grp_sync(1);
-        if (!ok) break;
-        for (int i = threadIdx.x - 128; i < kH * R2; i += 32 * kSoftWarps)
-          qr_s[i] = __ldg(a.qrope + (size_t)it.b * kH * R2 + i);
-        ok = grp_sync(1);
-        if (!ok) break;
+      if (first) {   // this piece's RoPE queries are in qr_s[u & 1] (loaded one piece ahead)
 #pragma unroll
         for (int h = 0; h < kHh; ++h) { m[h] = -INFINITY; l[h] = 0.f; }
+        if (warp == 4 && lane == 0) MLA_TRACE(43, n);
       }
+      const float* qr = qr_s + (u & 1) * (kH * R2);
       const int sb = n & 1, pb = n % a.NP, ob = u % a.NO;
       const int nvalid = min(kTile, it.t1 - it.t);
       const bool valid = tr < nvalid;
@@ -558,8 +559,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
       for (int h = 0; h < kHh; ++h) {
         const int H = kHh * hh + h;
         const uint4 kw = kr[h];
-        const float4 qa = *reinterpret_cast<const float4*>(qr_s + H * R2);
-        const float4 qb = *reinterpret_cast<const float4*>(qr_s + H * R2 + 4);
+        const float4 qa = *reinterpret_cast<const float4*>(qr + H * R2);
+        const float4 qb = *reinterpret_cast<const float4*>(qr + H * R2 + 4);
         v[h] += qa.x * bf16lo(kw.x) + qa.y * bf16hi(kw.x) + qa.z * bf16lo(kw.y) + qa.w * bf16hi(kw.y) +
                 qb.x * bf16lo(kw.z) + qb.y * bf16hi(kw.z) + qb.z * bf16lo(kw.w) + qb.w * bf16hi(kw.w);
       }
@@ -579,23 +580,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
 #pragma unroll
         for (int h = 0; h < kHh; ++h) v[h] = -INFINITY;
       }
-      // does any score exceed its head's running max by more than tau?
-      bool need = false;
-      if (valid) {
-#pragma unroll
-        for (int h = 0; h < kHh; ++h) need |= (v[h] - m[h] > kTau);
-      }
-      need = __any_sync(0xffffffffu, need);
-      if (lane == 0) MLA_TRACE(32 + sw, n);
-      if (lane == 0) misc->vote[n & 1][sw] = need ? 1 : 0;
-      ok = grp_sync(0);
-      if (!ok) break;
-      bool need_all = false;
-#pragma unroll
-      for (int i = 0; i < kSoftWarps; ++i) need_all |= misc->vote[n & 1][i] != 0;
-      if (warp == 4 && lane == 0) MLA_TRACE(11, n);
-      if (need_all) {
-        // exact tile max per head: over the 32 tokens of the warp, then over the 4 quarters
+      // per-head maximum over this warp's 32 tokens, published for the other quarters; after
+      // the barrier every warp knows the tile's exact per-head maximum, and raises its running
+      // max (lazily: only when some score exceeds it by more than tau) identically with the
+      // other warps of its head half
+      {
         float wmax = -INFINITY;   // lane h ends with head 16hh + h
 #pragma unroll
         for (int h = 0; h < kHh; ++h) {
@@ -603,19 +592,32 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
           wmax = (lane == h) ? r : wmax;
         }
         if (lane < 16) misc->red_max[n & 1][q][kHh * hh + lane] = wmax;
-        ok = grp_sync(1);
-        if (!ok) break;
-        if (lane < 16) {
-          const int H = kHh * hh + lane;
-          misc->mt[sw][lane] = fmaxf(fmaxf(misc->red_max[n & 1][0][H], misc->red_max[n & 1][1][H]),
-                                     fmaxf(misc->red_max[n & 1][2][H], misc->red_max[n & 1][3][H]));
-        }
-        __syncwarp();
+      }
+      if (lane == 0) MLA_TRACE(32 + sw, n);
+      ok = grp_sync(0);
+      if (!ok) break;
+      if (warp == 4 && lane == 0) MLA_TRACE(11, n);
+      float tmax[kHh];
+#pragma unroll
+      for (int h4 = 0; h4 < kHh; h4 += 4) {
+        const float4 q0 = *reinterpret_cast<const float4*>(&misc->red_max[n & 1][0][kHh * hh + h4]);
+        const float4 q1 = *reinterpret_cast<const float4*>(&misc->red_max[n & 1][1][kHh * hh + h4]);
+        const float4 q2 = *reinterpret_cast<const float4*>(&misc->red_max[n & 1][2][kHh * hh + h4]);
+        const float4 q3 = *reinterpret_cast<const float4*>(&misc->red_max[n & 1][3][kHh * hh + h4]);
+        tmax[h4 + 0] = fmaxf(fmaxf(q0.x, q1.x), fmaxf(q2.x, q3.x));
+        tmax[h4 + 1] = fmaxf(fmaxf(q0.y, q1.y), fmaxf(q2.y, q3.y));
+        tmax[h4 + 2] = fmaxf(fmaxf(q0.z, q1.z), fmaxf(q2.z, q3.z));
+        tmax[h4 + 3] = fmaxf(fmaxf(q0.w, q1.w), fmaxf(q2.w, q3.w));
+      }
+      bool need = false;
+#pragma unroll
+      for (int h = 0; h < kHh; ++h) need |= (tmax[h] - m[h] > kTau);
+      if (need) {
         bool any_scale = false;
         float my_alpha = 1.f;   // the factor of head 16hh + lane (lanes < 16)
 #pragma unroll
         for (int h = 0; h < kHh; ++h) {
-          const float mn = fmaxf(m[h], misc->mt[sw][h]);
+          const float mn = fmaxf(m[h], tmax[h]);
           const float al = exp2f(m[h] - mn);   // m = -inf on a piece's first tile -> 0
           any_scale |= (mn != m[h]);
           m[h] = mn;
@@ -681,8 +683,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
         // ---------------- piece epilogue: partial (m, l, O) for the split merge
         const float lsum = transpose_reduce16<false>(l, lane);   // l is reset by the next piece
         if (lane < 16) misc->red_l[q][kHh * hh + lane] = lsum;
+        {   // the next piece's RoPE queries, into the other buffer (visible after the barrier)
+          TileIter nx = it;
+          nx.next();
+          if (nx.valid())
+            for (int i = threadIdx.x - 128; i < kH * R2; i += 32 * kSoftWarps)
+              qr_s[((u + 1) & 1) * (kH * R2) + i] = __ldg(a.qrope + (size_t)nx.b * kH * R2 + i);
+        }
+        if (warp == 4 && lane == 0) MLA_TRACE(44, u);
         ok = grp_sync(1);
         if (!ok) break;
+        if (warp == 4 && lane == 0) MLA_TRACE(40, u);
         if (q == 0 && lane < 16) {
           const int H = kHh * hh + lane;
           const float L = misc->red_l[0][H] + misc->red_l[1][H] + misc->red_l[2][H] + misc->red_l[3][H];
@@ -694,24 +705,30 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
         }
         ok = wwait(bars.o_full(ob), (u / a.NO) & 1);
         if (!ok) break;
+        if (warp == 4 && lane == 0) MLA_TRACE(41, u);
         tc_fence_after();
         if (q < 2) {
           // O^T rows (M = 64 layout): head 16q + lane in lane `lane` (< 16) of quarter q; the
-          // two warps of the quarter take alternate 16-column chunks
+          // two warps of the quarter take one half of the columns each, 32 per TMEM wait
           const int H = 16 * q + lane;
-          float* dst = a.opart + ((size_t)H * a.P + pc) * dc;
-          for (int cc = hh; cc < dc / 16; cc += 2) {
-            uint32_t o[16];
-            tmem_ld16(taddr(tmem, 32 * q, O_COL + ob * dc + 16 * cc), o);
+          float* dst = a.opart + ((size_t)pc * kH + H) * dc;
+          const int half = dc / 2;   // a multiple of 32
+          for (int c0 = hh * half; c0 < (hh + 1) * half; c0 += 32) {
+            uint32_t o[2][16];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) tmem_ld16(taddr(tmem, 32 * q, O_COL + ob * dc + c0 + 16 * k), o[k]);
             tmem_wait_ld();
             if (lane < 16) {
 #pragma unroll
-              for (int k = 0; k < 16; k += 4)
-                *reinterpret_cast<float4*>(dst + 16 * cc + k) = make_float4(u2f(o[k]), u2f(o[k + 1]), u2f(o[k + 2]),
-                                                                            u2f(o[k + 3]));
+              for (int k = 0; k < 2; ++k)
+#pragma unroll
+                  for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<float4*>(dst + c0 + 16 * k + e) =
+                        make_float4(u2f(o[k][e]), u2f(o[k][e + 1]), u2f(o[k][e + 2]), u2f(o[k][e + 3]));
             }
           }
         }
+        if (warp == 4 && lane == 0) MLA_TRACE(42, u);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.o_empty(ob));
@@ -782,7 +799,7 @@ static TcLayout tc_layout(int dc, int R, int r2, bool int4) {
   const uint32_t c_stage = (uint32_t)(dc / 64) * kBox;
   const uint32_t raw_stage = (uint32_t)kTile * (dc / 2) + (uint32_t)kTile * (dc / 16);
   const uint32_t q_bytes = (uint32_t)(dc / 64 > 2 ? dc / 64 - 2 : 0) * kQBox;  // boxes 0-1 sit in P^T padding
-  const uint32_t qr_bytes = (uint32_t)kH * r2 * 4;
+  const uint32_t qr_bytes = 2u * kH * r2 * 4;   // two pieces' RoPE queries
   const uint32_t kr_bytes = (uint32_t)kTile * R * 2;
   auto size = [&](int nc, int nraw, int np) {
     uint32_t s = nc * c_stage + q_bytes + np * kPtBytes + kr_bytes;
