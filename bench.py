@@ -16,6 +16,7 @@ max-over-ranks time.
 """
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -179,6 +180,41 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def code_sha1(path):
+    """SHA-1 of a C++/CUDA source with // comments and blank lines removed, so an edit of
+    comments alone keeps the recorded counters valid while any code change voids them."""
+    lines = []
+    with open(path) as f:
+        for line in f:
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                lines.append(code)
+    return hashlib.sha1("\n".join(lines).encode()).hexdigest()
+
+
+def measured_traffic(workload_name, kernel_used):
+    """DRAM bytes (read + write) per launch of the tensor-core attention kernel, from the
+    committed ncu summary, when that summary was taken on this workload and on the current
+    kernel code (else None: the counters no longer describe the kernel)."""
+    if kernel_used != 2:
+        return None
+    path = os.path.join(ROOT, "profiles", "decode_tc_traffic.txt")
+    src = os.path.join(ROOT, "mha_mla_latent_b200", "csrc", "decode_tc.cu")
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if "=" in line and not line.startswith("#"):
+                    k, v = line.strip().split("=", 1)
+                    kv[k] = v
+        sha = code_sha1(src)
+        if kv.get("workload") != workload_name or kv.get("source_sha1") != sha:
+            return None
+        return int(kv["traffic_bytes"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def measured_peak_hbm():
@@ -385,7 +421,8 @@ def run_ours(args):
         "config": dict(wl_config(wl, lens), parallelism=f"replicas x{world}" if world > 1 else "single GPU",
                        l2=f"{n_rep} cache replicas rotated per step ({n_rep * cache_bytes / 2**20:.0f} MiB > 2x L2)"),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "kernel": kernel_name,
+                     "frac": achieved / peak, "traffic": measured_traffic(args.workload, kernel_used),
+                     "kernel": kernel_name,
                      "bytes_per_launch": kern_bytes, "avg_launch_ms": kern_avg_ms, "peak_source": peak_src},
         "decode_only_ms": decode_ms, "decode_roofline_frac": decode_frac,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

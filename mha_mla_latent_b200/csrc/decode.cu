@@ -55,8 +55,6 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
   const int n_rb = (rows_total + kAbsRows - 1) / kAbsRows;
   const int n_cc = (a.d_c + kAbsCols - 1) / kAbsCols;
   if (blockIdx.x == a.n_kv * n_rb * n_cc) {  // the last CTA builds the split-K schedule
-    pdl_wait();
-    pdl_trigger();
     build_schedule(a.seq_lens, a.B, a.T_cap, a.tile, a.G, a.sched, a.err, reinterpret_cast<int32_t*>(sm),
                    a.sched_ints);
     return;

@@ -41,9 +41,10 @@ __device__ inline int block_exscan(int v, int* total, int* s_warp) {
 }
 
 // Single-block schedule builder.  Must be run by one whole CTA.  When `scratch` (shared
-// memory, `scratch_ints` ints) can hold all of it, the schedule is built there and copied out
-// once at the end, so no step waits on a global-memory round trip; otherwise it is built in
-// the workspace directly.
+// memory, `scratch_ints` ints) can hold all of it, the schedule is built there (it depends
+// on the sequence lengths only, so this overlaps the kernel before) and copied out once,
+// after the programmatic dependency wait; otherwise the wait comes first and the schedule
+// is built in the workspace directly.
 __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int B, int T_cap,
                                       int tile, int G, Sched out, int32_t* err, int32_t* scratch,
                                       int scratch_ints) {
@@ -65,6 +66,9 @@ __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int 
     s.piece_t0 = q; q += Pcap;
     s.piece_t1 = q; q += Pcap;
     seq_len = q;  // [B]
+  } else {
+    pdl_wait();
+    pdl_trigger();
   }
   // 1. tiles per sequence; exclusive prefix sums of tiles and of non-empty sequences
   int carry_t = 0, carry_ne = 0;
@@ -154,6 +158,8 @@ __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int 
   }
   if (local) {   // copy the schedule out (coalesced)
     __syncthreads();
+    pdl_wait();   // the previous call's kernels may still read the workspace
+    pdl_trigger();
     for (int i = tid; i < B; i += nt) {
       out.seq_tile0[i] = s.seq_tile0[i];
       out.seq_ntiles[i] = s.seq_ntiles[i];

@@ -6,27 +6,25 @@
 // latent taken through W_uv.  Because every head reads the same c_kv row, the per-tile
 // work is a real dense contraction.  For a tile of 128 cached tokens of one sequence:
 //     S[t][h]   = sum_c C[t][c] * Qlat[h][c]            MMA1  M = 128 tokens, N = 32 heads
-//     S[t][h]  += sum_j KR[t][g(h)][j] * Qrope[h][j]    CUDA cores (fp32), from the KR tile
+//     S[t][h]  += sum_j KR[t][g(h)][j] * Qrope[h][j]    CUDA cores (fp32)
 //     O^T[h][d] += sum_t P^T[h][t] * C[t][d]            MMA2  M = 64 (32 heads + pad), N = d_c
 // MMA2 reuses the C tile already in shared memory as an MN-major B operand, so each
-// cached byte is read from HBM once.  A tcgen05.mma costs about the same issue time
-// whatever its shape, so the orientations maximise work per instruction: per 128
-// tokens d_c/16 + 8 instructions (24 at d_c = 256).
+// cached byte is read from HBM once.  The RoPE term has 8 dims per head; as extra K of
+// MMA1 it would double the MMAs per tile, so it runs on the CUDA cores beside them.
 //
 // One persistent CTA per SM walks its contiguous range of tiles (split-K schedule).
-// Warp roles:
-//   warp 0      TMA producer: Q_lat per piece; C and KR tiles into two rings of stages
-//               (int4 cache: codes + scales into a raw ring instead of C); L2 prefetch of
-//               the tiles after the rings
-//   warp 1      TMEM owner and single-thread MMA issuer; MMA1(n+1) is issued before
-//               MMA2(n) so the tensor pipe works while the softmax of tile n finishes
-//   warps 2-9   softmax: one token per thread (TMEM lane), 16 heads per thread (two warps
-//               per lane quarter); adds the
+// Warp roles (12 warps, three warpgroups; setmaxnreg gives warpgroups 1-2 224 registers):
+//   warp 0      TMA producer: Q_lat per piece, C tiles into a ring of stages (int4 cache:
+//               codes + scales into a raw ring instead)
+//   warp 1      TMEM owner and single-thread MMA issuer; it polls and issues MMA2 of the
+//               pending tile as soon as its P^T is ready, else MMA1 of the next tile
+//   warps 2-3   (int4 cache) dequantise codes*scale into the bf16 C stage
+//   warps 4-11  softmax: one token per thread (TMEM lane), 16 heads per thread (two warps
+//               per lane quarter); RoPE keys from a bulk-copied stage via registers, the
 //               RoPE score, online softmax in log2 units with lazy rescaling (the running
 //               max is raised only when a score exceeds it by more than 2^8, then the O
-//               rows are rescaled in TMEM), writes P^T (bf16) for MMA2, and per piece the
+//               rows are rescaled in TMEM), P^T (bf16) for MMA2, and per piece the
 //               partial (m, l, O) for the split merge
-//   warps 10-11 (int4 cache) dequantise codes*scale into the bf16 C stage
 // Every wait is bounded (about 1 s); a timeout sets MLA_DEVERR_TIMEOUT, all roles stop,
 // in-flight copies and MMAs are drained and TMEM is released before the CTA exits.
 #include <cuda.h>
