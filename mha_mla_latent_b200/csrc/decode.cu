@@ -41,8 +41,8 @@ struct AbsorbArgs {
 constexpr int kAbsRows = 8;    // (b, h) rows per CTA: one per warp in the product
 constexpr int kAbsCols = 64;   // latent columns per CTA: two per lane
 
-// grid: n_kv * (row blocks) * (column chunks) CTAs, plus one CTA that builds the split-K
-// schedule.  A CTA reads everything it needs (its W_uk^T slice, its query rows, the NoPE
+// grid: one CTA that builds the split-K schedule (block 0, so it is dispatched first), then
+// n_kv * (row blocks) * (column chunks) CTAs.  A CTA reads everything it needs (its W_uk^T slice, its query rows, the NoPE
 // index table, and for the first column chunk the RoPE tables and positions) in one batch
 // of loads, then q_lat[row][c] = scale * sum_j q[row][nope_j] * W_uk^T[g][j][c] with warp r
 // owning row r and lane l columns 2l, 2l+1 of the chunk.
@@ -53,15 +53,15 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
   const int G = a.H / a.n_kv;
   const int rows_total = a.B * G;
   const int n_rb = (rows_total + kAbsRows - 1) / kAbsRows;
-  const int n_cc = (a.d_c + kAbsCols - 1) / kAbsCols;
-  if (blockIdx.x == a.n_kv * n_rb * n_cc) {  // the last CTA builds the split-K schedule
+  if (blockIdx.x == 0) {  // the split-K schedule
     build_schedule(a.seq_lens, a.B, a.T_cap, a.tile, a.G, a.sched, a.err, reinterpret_cast<int32_t*>(sm),
                    a.sched_ints);
     return;
   }
-  const int g = blockIdx.x % a.n_kv;
-  const int rb = (blockIdx.x / a.n_kv) % n_rb;
-  const int cc = blockIdx.x / (a.n_kv * n_rb);
+  const int blk = blockIdx.x - 1;
+  const int g = blk % a.n_kv;
+  const int rb = (blk / a.n_kv) % n_rb;
+  const int cc = blk / (a.n_kv * n_rb);
   const int row0 = rb * kAbsRows, c0 = cc * kAbsCols;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int dn = a.dn, dh = a.dh, dnp = (dn + 3) & ~3;
@@ -98,19 +98,20 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
   }
   __syncthreads();
   for (int i = tid; i < kAbsRows * dn; i += 256) s_qn[(i / dn) * dnp + i % dn] = s_q[(i / dn) * dh + s_idx[i % dn]];
-  // outputs are read by the attention kernel of the previous call until it has finished
+  // the outputs below are read by the attention kernel of the previous call until it has
+  // finished (computing before this wait, while that kernel runs, measured slower)
   pdl_wait();
   pdl_trigger();
+  // RoPE query part: rotate the kept pairs at position L-1 (angle in double), scale
+  float ro0 = 0.f, ro1 = 0.f;
   if (rope_item) {
-    const int r = tid / a.r, j = tid % a.r, row = row0 + r;
-    const int b = row / G, h = g * G + row % G;
+    const int r = tid / a.r;
     const int p = (rp_pos >= 1 && rp_pos <= a.T_cap) ? rp_pos - 1 : 0;
     const double x0 = s_q[r * dh + 2 * rp_k], x1 = s_q[r * dh + 2 * rp_k + 1];
     double sn, cs;
     sincos((double)p * rp_th, &sn, &cs);
-    const size_t o = ((size_t)b * a.H + h) * 2 * a.r + 2 * j;
-    a.qrope[o] = (float)((x0 * cs - x1 * sn) * (double)scale);
-    a.qrope[o + 1] = (float)((x0 * sn + x1 * cs) * (double)scale);
+    ro0 = (float)((x0 * cs - x1 * sn) * (double)scale);
+    ro1 = (float)((x0 * sn + x1 * cs) * (double)scale);
   }
   __syncthreads();
   // ---- product: warp r -> row r, lane l -> columns 2l, 2l+1 of the chunk
@@ -131,6 +132,12 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
     const float2 w = *reinterpret_cast<const float2*>(s_w + j * kAbsCols + 2 * lane);
     acc0 += qn[j] * w.x;
     acc1 += qn[j] * w.y;
+  }
+  if (rope_item) {
+    const int rr = tid / a.r, jr = tid % a.r, rrow = row0 + rr;
+    const size_t o = ((size_t)(rrow / G) * a.H + g * G + rrow % G) * 2 * a.r + 2 * jr;
+    a.qrope[o] = ro0;
+    a.qrope[o + 1] = ro1;
   }
   if (row < rows_total && c < a.d_c) {
     const size_t o = ((size_t)(row / G) * a.H + g * G + row % G) * a.d_c + c;
@@ -318,14 +325,21 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
       for (int i = tid; i < dc * NCOL; i += 256) s_w[i] = 0.f;   // columns past d_h
     stage_rows_f32<T>(s_w, NCOL, dc, ncol, a.vec_ok && ncol == NCOL, [&](int c) { return W + (size_t)c * a.dh + d0; });
   }
+  // the schedule was written two kernels back (complete before the attention kernel let
+  // this one launch); the partials need the dependency wait
+  int first = 0, np = 0;
+  if (row0 + warp < rows_total) {
+    const int b = (row0 + warp) / G;
+    first = __ldg(a.sched.seq_first + b);
+    np = __ldg(a.sched.seq_np + b);
+  }
   pdl_wait();   // the partials of the attention kernel
   pdl_trigger();
   {
     const int r = warp, row = row0 + r;
     float* o = s_o + r * dc;
     if (row < rows_total) {
-      const int b = row / G, h = g * G + row % G;
-      const int first = __ldg(a.sched.seq_first + b), np = __ldg(a.sched.seq_np + b);
+      const int h = g * G + row % G;
       const float* ml = a.mlpart + ((size_t)h * a.P + first) * 2;
       const float* op = a.opart + ((size_t)first * a.H + h) * dc;   // piece j at op + j * H * d_c
       const size_t ps = (size_t)a.H * dc;
