@@ -129,6 +129,24 @@ MLA_API size_t mla_cache_bytes_per_token(const mla_config_t* cfg);
 MLA_API mla_status_t mla_select_pairs(const mla_config_t* cfg, const void* q_cal, const void* k_cal,
                               int32_t T, int32_t* pair_idx, float* contrib, void* stream);
 
+/* Fixed partial-RoPE pair sets, the alternatives to the 2-norm selection that the README
+ * "MHA2MLA" (§Fine-Tuning strategy tables: partial-RoPE versions) lists and the Notes
+ * (§消融实验, Partial-RoPE strategy comparison) compare.  With P = d_h/2 pairs, r = r_pairs
+ * and theta_k = base^(-2k/d_h) (k = 0 is the highest frequency):
+ *   MLA_PAIRS_HIGH     k = 0 .. r-1            (highest frequencies)
+ *   MLA_PAIRS_LOW      k = P-r .. P-1          (lowest frequencies)
+ *   MLA_PAIRS_UNIFORM  k_j = floor(j*P/r), j = 0 .. r-1   (evenly spaced)
+ *   MLA_PAIRS_FULL     every pair (requires r == P: full RoPE)
+ * The same set is used for every KV head.  pair_idx: HOST [n_kv][r] int32, ascending.
+ * Returns MLA_ERR_INVALID_ARG for an unknown strategy or r out of range.  No GPU use. */
+enum {
+  MLA_PAIRS_HIGH = 1,
+  MLA_PAIRS_UNIFORM = 2,
+  MLA_PAIRS_LOW = 5,
+  MLA_PAIRS_FULL = 0
+};
+MLA_API mla_status_t mla_fixed_pairs(const mla_config_t* cfg, int32_t strategy, int32_t* pair_idx);
+
 /* Build a plan: validate the config and copy/pack the converted weights into
  * plan-owned device memory.  All weight pointers are HOST memory in the config dtype.
  *   W_dkv    [d][d_c]            joint-SVD down-projection (U_trunc)

@@ -25,7 +25,9 @@ EXPORTED = (
     "mla_status_string", "mla_version", "mla_cache_bytes_per_token", "mla_select_pairs",
     "mla_plan_create", "mla_plan_destroy", "mla_plan_set_option", "mla_append",
     "mla_decode_workspace_bytes", "mla_decode", "mla_device_error", "mla_decode_noalloc",
+    "mla_fixed_pairs",
 )
+MLA_PAIRS_FULL, MLA_PAIRS_HIGH, MLA_PAIRS_UNIFORM, MLA_PAIRS_LOW = 0, 1, 2, 5
 MLA_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -59,6 +61,7 @@ def _load():
         "mla_version": (ctypes.c_char_p, []),
         "mla_cache_bytes_per_token": (sz, [cfgp]),
         "mla_select_pairs": (i32, [cfgp, vp, vp, i32, vp, vp, vp]),
+        "mla_fixed_pairs": (i32, [cfgp, i32, vp]),
         "mla_plan_create": (i32, [cfgp, vp, vp, vp, vp, vp, ctypes.POINTER(vp)]),
         "mla_plan_destroy": (None, [vp]),
         "mla_plan_set_option": (i32, [vp, i32, i64]),
@@ -127,6 +130,15 @@ def mla_status_string(status: int) -> str:
 
 def mla_cache_bytes_per_token(cfg: MlaConfig) -> int:
     return int(_lib.mla_cache_bytes_per_token(ctypes.byref(cfg)))
+
+
+def mla_fixed_pairs(cfg: MlaConfig, strategy: int, check=True):
+    """Fixed partial-RoPE pair set (MLA_PAIRS_*) -> numpy int32 [n_kv][r]."""
+    out = np.zeros((cfg.n_kv_heads, max(cfg.r_pairs, 0)), dtype=np.int32)
+    st = _lib.mla_fixed_pairs(ctypes.byref(cfg), int(strategy), out.ctypes.data_as(ctypes.c_void_p))
+    if check:
+        _check(st, "mla_fixed_pairs")
+    return out if st == MLA_OK else None
 
 
 def mla_select_pairs(cfg: MlaConfig, q_cal, k_cal, pair_idx, contrib=None, stream=None, check=True):

@@ -88,6 +88,35 @@ size_t mla_cache_bytes_per_token(const mla_config_t* cfg) {
   return (size_t)cfg->d_c * eb + rope;
 }
 
+mla_status_t mla_fixed_pairs(const mla_config_t* cfg, int32_t strategy, int32_t* pair_idx) {
+  if (!cfg || !pair_idx) return MLA_ERR_INVALID_ARG;
+  mla_status_t st = validate_config(cfg);
+  if (st != MLA_OK) return st;
+  const int P = cfg->head_dim / 2, r = cfg->r_pairs, nkv = cfg->n_kv_heads;
+  if (r < 0 || r > P) return MLA_ERR_INVALID_ARG;
+  std::vector<int32_t> ks(r);
+  switch (strategy) {
+    case MLA_PAIRS_HIGH:
+      for (int j = 0; j < r; ++j) ks[j] = j;
+      break;
+    case MLA_PAIRS_LOW:
+      for (int j = 0; j < r; ++j) ks[j] = P - r + j;
+      break;
+    case MLA_PAIRS_UNIFORM:
+      for (int j = 0; j < r; ++j) ks[j] = (int32_t)(((long long)j * P) / r);
+      break;
+    case MLA_PAIRS_FULL:
+      if (r != P) return MLA_ERR_INVALID_ARG;
+      for (int j = 0; j < r; ++j) ks[j] = j;
+      break;
+    default:
+      return MLA_ERR_INVALID_ARG;
+  }
+  for (int g = 0; g < nkv; ++g)
+    for (int j = 0; j < r; ++j) pair_idx[(size_t)g * r + j] = ks[j];
+  return MLA_OK;
+}
+
 mla_status_t mla_select_pairs(const mla_config_t* cfg, const void* q_cal, const void* k_cal,
                               int32_t T, int32_t* pair_idx, float* contrib, void* stream) {
   mla_status_t st = validate_config(cfg);

@@ -27,6 +27,9 @@ Pinning status (see tests/test_oracle_pins.py):
   hand-derived codes.
   cache_bytes_per_token — pinned by the pages' printed reduction figures under a
   stated reading of the unstated configuration.
+  fixed_pairs — the pages name the high / low / uniform / full strategies without
+  formulas; the reading is pinned by its frequency meaning (rope_theta ordering),
+  hand-written sets and the full-RoPE case, which reduces to textbook RoPE MHA.
 """
 
 from .mha2mla import *  # noqa: F401,F403

@@ -22,7 +22,7 @@ Readings taken where the pages are silent (each also listed in the design doc):
 import numpy as np
 
 __all__ = [
-    "rope_theta", "rotate", "pair_norms", "pair_scores", "select_pairs", "split_dims",
+    "rope_theta", "rotate", "pair_norms", "pair_scores", "select_pairs", "fixed_pairs", "split_dims",
     "svd_joint", "krope_weights", "convert", "append", "quant_int4_g32", "dequant_int4_g32",
     "pack_int4", "unpack_int4", "decode_unabsorbed", "decode_absorbed", "decode_sequence",
     "mha_textbook_rope", "cache_bytes_per_token", "mha_cache_bytes_per_token",
@@ -100,6 +100,38 @@ def select_pairs(contrib: np.ndarray, r: int) -> np.ndarray:
     return out
 
 
+def fixed_pairs(strategy: str, head_dim: int, r: int, n_kv: int) -> np.ndarray:
+    """The fixed partial-RoPE pair sets the 2-norm selection is compared against.
+
+    README "MHA2MLA" §Fine-Tuning strategy tables (partial-RoPE versions: full-RoPE,
+    S_high, S_uniform, S_2-norm, S_low) and Notes §消融实验 (Partial-RoPE strategy
+    comparison: keep high-frequency / low-frequency / uniformly spaced subspaces).  The
+    pages give no formulas; the reading: with P = d_h/2 pairs and theta_k = base^(-2k/d_h)
+    (pair 0 rotates fastest),
+      'high'    the r highest frequencies, k = 0 .. r-1
+      'low'     the r lowest frequencies,  k = P-r .. P-1
+      'uniform' r pairs evenly spaced from k = 0, k_j = floor(j * P / r)
+      'full'    every pair (r = P)
+    The same set serves every KV head.  Returns [n_kv][r] int64, ascending.
+    """
+    P = head_dim // 2
+    if not 0 <= r <= P:
+        raise ValueError("r out of range")
+    if strategy == "high":
+        ks = list(range(r))
+    elif strategy == "low":
+        ks = list(range(P - r, P))
+    elif strategy == "uniform":
+        ks = [(j * P) // r for j in range(r)]
+    elif strategy == "full":
+        if r != P:
+            raise ValueError("full RoPE keeps every pair")
+        ks = list(range(P))
+    else:
+        raise ValueError(strategy)
+    return np.array([ks] * n_kv, dtype=np.int64).reshape(n_kv, r)
+
+
 def split_dims(pair_idx: np.ndarray, head_dim: int):
     """(rope_dims [n_kv][2r], nope_dims [n_kv][d_h-2r]) for each KV head.
 
@@ -161,14 +193,16 @@ def krope_weights(W_k: np.ndarray, pair_idx: np.ndarray, head_dim: int) -> np.nd
     return np.stack([W_k[:, g * head_dim + rope[g]] for g in range(n_kv)], axis=1)
 
 
-def convert(weights: dict, q_cal: np.ndarray, k_cal: np.ndarray, wl, cast=None) -> dict:
-    """Partial-RoPE (2-norm top-r) followed by SVDjoint (NOTES §方法详解/整体框架).
+def convert(weights: dict, q_cal: np.ndarray, k_cal: np.ndarray, wl, cast=None, pair_idx=None) -> dict:
+    """Partial-RoPE (2-norm top-r, or the given pair set) followed by SVDjoint (NOTES
+    §方法详解/整体框架).
 
     ``cast`` (optional) rounds the deployed matrices to the storage dtype; the
     uncast float64 results are kept under '*_exact'.
     """
     contrib = pair_scores(q_cal, k_cal)
-    pair_idx = select_pairs(contrib, wl.r_pairs)
+    if pair_idx is None:
+        pair_idx = select_pairs(contrib, wl.r_pairs)
     W_dkv, W_uk, W_uv, sigma = svd_joint(weights["W_k"], weights["W_v"], pair_idx, wl.d_c, wl.head_dim)
     W_kr = krope_weights(weights["W_k"], pair_idx, wl.head_dim)
     out = {"contrib": contrib, "pair_idx": pair_idx, "sigma": sigma,

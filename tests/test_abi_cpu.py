@@ -2,6 +2,8 @@
 and rejects bad arguments with the documented status before touching the device."""
 
 import ctypes
+
+import numpy as np
 import os
 import re
 
@@ -93,3 +95,19 @@ def test_append_and_decode_need_a_plan(mla):
     assert mla._lib.mla_plan_set_option(None, 1, 0) == mla.MLA_ERR_INVALID_ARG
     code = ctypes.c_int32()
     assert mla._lib.mla_device_error(None, ctypes.byref(code)) == mla.MLA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("dh,r", [(32, 2), (64, 4), (128, 4), (128, 13)])
+def test_fixed_pairs_match_oracle(mla, dh, r):
+    """mla_fixed_pairs (library, host) equals the oracle's sets bit for bit."""
+    import oracle as O
+    cfg = mla.make_config(512, 8, 4, dh, r, 64)
+    for name, code in (("high", mla.MLA_PAIRS_HIGH), ("low", mla.MLA_PAIRS_LOW),
+                       ("uniform", mla.MLA_PAIRS_UNIFORM)):
+        got = mla.mla_fixed_pairs(cfg, code)
+        assert np.array_equal(got, O.fixed_pairs(name, dh, r, 4).astype(np.int32)), name
+    full_cfg = mla.make_config(512, 8, 4, dh, dh // 2, 64)
+    assert np.array_equal(mla.mla_fixed_pairs(full_cfg, mla.MLA_PAIRS_FULL),
+                          O.fixed_pairs("full", dh, dh // 2, 4).astype(np.int32))
+    assert mla.mla_fixed_pairs(cfg, mla.MLA_PAIRS_FULL, check=False) is None     # r != d_h / 2
+    assert mla.mla_fixed_pairs(cfg, 3, check=False) is None                      # unknown strategy

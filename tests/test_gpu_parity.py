@@ -232,3 +232,21 @@ def test_end_to_end_conversion_append_decode(wl):
     assert mla.mla_device_error(plan) == 0
     for b in case.seqs:
         assert_close(got[b], case.reference(b), wl.dtype, f"end-to-end seq {b}")
+
+
+@pytest.mark.parametrize("wl,pairs", [(PARITY_WORKLOADS[2], "uniform"), (PARITY_WORKLOADS[2], "low"),
+                                      (PARITY_WORKLOADS[1], "high"),
+                                      (PARITY_WORKLOADS[0].with_(name="tiny_full_rope", r_pairs=16), "full")],
+                         ids=["llama_uniform", "llama_low", "smollm_high", "tiny_full"])
+def test_decode_parity_fixed_pair_sets(wl, pairs):
+    """The other partial-RoPE strategies through the same conversion, plan and decode."""
+    case = OracleCase(wl, pairs=pairs)
+    cfg = mla.config_from_workload(wl)
+    fixed = {"high": mla.MLA_PAIRS_HIGH, "low": mla.MLA_PAIRS_LOW, "uniform": mla.MLA_PAIRS_UNIFORM,
+             "full": mla.MLA_PAIRS_FULL}[pairs]
+    assert np.array_equal(mla.mla_fixed_pairs(cfg, fixed), case.conv["pair_idx"].astype(np.int32))
+    plan = mla.mla_plan_create(cfg, **plan_inputs(case))
+    got = run_decode(case, plan, cfg)
+    assert mla.mla_device_error(plan) == 0
+    for b in case.seqs:
+        assert_close(got[b], case.reference(b), wl.dtype, f"{pairs} decode seq {b}")

@@ -310,3 +310,46 @@ def test_generators_are_seeded_and_cast():
     x1 = gen.context_tokens(wl, 1, 80)[:50]
     np.testing.assert_array_equal(x0, x1)
     assert gen.seq_lens(WORKLOADS[3]).min() >= 1024 and gen.seq_lens(WORKLOADS[3]).max() <= 32768
+
+
+# ------------------------------------------------------------------ T10 fixed pair sets
+def test_T10_fixed_pair_sets_hand_written():
+    """README §Fine-Tuning (partial-RoPE versions) / Notes §消融实验: the high, low,
+    uniform and full strategies, written out by hand for small cases."""
+    assert O.fixed_pairs("high", 128, 4, 1).tolist() == [[0, 1, 2, 3]]
+    assert O.fixed_pairs("low", 128, 4, 1).tolist() == [[60, 61, 62, 63]]
+    assert O.fixed_pairs("uniform", 128, 4, 1).tolist() == [[0, 16, 32, 48]]
+    assert O.fixed_pairs("uniform", 12, 4, 1).tolist() == [[0, 1, 3, 4]]   # P = 6: 0, 1.5, 3, 4.5
+    assert O.fixed_pairs("full", 8, 4, 2).tolist() == [[0, 1, 2, 3], [0, 1, 2, 3]]
+    with pytest.raises(ValueError):
+        O.fixed_pairs("full", 8, 3, 1)
+
+
+@pytest.mark.parametrize("dh,r", [(32, 2), (64, 4), (128, 4), (128, 13), (64, 31)])
+def test_T10_fixed_pairs_frequency_meaning(dh, r):
+    """'high' keeps the fastest-rotating pairs, 'low' the slowest (theta_k from rope_theta,
+    pair 0 fastest); 'uniform' starts at pair 0 with steps of floor or ceil of P/r."""
+    theta = O.rope_theta(dh, 10000.0)
+    P = dh // 2
+    for strat, faster in (("high", True), ("low", False)):
+        ks = O.fixed_pairs(strat, dh, r, 1)[0]
+        rest = [k for k in range(P) if k not in set(ks.tolist())]
+        if rest:
+            if faster:
+                assert theta[ks].min() > theta[rest].max()
+            else:
+                assert theta[ks].max() < theta[rest].min()
+    u = O.fixed_pairs("uniform", dh, r, 1)[0]
+    assert u[0] == 0 and len(set(u.tolist())) == r and u.max() < P
+    steps = np.diff(u)
+    assert set(steps.tolist()) <= {P // r, -(-P // r)}
+
+
+def test_T10_full_strategy_is_every_pair_and_rope_mha():
+    """Full RoPE keeps every pair, the same set the 2-norm top-P selection returns; at
+    full latent rank the converted layer then reproduces textbook RoPE MHA (pin T3)."""
+    wl = WORKLOADS[0].with_(name="tiny_full_rope", r_pairs=WORKLOADS[0].head_dim // 2,
+                            d_c=WORKLOADS[0].n_kv_heads * (2 * WORKLOADS[0].head_dim))
+    full = O.fixed_pairs("full", wl.head_dim, wl.r_pairs, wl.n_kv_heads)
+    contrib = np.random.default_rng(7).random((wl.n_kv_heads, wl.head_dim // 2))
+    assert np.array_equal(full, O.select_pairs(contrib, wl.r_pairs))
