@@ -57,13 +57,60 @@ def svd_joint(W_k: torch.Tensor, W_v: torch.Tensor, pair_idx: torch.Tensor, d_c:
     return U, W_uk, W_uv
 
 
+def _truncated_svd(W: torch.Tensor, rank: int):
+    """U[:, :rank] and Sigma V^T[:rank] (float64) with the sign convention of svd_joint; a
+    rank beyond the matrix's own leaves the extra latent dims empty (zeros)."""
+    U, S, Vh = torch.linalg.svd(W, full_matrices=False)
+    k = min(rank, S.shape[0])
+    U, Vh = U[:, :k], Vh[:k]
+    idx = U.abs().argmax(dim=0)
+    sgn = torch.sign(U[idx, torch.arange(k, device=U.device)])
+    sgn[sgn == 0] = 1.0
+    Uk = torch.zeros(W.shape[0], rank, dtype=W.dtype, device=W.device)
+    M = torch.zeros(rank, W.shape[1], dtype=W.dtype, device=W.device)
+    Uk[:, :k] = U * sgn
+    M[:k] = (S[:k, None] * Vh) * sgn[:, None]
+    return Uk, M
+
+
+def svd_split(W_k: torch.Tensor, W_v: torch.Tensor, pair_idx: torch.Tensor, d_c: int, head_dim: int):
+    """SVD_split (README §Fine-Tuning, SVD version 2): separate truncated SVDs of the NoPE
+    key projection and of W_v, d_c/2 latent dims each, in the shared-latent form the cache
+    and the decode use: W_dkv = [U_k | U_v], W_uk rows of the c_v half and W_uv rows of the
+    c_k half are zero."""
+    n_kv = W_v.shape[1] // head_dim
+    r = pair_idx.shape[1]
+    dn = head_dim - 2 * r
+    dk = d_c // 2
+    dv = d_c - dk
+    Wk = W_k.to(torch.float64)
+    pidx = pair_idx.to("cpu").tolist()
+    blocks = []
+    for g in range(n_kv):
+        rope = set()
+        for k in pidx[g]:
+            rope.update((2 * k, 2 * k + 1))
+        blocks.append(Wk[:, [g * head_dim + i for i in range(head_dim) if i not in rope]])
+    U_k, M_k = _truncated_svd(torch.cat(blocks, dim=1), dk)
+    U_v, M_v = _truncated_svd(W_v.to(torch.float64), dv)
+    W_dkv = torch.cat([U_k, U_v], dim=1)
+    W_uk = torch.zeros(n_kv, d_c, dn, dtype=torch.float64, device=W_k.device)
+    W_uv = torch.zeros(n_kv, d_c, head_dim, dtype=torch.float64, device=W_k.device)
+    for g in range(n_kv):
+        W_uk[g, :dk] = M_k[:, g * dn:(g + 1) * dn]
+        W_uv[g, dk:] = M_v[:, g * head_dim:(g + 1) * head_dim]
+    return W_dkv, W_uk, W_uv
+
+
 def convert_layer(cfg: "_lib.MlaConfig", W_k: torch.Tensor, W_v: torch.Tensor,
-                  q_cal: torch.Tensor, k_cal: torch.Tensor) -> dict:
-    """Full conversion; returns host tensors in the storage dtype ready for mla_plan_create."""
+                  q_cal: torch.Tensor, k_cal: torch.Tensor, svd: str = "joint") -> dict:
+    """Full conversion; returns host tensors in the storage dtype ready for mla_plan_create.
+    svd: "joint" (SVDjoint) or "split" (SVD_split)."""
     dtype = "bf16" if cfg.dtype == _lib.MLA_BF16 else "f32"
     tdt = _DT[dtype]
     pair_idx, contrib = select_pairs(cfg, q_cal, k_cal)
-    W_dkv, W_uk, W_uv = svd_joint(W_k, W_v, pair_idx, cfg.d_c, cfg.head_dim)
+    low_rank = svd_split if svd == "split" else svd_joint
+    W_dkv, W_uk, W_uv = low_rank(W_k, W_v, pair_idx, cfg.d_c, cfg.head_dim)
     host = lambda t: t.to(tdt).contiguous().cpu()  # noqa: E731
     return {
         "pair_idx": pair_idx.to(torch.int32).contiguous().cpu(),

@@ -23,7 +23,7 @@ import numpy as np
 
 __all__ = [
     "rope_theta", "rotate", "pair_norms", "pair_scores", "select_pairs", "fixed_pairs", "split_dims",
-    "svd_joint", "krope_weights", "convert", "append", "quant_int4_g32", "dequant_int4_g32",
+    "svd_joint", "svd_split", "krope_weights", "convert", "append", "quant_int4_g32", "dequant_int4_g32",
     "pack_int4", "unpack_int4", "decode_unabsorbed", "decode_absorbed", "decode_sequence",
     "mha_textbook_rope", "cache_bytes_per_token", "mha_cache_bytes_per_token",
 ]
@@ -183,6 +183,55 @@ def svd_joint(W_k: np.ndarray, W_v: np.ndarray, pair_idx: np.ndarray, d_c: int, 
     return U, W_uk, W_uv, s
 
 
+def _truncated_svd(W: np.ndarray, rank: int):
+    """U[:, :rank], Sigma V^T[:rank] with the sign convention of svd_joint, and all sigmas.
+    A rank beyond the matrix's own leaves the extra latent dims empty (zero columns of U
+    and zero rows of Sigma V^T)."""
+    U, s, Vt = np.linalg.svd(W, full_matrices=False)
+    k = min(rank, s.shape[0])
+    Uk = np.zeros((W.shape[0], rank))
+    M = np.zeros((rank, W.shape[1]))
+    Uk[:, :k] = U[:, :k]
+    M[:k] = s[:k, None] * Vt[:k]
+    for i in range(k):
+        j = int(np.argmax(np.abs(Uk[:, i])))
+        if Uk[j, i] < 0:
+            Uk[:, i] *= -1.0
+            M[i] *= -1.0
+    return Uk, M, s
+
+
+def svd_split(W_k: np.ndarray, W_v: np.ndarray, pair_idx: np.ndarray, d_c: int, head_dim: int):
+    """SVDsplit low-rank initialisation: separate truncated SVDs of the NoPE key projection
+    [W_k,nope(g) for all g] and of W_v.
+
+    README "MHA2MLA" §Fine-Tuning strategy tables (SVD version 2, SVD_split); Notes
+    §消融实验 (SVD strategy comparison: SVDsplit and SVDjoint have the same KV cache size).
+    Reading: the d_c cached latent dims are split evenly, c = [c_k | c_v] with c_k = x U_k
+    (d_c/2 dims) and c_v = x U_v (d_c - d_c/2 dims).  In the shared-latent form used by
+    the cache and the decode, W_dkv = [U_k | U_v], W_uk[g] has zero rows for c_v and
+    W_uv[g] zero rows for c_k, so K_nope = c_k (Sigma V^T)_k and V = c_v (Sigma V^T)_v.
+
+    Returns W_dkv [d][d_c], W_uk [n_kv][d_c][d_h-2r], W_uv [n_kv][d_c][d_h],
+    (sigma_k, sigma_v) (all singular values of each part).
+    """
+    n_kv = W_v.shape[1] // head_dim
+    _, nope = split_dims(pair_idx, head_dim)
+    dn = nope.shape[1]
+    dk = d_c // 2
+    dv = d_c - dk
+    Wk_nope = np.concatenate([W_k[:, g * head_dim + nope[g]] for g in range(n_kv)], axis=1)
+    U_k, M_k, s_k = _truncated_svd(Wk_nope, dk)
+    U_v, M_v, s_v = _truncated_svd(W_v, dv)
+    W_dkv = np.concatenate([U_k, U_v], axis=1)
+    W_uk = np.zeros((n_kv, d_c, dn))
+    W_uv = np.zeros((n_kv, d_c, head_dim))
+    for g in range(n_kv):
+        W_uk[g, :dk] = M_k[:, g * dn:(g + 1) * dn]
+        W_uv[g, dk:] = M_v[:, g * head_dim:(g + 1) * head_dim]
+    return W_dkv, W_uk, W_uv, (s_k, s_v)
+
+
 def krope_weights(W_k: np.ndarray, pair_idx: np.ndarray, head_dim: int) -> np.ndarray:
     """W_krope [d][n_kv][2r]: the columns of W_k that keep RoPE (ascending pair order).
 
@@ -193,9 +242,10 @@ def krope_weights(W_k: np.ndarray, pair_idx: np.ndarray, head_dim: int) -> np.nd
     return np.stack([W_k[:, g * head_dim + rope[g]] for g in range(n_kv)], axis=1)
 
 
-def convert(weights: dict, q_cal: np.ndarray, k_cal: np.ndarray, wl, cast=None, pair_idx=None) -> dict:
+def convert(weights: dict, q_cal: np.ndarray, k_cal: np.ndarray, wl, cast=None, pair_idx=None,
+            svd: str = "joint") -> dict:
     """Partial-RoPE (2-norm top-r, or the given pair set) followed by SVDjoint (NOTES
-    §方法详解/整体框架).
+    §方法详解/整体框架), or SVDsplit when svd == "split".
 
     ``cast`` (optional) rounds the deployed matrices to the storage dtype; the
     uncast float64 results are kept under '*_exact'.
@@ -203,7 +253,8 @@ def convert(weights: dict, q_cal: np.ndarray, k_cal: np.ndarray, wl, cast=None, 
     contrib = pair_scores(q_cal, k_cal)
     if pair_idx is None:
         pair_idx = select_pairs(contrib, wl.r_pairs)
-    W_dkv, W_uk, W_uv, sigma = svd_joint(weights["W_k"], weights["W_v"], pair_idx, wl.d_c, wl.head_dim)
+    low_rank = svd_split if svd == "split" else svd_joint
+    W_dkv, W_uk, W_uv, sigma = low_rank(weights["W_k"], weights["W_v"], pair_idx, wl.d_c, wl.head_dim)
     W_kr = krope_weights(weights["W_k"], pair_idx, wl.head_dim)
     out = {"contrib": contrib, "pair_idx": pair_idx, "sigma": sigma,
            "W_dkv_exact": W_dkv, "W_uk_exact": W_uk, "W_uv_exact": W_uv, "W_krope_exact": W_kr}

@@ -66,15 +66,15 @@ def assert_stored_close(got, exact, dtype: str, what: str = ""):
 class OracleCase:
     """Oracle conversion, cache and reference outputs for one workload (float64)."""
 
-    def __init__(self, wl, seqs=None, pairs=None):
+    def __init__(self, wl, seqs=None, pairs=None, svd="joint"):
         """pairs: None for the 2-norm selection, else a fixed strategy name of
-        oracle.fixed_pairs ('high', 'low', 'uniform', 'full')."""
+        oracle.fixed_pairs ('high', 'low', 'uniform', 'full'); svd: 'joint' or 'split'."""
         self.wl = wl
         self.w = gen.layer_weights(wl)
         self.q_cal, self.k_cal = gen.calib_activations(wl, self.w)
         cast = lambda a: gen.cast(a, wl.dtype)  # noqa: E731
         pair_idx = None if pairs is None else O.fixed_pairs(pairs, wl.head_dim, wl.r_pairs, wl.n_kv_heads)
-        self.conv = O.convert(self.w, self.q_cal, self.k_cal, wl, cast=cast, pair_idx=pair_idx)
+        self.conv = O.convert(self.w, self.q_cal, self.k_cal, wl, cast=cast, pair_idx=pair_idx, svd=svd)
         self.theta = O.rope_theta(wl.head_dim, wl.rope_base)
         self.lens = gen.seq_lens(wl)
         self.q = gen.decode_queries(wl, self.w)

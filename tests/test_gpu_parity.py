@@ -250,3 +250,34 @@ def test_decode_parity_fixed_pair_sets(wl, pairs):
     assert mla.mla_device_error(plan) == 0
     for b in case.seqs:
         assert_close(got[b], case.reference(b), wl.dtype, f"{pairs} decode seq {b}")
+
+
+@pytest.mark.parametrize("wl", [PARITY_WORKLOADS[2], PARITY_WORKLOADS[1], PARITY_WORKLOADS[4]],
+                         ids=["llama", "smollm", "int4"])
+def test_svd_split_conversion_append_decode(wl):
+    """SVD_split end to end: the product conversion (device SVDs) gives the oracle's pair set
+    and decodes, after GPU append, to the oracle's SVD_split reference."""
+    case = OracleCase(wl, svd="split")
+    from mha_mla_latent_b200.convert import convert_layer, plan_from_converted
+    cfg = mla.config_from_workload(wl)
+    conv = convert_layer(cfg, gen.to_torch(case.w["W_k"], wl.dtype, "cuda"),
+                         gen.to_torch(case.w["W_v"], wl.dtype, "cuda"),
+                         gen.to_torch(case.q_cal, wl.dtype, "cuda"), gen.to_torch(case.k_cal, wl.dtype, "cuda"),
+                         svd="split")
+    assert conv["pair_idx"].numpy().tolist() == case.conv["pair_idx"].tolist()
+    dk = wl.d_c // 2
+    assert bool((conv["W_uk"][:, dk:] == 0).all()) and bool((conv["W_uv"][:, :dk] == 0).all())
+    plan = plan_from_converted(cfg, conv)
+    T_cap = max(1, int(max(case.lens)))
+    cache = LatentCache(cfg, wl.batch, T_cap, "cuda")
+    for b in case.seqs:
+        x = case.tokens(b)
+        if x.shape[0] == 0:
+            continue
+        mla.mla_append(plan, gen.to_torch(x, wl.dtype, "cuda"),
+                       torch.full((x.shape[0],), b, dtype=torch.int32, device="cuda"),
+                       torch.arange(x.shape[0], dtype=torch.int32, device="cuda"), cache.struct)
+    got = run_decode(case, plan, cfg, cache=cache)
+    assert mla.mla_device_error(plan) == 0
+    for b in case.seqs:
+        assert_close(got[b], case.reference(b), wl.dtype, f"SVD_split seq {b}")

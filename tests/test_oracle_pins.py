@@ -29,7 +29,7 @@ def _rand_layer(rng, d, H, n_kv, dh):
     return W_q, W_k, W_v
 
 
-def _converted_decode(rng, d, H, n_kv, dh, r, d_c, L, absorbed=False, pair_idx=None):
+def _converted_decode(rng, d, H, n_kv, dh, r, d_c, L, absorbed=False, pair_idx=None, svd="joint"):
     """Run the oracle's convert -> append -> decode on random data; also return raw pieces."""
     W_q, W_k, W_v = _rand_layer(rng, d, H, n_kv, dh)
     if pair_idx is None:
@@ -37,7 +37,8 @@ def _converted_decode(rng, d, H, n_kv, dh, r, d_c, L, absorbed=False, pair_idx=N
         k_cal = rng.standard_normal((64, d)) @ W_k
         contrib = O.pair_scores(q_cal.reshape(64, H, dh), k_cal.reshape(64, n_kv, dh))
         pair_idx = O.select_pairs(contrib, r)
-    W_dkv, W_uk, W_uv, _ = O.svd_joint(W_k, W_v, pair_idx, d_c, dh)
+    low_rank = O.svd_split if svd == "split" else O.svd_joint
+    W_dkv, W_uk, W_uv, _ = low_rank(W_k, W_v, pair_idx, d_c, dh)
     W_kr = O.krope_weights(W_k, pair_idx, dh)
     theta = O.rope_theta(dh, 10000.0)
     x = rng.standard_normal((L, d))
@@ -353,3 +354,40 @@ def test_T10_full_strategy_is_every_pair_and_rope_mha():
     full = O.fixed_pairs("full", wl.head_dim, wl.r_pairs, wl.n_kv_heads)
     contrib = np.random.default_rng(7).random((wl.n_kv_heads, wl.head_dim // 2))
     assert np.array_equal(full, O.select_pairs(contrib, wl.r_pairs))
+
+
+# ------------------------------------------------------------------ T4s SVD_split
+def test_T4s_split_eckart_young_per_part_and_zero_blocks():
+    """SVD_split: each half is the truncated SVD of its own matrix (Eckart-Young per part,
+    orthonormal columns per half); the key up-projection reads only c_k and the value
+    up-projection only c_v."""
+    rng = np.random.default_rng(18)
+    d, n_kv, dh, r, d_c = 80, 3, 16, 2, 24
+    _, W_k, W_v = _rand_layer(rng, d, 3, n_kv, dh)
+    pair_idx = np.array([[0, 5], [1, 7], [2, 3]])
+    W_dkv, W_uk, W_uv, (s_k, s_v) = O.svd_split(W_k, W_v, pair_idx, d_c, dh)
+    dk = d_c // 2
+    U_k, U_v = W_dkv[:, :dk], W_dkv[:, dk:]
+    np.testing.assert_allclose(U_k.T @ U_k, np.eye(dk), atol=1e-12)
+    np.testing.assert_allclose(U_v.T @ U_v, np.eye(d_c - dk), atol=1e-12)
+    assert np.all(W_uk[:, dk:] == 0) and np.all(W_uv[:, :dk] == 0)
+    _, nope = O.split_dims(pair_idx, dh)
+    Wk_nope = np.concatenate([W_k[:, g * dh + nope[g]] for g in range(n_kv)], axis=1)
+    rec_k = np.concatenate([W_dkv @ W_uk[g] for g in range(n_kv)], axis=1)
+    rec_v = np.concatenate([W_dkv @ W_uv[g] for g in range(n_kv)], axis=1)
+    np.testing.assert_allclose(np.linalg.norm(Wk_nope - rec_k) ** 2, np.sum(s_k[dk:] ** 2), rtol=1e-9)
+    np.testing.assert_allclose(np.linalg.norm(W_v - rec_v) ** 2, np.sum(s_v[d_c - dk:] ** 2), rtol=1e-9)
+    # at the same total rank the joint SVD of the concatenation loses no more energy
+    _, _, _, s_j = O.svd_joint(W_k, W_v, pair_idx, d_c, dh)
+    assert np.sum(s_k[dk:] ** 2) + np.sum(s_v[d_c - dk:] ** 2) >= np.sum(s_j[d_c:] ** 2) - 1e-9
+
+
+@pytest.mark.parametrize("H,n_kv", [(4, 4), (8, 2)])
+def test_T3s_split_full_rank_matches_masked_rope_mha(H, n_kv):
+    """SVD_split with each half at full rank reproduces MHA with RoPE on the kept pairs."""
+    rng = np.random.default_rng(19)
+    dh, d, L, r = 8, 96, 11, 2
+    d_c = 2 * max(n_kv * (dh - 2 * r), n_kv * dh)
+    o, q, k, v, theta, pair_idx, _ = _converted_decode(rng, d, H, n_kv, dh, r, d_c, L, svd="split")
+    ref = O.mha_textbook_rope(q, k, v, theta, rope_pairs=pair_idx)
+    np.testing.assert_allclose(o, ref, rtol=1e-10, atol=1e-11)
