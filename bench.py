@@ -61,7 +61,8 @@ def wl_config(wl, lens):
             "ctx": wl.ctx if wl.ctx is not None else f"ragged U[{wl.ctx_range[0]},{wl.ctx_range[1]}]",
             "cached_tokens_per_step": int(np.sum(lens)), "hidden": wl.hidden, "heads": wl.n_heads,
             "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "r_pairs": wl.r_pairs, "d_c": wl.d_c,
-            "latent_cache": "int4 g32 + fp16 scales" if wl.cache == "int4_g32" else wl.dtype,
+            "latent_cache": ("int4 g32 + fp16 scales" + (f", {wl.resid}-token bf16 residual window" if wl.resid else "")
+                             if wl.cache == "int4_g32" else wl.dtype),
             "step": "mla_append(B new tokens) + mla_decode(B queries)"}
 
 
@@ -83,6 +84,7 @@ def oracle_decode_sample(wl, n_tokens, rounds, seconds_cap=None):
     kr = gen.cast(kr, wl.dtype)
     if wl.cache == "int4_g32":
         codes, scales = O.quant_int4_g32(c)
+        plain = gen.cast(c, wl.dtype)
     else:
         c = gen.cast(c, wl.dtype)
     q = gen.decode_queries(small, w)[0]
@@ -91,6 +93,8 @@ def oracle_decode_sample(wl, n_tokens, rounds, seconds_cap=None):
     for _ in range(rounds):
         t0 = time.perf_counter()
         cc = O.dequant_int4_g32(codes, scales) if wl.cache == "int4_g32" else c
+        if wl.cache == "int4_g32" and wl.resid:
+            cc = O.residual_window(cc, plain, wl.resid)
         O.decode_unabsorbed(q, cc, kr, conv["W_uk"], conv["W_uv"], conv["pair_idx"], theta)
         times.append(time.perf_counter() - t0)
         if seconds_cap and time.perf_counter() - t_start > seconds_cap:
@@ -265,6 +269,8 @@ def run_ours(args):
     # ---- caches: enough replicas that consecutive steps never hit L2 from the previous one
     per_tok = mla.mla_cache_bytes_per_token(cfg)
     cache_bytes = int(np.sum(lens)) * per_tok
+    if wl.resid:   # + the window's ring rows (dtype) and their position tags
+        cache_bytes += int(np.sum(np.minimum(lens, wl.resid))) * (wl.d_c * 2 + 4)
     n_rep = max(1, -(-2 * L2_BYTES // cache_bytes))
     T_cap = int(lens.max())
     caches = [LatentCache(cfg, B, T_cap, dev) for _ in range(n_rep)]
@@ -286,6 +292,9 @@ def run_ours(args):
             c.c_scales.copy_(caches[0].c_scales)
         if c.k_rope is not None:
             c.k_rope.copy_(caches[0].k_rope)
+        if c.c_resid is not None:
+            c.c_resid.copy_(caches[0].c_resid)
+            c.resid_pos.copy_(caches[0].resid_pos)
     prefill_s = time.perf_counter() - t0
     assert mla.mla_device_error(plan) == 0
 
@@ -314,7 +323,8 @@ def run_ours(args):
         mla.mla_append(plan, xd, seq_idx, pos, c, stream=stream)
         mla.mla_decode(plan, c, seq_lens, q, out, ws, stream=stream)
 
-    launches_per_step = 4   # append, absorb(+schedule), split-K attention, combine(+W_uv)
+    # append, absorb(+schedule), split-K attention, combine(+W_uv); + the ring-slot claim
+    launches_per_step = 4 + (1 if wl.resid else 0)
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()

@@ -63,8 +63,18 @@ typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype_t;
  * scale s = fp16(absmax/7) per group and 4-bit two's-complement codes
  * clamp(round_half_even(c/s), -7, 7) (codes 0 when s == 0), element 2i in the low
  * nibble of byte i; value = code*s.  (Notes §关键设计: 4-bit quantisation stacks on
- * the latent; the group layout is this library's choice.)  RoPE dims stay in dtype. */
-typedef enum { MLA_CACHE_SAME = 0, MLA_CACHE_INT4_G32 = 1 } mla_cache_kind_t;
+ * the latent; the group layout is this library's choice.)  RoPE dims stay in dtype.
+ * MLA_CACHE_INT4_G32_R128 is MLA_CACHE_INT4_G32 plus an unquantised residual window:
+ * each sequence's MLA_RESID_WINDOW most recent tokens are read at full precision.  The
+ * README "MHA2MLA" (§LongBench evaluation: the 4-bit HQQ quantised cache is run with a
+ * residual length of 128) deploys the 4-bit cache this way.  Every token still gets its
+ * int4 row; in addition the latent of token t, in dtype, goes to slot t % 128 of the
+ * sequence's ring c_resid, and resid_pos[slot] records which position the slot holds
+ * (the largest one appended there: it only grows).  Decode reads token t of a sequence
+ * of length L from the ring when t >= L - 128 and resid_pos[t % 128] == t, else from the
+ * int4 row, so with positions appended in order the window is exactly [L-128, L). */
+typedef enum { MLA_CACHE_SAME = 0, MLA_CACHE_INT4_G32 = 1, MLA_CACHE_INT4_G32_R128 = 2 } mla_cache_kind_t;
+#define MLA_RESID_WINDOW 128
 
 typedef struct {
   int32_t hidden;       /* d */
@@ -75,22 +85,28 @@ typedef struct {
   int32_t d_c;          /* latent width, multiple of 4 (of 32 for the int4 cache) */
   double rope_base;     /* RoPE base (10000 for the Llama/SmolLM shapes) */
   int32_t dtype;        /* mla_dtype_t */
-  int32_t cache_kind;   /* mla_cache_kind_t (int4 requires dtype MLA_BF16) */
+  int32_t cache_kind;   /* mla_cache_kind_t (the int4 kinds require dtype MLA_BF16) */
 } mla_config_t;
 
 /* Caller-owned cache, device memory, capacity T_cap tokens per sequence.
- *   c_kv     SAME: [B][T_cap][d_c] dtype;  INT4: [B][T_cap][d_c/2] uint8 codes
- *   c_scales INT4: [B][T_cap][d_c/32] fp16;  SAME: must be NULL
- *   k_rope   [B][ceil(T_cap/32)][n_kv][32][2r] dtype (may be NULL when r == 0): the kept
- *            RoPE key dims in blocks of 32 tokens, KV-head-major inside a block, so the
- *            2r dims of one KV head for 32 consecutive tokens are contiguous; element
- *            (b, t, g, j) sits at ((b*ceil(T_cap/32) + t/32)*n_kv + g)*32*2r + (t%32)*2r + j */
+ *   c_kv      SAME: [B][T_cap][d_c] dtype;  INT4*: [B][T_cap][d_c/2] uint8 codes
+ *   c_scales  INT4*: [B][T_cap][d_c/32] fp16;  SAME: must be NULL
+ *   k_rope    [B][ceil(T_cap/32)][n_kv][32][2r] dtype (may be NULL when r == 0): the kept
+ *             RoPE key dims in blocks of 32 tokens, KV-head-major inside a block, so the
+ *             2r dims of one KV head for 32 consecutive tokens are contiguous; element
+ *             (b, t, g, j) sits at ((b*ceil(T_cap/32) + t/32)*n_kv + g)*32*2r + (t%32)*2r + j
+ *   c_resid   INT4_G32_R128: [B][128][d_c] dtype, the residual ring; otherwise NULL
+ *   resid_pos INT4_G32_R128: [B][128] int32, the position each ring slot holds; set every
+ *             entry to -1 before a sequence's first append (and again when a sequence
+ *             slot is reused for a new sequence); otherwise NULL */
 typedef struct {
   void* c_kv;
   void* c_scales;
   void* k_rope;
   int32_t B;
   int32_t T_cap;
+  void* c_resid;
+  int32_t* resid_pos;
 } mla_cache_t;
 
 typedef struct mla_plan mla_plan_t;   /* opaque, created by mla_plan_create */
@@ -170,7 +186,10 @@ MLA_API mla_status_t mla_plan_set_option(mla_plan_t* plan, int32_t option, int64
  *   x       device [N][d] dtype
  *   seq_idx device [N] int32 in [0, B);  pos device [N] int32 in [0, T_cap)
  * Tokens with an out-of-range seq_idx/pos are skipped and flag the device error word.
- * Distinct tokens must target distinct (seq, pos) slots. */
+ * Distinct tokens must target distinct (seq, pos) slots.  With the residual window
+ * (MLA_CACHE_INT4_G32_R128) one call may carry any number of a sequence's tokens: a first
+ * kernel raises resid_pos[slot] to the largest position of the call that maps to the slot,
+ * and only that token writes the ring row. */
 MLA_API mla_status_t mla_append(const mla_plan_t* plan, const void* x, const int32_t* seq_idx,
                         const int32_t* pos, int32_t N, const mla_cache_t* cache, void* stream);
 

@@ -17,7 +17,8 @@ LIB_PATH = os.environ.get("MLA_B200_LIB", os.path.join(_PKG, "lib", "libmla_b200
 MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_ALIGNMENT = 0, 1, 2, 3
 MLA_ERR_WORKSPACE_TOO_SMALL, MLA_ERR_CUDA, MLA_ERR_DEVICE = 4, 5, 6
 MLA_F32, MLA_BF16 = 0, 1
-MLA_CACHE_SAME, MLA_CACHE_INT4_G32 = 0, 1
+MLA_CACHE_SAME, MLA_CACHE_INT4_G32, MLA_CACHE_INT4_G32_R128 = 0, 1, 2
+MLA_RESID_WINDOW = 128
 MLA_OPT_DECODE_KERNEL, MLA_OPT_DECODE_SPLITS, MLA_OPT_PROFILE_EVENTS, MLA_OPT_OVERLAP_LAUNCH = 1, 2, 3, 4
 MLA_DEVERR_SEQ_LEN, MLA_DEVERR_APPEND_SLOT, MLA_DEVERR_TIMEOUT = 1, 2, 4
 
@@ -41,7 +42,8 @@ class MlaConfig(ctypes.Structure):
 
 class MlaCache(ctypes.Structure):
     _fields_ = [("c_kv", ctypes.c_void_p), ("c_scales", ctypes.c_void_p),
-                ("k_rope", ctypes.c_void_p), ("B", ctypes.c_int32), ("T_cap", ctypes.c_int32)]
+                ("k_rope", ctypes.c_void_p), ("B", ctypes.c_int32), ("T_cap", ctypes.c_int32),
+                ("c_resid", ctypes.c_void_p), ("resid_pos", ctypes.c_void_p)]
 
 
 class MlaError(RuntimeError):
@@ -109,15 +111,24 @@ def _stream(stream):
 
 
 def make_config(hidden, n_heads, n_kv_heads, head_dim, r_pairs, d_c, rope_base=10000.0,
-                dtype="bf16", cache="same") -> MlaConfig:
+                dtype="bf16", cache="same", resid=0) -> MlaConfig:
+    """cache: "same" or "int4_g32"; resid: 0, or MLA_RESID_WINDOW for the int4 cache with
+    the unquantised residual window (MLA_CACHE_INT4_G32_R128)."""
+    if cache == "int4_g32":
+        if resid not in (0, MLA_RESID_WINDOW):
+            raise ValueError(f"residual window {resid}: this library keeps {MLA_RESID_WINDOW} tokens")
+        kind = MLA_CACHE_INT4_G32_R128 if resid else MLA_CACHE_INT4_G32
+    else:
+        if resid:
+            raise ValueError("the residual window needs the int4 cache")
+        kind = MLA_CACHE_SAME
     return MlaConfig(hidden, n_heads, n_kv_heads, head_dim, r_pairs, d_c, float(rope_base),
-                     MLA_BF16 if dtype == "bf16" else MLA_F32,
-                     MLA_CACHE_INT4_G32 if cache == "int4_g32" else MLA_CACHE_SAME)
+                     MLA_BF16 if dtype == "bf16" else MLA_F32, kind)
 
 
 def config_from_workload(wl) -> MlaConfig:
     return make_config(wl.hidden, wl.n_heads, wl.n_kv_heads, wl.head_dim, wl.r_pairs, wl.d_c,
-                       wl.rope_base, wl.dtype, wl.cache)
+                       wl.rope_base, wl.dtype, wl.cache, wl.resid)
 
 
 def mla_version() -> str:
@@ -184,8 +195,9 @@ def mla_plan_set_option(plan: Plan, option: int, value: int):
     _check(_lib.mla_plan_set_option(plan.handle, option, int(value)), "mla_plan_set_option")
 
 
-def cache_struct(c_kv, c_scales, k_rope, B, T_cap) -> MlaCache:
-    return MlaCache(_ptr(c_kv), _ptr(c_scales), _ptr(k_rope), int(B), int(T_cap))
+def cache_struct(c_kv, c_scales, k_rope, B, T_cap, c_resid=None, resid_pos=None) -> MlaCache:
+    return MlaCache(_ptr(c_kv), _ptr(c_scales), _ptr(k_rope), int(B), int(T_cap), _ptr(c_resid),
+                    _ptr(resid_pos))
 
 
 def mla_append(plan: Plan, x, seq_idx, pos, cache: MlaCache, stream=None, check=True):

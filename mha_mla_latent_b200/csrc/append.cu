@@ -42,6 +42,30 @@ struct AppendArgs {
   int vec_ok;               // x rows and W rows allow 16-byte vector loads
 };
 
+// Residual window (MLA_CACHE_INT4_G32_R128): the unquantised latent of token (sq, p), in
+// the config dtype (bf16), goes to ring slot p % 128 when the slot is claimed by p (the
+// claim kernel ran first and left there the largest position of the call for the slot).
+__device__ __forceinline__ void resid_store(const mla_cache_t& c, int sq, int p, int d_c, int col, float v) {
+  if (!c.c_resid) return;
+  const size_t rs = (size_t)sq * MLA_RESID_WINDOW + (p & (MLA_RESID_WINDOW - 1));
+  if (c.resid_pos[rs] == p) ((__nv_bfloat16*)c.c_resid)[rs * d_c + col] = __float2bfloat16_rn(v);
+}
+
+// Claims the residual ring slots of a call's tokens: resid_pos[seq][p % 128] becomes the
+// largest position that maps there (an atomic maximum, so the newest token owns the slot
+// whatever the order of the call's tokens).
+__global__ void __launch_bounds__(256) resid_claim_kernel(const int32_t* __restrict__ seq_idx,
+                                                          const int32_t* __restrict__ pos, int N,
+                                                          mla_cache_t c) {
+  pdl_wait();   // the kernel before may still read the ring
+  pdl_trigger();
+  for (int n = blockIdx.x * blockDim.x + threadIdx.x; n < N; n += gridDim.x * blockDim.x) {
+    const int sq = seq_idx[n], p = pos[n];
+    if (sq < 0 || sq >= c.B || p < 0 || p >= c.T_cap) continue;   // reported by the append
+    atomicMax(c.resid_pos + (size_t)sq * MLA_RESID_WINDOW + (p & (MLA_RESID_WINDOW - 1)), p);
+  }
+}
+
 // Epilogue on a finished [TOK][COLS] tile of x [W_dkv | W_krope] sums held in shared
 // memory: latent columns are stored in the cache encoding, RoPE columns are rotated at
 // the token's position (angle in double) and stored; everything goes to (seq, pos).
@@ -99,6 +123,7 @@ __device__ void append_epilogue(const AppendArgs& a, const float* tile, int tok0
       const uint32_t hi = __shfl_down_sync(0xffffffffu, nib, 1);
       if ((lane & 1) == 0) ((uint8_t*)c.c_kv)[slot * (a.d_c / 2) + col / 2] = (uint8_t)(nib | (hi << 4));
       if (lane == 0) ((__half*)c.c_scales)[slot * (a.d_c / 32) + col / 32] = sh;
+      resid_store(c, sq, p, a.d_c, col, v);
     }
   }
 }
@@ -278,6 +303,7 @@ __device__ __forceinline__ void append_small_finish(const AppendSmallArgs& sa, f
       const uint32_t hi = __shfl_down_sync(0xffffffffu, nib, 1);
       if ((lane & 1) == 0) ((uint8_t*)c.c_kv)[slot * (a.d_c / 2) + (col0 + lane) / 2] = (uint8_t)(nib | (hi << 4));
       if (lane == 0) ((__half*)c.c_scales)[slot * (a.d_c / 32) + col0 / 32] = sh;
+      resid_store(c, sq, p, a.d_c, col0 + lane, v);
     }
   }
 }
@@ -548,7 +574,12 @@ cudaError_t mla_launch_append(const mla_plan& p, const void* x, const int32_t* s
   a.rope_pair = p.rope_pair; a.theta = p.theta; a.err = p.err;
   const size_t eb = cfg.dtype == MLA_BF16 ? 2 : 4;
   a.vec_ok = ((uintptr_t)x % 16 == 0) && ((size_t)cfg.hidden * eb) % 16 == 0 && ((size_t)p.ncols * eb) % 16 == 0;
-  const bool int4 = cfg.cache_kind == MLA_CACHE_INT4_G32;
+  const bool int4 = mla_kind_int4(cfg.cache_kind);
+  if (c.c_resid) {   // residual window: claim the ring slots first
+    const int grid = std::max(1, std::min((N + 255) / 256, 4 * p.num_sms));
+    cudaError_t e = mla_launch_kernel(resid_claim_kernel, dim3(grid), dim3(256), 0, s, p.opt_pdl, seq_idx, pos, N, c);
+    if (e != cudaSuccess) return e;
+  }
   if (N <= kAppMaxSmallTokens && p.app_part && p.app_ticket && cfg.dtype == MLA_BF16 && a.vec_ok) {
     int ks = (cfg.hidden + kAppSplit - 1) / kAppSplit;
     a.kslice = (ks + 127) / 128 * 128;

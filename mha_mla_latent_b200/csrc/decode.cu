@@ -155,6 +155,7 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
 // ------------------------------------------------------------ CUDA-core split-K decode
 struct DecodeArgs {
   mla_cache_t cache;
+  const int32_t* seq_lens;   // read for the residual window only
   int B, H, n_kv, r, d_c, R;
   const float* qlat;
   const float* qrope;
@@ -192,6 +193,8 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(DecodeArgs a) {
     for (int i = tid; i < H * dc; i += 256) s_qlat[i] = a.qlat[(size_t)b * H * dc + i];
     for (int i = tid; i < H * r2; i += 256) s_qrope[i] = a.qrope[(size_t)b * H * r2 + i];
     if (tid < H) { s_m[tid] = -INFINITY; s_l[tid] = 0.f; }
+    // residual window: tokens from lo on may be read unquantised from the ring
+    const int lo = (INT4 && a.cache.c_resid) ? __ldg(a.seq_lens + b) - MLA_RESID_WINDOW : INT_MAX;
     float O[kSimtMaxE];
 #pragma unroll
     for (int e = 0; e < kSimtMaxE; ++e) O[e] = 0.f;
@@ -203,10 +206,16 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(DecodeArgs a) {
         int tt = i / dc, cc = i % dc;
         float v;
         if (INT4) {
-          const uint8_t* codes = (const uint8_t*)a.cache.c_kv + (slot0 + tt) * (dc / 2);
-          const __half* sc = (const __half*)a.cache.c_scales + (slot0 + tt) * (dc / 32);
-          uint32_t byte = codes[cc / 2];
-          v = (float)nib_to_int((cc & 1) ? (byte >> 4) : (byte & 15u)) * __half2float(sc[cc / 32]);
+          const int tp = t + tt;
+          const size_t rs = (size_t)b * MLA_RESID_WINDOW + (tp & (MLA_RESID_WINDOW - 1));
+          if (tp >= lo && a.cache.resid_pos[rs] == tp) {
+            v = __bfloat162float(((const __nv_bfloat16*)a.cache.c_resid)[rs * dc + cc]);
+          } else {
+            const uint8_t* codes = (const uint8_t*)a.cache.c_kv + (slot0 + tt) * (dc / 2);
+            const __half* sc = (const __half*)a.cache.c_scales + (slot0 + tt) * (dc / 32);
+            uint32_t byte = codes[cc / 2];
+            v = (float)nib_to_int((cc & 1) ? (byte >> 4) : (byte & 15u)) * __half2float(sc[cc / 32]);
+          }
         } else {
           v = to_f32(((const T*)a.cache.c_kv)[(slot0 + tt) * dc + cc]);
         }
@@ -491,7 +500,7 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
   // 2. split-K attention over the latent cache
   if (L.kernel == 1) {
     DecodeArgs da;
-    da.cache = c; da.B = B; da.H = H; da.n_kv = cfg.n_kv_heads; da.r = cfg.r_pairs;
+    da.cache = c; da.seq_lens = seq_lens; da.B = B; da.H = H; da.n_kv = cfg.n_kv_heads; da.r = cfg.r_pairs;
     da.d_c = cfg.d_c; da.R = p.R; da.qlat = aa.qlat; da.qrope = aa.qrope;
     da.opart = (float*)(base + L.off_opart); da.mlpart = (float*)(base + L.off_mlpart);
     da.P = L.P;
@@ -507,7 +516,7 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
     if (e != cudaSuccess) return e;
     if ((e = mla_profile_event(p, 1, s)) != cudaSuccess) return e;
   } else {
-    e = mla_launch_decode_tc(p, c, B, sched, base + L.off_qlat, (const float*)(base + L.off_qrope),
+    e = mla_launch_decode_tc(p, c, seq_lens, B, sched, base + L.off_qlat, (const float*)(base + L.off_qrope),
                              (float*)(base + L.off_opart), (float*)(base + L.off_mlpart), L.P, L.G, s);
     if (e != cudaSuccess) return e;
   }
@@ -581,7 +590,7 @@ cudaError_t mla_launch_decode(const mla_plan& p, const mla_cache_t& c, const int
                               const void* q, int B, void* out, void* ws, const DecodeLayout& L,
                               cudaStream_t s) {
   using namespace mla;
-  bool int4 = p.cfg.cache_kind == MLA_CACHE_INT4_G32;
+  bool int4 = mla_kind_int4(p.cfg.cache_kind);
   if (p.cfg.dtype == MLA_BF16)
     return int4 ? launch_decode_t<__nv_bfloat16, true>(p, c, seq_lens, q, B, out, ws, L, s)
                 : launch_decode_t<__nv_bfloat16, false>(p, c, seq_lens, q, B, out, ws, L, s);

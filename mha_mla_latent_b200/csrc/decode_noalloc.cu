@@ -42,7 +42,7 @@ extern "C" mla_status_t mla_decode_noalloc(const mla_plan_t* plan, const mla_cac
                                            void* stream) {
   if (!plan || !cache || !seq_lens || !q || !out || B <= 0) return MLA_ERR_INVALID_ARG;
   const mla_config_t& cfg = plan->cfg;
-  const bool int4 = cfg.cache_kind == MLA_CACHE_INT4_G32;
+  const bool int4 = mla_kind_int4(cfg.cache_kind);
   if (!cache->c_kv || cache->B <= 0 || cache->T_cap <= 0 || B > cache->B) return MLA_ERR_INVALID_ARG;
   if (int4 != (cache->c_scales != nullptr)) return MLA_ERR_INVALID_ARG;
   if (cfg.r_pairs > 0 && !cache->k_rope) return MLA_ERR_INVALID_ARG;

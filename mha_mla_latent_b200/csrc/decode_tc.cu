@@ -54,6 +54,9 @@ struct TcArgs {
   float* mlpart;          // [H][P][2]
   const float* qrope;     // [B][H][2r] rotated, scaled RoPE query part
   const __half* scales;   // int4: [B*T_cap][d_c/32]
+  const int32_t* seq_lens;            // residual window only
+  const __nv_bfloat16* c_resid;       // int4 with the residual window: [B][128][d_c], else null
+  const int32_t* resid_pos;           // [B][128]
   const uint8_t* kr_base;
   uint32_t c_row, kr_row;
   int32_t* err;
@@ -412,8 +415,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
       it.init(&a.sched, w);
       int n = 0;
       bool ok = true;
+      int lo_b = -1, lo = INT_MAX;   // residual window: tokens from lo on may sit in the ring
       while (ok && it.valid()) {
         const int rs = n % a.NRAW, cs = n % a.NC;
+        if (a.c_resid && it.b != lo_b) {   // once per sequence, ahead of the stage wait
+          lo_b = it.b;
+          lo = __ldg(a.seq_lens + it.b) - MLA_RESID_WINDOW;
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_full(rs), (n / a.NRAW) & 1, abort_flag));
         if (ok && n >= a.NC)
           ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag));
@@ -423,7 +431,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
         for (int rr = 0; rr < 2; ++rr) {
           const int tok = tid_dq + 64 * rr;
           uint8_t* C = sbase + a.off_c + cs * c_stage + tok * 128;
-          if (tok < nvalid) {
+          const int tp = it.t + tok;
+          const size_t rslot = (size_t)it.b * MLA_RESID_WINDOW + (tp & (MLA_RESID_WINDOW - 1));
+          if (tok < nvalid && tp >= lo && __ldg(a.resid_pos + rslot) == tp) {
+            const uint4* src = reinterpret_cast<const uint4*>(a.c_resid + rslot * dc);
+            for (int half = 0; half < dc / 64; ++half)
+  #pragma unroll
+              for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4*>(C + half * kBox + ((ch ^ (tok & 7)) * 16)) = __ldg(src + half * 8 + ch);
+          } else if (tok < nvalid) {
             const __half* sc = reinterpret_cast<const __half*>(raw + raw_codes) + tok * (dc / 32);
             for (int half = 0; half < dc / 64; ++half) {
               const uint4 c0 = *reinterpret_cast<const uint4*>(raw + tok * (dc / 2) + half * 32);
@@ -842,24 +858,25 @@ bool mla_tc_capable(const mla_plan& p) {
   if (cfg.dtype != MLA_BF16 || cfg.n_heads != mla::tc::kH) return false;
   if (cfg.d_c % 64 != 0 || cfg.d_c > 256) return false;
   if (p.R == 0 || p.R % 64 != 0 || 2 * cfg.r_pairs != 8) return false;   // 2r = 8 (r = 4) build
-  if (cfg.cache_kind == MLA_CACHE_INT4_G32 && cfg.d_c != 128) return false;
-  const mla::tc::TcLayout L = mla::tc::tc_layout(cfg.d_c, p.R, 2 * cfg.r_pairs, cfg.cache_kind == MLA_CACHE_INT4_G32);
+  if (mla_kind_int4(cfg.cache_kind) && cfg.d_c != 128) return false;
+  const mla::tc::TcLayout L = mla::tc::tc_layout(cfg.d_c, p.R, 2 * cfg.r_pairs, mla_kind_int4(cfg.cache_kind));
   return L.total <= 232448;
 }
 
 // The int4 scale rows are fetched with 1-D bulk copies, which need an even capacity.
 bool mla_tc_supported(const mla_plan& p, const mla_cache_t& c) {
   if (!mla_tc_capable(p)) return false;
-  if (p.cfg.cache_kind == MLA_CACHE_INT4_G32 && c.T_cap % 2 != 0) return false;
+  if (mla_kind_int4(p.cfg.cache_kind) && c.T_cap % 2 != 0) return false;
   return true;
 }
 
-cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, int B, const Sched& sched,
+cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B,
+                                 const Sched& sched,
                                  const void* qlat, const float* qrope, float* opart, float* mlpart, int P, int G,
                                  cudaStream_t s) {
   using namespace mla::tc;
   const mla_config_t& cfg = p.cfg;
-  const bool int4 = cfg.cache_kind == MLA_CACHE_INT4_G32;
+  const bool int4 = mla_kind_int4(cfg.cache_kind);
   const int dc = cfg.d_c, R = p.R;
   CUtensorMap tm_c, tm_q;
   const uint64_t rows = (uint64_t)c.B * c.T_cap;
@@ -878,6 +895,9 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, int B,
   a.B = B; a.H = kH; a.d_c = dc; a.R = R; a.r2 = 2 * cfg.r_pairs; a.T_cap = c.T_cap; a.P = P;
   a.sched = sched; a.opart = opart; a.mlpart = mlpart; a.qrope = qrope;
   a.scales = (const __half*)c.c_scales; a.err = p.err;
+  a.seq_lens = seq_lens;
+  a.c_resid = (const __nv_bfloat16*)c.c_resid;
+  a.resid_pos = c.resid_pos;
   a.kr_base = (const uint8_t*)c.k_rope;
   a.c_row = int4 ? (uint32_t)dc / 2 : (uint32_t)dc * 2;
   a.kr_row = (uint32_t)R * 2;

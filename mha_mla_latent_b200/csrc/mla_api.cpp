@@ -24,8 +24,8 @@ mla_status_t validate_config(const mla_config_t* c) {
   if (c->r_pairs < 0 || 2 * c->r_pairs > c->head_dim) return MLA_ERR_INVALID_ARG;
   if (!(c->rope_base > 1.0)) return MLA_ERR_INVALID_ARG;
   if (c->dtype != MLA_F32 && c->dtype != MLA_BF16) return MLA_ERR_INVALID_ARG;
-  if (c->cache_kind != MLA_CACHE_SAME && c->cache_kind != MLA_CACHE_INT4_G32) return MLA_ERR_INVALID_ARG;
-  if (c->cache_kind == MLA_CACHE_INT4_G32 && (c->dtype != MLA_BF16 || c->d_c % 32 != 0))
+  if (c->cache_kind != MLA_CACHE_SAME && !mla_kind_int4(c->cache_kind)) return MLA_ERR_INVALID_ARG;
+  if (mla_kind_int4(c->cache_kind) && (c->dtype != MLA_BF16 || c->d_c % 32 != 0))
     return MLA_ERR_UNSUPPORTED;
   // limits of the kernels in this build
   if (c->head_dim > 256 || c->d_c > 1024 || c->n_heads > 256) return MLA_ERR_UNSUPPORTED;
@@ -35,12 +35,15 @@ mla_status_t validate_config(const mla_config_t* c) {
 
 mla_status_t validate_cache(const mla_config_t& cfg, const mla_cache_t* c) {
   if (!c || !c->c_kv || c->B <= 0 || c->T_cap <= 0) return MLA_ERR_INVALID_ARG;
-  bool int4 = cfg.cache_kind == MLA_CACHE_INT4_G32;
+  bool int4 = mla_kind_int4(cfg.cache_kind);
   if (int4 && !c->c_scales) return MLA_ERR_INVALID_ARG;
   if (!int4 && c->c_scales) return MLA_ERR_INVALID_ARG;
   if (cfg.r_pairs > 0 && !c->k_rope) return MLA_ERR_INVALID_ARG;
+  const bool resid = cfg.cache_kind == MLA_CACHE_INT4_G32_R128;
+  if (resid != (c->c_resid != nullptr) || resid != (c->resid_pos != nullptr)) return MLA_ERR_INVALID_ARG;
   if (!aligned16(c->c_kv) || (c->c_scales && !aligned16(c->c_scales)) ||
-      (c->k_rope && !aligned16(c->k_rope)))
+      (c->k_rope && !aligned16(c->k_rope)) || (c->c_resid && !aligned16(c->c_resid)) ||
+      (c->resid_pos && !aligned16(c->resid_pos)))
     return MLA_ERR_ALIGNMENT;
   return MLA_OK;
 }
@@ -84,7 +87,7 @@ size_t mla_cache_bytes_per_token(const mla_config_t* cfg) {
   if (validate_config(cfg) == MLA_ERR_INVALID_ARG) return 0;
   size_t eb = elem_bytes(*cfg);
   size_t rope = (size_t)cfg->n_kv_heads * 2 * cfg->r_pairs * eb;
-  if (cfg->cache_kind == MLA_CACHE_INT4_G32) return (size_t)cfg->d_c / 2 + 2 * ((size_t)cfg->d_c / 32) + rope;
+  if (mla_kind_int4(cfg->cache_kind)) return (size_t)cfg->d_c / 2 + 2 * ((size_t)cfg->d_c / 32) + rope;
   return (size_t)cfg->d_c * eb + rope;
 }
 

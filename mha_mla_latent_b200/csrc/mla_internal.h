@@ -15,6 +15,11 @@ inline __host__ __device__ size_t mla_kr_offset(int b, int t, int g, int j, int 
   return (((size_t)b * blocks + (size_t)(t >> 5)) * n_kv + g) * 32u * r2 + (size_t)(t & 31) * r2 + j;
 }
 
+// True for the int4 cache encodings (with or without the residual window).
+inline __host__ __device__ bool mla_kind_int4(int kind) {
+  return kind == MLA_CACHE_INT4_G32 || kind == MLA_CACHE_INT4_G32_R128;
+}
+
 // Largest token count the decode-step append path takes (its scratch is sized for it).
 constexpr int kAppMaxSmallTokens = 128;
 
@@ -102,7 +107,8 @@ struct Sched {
 DecodeLayout mla_decode_layout(const mla_plan& p, int B, int kernel);
 bool mla_tc_supported(const mla_plan& p, const mla_cache_t& c);
 bool mla_tc_capable(const mla_plan& p);   // shape/dtype allow the tensor-core kernel
-cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, int B, const Sched& sched,
+cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B,
+                                 const Sched& sched,
                                  const void* qlat, const float* qrope, float* opart, float* mlpart, int P, int G,
                                  cudaStream_t s);
 Sched mla_sched_view(const DecodeLayout& L, void* ws, int B);

@@ -30,6 +30,11 @@ Pinning status (see tests/test_oracle_pins.py):
   fixed_pairs — the pages name the high / low / uniform / full strategies without
   formulas; the reading is pinned by its frequency meaning (rope_theta ordering),
   hand-written sets and the full-RoPE case, which reduces to textbook RoPE MHA.
+  residual_window — the README gives only the residual length (128) of the quantised
+  cache; the reading (the most recent tokens read unquantised) is pinned by its special
+  cases (no window: the int4 values; a window over the whole sequence: the plain values),
+  by a brute-force ring-with-position-tags model for in-order appends, and by the decodes
+  it reduces to.
 """
 
 from .mha2mla import *  # noqa: F401,F403

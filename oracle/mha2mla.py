@@ -24,7 +24,7 @@ import numpy as np
 __all__ = [
     "rope_theta", "rotate", "pair_norms", "pair_scores", "select_pairs", "fixed_pairs", "split_dims",
     "svd_joint", "svd_split", "krope_weights", "convert", "append", "quant_int4_g32", "dequant_int4_g32",
-    "pack_int4", "unpack_int4", "decode_unabsorbed", "decode_absorbed", "decode_sequence",
+    "pack_int4", "unpack_int4", "residual_window", "decode_unabsorbed", "decode_absorbed", "decode_sequence",
     "mha_textbook_rope", "cache_bytes_per_token", "mha_cache_bytes_per_token",
 ]
 
@@ -333,6 +333,27 @@ def unpack_int4(packed: np.ndarray) -> np.ndarray:
     out = np.empty((packed.shape[0], packed.shape[1] * 2), dtype=np.int8)
     out[:, 0::2] = lo
     out[:, 1::2] = hi
+    return out
+
+
+def residual_window(c_quant: np.ndarray, c_plain: np.ndarray, window: int) -> np.ndarray:
+    """Latent values a decode reads from the int4 cache with an unquantised residual window.
+
+    README "MHA2MLA" (LongBench evaluation of the 4-bit quantised cache) runs the cache with
+    a residual length of 128; the reading taken here: the `window` most recent tokens are
+    read with their unquantised value (as stored, in the cache dtype) and every older token
+    with its int4 value.  Tokens are appended in position order, so for a sequence of L
+    tokens the window is rows [max(0, L - window), L).
+
+    c_quant, c_plain [L][d_c] -> [L][d_c] (float64)
+    """
+    c_quant = np.asarray(c_quant, dtype=np.float64)
+    c_plain = np.asarray(c_plain, dtype=np.float64)
+    assert c_quant.shape == c_plain.shape and window >= 0
+    L = c_quant.shape[0]
+    out = c_quant.copy()
+    lo = max(0, L - window)
+    out[lo:] = c_plain[lo:]
     return out
 
 

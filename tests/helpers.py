@@ -100,7 +100,10 @@ class OracleCase:
         out = {"c_exact": c, "kr_exact": kr, "kr": gen.cast(kr, wl.dtype)}
         if wl.cache == "int4_g32":
             codes, scales = O.quant_int4_g32(c)
-            out.update(codes=codes, scales=scales, c=O.dequant_int4_g32(codes, scales))
+            deq = O.dequant_int4_g32(codes, scales)
+            out.update(codes=codes, scales=scales, c=deq)
+            if wl.resid:   # the most recent tokens are read unquantised, as stored (dtype)
+                out["c"] = O.residual_window(deq, gen.cast(c, wl.dtype), wl.resid)
         else:
             out["c"] = gen.cast(c, wl.dtype)
         return out
@@ -132,6 +135,11 @@ def upload_oracle_cache(case: OracleCase, cache, T_cap):
         if wl.cache == "int4_g32":
             cache.c_kv[b, :L] = torch.from_numpy(O.pack_int4(cc["codes"])).to(cache.c_kv.device)
             cache.c_scales[b, :L] = torch.from_numpy(cc["scales"]).to(cache.c_scales.device)
+            if wl.resid:   # ring slot t % W holds token t for the window's tokens
+                W = cache.c_resid.shape[1]
+                t = np.arange(max(0, L - W), L)
+                cache.c_resid[b, t % W] = gen.to_torch(cc["c_exact"][t], wl.dtype, cache.c_resid.device)
+                cache.resid_pos[b, t % W] = torch.from_numpy(t.astype(np.int32)).to(cache.resid_pos.device)
         else:
             cache.c_kv[b, :L] = gen.to_torch(cc["c"], wl.dtype, cache.c_kv.device)
         if cache.k_rope is not None:

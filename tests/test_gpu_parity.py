@@ -104,9 +104,11 @@ def test_append_parity(wl):
             codes = O.unpack_int4(cache.c_kv[b, :L].cpu().numpy())
             scales = cache.c_scales[b, :L].cpu().numpy()
             deq = O.dequant_int4_g32(codes, scales)
-            assert_close(deq, cc["c"], wl.dtype, f"int4 latent seq {b}")
+            assert_close(deq, O.dequant_int4_g32(cc["codes"], cc["scales"]), wl.dtype, f"int4 latent seq {b}")
             # codes differ only where the float32 latents straddle a rounding boundary
             assert np.mean(codes != cc["codes"]) < 1e-3
+            if wl.resid:
+                _check_ring(cache, b, L, cc["c_exact"], wl)
         else:
             c = cache.c_kv[b, :L].double().cpu().numpy()
             assert_stored_close(c, cc["c_exact"], wl.dtype, f"latent seq {b}")
@@ -133,9 +135,70 @@ def test_append_decode_step_batch(wl):
         if wl.cache == "int4_g32":
             codes = O.unpack_int4(cache.c_kv[b, p_:p_ + 1].cpu().numpy())
             deq = O.dequant_int4_g32(codes, cache.c_scales[b, p_:p_ + 1].cpu().numpy())
-            assert_close(deq[0], cc["c"][p_], wl.dtype, f"int4 latent {b}")
+            assert_close(deq[0], O.dequant_int4_g32(cc["codes"][p_:p_ + 1], cc["scales"][p_:p_ + 1])[0],
+                         wl.dtype, f"int4 latent {b}")
+            if wl.resid:   # only the appended token's slot is claimed and written
+                W = cache.resid_pos.shape[1]
+                tags = cache.resid_pos[b].cpu().numpy()
+                assert tags[p_ % W] == p_ and np.sum(tags >= 0) == 1
+                assert_stored_close(cache.c_resid[b, p_ % W].double().cpu().numpy(), cc["c_exact"][p_],
+                                    wl.dtype, f"ring {b}")
         else:
             assert_stored_close(cache.c_kv[b, p_].double().cpu().numpy(), cc["c_exact"][p_], wl.dtype, f"c {b}")
+
+
+def _check_ring(cache, b, L, c_exact, wl):
+    """The ring after in-order appends of tokens [0, L): slot t % W holds token t for the
+    W most recent tokens (tag t, row = the unquantised latent in the cache dtype); slots
+    never written keep tag -1."""
+    W = cache.resid_pos.shape[1]
+    tags = cache.resid_pos[b].cpu().numpy()
+    t = np.arange(max(0, L - W), L)
+    np.testing.assert_array_equal(tags[t % W], t)
+    if L < W:
+        assert np.all(tags[L:] == -1)
+    rows = cache.c_resid[b, t % W].double().cpu().numpy()
+    assert_stored_close(rows, c_exact[t], wl.dtype, f"ring rows seq {b}")
+
+
+RESID_WORKLOADS = [w for w in PARITY_WORKLOADS if w.resid]
+
+
+@pytest.mark.parametrize("wl", RESID_WORKLOADS, ids=[w.name for w in RESID_WORKLOADS])
+def test_residual_window_slides_with_decode_steps(wl):
+    """Prefill in one call (positions wrap the ring several times: the newest token of
+    each slot must win), then one-token decode steps; after each, the decode reads the
+    128 most recent tokens unquantised and the rest as int4, as the oracle does."""
+    case = case_for(wl)
+    cfg, plan = make_plan(case)
+    b = int(np.argmax(case.lens))
+    x = case.tokens(b)
+    L_end = x.shape[0]
+    L0 = L_end - 80
+    cache = LatentCache(cfg, 1, L_end, "cuda")
+    mla.mla_append(plan, gen.to_torch(x[:L0], wl.dtype, "cuda"), torch.zeros(L0, dtype=torch.int32, device="cuda"),
+                   torch.arange(L0, dtype=torch.int32, device="cuda"), cache.struct)
+    cc = case.cache[b]
+    _check_ring(cache, 0, L0, cc["c_exact"], wl)
+    deq = O.dequant_int4_g32(cc["codes"], cc["scales"])
+    plain = gen.cast(cc["c_exact"], wl.dtype)
+    q = gen.to_torch(case.q[b:b + 1], wl.dtype, "cuda")
+    out = torch.empty_like(q)
+    ws = workspace(plan, 1, "cuda")
+    checks = {L0 + 1, L_end - 59, L_end - 58, L_end}
+    for L in range(L0 + 1, L_end + 1):
+        mla.mla_append(plan, gen.to_torch(x[L - 1:L], wl.dtype, "cuda"), torch.zeros(1, dtype=torch.int32, device="cuda"),
+                       torch.full((1,), L - 1, dtype=torch.int32, device="cuda"), cache.struct)
+        if L not in checks:
+            continue
+        mla.mla_decode(plan, cache.struct, torch.tensor([L], dtype=torch.int32, device="cuda"), q, out, ws)
+        torch.cuda.synchronize()
+        c_mix = O.residual_window(deq[:L], plain[:L], wl.resid)
+        ref = O.decode_unabsorbed(case.q[b], c_mix, cc["kr"][:L], case.conv["W_uk"], case.conv["W_uv"],
+                                  case.conv["pair_idx"], case.theta)
+        assert_close(out[0].double().cpu().numpy(), ref, wl.dtype, f"{wl.name} L={L}")
+    assert mla.mla_device_error(plan) == 0
+    _check_ring(cache, 0, L_end, cc["c_exact"], wl)
 
 
 def test_append_int4_codes_bit_exact_on_exact_latents():

@@ -391,3 +391,56 @@ def test_T3s_split_full_rank_matches_masked_rope_mha(H, n_kv):
     o, q, k, v, theta, pair_idx, _ = _converted_decode(rng, d, H, n_kv, dh, r, d_c, L, svd="split")
     ref = O.mha_textbook_rope(q, k, v, theta, rope_pairs=pair_idx)
     np.testing.assert_allclose(o, ref, rtol=1e-10, atol=1e-11)
+
+
+# ------------------------------------------------------------------ T11 residual window
+def test_T11_residual_window_special_cases_and_rows():
+    rng = np.random.default_rng(23)
+    L, dc = 5, 64
+    c = rng.standard_normal((L, dc))
+    codes, scales = O.quant_int4_g32(c)
+    deq = O.dequant_int4_g32(codes, scales)
+    plain = gen.cast(c, "bf16")
+    np.testing.assert_array_equal(O.residual_window(deq, plain, 0), deq)        # no window: int4 only
+    np.testing.assert_array_equal(O.residual_window(deq, plain, L), plain)      # window covers all
+    np.testing.assert_array_equal(O.residual_window(deq, plain, 128), plain)
+    got = O.residual_window(deq, plain, 2)                                       # rows 3, 4 are recent
+    for t, src in enumerate([deq, deq, deq, plain, plain]):
+        np.testing.assert_array_equal(got[t], src[t])
+
+
+def test_T11_ring_with_position_tags_selects_the_window():
+    """A ring of W slots (slot t % W, each slot keeping the largest position written to it,
+    whatever the order inside one append call), read for t >= L - W when the slot's tag is
+    t, selects exactly the rows residual_window takes from the unquantised values."""
+    rng = np.random.default_rng(29)
+    W = 8
+    for trial in range(200):
+        L = int(rng.integers(0, 40))
+        tags = np.full(W, -1)
+        done = 0
+        while done < L:          # in-order calls of random size; tokens of a call in random order
+            n = int(rng.integers(1, 20))
+            call = rng.permutation(np.arange(done, min(L, done + n)))
+            for t in call:
+                tags[t % W] = max(tags[t % W], t)
+            done = min(L, done + n)
+        from_ring = np.array([t >= L - W and tags[t % W] == t for t in range(L)], dtype=bool)
+        quant = np.zeros((L, 1))
+        plain = np.ones((L, 1))
+        sel = O.residual_window(quant, plain, W)[:, 0] == 1
+        np.testing.assert_array_equal(from_ring, sel)
+
+
+def test_T11_decode_over_window_reduces_to_pinned_decodes():
+    """Window >= L: the decode over the plain (bf16) latents; window 0: over the int4 values."""
+    rng = np.random.default_rng(31)
+    o, q, k, v, theta, pair_idx, (c, kr, W_uk, W_uv) = _converted_decode(rng, 64, 4, 2, 16, 2, 32, 40)
+    codes, scales = O.quant_int4_g32(c)
+    deq = O.dequant_int4_g32(codes, scales)
+    plain = gen.cast(c, "bf16")
+    dec = lambda cc: O.decode_unabsorbed(q, cc, kr, W_uk, W_uv, pair_idx, theta)  # noqa: E731
+    np.testing.assert_array_equal(dec(O.residual_window(deq, plain, 40)), dec(plain))
+    np.testing.assert_array_equal(dec(O.residual_window(deq, plain, 0)), dec(deq))
+    mixed = dec(O.residual_window(deq, plain, 16))
+    assert not np.array_equal(mixed, dec(deq)) and not np.array_equal(mixed, dec(plain))

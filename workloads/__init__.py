@@ -7,5 +7,5 @@ scoring, no SVD, no RoPE, no attention), so that the CPU oracle and the CUDA
 path can both draw their inputs from it without sharing any computation.
 """
 
-from .configs import WORKLOADS, PARITY_WORKLOADS, Workload, get  # noqa: F401
+from .configs import WORKLOADS, PARITY_WORKLOADS, EXTRA_WORKLOADS, Workload, get  # noqa: F401
 from . import generate  # noqa: F401

@@ -34,6 +34,7 @@ class Workload:
     rope_base: float = 10000.0
     seed: int = 0
     fixed_lens: Optional[Tuple[int, ...]] = field(default=None)  # explicit lengths (parity cases)
+    resid: int = 0             # int4 cache: unquantised residual window of the most recent tokens (0 or 128)
 
     @property
     def group(self) -> int:
@@ -78,13 +79,27 @@ PARITY_WORKLOADS = [
                        ctx_range=None, fixed_lens=(2500, 129, 64, 1), t_cal=512),
     WORKLOADS[4].with_(name="llama_int4_small", hidden=512, batch=3, ctx=None,
                        fixed_lens=(700, 65, 1), t_cal=512),
+    # the int4 cache with the 128-token residual window: on the tensor-core kernel (window
+    # across a tile boundary, a window covering the whole sequence, a single token) and on
+    # the CUDA-core kernel (9 heads)
+    WORKLOADS[4].with_(name="llama_int4_r128_small", hidden=512, batch=4, ctx=None,
+                       fixed_lens=(700, 200, 128, 1), t_cal=512, resid=128),
+    WORKLOADS[1].with_(name="smollm_int4_r128_small", cache="int4_g32", batch=3, ctx=None,
+                       fixed_lens=(300, 129, 5), t_cal=512, resid=128),
+]
+
+# The int4 workload as the pages deploy the 4-bit cache: with a residual window of the 128
+# most recent tokens kept unquantised (README "MHA2MLA", LongBench evaluation of the
+# quantised cache).
+EXTRA_WORKLOADS = [
+    WORKLOADS[4].with_(name="llama2_7b_int4_r128", resid=128),
 ]
 
 
 def get(name_or_index) -> Workload:
     if isinstance(name_or_index, int):
         return WORKLOADS[name_or_index]
-    for w in WORKLOADS + PARITY_WORKLOADS:
+    for w in WORKLOADS + PARITY_WORKLOADS + EXTRA_WORKLOADS:
         if w.name == name_or_index:
             return w
     raise KeyError(name_or_index)
