@@ -89,6 +89,15 @@ typedef struct {
 } mla_config_t;
 
 /* Caller-owned cache, device memory, capacity T_cap tokens per sequence.
+ * Contiguous (block_table == NULL): each sequence owns T_cap token rows, in the arrays below.
+ * Paged (block_table != NULL): the arrays are pools of n_blocks blocks of MLA_BLOCK_TOKENS
+ * (128) tokens, and token t of sequence b lives in token row t % 128 of pool block
+ * block_table[b][t / 128]; every array below is then read with B := n_blocks and
+ * T_cap := 128 (so k_rope holds 4 blocks of 32 tokens per pool block).  T_cap must be a
+ * multiple of 128 (the logical capacity: T_cap / 128 table entries per sequence).  The
+ * README "MHA2MLA" runs ragged LongBench batches; 128-token blocks match the decode tile,
+ * so each tile of the attention kernel reads one block.  A table entry outside
+ * [0, n_blocks) flags MLA_DEVERR_BLOCK and reads or writes block 0 instead.
  *   c_kv      SAME: [B][T_cap][d_c] dtype;  INT4*: [B][T_cap][d_c/2] uint8 codes
  *   c_scales  INT4*: [B][T_cap][d_c/32] fp16;  SAME: must be NULL
  *   k_rope    [B][ceil(T_cap/32)][n_kv][32][2r] dtype (may be NULL when r == 0): the kept
@@ -107,7 +116,10 @@ typedef struct {
   int32_t T_cap;
   void* c_resid;
   int32_t* resid_pos;
+  const int32_t* block_table;   /* paged: device [B][T_cap/128] int32 pool block ids; else NULL */
+  int32_t n_blocks;             /* paged: blocks in the pool; else 0 */
 } mla_cache_t;
+#define MLA_BLOCK_TOKENS 128
 
 typedef struct mla_plan mla_plan_t;   /* opaque, created by mla_plan_create */
 
@@ -243,7 +255,8 @@ MLA_API mla_status_t mla_decode_noalloc(const mla_plan_t* plan, const mla_cache_
 enum {
   MLA_DEVERR_SEQ_LEN = 1,     /* a seq_lens entry was < 0 or > T_cap (treated as 0) */
   MLA_DEVERR_APPEND_SLOT = 2, /* an append token had seq_idx/pos out of range (skipped) */
-  MLA_DEVERR_TIMEOUT = 4      /* a pipeline wait exceeded its bound (output invalid) */
+  MLA_DEVERR_TIMEOUT = 4,     /* a pipeline wait exceeded its bound (output invalid) */
+  MLA_DEVERR_BLOCK = 8        /* a paged cache's block table named a block outside the pool */
 };
 MLA_API mla_status_t mla_device_error(mla_plan_t* plan, int32_t* code);
 

@@ -20,7 +20,8 @@ MLA_F32, MLA_BF16 = 0, 1
 MLA_CACHE_SAME, MLA_CACHE_INT4_G32, MLA_CACHE_INT4_G32_R128 = 0, 1, 2
 MLA_RESID_WINDOW = 128
 MLA_OPT_DECODE_KERNEL, MLA_OPT_DECODE_SPLITS, MLA_OPT_PROFILE_EVENTS, MLA_OPT_OVERLAP_LAUNCH = 1, 2, 3, 4
-MLA_DEVERR_SEQ_LEN, MLA_DEVERR_APPEND_SLOT, MLA_DEVERR_TIMEOUT = 1, 2, 4
+MLA_DEVERR_SEQ_LEN, MLA_DEVERR_APPEND_SLOT, MLA_DEVERR_TIMEOUT, MLA_DEVERR_BLOCK = 1, 2, 4, 8
+MLA_BLOCK_TOKENS = 128
 
 EXPORTED = (
     "mla_status_string", "mla_version", "mla_cache_bytes_per_token", "mla_select_pairs",
@@ -43,7 +44,8 @@ class MlaConfig(ctypes.Structure):
 class MlaCache(ctypes.Structure):
     _fields_ = [("c_kv", ctypes.c_void_p), ("c_scales", ctypes.c_void_p),
                 ("k_rope", ctypes.c_void_p), ("B", ctypes.c_int32), ("T_cap", ctypes.c_int32),
-                ("c_resid", ctypes.c_void_p), ("resid_pos", ctypes.c_void_p)]
+                ("c_resid", ctypes.c_void_p), ("resid_pos", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p), ("n_blocks", ctypes.c_int32)]
 
 
 class MlaError(RuntimeError):
@@ -195,9 +197,10 @@ def mla_plan_set_option(plan: Plan, option: int, value: int):
     _check(_lib.mla_plan_set_option(plan.handle, option, int(value)), "mla_plan_set_option")
 
 
-def cache_struct(c_kv, c_scales, k_rope, B, T_cap, c_resid=None, resid_pos=None) -> MlaCache:
+def cache_struct(c_kv, c_scales, k_rope, B, T_cap, c_resid=None, resid_pos=None, block_table=None,
+                 n_blocks=0) -> MlaCache:
     return MlaCache(_ptr(c_kv), _ptr(c_scales), _ptr(k_rope), int(B), int(T_cap), _ptr(c_resid),
-                    _ptr(resid_pos))
+                    _ptr(resid_pos), _ptr(block_table), int(n_blocks))
 
 
 def mla_append(plan: Plan, x, seq_idx, pos, cache: MlaCache, stream=None, check=True):

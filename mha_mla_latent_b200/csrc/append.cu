@@ -82,7 +82,8 @@ __device__ void append_epilogue(const AppendArgs& a, const float* tile, int tok0
       if (col == 0) raise_error(a.err, MLA_DEVERR_APPEND_SLOT);
       continue;
     }
-    const size_t slot = (size_t)sq * c.T_cap + p;
+    const MlaLoc lc = mla_loc(c, sq, p, a.err);
+    const size_t slot = (size_t)lc.pb * lc.cap + lc.pt;
     const float v0 = tile[t * COLS + 2 * cp], v1 = tile[t * COLS + 2 * cp + 1];
     if (col < a.d_c) {
       if (!INT4) {
@@ -96,7 +97,7 @@ __device__ void append_epilogue(const AppendArgs& a, const float* tile, int tok0
       const int kpair = a.rope_pair[g * a.r + j];
       double sn, cs;
       sincos((double)p * a.theta[kpair], &sn, &cs);
-      T* dst = (T*)c.k_rope + mla_kr_offset(sq, p, g, rc % (2 * a.r), c.T_cap, a.R / (2 * a.r), 2 * a.r);
+      T* dst = (T*)c.k_rope + mla_kr_offset(lc.pb, lc.pt, g, rc % (2 * a.r), lc.cap, a.R / (2 * a.r), 2 * a.r);
       dst[0] = from_f64<T>((double)v0 * cs - (double)v1 * sn);
       dst[1] = from_f64<T>((double)v0 * sn + (double)v1 * cs);
     }
@@ -110,7 +111,8 @@ __device__ void append_epilogue(const AppendArgs& a, const float* tile, int tok0
       if (n >= a.N || col0 + gi * 32 >= a.d_c) continue;   // whole group outside the latent
       const int sq = a.seq_idx[n], p = a.pos[n];
       if (sq < 0 || sq >= c.B || p < 0 || p >= c.T_cap) continue;
-      const size_t slot = (size_t)sq * c.T_cap + p;
+      const MlaLoc lc = mla_loc(c, sq, p, a.err);
+      const size_t slot = (size_t)lc.pb * lc.cap + lc.pt;
       const float v = tile[t * COLS + gi * 32 + lane];
       float am = fabsf(v);
 #pragma unroll
@@ -269,9 +271,10 @@ __device__ __forceinline__ void append_small_finish(const AppendSmallArgs& sa, f
       continue;
     }
     const float v0 = tileb[t * kSmCols + 2 * cp], v1 = tileb[t * kSmCols + 2 * cp + 1];
+    const MlaLoc lc = mla_loc(c, sq, p, a.err);
     if (col < a.d_c) {
       if (!INT4) {
-        T* dst = (T*)c.c_kv + ((size_t)sq * c.T_cap + p) * a.d_c + col;
+        T* dst = (T*)c.c_kv + ((size_t)lc.pb * lc.cap + lc.pt) * a.d_c + col;
         dst[0] = from_f32<T>(v0);
         dst[1] = from_f32<T>(v1);
       }
@@ -279,7 +282,7 @@ __device__ __forceinline__ void append_small_finish(const AppendSmallArgs& sa, f
       const int rc = col - a.d_c;
       double sn, cs;
       sincos((double)p * s_theta[cp], &sn, &cs);
-      T* dst = (T*)c.k_rope + mla_kr_offset(sq, p, rc / (2 * a.r), rc % (2 * a.r), c.T_cap, n_kv, 2 * a.r);
+      T* dst = (T*)c.k_rope + mla_kr_offset(lc.pb, lc.pt, rc / (2 * a.r), rc % (2 * a.r), lc.cap, n_kv, 2 * a.r);
       dst[0] = from_f64<T>((double)v0 * cs - (double)v1 * sn);
       dst[1] = from_f64<T>((double)v0 * sn + (double)v1 * cs);
     }
@@ -290,7 +293,8 @@ __device__ __forceinline__ void append_small_finish(const AppendSmallArgs& sa, f
       const int n = tok0 + t;
       const int sq = s_sq[t], p = s_pos[t];
       if (n >= a.N || sq < 0 || sq >= c.B || p < 0 || p >= c.T_cap) continue;
-      const size_t slot = (size_t)sq * c.T_cap + p;
+      const MlaLoc lc = mla_loc(c, sq, p, a.err);
+      const size_t slot = (size_t)lc.pb * lc.cap + lc.pt;
       const float v = tileb[t * kSmCols + lane];
       float am = fabsf(v);
 #pragma unroll

@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
 struct DecodeArgs {
   mla_cache_t cache;
   const int32_t* seq_lens;   // read for the residual window only
+  int32_t* err;
   int B, H, n_kv, r, d_c, R;
   const float* qlat;
   const float* qrope;
@@ -201,7 +202,8 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(DecodeArgs a) {
     __syncthreads();
     for (int t = t0; t < t1; t += kSimtTile) {
       const int n = min(kSimtTile, t1 - t);
-      const size_t slot0 = (size_t)b * a.cache.T_cap + t;
+      const MlaLoc lc = mla_loc(a.cache, b, t, a.err);   // a 32-token tile lies in one block
+      const size_t slot0 = (size_t)lc.pb * lc.cap + lc.pt;
       for (int i = tid; i < n * dc; i += 256) {
         int tt = i / dc, cc = i % dc;
         float v;
@@ -224,7 +226,7 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(DecodeArgs a) {
       for (int i = tid; i < n * R; i += 256) {
         int tt = i / R, j = i % R;
         s_kr[tt * (R + 1) + j] =
-            to_f32(((const T*)a.cache.k_rope)[mla_kr_offset(b, t + tt, j / r2, j % r2, a.cache.T_cap, a.n_kv, r2)]);
+            to_f32(((const T*)a.cache.k_rope)[mla_kr_offset(lc.pb, lc.pt + tt, j / r2, j % r2, lc.cap, a.n_kv, r2)]);
       }
       __syncthreads();
       for (int i = tid; i < n * H; i += 256) {
@@ -500,7 +502,7 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
   // 2. split-K attention over the latent cache
   if (L.kernel == 1) {
     DecodeArgs da;
-    da.cache = c; da.seq_lens = seq_lens; da.B = B; da.H = H; da.n_kv = cfg.n_kv_heads; da.r = cfg.r_pairs;
+    da.cache = c; da.seq_lens = seq_lens; da.err = p.err; da.B = B; da.H = H; da.n_kv = cfg.n_kv_heads; da.r = cfg.r_pairs;
     da.d_c = cfg.d_c; da.R = p.R; da.qlat = aa.qlat; da.qrope = aa.qrope;
     da.opart = (float*)(base + L.off_opart); da.mlpart = (float*)(base + L.off_mlpart);
     da.P = L.P;

@@ -55,6 +55,7 @@ struct TcArgs {
   const float* qrope;     // [B][H][2r] rotated, scaled RoPE query part
   const __half* scales;   // int4: [B*T_cap][d_c/32]
   const int32_t* seq_lens;            // residual window only
+  mla_cache_t cache;                  // block table (paged cache) and geometry
   const __nv_bfloat16* c_resid;       // int4 with the residual window: [B][128][d_c], else null
   const int32_t* resid_pos;           // [B][128]
   const uint8_t* kr_base;
@@ -191,7 +192,17 @@ __device__ __forceinline__ int trace_slot() {   // CTAs 0, 1 and two that stradd
 #define MLA_TRACE(ev, n) do { } while (0)
 #endif
 
-template <bool INT4, int R2>
+// Storage location of (b, t): compile-time contiguous, or through the paged block table.
+template <bool PAGED>
+__device__ __forceinline__ MlaLoc tc_loc(const TcArgs& a, int b, int t) {
+  if (!PAGED) return MlaLoc{b, t, a.T_cap};
+  return mla_loc(a.cache, b, t, a.err);
+}
+
+// INT4: int4 latent cache (dequantised in shared memory); RESID: with the residual window
+// ring (INT4 only); PAGED: cache addressed through a block table.  Each combination is its
+// own instantiation, so the common ones carry no code of the others.
+template <bool INT4, bool RESID, bool PAGED, int R2>
 __global__ void __launch_bounds__(384, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
                  const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ TcArgs a) {
@@ -279,7 +290,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
               tma_load_2d(qbox(kb), &tm_q, bars.q_full(), kb * 64, it.b * a.H);
             ++q_loads;
           }
-          const int row = it.b * a.T_cap + it.t;
+          const MlaLoc lc = tc_loc<PAGED>(a, it.b, it.t);   // a tile is one paged block
+          const int row = lc.pb * lc.cap + lc.pt;
           MLA_TRACE(0, n);
           if (!INT4) {
             const int cs = n % a.NC;
@@ -418,7 +430,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
       int lo_b = -1, lo = INT_MAX;   // residual window: tokens from lo on may sit in the ring
       while (ok && it.valid()) {
         const int rs = n % a.NRAW, cs = n % a.NC;
-        if (a.c_resid && it.b != lo_b) {   // once per sequence, ahead of the stage wait
+        if (RESID && it.b != lo_b) {   // once per sequence, ahead of the stage wait
           lo_b = it.b;
           lo = __ldg(a.seq_lens + it.b) - MLA_RESID_WINDOW;
         }
@@ -433,7 +445,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
           uint8_t* C = sbase + a.off_c + cs * c_stage + tok * 128;
           const int tp = it.t + tok;
           const size_t rslot = (size_t)it.b * MLA_RESID_WINDOW + (tp & (MLA_RESID_WINDOW - 1));
-          if (tok < nvalid && tp >= lo && __ldg(a.resid_pos + rslot) == tp) {
+          if (RESID && tok < nvalid && tp >= lo && __ldg(a.resid_pos + rslot) == tp) {
             const uint4* src = reinterpret_cast<const uint4*>(a.c_resid + rslot * dc);
             for (int half = 0; half < dc / 64; ++half)
   #pragma unroll
@@ -511,7 +523,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
     auto issue_kr = [&](const TileIter& ti) {   // one thread
       if (!ti.valid()) return;
       const int nblk = min(4, (ti.t1 - ti.t + 31) / 32);
-      const uint8_t* src = a.kr_base + mla_kr_offset(ti.b, ti.t, 0, 0, a.T_cap, n_kv, R2) * 2;
+      const MlaLoc lc = tc_loc<PAGED>(a, ti.b, ti.t);
+      const uint8_t* src = a.kr_base + mla_kr_offset(lc.pb, lc.pt, 0, 0, lc.cap, n_kv, R2) * 2;
       fence_proxy_async_smem();
       mbar_expect_tx(bars.kr_full(), nblk * kr_blk);
       for (int k = 0; k < nblk; ++k)   // one copy per 32-token block: they proceed in parallel
@@ -879,7 +892,7 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
   const bool int4 = mla_kind_int4(cfg.cache_kind);
   const int dc = cfg.d_c, R = p.R;
   CUtensorMap tm_c, tm_q;
-  const uint64_t rows = (uint64_t)c.B * c.T_cap;
+  const uint64_t rows = mla_cache_rows(c);
   bool ok = true;
   if (int4)
     ok &= make_map_2d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.c_kv, dc / 2, rows, dc / 2, dc / 2, kTile,
@@ -896,6 +909,7 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
   a.sched = sched; a.opart = opart; a.mlpart = mlpart; a.qrope = qrope;
   a.scales = (const __half*)c.c_scales; a.err = p.err;
   a.seq_lens = seq_lens;
+  a.cache = c;
   a.c_resid = (const __nv_bfloat16*)c.c_resid;
   a.resid_pos = c.resid_pos;
   a.kr_base = (const uint8_t*)c.k_rope;
@@ -906,7 +920,10 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
   a.off_qr = L.off_qr; a.off_kr = L.off_kr; a.off_bar = L.off_bar; a.off_misc = L.off_misc;
   // the RoPE width per KV head is a compile-time constant so the score loop fully unrolls
   // and the per-head registers never move to local memory
-  auto kern = int4 ? decode_tc_kernel<true, 8> : decode_tc_kernel<false, 8>;
+  const bool resid = int4 && c.c_resid, paged = c.block_table != nullptr;
+  auto kern = int4 ? (resid ? (paged ? decode_tc_kernel<true, true, true, 8> : decode_tc_kernel<true, true, false, 8>)
+                            : (paged ? decode_tc_kernel<true, false, true, 8> : decode_tc_kernel<true, false, false, 8>))
+                   : (paged ? decode_tc_kernel<false, false, true, 8> : decode_tc_kernel<false, false, false, 8>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
   // the optional profiling events bracket the launch alone, after all host-side set-up

@@ -39,6 +39,12 @@ mla_status_t validate_cache(const mla_config_t& cfg, const mla_cache_t* c) {
   if (int4 && !c->c_scales) return MLA_ERR_INVALID_ARG;
   if (!int4 && c->c_scales) return MLA_ERR_INVALID_ARG;
   if (cfg.r_pairs > 0 && !c->k_rope) return MLA_ERR_INVALID_ARG;
+  if (c->block_table) {   // paged: 128-token blocks, a table row per sequence
+    if (c->n_blocks <= 0 || c->T_cap % MLA_BLOCK_TOKENS != 0) return MLA_ERR_INVALID_ARG;
+    if ((uintptr_t)c->block_table % 4 != 0) return MLA_ERR_ALIGNMENT;
+  } else if (c->n_blocks != 0) {
+    return MLA_ERR_INVALID_ARG;
+  }
   const bool resid = cfg.cache_kind == MLA_CACHE_INT4_G32_R128;
   if (resid != (c->c_resid != nullptr) || resid != (c->resid_pos != nullptr)) return MLA_ERR_INVALID_ARG;
   if (!aligned16(c->c_kv) || (c->c_scales && !aligned16(c->c_scales)) ||

@@ -15,6 +15,29 @@ inline __host__ __device__ size_t mla_kr_offset(int b, int t, int g, int j, int 
   return (((size_t)b * blocks + (size_t)(t >> 5)) * n_kv + g) * 32u * r2 + (size_t)(t & 31) * r2 + j;
 }
 
+// Storage location of token t of sequence b: (row-space sequence pb, token pt, capacity cap).
+// Contiguous cache: (b, t, T_cap).  Paged cache: (block_table[b][t/128], t % 128, 128), the
+// block id checked against the pool (outside it: error flag, block 0).  A token row index
+// is pb * cap + pt; RoPE keys sit at mla_kr_offset(pb, pt, g, j, cap, n_kv, 2r).
+struct MlaLoc {
+  int pb, pt, cap;
+};
+#ifdef __CUDACC__
+inline __device__ MlaLoc mla_loc(const mla_cache_t& c, int b, int t, int32_t* err) {
+  if (!c.block_table) return MlaLoc{b, t, c.T_cap};
+  int blk = __ldg(c.block_table + (size_t)b * (c.T_cap / MLA_BLOCK_TOKENS) + t / MLA_BLOCK_TOKENS);
+  if (blk < 0 || blk >= c.n_blocks) {
+    atomicOr(err, MLA_DEVERR_BLOCK);
+    blk = 0;
+  }
+  return MlaLoc{blk, t & (MLA_BLOCK_TOKENS - 1), MLA_BLOCK_TOKENS};
+}
+#endif
+// Token rows in the arrays of the cache (the pool's rows when paged).
+inline __host__ __device__ size_t mla_cache_rows(const mla_cache_t& c) {
+  return c.block_table ? (size_t)c.n_blocks * MLA_BLOCK_TOKENS : (size_t)c.B * c.T_cap;
+}
+
 // True for the int4 cache encodings (with or without the residual window).
 inline __host__ __device__ bool mla_kind_int4(int kind) {
   return kind == MLA_CACHE_INT4_G32 || kind == MLA_CACHE_INT4_G32_R128;

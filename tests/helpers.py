@@ -133,15 +133,15 @@ def upload_oracle_cache(case: OracleCase, cache, T_cap):
             continue
         cc = case.cache[b]
         if wl.cache == "int4_g32":
-            cache.c_kv[b, :L] = torch.from_numpy(O.pack_int4(cc["codes"])).to(cache.c_kv.device)
-            cache.c_scales[b, :L] = torch.from_numpy(cc["scales"]).to(cache.c_scales.device)
+            cache.set_latent_rows(b, 0, torch.from_numpy(O.pack_int4(cc["codes"])))
+            cache.set_scale_rows(b, 0, torch.from_numpy(cc["scales"]))
             if wl.resid:   # ring slot t % W holds token t for the window's tokens
                 W = cache.c_resid.shape[1]
                 t = np.arange(max(0, L - W), L)
                 cache.c_resid[b, t % W] = gen.to_torch(cc["c_exact"][t], wl.dtype, cache.c_resid.device)
                 cache.resid_pos[b, t % W] = torch.from_numpy(t.astype(np.int32)).to(cache.resid_pos.device)
         else:
-            cache.c_kv[b, :L] = gen.to_torch(cc["c"], wl.dtype, cache.c_kv.device)
+            cache.set_latent_rows(b, 0, gen.to_torch(cc["c"], wl.dtype, cache.c_kv.device))
         if cache.k_rope is not None:
             cache.set_k_rope_tokens(b, 0, gen.to_torch(cc["kr"], wl.dtype, cache.k_rope.device))
 

@@ -101,8 +101,8 @@ def test_append_parity(wl):
         kr = cache.k_rope_tokens(b, 0, L).double().cpu().numpy()
         assert_stored_close(kr, cc["kr_exact"], wl.dtype, f"k_rope seq {b}")
         if wl.cache == "int4_g32":
-            codes = O.unpack_int4(cache.c_kv[b, :L].cpu().numpy())
-            scales = cache.c_scales[b, :L].cpu().numpy()
+            codes = O.unpack_int4(cache.latent_rows(b, 0, L).cpu().numpy())
+            scales = cache.scale_rows(b, 0, L).cpu().numpy()
             deq = O.dequant_int4_g32(codes, scales)
             assert_close(deq, O.dequant_int4_g32(cc["codes"], cc["scales"]), wl.dtype, f"int4 latent seq {b}")
             # codes differ only where the float32 latents straddle a rounding boundary
@@ -110,7 +110,7 @@ def test_append_parity(wl):
             if wl.resid:
                 _check_ring(cache, b, L, cc["c_exact"], wl)
         else:
-            c = cache.c_kv[b, :L].double().cpu().numpy()
+            c = cache.latent_rows(b, 0, L).double().cpu().numpy()
             assert_stored_close(c, cc["c_exact"], wl.dtype, f"latent seq {b}")
 
 
@@ -133,8 +133,8 @@ def test_append_decode_step_batch(wl):
         assert_stored_close(cache.k_rope_tokens(b, p_, p_ + 1)[0].double().cpu().numpy(), cc["kr_exact"][p_],
                             wl.dtype, f"kr {b}")
         if wl.cache == "int4_g32":
-            codes = O.unpack_int4(cache.c_kv[b, p_:p_ + 1].cpu().numpy())
-            deq = O.dequant_int4_g32(codes, cache.c_scales[b, p_:p_ + 1].cpu().numpy())
+            codes = O.unpack_int4(cache.latent_rows(b, p_, p_ + 1).cpu().numpy())
+            deq = O.dequant_int4_g32(codes, cache.scale_rows(b, p_, p_ + 1).cpu().numpy())
             assert_close(deq[0], O.dequant_int4_g32(cc["codes"][p_:p_ + 1], cc["scales"][p_:p_ + 1])[0],
                          wl.dtype, f"int4 latent {b}")
             if wl.resid:   # only the appended token's slot is claimed and written
@@ -144,7 +144,8 @@ def test_append_decode_step_batch(wl):
                 assert_stored_close(cache.c_resid[b, p_ % W].double().cpu().numpy(), cc["c_exact"][p_],
                                     wl.dtype, f"ring {b}")
         else:
-            assert_stored_close(cache.c_kv[b, p_].double().cpu().numpy(), cc["c_exact"][p_], wl.dtype, f"c {b}")
+            assert_stored_close(cache.latent_rows(b, p_, p_ + 1)[0].double().cpu().numpy(), cc["c_exact"][p_],
+                                wl.dtype, f"c {b}")
 
 
 def _check_ring(cache, b, L, c_exact, wl):
@@ -344,3 +345,98 @@ def test_svd_split_conversion_append_decode(wl):
     assert mla.mla_device_error(plan) == 0
     for b in case.seqs:
         assert_close(got[b], case.reference(b), wl.dtype, f"SVD_split seq {b}")
+
+
+# --------------------------------------------------------------------------- paged cache
+def _paged_cache(cfg, B, lens, seed, spare=3):
+    """A paged cache whose sequences' 128-token blocks sit at shuffled pool positions
+    (plus spare blocks nobody uses); unused table entries name a spare block."""
+    BT = mla.MLA_BLOCK_TOKENS
+    T_cap = max(BT, -(-int(max(lens)) // BT) * BT)
+    need = [-(-int(L) // BT) for L in lens]
+    n_blocks = sum(need) + spare
+    ids = np.random.default_rng(seed).permutation(n_blocks)
+    table = np.full((B, T_cap // BT), ids[-1], dtype=np.int32)
+    k = 0
+    for b, nb in enumerate(need):
+        table[b, :nb] = ids[k:k + nb]
+        k += nb
+    return LatentCache(cfg, B, T_cap, "cuda", block_table=table, n_blocks=n_blocks)
+
+
+PAGED = [PARITY_WORKLOADS[0], PARITY_WORKLOADS[1], PARITY_WORKLOADS[2], PARITY_WORKLOADS[3],
+         PARITY_WORKLOADS[4]] + RESID_WORKLOADS
+
+
+@pytest.mark.parametrize("wl", PAGED, ids=[w.name for w in PAGED])
+def test_paged_append_matches_contiguous(wl):
+    """All tokens of all sequences in one append call, into a contiguous and a paged cache:
+    every token's stored latent (or int4 codes and scales), RoPE keys and ring row agree
+    bit for bit (the same arithmetic, only the addresses differ)."""
+    case = case_for(wl)
+    cfg, plan = make_plan(case)
+    lens = [int(L) for L in case.lens]
+    flat = LatentCache(cfg, wl.batch, max(1, max(lens)), "cuda")
+    paged = _paged_cache(cfg, wl.batch, lens, seed=5)
+    xs, sidx, pos = [], [], []
+    for b in case.seqs:
+        x = case.tokens(b)
+        xs.append(x)
+        sidx += [b] * x.shape[0]
+        pos += list(range(x.shape[0]))
+    x = gen.to_torch(np.concatenate(xs), wl.dtype, "cuda")
+    si = torch.tensor(sidx, dtype=torch.int32, device="cuda")
+    po = torch.tensor(pos, dtype=torch.int32, device="cuda")
+    for c in (flat, paged):
+        mla.mla_append(plan, x, si, po, c.struct)
+    assert mla.mla_device_error(plan) == 0
+    for b in case.seqs:
+        L = lens[b]
+        if L == 0:
+            continue
+        assert torch.equal(flat.latent_rows(b, 0, L), paged.latent_rows(b, 0, L)), f"latent seq {b}"
+        if flat.c_scales is not None:
+            assert torch.equal(flat.scale_rows(b, 0, L), paged.scale_rows(b, 0, L)), f"scales seq {b}"
+        if flat.k_rope is not None:
+            assert torch.equal(flat.k_rope_tokens(b, 0, L), paged.k_rope_tokens(b, 0, L)), f"k_rope seq {b}"
+        if flat.c_resid is not None:
+            assert torch.equal(flat.resid_pos[b], paged.resid_pos[b])
+            assert torch.equal(flat.c_resid[b], paged.c_resid[b])
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
+@pytest.mark.parametrize("wl", PAGED, ids=[w.name for w in PAGED])
+def test_paged_decode_parity(wl, kernel):
+    """Decode over a paged cache (shuffled blocks) equals the decode over the contiguous
+    cache bit for bit, and the oracle within tolerance."""
+    if kernel == 2 and (wl.dtype == "f32" or wl.n_heads != 32):
+        pytest.skip("shape outside the tensor-core kernel (fp32 or H != 32)")
+    case = case_for(wl)
+    cfg, plan = make_plan(case, kernel=kernel)
+    lens = [int(L) for L in case.lens]
+    flat = run_decode(case, plan, cfg)
+    paged = _paged_cache(cfg, wl.batch, lens, seed=7)
+    upload_oracle_cache(case, paged, paged.T_cap)
+    got = run_decode(case, plan, cfg, cache=paged)
+    assert mla.mla_device_error(plan) == 0
+    np.testing.assert_array_equal(got, flat)
+    for b in case.seqs:
+        assert_close(got[b], case.reference(b), wl.dtype, f"paged decode seq {b} (L={lens[b]})")
+
+
+def test_paged_block_outside_pool_is_flagged():
+    """A table entry outside the pool is reported (and block 0 read or written instead)."""
+    wl = PARITY_WORKLOADS[2]
+    case = case_for(wl)
+    lens = [int(L) for L in case.lens]
+    for kernel in (1, 2):
+        cfg, plan = make_plan(case, kernel=kernel)
+        paged = _paged_cache(cfg, wl.batch, lens, seed=9)
+        upload_oracle_cache(case, paged, paged.T_cap)
+        paged.block_table[0, 0] = paged.n_blocks          # sequence 0's first block: outside
+        run_decode(case, plan, cfg, cache=paged)
+        assert mla.mla_device_error(plan) & mla.MLA_DEVERR_BLOCK
+        x = gen.to_torch(case.x_dec[:1], wl.dtype, "cuda")
+        mla.mla_append(plan, x, torch.zeros(1, dtype=torch.int32, device="cuda"),
+                       torch.zeros(1, dtype=torch.int32, device="cuda"), paged.struct)
+        assert mla.mla_device_error(plan) & mla.MLA_DEVERR_BLOCK
