@@ -30,6 +30,10 @@ Pinning status (see tests/test_oracle_pins.py):
   fixed_pairs — the pages name the high / low / uniform / full strategies without
   formulas; the reading is pinned by its frequency meaning (rope_theta ordering),
   hand-written sets and the full-RoPE case, which reduces to textbook RoPE MHA.
+  quant_int2_g32 / dequant_int2_g32 / pack_int2 — the Notes name 2-bit quantisation of
+  the latent without an encoding; the reading (the int4 scheme at 2 bits) is pinned by
+  its error bound, the group maximum landing on +-1, exact round trips, hand-derived codes
+  and a hand-derived byte.
   residual_window — the README gives only the residual length (128) of the quantised
   cache; the reading (the most recent tokens read unquantised) is pinned by its special
   cases (no window: the int4 values; a window over the whole sequence: the plain values),

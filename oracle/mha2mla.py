@@ -24,7 +24,8 @@ import numpy as np
 __all__ = [
     "rope_theta", "rotate", "pair_norms", "pair_scores", "select_pairs", "fixed_pairs", "split_dims",
     "svd_joint", "svd_split", "krope_weights", "convert", "append", "quant_int4_g32", "dequant_int4_g32",
-    "pack_int4", "unpack_int4", "residual_window", "decode_unabsorbed", "decode_absorbed", "decode_sequence",
+    "pack_int4", "unpack_int4", "residual_window", "quant_int2_g32", "dequant_int2_g32", "pack_int2",
+    "unpack_int2", "decode_unabsorbed", "decode_absorbed", "decode_sequence",
     "mha_textbook_rope", "cache_bytes_per_token", "mha_cache_bytes_per_token",
 ]
 
@@ -333,6 +334,47 @@ def unpack_int4(packed: np.ndarray) -> np.ndarray:
     out = np.empty((packed.shape[0], packed.shape[1] * 2), dtype=np.int8)
     out[:, 0::2] = lo
     out[:, 1::2] = hi
+    return out
+
+
+def quant_int2_g32(c: np.ndarray):
+    """Per-token 2-bit quantisation of the latent in groups of 32.
+
+    NOTES §关键设计 / KV-cache quantisation: 4-bit or 2-bit quantisation stacks on the
+    latent.  The reading is the int4 encoding's scheme at 2 bits: symmetric, zero is a
+    level, codes clamp(rint_half_even(c/scale), -1, 1) (the largest magnitude 2^(2-1)-1),
+    scale fp16(absmax / 1); an all-zero group (or a scale that rounds to 0) gives scale 0
+    and codes 0.  Decisions are taken in float32.
+
+    c [N][d_c] -> codes int8 [N][d_c] in {-1, 0, 1}, scales float16 [N][d_c/32]
+    """
+    c32 = np.asarray(c, dtype=np.float64).astype(np.float32)
+    N, dc = c32.shape
+    g = c32.reshape(N, dc // 32, 32)
+    scale16 = np.abs(g).max(axis=-1).astype(np.float16)
+    sc32 = scale16.astype(np.float32)
+    safe = np.where(sc32 > 0, sc32, np.float32(1.0))
+    q = np.clip(np.rint((g / safe[..., None]).astype(np.float32)), -1, 1)
+    q = np.where(sc32[..., None] > 0, q, 0)
+    return q.astype(np.int8).reshape(N, dc), scale16
+
+
+def dequant_int2_g32(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """value = code * scale (exact in float64)."""
+    return dequant_int4_g32(codes, scales)
+
+
+def pack_int2(codes: np.ndarray) -> np.ndarray:
+    """Two's-complement 2-bit fields, element 4i + k in bits 2k, 2k+1 of byte i."""
+    u = (codes.astype(np.int16) & 0x3).astype(np.uint8)
+    return (u[:, 0::4] | (u[:, 1::4] << 2) | (u[:, 2::4] << 4) | (u[:, 3::4] << 6)).astype(np.uint8)
+
+
+def unpack_int2(packed: np.ndarray) -> np.ndarray:
+    out = np.empty((packed.shape[0], packed.shape[1] * 4), dtype=np.int8)
+    for k in range(4):
+        f = ((packed >> (2 * k)) & 0x3).astype(np.int16)
+        out[:, k::4] = np.where(f >= 2, f - 4, f)
     return out
 
 

@@ -444,3 +444,41 @@ def test_T11_decode_over_window_reduces_to_pinned_decodes():
     np.testing.assert_array_equal(dec(O.residual_window(deq, plain, 0)), dec(deq))
     mixed = dec(O.residual_window(deq, plain, 16))
     assert not np.array_equal(mixed, dec(deq)) and not np.array_equal(mixed, dec(plain))
+
+
+# ------------------------------------------------------------------ T12 2-bit latent
+def test_T12_int2_hand_derived_codes_and_bytes():
+    g = np.zeros((1, 32))
+    g[0, :8] = [3.0, -3.0, 1.4, -1.6, 1.5, -1.5, 0.2, 2.9]
+    codes, scales = O.quant_int2_g32(g)
+    assert scales[0, 0] == np.float16(3.0)
+    # c/s = 1, -1, 0.467, -0.533, 0.5 (half to even: 0), -0.5 (0), 0.067, 0.967
+    assert codes[0, :8].tolist() == [1, -1, 0, -1, 0, 0, 0, 1]
+    assert np.all(codes[0, 8:] == 0)
+    # bytes: element 4i + k in bits 2k..2k+1, two's complement (-1 = 0b11)
+    packed = O.pack_int2(codes)
+    assert packed[0, 0] == (1 | (3 << 2) | (0 << 4) | (3 << 6))
+    assert packed[0, 1] == (0 | (0 << 2) | (0 << 4) | (1 << 6))
+    np.testing.assert_array_equal(O.unpack_int2(packed), codes)
+    z, zs = O.quant_int2_g32(np.zeros((2, 64)))
+    assert np.all(z == 0) and np.all(zs == 0)
+
+
+def test_T12_int2_error_bound_and_round_trip():
+    rng = np.random.default_rng(37)
+    c = rng.standard_normal((40, 128)) * rng.lognormal(0, 1, size=(40, 1))
+    codes, scales = O.quant_int2_g32(c)
+    assert set(np.unique(codes).tolist()) <= {-1, 0, 1}
+    deq = O.dequant_int2_g32(codes, scales)
+    sc = np.repeat(scales.astype(np.float64), 32, axis=1)
+    c32 = c.astype(np.float32).astype(np.float64)
+    # within half a step (plus the fp16 rounding of the scale), and the group max lands on +-1
+    assert np.all(np.abs(deq - c32) <= sc * (0.5 + 1e-3) + 1e-30)
+    assert np.all(np.abs(codes.reshape(40, 4, 32)).max(axis=-1) == 1)
+    codes2, scales2 = O.quant_int2_g32(deq)
+    np.testing.assert_array_equal(codes2, codes)
+    np.testing.assert_array_equal(scales2, scales)
+    np.testing.assert_array_equal(O.unpack_int2(O.pack_int2(codes)), codes)
+    # 2 bits lose more than 4 on the same latents
+    c4, s4 = O.quant_int4_g32(c)
+    assert np.linalg.norm(O.dequant_int4_g32(c4, s4) - c32) < np.linalg.norm(deq - c32)
