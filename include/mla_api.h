@@ -73,7 +73,14 @@ typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype_t;
  * (the largest one appended there: it only grows).  Decode reads token t of a sequence
  * of length L from the ring when t >= L - 128 and resid_pos[t % 128] == t, else from the
  * int4 row, so with positions appended in order the window is exactly [L-128, L). */
-typedef enum { MLA_CACHE_SAME = 0, MLA_CACHE_INT4_G32 = 1, MLA_CACHE_INT4_G32_R128 = 2 } mla_cache_kind_t;
+typedef enum {
+  MLA_CACHE_SAME = 0, MLA_CACHE_INT4_G32 = 1, MLA_CACHE_INT4_G32_R128 = 2, MLA_CACHE_INT2_G32 = 3
+} mla_cache_kind_t;
+/* MLA_CACHE_INT2_G32 is the same scheme at 2 bits (Notes §关键设计: 4-bit or 2-bit
+ * quantisation stacks on the latent): per token, groups of 32, fp16 scale s = fp16(absmax),
+ * codes clamp(round_half_even(c/s), -1, 1) (0 when s == 0), two's-complement 2-bit fields,
+ * element 4i+k in bits 2k..2k+1 of byte i; value = code*s.  Decoded by the CUDA-core
+ * kernel (the tensor-core kernel reports MLA_ERR_UNSUPPORTED when forced). */
 #define MLA_RESID_WINDOW 128
 
 typedef struct {
@@ -85,7 +92,7 @@ typedef struct {
   int32_t d_c;          /* latent width, multiple of 4 (of 32 for the int4 cache) */
   double rope_base;     /* RoPE base (10000 for the Llama/SmolLM shapes) */
   int32_t dtype;        /* mla_dtype_t */
-  int32_t cache_kind;   /* mla_cache_kind_t (the int4 kinds require dtype MLA_BF16) */
+  int32_t cache_kind;   /* mla_cache_kind_t (the int4 and int2 kinds require dtype MLA_BF16) */
 } mla_config_t;
 
 /* Caller-owned cache, device memory, capacity T_cap tokens per sequence.
@@ -98,8 +105,9 @@ typedef struct {
  * README "MHA2MLA" runs ragged LongBench batches; 128-token blocks match the decode tile,
  * so each tile of the attention kernel reads one block.  A table entry outside
  * [0, n_blocks) flags MLA_DEVERR_BLOCK and reads or writes block 0 instead.
- *   c_kv      SAME: [B][T_cap][d_c] dtype;  INT4*: [B][T_cap][d_c/2] uint8 codes
- *   c_scales  INT4*: [B][T_cap][d_c/32] fp16;  SAME: must be NULL
+ *   c_kv      SAME: [B][T_cap][d_c] dtype;  INT4*: [B][T_cap][d_c/2] uint8 codes;
+ *             INT2: [B][T_cap][d_c/4] uint8 codes
+ *   c_scales  INT4*, INT2: [B][T_cap][d_c/32] fp16;  SAME: must be NULL
  *   k_rope    [B][ceil(T_cap/32)][n_kv][32][2r] dtype (may be NULL when r == 0): the kept
  *             RoPE key dims in blocks of 32 tokens, KV-head-major inside a block, so the
  *             2r dims of one KV head for 32 consecutive tokens are contiguous; element

@@ -17,7 +17,7 @@ LIB_PATH = os.environ.get("MLA_B200_LIB", os.path.join(_PKG, "lib", "libmla_b200
 MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_ALIGNMENT = 0, 1, 2, 3
 MLA_ERR_WORKSPACE_TOO_SMALL, MLA_ERR_CUDA, MLA_ERR_DEVICE = 4, 5, 6
 MLA_F32, MLA_BF16 = 0, 1
-MLA_CACHE_SAME, MLA_CACHE_INT4_G32, MLA_CACHE_INT4_G32_R128 = 0, 1, 2
+MLA_CACHE_SAME, MLA_CACHE_INT4_G32, MLA_CACHE_INT4_G32_R128, MLA_CACHE_INT2_G32 = 0, 1, 2, 3
 MLA_RESID_WINDOW = 128
 MLA_OPT_DECODE_KERNEL, MLA_OPT_DECODE_SPLITS, MLA_OPT_PROFILE_EVENTS, MLA_OPT_OVERLAP_LAUNCH = 1, 2, 3, 4
 MLA_DEVERR_SEQ_LEN, MLA_DEVERR_APPEND_SLOT, MLA_DEVERR_TIMEOUT, MLA_DEVERR_BLOCK = 1, 2, 4, 8
@@ -114,9 +114,13 @@ def _stream(stream):
 
 def make_config(hidden, n_heads, n_kv_heads, head_dim, r_pairs, d_c, rope_base=10000.0,
                 dtype="bf16", cache="same", resid=0) -> MlaConfig:
-    """cache: "same" or "int4_g32"; resid: 0, or MLA_RESID_WINDOW for the int4 cache with
-    the unquantised residual window (MLA_CACHE_INT4_G32_R128)."""
-    if cache == "int4_g32":
+    """cache: "same", "int4_g32" or "int2_g32"; resid: 0, or MLA_RESID_WINDOW for the int4
+    cache with the unquantised residual window (MLA_CACHE_INT4_G32_R128)."""
+    if cache == "int2_g32":
+        if resid:
+            raise ValueError("the residual window is built for the int4 cache")
+        kind = MLA_CACHE_INT2_G32
+    elif cache == "int4_g32":
         if resid not in (0, MLA_RESID_WINDOW):
             raise ValueError(f"residual window {resid}: this library keeps {MLA_RESID_WINDOW} tokens")
         kind = MLA_CACHE_INT4_G32_R128 if resid else MLA_CACHE_INT4_G32

@@ -34,8 +34,9 @@ class LatentCache:
         else:
             self.block_table, self.n_blocks = None, 0
             rows, cap = B, T_cap
-        if cfg.cache_kind in (_lib.MLA_CACHE_INT4_G32, _lib.MLA_CACHE_INT4_G32_R128):
-            self.c_kv = torch.zeros(rows, cap, cfg.d_c // 2, dtype=torch.uint8, device=device)
+        if cfg.cache_kind in (_lib.MLA_CACHE_INT4_G32, _lib.MLA_CACHE_INT4_G32_R128, _lib.MLA_CACHE_INT2_G32):
+            per_byte = 4 if cfg.cache_kind == _lib.MLA_CACHE_INT2_G32 else 2   # codes per byte
+            self.c_kv = torch.zeros(rows, cap, cfg.d_c // per_byte, dtype=torch.uint8, device=device)
             self.c_scales = torch.zeros(rows, cap, cfg.d_c // 32, dtype=torch.float16, device=device)
         else:
             self.c_kv = torch.zeros(rows, cap, cfg.d_c, dtype=dt, device=device)

@@ -38,6 +38,7 @@ struct AppendArgs {
   const int32_t* rope_pair;  // [n_kv][r]
   const double* theta;
   int32_t* err;
+  int qbits;                // quantised latent (INT4 instantiations): code width, 4 or 2
   int kslice;               // hidden dims per cluster rank
   int vec_ok;               // x rows and W rows allow 16-byte vector loads
 };
@@ -49,6 +50,33 @@ __device__ __forceinline__ void resid_store(const mla_cache_t& c, int sq, int p,
   if (!c.c_resid) return;
   const size_t rs = (size_t)sq * MLA_RESID_WINDOW + (p & (MLA_RESID_WINDOW - 1));
   if (c.resid_pos[rs] == p) ((__nv_bfloat16*)c.c_resid)[rs * d_c + col] = __float2bfloat16_rn(v);
+}
+
+// Quantises one group of 32 latent values held one per lane (lane l: element col, the
+// group's start + l) and stores codes and scale at token row `slot`.  4 bits: scale
+// fp16(absmax/7), codes in [-7, 7], two per byte; 2 bits: scale fp16(absmax), codes in
+// [-1, 1], four per byte.  Decisions in float32 (the division correctly rounded).
+__device__ __forceinline__ void quant_group_store(const mla_cache_t& c, size_t slot, int d_c, int col, int lane,
+                                                  float v, int qbits) {
+  float am = fabsf(v);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  const int qmax = qbits == 4 ? 7 : 1;
+  const __half sh = __float2half_rn(qbits == 4 ? __fdiv_rn(am, 7.0f) : am);
+  const float sc = __half2float(sh);
+  int code = 0;
+  if (sc > 0.f) code = max(-qmax, min(qmax, (int)rintf(__fdiv_rn(v, sc))));
+  if (qbits == 4) {
+    const uint32_t nib = (uint32_t)code & 15u;
+    const uint32_t hi = __shfl_down_sync(0xffffffffu, nib, 1);
+    if ((lane & 1) == 0) ((uint8_t*)c.c_kv)[slot * (d_c / 2) + col / 2] = (uint8_t)(nib | (hi << 4));
+  } else {
+    const uint32_t f = (uint32_t)code & 3u;
+    const uint32_t f1 = __shfl_down_sync(0xffffffffu, f, 1), f2 = __shfl_down_sync(0xffffffffu, f, 2),
+                   f3 = __shfl_down_sync(0xffffffffu, f, 3);
+    if ((lane & 3) == 0) ((uint8_t*)c.c_kv)[slot * (d_c / 4) + col / 4] = (uint8_t)(f | (f1 << 2) | (f2 << 4) | (f3 << 6));
+  }
+  if (lane == 0) ((__half*)c.c_scales)[slot * (d_c / 32) + col / 32] = sh;
 }
 
 // Claims the residual ring slots of a call's tokens: resid_pos[seq][p % 128] becomes the
@@ -114,17 +142,7 @@ __device__ void append_epilogue(const AppendArgs& a, const float* tile, int tok0
       const MlaLoc lc = mla_loc(c, sq, p, a.err);
       const size_t slot = (size_t)lc.pb * lc.cap + lc.pt;
       const float v = tile[t * COLS + gi * 32 + lane];
-      float am = fabsf(v);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-      const __half sh = __float2half_rn(__fdiv_rn(am, 7.0f));
-      const float sc = __half2float(sh);
-      int code = 0;
-      if (sc > 0.f) code = max(-7, min(7, (int)rintf(__fdiv_rn(v, sc))));
-      const uint32_t nib = (uint32_t)code & 15u;
-      const uint32_t hi = __shfl_down_sync(0xffffffffu, nib, 1);
-      if ((lane & 1) == 0) ((uint8_t*)c.c_kv)[slot * (a.d_c / 2) + col / 2] = (uint8_t)(nib | (hi << 4));
-      if (lane == 0) ((__half*)c.c_scales)[slot * (a.d_c / 32) + col / 32] = sh;
+      quant_group_store(c, slot, a.d_c, col, lane, v, a.qbits);
       resid_store(c, sq, p, a.d_c, col, v);
     }
   }
@@ -296,17 +314,7 @@ __device__ __forceinline__ void append_small_finish(const AppendSmallArgs& sa, f
       const MlaLoc lc = mla_loc(c, sq, p, a.err);
       const size_t slot = (size_t)lc.pb * lc.cap + lc.pt;
       const float v = tileb[t * kSmCols + lane];
-      float am = fabsf(v);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-      const __half sh = __float2half_rn(__fdiv_rn(am, 7.0f));
-      const float sc = __half2float(sh);
-      int code = 0;
-      if (sc > 0.f) code = max(-7, min(7, (int)rintf(__fdiv_rn(v, sc))));
-      const uint32_t nib = (uint32_t)code & 15u;
-      const uint32_t hi = __shfl_down_sync(0xffffffffu, nib, 1);
-      if ((lane & 1) == 0) ((uint8_t*)c.c_kv)[slot * (a.d_c / 2) + (col0 + lane) / 2] = (uint8_t)(nib | (hi << 4));
-      if (lane == 0) ((__half*)c.c_scales)[slot * (a.d_c / 32) + col0 / 32] = sh;
+      quant_group_store(c, slot, a.d_c, col0 + lane, lane, v, a.qbits);
       resid_store(c, sq, p, a.d_c, col0 + lane, v);
     }
   }
@@ -578,7 +586,8 @@ cudaError_t mla_launch_append(const mla_plan& p, const void* x, const int32_t* s
   a.rope_pair = p.rope_pair; a.theta = p.theta; a.err = p.err;
   const size_t eb = cfg.dtype == MLA_BF16 ? 2 : 4;
   a.vec_ok = ((uintptr_t)x % 16 == 0) && ((size_t)cfg.hidden * eb) % 16 == 0 && ((size_t)p.ncols * eb) % 16 == 0;
-  const bool int4 = mla_kind_int4(cfg.cache_kind);
+  const bool int4 = mla_kind_quant(cfg.cache_kind);   // quantised latent (int4 or int2 codes)
+  a.qbits = mla_quant_bits(cfg.cache_kind);
   if (c.c_resid) {   // residual window: claim the ring slots first
     const int grid = std::max(1, std::min((N + 255) / 256, 4 * p.num_sms));
     cudaError_t e = mla_launch_kernel(resid_claim_kernel, dim3(grid), dim3(256), 0, s, p.opt_pdl, seq_idx, pos, N, c);

@@ -157,6 +157,7 @@ struct DecodeArgs {
   mla_cache_t cache;
   const int32_t* seq_lens;   // read for the residual window only
   int32_t* err;
+  int qbits;                 // quantised cache: code width (4 or 2)
   int B, H, n_kv, r, d_c, R;
   const float* qlat;
   const float* qrope;
@@ -212,11 +213,16 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(DecodeArgs a) {
           const size_t rs = (size_t)b * MLA_RESID_WINDOW + (tp & (MLA_RESID_WINDOW - 1));
           if (tp >= lo && a.cache.resid_pos[rs] == tp) {
             v = __bfloat162float(((const __nv_bfloat16*)a.cache.c_resid)[rs * dc + cc]);
-          } else {
+          } else if (a.qbits == 4) {
             const uint8_t* codes = (const uint8_t*)a.cache.c_kv + (slot0 + tt) * (dc / 2);
             const __half* sc = (const __half*)a.cache.c_scales + (slot0 + tt) * (dc / 32);
             uint32_t byte = codes[cc / 2];
             v = (float)nib_to_int((cc & 1) ? (byte >> 4) : (byte & 15u)) * __half2float(sc[cc / 32]);
+          } else {   // 2-bit: element 4i+k in bits 2k..2k+1 of byte i, two's complement
+            const uint8_t* codes = (const uint8_t*)a.cache.c_kv + (slot0 + tt) * (dc / 4);
+            const __half* sc = (const __half*)a.cache.c_scales + (slot0 + tt) * (dc / 32);
+            const int f = (codes[cc / 4] >> (2 * (cc & 3))) & 3;
+            v = (float)(f >= 2 ? f - 4 : f) * __half2float(sc[cc / 32]);
           }
         } else {
           v = to_f32(((const T*)a.cache.c_kv)[(slot0 + tt) * dc + cc]);
@@ -502,7 +508,7 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
   // 2. split-K attention over the latent cache
   if (L.kernel == 1) {
     DecodeArgs da;
-    da.cache = c; da.seq_lens = seq_lens; da.err = p.err; da.B = B; da.H = H; da.n_kv = cfg.n_kv_heads; da.r = cfg.r_pairs;
+    da.cache = c; da.seq_lens = seq_lens; da.err = p.err; da.qbits = mla_quant_bits(cfg.cache_kind); da.B = B; da.H = H; da.n_kv = cfg.n_kv_heads; da.r = cfg.r_pairs;
     da.d_c = cfg.d_c; da.R = p.R; da.qlat = aa.qlat; da.qrope = aa.qrope;
     da.opart = (float*)(base + L.off_opart); da.mlpart = (float*)(base + L.off_mlpart);
     da.P = L.P;
@@ -592,9 +598,9 @@ cudaError_t mla_launch_decode(const mla_plan& p, const mla_cache_t& c, const int
                               const void* q, int B, void* out, void* ws, const DecodeLayout& L,
                               cudaStream_t s) {
   using namespace mla;
-  bool int4 = mla_kind_int4(p.cfg.cache_kind);
+  const bool quant = mla_kind_quant(p.cfg.cache_kind);   // int4 or int2 codes
   if (p.cfg.dtype == MLA_BF16)
-    return int4 ? launch_decode_t<__nv_bfloat16, true>(p, c, seq_lens, q, B, out, ws, L, s)
+    return quant ? launch_decode_t<__nv_bfloat16, true>(p, c, seq_lens, q, B, out, ws, L, s)
                 : launch_decode_t<__nv_bfloat16, false>(p, c, seq_lens, q, B, out, ws, L, s);
   return launch_decode_t<float, false>(p, c, seq_lens, q, B, out, ws, L, s);
 }

@@ -42,14 +42,10 @@ extern "C" mla_status_t mla_decode_noalloc(const mla_plan_t* plan, const mla_cac
                                            void* stream) {
   if (!plan || !cache || !seq_lens || !q || !out || B <= 0) return MLA_ERR_INVALID_ARG;
   const mla_config_t& cfg = plan->cfg;
-  const bool int4 = mla_kind_int4(cfg.cache_kind);
-  if (!cache->c_kv || cache->B <= 0 || cache->T_cap <= 0 || B > cache->B) return MLA_ERR_INVALID_ARG;
-  if (int4 != (cache->c_scales != nullptr)) return MLA_ERR_INVALID_ARG;
-  if (cfg.r_pairs > 0 && !cache->k_rope) return MLA_ERR_INVALID_ARG;
-  if (!aligned16(cache->c_kv) || (cache->c_scales && !aligned16(cache->c_scales)) ||
-      (cache->k_rope && !aligned16(cache->k_rope)) || !aligned16(q) || !aligned16(out) ||
-      ((uintptr_t)seq_lens & 3))
-    return MLA_ERR_ALIGNMENT;
+  const mla_status_t st = mla_validate_cache(cfg, cache);   // the same checks as mla_decode
+  if (st != MLA_OK) return st;
+  if (B > cache->B) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || ((uintptr_t)seq_lens & 3)) return MLA_ERR_ALIGNMENT;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
   if (dev != plan->device) return MLA_ERR_INVALID_ARG;   // the plan's weights live on its device
@@ -58,7 +54,7 @@ extern "C" mla_status_t mla_decode_noalloc(const mla_plan_t* plan, const mla_cac
   if (g_scratch_err[dev] != cudaSuccess || !g_scratch[dev]) return MLA_ERR_CUDA;
 
   int kernel = 1;
-  if (plan->opt_kernel != 1 && mla_tc_supported(*plan, *cache)) kernel = 2;
+  if (plan->opt_kernel != 1 && mla_tc_kind_ok(cfg) && mla_tc_supported(*plan, *cache)) kernel = 2;
   if (plan->opt_kernel == 2 && kernel != 2) return MLA_ERR_UNSUPPORTED;
   if (kernel == 1 && (size_t)cfg.n_heads * cfg.d_c > 8192) return MLA_ERR_UNSUPPORTED;
   const DecodeLayout L = mla_decode_layout(*plan, B, kernel);

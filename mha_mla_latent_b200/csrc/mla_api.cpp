@@ -24,8 +24,8 @@ mla_status_t validate_config(const mla_config_t* c) {
   if (c->r_pairs < 0 || 2 * c->r_pairs > c->head_dim) return MLA_ERR_INVALID_ARG;
   if (!(c->rope_base > 1.0)) return MLA_ERR_INVALID_ARG;
   if (c->dtype != MLA_F32 && c->dtype != MLA_BF16) return MLA_ERR_INVALID_ARG;
-  if (c->cache_kind != MLA_CACHE_SAME && !mla_kind_int4(c->cache_kind)) return MLA_ERR_INVALID_ARG;
-  if (mla_kind_int4(c->cache_kind) && (c->dtype != MLA_BF16 || c->d_c % 32 != 0))
+  if (c->cache_kind != MLA_CACHE_SAME && !mla_kind_quant(c->cache_kind)) return MLA_ERR_INVALID_ARG;
+  if (mla_kind_quant(c->cache_kind) && (c->dtype != MLA_BF16 || c->d_c % 32 != 0))
     return MLA_ERR_UNSUPPORTED;
   // limits of the kernels in this build
   if (c->head_dim > 256 || c->d_c > 1024 || c->n_heads > 256) return MLA_ERR_UNSUPPORTED;
@@ -33,11 +33,12 @@ mla_status_t validate_config(const mla_config_t* c) {
   return MLA_OK;
 }
 
-mla_status_t validate_cache(const mla_config_t& cfg, const mla_cache_t* c) {
+}  // namespace
+
+mla_status_t mla_validate_cache(const mla_config_t& cfg, const mla_cache_t* c) {
   if (!c || !c->c_kv || c->B <= 0 || c->T_cap <= 0) return MLA_ERR_INVALID_ARG;
-  bool int4 = mla_kind_int4(cfg.cache_kind);
-  if (int4 && !c->c_scales) return MLA_ERR_INVALID_ARG;
-  if (!int4 && c->c_scales) return MLA_ERR_INVALID_ARG;
+  const bool quant = mla_kind_quant(cfg.cache_kind);
+  if (quant != (c->c_scales != nullptr)) return MLA_ERR_INVALID_ARG;
   if (cfg.r_pairs > 0 && !c->k_rope) return MLA_ERR_INVALID_ARG;
   if (c->block_table) {   // paged: 128-token blocks, a table row per sequence
     if (c->n_blocks <= 0 || c->T_cap % MLA_BLOCK_TOKENS != 0) return MLA_ERR_INVALID_ARG;
@@ -53,6 +54,8 @@ mla_status_t validate_cache(const mla_config_t& cfg, const mla_cache_t* c) {
     return MLA_ERR_ALIGNMENT;
   return MLA_OK;
 }
+
+namespace {
 
 mla_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
@@ -94,6 +97,7 @@ size_t mla_cache_bytes_per_token(const mla_config_t* cfg) {
   size_t eb = elem_bytes(*cfg);
   size_t rope = (size_t)cfg->n_kv_heads * 2 * cfg->r_pairs * eb;
   if (mla_kind_int4(cfg->cache_kind)) return (size_t)cfg->d_c / 2 + 2 * ((size_t)cfg->d_c / 32) + rope;
+  if (mla_kind_int2(cfg->cache_kind)) return (size_t)cfg->d_c / 4 + 2 * ((size_t)cfg->d_c / 32) + rope;
   return (size_t)cfg->d_c * eb + rope;
 }
 
@@ -245,7 +249,7 @@ mla_status_t mla_plan_set_option(mla_plan_t* plan, int32_t option, int64_t value
 mla_status_t mla_append(const mla_plan_t* plan, const void* x, const int32_t* seq_idx,
                         const int32_t* pos, int32_t N, const mla_cache_t* cache, void* stream) {
   if (!plan || !x || !seq_idx || !pos || N <= 0) return MLA_ERR_INVALID_ARG;
-  mla_status_t st = validate_cache(plan->cfg, cache);
+  mla_status_t st = mla_validate_cache(plan->cfg, cache);
   if (st != MLA_OK) return st;
   if (!aligned16(x) || ((uintptr_t)seq_idx & 3) || ((uintptr_t)pos & 3)) return MLA_ERR_ALIGNMENT;
   return cuda_status(mla_launch_append(*plan, x, seq_idx, pos, N, *cache, (cudaStream_t)stream));
@@ -254,7 +258,7 @@ mla_status_t mla_append(const mla_plan_t* plan, const void* x, const int32_t* se
 size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B) {
   if (!plan || B <= 0) return 0;
   size_t n = mla_decode_layout(*plan, B, 1).total;
-  if (mla_tc_capable(*plan)) n = std::max(n, mla_decode_layout(*plan, B, 2).total);
+  if (mla_tc_kind_ok(plan->cfg) && mla_tc_capable(*plan)) n = std::max(n, mla_decode_layout(*plan, B, 2).total);
   return n;
 }
 
@@ -262,13 +266,13 @@ mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache, const 
                         const void* q, int32_t B, void* out, void* workspace, size_t ws_bytes,
                         void* stream) {
   if (!plan || !seq_lens || !q || !out || !workspace || B <= 0) return MLA_ERR_INVALID_ARG;
-  mla_status_t st = validate_cache(plan->cfg, cache);
+  mla_status_t st = mla_validate_cache(plan->cfg, cache);
   if (st != MLA_OK) return st;
   if (B > cache->B) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace) || ((uintptr_t)seq_lens & 3))
     return MLA_ERR_ALIGNMENT;
   int kernel = 1;
-  if (plan->opt_kernel != 1 && mla_tc_supported(*plan, *cache)) kernel = 2;
+  if (plan->opt_kernel != 1 && mla_tc_kind_ok(plan->cfg) && mla_tc_supported(*plan, *cache)) kernel = 2;
   if (plan->opt_kernel == 2 && kernel != 2) return MLA_ERR_UNSUPPORTED;
   if (kernel == 1 && (size_t)plan->cfg.n_heads * plan->cfg.d_c > 8192) return MLA_ERR_UNSUPPORTED;
   DecodeLayout L = mla_decode_layout(*plan, B, kernel);

@@ -43,6 +43,14 @@ inline __host__ __device__ bool mla_kind_int4(int kind) {
   return kind == MLA_CACHE_INT4_G32 || kind == MLA_CACHE_INT4_G32_R128;
 }
 
+inline __host__ __device__ bool mla_kind_int2(int kind) { return kind == MLA_CACHE_INT2_G32; }
+// Quantised latent (codes + fp16 group scales), and the code width in bits.
+inline __host__ __device__ bool mla_kind_quant(int kind) { return mla_kind_int4(kind) || mla_kind_int2(kind); }
+inline __host__ __device__ int mla_quant_bits(int kind) { return mla_kind_int2(kind) ? 2 : 4; }
+
+// Host validation of a cache view against a config (mla_api.cpp); MLA_OK when usable.
+mla_status_t mla_validate_cache(const mla_config_t& cfg, const mla_cache_t* c);
+
 // Largest token count the decode-step append path takes (its scratch is sized for it).
 constexpr int kAppMaxSmallTokens = 128;
 
@@ -130,6 +138,8 @@ struct Sched {
 DecodeLayout mla_decode_layout(const mla_plan& p, int B, int kernel);
 bool mla_tc_supported(const mla_plan& p, const mla_cache_t& c);
 bool mla_tc_capable(const mla_plan& p);   // shape/dtype allow the tensor-core kernel
+// The tensor-core kernel reads bf16 or int4 latents; the 2-bit cache stays on the CUDA-core kernel.
+inline bool mla_tc_kind_ok(const mla_config_t& c) { return !mla_kind_int2(c.cache_kind); }
 cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B,
                                  const Sched& sched,
                                  const void* qlat, const float* qrope, float* opart, float* mlpart, int P, int G,

@@ -63,6 +63,15 @@ def assert_stored_close(got, exact, dtype: str, what: str = ""):
     return rl
 
 
+def quant_scheme(wl):
+    """(quantise, dequantise, pack, unpack) of the workload's quantised latent cache, or None."""
+    if wl.cache == "int4_g32":
+        return O.quant_int4_g32, O.dequant_int4_g32, O.pack_int4, O.unpack_int4
+    if wl.cache == "int2_g32":
+        return O.quant_int2_g32, O.dequant_int2_g32, O.pack_int2, O.unpack_int2
+    return None
+
+
 class OracleCase:
     """Oracle conversion, cache and reference outputs for one workload (float64)."""
 
@@ -98,9 +107,10 @@ class OracleCase:
         L = x.shape[0]
         c, kr = O.append(x, np.arange(L), cv["W_dkv"], cv["W_krope"], cv["pair_idx"], self.theta)
         out = {"c_exact": c, "kr_exact": kr, "kr": gen.cast(kr, wl.dtype)}
-        if wl.cache == "int4_g32":
-            codes, scales = O.quant_int4_g32(c)
-            deq = O.dequant_int4_g32(codes, scales)
+        qs = quant_scheme(wl)
+        if qs is not None:
+            codes, scales = qs[0](c)
+            deq = qs[1](codes, scales)
             out.update(codes=codes, scales=scales, c=deq)
             if wl.resid:   # the most recent tokens are read unquantised, as stored (dtype)
                 out["c"] = O.residual_window(deq, gen.cast(c, wl.dtype), wl.resid)
@@ -132,8 +142,9 @@ def upload_oracle_cache(case: OracleCase, cache, T_cap):
         if L == 0:
             continue
         cc = case.cache[b]
-        if wl.cache == "int4_g32":
-            cache.set_latent_rows(b, 0, torch.from_numpy(O.pack_int4(cc["codes"])))
+        qs = quant_scheme(wl)
+        if qs is not None:
+            cache.set_latent_rows(b, 0, torch.from_numpy(qs[2](cc["codes"])))
             cache.set_scale_rows(b, 0, torch.from_numpy(cc["scales"]))
             if wl.resid:   # ring slot t % W holds token t for the window's tokens
                 W = cache.c_resid.shape[1]

@@ -111,3 +111,33 @@ def test_fixed_pairs_match_oracle(mla, dh, r):
                           O.fixed_pairs("full", dh, dh // 2, 4).astype(np.int32))
     assert mla.mla_fixed_pairs(cfg, mla.MLA_PAIRS_FULL, check=False) is None     # r != d_h / 2
     assert mla.mla_fixed_pairs(cfg, 3, check=False) is None                      # unknown strategy
+
+
+def test_int2_and_residual_window_configs(mla):
+    """2-bit cache accounting (d_c/4 code bytes + one fp16 scale per 32 + RoPE dims), the
+    int2/int4 dtype rule, and the binding's cache-kind mapping."""
+    import pytest
+    c2 = mla.make_config(4096, 32, 32, 128, 4, 128, cache="int2_g32")
+    assert c2.cache_kind == mla.MLA_CACHE_INT2_G32
+    assert mla.mla_cache_bytes_per_token(c2) == 128 // 4 + 2 * (128 // 32) + 32 * 8 * 2
+    c4r = mla.make_config(4096, 32, 32, 128, 4, 128, cache="int4_g32", resid=128)
+    assert c4r.cache_kind == mla.MLA_CACHE_INT4_G32_R128
+    assert mla.mla_cache_bytes_per_token(c4r) == 128 // 2 + 2 * (128 // 32) + 32 * 8 * 2
+    out = ctypes.c_void_p()
+    f32_int2 = mla.make_config(512, 8, 4, 64, 4, 64, dtype="f32", cache="int2_g32")
+    st = mla._lib.mla_plan_create(ctypes.byref(f32_int2), None, None, None, None, None, ctypes.byref(out))
+    assert st == mla.MLA_ERR_UNSUPPORTED
+    with pytest.raises(ValueError):
+        mla.make_config(512, 8, 4, 64, 4, 64, cache="int2_g32", resid=128)
+    with pytest.raises(ValueError):
+        mla.make_config(512, 8, 4, 64, 4, 64, cache="int4_g32", resid=64)
+
+
+def test_cache_view_layout_matches_header(mla):
+    """The ctypes mirror of mla_cache_t: field order and offsets of the C struct
+    (three pointers, two int32, two pointers, a pointer and an int32)."""
+    C = mla.MlaCache
+    offs = {name: getattr(C, name).offset for name, _ in C._fields_}
+    assert offs == {"c_kv": 0, "c_scales": 8, "k_rope": 16, "B": 24, "T_cap": 28, "c_resid": 32,
+                    "resid_pos": 40, "block_table": 48, "n_blocks": 56}
+    assert ctypes.sizeof(C) == 64

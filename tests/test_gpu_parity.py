@@ -11,7 +11,8 @@ import pytest
 import torch
 
 import oracle as O
-from tests.helpers import OracleCase, assert_close, assert_stored_close, plan_inputs, upload_oracle_cache
+from tests.helpers import (OracleCase, assert_close, assert_stored_close, plan_inputs, quant_scheme,
+                           upload_oracle_cache)
 from workloads import PARITY_WORKLOADS, generate as gen
 
 pytestmark = pytest.mark.gpu
@@ -100,11 +101,12 @@ def test_append_parity(wl):
         cc = case.cache[b]
         kr = cache.k_rope_tokens(b, 0, L).double().cpu().numpy()
         assert_stored_close(kr, cc["kr_exact"], wl.dtype, f"k_rope seq {b}")
-        if wl.cache == "int4_g32":
-            codes = O.unpack_int4(cache.latent_rows(b, 0, L).cpu().numpy())
+        qs = quant_scheme(wl)
+        if qs is not None:
+            codes = qs[3](cache.latent_rows(b, 0, L).cpu().numpy())
             scales = cache.scale_rows(b, 0, L).cpu().numpy()
-            deq = O.dequant_int4_g32(codes, scales)
-            assert_close(deq, O.dequant_int4_g32(cc["codes"], cc["scales"]), wl.dtype, f"int4 latent seq {b}")
+            deq = qs[1](codes, scales)
+            assert_close(deq, qs[1](cc["codes"], cc["scales"]), wl.dtype, f"{wl.cache} latent seq {b}")
             # codes differ only where the float32 latents straddle a rounding boundary
             assert np.mean(codes != cc["codes"]) < 1e-3
             if wl.resid:
@@ -132,11 +134,12 @@ def test_append_decode_step_batch(wl):
         cc = case.cache[b]
         assert_stored_close(cache.k_rope_tokens(b, p_, p_ + 1)[0].double().cpu().numpy(), cc["kr_exact"][p_],
                             wl.dtype, f"kr {b}")
-        if wl.cache == "int4_g32":
-            codes = O.unpack_int4(cache.latent_rows(b, p_, p_ + 1).cpu().numpy())
-            deq = O.dequant_int4_g32(codes, cache.scale_rows(b, p_, p_ + 1).cpu().numpy())
-            assert_close(deq[0], O.dequant_int4_g32(cc["codes"][p_:p_ + 1], cc["scales"][p_:p_ + 1])[0],
-                         wl.dtype, f"int4 latent {b}")
+        qs = quant_scheme(wl)
+        if qs is not None:
+            codes = qs[3](cache.latent_rows(b, p_, p_ + 1).cpu().numpy())
+            deq = qs[1](codes, cache.scale_rows(b, p_, p_ + 1).cpu().numpy())
+            assert_close(deq[0], qs[1](cc["codes"][p_:p_ + 1], cc["scales"][p_:p_ + 1])[0],
+                         wl.dtype, f"{wl.cache} latent {b}")
             if wl.resid:   # only the appended token's slot is claimed and written
                 W = cache.resid_pos.shape[1]
                 tags = cache.resid_pos[b].cpu().numpy()
@@ -202,10 +205,14 @@ def test_residual_window_slides_with_decode_steps(wl):
     _check_ring(cache, 0, L_end, cc["c_exact"], wl)
 
 
-def test_append_int4_codes_bit_exact_on_exact_latents():
+QUANT_WORKLOADS = [w for w in PARITY_WORKLOADS if w.cache != "same" and not w.resid]
+
+
+@pytest.mark.parametrize("wl", QUANT_WORKLOADS, ids=[w.name for w in QUANT_WORKLOADS])
+def test_append_quant_codes_bit_exact_on_exact_latents(wl):
     """One-hot tokens make c = a row of W_dkv exactly; codes and scales must match bit for bit."""
-    wl = PARITY_WORKLOADS[4]
     case = case_for(wl)
+    quant, _, pack, _ = quant_scheme(wl)
     cfg, plan = make_plan(case)
     n = 64
     x = np.zeros((n, wl.hidden))
@@ -216,8 +223,8 @@ def test_append_int4_codes_bit_exact_on_exact_latents():
                    torch.arange(n, dtype=torch.int32, device="cuda"), cache.struct)
     torch.cuda.synchronize()
     c = case.conv["W_dkv"][rows]
-    codes_ref, scales_ref = O.quant_int4_g32(c)
-    np.testing.assert_array_equal(cache.c_kv[0].cpu().numpy(), O.pack_int4(codes_ref))
+    codes_ref, scales_ref = quant(c)
+    np.testing.assert_array_equal(cache.c_kv[0].cpu().numpy(), pack(codes_ref))
     np.testing.assert_array_equal(cache.c_scales[0].cpu().numpy().view(np.uint16), scales_ref.view(np.uint16))
 
 
@@ -228,11 +235,11 @@ def test_decode_parity(wl, kernel):
     """kernel 0: the plan's choice; 1: CUDA-core split-K; 2: tcgen05 (bf16, 32 heads)."""
     case = case_for(wl)
     cfg, plan = make_plan(case, kernel=kernel)
-    if kernel == 2 and (wl.dtype == "f32" or wl.n_heads != 32):
+    if kernel == 2 and (wl.dtype == "f32" or wl.n_heads != 32 or wl.cache == "int2_g32"):
         with pytest.raises(mla.MlaError) as ei:
             run_decode(case, plan, cfg)
         assert ei.value.status == mla.MLA_ERR_UNSUPPORTED
-        pytest.skip("shape outside the tensor-core kernel (fp32 or H != 32)")
+        pytest.skip("outside the tensor-core kernel (fp32, H != 32 or the 2-bit cache)")
     got = run_decode(case, plan, cfg)
     assert mla.mla_device_error(plan) == 0
     for b in case.seqs:
@@ -365,7 +372,7 @@ def _paged_cache(cfg, B, lens, seed, spare=3):
 
 
 PAGED = [PARITY_WORKLOADS[0], PARITY_WORKLOADS[1], PARITY_WORKLOADS[2], PARITY_WORKLOADS[3],
-         PARITY_WORKLOADS[4]] + RESID_WORKLOADS
+         PARITY_WORKLOADS[4]] + RESID_WORKLOADS + [w for w in PARITY_WORKLOADS if w.cache == "int2_g32"]
 
 
 @pytest.mark.parametrize("wl", PAGED, ids=[w.name for w in PAGED])
@@ -409,8 +416,8 @@ def test_paged_append_matches_contiguous(wl):
 def test_paged_decode_parity(wl, kernel):
     """Decode over a paged cache (shuffled blocks) equals the decode over the contiguous
     cache bit for bit, and the oracle within tolerance."""
-    if kernel == 2 and (wl.dtype == "f32" or wl.n_heads != 32):
-        pytest.skip("shape outside the tensor-core kernel (fp32 or H != 32)")
+    if kernel == 2 and (wl.dtype == "f32" or wl.n_heads != 32 or wl.cache == "int2_g32"):
+        pytest.skip("outside the tensor-core kernel (fp32, H != 32 or the 2-bit cache)")
     case = case_for(wl)
     cfg, plan = make_plan(case, kernel=kernel)
     lens = [int(L) for L in case.lens]

@@ -66,3 +66,31 @@ def test_noalloc_rejects_a_batch_beyond_the_scratch():
     st = mla.mla_decode_noalloc(plan, cache.struct, seq, q, out, check=False)
     assert st == mla.MLA_ERR_WORKSPACE_TOO_SMALL
     plan.close()
+
+
+def test_noalloc_validates_the_cache_view_like_decode():
+    """The same cache-view checks as mla_decode, before anything is launched: a paged view
+    whose capacity is not a whole number of 128-token blocks, a block table without a pool
+    size, and a residual-window field on a cache kind without a window are all refused."""
+    import mha_mla_latent_b200 as mla
+    from mha_mla_latent_b200 import _lib
+    from mha_mla_latent_b200.cache import LatentCache
+
+    wl = PARITY_WORKLOADS[2]
+    case = OracleCase(wl, seqs=[])
+    cfg = mla.config_from_workload(wl)
+    plan = mla.mla_plan_create(cfg, **plan_inputs(case))
+    cache = LatentCache(cfg, 2, 256, "cuda")
+    table = torch.zeros(2, 2, dtype=torch.int32, device="cuda")
+    seq = torch.ones(2, dtype=torch.int32, device="cuda")
+    q = torch.zeros(2, wl.n_heads, wl.head_dim, dtype=gen.torch_dtype(wl.dtype), device="cuda")
+    out = torch.empty_like(q)
+    ring = torch.zeros(2, 128, wl.d_c, dtype=gen.torch_dtype(wl.dtype), device="cuda")
+    bad = [
+        _lib.cache_struct(cache.c_kv, None, cache.k_rope, 2, 200, block_table=table, n_blocks=4),
+        _lib.cache_struct(cache.c_kv, None, cache.k_rope, 2, 256, block_table=table, n_blocks=0),
+        _lib.cache_struct(cache.c_kv, None, cache.k_rope, 2, 256, c_resid=ring),
+    ]
+    for view in bad:
+        assert mla.mla_decode_noalloc(plan, view, seq, q, out, check=False) == mla.MLA_ERR_INVALID_ARG
+    plan.close()

@@ -20,7 +20,7 @@ from typing import Optional, Tuple
 class Workload:
     name: str
     dtype: str                 # arithmetic/storage dtype of weights, activations, cache: "f32" | "bf16"
-    cache: str                 # latent cache encoding: "same" (dtype) | "int4_g32"
+    cache: str                 # latent cache encoding: "same" (dtype) | "int4_g32" | "int2_g32"
     hidden: int                # d
     n_heads: int               # H
     n_kv_heads: int            # n_kv
@@ -86,6 +86,9 @@ PARITY_WORKLOADS = [
                        fixed_lens=(700, 200, 128, 1), t_cal=512, resid=128),
     WORKLOADS[1].with_(name="smollm_int4_r128_small", cache="int4_g32", batch=3, ctx=None,
                        fixed_lens=(300, 129, 5), t_cal=512, resid=128),
+    # the 2-bit latent cache (CUDA-core kernel)
+    WORKLOADS[4].with_(name="llama_int2_small", cache="int2_g32", hidden=512, batch=3, ctx=None,
+                       fixed_lens=(700, 65, 1), t_cal=512),
 ]
 
 # The int4 workload as the pages deploy the 4-bit cache: with a residual window of the 128
