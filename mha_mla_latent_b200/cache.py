@@ -83,6 +83,24 @@ class LatentCache:
     def set_scale_rows(self, b: int, t0: int, values: torch.Tensor) -> None:
         self._set_rows(self.c_scales, b, t0, values)
 
+    def query_view(self, seq_of_query) -> "_lib.MlaCache":
+        """A cache view with one row per query: query j reads sequence seq_of_query[j]'s blocks.
+
+        Many queries of one sequence (a chunk of new tokens, or drafted tokens to verify)
+        then attend causally in a single mla_decode: query j at position p_j is passed with
+        seq_lens[j] = p_j + 1, so it is rotated at p_j and attends over tokens [0, p_j].
+        Needs the paged layout (the table rows alias the sequence's blocks) and no residual
+        window (the ring belongs to a sequence row).  The view holds its own table; keep the
+        returned object alive while the call runs."""
+        if not self.paged or self.c_resid is not None:
+            raise ValueError("query_view needs a paged cache without a residual window")
+        idx = torch.as_tensor(seq_of_query, dtype=torch.long)
+        table = self.block_table[idx.to(self.block_table.device)].contiguous()
+        view = _lib.cache_struct(self.c_kv, self.c_scales, self.k_rope, len(idx), self.T_cap,
+                                 block_table=table, n_blocks=self.n_blocks)
+        view._table_ref = table   # the struct holds a raw pointer
+        return view
+
     def reset_sequence(self, b: int) -> None:
         """Forget sequence b's residual window before a new sequence takes slot b."""
         if self.resid_pos is not None:

@@ -447,3 +447,36 @@ def test_paged_block_outside_pool_is_flagged():
         mla.mla_append(plan, x, torch.zeros(1, dtype=torch.int32, device="cuda"),
                        torch.zeros(1, dtype=torch.int32, device="cuda"), paged.struct)
         assert mla.mla_device_error(plan) & mla.MLA_DEVERR_BLOCK
+
+
+# --------------------------------------------------------------------------- many queries per sequence
+@pytest.mark.parametrize("wl,kernel", [(PARITY_WORKLOADS[2], 2), (PARITY_WORKLOADS[2], 1),
+                                       (PARITY_WORKLOADS[1], 1), (PARITY_WORKLOADS[4], 2)],
+                         ids=["llama_tc", "llama_cuda_core", "smollm_gqa", "int4_tc"])
+def test_multi_query_causal_decode(wl, kernel):
+    """A chunk of Q new tokens of one sequence attends causally in one call: query j, at
+    position p_j, over tokens [0, p_j], through per-query rows of the block table that
+    alias the sequence's blocks (the queries are the chunk tokens' own projections)."""
+    case = case_for(wl)
+    cfg, plan = make_plan(case, kernel=kernel)
+    lens = [int(L) for L in case.lens]
+    b = int(np.argmax(lens))
+    L = lens[b]
+    paged = _paged_cache(cfg, wl.batch, lens, seed=11)
+    upload_oracle_cache(case, paged, paged.T_cap)
+    Q = 12
+    pos = np.arange(L - Q, L)
+    x = case.tokens(b)
+    q = gen.cast((x[pos] @ case.w["W_q"]).reshape(Q, wl.n_heads, wl.head_dim), wl.dtype)
+    view = paged.query_view([b] * Q)
+    out = torch.empty(Q, wl.n_heads, wl.head_dim, dtype=gen.torch_dtype(wl.dtype), device="cuda")
+    mla.mla_decode(plan, view, torch.tensor(pos + 1, dtype=torch.int32, device="cuda"),
+                   gen.to_torch(q, wl.dtype, "cuda"), out, workspace(plan, Q, "cuda"))
+    torch.cuda.synchronize()
+    assert mla.mla_device_error(plan) == 0
+    got = out.double().cpu().numpy()
+    cc = case.cache[b]
+    for j, p in enumerate(pos):
+        ref = O.decode_unabsorbed(q[j], cc["c"][:p + 1], cc["kr"][:p + 1], case.conv["W_uk"], case.conv["W_uv"],
+                                  case.conv["pair_idx"], case.theta)
+        assert_close(got[j], ref, wl.dtype, f"query at position {p}")
