@@ -230,6 +230,19 @@ def measured_peak_hbm():
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s pool figure)"
 
 
+def replica_aggregate(local_ms, tokens_per_rank, world, device):
+    """Whole-job timing of N independent replicas: the slowest rank's time of the timed
+    region (an all-reduce MAX over the process group when world > 1) and the job's value,
+    tokens of all ranks / that time.  Every rank calls it at the same point."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    return max_ms, tokens_per_rank * world / (max_ms * 1e-3)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -372,12 +385,9 @@ def run_ours(args):
     total_ms = start.elapsed_time(end)
     kern_ms = [a.elapsed_time(b) for a, b in ev]
     kern_avg_ms = statistics.mean(kern_ms)
-    t_local = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
-    total_ms = float(t_local.item())
-    ms_per_step = total_ms / K
     tokens = int(np.sum(lens))
+    total_ms, _ = replica_aggregate(total_ms, tokens * K, world, dev)
+    ms_per_step = total_ms / K
     value = tokens * world / (ms_per_step * 1e-3)
 
     # ---- decode-only timing (same inputs, no append) for the whole-decode roofline
@@ -406,10 +416,7 @@ def run_ours(args):
         oh.copy_(out, non_blocking=True)
     e3.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([s3.elapsed_time(e3) / E], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = tokens * world / (float(e2e_ms.item()) * 1e-3)
+    _, e2e_value = replica_aggregate(s3.elapsed_time(e3) / E, tokens, world, dev)
     h2d = xd.numel() * xd.element_size() + q.numel() * q.element_size()
     d2h = out.numel() * out.element_size()
 
