@@ -5,7 +5,7 @@ heads, n_kv KV heads, G = H / n_kv, g(h) = floor(h / G), d_h head dim, r kept
 frequency pairs per KV head, d_c latent width.  Pairs are the 2-D subspaces
 (2k, 2k+1), k = 0 .. d_h/2 - 1.
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * RoPE: interleaved pairs (2k, 2k+1) as the notes write them; frequency
     theta_k = base^(-2k/d_h); 0-based positions; rotation
     (a, b) -> (a cos p*theta - b sin p*theta, a sin p*theta + b cos p*theta).

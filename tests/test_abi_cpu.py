@@ -141,3 +141,23 @@ def test_cache_view_layout_matches_header(mla):
     assert offs == {"c_kv": 0, "c_scales": 8, "k_rope": 16, "B": 24, "T_cap": 28, "c_resid": 32,
                     "resid_pos": 40, "block_table": 48, "n_blocks": 56}
     assert ctypes.sizeof(C) == 64
+
+
+def test_binding_constants_match_the_header(mla):
+    """Every enumerator and #define value of include/mla_api.h that the binding mirrors
+    carries the same value on both sides (an ABI drift check)."""
+    text = open(HEADER).read()
+    body = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    values = {}
+    for m in re.finditer(r"\b(MLA_[A-Z0-9_]+)\s*=\s*(\d+)", body):
+        values[m.group(1)] = int(m.group(2))
+    for m in re.finditer(r"#define\s+(MLA_[A-Z0-9_]+)\s+\(?(\d+)u?\s*(?:<<\s*(\d+))?\)?", body):
+        v = int(m.group(2))
+        values[m.group(1)] = v << int(m.group(3)) if m.group(3) else v
+    mirrored = [n for n in values if hasattr(mla, n)]
+    assert len(mirrored) >= 25, mirrored
+    for n in mirrored:
+        assert getattr(mla, n) == values[n], (n, getattr(mla, n), values[n])
+    for n in ("MLA_CACHE_INT2_G32", "MLA_CACHE_INT4_G32_R128", "MLA_RESID_WINDOW", "MLA_BLOCK_TOKENS",
+              "MLA_DEVERR_BLOCK", "MLA_NOALLOC_SCRATCH_BYTES"):
+        assert n in mirrored, n
