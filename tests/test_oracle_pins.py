@@ -460,6 +460,9 @@ def test_T12_int2_hand_derived_codes_and_bytes():
     assert packed[0, 0] == (1 | (3 << 2) | (0 << 4) | (3 << 6))
     assert packed[0, 1] == (0 | (0 << 2) | (0 << 4) | (1 << 6))
     np.testing.assert_array_equal(O.unpack_int2(packed), codes)
+    # every 2-bit field value, two's complement: 00 -> 0, 01 -> 1, 11 -> -1, 10 -> -2
+    byte = np.array([[0b10_11_01_00]], dtype=np.uint8)
+    assert O.unpack_int2(byte)[0].tolist() == [0, 1, -1, -2]
     z, zs = O.quant_int2_g32(np.zeros((2, 64)))
     assert np.all(z == 0) and np.all(zs == 0)
 
