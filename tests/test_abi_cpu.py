@@ -161,3 +161,49 @@ def test_binding_constants_match_the_header(mla):
     for n in ("MLA_CACHE_INT2_G32", "MLA_CACHE_INT4_G32_R128", "MLA_RESID_WINDOW", "MLA_BLOCK_TOKENS",
               "MLA_DEVERR_BLOCK", "MLA_NOALLOC_SCRATCH_BYTES"):
         assert n in mirrored, n
+
+
+def test_cache_accessors_follow_the_documented_layout(mla):
+    """LatentCache's token accessors (used by the parity tests to read and write the cache)
+    against the layout mla_cache_t documents, on CPU tensors: contiguous rows [b][t], paged
+    rows [block_table[b][t/128]][t%128], RoPE keys at
+    ((pb*ceil(cap/32) + pt/32)*n_kv + g)*32*2r + (pt%32)*2r + j."""
+    from mha_mla_latent_b200.cache import LatentCache
+    import torch
+    cfg = mla.make_config(256, 8, 4, 32, 2, 64, cache="int4_g32", resid=128)
+    n_kv, r2, B = 4, 4, 3
+    table = np.array([[5, 0, 2], [1, 4, 3], [6, 6, 6]], dtype=np.int32)
+    caches = {"flat": LatentCache(cfg, B, 384, "cpu"),
+              "paged": LatentCache(cfg, B, 384, "cpu", block_table=table, n_blocks=7)}
+    rng = np.random.default_rng(1)
+    for kind, c in caches.items():
+        b, t0, n = 1, 100, 200                       # crosses the 128-token block boundary
+        kr = torch.from_numpy(rng.standard_normal((n, n_kv, r2)).astype(np.float32))
+        codes = torch.from_numpy(rng.integers(0, 256, size=(n, 32), dtype=np.uint8))
+        c.set_k_rope_tokens(b, t0, kr)
+        c.set_latent_rows(b, t0, codes)
+        assert torch.equal(c.latent_rows(b, t0, t0 + n), codes)
+        np.testing.assert_array_equal(c.k_rope_tokens(b, t0, t0 + n).float().numpy(),
+                                      kr.to(torch.bfloat16).float().numpy())
+        flat_kr = c.k_rope.reshape(-1).float().numpy()
+        flat_c = c.c_kv.reshape(-1, 32).numpy()
+        for i in (0, 27, 28, 150, 199):
+            t = t0 + i
+            if kind == "flat":
+                pb, pt, cap = b, t, 384
+            else:
+                pb, pt, cap = int(table[b][t // 128]), t % 128, 128
+            np.testing.assert_array_equal(flat_c[pb * cap + pt], codes[i].numpy())
+            for g in range(n_kv):
+                for j in range(r2):
+                    off = ((pb * ((cap + 31) // 32) + pt // 32) * n_kv + g) * 32 * r2 + (pt % 32) * r2 + j
+                    assert flat_kr[off] == float(kr[i, g, j].to(torch.bfloat16))
+    # per-query views alias a sequence's table row and keep the pool (no residual window:
+    # its ring belongs to a sequence row)
+    with pytest.raises(ValueError):
+        caches["paged"].query_view([1])
+    plain = LatentCache(mla.make_config(256, 8, 4, 32, 2, 64, cache="int4_g32"), B, 384, "cpu",
+                        block_table=table, n_blocks=7)
+    v = plain.query_view([1, 1, 0])
+    assert v.B == 3 and v.n_blocks == 7 and v.T_cap == 384
+    assert v._table_ref.tolist() == [table[1].tolist(), table[1].tolist(), table[0].tolist()]
