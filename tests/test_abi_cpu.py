@@ -207,3 +207,23 @@ def test_cache_accessors_follow_the_documented_layout(mla):
     v = plain.query_view([1, 1, 0])
     assert v.B == 3 and v.n_blocks == 7 and v.T_cap == 384
     assert v._table_ref.tolist() == [table[1].tolist(), table[1].tolist(), table[0].tolist()]
+
+
+def test_plain_c_host_program_links_and_runs(mla, tmp_path):
+    """The boundary is a C ABI: a C99 program built with gcc -Wall -Werror against
+    include/mla_api.h links the library and gets the documented results from the entry
+    points that need no GPU."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = os.path.join(ROOT, "tests", "c_abi", "abi_host.c")
+    exe = str(tmp_path / "abi_host")
+    libdir = os.path.dirname(mla.LIB_PATH)
+    name = os.path.basename(mla.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), src,
+                    "-o", exe, "-L", libdir, f"-l:{name}", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "0 failed" in r.stdout
