@@ -33,18 +33,21 @@ METRIC = "MLA decode cached tokens/s (batch×ctx per step) and % of B200 HBM pea
 UNIT = "cached tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+PER_WORKLOADS = ("llama2_7b_ragged_bf16", "llama2_7b_int4", "llama2_7b_int4_r128")
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama2_7b_bf16")
     ap.add_argument("--kernel", type=int, default=0, help="decode kernel: 0 auto, 1 CUDA-core, 2 tcgen05")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--no-per-workload", dest="per_workload", action="store_false",
+                    help="measure only --workload (default: also the ragged and int4 workloads at N=1)")
     return ap.parse_args()
 
 
@@ -243,6 +246,204 @@ def replica_aggregate(local_ms, tokens_per_rank, world, device):
     return max_ms, tokens_per_rank * world / (max_ms * 1e-3)
 
 
+class Bench:
+    """One workload set up on one GPU: the converted plan, cache replicas that together
+    exceed twice the L2, the step's inputs, and the measurements of one step."""
+
+    def __init__(self, name, dev, kernel=0):
+        import torch
+        import mha_mla_latent_b200 as mla
+        from mha_mla_latent_b200.cache import LatentCache, workspace
+        from mha_mla_latent_b200.convert import convert_layer, plan_from_converted
+        from workloads import generate as gen
+
+        self.mla, self.torch = mla, torch
+        wl = self.wl = workload(name)
+        self.dev = dev
+        cfg = self.cfg = mla.config_from_workload(wl)
+        lens = self.lens = gen.seq_lens(wl)
+        B = wl.batch
+        # ---- conversion (once): GPU pair selection + device SVD
+        t0 = time.perf_counter()
+        w = gen.layer_weights(wl)
+        q_cal, k_cal = gen.calib_activations(wl, w)
+        conv = convert_layer(cfg, gen.to_torch(w["W_k"], wl.dtype, dev), gen.to_torch(w["W_v"], wl.dtype, dev),
+                             gen.to_torch(q_cal, wl.dtype, dev), gen.to_torch(k_cal, wl.dtype, dev))
+        self.plan = plan = plan_from_converted(cfg, conv)
+        torch.cuda.synchronize()
+        self.conversion_s = time.perf_counter() - t0
+
+        # ---- caches: enough replicas that consecutive steps never hit L2 from the previous one
+        per_tok = mla.mla_cache_bytes_per_token(cfg)
+        cache_bytes = int(np.sum(lens)) * per_tok
+        if wl.resid:   # + the window's ring rows (dtype) and their position tags
+            cache_bytes += int(np.sum(np.minimum(lens, wl.resid))) * (wl.d_c * 2 + 4)
+        self.cache_bytes = cache_bytes
+        self.n_rep = n_rep = max(1, -(-2 * L2_BYTES // cache_bytes))
+        T_cap = int(lens.max())
+        T_cap += T_cap % 2
+        self.caches = caches = [LatentCache(cfg, B, T_cap, dev) for _ in range(n_rep)]
+        t0 = time.perf_counter()
+        chunk = 16384
+        for b in range(B):
+            L = int(lens[b])
+            ctx = gen.context_tokens(wl, b, L - 1)
+            for s in range(0, L - 1, chunk):
+                e = min(L - 1, s + chunk)
+                xt = gen.to_torch(ctx[s:e], wl.dtype, dev)
+                mla.mla_append(plan, xt, torch.full((e - s,), b, dtype=torch.int32, device=dev),
+                               torch.arange(s, e, dtype=torch.int32, device=dev), caches[0].struct)
+        torch.cuda.synchronize()
+        for c in caches[1:]:
+            for name_ in ("c_kv", "c_scales", "k_rope", "c_resid", "resid_pos"):
+                src, dst = getattr(caches[0], name_), getattr(c, name_)
+                if src is not None:
+                    dst.copy_(src)
+        self.prefill_s = time.perf_counter() - t0
+        assert mla.mla_device_error(plan) == 0
+
+        # ---- step inputs
+        self.xd = gen.to_torch(gen.decode_tokens(wl), wl.dtype, dev)
+        self.q = gen.to_torch(gen.decode_queries(wl, w), wl.dtype, dev)
+        self.seq_idx = torch.arange(B, dtype=torch.int32, device=dev)
+        self.pos = torch.tensor(lens - 1, dtype=torch.int32, device=dev)
+        self.seq_lens = torch.tensor(lens, dtype=torch.int32, device=dev)
+        self.out = torch.empty_like(self.q)
+        self.ws = workspace(plan, B, dev)
+        self.stream = torch.cuda.current_stream(dev)
+
+        # which split-K kernel runs: the tcgen05 kernel where the shape allows it
+        kernel_used = kernel
+        if kernel_used == 0:
+            mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, 2)
+            st = mla.mla_decode(plan, caches[0].struct, self.seq_lens, self.q, self.out, self.ws,
+                                stream=self.stream, check=False)
+            kernel_used = 2 if st == mla.MLA_OK else 1
+        self.kernel_used = kernel_used
+        mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, kernel_used)
+        torch.cuda.synchronize()
+        assert mla.mla_device_error(plan) == 0
+        self.tokens = int(np.sum(lens))
+        # append, absorb(+schedule), split-K attention, combine(+W_uv); + the ring-slot claim
+        self.launches_per_step = 4 + (1 if wl.resid else 0)
+
+    def step(self, i):
+        c = self.caches[i % self.n_rep].struct
+        self.mla.mla_append(self.plan, self.xd, self.seq_idx, self.pos, c, stream=self.stream)
+        self.mla.mla_decode(self.plan, c, self.seq_lens, self.q, self.out, self.ws, stream=self.stream)
+
+    def timed_steps(self, K, world=1, sampler=None):
+        """ms per step over K steps (device time, CUDA events on the launching stream), the
+        clocks sampled during the region; nothing but the steps is enqueued inside it."""
+        torch = self.torch
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if sampler:
+            sampler.start()
+        # keep the GPU under the same load for ~1.5 s before the timed region so that the
+        # 100 ms clock samples cover the timed region and its steady state
+        t_soak = time.perf_counter()
+        i = 0
+        while time.perf_counter() - t_soak < 1.5:
+            self.step(i)
+            i += 1
+            if i % 64 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+        start.record(self.stream)
+        for i in range(K):
+            self.step(i)
+        end.record(self.stream)
+        torch.cuda.synchronize()
+        clocks = sampler.stop() if sampler else None
+        dev_err = self.mla.mla_device_error(self.plan)
+        if dev_err:
+            raise RuntimeError(f"device error word {dev_err} after the timed region: result invalid")
+        return start.elapsed_time(end) / K, clocks
+
+    def kernel_times(self, K):
+        """Average ms of each kernel of the step, from events the library records right
+        around each launch on its stream (MLA_OPT_PROFILE_KERNELS).  The events keep the
+        kernels from overlapping, so these run in a separate loop from the timed steps."""
+        import ctypes
+        torch, mla = self.torch, self.mla
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)]
+        for row in ev:
+            for e in row:
+                e.record(self.stream)
+        handles = [(ctypes.c_void_p * 8)(*[e.cuda_event for e in row]) for row in ev]
+        torch.cuda.synchronize()
+        for i in range(K):
+            mla.mla_plan_set_option(self.plan, mla.MLA_OPT_PROFILE_KERNELS, ctypes.addressof(handles[i]))
+            self.step(i)
+        torch.cuda.synchronize()
+        mla.mla_plan_set_option(self.plan, mla.MLA_OPT_PROFILE_KERNELS, 0)
+        names = ("append", "absorb", "attention", "combine")
+        return {n: statistics.mean(ev[i][2 * k].elapsed_time(ev[i][2 * k + 1]) for i in range(K))
+                for k, n in enumerate(names)}
+
+    def decode_only_ms(self, K):
+        torch = self.torch
+        torch.cuda.synchronize()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(self.stream)
+        for i in range(K):
+            self.mla.mla_decode(self.plan, self.caches[i % self.n_rep].struct, self.seq_lens, self.q, self.out,
+                                self.ws, stream=self.stream)
+        e2.record(self.stream)
+        torch.cuda.synchronize()
+        return s2.elapsed_time(e2) / K
+
+    def e2e(self, E):
+        """The same step end to end through the public API with host buffers: pinned host
+        x and q copied in and the output read back inside the timed region, every step."""
+        torch = self.torch
+        xh = self.xd.cpu().pin_memory()
+        qh = self.q.cpu().pin_memory()
+        oh = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        torch.cuda.synchronize()
+        s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s3.record(self.stream)
+        for i in range(E):
+            self.xd.copy_(xh, non_blocking=True)
+            self.q.copy_(qh, non_blocking=True)
+            self.step(i)
+            oh.copy_(self.out, non_blocking=True)
+        e3.record(self.stream)
+        torch.cuda.synchronize()
+        h2d = self.xd.numel() * self.xd.element_size() + self.q.numel() * self.q.element_size()
+        d2h = self.out.numel() * self.out.element_size()
+        return s3.elapsed_time(e3) / E, h2d, d2h
+
+    def roofline(self, attention_ms, workload_name):
+        peak, peak_src = measured_peak_hbm()
+        achieved = self.cache_bytes / (attention_ms * 1e-3) / 1e9
+        kernel_name = ("tcgen05 split-K latent attention (decode_tc_kernel)" if self.kernel_used == 2
+                       else "CUDA-core split-K latent attention (decode_simt_kernel)")
+        return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": measured_traffic(workload_name, self.kernel_used), "kernel": kernel_name,
+                "bytes_per_launch": self.cache_bytes, "avg_launch_ms": attention_ms, "peak_source": peak_src}
+
+    def weight_bytes(self):
+        wl = self.wl
+        eb = 2 if wl.dtype == "bf16" else 4
+        return wl.n_kv_heads * wl.d_c * (wl.head_dim - 2 * wl.r_pairs) * eb + wl.n_kv_heads * wl.d_c * wl.head_dim * eb
+
+    def cpu_baseline(self, seconds_cap):
+        n_tok = int(min(self.lens[0], 4096))
+        times = oracle_decode_sample(self.wl, n_tok, 50, seconds_cap=seconds_cap)
+        return {"value": n_tok / statistics.median(times), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                "sample": f"float64 oracle decode of one query (all {self.wl.n_heads} heads) over "
+                          f"{n_tok} cached tokens, median of {len(times)} runs"}
+
+    def close(self):
+        self.plan.close()
+        self.caches = None
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -257,206 +458,76 @@ def run_ours(args):
 
     from mha_mla_latent_b200 import build
     build.build()
-    import mha_mla_latent_b200 as mla
-    from mha_mla_latent_b200.cache import LatentCache, workspace
-    from mha_mla_latent_b200.convert import convert_layer, plan_from_converted
-    from workloads import generate as gen
 
-    wl = workload(args.workload)
     dev = torch.device("cuda", local)
-    dt = gen.torch_dtype(wl.dtype)
-    cfg = mla.config_from_workload(wl)
-    lens = gen.seq_lens(wl)
-    B = wl.batch
-
-    # ---- conversion (once): GPU pair selection + device SVD
-    t0 = time.perf_counter()
-    w = gen.layer_weights(wl)
-    q_cal, k_cal = gen.calib_activations(wl, w)
-    conv = convert_layer(cfg, gen.to_torch(w["W_k"], wl.dtype, dev), gen.to_torch(w["W_v"], wl.dtype, dev),
-                         gen.to_torch(q_cal, wl.dtype, dev), gen.to_torch(k_cal, wl.dtype, dev))
-    plan = plan_from_converted(cfg, conv)
-    torch.cuda.synchronize()
-    conversion_s = time.perf_counter() - t0
-
-    # ---- caches: enough replicas that consecutive steps never hit L2 from the previous one
-    per_tok = mla.mla_cache_bytes_per_token(cfg)
-    cache_bytes = int(np.sum(lens)) * per_tok
-    if wl.resid:   # + the window's ring rows (dtype) and their position tags
-        cache_bytes += int(np.sum(np.minimum(lens, wl.resid))) * (wl.d_c * 2 + 4)
-    n_rep = max(1, -(-2 * L2_BYTES // cache_bytes))
-    T_cap = int(lens.max())
-    caches = [LatentCache(cfg, B, T_cap, dev) for _ in range(n_rep)]
-    x_dec = gen.decode_tokens(wl)
-    t0 = time.perf_counter()
-    chunk = 16384
-    for b in range(B):
-        L = int(lens[b])
-        ctx = gen.context_tokens(wl, b, L - 1)
-        for s in range(0, L - 1, chunk):
-            e = min(L - 1, s + chunk)
-            xt = gen.to_torch(ctx[s:e], wl.dtype, dev)
-            mla.mla_append(plan, xt, torch.full((e - s,), b, dtype=torch.int32, device=dev),
-                           torch.arange(s, e, dtype=torch.int32, device=dev), caches[0].struct)
-    torch.cuda.synchronize()
-    for c in caches[1:]:
-        c.c_kv.copy_(caches[0].c_kv)
-        if c.c_scales is not None:
-            c.c_scales.copy_(caches[0].c_scales)
-        if c.k_rope is not None:
-            c.k_rope.copy_(caches[0].k_rope)
-        if c.c_resid is not None:
-            c.c_resid.copy_(caches[0].c_resid)
-            c.resid_pos.copy_(caches[0].resid_pos)
-    prefill_s = time.perf_counter() - t0
-    assert mla.mla_device_error(plan) == 0
-
-    # ---- step inputs
-    xd = gen.to_torch(x_dec, wl.dtype, dev)
-    q = gen.to_torch(gen.decode_queries(wl, w), wl.dtype, dev)
-    seq_idx = torch.arange(B, dtype=torch.int32, device=dev)
-    pos = torch.tensor(lens - 1, dtype=torch.int32, device=dev)
-    seq_lens = torch.tensor(lens, dtype=torch.int32, device=dev)
-    out = torch.empty_like(q)
-    ws = workspace(plan, B, dev)
-    stream = torch.cuda.current_stream(dev)
-
-    # which split-K kernel runs: the tcgen05 kernel where the shape allows it
-    kernel_used = args.kernel
-    if kernel_used == 0:
-        mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, 2)
-        st = mla.mla_decode(plan, caches[0].struct, seq_lens, q, out, ws, stream=stream, check=False)
-        kernel_used = 2 if st == mla.MLA_OK else 1
-    mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, kernel_used)
-    torch.cuda.synchronize()
-    assert mla.mla_device_error(plan) == 0
-
-    def step(i):
-        c = caches[i % n_rep].struct
-        mla.mla_append(plan, xd, seq_idx, pos, c, stream=stream)
-        mla.mla_decode(plan, c, seq_lens, q, out, ws, stream=stream)
-
-    # append, absorb(+schedule), split-K attention, combine(+W_uv); + the ring-slot claim
-    launches_per_step = 4 + (1 if wl.resid else 0)
+    bn = Bench(args.workload, dev, args.kernel)
+    wl, K = bn.wl, args.steps
     for i in range(args.warmup):
-        step(i)
+        bn.step(i)
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps, dominant-kernel events recorded on the launching stream
-    import ctypes
-    K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    for a, b in ev:
-        a.record(stream); b.record(stream)
-    handles = [(ctypes.c_void_p * 2)(a.cuda_event, b.cuda_event) for a, b in ev]
-    torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     sampler = ClockSampler(vis.split(",")[local] if vis else local)
-    sampler.start()
-    # keep the GPU under the same load for ~1.5 s before the timed region so that the
-    # 100 ms clock samples cover the timed region and its steady state
-    t_soak = time.perf_counter()
-    i = 0
-    while time.perf_counter() - t_soak < 1.5:
-        step(i)
-        i += 1
-        if i % 64 == 0:
-            torch.cuda.synchronize()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    start.record(stream)
-    for i in range(K):
-        mla.mla_plan_set_option(plan, mla.MLA_OPT_PROFILE_EVENTS, ctypes.addressof(handles[i]))
-        step(i)
-    end.record(stream)
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
-    mla.mla_plan_set_option(plan, mla.MLA_OPT_PROFILE_EVENTS, 0)
-    dev_err = mla.mla_device_error(plan)
-    if dev_err:
-        raise RuntimeError(f"device error word {dev_err} after the timed region: result invalid")
-    if world > 1:
-        dist.barrier()
-    total_ms = start.elapsed_time(end)
-    kern_ms = [a.elapsed_time(b) for a, b in ev]
-    kern_avg_ms = statistics.mean(kern_ms)
-    tokens = int(np.sum(lens))
-    total_ms, _ = replica_aggregate(total_ms, tokens * K, world, dev)
-    ms_per_step = total_ms / K
-    value = tokens * world / (ms_per_step * 1e-3)
-
-    # ---- decode-only timing (same inputs, no append) for the whole-decode roofline
-    torch.cuda.synchronize()
-    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    nd = min(K, 1000)
-    s2.record(stream)
-    for i in range(nd):
-        mla.mla_decode(plan, caches[i % n_rep].struct, seq_lens, q, out, ws, stream=stream)
-    e2.record(stream)
-    torch.cuda.synchronize()
-    decode_ms = s2.elapsed_time(e2) / nd
-
-    # ---- end to end through the public API with host buffers (pinned), copies inside
-    xh = xd.cpu().pin_memory()
-    qh = q.cpu().pin_memory()
-    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    E = args.e2e_steps
-    torch.cuda.synchronize()
-    s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s3.record(stream)
-    for i in range(E):
-        xd.copy_(xh, non_blocking=True)
-        q.copy_(qh, non_blocking=True)
-        step(i)
-        oh.copy_(out, non_blocking=True)
-    e3.record(stream)
-    torch.cuda.synchronize()
-    _, e2e_value = replica_aggregate(s3.elapsed_time(e3) / E, tokens, world, dev)
-    h2d = xd.numel() * xd.element_size() + q.numel() * q.element_size()
-    d2h = out.numel() * out.element_size()
-
-    # ---- roofline of the dominant kernel (split-K attention over the cache)
-    peak, peak_src = measured_peak_hbm()
-    kern_bytes = cache_bytes                      # algorithmic: every cached byte read once
-    achieved = kern_bytes / (kern_avg_ms * 1e-3) / 1e9
-    wuk = wl.n_kv_heads * wl.d_c * (wl.head_dim - 2 * wl.r_pairs) * (2 if wl.dtype == "bf16" else 4)
-    wuv = wl.n_kv_heads * wl.d_c * wl.head_dim * (2 if wl.dtype == "bf16" else 4)
-    decode_frac = (cache_bytes + wuk + wuv) / (decode_ms * 1e-3) / 1e9 / peak
-    kernel_name = ("tcgen05 split-K latent attention (decode_tc_kernel)" if kernel_used == 2
-                   else "CUDA-core split-K latent attention (decode_simt_kernel)")
-
+    local_ms, clocks = bn.timed_steps(K, world, sampler)
+    ms_per_step, value = replica_aggregate(local_ms, bn.tokens, world, dev)
+    kt = bn.kernel_times(K)
+    decode_ms = bn.decode_only_ms(min(K, 1000))
+    e2e_ms, h2d, d2h = bn.e2e(args.e2e_steps)
+    _, e2e_value = replica_aggregate(e2e_ms, bn.tokens, world, dev)
+    peak, _ = measured_peak_hbm()
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype if wl.cache != "int4_g32" else "bf16 (int4 latent cache)",
         "data": "synthetic (seeded generators; random-init layer of the named shape)",
-        "config": dict(wl_config(wl, lens), parallelism=f"replicas x{world}" if world > 1 else "single GPU",
-                       l2=f"{n_rep} cache replicas rotated per step ({n_rep * cache_bytes / 2**20:.0f} MiB > 2x L2)"),
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": measured_traffic(args.workload, kernel_used),
-                     "kernel": kernel_name,
-                     "bytes_per_launch": kern_bytes, "avg_launch_ms": kern_avg_ms, "peak_source": peak_src},
-        "decode_only_ms": decode_ms, "decode_roofline_frac": decode_frac,
+        "config": dict(wl_config(wl, bn.lens), parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                       l2=f"{bn.n_rep} cache replicas rotated per step "
+                          f"({bn.n_rep * bn.cache_bytes / 2**20:.0f} MiB > 2x L2)"),
+        "roofline": bn.roofline(kt["attention"], args.workload),
+        "decode_only_ms": decode_ms,
+        "decode_roofline_frac": (bn.cache_bytes + bn.weight_bytes()) / (decode_ms * 1e-3) / 1e9 / peak,
+        "kernel_ms": kt,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": bn.launches_per_step * K,
         "clocks": clocks,
-        "conversion_s": conversion_s, "prefill_s": prefill_s,
+        "conversion_s": bn.conversion_s, "prefill_s": bn.prefill_s,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_tok = int(min(lens[0], 4096))
-        times = oracle_decode_sample(wl, n_tok, 50, seconds_cap=20.0)
-        cpu_val = n_tok / statistics.median(times)
-        line["cpu_baseline"] = {"value": cpu_val, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                                "sample": f"float64 oracle decode of one query (all {wl.n_heads} heads) over "
-                                          f"{n_tok} cached tokens, median of {len(times)} runs"}
+        line["cpu_baseline"] = bn.cpu_baseline(20.0)
+    bn.close()
+    del bn
+    torch.cuda.empty_cache()
+
+    # the other Llama-2-7B-shaped workloads, measured in the same run on one GPU: the
+    # ragged long-context batch, the int4 latent cache, and the int4 cache with its
+    # 128-token residual window
+    if world == 1 and args.per_workload:
+        per = {}
+        for name in PER_WORKLOADS:
+            if name == args.workload:
+                continue
+            b2 = Bench(name, dev, args.kernel)
+            Kw = max(20, min(K, 500))
+            for i in range(args.warmup):
+                b2.step(i)
+            torch.cuda.synchronize()
+            ms, ck = b2.timed_steps(Kw, 1, ClockSampler(vis.split(",")[local] if vis else local))
+            kt2 = b2.kernel_times(Kw)
+            dms = b2.decode_only_ms(Kw)
+            entry = {"value": b2.tokens / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "steps": Kw,
+                     "config": wl_config(b2.wl, b2.lens), "roofline": b2.roofline(kt2["attention"], name),
+                     "decode_only_ms": dms,
+                     "decode_roofline_frac": (b2.cache_bytes + b2.weight_bytes()) / (dms * 1e-3) / 1e9 / peak,
+                     "kernel_ms": kt2, "clocks": ck}
+            if not args.no_cpu_baseline:
+                entry["cpu_baseline"] = b2.cpu_baseline(5.0)
+            per[name] = entry
+            b2.close()
+            del b2
+            torch.cuda.empty_cache()
+        line["per_workload"] = per
     if rank == 0:
         print(json.dumps(line), flush=True)
-    plan.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

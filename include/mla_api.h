@@ -91,6 +91,7 @@ typedef struct {
   int32_t r_pairs;      /* r, 0 <= r <= d_h/2 */
   int32_t d_c;          /* latent width, multiple of 4 (of 32 for the int4 cache) */
   double rope_base;     /* RoPE base (10000 for the Llama/SmolLM shapes) */
+  float softmax_scale;  /* score scale; 0 = 1/sqrt(d_h), the original layer's (must be >= 0) */
   int32_t dtype;        /* mla_dtype_t */
   int32_t cache_kind;   /* mla_cache_kind_t (the int4 and int2 kinds require dtype MLA_BF16) */
 } mla_config_t;
@@ -140,10 +141,34 @@ enum {
                                  mla_decode records [0] just before and [1] just after its
                                  split-K attention kernel on the call's stream (0 = off).
                                  The array must stay valid while the option is set. */
-  MLA_OPT_OVERLAP_LAUNCH = 4  /* 1 (default): launch the kernels of mla_append / mla_decode
+  MLA_OPT_OVERLAP_LAUNCH = 4, /* 1 (default): launch the kernels of mla_append / mla_decode
                                  with programmatic stream serialization, so each one's
                                  independent prologue (weight loads, set-up) overlaps the
                                  tail of the kernel before it; 0: plain stream order */
+  MLA_OPT_WAIT_LIMIT_US = 5,  /* bound of every pipeline wait of the tensor-core decode
+                                 kernel, in microseconds, 100 .. 10^7 (default 10^6 = 1 s).
+                                 A wait that runs out sets MLA_DEVERR_TIMEOUT; the kernel
+                                 then drains its copies, releases its tensor memory and
+                                 returns, and the decode output of that call is invalid. */
+  MLA_OPT_TEST_SKIP_COPY = 6, /* testing the timeout path only (0 = off, the default): with
+                                 value k > 0 every CTA of the tensor-core kernel leaves out
+                                 the latent copy of its k-th tile, so the waits for that tile
+                                 run out (after MLA_OPT_WAIT_LIMIT_US) and the call reports
+                                 MLA_DEVERR_TIMEOUT.  Nothing faults; later calls with the
+                                 option cleared run normally. */
+  MLA_OPT_PROFILE_KERNELS = 8, /* value: address of a host array of eight cudaEvent_t (0 =
+                                 off); each call records [2k] just before and [2k+1] just
+                                 after its kernel k on the call's stream: k = 0 the append
+                                 kernel (mla_append), 1 the query absorption, 2 the split-K
+                                 attention, 3 the split merge (mla_decode).  Events between
+                                 kernels stop their launches from overlapping, so each
+                                 interval times its kernel alone.  Overrides
+                                 MLA_OPT_PROFILE_EVENTS while set. */
+  MLA_OPT_L2_PREFETCH = 7     /* L2 prefetch lookahead of the tensor-core kernel: the low 8
+                                 bits give how many tiles ahead of its shared-memory copies
+                                 it asks L2 for cache bytes (0 = off, at most 16; default 2);
+                                 bits 8.. select the form when non-zero: 1 line prefetches,
+                                 2 bulk prefetches (default 1). */
 };
 
 MLA_API const char* mla_status_string(mla_status_t s);
@@ -213,7 +238,9 @@ MLA_API mla_status_t mla_plan_set_option(mla_plan_t* plan, int32_t option, int64
 MLA_API mla_status_t mla_append(const mla_plan_t* plan, const void* x, const int32_t* seq_idx,
                         const int32_t* pos, int32_t N, const mla_cache_t* cache, void* stream);
 
-/* Device workspace mla_decode needs for a batch of B sequences (bytes, 256-aligned). */
+/* Device workspace mla_decode, mla_decode_step and mla_decode_step_host need for a batch
+ * of B sequences (bytes, 256-aligned; it includes the host variant's staging of the step's
+ * inputs and output). */
 MLA_API size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B);
 
 /* One decode step: attention of each sequence's new query over its cached tokens
@@ -231,6 +258,35 @@ MLA_API mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache
                         const void* q, int32_t B, void* out, void* workspace, size_t ws_bytes,
                         void* stream);
 
+/* One serving-loop decode step in a single call: the append of every sequence's new
+ * token, then the decode of every sequence's new query.  Token b (row b of x) is the
+ * newest token of sequence b: it is appended at position seq_lens[b] - 1 (the length
+ * already counts it), and query b then attends over tokens [0, seq_lens[b]).  The result
+ * equals mla_append(x, seq_idx = 0..B-1, pos = seq_lens - 1) followed by mla_decode;
+ * the append and the query absorption, which do not depend on each other, run in one
+ * launch (bf16, B <= 128), so a step is three kernels.  Notes §关键设计 (the cache holds
+ * c_kv = x W_dkv and the kept RoPE key dims; decode absorbs W_uk and applies W_uv after
+ * the weighted sum).  With the residual window, each new token claims its ring slot itself.
+ *   seq_lens  device [B] int32, 1 <= L <= T_cap
+ *   x         device [B][d] dtype, the new tokens' hidden states
+ *   q         device [B][H][d_h] dtype, unrotated queries
+ *   out       device [B][H][d_h] dtype
+ *   workspace device, >= mla_decode_workspace_bytes(plan, B) bytes              */
+MLA_API mla_status_t mla_decode_step(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
+                                     const void* x, const void* q, int32_t B, void* out, void* workspace,
+                                     size_t ws_bytes, void* stream);
+
+/* mla_decode_step with the step's inputs and output in HOST memory (page-locked memory
+ * lets the copies run asynchronously): seq_lens [B] int32, x [B][d], q [B][H][d_h] and out
+ * [B][H][d_h] are host pointers; the cache and the workspace are device memory.  The call
+ * enqueues the host-to-device copies of seq_lens, x and q into the workspace, the step's
+ * kernels, and the device-to-host copy of the output, all on `stream`: out is complete
+ * once the stream reaches that point (e.g. after cudaStreamSynchronize).  The host buffers
+ * must stay untouched until then.  workspace >= mla_decode_workspace_bytes(plan, B). */
+MLA_API mla_status_t mla_decode_step_host(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
+                                          const void* x, const void* q, int32_t B, void* out, void* workspace,
+                                          size_t ws_bytes, void* stream);
+
 /* Size of the static scratch array behind mla_decode_noalloc (bytes, per device). */
 #define MLA_NOALLOC_SCRATCH_BYTES (16u << 20)
 
@@ -245,8 +301,10 @@ MLA_API mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache
  * the library until the process exits.
  *   - Returns MLA_ERR_WORKSPACE_TOO_SMALL when the batch needs more workspace than the
  *     array holds (mla_decode_workspace_bytes(plan, B) tells how much a batch needs).
- *   - The first call on a device looks up the array's device address (once per device,
- *     with that device current); make that first call before any stream capture.
+ *   - The first successful call on a device looks up the array's device address (with
+ *     that device current) and keeps it; a failed lookup returns MLA_ERR_CUDA, leaves no
+ *     pending CUDA error behind and is retried by the next call.  Make the first call
+ *     before any stream capture.
  *   - The plan must belong to the current device (MLA_ERR_INVALID_ARG otherwise).
  *   - All calls share the one array and each leaves its contents behind.  Nothing in
  *     it needs clearing: every call writes each part of the workspace before reading it.

@@ -20,6 +20,7 @@ MLA_F32, MLA_BF16 = 0, 1
 MLA_CACHE_SAME, MLA_CACHE_INT4_G32, MLA_CACHE_INT4_G32_R128, MLA_CACHE_INT2_G32 = 0, 1, 2, 3
 MLA_RESID_WINDOW = 128
 MLA_OPT_DECODE_KERNEL, MLA_OPT_DECODE_SPLITS, MLA_OPT_PROFILE_EVENTS, MLA_OPT_OVERLAP_LAUNCH = 1, 2, 3, 4
+MLA_OPT_WAIT_LIMIT_US, MLA_OPT_TEST_SKIP_COPY, MLA_OPT_L2_PREFETCH, MLA_OPT_PROFILE_KERNELS = 5, 6, 7, 8
 MLA_DEVERR_SEQ_LEN, MLA_DEVERR_APPEND_SLOT, MLA_DEVERR_TIMEOUT, MLA_DEVERR_BLOCK = 1, 2, 4, 8
 MLA_BLOCK_TOKENS = 128
 
@@ -27,7 +28,7 @@ EXPORTED = (
     "mla_status_string", "mla_version", "mla_cache_bytes_per_token", "mla_select_pairs",
     "mla_plan_create", "mla_plan_destroy", "mla_plan_set_option", "mla_append",
     "mla_decode_workspace_bytes", "mla_decode", "mla_device_error", "mla_decode_noalloc",
-    "mla_fixed_pairs",
+    "mla_fixed_pairs", "mla_decode_step", "mla_decode_step_host",
 )
 MLA_PAIRS_FULL, MLA_PAIRS_HIGH, MLA_PAIRS_UNIFORM, MLA_PAIRS_LOW = 0, 1, 2, 5
 MLA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -37,8 +38,8 @@ class MlaConfig(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int32), ("n_heads", ctypes.c_int32),
                 ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("r_pairs", ctypes.c_int32), ("d_c", ctypes.c_int32),
-                ("rope_base", ctypes.c_double), ("dtype", ctypes.c_int32),
-                ("cache_kind", ctypes.c_int32)]
+                ("rope_base", ctypes.c_double), ("softmax_scale", ctypes.c_float),
+                ("dtype", ctypes.c_int32), ("cache_kind", ctypes.c_int32)]
 
 
 class MlaCache(ctypes.Structure):
@@ -74,6 +75,8 @@ def _load():
         "mla_decode": (i32, [vp, cachep, vp, vp, i32, vp, vp, sz, vp]),
         "mla_device_error": (i32, [vp, ctypes.POINTER(i32)]),
         "mla_decode_noalloc": (i32, [vp, cachep, vp, vp, i32, vp, vp]),
+        "mla_decode_step": (i32, [vp, cachep, vp, vp, vp, i32, vp, vp, sz, vp]),
+        "mla_decode_step_host": (i32, [vp, cachep, vp, vp, vp, i32, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -113,9 +116,10 @@ def _stream(stream):
 
 
 def make_config(hidden, n_heads, n_kv_heads, head_dim, r_pairs, d_c, rope_base=10000.0,
-                dtype="bf16", cache="same", resid=0) -> MlaConfig:
+                dtype="bf16", cache="same", resid=0, softmax_scale=0.0) -> MlaConfig:
     """cache: "same", "int4_g32" or "int2_g32"; resid: 0, or MLA_RESID_WINDOW for the int4
-    cache with the unquantised residual window (MLA_CACHE_INT4_G32_R128)."""
+    cache with the unquantised residual window (MLA_CACHE_INT4_G32_R128); softmax_scale: 0
+    for 1/sqrt(head_dim)."""
     if cache == "int2_g32":
         if resid:
             raise ValueError("the residual window is built for the int4 cache")
@@ -128,7 +132,7 @@ def make_config(hidden, n_heads, n_kv_heads, head_dim, r_pairs, d_c, rope_base=1
         if resid:
             raise ValueError("the residual window needs the int4 cache")
         kind = MLA_CACHE_SAME
-    return MlaConfig(hidden, n_heads, n_kv_heads, head_dim, r_pairs, d_c, float(rope_base),
+    return MlaConfig(hidden, n_heads, n_kv_heads, head_dim, r_pairs, d_c, float(rope_base), float(softmax_scale),
                      MLA_BF16 if dtype == "bf16" else MLA_F32, kind)
 
 
@@ -225,6 +229,28 @@ def mla_decode(plan: Plan, cache: MlaCache, seq_lens, q, out, workspace, stream=
                          _ptr(out), _ptr(workspace), ws_bytes, _stream(stream))
     if check:
         _check(st, "mla_decode")
+    return st
+
+
+def mla_decode_step(plan: Plan, cache: MlaCache, seq_lens, x, q, out, workspace, stream=None, check=True):
+    """Append every sequence's new token (row b of x at position seq_lens[b]-1 of sequence
+    b) and decode every query, in one call (device tensors)."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _lib.mla_decode_step(plan.handle, ctypes.byref(cache), _ptr(seq_lens), _ptr(x), _ptr(q), int(q.shape[0]),
+                              _ptr(out), _ptr(workspace), ws_bytes, _stream(stream))
+    if check:
+        _check(st, "mla_decode_step")
+    return st
+
+
+def mla_decode_step_host(plan: Plan, cache: MlaCache, seq_lens, x, q, out, workspace, stream=None, check=True):
+    """mla_decode_step with seq_lens, x, q and out in host memory (pinned torch CPU tensors
+    or numpy arrays); the copies in and out are enqueued on the stream with the kernels."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _lib.mla_decode_step_host(plan.handle, ctypes.byref(cache), _ptr(seq_lens), _ptr(x), _ptr(q),
+                                   int(q.shape[0]), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream))
+    if check:
+        _check(st, "mla_decode_step_host")
     return st
 
 

@@ -14,70 +14,12 @@
 
 #include <algorithm>
 
-#include "common.cuh"
-#include "sm100.cuh"
-#include "warp_mma.cuh"
+#include "append_common.cuh"
 
 namespace cg = cooperative_groups;
 
-MLA_KSPAN_DEFINE(append)
 
 namespace mla {
-
-constexpr int kAppTokens = 32;
-constexpr int kAppCols = 64;
-constexpr int kAppK = 32;
-
-struct AppendArgs {
-  const void* x;
-  const void* W;            // [d][ncols]
-  int d, ncols, d_c, R, r, N;
-  const int32_t* seq_idx;
-  const int32_t* pos;
-  mla_cache_t cache;
-  const int32_t* rope_pair;  // [n_kv][r]
-  const double* theta;
-  int32_t* err;
-  int qbits;                // quantised latent (INT4 instantiations): code width, 4 or 2
-  int kslice;               // hidden dims per cluster rank
-  int vec_ok;               // x rows and W rows allow 16-byte vector loads
-};
-
-// Residual window (MLA_CACHE_INT4_G32_R128): the unquantised latent of token (sq, p), in
-// the config dtype (bf16), goes to ring slot p % 128 when the slot is claimed by p (the
-// claim kernel ran first and left there the largest position of the call for the slot).
-__device__ __forceinline__ void resid_store(const mla_cache_t& c, int sq, int p, int d_c, int col, float v) {
-  if (!c.c_resid) return;
-  const size_t rs = (size_t)sq * MLA_RESID_WINDOW + (p & (MLA_RESID_WINDOW - 1));
-  if (c.resid_pos[rs] == p) ((__nv_bfloat16*)c.c_resid)[rs * d_c + col] = __float2bfloat16_rn(v);
-}
-
-// Quantises one group of 32 latent values held one per lane (lane l: element col, the
-// group's start + l) and stores codes and scale at token row `slot`.  4 bits: scale
-// fp16(absmax/7), codes in [-7, 7], two per byte; 2 bits: scale fp16(absmax), codes in
-// [-1, 1], four per byte.  Decisions in float32 (the division correctly rounded).
-__device__ __forceinline__ void quant_group_store(const mla_cache_t& c, size_t slot, int d_c, int col, int lane,
-                                                  float v, int qbits) {
-  float am = fabsf(v);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-  const int qmax = qbits == 4 ? 7 : 1;
-  const __half sh = __float2half_rn(qbits == 4 ? __fdiv_rn(am, 7.0f) : am);
-  const float sc = __half2float(sh);
-  int code = 0;
-  if (sc > 0.f) code = max(-qmax, min(qmax, (int)rintf(__fdiv_rn(v, sc))));
-  if (qbits == 4) {
-    const uint32_t nib = (uint32_t)code & 15u;
-    const uint32_t hi = __shfl_down_sync(0xffffffffu, nib, 1);
-    if ((lane & 1) == 0) ((uint8_t*)c.c_kv)[slot * (d_c / 2) + col / 2] = (uint8_t)(nib | (hi << 4));
-  } else {
-    const uint32_t f = (uint32_t)code & 3u;
-    const uint32_t f1 = __shfl_down_sync(0xffffffffu, f, 1), f2 = __shfl_down_sync(0xffffffffu, f, 2),
-                   f3 = __shfl_down_sync(0xffffffffu, f, 3);
-    if ((lane & 3) == 0) ((uint8_t*)c.c_kv)[slot * (d_c / 4) + col / 4] = (uint8_t)(f | (f1 << 2) | (f2 << 4) | (f3 << 6));
-  }
-  if (lane == 0) ((__half*)c.c_scales)[slot * (d_c / 32) + col / 32] = sh;
-}
 
 // Claims the residual ring slots of a call's tokens: resid_pos[seq][p % 128] becomes the
 // largest position that maps there (an atomic maximum, so the newest token owns the slot
@@ -105,7 +47,8 @@ __device__ void append_epilogue(const AppendArgs& a, const float* tile, int tok0
     const int t = i / (COLS / 2), cp = i % (COLS / 2);
     const int n = tok0 + t, col = col0 + 2 * cp;
     if (n >= a.N || col >= a.ncols) continue;
-    const int sq = a.seq_idx[n], p = a.pos[n];
+    int sq, p;
+    append_slot(a, n, &sq, &p);
     if (sq < 0 || sq >= c.B || p < 0 || p >= c.T_cap) {
       if (col == 0) raise_error(a.err, MLA_DEVERR_APPEND_SLOT);
       continue;
@@ -137,20 +80,21 @@ __device__ void append_epilogue(const AppendArgs& a, const float* tile, int tok0
       const int t = w / (COLS / 32), gi = w % (COLS / 32);
       const int n = tok0 + t, col = col0 + gi * 32 + lane;
       if (n >= a.N || col0 + gi * 32 >= a.d_c) continue;   // whole group outside the latent
-      const int sq = a.seq_idx[n], p = a.pos[n];
+      int sq, p;
+      append_slot(a, n, &sq, &p);
       if (sq < 0 || sq >= c.B || p < 0 || p >= c.T_cap) continue;
       const MlaLoc lc = mla_loc(c, sq, p, a.err);
       const size_t slot = (size_t)lc.pb * lc.cap + lc.pt;
       const float v = tile[t * COLS + gi * 32 + lane];
       quant_group_store(c, slot, a.d_c, col, lane, v, a.qbits);
-      resid_store(c, sq, p, a.d_c, col, v);
+      const bool own = __shfl_sync(0xffffffffu, lane == 0 ? resid_owns(c, sq, p, a.step_lens != nullptr) : false, 0);
+      if (own) resid_store(c, sq, p, a.d_c, col, v);
     }
   }
 }
 
 template <typename T, bool INT4>
 __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
-  MLA_KSPAN(1);
   __shared__ float xs[kAppTokens][kAppK + 1];
   __shared__ __align__(16) float ws[kAppK][kAppCols];
   __shared__ __align__(16) float red[kAppTokens][kAppCols];
@@ -165,6 +109,9 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   const int k_end = min(a.d, k_begin + a.kslice);
   const T* x = (const T*)a.x;
   const T* W = (const T*)a.W;
+  // x and the token slots come from the caller, possibly from the kernel just before
+  pdl_wait();
+  pdl_trigger();
 
   float acc[2][4] = {};
   for (int k0 = k_begin; k0 < k_end; k0 += kAppK) {
@@ -189,8 +136,6 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
     __syncthreads();
   }
 
-  pdl_wait();   // the cache may still be read by the kernel before this one
-  pdl_trigger();
   // Partial tile to shared memory; cluster reduction when the hidden dim is split.
 #pragma unroll
   for (int i = 0; i < 2; ++i)
@@ -220,106 +165,6 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   append_epilogue<T, INT4, kAppTokens, kAppCols>(a, &red[0][0], tok0, col0);
 }
 
-// Decode-step append (few tokens).  The product out[N][ncols] = x W_app is split into
-// 32-token x 32-column tiles and kAppSplit slices of the hidden dim, one CTA each.  A CTA
-// stages its x and W slices in one batch of loads, its eight warps each take an eighth of
-// the slice with 8 x 4 register tiles, and the warps' tiles are summed in shared memory.
-// The slice's partial tile goes to the plan's scratch; the last CTA of a tile to finish
-// (ticket counter) sums the kAppSplit partials in slice order (deterministic) and runs the
-// epilogue, whose per-token and per-column inputs every CTA prefetched at its start.
-constexpr int kSmTok = 32, kSmCols = 32, kAppSplit = 8;
-
-struct AppendSmallArgs {
-  AppendArgs a;
-  float* part;        // [kAppSplit][tiles][32 * 32] partial tiles
-  int32_t* ticket;    // [tiles] arrival counters (the last CTA resets its counter)
-};
-
-// Second half of the decode-step append, after the eight warps' 32 x 32 tiles of this hidden-dim
-// slice are in red[8][32 * 32]: sum them into the slice's partial, and let the last CTA of the
-// tile sum the partials in slice order and write the cache (latent, RoPE keys rotated at the
-// token's position, int4 codes).
-template <typename T, bool INT4>
-__device__ __forceinline__ void append_small_finish(const AppendSmallArgs& sa, float* red, const int* s_sq,
-                                                    const int* s_pos, const double* s_theta, int* s_last,
-                                                    int tok0, int col0, int tile, int ntile, int split) {
-  const AppendArgs& a = sa.a;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // the scratch and the cache may still be in use by the kernels before this one
-  pdl_wait();
-  pdl_trigger();
-  float* my_part = sa.part + ((size_t)split * ntile + tile) * (kSmTok * kSmCols);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int o = tid + 256 * e;
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) v += red[w * kSmTok * kSmCols + o];
-    my_part[o] = v;
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int prev = atomicAdd(sa.ticket + tile, 1);
-    *s_last = prev == kAppSplit - 1;
-    if (*s_last) sa.ticket[tile] = 0;   // ready for the next call
-  }
-  __syncthreads();
-  if (!*s_last) return;
-  __threadfence();
-  // ---- last CTA of the tile: sum the partials in slice order, then the epilogue
-  float* tileb = red;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int o = tid + 256 * e;
-    float v = 0.f;
-    for (int sp = 0; sp < kAppSplit; ++sp) v += __ldcg(sa.part + ((size_t)sp * ntile + tile) * (kSmTok * kSmCols) + o);
-    tileb[o] = v;
-  }
-  __syncthreads();
-  const mla_cache_t& c = a.cache;
-  const int n_kv = a.R / max(2 * a.r, 1);
-  for (int i = tid; i < kSmTok * (kSmCols / 2); i += 256) {
-    const int t = i / (kSmCols / 2), cp = i % (kSmCols / 2);
-    const int n = tok0 + t, col = col0 + 2 * cp;
-    if (n >= a.N || col >= a.ncols) continue;
-    const int sq = s_sq[t], p = s_pos[t];
-    if (sq < 0 || sq >= c.B || p < 0 || p >= c.T_cap) {
-      if (col == 0) raise_error(a.err, MLA_DEVERR_APPEND_SLOT);
-      continue;
-    }
-    const float v0 = tileb[t * kSmCols + 2 * cp], v1 = tileb[t * kSmCols + 2 * cp + 1];
-    const MlaLoc lc = mla_loc(c, sq, p, a.err);
-    if (col < a.d_c) {
-      if (!INT4) {
-        T* dst = (T*)c.c_kv + ((size_t)lc.pb * lc.cap + lc.pt) * a.d_c + col;
-        dst[0] = from_f32<T>(v0);
-        dst[1] = from_f32<T>(v1);
-      }
-    } else {
-      const int rc = col - a.d_c;
-      double sn, cs;
-      sincos((double)p * s_theta[cp], &sn, &cs);
-      T* dst = (T*)c.k_rope + mla_kr_offset(lc.pb, lc.pt, rc / (2 * a.r), rc % (2 * a.r), lc.cap, n_kv, 2 * a.r);
-      dst[0] = from_f64<T>((double)v0 * cs - (double)v1 * sn);
-      dst[1] = from_f64<T>((double)v0 * sn + (double)v1 * cs);
-    }
-  }
-  if (INT4 && col0 < a.d_c) {
-    // one warp per token: the tile's 32 latent columns are one quantisation group
-    for (int t = warp; t < kSmTok; t += 8) {
-      const int n = tok0 + t;
-      const int sq = s_sq[t], p = s_pos[t];
-      if (n >= a.N || sq < 0 || sq >= c.B || p < 0 || p >= c.T_cap) continue;
-      const MlaLoc lc = mla_loc(c, sq, p, a.err);
-      const size_t slot = (size_t)lc.pb * lc.cap + lc.pt;
-      const float v = tileb[t * kSmCols + lane];
-      quant_group_store(c, slot, a.d_c, col0 + lane, lane, v, a.qbits);
-      resid_store(c, sq, p, a.d_c, col0 + lane, v);
-    }
-  }
-}
-
 template <typename T, bool INT4>
 cudaError_t launch_append_t(const AppendArgs& args, int ksplit, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
@@ -339,7 +184,6 @@ cudaError_t launch_append_t(const AppendArgs& args, int ksplit, cudaStream_t s) 
 
 template <typename T, bool INT4>
 __global__ void __launch_bounds__(256) append_small_kernel(AppendSmallArgs sa) {
-  MLA_KSPAN(0);
   const AppendArgs& a = sa.a;
   extern __shared__ __align__(16) float smf[];
   const int ks = a.kslice;                       // multiple of 64
@@ -358,10 +202,11 @@ __global__ void __launch_bounds__(256) append_small_kernel(AppendSmallArgs sa) {
   const T* W = (const T*)a.W;
   constexpr int VEC = 16 / sizeof(T);
   // ---- epilogue inputs (token slots, rotation frequencies), prefetched
+  // the token slots and x come from the caller, possibly from the kernel just before
+  pdl_wait();
+  pdl_trigger();
   if (tid < kSmTok) {
-    const int n = tok0 + tid;
-    s_sq[tid] = n < a.N ? __ldg(a.seq_idx + n) : -1;
-    s_pos[tid] = n < a.N ? __ldg(a.pos + n) : -1;
+    append_slot(a, tok0 + tid, &s_sq[tid], &s_pos[tid]);
   } else if (tid < kSmTok + kSmCols / 2) {
     const int cp = tid - kSmTok, col = col0 + 2 * cp;
     double th = 0.0;
@@ -451,117 +296,10 @@ __global__ void __launch_bounds__(256) append_small_kernel(AppendSmallArgs sa) {
   append_small_finish<T, INT4>(sa, red, s_sq, s_pos, s_theta, &s_last, tok0, col0, tile, ntile, split);
 }
 
-// bf16 form of the decode-step append: the slice product runs on the tensor cores as
-// m16n8k16 warp MMAs from bf16 tiles staged with cp.async (x [32][ks], W [ks][32], rows
-// padded by 16 bytes so the ldmatrix reads are conflict-free); warp w takes hidden dims
-// [w ks/8, (w+1) ks/8) for the whole 32 x 32 tile.
 template <bool INT4>
 __global__ void __launch_bounds__(256) append_small_mma_kernel(AppendSmallArgs sa) {
-  MLA_KSPAN(2);
-  using bf16 = __nv_bfloat16;
-  const AppendArgs& a = sa.a;
   extern __shared__ __align__(16) uint8_t sm8[];
-  const int ks = a.kslice;                       // multiple of 128
-  const int XLD = ks + 8;
-  constexpr int WLD = kSmCols + 8;
-  bf16* xs = reinterpret_cast<bf16*>(sm8);       // [kSmTok][XLD]
-  bf16* wsm = xs + kSmTok * XLD;                 // [ks][WLD]
-  float* red = reinterpret_cast<float*>(sm8);    // [8][kSmTok * kSmCols], after the product
-  __shared__ int s_sq[kSmTok], s_pos[kSmTok];
-  __shared__ double s_theta[kSmCols / 2];
-  __shared__ int s_last;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int col0 = blockIdx.x * kSmCols, tok0 = blockIdx.y * kSmTok;
-  const int split = blockIdx.z;
-  const int tile = blockIdx.y * gridDim.x + blockIdx.x, ntile = gridDim.x * gridDim.y;
-  const int k_begin = split * ks, k_end = min(a.d, k_begin + ks);
-  const bf16* x = (const bf16*)a.x;
-  const bf16* W = (const bf16*)a.W;
-  if (tid < kSmTok) {
-    const int n = tok0 + tid;
-    s_sq[tid] = n < a.N ? __ldg(a.seq_idx + n) : -1;
-    s_pos[tid] = n < a.N ? __ldg(a.pos + n) : -1;
-  } else if (tid < kSmTok + kSmCols / 2) {
-    const int cp = tid - kSmTok, col = col0 + 2 * cp;
-    double th = 0.0;
-    if (col >= a.d_c && col < a.ncols) {
-      const int rc = col - a.d_c, g = rc / (2 * a.r), j = (rc % (2 * a.r)) / 2;
-      th = __ldg(a.theta + __ldg(a.rope_pair + g * a.r + j));
-    }
-    s_theta[cp] = th;
-  }
-  // ---- stage: 16-byte asynchronous copies, all in flight together (missing rows and
-  // columns are zero-filled)
-  {
-    const int nxv = kSmTok * (ks / 8), nwv = ks * (kSmCols / 8);
-    for (int v = tid; v < nxv + nwv; v += 256) {
-      if (v < nxv) {
-        const int t = v / (ks / 8), ch = v % (ks / 8);
-        const int n = tok0 + t, kd = k_begin + ch * 8;
-        const bool ok = n < a.N && kd + 8 <= k_end;
-        sm100::cp_async16(wmma16::smem_addr(xs + t * XLD + ch * 8), ok ? (const void*)(x + (size_t)n * a.d + kd) : a.x,
-                          ok ? 16u : 0u);
-      } else {
-        const int vw = v - nxv;
-        const int kk = vw / (kSmCols / 8), part = vw % (kSmCols / 8);
-        const int kd = k_begin + kk, col = col0 + part * 8;
-        const bool ok = kd < k_end && col + 8 <= a.ncols;
-        sm100::cp_async16(wmma16::smem_addr(wsm + kk * WLD + part * 8),
-                          ok ? (const void*)(W + (size_t)kd * a.ncols + col) : a.W, ok ? 16u : 0u);
-      }
-    }
-    sm100::cp_async_commit();
-    sm100::cp_async_wait_all();
-  }
-  __syncthreads();
-  float acc[2][4][4];
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-  const int kw = ks / 8;
-  for (int k0 = warp * kw; k0 < (warp + 1) * kw; k0 += 16) {
-    uint32_t a0[4], a1[4], b0[4], b1[4];
-    wmma16::load_a(a0, xs, XLD, 0, k0, lane);
-    wmma16::load_a(a1, xs, XLD, 16, k0, lane);
-    wmma16::load_b2(b0, wsm, WLD, k0, 0, lane);
-    wmma16::load_b2(b1, wsm, WLD, k0, 16, lane);
-    wmma16::mma_16816(acc[0][0], a0, b0[0], b0[1]);
-    wmma16::mma_16816(acc[0][1], a0, b0[2], b0[3]);
-    wmma16::mma_16816(acc[0][2], a0, b1[0], b1[1]);
-    wmma16::mma_16816(acc[0][3], a0, b1[2], b1[3]);
-    wmma16::mma_16816(acc[1][0], a1, b0[0], b0[1]);
-    wmma16::mma_16816(acc[1][1], a1, b0[2], b0[3]);
-    wmma16::mma_16816(acc[1][2], a1, b1[0], b1[1]);
-    wmma16::mma_16816(acc[1][3], a1, b1[2], b1[3]);
-  }
-  __syncthreads();   // the staging area is reused for the warps' tiles
-  float* my = red + warp * kSmTok * kSmCols;
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int row = 16 * i + (lane >> 2), col = 8 * j + 2 * (lane & 3);
-      *reinterpret_cast<float2*>(my + row * kSmCols + col) = make_float2(acc[i][j][0], acc[i][j][1]);
-      *reinterpret_cast<float2*>(my + (row + 8) * kSmCols + col) = make_float2(acc[i][j][2], acc[i][j][3]);
-    }
-  __syncthreads();
-  append_small_finish<bf16, INT4>(sa, red, s_sq, s_pos, s_theta, &s_last, tok0, col0, tile, ntile, split);
-}
-
-template <bool INT4>
-cudaError_t launch_append_small_mma(const AppendSmallArgs& sa, cudaStream_t s, bool pdl) {
-  const AppendArgs& a = sa.a;
-  dim3 grid((a.ncols + kSmCols - 1) / kSmCols, (a.N + kSmTok - 1) / kSmTok, kAppSplit);
-  const size_t smem = std::max<size_t>(sizeof(__nv_bfloat16) * ((size_t)kSmTok * (a.kslice + 8) +
-                                                                (size_t)a.kslice * (kSmCols + 8)),
-                                       sizeof(float) * 8 * kSmTok * kSmCols);
-  cudaError_t e = cudaFuncSetAttribute(append_small_mma_kernel<INT4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
-  return mla_launch_kernel(append_small_mma_kernel<INT4>, grid, dim3(256), smem, s, pdl, sa);
+  append_small_mma_body<INT4>(sa, blockIdx.x, blockIdx.y, blockIdx.z, gridDim.x, gridDim.y, sm8);
 }
 
 template <typename T, bool INT4>
@@ -576,32 +314,58 @@ cudaError_t launch_append_small_t(const AppendSmallArgs& sa, size_t smem, cudaSt
 
 }  // namespace mla
 
-cudaError_t mla_launch_append(const mla_plan& p, const void* x, const int32_t* seq_idx,
-                              const int32_t* pos, int N, const mla_cache_t& c, cudaStream_t s) {
-  using namespace mla;
+namespace {
+
+mla::AppendArgs make_append_args(const mla_plan& p, const void* x, int N, const mla_cache_t& c) {
   const mla_config_t& cfg = p.cfg;
-  AppendArgs a;
+  mla::AppendArgs a;
   a.x = x; a.W = p.W_app; a.d = cfg.hidden; a.ncols = p.ncols; a.d_c = cfg.d_c; a.R = p.R;
-  a.r = cfg.r_pairs; a.N = N; a.seq_idx = seq_idx; a.pos = pos; a.cache = c;
-  a.rope_pair = p.rope_pair; a.theta = p.theta; a.err = p.err;
+  a.r = cfg.r_pairs; a.N = N; a.seq_idx = nullptr; a.pos = nullptr; a.cache = c;
+  a.rope_pair = p.rope_pair; a.theta = p.theta; a.err = p.err; a.step_lens = nullptr;
   const size_t eb = cfg.dtype == MLA_BF16 ? 2 : 4;
   a.vec_ok = ((uintptr_t)x % 16 == 0) && ((size_t)cfg.hidden * eb) % 16 == 0 && ((size_t)p.ncols * eb) % 16 == 0;
-  const bool int4 = mla_kind_quant(cfg.cache_kind);   // quantised latent (int4 or int2 codes)
   a.qbits = mla_quant_bits(cfg.cache_kind);
-  if (c.c_resid) {   // residual window: claim the ring slots first
+  a.kslice = 0;
+  return a;
+}
+
+// The bf16 decode-step form (tensor-core slice products, ticket reduction), when it applies.
+bool mma_form(const mla_plan& p, mla::AppendArgs a, mla::AppendSmallArgs* sa, dim3* grid, size_t* smem) {
+  using namespace mla;
+  const mla_config_t& cfg = p.cfg;
+  if (!(a.N <= kAppMaxSmallTokens && p.app_part && p.app_ticket && cfg.dtype == MLA_BF16 && a.vec_ok)) return false;
+  const int ks = (cfg.hidden + kAppSplit - 1) / kAppSplit;
+  a.kslice = (ks + 127) / 128 * 128;
+  if ((size_t)a.kslice * (kSmTok + kSmCols + 16) * 2 > 200 * 1024) return false;
+  sa->a = a;
+  sa->part = p.app_part;
+  sa->ticket = p.app_ticket;
+  *grid = dim3((a.ncols + kSmCols - 1) / kSmCols, (a.N + kSmTok - 1) / kSmTok, kAppSplit);
+  *smem = std::max<size_t>(sizeof(__nv_bfloat16) * ((size_t)kSmTok * (a.kslice + 8) + (size_t)a.kslice * (kSmCols + 8)),
+                           sizeof(float) * 8 * kSmTok * kSmCols);
+  return true;
+}
+
+cudaError_t launch_append_args(const mla_plan& p, mla::AppendArgs a, const mla_cache_t& c, cudaStream_t s) {
+  using namespace mla;
+  const mla_config_t& cfg = p.cfg;
+  const int N = a.N;
+  const bool int4 = mla_kind_quant(cfg.cache_kind);   // quantised latent (int4 or int2 codes)
+  if (c.c_resid && !a.step_lens) {   // residual window: claim the ring slots first
     const int grid = std::max(1, std::min((N + 255) / 256, 4 * p.num_sms));
-    cudaError_t e = mla_launch_kernel(resid_claim_kernel, dim3(grid), dim3(256), 0, s, p.opt_pdl, seq_idx, pos, N, c);
+    cudaError_t e =
+        mla_launch_kernel(resid_claim_kernel, dim3(grid), dim3(256), 0, s, p.opt_pdl, a.seq_idx, a.pos, N, c);
     if (e != cudaSuccess) return e;
   }
-  if (N <= kAppMaxSmallTokens && p.app_part && p.app_ticket && cfg.dtype == MLA_BF16 && a.vec_ok) {
-    int ks = (cfg.hidden + kAppSplit - 1) / kAppSplit;
-    a.kslice = (ks + 127) / 128 * 128;
-    if ((size_t)a.kslice * (kSmTok + kSmCols + 16) * 2 <= 200 * 1024) {
-      AppendSmallArgs sa;
-      sa.a = a;
-      sa.part = p.app_part;
-      sa.ticket = p.app_ticket;
-      return int4 ? launch_append_small_mma<true>(sa, s, p.opt_pdl) : launch_append_small_mma<false>(sa, s, p.opt_pdl);
+  {
+    AppendSmallArgs sa;
+    dim3 grid;
+    size_t smem;
+    if (mma_form(p, a, &sa, &grid, &smem)) {
+      auto kern = int4 ? append_small_mma_kernel<true> : append_small_mma_kernel<false>;
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      return mla_launch_kernel(kern, grid, dim3(256), smem, s, p.opt_pdl, sa);
     }
   }
   if (N <= kAppMaxSmallTokens && p.app_part && p.app_ticket) {
@@ -634,4 +398,28 @@ cudaError_t mla_launch_append(const mla_plan& p, const void* x, const int32_t* s
     return int4 ? launch_append_t<__nv_bfloat16, true>(a, ksplit, s)
                 : launch_append_t<__nv_bfloat16, false>(a, ksplit, s);
   return launch_append_t<float, false>(a, ksplit, s);
+}
+
+}  // namespace
+
+bool mla_append_step_mma_form(const mla_plan& p, const void* x, const int32_t* seq_lens, int B,
+                              const mla_cache_t& c, mla::AppendSmallArgs* sa, dim3* grid, size_t* smem) {
+  mla::AppendArgs a = make_append_args(p, x, B, c);
+  a.step_lens = seq_lens;
+  return mma_form(p, a, sa, grid, smem);
+}
+
+cudaError_t mla_launch_append(const mla_plan& p, const void* x, const int32_t* seq_idx,
+                              const int32_t* pos, int N, const mla_cache_t& c, cudaStream_t s) {
+  mla::AppendArgs a = make_append_args(p, x, N, c);
+  a.seq_idx = seq_idx;
+  a.pos = pos;
+  return launch_append_args(p, a, c, s);
+}
+
+cudaError_t mla_launch_append_step(const mla_plan& p, const void* x, const int32_t* seq_lens, int B,
+                                   const mla_cache_t& c, cudaStream_t s) {
+  mla::AppendArgs a = make_append_args(p, x, B, c);
+  a.step_lens = seq_lens;
+  return launch_append_args(p, a, c, s);
 }

@@ -7,34 +7,6 @@
 
 #include "mla_internal.h"
 
-#ifdef MLA_TC_TRACE
-// Development builds only (-DMLA_TC_TRACE): each CTA's start and end %globaltimer stamps,
-// per kernel id, in a translation-unit-local array with an exported reader.
-#define MLA_KSPAN_DEFINE(name)                                                                  \
-  static __device__ unsigned long long g_kspan[8 * 1024 * 2];                                   \
-  extern "C" __attribute__((visibility("default"))) int mla_kspan_read_##name(unsigned long long* h) { \
-    return cudaMemcpyFromSymbol(h, g_kspan, sizeof(g_kspan)) == cudaSuccess ? 8 * 1024 * 2 : -1;  \
-  }
-#define MLA_KSPAN(k)                                                                            \
-  struct KSpanT {                                                                               \
-    unsigned long long t0;                                                                      \
-    __device__ static unsigned long long now() {                                                \
-      unsigned long long t;                                                                     \
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));                                     \
-      return t;                                                                                 \
-    }                                                                                           \
-    __device__ ~KSpanT() {                                                                      \
-      const int blk = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);           \
-      if (threadIdx.x == 0 && blk < 1024) {                                                     \
-        g_kspan[((k) * 1024 + blk) * 2] = t0;                                                   \
-        g_kspan[((k) * 1024 + blk) * 2 + 1] = now();                                            \
-      }                                                                                         \
-    }                                                                                           \
-  } kspan_{KSpanT::now()}
-#else
-#define MLA_KSPAN_DEFINE(name)
-#define MLA_KSPAN(k) do { } while (0)
-#endif
 
 namespace mla {
 

@@ -7,15 +7,15 @@
 // scores the NoPE part directly against c_kv; the probability-weighted latent is taken
 // through W_uv after the softmax sum.  Scores are kept in log2 units (the query is
 // pre-scaled by log2(e)/sqrt(d_h)) so the softmax uses exp2.
+#include <math.h>
+
 #include <algorithm>
 
+#include "append_common.cuh"
 #include "decode_common.cuh"
-#include "sm100.cuh"
-#include "warp_mma.cuh"
 
 #include <type_traits>
 
-MLA_KSPAN_DEFINE(decode)
 
 namespace mla {
 
@@ -35,30 +35,31 @@ struct AbsorbArgs {
   int tile, G;
   int32_t* err;
   int sched_ints;             // shared memory of the schedule CTA, in ints
+  float sm_scale;             // softmax scale of the scores (1/sqrt(d_h) unless the config sets one)
   int vec_ok;                 // q and W_uk^T rows allow 16-byte loads
 };
 
 constexpr int kAbsRows = 8;    // (b, h) rows per CTA: one per warp in the product
 constexpr int kAbsCols = 64;   // latent columns per CTA: two per lane
 
-// grid: one CTA that builds the split-K schedule (block 0, so it is dispatched first), then
-// n_kv * (row blocks) * (column chunks) CTAs.  A CTA reads everything it needs (its W_uk^T slice, its query rows, the NoPE
-// index table, and for the first column chunk the RoPE tables and positions) in one batch
-// of loads, then q_lat[row][c] = scale * sum_j q[row][nope_j] * W_uk^T[g][j][c] with warp r
-// owning row r and lane l columns 2l, 2l+1 of the chunk.
+// Block `blk` of the absorption grid: block 0 builds the split-K schedule (dispatched
+// first), blocks 1 .. n_kv * (row blocks) * (column chunks) compute q_lat.  A CTA stages
+// what comes from the plan (its W_uk^T slice, the NoPE index table, the RoPE pair table
+// and frequencies) before the dependency wait and the caller's queries and sequence lengths
+// after it, then q_lat[row][c] = scale * sum_j q[row][nope_j] * W_uk^T[g][j][c] with warp r
+// owning row r and lane l columns 2l, 2l+1 of the chunk.  `sm` is the CTA's dynamic shared
+// memory.
 template <typename T>
-__global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
-  MLA_KSPAN(0);
-  extern __shared__ __align__(16) float sm[];
+__device__ __forceinline__ void absorb_body(const AbsorbArgs& a, int blk_id, float* sm) {
   const int G = a.H / a.n_kv;
   const int rows_total = a.B * G;
   const int n_rb = (rows_total + kAbsRows - 1) / kAbsRows;
-  if (blockIdx.x == 0) {  // the split-K schedule
+  if (blk_id == 0) {  // the split-K schedule
     build_schedule(a.seq_lens, a.B, a.T_cap, a.tile, a.G, a.sched, a.err, reinterpret_cast<int32_t*>(sm),
                    a.sched_ints);
     return;
   }
-  const int blk = blockIdx.x - 1;
+  const int blk = blk_id - 1;
   const int g = blk % a.n_kv;
   const int rb = (blk / a.n_kv) % n_rb;
   const int cc = blk / (a.n_kv * n_rb);
@@ -71,37 +72,34 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
   int* s_idx = reinterpret_cast<int*>(s_qn + kAbsRows * dnp);   // [dn]
   const T* q = (const T*)a.q;
   const T* W = (const T*)a.W_ukT + (size_t)g * dn * a.d_c;
-  // ---- loads: W slice, query rows, NoPE indices (inputs and plan tables only)
+  // ---- plan data: W slice, NoPE indices, RoPE pair frequencies
   const int ncol = min(kAbsCols, a.d_c - c0);
   if (ncol < kAbsCols)
     for (int i = tid; i < dn * kAbsCols; i += 256) s_w[i] = 0.f;   // columns past d_c
   stage_rows_f32<T>(s_w, kAbsCols, dn, ncol, a.vec_ok && ncol == kAbsCols,
                     [&](int j) { return W + (size_t)j * a.d_c + c0; });
+  for (int j = tid; j < dn; j += 256) s_idx[j] = __ldg(a.nope_idx + g * dn + j);
+  const float scale = kLog2e * a.sm_scale;
+  const int nrope = (cc == 0) ? kAbsRows * a.r : 0;
+  int rp_k = 0;
+  double rp_th = 0.0;
+  const bool rope_item = tid < nrope && row0 + tid / max(a.r, 1) < rows_total;
+  if (rope_item) {
+    rp_k = __ldg(a.rope_pair + g * a.r + tid % a.r);
+    rp_th = __ldg(a.theta + rp_k);
+  }
+  // ---- the caller's queries and lengths; the outputs are read by the attention kernel of
+  // the previous call until it has finished
+  pdl_wait();
+  pdl_trigger();
   const int nrow = min(kAbsRows, rows_total - row0);
   stage_rows_f32<T>(s_q, dh, nrow, dh, a.vec_ok, [&](int r) {
     const int row = row0 + r;
     return q + ((size_t)(row / G) * a.H + g * G + row % G) * dh;
   });
-  for (int j = tid; j < dn; j += 256) s_idx[j] = __ldg(a.nope_idx + g * dn + j);
-  // RoPE query part (first column chunk): rotate the kept pairs at position L-1 (angle in
-  // double), scale.  Positions and frequencies are loaded in the same batch.
-  const float scale = kLog2e * rsqrtf((float)dh);
-  const int nrope = (cc == 0) ? kAbsRows * a.r : 0;
-  int rp_pos = 0, rp_k = 0;
-  double rp_th = 0.0;
-  const bool rope_item = tid < nrope && row0 + tid / max(a.r, 1) < rows_total;
-  if (rope_item) {
-    const int r = tid / a.r, row = row0 + r;
-    rp_k = __ldg(a.rope_pair + g * a.r + tid % a.r);
-    rp_th = __ldg(a.theta + rp_k);
-    rp_pos = __ldg(a.seq_lens + row / G);
-  }
+  const int rp_pos = rope_item ? __ldg(a.seq_lens + (row0 + tid / a.r) / G) : 0;
   __syncthreads();
   for (int i = tid; i < kAbsRows * dn; i += 256) s_qn[(i / dn) * dnp + i % dn] = s_q[(i / dn) * dh + s_idx[i % dn]];
-  // the outputs below are read by the attention kernel of the previous call until it has
-  // finished (computing before this wait, while that kernel runs, measured slower)
-  pdl_wait();
-  pdl_trigger();
   // RoPE query part: rotate the kept pairs at position L-1 (angle in double), scale
   float ro0 = 0.f, ro1 = 0.f;
   if (rope_item) {
@@ -152,6 +150,12 @@ __global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
   }
 }
 
+template <typename T>
+__global__ void __launch_bounds__(256) absorb_kernel(AbsorbArgs a) {
+  extern __shared__ __align__(16) float sm[];
+  absorb_body<T>(a, blockIdx.x, sm);
+}
+
 // ------------------------------------------------------------ CUDA-core split-K decode
 struct DecodeArgs {
   mla_cache_t cache;
@@ -172,7 +176,6 @@ constexpr int kSimtMaxE = 32;   // H*d_c / 256 owned accumulators per thread
 
 template <typename T, bool INT4>
 __global__ void __launch_bounds__(256) decode_simt_kernel(DecodeArgs a) {
-  MLA_KSPAN(1);
   const int H = a.H, dc = a.d_c, R = a.R, r2 = 2 * a.r;
   const int G = H / a.n_kv;
   extern __shared__ float sm[];
@@ -309,7 +312,6 @@ constexpr int kCmbRows = 8;    // (b, h) rows per CTA, one warp each
 // out[row][d] = sum_c O_lat[row][c] W_uv[g][c][d] with lane l on columns 2l, 2l+1.
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
-  MLA_KSPAN(2);
   extern __shared__ __align__(16) float sm[];
   const int G = a.H / a.n_kv;
   const int rows_total = a.B * G;
@@ -470,42 +472,45 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   }
 }
 
-template <typename T, bool INT4>
-cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens,
-                            const void* q, int B, void* out, void* ws, const DecodeLayout& L,
-                            cudaStream_t s) {
+// Arguments and shared memory of the absorption grid (block 0: the split-K schedule).
+template <typename T>
+void absorb_setup(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, const void* q, int B, void* ws,
+                  const DecodeLayout& L, AbsorbArgs* aa, size_t* smem, int* nblocks) {
   const mla_config_t& cfg = p.cfg;
   const int H = cfg.n_heads, G = H / cfg.n_kv_heads;
   char* base = (char*)ws;
-  Sched sched = mla_sched_view(L, ws, B);
-  // 1. absorb + schedule
-  AbsorbArgs aa;
-  aa.q = q; aa.seq_lens = seq_lens; aa.B = B; aa.T_cap = c.T_cap; aa.H = H;
-  aa.n_kv = cfg.n_kv_heads; aa.dh = cfg.head_dim; aa.r = cfg.r_pairs; aa.d_c = cfg.d_c;
-  aa.dn = p.dn; aa.W_ukT = p.W_ukT; aa.nope_idx = p.nope_idx;
-  aa.rope_pair = p.rope_pair; aa.theta = p.theta;
-  aa.qlat = L.kernel == 1 ? (float*)(base + L.off_qlat) : nullptr;
-  aa.qlat16 = L.kernel == 2 ? (__nv_bfloat16*)(base + L.off_qlat) : nullptr;
-  aa.qrope = (float*)(base + L.off_qrope);
-  aa.sched = sched; aa.tile = L.tile; aa.G = L.G; aa.err = p.err;
+  aa->q = q; aa->seq_lens = seq_lens; aa->B = B; aa->T_cap = c.T_cap; aa->H = H;
+  aa->n_kv = cfg.n_kv_heads; aa->dh = cfg.head_dim; aa->r = cfg.r_pairs; aa->d_c = cfg.d_c;
+  aa->dn = p.dn; aa->W_ukT = p.W_ukT; aa->nope_idx = p.nope_idx;
+  aa->rope_pair = p.rope_pair; aa->theta = p.theta;
+  aa->qlat = L.kernel == 1 ? (float*)(base + L.off_qlat) : nullptr;
+  aa->qlat16 = L.kernel == 2 ? (__nv_bfloat16*)(base + L.off_qlat) : nullptr;
+  aa->qrope = (float*)(base + L.off_qrope);
+  aa->sched = mla_sched_view(L, ws, B); aa->tile = L.tile; aa->G = L.G; aa->err = p.err;
+  aa->sm_scale = cfg.softmax_scale > 0.0f ? cfg.softmax_scale : (float)(1.0 / sqrt((double)cfg.head_dim));
   {
     const int vecn = 16 / (int)sizeof(T);   // elements per 16-byte load
-    aa.vec_ok = ((uintptr_t)q % 16 == 0) && cfg.d_c % vecn == 0 && cfg.head_dim % vecn == 0;
+    aa->vec_ok = ((uintptr_t)q % 16 == 0) && cfg.d_c % vecn == 0 && cfg.head_dim % vecn == 0;
   }
   const int n_rb = (B * G + kAbsRows - 1) / kAbsRows, n_cc = (cfg.d_c + kAbsCols - 1) / kAbsCols;
   const int dnp = (p.dn + 3) & ~3;
   const size_t smem_work = sizeof(float) * ((size_t)p.dn * kAbsCols + (size_t)kAbsRows * cfg.head_dim +
                                             (size_t)kAbsRows * dnp + p.dn);
   const size_t sched_ints = (size_t)9 * B + 4 * L.G + 2;
-  const size_t smem_abs = std::min<size_t>(std::max(smem_work, sched_ints * sizeof(int32_t)),
-                                           std::max<size_t>(smem_work, 160 * 1024));
-  aa.sched_ints = (int)(smem_abs / sizeof(int32_t));
-  cudaError_t e = cudaFuncSetAttribute(absorb_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_abs);
-  if (e != cudaSuccess) return e;
-  e = mla_launch_kernel(absorb_kernel<T>, dim3(cfg.n_kv_heads * n_rb * n_cc + 1), dim3(256), smem_abs, s, p.opt_pdl,
-                        aa);
-  if (e != cudaSuccess) return e;
-  // 2. split-K attention over the latent cache
+  *smem = std::min<size_t>(std::max(smem_work, sched_ints * sizeof(int32_t)), std::max<size_t>(smem_work, 160 * 1024));
+  aa->sched_ints = (int)(*smem / sizeof(int32_t));
+  *nblocks = cfg.n_kv_heads * n_rb * n_cc + 1;
+}
+
+// Split-K attention over the latent cache, then the split merge with W_uv.
+template <typename T, bool INT4>
+cudaError_t launch_attention_combine(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B,
+                                     void* out, void* ws, const DecodeLayout& L, const AbsorbArgs& aa, cudaStream_t s) {
+  const mla_config_t& cfg = p.cfg;
+  const int H = cfg.n_heads;
+  char* base = (char*)ws;
+  const Sched sched = aa.sched;
+  cudaError_t e;
   if (L.kernel == 1) {
     DecodeArgs da;
     da.cache = c; da.seq_lens = seq_lens; da.err = p.err; da.qbits = mla_quant_bits(cfg.cache_kind); da.B = B; da.H = H; da.n_kv = cfg.n_kv_heads; da.r = cfg.r_pairs;
@@ -519,16 +524,16 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
     e = cudaFuncSetAttribute(decode_simt_kernel<T, INT4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    if ((e = mla_profile_event(p, 0, s)) != cudaSuccess) return e;
+    if ((e = mla_profile_event(p, kProfAttention, false, s)) != cudaSuccess) return e;
     e = mla_launch_kernel(decode_simt_kernel<T, INT4>, dim3(L.G), dim3(256), smem, s, p.opt_pdl, da);
     if (e != cudaSuccess) return e;
-    if ((e = mla_profile_event(p, 1, s)) != cudaSuccess) return e;
+    if ((e = mla_profile_event(p, kProfAttention, true, s)) != cudaSuccess) return e;
   } else {
     e = mla_launch_decode_tc(p, c, seq_lens, B, sched, base + L.off_qlat, (const float*)(base + L.off_qrope),
                              (float*)(base + L.off_opart), (float*)(base + L.off_mlpart), L.P, L.G, s);
     if (e != cudaSuccess) return e;
   }
-  // 3. merge the splits and apply W_uv
+  // merge the splits and apply W_uv
   CombineArgs ca;
   ca.B = B; ca.H = H; ca.n_kv = cfg.n_kv_heads; ca.d_c = cfg.d_c; ca.dh = cfg.head_dim;
   ca.opart = (const float*)(base + L.off_opart); ca.mlpart = (const float*)(base + L.off_mlpart);
@@ -537,11 +542,86 @@ cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32
   ca.vec_ok = cfg.head_dim % (16 / (int)sizeof(T)) == 0;
   const size_t smem_c = (size_t)cfg.d_c * (ca.ncols + kCmbRows) * sizeof(float) +
                         (size_t)16 * (cfg.d_c + 8) * sizeof(__nv_bfloat16);   // + the MMA form's A tile
+  const int G = H / cfg.n_kv_heads;
   const int n_rbc = (B * G + kCmbRows - 1) / kCmbRows, n_dc = (cfg.head_dim + ca.ncols - 1) / ca.ncols;
   e = cudaFuncSetAttribute(combine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
   if (e != cudaSuccess) return e;
-  return mla_launch_kernel(combine_kernel<T>, dim3(cfg.n_kv_heads * n_rbc * n_dc), dim3(256), smem_c, s, p.opt_pdl,
-                           ca);
+  if ((e = mla_profile_event(p, kProfCombine, false, s)) != cudaSuccess) return e;
+  e = mla_launch_kernel(combine_kernel<T>, dim3(cfg.n_kv_heads * n_rbc * n_dc), dim3(256), smem_c, s, p.opt_pdl, ca);
+  if (e != cudaSuccess) return e;
+  return mla_profile_event(p, kProfCombine, true, s);
+}
+
+template <typename T, bool INT4>
+cudaError_t launch_decode_t(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens,
+                            const void* q, int B, void* out, void* ws, const DecodeLayout& L,
+                            cudaStream_t s) {
+  AbsorbArgs aa;
+  size_t smem_abs;
+  int nblk;
+  absorb_setup<T>(p, c, seq_lens, q, B, ws, L, &aa, &smem_abs, &nblk);
+  cudaError_t e = cudaFuncSetAttribute(absorb_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_abs);
+  if (e != cudaSuccess) return e;
+  if ((e = mla_profile_event(p, kProfAbsorb, false, s)) != cudaSuccess) return e;
+  e = mla_launch_kernel(absorb_kernel<T>, dim3(nblk), dim3(256), smem_abs, s, p.opt_pdl, aa);
+  if (e != cudaSuccess) return e;
+  if ((e = mla_profile_event(p, kProfAbsorb, true, s)) != cudaSuccess) return e;
+  return launch_attention_combine<T, INT4>(p, c, seq_lens, B, out, ws, L, aa, s);
+}
+
+// ------------------------------------------------------------ fused decode step
+// The first kernel of a decode step: the append of every sequence's new token and the
+// query absorption (with the split-K schedule) in one launch, as they depend on nothing
+// of each other.  Blocks [0, n_abs) run the absorption grid (block 0, the schedule, is
+// dispatched first), blocks [n_abs, n_abs + n_app) the append grid.
+struct StepPreArgs {
+  AbsorbArgs abs;
+  AppendSmallArgs app;
+  int n_abs, app_gx, app_gy;
+};
+
+template <bool INT4>
+__global__ void __launch_bounds__(256) step_pre_kernel(StepPreArgs sp) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int b = blockIdx.x;
+  if (b < sp.n_abs) {
+    absorb_body<__nv_bfloat16>(sp.abs, b, reinterpret_cast<float*>(smem));
+  } else {
+    const int k = b - sp.n_abs, gxy = sp.app_gx * sp.app_gy;
+    append_small_mma_body<INT4>(sp.app, k % sp.app_gx, (k / sp.app_gx) % sp.app_gy, k / gxy, sp.app_gx, sp.app_gy,
+                                smem);
+  }
+}
+
+template <bool INT4>
+cudaError_t launch_step_t(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, const void* x,
+                          const void* q, int B, void* out, void* ws, const DecodeLayout& L, cudaStream_t s) {
+  using bf16 = __nv_bfloat16;
+  StepPreArgs sp;
+  dim3 agrid;
+  size_t smem_app = 0, smem_abs;
+  int nabs;
+  absorb_setup<bf16>(p, c, seq_lens, q, B, ws, L, &sp.abs, &smem_abs, &nabs);
+  if (!mla_append_step_mma_form(p, x, seq_lens, B, c, &sp.app, &agrid, &smem_app)) {
+    // no fused form for this shape: the append, then the decode, as separate launches
+    cudaError_t e = mla_profile_event(p, kProfAppend, false, s);
+    if (e == cudaSuccess) e = mla_launch_append_step(p, x, seq_lens, B, c, s);
+    if (e == cudaSuccess) e = mla_profile_event(p, kProfAppend, true, s);
+    if (e != cudaSuccess) return e;
+    return launch_decode_t<bf16, INT4>(p, c, seq_lens, q, B, out, ws, L, s);
+  }
+  sp.n_abs = nabs;
+  sp.app_gx = (int)agrid.x;
+  sp.app_gy = (int)agrid.y;
+  const int nblk = nabs + (int)(agrid.x * agrid.y * agrid.z);
+  const size_t smem = std::max(smem_app, smem_abs);
+  cudaError_t e = cudaFuncSetAttribute(step_pre_kernel<INT4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  if ((e = mla_profile_event(p, kProfAbsorb, false, s)) != cudaSuccess) return e;
+  e = mla_launch_kernel(step_pre_kernel<INT4>, dim3(nblk), dim3(256), smem, s, p.opt_pdl, sp);
+  if (e != cudaSuccess) return e;
+  if ((e = mla_profile_event(p, kProfAbsorb, true, s)) != cudaSuccess) return e;
+  return launch_attention_combine<bf16, INT4>(p, c, seq_lens, B, out, ws, L, sp.abs, s);
 }
 
 }  // namespace mla
@@ -602,5 +682,20 @@ cudaError_t mla_launch_decode(const mla_plan& p, const mla_cache_t& c, const int
   if (p.cfg.dtype == MLA_BF16)
     return quant ? launch_decode_t<__nv_bfloat16, true>(p, c, seq_lens, q, B, out, ws, L, s)
                 : launch_decode_t<__nv_bfloat16, false>(p, c, seq_lens, q, B, out, ws, L, s);
+  return launch_decode_t<float, false>(p, c, seq_lens, q, B, out, ws, L, s);
+}
+
+cudaError_t mla_launch_step(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, const void* x,
+                            const void* q, int B, void* out, void* ws, const DecodeLayout& L, cudaStream_t s) {
+  using namespace mla;
+  const bool quant = mla_kind_quant(p.cfg.cache_kind);
+  if (p.cfg.dtype == MLA_BF16)
+    return quant ? launch_step_t<true>(p, c, seq_lens, x, q, B, out, ws, L, s)
+                 : launch_step_t<false>(p, c, seq_lens, x, q, B, out, ws, L, s);
+  // float32: no fused form
+  cudaError_t e = mla_profile_event(p, kProfAppend, false, s);
+  if (e == cudaSuccess) e = mla_launch_append_step(p, x, seq_lens, B, c, s);
+  if (e == cudaSuccess) e = mla_profile_event(p, kProfAppend, true, s);
+  if (e != cudaSuccess) return e;
   return launch_decode_t<float, false>(p, c, seq_lens, q, B, out, ws, L, s);
 }

@@ -40,11 +40,11 @@ __device__ inline int block_exscan(int v, int* total, int* s_warp) {
   return base + x - v;
 }
 
-// Single-block schedule builder.  Must be run by one whole CTA.  When `scratch` (shared
-// memory, `scratch_ints` ints) can hold all of it, the schedule is built there (it depends
-// on the sequence lengths only, so this overlaps the kernel before) and copied out once,
-// after the programmatic dependency wait; otherwise the wait comes first and the schedule
-// is built in the workspace directly.
+// Single-block schedule builder.  Must be run by one whole CTA.  It first waits for the
+// kernel before (the sequence lengths are the caller's input and the workspace may still
+// be read by the previous call).  When `scratch` (shared memory, `scratch_ints` ints) can
+// hold all of it, the schedule is built there and copied out once, coalesced; otherwise
+// it is built in the workspace directly.
 __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int B, int T_cap,
                                       int tile, int G, Sched out, int32_t* err, int32_t* scratch,
                                       int scratch_ints) {
@@ -54,6 +54,8 @@ __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int 
   const bool local = scratch && (long long)9 * B + 4 * G + 2 <= scratch_ints;
   Sched s = out;
   int32_t* seq_len = nullptr;
+  pdl_wait();
+  pdl_trigger();
   if (local) {
     int32_t* q = scratch;
     s.seq_tile0 = q; q += B;
@@ -66,9 +68,6 @@ __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int 
     s.piece_t0 = q; q += Pcap;
     s.piece_t1 = q; q += Pcap;
     seq_len = q;  // [B]
-  } else {
-    pdl_wait();
-    pdl_trigger();
   }
   // 1. tiles per sequence; exclusive prefix sums of tiles and of non-empty sequences
   int carry_t = 0, carry_ne = 0;
@@ -158,8 +157,6 @@ __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int 
   }
   if (local) {   // copy the schedule out (coalesced)
     __syncthreads();
-    pdl_wait();   // the previous call's kernels may still read the workspace
-    pdl_trigger();
     for (int i = tid; i < B; i += nt) {
       out.seq_tile0[i] = s.seq_tile0[i];
       out.seq_ntiles[i] = s.seq_ntiles[i];

@@ -21,16 +21,24 @@ static_assert(kNoAllocScratchBytes == (size_t)MLA_NOALLOC_SCRATCH_BYTES, "header
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-void* g_scratch[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+std::mutex g_mutex;
+void* g_scratch[kMaxDevices];   // device address of the array per device, once resolved
 
-// Runs once per device, with that device current.
-void resolve_scratch(int dev) {
-  void* p = nullptr;
-  cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
-  g_scratch_err[dev] = e;
-  g_scratch[dev] = e == cudaSuccess ? p : nullptr;
+// The array's device address on `dev` (the current device), looked up the first time it
+// succeeds and kept from then on.  A failed lookup is not remembered: the next call tries
+// again, and the lookup's error is cleared so a later, unrelated status check does not
+// pick it up.
+void* scratch_address(int dev) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_scratch[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) == cudaSuccess) {
+      g_scratch[dev] = p;
+    } else {
+      (void)cudaGetLastError();
+    }
+  }
+  return g_scratch[dev];
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
@@ -50,8 +58,8 @@ extern "C" mla_status_t mla_decode_noalloc(const mla_plan_t* plan, const mla_cac
   if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
   if (dev != plan->device) return MLA_ERR_INVALID_ARG;   // the plan's weights live on its device
   if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
-  std::call_once(g_once[dev], resolve_scratch, dev);
-  if (g_scratch_err[dev] != cudaSuccess || !g_scratch[dev]) return MLA_ERR_CUDA;
+  void* scratch = scratch_address(dev);
+  if (!scratch) return MLA_ERR_CUDA;
 
   int kernel = 1;
   if (plan->opt_kernel != 1 && mla_tc_kind_ok(cfg) && mla_tc_supported(*plan, *cache)) kernel = 2;
@@ -60,6 +68,6 @@ extern "C" mla_status_t mla_decode_noalloc(const mla_plan_t* plan, const mla_cac
   const DecodeLayout L = mla_decode_layout(*plan, B, kernel);
   if (L.total > kNoAllocScratchBytes) return MLA_ERR_WORKSPACE_TOO_SMALL;
   const cudaError_t e =
-      mla_launch_decode(*plan, *cache, seq_lens, q, B, out, g_scratch[dev], L, (cudaStream_t)stream);
+      mla_launch_decode(*plan, *cache, seq_lens, q, B, out, scratch, L, (cudaStream_t)stream);
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }

@@ -61,6 +61,9 @@ struct TcArgs {
   const uint8_t* kr_base;
   uint32_t c_row, kr_row;
   int32_t* err;
+  uint64_t wait_ns;       // bound of every pipeline wait
+  int pf_dist, pf_mode;   // L2 prefetch: tiles ahead of the copies (0 = off); 1 lines, 2 bulk
+  int skip_tile;          // testing only: 1-based tile whose latent copy is left out (0 = none)
   int NC, NRAW, NP, NO;  // ring depths; P^T and O buffers
   uint32_t off_c, off_q, off_p, off_raw, off_qr, off_bar, off_misc;
   uint32_t off_kr;        // RoPE key stage: one tile, 4 blocks of [n_kv][32][2r]
@@ -173,24 +176,6 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[kH], int lane) {
   return v[0];
 }
 
-#ifdef MLA_TC_TRACE
-// Timeline instrumentation for development builds only (-DMLA_TC_TRACE): %globaltimer
-// stamps per (CTA, event, tile) for the first kTraceCtas CTAs.
-constexpr int kTraceCtas = 4, kTraceEv = 48, kTraceTiles = 64;
-__device__ unsigned long long g_trace[kTraceCtas * kTraceEv * kTraceTiles];
-__device__ unsigned long long g_cta_span[1024 * 2];
-__device__ __forceinline__ int trace_slot() {   // CTAs 0, 1 and two that straddle sequences
-  return blockIdx.x < 2 ? (int)blockIdx.x : blockIdx.x == 23 ? 2 : blockIdx.x == 60 ? 3 : -1;
-}
-#define MLA_TRACE(ev, n)                                                                          \
-  do {                                                                                            \
-    const int ts_ = trace_slot();                                                                 \
-    if (ts_ >= 0 && (n) < kTraceTiles)                                                            \
-      g_trace[(ts_ * kTraceEv + (ev)) * kTraceTiles + (n)] = globaltimer();                       \
-  } while (0)
-#else
-#define MLA_TRACE(ev, n) do { } while (0)
-#endif
 
 // Storage location of (b, t): compile-time contiguous, or through the paged block table.
 template <bool PAGED>
@@ -210,9 +195,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
   const uint32_t sbase_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (sbase_u32 - smem_u32(smem_raw));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-#ifdef MLA_TC_TRACE
-  if (threadIdx.x == 0 && blockIdx.x < 1024) g_cta_span[2 * blockIdx.x] = globaltimer();
-#endif
   const int dc = a.d_c, R = a.R;
   const int n_cbox = dc / 64;
   const uint32_t c_stage = (uint32_t)n_cbox * kBox;
@@ -267,7 +249,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
   pdl_trigger();
   const uint32_t tmem = misc->tmem_base;
   const int w = blockIdx.x;
-  if (threadIdx.x == 0) MLA_TRACE(7, 0);
+  const uint64_t lim = a.wait_ns;
 
   // register split: the control warpgroup (producer, MMA issuer, int4 dequant) gives up
   // registers to the two softmax warpgroups: 128 * 56 + 256 * 224 = 384 * 168 at launch
@@ -275,62 +257,98 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
     setmaxnreg_dec<56>();
     if (warp == 0) {
       // ============================================================ TMA producer
-      if (lane == 0) {
-        TileIter it;
-        it.init(&a.sched, w);
-        int n = 0, u = 0, q_loads = 0;
-        int last_c = -1, last_raw = -1;
-        bool ok = true;
-        while (ok && it.valid()) {
-          if (it.first_of_piece()) {
-            if (u > 0) ok = mbar_wait(bars.q_empty(), (u - 1) & 1, abort_flag);
-            if (!ok) break;
+      // Lane 0 issues the copies; the whole warp walks the schedule a.pf_dist tiles ahead
+      // and asks L2 to fetch those tiles' cache bytes (latent rows, int4 scales, RoPE-key
+      // blocks), so HBM keeps streaming while the shared-memory stages are all busy.
+      TileIter it, pf;
+      it.init(&a.sched, w);
+      pf = it;
+      auto prefetch_tile = [&](const TileIter& ti) {
+        const int nvalid = min(kTile, ti.t1 - ti.t);
+        const MlaLoc lc = tc_loc<PAGED>(a, ti.b, ti.t);
+        const size_t row = (size_t)lc.pb * lc.cap + lc.pt;
+        const uint8_t* cp = reinterpret_cast<const uint8_t*>(a.cache.c_kv) + row * a.c_row;
+        const uint8_t* kp = a.kr_base + mla_kr_offset(lc.pb, lc.pt, 0, 0, lc.cap, R / R2, R2) * 2;
+        const uint8_t* sp = INT4 ? reinterpret_cast<const uint8_t*>(a.scales) + row * (dc / 16) : nullptr;
+        const uint32_t cbytes = (uint32_t)nvalid * a.c_row;
+        const uint32_t kbytes = (uint32_t)((nvalid + 31) / 32) * (uint32_t)(R / R2) * 32u * R2 * 2u;
+        const uint32_t sbytes = INT4 ? (uint32_t)nvalid * (dc / 16) : 0u;
+        if (a.pf_mode == 2) {   // bulk prefetches (sizes rounded down to 16 bytes: a hint)
+          if (lane == 0) {
+            prefetch_l2(cp, cbytes & ~15u);
+            prefetch_l2(kp, kbytes & ~15u);
+            if (INT4 && sbytes >= 16) prefetch_l2(sp, sbytes & ~15u);
+          }
+        } else {                // one 128-byte line per lane and instruction
+          for (uint32_t o = lane * 128u; o < cbytes; o += 32u * 128u) prefetch_l2_line(cp + o);
+          for (uint32_t o = lane * 128u; o < kbytes; o += 32u * 128u) prefetch_l2_line(kp + o);
+          if (INT4)
+            for (uint32_t o = lane * 128u; o < sbytes; o += 32u * 128u) prefetch_l2_line(sp + o);
+        }
+      };
+      if (a.pf_dist > 0) {   // tiles 1 .. pf_dist ahead of the first copy
+        pf.next();
+        for (int k = 0; k < a.pf_dist && pf.valid(); ++k) { prefetch_tile(pf); pf.next(); }
+      }
+      int n = 0, u = 0, q_loads = 0;
+      int last_c = -1, last_raw = -1, skipped = -1;
+      bool ok = true;
+      while (ok && it.valid()) {
+        if (a.pf_dist > 0 && pf.valid()) { prefetch_tile(pf); pf.next(); }
+        if (it.first_of_piece()) {
+          if (u > 0) ok = __all_sync(0xffffffffu, mbar_wait(bars.q_empty(), (u - 1) & 1, abort_flag, lim));
+          if (!ok) break;
+          if (lane == 0) {
             mbar_expect_tx(bars.q_full(), (uint32_t)n_cbox * kQBox);
             for (int kb = 0; kb < n_cbox; ++kb)
               tma_load_2d(qbox(kb), &tm_q, bars.q_full(), kb * 64, it.b * a.H);
-            ++q_loads;
           }
-          const MlaLoc lc = tc_loc<PAGED>(a, it.b, it.t);   // a tile is one paged block
-          const int row = lc.pb * lc.cap + lc.pt;
-          MLA_TRACE(0, n);
-          if (!INT4) {
-            const int cs = n % a.NC;
-            if (n >= a.NC) ok = mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag);
-            if (!ok) break;
+          ++q_loads;
+        }
+        const MlaLoc lc = tc_loc<PAGED>(a, it.b, it.t);   // a tile is one paged block
+        const int row = lc.pb * lc.cap + lc.pt;
+        // testing hook (off unless set): leave this tile's latent copy out, so the waits
+        // on it run out and the kernel reports MLA_DEVERR_TIMEOUT
+        const bool skip = (n + 1 == a.skip_tile);
+        if (!INT4) {
+          const int cs = n % a.NC;
+          if (n >= a.NC) ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag, lim));
+          if (!ok) break;
+          if (lane == 0 && !skip) {
             mbar_expect_tx(bars.c_full(cs), c_stage);
             for (int cb = 0; cb < n_cbox; ++cb)
               tma_load_2d(sbase_u32 + a.off_c + cs * c_stage + cb * kBox, &tm_c, bars.c_full(cs), cb * 64, row);
-            last_c = n;
-          } else {
-            const int rs = n % a.NRAW;
-            if (n >= a.NRAW) ok = mbar_wait(bars.raw_empty(rs), ((n / a.NRAW) - 1) & 1, abort_flag);
-            if (!ok) break;
-            const int nvalid = min(kTile, it.t1 - it.t);
-            const uint32_t sbytes = (uint32_t)((((nvalid + 1) & ~1) * (dc / 16) + 15) & ~15);
+          }
+          last_c = n;
+        } else {
+          const int rs = n % a.NRAW;
+          if (n >= a.NRAW) ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_empty(rs), ((n / a.NRAW) - 1) & 1, abort_flag, lim));
+          if (!ok) break;
+          const int nvalid = min(kTile, it.t1 - it.t);
+          const uint32_t sbytes = (uint32_t)((((nvalid + 1) & ~1) * (dc / 16) + 15) & ~15);
+          if (lane == 0 && !skip) {
             mbar_expect_tx(bars.raw_full(rs), raw_codes + sbytes);
             tma_load_2d(sbase_u32 + a.off_raw + rs * raw_stage, &tm_c, bars.raw_full(rs), 0, row);
             bulk_load(sbase_u32 + a.off_raw + rs * raw_stage + raw_codes, a.scales + (size_t)row * (dc / 32), sbytes,
                       bars.raw_full(rs));
-            last_raw = n;
           }
-          MLA_TRACE(1, n);
-          if (it.last_of_piece()) ++u;
-          it.next();
-          ++n;
+          last_raw = n;
         }
-        // drain: every issued copy must land before the CTA can exit
+        if (skip) skipped = n;
+        if (it.last_of_piece()) ++u;
+        it.next();
+        ++n;
+      }
+      // drain: every issued copy must land before the CTA can exit (a skipped copy's
+      // stage waits for the copy before it instead)
+      if (lane == 0) {
         volatile int never = 0;
-        if (q_loads > 0) mbar_wait(bars.q_full(), (q_loads - 1) & 1, &never);
-        if (!INT4) {
-          for (int s = 0; s < a.NC; ++s) {
-            const int k = last_c - ((last_c - s) % a.NC + a.NC) % a.NC;
-            if (last_c >= 0 && k >= 0) mbar_wait(bars.c_full(s), (k / a.NC) & 1, &never);
-          }
-        } else {
-          for (int s = 0; s < a.NRAW; ++s) {
-            const int k = last_raw - ((last_raw - s) % a.NRAW + a.NRAW) % a.NRAW;
-            if (last_raw >= 0 && k >= 0) mbar_wait(bars.raw_full(s), (k / a.NRAW) & 1, &never);
-          }
+        if (q_loads > 0) mbar_wait(bars.q_full(), (q_loads - 1) & 1, &never, lim);
+        const int NS = INT4 ? a.NRAW : a.NC, last = INT4 ? last_raw : last_c;
+        for (int s = 0; s < NS; ++s) {
+          int k = last - ((last - s) % NS + NS) % NS;
+          if (k == skipped) k -= NS;
+          if (last >= 0 && k >= 0) mbar_wait(INT4 ? bars.raw_full(s) : bars.c_full(s), (k / NS) & 1, &never, lim);
         }
       }
     } else if (warp == 1) {
@@ -346,10 +364,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
         bool pend_first = false, pend_last = false;
         auto do_mma2 = [&](int pn, int pu, bool first, bool last) -> bool {
           const int pb = pn % a.NP, cs = pn % a.NC, ob = pu % a.NO;
-          if (!mbar_wait(bars.p_full(pb), (pn / a.NP) & 1, abort_flag)) return false;
+          if (!mbar_wait(bars.p_full(pb), (pn / a.NP) & 1, abort_flag, lim)) return false;
           if (first && pu >= a.NO)
-            if (!mbar_wait(bars.o_empty(ob), ((pu / a.NO) - 1) & 1, abort_flag)) return false;
-          MLA_TRACE(4, pn);
+            if (!mbar_wait(bars.o_empty(ob), ((pu / a.NO) - 1) & 1, abort_flag, lim)) return false;
           tc_fence_after();
           const uint32_t c0 = sbase_u32 + a.off_c + cs * c_stage;
           const uint32_t p0 = sbase_u32 + a.off_p + pb * kPtBytes;
@@ -383,7 +400,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
               if ((n < 2 || mbar_test(bars.s_empty(sb), ((n >> 1) - 1) & 1)) &&
                   (!first || mbar_test(bars.q_full(), u & 1)) && mbar_test(bars.c_full(cs), (n / a.NC) & 1))
                 break;
-              if (*abort_flag || globaltimer() - t_start > kWaitLimitNs) {
+              if (*abort_flag || globaltimer() - t_start > lim) {
                 *abort_flag = 1;
                 ok = false;
                 break;
@@ -391,7 +408,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
             }
           }
           if (!ok) break;
-          MLA_TRACE(2, n);
           tc_fence_after();
           {  // MMA1: S = C Q_lat^T
             const uint32_t d = tmem + S_COL + sb * kH;
@@ -403,7 +419,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
             }
             tc_commit(bars.s_full(sb));
             if (it.last_of_piece()) tc_commit(bars.q_empty());
-            MLA_TRACE(3, n);
           }
           if (pend_n >= 0) {   // one pending tile at most: MMA2(n-1) before tile n waits
             ok = do_mma2(pend_n, pend_u, pend_first, pend_last);
@@ -418,7 +433,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
         // drain: all issued MMAs complete before TMEM is released
         tc_commit(bars.mma_done());
         volatile int never = 0;
-        mbar_wait(bars.mma_done(), 0, &never);
+        mbar_wait(bars.mma_done(), 0, &never, lim);
       }
     } else if (INT4 && warp >= 2) {
       // ============================================================ int4 dequantisation
@@ -434,9 +449,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
           lo_b = it.b;
           lo = __ldg(a.seq_lens + it.b) - MLA_RESID_WINDOW;
         }
-        ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_full(rs), (n / a.NRAW) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_full(rs), (n / a.NRAW) & 1, abort_flag, lim));
         if (ok && n >= a.NC)
-          ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag));
+          ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag, lim));
         if (!ok) break;
         const int nvalid = min(kTile, it.t1 - it.t);
         const uint8_t* raw = sbase + a.off_raw + rs * raw_stage;
@@ -501,7 +516,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
     bool ok = true;
     float m[kHh], l[kHh];
     auto wwait = [&](uint32_t bar, int parity) -> bool {  // warp-uniform outcome
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, lim));
     };
     auto grp_sync = [&](int i) -> bool {  // all softmax warps, bounded
       __syncwarp();
@@ -559,7 +574,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
       if (first) {   // this piece's RoPE queries are in qr_s[u & 1] (loaded one piece ahead)
 #pragma unroll
         for (int h = 0; h < kHh; ++h) { m[h] = -INFINITY; l[h] = 0.f; }
-        if (warp == 4 && lane == 0) MLA_TRACE(43, n);
       }
       const float* qr = qr_s + (u & 1) * (kH * R2);
       const int sb = n & 1, pb = n % a.NP, ob = u % a.NO;
@@ -567,7 +581,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
       const bool valid = tr < nvalid;
       ok = wwait(bars.s_full(sb), (n >> 1) & 1);
       if (!ok) break;
-      if (warp == 4 && lane == 0) MLA_TRACE(5, n);
       tc_fence_after();
       float v[kHh];
       {
@@ -577,7 +590,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
 #pragma unroll
         for (int h = 0; h < kHh; ++h) v[h] = u2f(raw[h]);
       }
-      if (lane == 0) MLA_TRACE(16 + sw, n);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.s_empty(sb));
@@ -591,7 +603,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
         v[h] += qa.x * bf16lo(kw.x) + qa.y * bf16hi(kw.x) + qa.z * bf16lo(kw.y) + qa.w * bf16hi(kw.y) +
                 qb.x * bf16lo(kw.z) + qb.y * bf16hi(kw.z) + qb.z * bf16lo(kw.w) + qb.w * bf16hi(kw.w);
       }
-      if (lane == 0) MLA_TRACE(24 + sw, n);
       {
         TileIter nx = it;
         nx.next();
@@ -602,7 +613,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
           if (!ok) break;
         }
       }
-      if (warp == 4 && lane == 0) MLA_TRACE(10, n);
       if (!valid) {
 #pragma unroll
         for (int h = 0; h < kHh; ++h) v[h] = -INFINITY;
@@ -620,10 +630,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
         }
         if (lane < 16) misc->red_max[n & 1][q][kHh * hh + lane] = wmax;
       }
-      if (lane == 0) MLA_TRACE(32 + sw, n);
       ok = grp_sync(0);
       if (!ok) break;
-      if (warp == 4 && lane == 0) MLA_TRACE(11, n);
       float tmax[kHh];
 #pragma unroll
       for (int h4 = 0; h4 < kHh; h4 += 4) {
@@ -669,7 +677,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
           tmem_wait_st();
         }
       }
-      if (warp == 4 && lane == 0) MLA_TRACE(12, n);
       // probabilities of this tile, P^T for MMA2 (row h, column = token, bf16)
       float pr[kHh];
 #pragma unroll
@@ -677,12 +684,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
         pr[h] = valid ? exp2f(v[h] - m[h]) : 0.f;
         l[h] += pr[h];
       }
-      if (warp == 4 && lane == 0) MLA_TRACE(13, n);
       if (n >= a.NP) {
         ok = wwait(bars.p_empty(pb), ((n / a.NP) - 1) & 1);
         if (!ok) break;
       }
-      if (warp == 4 && lane == 0) MLA_TRACE(14, n);
       {
         uint8_t* Pt = sbase + a.off_p + pb * kPtBytes + (tr >> 6) * kPtAtom + (tr & 7) * 2;
         const int c8 = (tr & 63) >> 3;
@@ -704,7 +709,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.p_full(pb));
-      if (warp == 4 && lane == 0) MLA_TRACE(6, n);
 
       if (it.last_of_piece()) {
         // ---------------- piece epilogue: partial (m, l, O) for the split merge
@@ -717,10 +721,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
             for (int i = threadIdx.x - 128; i < kH * R2; i += 32 * kSoftWarps)
               qr_s[((u + 1) & 1) * (kH * R2) + i] = __ldg(a.qrope + (size_t)nx.b * kH * R2 + i);
         }
-        if (warp == 4 && lane == 0) MLA_TRACE(44, u);
         ok = grp_sync(1);
         if (!ok) break;
-        if (warp == 4 && lane == 0) MLA_TRACE(40, u);
         if (q == 0 && lane < 16) {
           const int H = kHh * hh + lane;
           const float L = misc->red_l[0][H] + misc->red_l[1][H] + misc->red_l[2][H] + misc->red_l[3][H];
@@ -732,7 +734,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
         }
         ok = wwait(bars.o_full(ob), (u / a.NO) & 1);
         if (!ok) break;
-        if (warp == 4 && lane == 0) MLA_TRACE(41, u);
         tc_fence_after();
         if (q < 2) {
           // O^T rows (M = 64 layout): head 16q + lane in lane `lane` (< 16) of quarter q; the
@@ -755,11 +756,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
             }
           }
         }
-        if (warp == 4 && lane == 0) MLA_TRACE(42, u);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.o_empty(ob));
-        if (warp == 4 && lane == 0) MLA_TRACE(9, u);
         ++u;
       }
       it.next();
@@ -768,7 +767,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
     // no RoPE key copy may still be landing when the CTA exits
     if (sw == 0 && lane == 0 && misc->kr_issued > 0) {
       volatile int never = 0;
-      mbar_wait(bars.kr_full(), (misc->kr_issued - 1) & 1, &never);
+      mbar_wait(bars.kr_full(), (misc->kr_issued - 1) & 1, &never, lim);
     }
   }
 
@@ -781,10 +780,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
     tmem_dealloc(tmem, tmem_cols);
   }
   if (threadIdx.x == 0 && misc->abort_flag) raise_error(a.err, MLA_DEVERR_TIMEOUT);
-  if (threadIdx.x == 0) MLA_TRACE(8, 0);
-#ifdef MLA_TC_TRACE
-  if (threadIdx.x == 0 && blockIdx.x < 1024) g_cta_span[2 * blockIdx.x + 1] = globaltimer();
-#endif
 }
 
 // ------------------------------------------------------------------ host side
@@ -915,6 +910,10 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
   a.kr_base = (const uint8_t*)c.k_rope;
   a.c_row = int4 ? (uint32_t)dc / 2 : (uint32_t)dc * 2;
   a.kr_row = (uint32_t)R * 2;
+  a.wait_ns = (uint64_t)p.opt_wait_us * 1000u;
+  a.pf_dist = p.opt_pf_dist;
+  a.pf_mode = p.opt_pf_mode;
+  a.skip_tile = p.opt_skip_tile;
   a.NC = L.NC; a.NRAW = L.NRAW; a.NP = L.NP; a.NO = L.NO;
   a.off_c = L.off_c; a.off_q = L.off_q; a.off_p = L.off_p; a.off_raw = L.off_raw;
   a.off_qr = L.off_qr; a.off_kr = L.off_kr; a.off_bar = L.off_bar; a.off_misc = L.off_misc;
@@ -927,23 +926,10 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
   // the optional profiling events bracket the launch alone, after all host-side set-up
-  if ((e = mla_profile_event(p, 0, s)) != cudaSuccess) return e;
+  if ((e = mla_profile_event(p, kProfAttention, false, s)) != cudaSuccess) return e;
   e = mla_launch_kernel(kern, dim3(G), dim3(384), L.total, s, p.opt_pdl, tm_c, tm_q, a);
   if (e != cudaSuccess) return e;
-  if ((e = mla_profile_event(p, 1, s)) != cudaSuccess) return e;
+  if ((e = mla_profile_event(p, kProfAttention, true, s)) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
-#ifdef MLA_TC_TRACE
-extern "C" __attribute__((visibility("default"))) int mla_tc_trace_read(unsigned long long* host, int n) {
-  const int total = mla::tc::kTraceCtas * mla::tc::kTraceEv * mla::tc::kTraceTiles;
-  if (n < total) return -1;
-  if (cudaMemcpyFromSymbol(host, mla::tc::g_trace, sizeof(unsigned long long) * total) != cudaSuccess) return -2;
-  return total;
-}
-extern "C" __attribute__((visibility("default"))) int mla_tc_span_read(unsigned long long* host, int n) {
-  if (n < 2048) return -1;
-  if (cudaMemcpyFromSymbol(host, mla::tc::g_cta_span, sizeof(unsigned long long) * 2048) != cudaSuccess) return -2;
-  return 2048;
-}
-#endif

@@ -23,6 +23,7 @@ mla_status_t validate_config(const mla_config_t* c) {
   if (c->n_heads % c->n_kv_heads != 0 || c->head_dim % 2 != 0) return MLA_ERR_INVALID_ARG;
   if (c->r_pairs < 0 || 2 * c->r_pairs > c->head_dim) return MLA_ERR_INVALID_ARG;
   if (!(c->rope_base > 1.0)) return MLA_ERR_INVALID_ARG;
+  if (!(c->softmax_scale >= 0.0f) || !isfinite(c->softmax_scale)) return MLA_ERR_INVALID_ARG;
   if (c->dtype != MLA_F32 && c->dtype != MLA_BF16) return MLA_ERR_INVALID_ARG;
   if (c->cache_kind != MLA_CACHE_SAME && !mla_kind_quant(c->cache_kind)) return MLA_ERR_INVALID_ARG;
   if (mla_kind_quant(c->cache_kind) && (c->dtype != MLA_BF16 || c->d_c % 32 != 0))
@@ -238,9 +239,25 @@ mla_status_t mla_plan_set_option(mla_plan_t* plan, int32_t option, int64_t value
     case MLA_OPT_PROFILE_EVENTS:
       plan->opt_events = (const void* const*)(uintptr_t)value;
       return MLA_OK;
+    case MLA_OPT_PROFILE_KERNELS:
+      plan->opt_kernel_events = (const void* const*)(uintptr_t)value;
+      return MLA_OK;
     case MLA_OPT_OVERLAP_LAUNCH:
       if (value < 0 || value > 1) return MLA_ERR_INVALID_ARG;
       plan->opt_pdl = (int)value;
+      return MLA_OK;
+    case MLA_OPT_WAIT_LIMIT_US:
+      if (value < 100 || value > 10000000) return MLA_ERR_INVALID_ARG;
+      plan->opt_wait_us = value;
+      return MLA_OK;
+    case MLA_OPT_TEST_SKIP_COPY:
+      if (value < 0 || value > (1 << 20)) return MLA_ERR_INVALID_ARG;
+      plan->opt_skip_tile = (int)value;
+      return MLA_OK;
+    case MLA_OPT_L2_PREFETCH:
+      if (value < 0 || (value & 0xFF) > 16 || (value >> 8) > 2) return MLA_ERR_INVALID_ARG;
+      plan->opt_pf_dist = (int)(value & 0xFF);
+      if ((value >> 8) != 0) plan->opt_pf_mode = (int)(value >> 8);
       return MLA_OK;
   }
   return MLA_ERR_INVALID_ARG;
@@ -252,14 +269,51 @@ mla_status_t mla_append(const mla_plan_t* plan, const void* x, const int32_t* se
   mla_status_t st = mla_validate_cache(plan->cfg, cache);
   if (st != MLA_OK) return st;
   if (!aligned16(x) || ((uintptr_t)seq_idx & 3) || ((uintptr_t)pos & 3)) return MLA_ERR_ALIGNMENT;
-  return cuda_status(mla_launch_append(*plan, x, seq_idx, pos, N, *cache, (cudaStream_t)stream));
+  const cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = mla_profile_event(*plan, kProfAppend, false, s);
+  if (e == cudaSuccess) e = mla_launch_append(*plan, x, seq_idx, pos, N, *cache, s);
+  if (e == cudaSuccess) e = mla_profile_event(*plan, kProfAppend, true, s);
+  return cuda_status(e);
 }
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Staging of mla_decode_step_host inside the workspace, after the decode's own part:
+// seq_lens, x, q and out, each 256-byte aligned.
+struct HostStage {
+  size_t off_lens, off_x, off_q, off_out, total;
+};
+HostStage host_stage(const mla_plan& p, int B, size_t base) {
+  const mla_config_t& c = p.cfg;
+  const size_t eb = elem_bytes(c), qo = (size_t)B * c.n_heads * c.head_dim * eb;
+  HostStage h;
+  h.off_lens = align256(base);
+  h.off_x = h.off_lens + align256((size_t)B * sizeof(int32_t));
+  h.off_q = h.off_x + align256((size_t)B * c.hidden * eb);
+  h.off_out = h.off_q + align256(qo);
+  h.total = h.off_out + align256(qo);
+  return h;
+}
+
+// The decode kernel a call runs: the tensor-core kernel where the plan, cache and options
+// allow it, else the CUDA-core kernel.  MLA_OK, or the status that refuses the call.
+mla_status_t pick_kernel(const mla_plan& p, const mla_cache_t& c, int* kernel) {
+  *kernel = 1;
+  if (p.opt_kernel != 1 && mla_tc_kind_ok(p.cfg) && mla_tc_supported(p, c)) *kernel = 2;
+  if (p.opt_kernel == 2 && *kernel != 2) return MLA_ERR_UNSUPPORTED;
+  if (*kernel == 1 && (size_t)p.cfg.n_heads * p.cfg.d_c > 8192) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+}  // namespace
 
 size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B) {
   if (!plan || B <= 0) return 0;
   size_t n = mla_decode_layout(*plan, B, 1).total;
   if (mla_tc_kind_ok(plan->cfg) && mla_tc_capable(*plan)) n = std::max(n, mla_decode_layout(*plan, B, 2).total);
-  return n;
+  return host_stage(*plan, B, n).total;
 }
 
 mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
@@ -272,13 +326,54 @@ mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache, const 
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace) || ((uintptr_t)seq_lens & 3))
     return MLA_ERR_ALIGNMENT;
   int kernel = 1;
-  if (plan->opt_kernel != 1 && mla_tc_kind_ok(plan->cfg) && mla_tc_supported(*plan, *cache)) kernel = 2;
-  if (plan->opt_kernel == 2 && kernel != 2) return MLA_ERR_UNSUPPORTED;
-  if (kernel == 1 && (size_t)plan->cfg.n_heads * plan->cfg.d_c > 8192) return MLA_ERR_UNSUPPORTED;
+  if ((st = pick_kernel(*plan, *cache, &kernel)) != MLA_OK) return st;
   DecodeLayout L = mla_decode_layout(*plan, B, kernel);
   if (ws_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
   return cuda_status(mla_launch_decode(*plan, *cache, seq_lens, q, B, out, workspace, L,
                                        (cudaStream_t)stream));
+}
+
+mla_status_t mla_decode_step(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
+                             const void* x, const void* q, int32_t B, void* out, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  if (!plan || !seq_lens || !x || !q || !out || !workspace || B <= 0) return MLA_ERR_INVALID_ARG;
+  mla_status_t st = mla_validate_cache(plan->cfg, cache);
+  if (st != MLA_OK) return st;
+  if (B > cache->B) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(out) || !aligned16(workspace) || ((uintptr_t)seq_lens & 3))
+    return MLA_ERR_ALIGNMENT;
+  int kernel = 1;
+  if ((st = pick_kernel(*plan, *cache, &kernel)) != MLA_OK) return st;
+  DecodeLayout L = mla_decode_layout(*plan, B, kernel);
+  if (ws_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  return cuda_status(mla_launch_step(*plan, *cache, seq_lens, x, q, B, out, workspace, L, (cudaStream_t)stream));
+}
+
+mla_status_t mla_decode_step_host(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
+                                  const void* x, const void* q, int32_t B, void* out, void* workspace,
+                                  size_t ws_bytes, void* stream) {
+  if (!plan || !seq_lens || !x || !q || !out || !workspace || B <= 0) return MLA_ERR_INVALID_ARG;
+  mla_status_t st = mla_validate_cache(plan->cfg, cache);
+  if (st != MLA_OK) return st;
+  if (B > cache->B) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return MLA_ERR_ALIGNMENT;
+  int kernel = 1;
+  if ((st = pick_kernel(*plan, *cache, &kernel)) != MLA_OK) return st;
+  DecodeLayout L = mla_decode_layout(*plan, B, kernel);
+  const HostStage h = host_stage(*plan, B, L.total);
+  if (ws_bytes < h.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  const mla_config_t& c = plan->cfg;
+  const size_t eb = elem_bytes(c), qo = (size_t)B * c.n_heads * c.head_dim * eb;
+  char* w = (char*)workspace;
+  const cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(w + h.off_lens, seq_lens, (size_t)B * sizeof(int32_t), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(w + h.off_x, x, (size_t)B * c.hidden * eb, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(w + h.off_q, q, qo, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = mla_launch_step(*plan, *cache, (const int32_t*)(w + h.off_lens), w + h.off_x, w + h.off_q, B, w + h.off_out,
+                        workspace, L, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(out, w + h.off_out, qo, cudaMemcpyDeviceToHost, s);
+  return cuda_status(e);
 }
 
 mla_status_t mla_device_error(mla_plan_t* plan, int32_t* code) {

@@ -75,7 +75,11 @@ struct mla_plan {
   int opt_kernel = 0;
   int opt_splits = 0;
   const void* const* opt_events = nullptr;  // cudaEvent_t[2] or null
+  const void* const* opt_kernel_events = nullptr;  // cudaEvent_t[8] or null
   int opt_pdl = 1;                            // programmatic dependent launch
+  int64_t opt_wait_us = 1000000;              // bound of each pipeline wait (tensor-core kernel)
+  int opt_skip_tile = 0;                      // testing: leave out one latent copy per CTA
+  int opt_pf_dist = 2, opt_pf_mode = 1;       // L2 prefetch lookahead (tiles) and form
 };
 
 // Launches a kernel, with programmatic stream serialization when `pdl` is set (the kernel
@@ -96,15 +100,23 @@ inline cudaError_t mla_launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 blo
   return cudaLaunchKernelEx(&lc, kern, std::forward<Args>(args)...);
 }
 
-// Records profiling event i (0 before, 1 after the split-K kernel) when the option is set.
-// Under stream capture the record becomes an external event node of the graph, so the
-// event still marks each replay.  A failed record is returned, never left pending.
-inline cudaError_t mla_profile_event(const mla_plan& p, int i, cudaStream_t s) {
-  if (!p.opt_events) return cudaSuccess;
+// Kernels of a call that the profiling options can bracket with events.
+enum MlaProfKernel { kProfAppend = 0, kProfAbsorb = 1, kProfAttention = 2, kProfCombine = 3 };
+
+// Records the profiling event before (`after` false) or after a kernel launch when an
+// option asks for it: MLA_OPT_PROFILE_EVENTS brackets the split-K attention kernel,
+// MLA_OPT_PROFILE_KERNELS every kernel.  Under stream capture the record becomes an
+// external event node of the graph, so the event still marks each replay.  A failed record
+// is returned, never left pending.
+inline cudaError_t mla_profile_event(const mla_plan& p, MlaProfKernel k, bool after, cudaStream_t s) {
+  const void* ev = nullptr;
+  if (p.opt_kernel_events) ev = p.opt_kernel_events[2 * (int)k + (after ? 1 : 0)];
+  else if (p.opt_events && k == kProfAttention) ev = p.opt_events[after ? 1 : 0];
+  if (!ev) return cudaSuccess;
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   cudaError_t e = cudaStreamIsCapturing(s, &cs);
   if (e != cudaSuccess) return e;
-  return cudaEventRecordWithFlags((cudaEvent_t)p.opt_events[i], s,
+  return cudaEventRecordWithFlags((cudaEvent_t)ev, s,
                                   cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal
                                                                       : cudaEventRecordDefault);
 }
@@ -150,6 +162,12 @@ cudaError_t mla_launch_select_pairs(const mla_config_t& cfg, const void* q, cons
                                     int32_t* pair_idx, float* contrib, cudaStream_t s);
 cudaError_t mla_launch_append(const mla_plan& p, const void* x, const int32_t* seq_idx,
                               const int32_t* pos, int N, const mla_cache_t& c, cudaStream_t s);
+// Append of a decode step: token b goes to sequence b at position seq_lens[b] - 1.
+cudaError_t mla_launch_append_step(const mla_plan& p, const void* x, const int32_t* seq_lens, int B,
+                                   const mla_cache_t& c, cudaStream_t s);
+// One decode step (append of each sequence's new token, then decode), fused where it can be.
+cudaError_t mla_launch_step(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, const void* x,
+                            const void* q, int B, void* out, void* ws, const DecodeLayout& L, cudaStream_t s);
 cudaError_t mla_launch_decode(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens,
                               const void* q, int B, void* out, void* ws, const DecodeLayout& L,
                               cudaStream_t s);

@@ -406,16 +406,18 @@ def _softmax(s: np.ndarray) -> np.ndarray:
 
 
 def decode_unabsorbed(q: np.ndarray, c: np.ndarray, kr: np.ndarray, W_uk: np.ndarray,
-                      W_uv: np.ndarray, pair_idx: np.ndarray, theta: np.ndarray) -> np.ndarray:
+                      W_uv: np.ndarray, pair_idx: np.ndarray, theta: np.ndarray, scale=None) -> np.ndarray:
     """Attention of one sequence's new query over its latent cache, by definition.
 
     NOTES §关键设计 / SVDjoint: keys' NoPE part is reconstructed as K_nope = c_kv W_uk and
     values as V = c_kv W_uv; the retained RoPE dims give a separate score term.  The
     query is split the same way: NoPE dims unrotated, kept pairs rotated at the query
-    position p = L - 1.  Scale 1/sqrt(d_h).
+    position p = L - 1.  Scale 1/sqrt(d_h), the original layer's, unless `scale` is given
+    (a caller-chosen softmax scale multiplies the scores in its place).
 
     q [H][d_h]; c [L][d_c]; kr [L][n_kv][2r] (already rotated)  ->  o [H][d_h]
     """
+    sc = 1.0 / np.sqrt(q.shape[1]) if scale is None else float(scale)
     H, dh = q.shape
     n_kv, r = pair_idx.shape
     G = H // n_kv
@@ -430,7 +432,7 @@ def decode_unabsorbed(q: np.ndarray, c: np.ndarray, kr: np.ndarray, W_uk: np.nda
         V = c @ W_uv[g]                           # [L][d_h]
         q_nope = q[h, nope[g]]
         q_rope = rotate(q[h, rope[g]].reshape(r, 2), p, th[g]).reshape(2 * r)
-        s = (K_nope @ q_nope + kr[:, g, :] @ q_rope) / np.sqrt(dh)
+        s = (K_nope @ q_nope + kr[:, g, :] @ q_rope) * sc
         o[h] = _softmax(s) @ V
     return o
 

@@ -33,6 +33,10 @@ int main(void) {
   CHECK(mla_cache_bytes_per_token(&cfg) == 32 + 8 + 512, "int2 cache bytes per token");
   cfg.cache_kind = MLA_CACHE_SAME; cfg.d_c = 256;
 
+  cfg.softmax_scale = -1.0f;
+  CHECK(mla_cache_bytes_per_token(&cfg) == 0, "a negative softmax scale is an invalid config");
+  cfg.softmax_scale = 0.0f;
+
   int32_t pairs[32 * 4];
   CHECK(mla_fixed_pairs(&cfg, MLA_PAIRS_HIGH, pairs) == MLA_OK && pairs[0] == 0 && pairs[3] == 3,
         "high-frequency pair set");

@@ -480,3 +480,25 @@ def test_multi_query_causal_decode(wl, kernel):
         ref = O.decode_unabsorbed(q[j], cc["c"][:p + 1], cc["kr"][:p + 1], case.conv["W_uk"], case.conv["W_uv"],
                                   case.conv["pair_idx"], case.theta)
         assert_close(got[j], ref, wl.dtype, f"query at position {p}")
+
+
+@pytest.mark.parametrize("idx", [2, 4, 1], ids=["bf16_dc256", "int4_dc128", "gqa_cuda_core"])
+def test_decode_softmax_scale(idx):
+    """A config softmax_scale other than 1/sqrt(d_h) scales every score (both kernels)."""
+    wl = PARITY_WORKLOADS[idx]
+    case = case_for(wl)
+    scale = 0.6 / np.sqrt(wl.head_dim)
+    cfg = mla.make_config(wl.hidden, wl.n_heads, wl.n_kv_heads, wl.head_dim, wl.r_pairs, wl.d_c, wl.rope_base,
+                          wl.dtype, wl.cache, wl.resid, softmax_scale=scale)
+    plan = mla.mla_plan_create(cfg, **plan_inputs(case))
+    got = run_decode(case, plan, cfg)
+    assert mla.mla_device_error(plan) == 0
+    for b in case.seqs:
+        if case.lens[b] == 0:
+            continue
+        cc = case.cache[b]
+        ref = O.decode_unabsorbed(case.q[b], cc["c"], cc["kr"], case.conv["W_uk"], case.conv["W_uv"],
+                                  case.conv["pair_idx"], case.theta, scale=scale)
+        assert_close(got[b], ref, wl.dtype, f"{wl.name} scale seq {b}")
+        assert not np.allclose(ref, case.reference(b), rtol=1e-3)
+    plan.close()

@@ -220,6 +220,29 @@ def test_T6_softmax_edge_cases():
         np.testing.assert_allclose(o[h], c[0] @ W_uv[h // G], rtol=1e-12, atol=1e-13)
 
 
+def test_T6s_softmax_scale():
+    """A caller-chosen score scale (the boundary's softmax_scale): the default is the
+    original layer's 1/sqrt(d_h); the scores are linear in q (the rotation is linear), so
+    scale k/sqrt(d_h) equals the default decode of k*q; scale 0 gives uniform weights."""
+    rng = np.random.default_rng(19)
+    W_q, W_dkv, W_kr, W_uk, W_uv, pair_idx, theta = _tiny_conv(rng)
+    H, G, dh = 4, 2, 8
+    x = rng.standard_normal((9, 40))
+    c, kr = O.append(x, np.arange(9), W_dkv, W_kr, pair_idx, theta)
+    q = (rng.standard_normal(40) @ W_q).reshape(H, dh)
+    base = O.decode_unabsorbed(q, c, kr, W_uk, W_uv, pair_idx, theta)
+    np.testing.assert_array_equal(O.decode_unabsorbed(q, c, kr, W_uk, W_uv, pair_idx, theta,
+                                                      scale=1.0 / np.sqrt(dh)), base)
+    for k in (0.37, 2.5):
+        np.testing.assert_allclose(O.decode_unabsorbed(q, c, kr, W_uk, W_uv, pair_idx, theta, scale=k / np.sqrt(dh)),
+                                   O.decode_unabsorbed(k * q, c, kr, W_uk, W_uv, pair_idx, theta),
+                                   rtol=1e-12, atol=1e-13)
+    assert not np.allclose(O.decode_unabsorbed(q, c, kr, W_uk, W_uv, pair_idx, theta, scale=2.5 / np.sqrt(dh)), base)
+    o0 = O.decode_unabsorbed(q, c, kr, W_uk, W_uv, pair_idx, theta, scale=0.0)
+    for h in range(H):
+        np.testing.assert_allclose(o0[h], (c @ W_uv[h // G]).mean(axis=0), rtol=1e-12, atol=1e-13)
+
+
 # ------------------------------------------------------------------ T7
 def test_T7_rope_relative_position_and_norms():
     rng = np.random.default_rng(10)
