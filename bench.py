@@ -33,7 +33,7 @@ METRIC = "MLA decode cached tokens/s (batch×ctx per step) and % of B200 HBM pea
 UNIT = "cached tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
-PER_WORKLOADS = ("llama2_7b_ragged_bf16", "llama2_7b_int4", "llama2_7b_int4_r128")
+PER_WORKLOADS = ("llama2_7b_ragged_bf16", "llama2_7b_int4", "llama2_7b_int4_r128", "llama2_7b_int2")
 
 
 def parse():
@@ -65,7 +65,8 @@ def wl_config(wl, lens):
             "cached_tokens_per_step": int(np.sum(lens)), "hidden": wl.hidden, "heads": wl.n_heads,
             "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "r_pairs": wl.r_pairs, "d_c": wl.d_c,
             "latent_cache": ("int4 g32 + fp16 scales" + (f", {wl.resid}-token bf16 residual window" if wl.resid else "")
-                             if wl.cache == "int4_g32" else wl.dtype),
+                             if wl.cache == "int4_g32" else
+                             "int2 g32 + fp16 scales" if wl.cache == "int2_g32" else wl.dtype),
             "step": "mla_append(B new tokens) + mla_decode(B queries)"}
 
 
@@ -85,8 +86,10 @@ def oracle_decode_sample(wl, n_tokens, rounds, seconds_cap=None):
     x = gen.context_tokens(small, 0, n_tokens)
     c, kr = O.append(x, np.arange(n_tokens), conv["W_dkv"], conv["W_krope"], conv["pair_idx"], theta)
     kr = gen.cast(kr, wl.dtype)
-    if wl.cache == "int4_g32":
-        codes, scales = O.quant_int4_g32(c)
+    quant = {"int4_g32": (O.quant_int4_g32, O.dequant_int4_g32),
+             "int2_g32": (O.quant_int2_g32, O.dequant_int2_g32)}.get(wl.cache)
+    if quant:
+        codes, scales = quant[0](c)
         plain = gen.cast(c, wl.dtype)
     else:
         c = gen.cast(c, wl.dtype)
@@ -95,8 +98,8 @@ def oracle_decode_sample(wl, n_tokens, rounds, seconds_cap=None):
     t_start = time.perf_counter()
     for _ in range(rounds):
         t0 = time.perf_counter()
-        cc = O.dequant_int4_g32(codes, scales) if wl.cache == "int4_g32" else c
-        if wl.cache == "int4_g32" and wl.resid:
+        cc = quant[1](codes, scales) if quant else c
+        if quant and wl.resid:
             cc = O.residual_window(cc, plain, wl.resid)
         O.decode_unabsorbed(q, cc, kr, conv["W_uk"], conv["W_uv"], conv["pair_idx"], theta)
         times.append(time.perf_counter() - t0)
@@ -478,7 +481,7 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": wl.dtype if wl.cache != "int4_g32" else "bf16 (int4 latent cache)",
+        "dtype": wl.dtype if wl.cache == "same" else f"bf16 ({wl.cache[:4]} latent cache)",
         "data": "synthetic (seeded generators; random-init layer of the named shape)",
         "config": dict(wl_config(wl, bn.lens), parallelism=f"replicas x{world}" if world > 1 else "single GPU",
                        l2=f"{bn.n_rep} cache replicas rotated per step "

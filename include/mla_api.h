@@ -79,8 +79,9 @@ typedef enum {
 /* MLA_CACHE_INT2_G32 is the same scheme at 2 bits (Notes §关键设计: 4-bit or 2-bit
  * quantisation stacks on the latent): per token, groups of 32, fp16 scale s = fp16(absmax),
  * codes clamp(round_half_even(c/s), -1, 1) (0 when s == 0), two's-complement 2-bit fields,
- * element 4i+k in bits 2k..2k+1 of byte i; value = code*s.  Decoded by the CUDA-core
- * kernel (the tensor-core kernel reports MLA_ERR_UNSUPPORTED when forced). */
+ * element 4i+k in bits 2k..2k+1 of byte i; value = code*s.  The quantised caches are
+ * decoded by the tensor-core kernel at d_c = 128 (32 heads, r = 4) and by the CUDA-core
+ * kernel otherwise. */
 #define MLA_RESID_WINDOW 128
 
 typedef struct {

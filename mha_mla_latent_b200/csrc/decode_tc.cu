@@ -184,21 +184,24 @@ __device__ __forceinline__ MlaLoc tc_loc(const TcArgs& a, int b, int t) {
   return mla_loc(a.cache, b, t, a.err);
 }
 
-// INT4: int4 latent cache (dequantised in shared memory); RESID: with the residual window
-// ring (INT4 only); PAGED: cache addressed through a block table.  Each combination is its
-// own instantiation, so the common ones carry no code of the others.
-template <bool INT4, bool RESID, bool PAGED, int R2>
+// QB: code width of a quantised latent cache (4 or 2; dequantised in shared memory), 0 for a
+// bf16 latent; RESID: with the residual window ring (4-bit only); PAGED: cache addressed
+// through a block table.  Each combination is its own instantiation, so the common ones
+// carry no code of the others.
+template <int QB, bool RESID, bool PAGED, int R2>
 __global__ void __launch_bounds__(384, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
                  const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (sbase_u32 - smem_u32(smem_raw));
+  constexpr bool INT4 = QB != 0;   // quantised latent (4- or 2-bit codes)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int dc = a.d_c, R = a.R;
   const int n_cbox = dc / 64;
   const uint32_t c_stage = (uint32_t)n_cbox * kBox;
-  const uint32_t raw_codes = (uint32_t)kTile * (dc / 2), raw_stage = raw_codes + (uint32_t)kTile * (dc / 16);
+  constexpr int kCodeBytes64 = QB * 8;   // code bytes of 64 latent values
+  const uint32_t raw_codes = (uint32_t)kTile * (dc / 64) * kCodeBytes64, raw_stage = raw_codes + (uint32_t)kTile * (dc / 16);
   const uint32_t S_COL = 0, O_COL = 2 * kH;
   Bars bars{sbase_u32 + a.off_bar, a.NC, a.NRAW, a.NP, a.NO};
   Misc* misc = reinterpret_cast<Misc*>(sbase + a.off_misc);
@@ -436,7 +439,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
         mbar_wait(bars.mma_done(), 0, &never, lim);
       }
     } else if (INT4 && warp >= 2) {
-      // ============================================================ int4 dequantisation
+      // ============================================================ dequantisation
       const int tid_dq = threadIdx.x - 64;   // 0..63: token rows tid_dq, tid_dq + 64
       TileIter it;
       it.init(&a.sched, w);
@@ -468,22 +471,40 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
                 *reinterpret_cast<uint4*>(C + half * kBox + ((ch ^ (tok & 7)) * 16)) = __ldg(src + half * 8 + ch);
           } else if (tok < nvalid) {
             const __half* sc = reinterpret_cast<const __half*>(raw + raw_codes) + tok * (dc / 32);
+            const uint8_t* codes = raw + tok * (dc / 64) * kCodeBytes64;
             for (int half = 0; half < dc / 64; ++half) {
-              const uint4 c0 = *reinterpret_cast<const uint4*>(raw + tok * (dc / 2) + half * 32);
-              const uint4 c1 = *reinterpret_cast<const uint4*>(raw + tok * (dc / 2) + half * 32 + 16);
               const float s0 = __half2float(sc[half * 2]), s1 = __half2float(sc[half * 2 + 1]);
-              const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+              if (QB == 4) {   // two's-complement nibbles, element 2i in the low nibble of byte i
+                const uint4 c0 = *reinterpret_cast<const uint4*>(codes + half * 32);
+                const uint4 c1 = *reinterpret_cast<const uint4*>(codes + half * 32 + 16);
+                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
   #pragma unroll
-              for (int ch = 0; ch < 8; ++ch) {           // 8 latent values per 16-byte chunk
-                const uint32_t wd = words[ch];
-                const float s = ch < 4 ? s0 : s1;
-                uint32_t o[4];
+                for (int ch = 0; ch < 8; ++ch) {           // 8 latent values per 16-byte chunk
+                  const uint32_t wd = words[ch];
+                  const float s = ch < 4 ? s0 : s1;
+                  uint32_t o[4];
   #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const uint32_t byte = (wd >> (8 * j)) & 0xFFu;
-                  o[j] = pack_bf16x2((float)nib_to_int(byte & 15u) * s, (float)nib_to_int(byte >> 4) * s);
+                  for (int j = 0; j < 4; ++j) {
+                    const uint32_t byte = (wd >> (8 * j)) & 0xFFu;
+                    o[j] = pack_bf16x2((float)nib_to_int(byte & 15u) * s, (float)nib_to_int(byte >> 4) * s);
+                  }
+                  *reinterpret_cast<uint4*>(C + half * kBox + ((ch ^ (tok & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
                 }
-                *reinterpret_cast<uint4*>(C + half * kBox + ((ch ^ (tok & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
+              } else {         // two's-complement 2-bit fields, element 4i+k in bits 2k..2k+1 of byte i
+                const uint4 c0 = *reinterpret_cast<const uint4*>(codes + half * 16);
+                const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
+  #pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {           // 8 latent values: 16 bits of codes
+                  const uint32_t bits = (words[ch >> 1] >> (16 * (ch & 1))) & 0xFFFFu;
+                  const float s = ch < 4 ? s0 : s1;
+                  uint32_t o[4];
+  #pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    const int f0 = (int)((bits >> (4 * j)) & 3u), f1 = (int)((bits >> (4 * j + 2)) & 3u);
+                    o[j] = pack_bf16x2((float)(f0 >= 2 ? f0 - 4 : f0) * s, (float)(f1 >= 2 ? f1 - 4 : f1) * s);
+                  }
+                  *reinterpret_cast<uint4*>(C + half * kBox + ((ch ^ (tok & 7)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
               }
             }
           } else {
@@ -816,10 +837,10 @@ struct TcLayout {
   uint32_t off_c, off_q, off_p, off_raw, off_qr, off_kr, off_bar, off_misc, total;
 };
 
-static TcLayout tc_layout(int dc, int R, int r2, bool int4) {
+static TcLayout tc_layout(int dc, int R, int r2, bool int4, int qbits) {
   const uint32_t budget = 232448 - 1024;   // max dynamic smem per block minus alignment slack
   const uint32_t c_stage = (uint32_t)(dc / 64) * kBox;
-  const uint32_t raw_stage = (uint32_t)kTile * (dc / 2) + (uint32_t)kTile * (dc / 16);
+  const uint32_t raw_stage = (uint32_t)kTile * (dc * qbits / 8) + (uint32_t)kTile * (dc / 16);
   const uint32_t q_bytes = (uint32_t)(dc / 64 > 2 ? dc / 64 - 2 : 0) * kQBox;  // boxes 0-1 sit in P^T padding
   const uint32_t qr_bytes = 2u * kH * r2 * 4;   // two pieces' RoPE queries
   const uint32_t kr_bytes = (uint32_t)kTile * R * 2;
@@ -860,21 +881,24 @@ static TcLayout tc_layout(int dc, int R, int r2, bool int4) {
 }  // namespace mla
 
 // Shapes the tensor-core kernel covers: bf16, 32 query heads, d_c in {64, 128, 256}, r = 4
-// kept pairs per KV head (RoPE width a multiple of 64); the int4 cache with d_c = 128.
+// kept pairs per KV head (RoPE width a multiple of 64); the int4 and 2-bit caches with d_c = 128.
 bool mla_tc_capable(const mla_plan& p) {
   const mla_config_t& cfg = p.cfg;
   if (cfg.dtype != MLA_BF16 || cfg.n_heads != mla::tc::kH) return false;
   if (cfg.d_c % 64 != 0 || cfg.d_c > 256) return false;
   if (p.R == 0 || p.R % 64 != 0 || 2 * cfg.r_pairs != 8) return false;   // 2r = 8 (r = 4) build
-  if (mla_kind_int4(cfg.cache_kind) && cfg.d_c != 128) return false;
-  const mla::tc::TcLayout L = mla::tc::tc_layout(cfg.d_c, p.R, 2 * cfg.r_pairs, mla_kind_int4(cfg.cache_kind));
+  const bool quant = mla_kind_quant(cfg.cache_kind);
+  if (quant && cfg.d_c != 128) return false;
+  const mla::tc::TcLayout L =
+      mla::tc::tc_layout(cfg.d_c, p.R, 2 * cfg.r_pairs, quant, mla_quant_bits(cfg.cache_kind));
   return L.total <= 232448;
 }
 
-// The int4 scale rows are fetched with 1-D bulk copies, which need an even capacity.
+// The scale rows of a quantised cache are fetched with 1-D bulk copies, which need an even
+// capacity.
 bool mla_tc_supported(const mla_plan& p, const mla_cache_t& c) {
   if (!mla_tc_capable(p)) return false;
-  if (mla_kind_int4(p.cfg.cache_kind) && c.T_cap % 2 != 0) return false;
+  if (mla_kind_quant(p.cfg.cache_kind) && c.T_cap % 2 != 0) return false;
   return true;
 }
 
@@ -884,13 +908,15 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
                                  cudaStream_t s) {
   using namespace mla::tc;
   const mla_config_t& cfg = p.cfg;
-  const bool int4 = mla_kind_int4(cfg.cache_kind);
+  const bool int4 = mla_kind_quant(cfg.cache_kind);   // quantised latent: 4- or 2-bit codes
+  const int qbits = mla_quant_bits(cfg.cache_kind);
   const int dc = cfg.d_c, R = p.R;
+  const int code_row = dc * qbits / 8;   // code bytes per token
   CUtensorMap tm_c, tm_q;
   const uint64_t rows = mla_cache_rows(c);
   bool ok = true;
   if (int4)
-    ok &= make_map_2d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.c_kv, dc / 2, rows, dc / 2, dc / 2, kTile,
+    ok &= make_map_2d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.c_kv, code_row, rows, code_row, code_row, kTile,
                       CU_TENSOR_MAP_SWIZZLE_NONE);
   else
     ok &= make_map_2d(&tm_c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.c_kv, dc, rows, (uint64_t)dc * 2, 64, kTile,
@@ -898,7 +924,7 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
   ok &= make_map_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qlat, dc, (uint64_t)B * kH, (uint64_t)dc * 2, 64, kH,
                     CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
-  const TcLayout L = tc_layout(dc, R, 2 * cfg.r_pairs, int4);
+  const TcLayout L = tc_layout(dc, R, 2 * cfg.r_pairs, int4, qbits);
   TcArgs a;
   a.B = B; a.H = kH; a.d_c = dc; a.R = R; a.r2 = 2 * cfg.r_pairs; a.T_cap = c.T_cap; a.P = P;
   a.sched = sched; a.opart = opart; a.mlpart = mlpart; a.qrope = qrope;
@@ -908,7 +934,7 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
   a.c_resid = (const __nv_bfloat16*)c.c_resid;
   a.resid_pos = c.resid_pos;
   a.kr_base = (const uint8_t*)c.k_rope;
-  a.c_row = int4 ? (uint32_t)dc / 2 : (uint32_t)dc * 2;
+  a.c_row = int4 ? (uint32_t)code_row : (uint32_t)dc * 2;
   a.kr_row = (uint32_t)R * 2;
   a.wait_ns = (uint64_t)p.opt_wait_us * 1000u;
   a.pf_dist = p.opt_pf_dist;
@@ -919,10 +945,11 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
   a.off_qr = L.off_qr; a.off_kr = L.off_kr; a.off_bar = L.off_bar; a.off_misc = L.off_misc;
   // the RoPE width per KV head is a compile-time constant so the score loop fully unrolls
   // and the per-head registers never move to local memory
-  const bool resid = int4 && c.c_resid, paged = c.block_table != nullptr;
-  auto kern = int4 ? (resid ? (paged ? decode_tc_kernel<true, true, true, 8> : decode_tc_kernel<true, true, false, 8>)
-                            : (paged ? decode_tc_kernel<true, false, true, 8> : decode_tc_kernel<true, false, false, 8>))
-                   : (paged ? decode_tc_kernel<false, false, true, 8> : decode_tc_kernel<false, false, false, 8>);
+  const bool resid = int4 && qbits == 4 && c.c_resid, paged = c.block_table != nullptr;
+  auto kern = !int4        ? (paged ? decode_tc_kernel<0, false, true, 8> : decode_tc_kernel<0, false, false, 8>)
+              : qbits == 2 ? (paged ? decode_tc_kernel<2, false, true, 8> : decode_tc_kernel<2, false, false, 8>)
+              : resid      ? (paged ? decode_tc_kernel<4, true, true, 8> : decode_tc_kernel<4, true, false, 8>)
+                           : (paged ? decode_tc_kernel<4, false, true, 8> : decode_tc_kernel<4, false, false, 8>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
   // the optional profiling events bracket the launch alone, after all host-side set-up

@@ -21,7 +21,8 @@ from workloads import get
 
 pytestmark = pytest.mark.gpu
 
-FULL = ["smollm135m_gqa_bf16", "llama2_7b_bf16", "llama2_7b_ragged_bf16", "llama2_7b_int4", "llama2_7b_int4_r128"]
+FULL = ["smollm135m_gqa_bf16", "llama2_7b_bf16", "llama2_7b_ragged_bf16", "llama2_7b_int4", "llama2_7b_int4_r128",
+        "llama2_7b_int2"]
 
 
 def _sampled(wl, lens):

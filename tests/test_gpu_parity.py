@@ -235,11 +235,11 @@ def test_decode_parity(wl, kernel):
     """kernel 0: the plan's choice; 1: CUDA-core split-K; 2: tcgen05 (bf16, 32 heads)."""
     case = case_for(wl)
     cfg, plan = make_plan(case, kernel=kernel)
-    if kernel == 2 and (wl.dtype == "f32" or wl.n_heads != 32 or wl.cache == "int2_g32"):
+    if kernel == 2 and (wl.dtype == "f32" or wl.n_heads != 32):
         with pytest.raises(mla.MlaError) as ei:
             run_decode(case, plan, cfg)
         assert ei.value.status == mla.MLA_ERR_UNSUPPORTED
-        pytest.skip("outside the tensor-core kernel (fp32, H != 32 or the 2-bit cache)")
+        pytest.skip("outside the tensor-core kernel (fp32 or H != 32)")
     got = run_decode(case, plan, cfg)
     assert mla.mla_device_error(plan) == 0
     for b in case.seqs:
@@ -416,8 +416,8 @@ def test_paged_append_matches_contiguous(wl):
 def test_paged_decode_parity(wl, kernel):
     """Decode over a paged cache (shuffled blocks) equals the decode over the contiguous
     cache bit for bit, and the oracle within tolerance."""
-    if kernel == 2 and (wl.dtype == "f32" or wl.n_heads != 32 or wl.cache == "int2_g32"):
-        pytest.skip("outside the tensor-core kernel (fp32, H != 32 or the 2-bit cache)")
+    if kernel == 2 and (wl.dtype == "f32" or wl.n_heads != 32):
+        pytest.skip("outside the tensor-core kernel (fp32 or H != 32)")
     case = case_for(wl)
     cfg, plan = make_plan(case, kernel=kernel)
     lens = [int(L) for L in case.lens]

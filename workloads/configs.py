@@ -96,6 +96,8 @@ PARITY_WORKLOADS = [
 # quantised cache).
 EXTRA_WORKLOADS = [
     WORKLOADS[4].with_(name="llama2_7b_int4_r128", resid=128),
+    # the same shape with the 2-bit latent (Notes §关键设计: 4- or 2-bit quantisation of the latent)
+    WORKLOADS[4].with_(name="llama2_7b_int2", cache="int2_g32"),
 ]
 
 
