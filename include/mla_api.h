@@ -102,7 +102,7 @@ typedef struct {
  * Paged (block_table != NULL): the arrays are pools of n_blocks blocks of MLA_BLOCK_TOKENS
  * (128) tokens, and token t of sequence b lives in token row t % 128 of pool block
  * block_table[b][t / 128]; every array below is then read with B := n_blocks and
- * T_cap := 128 (so k_rope holds 4 blocks of 32 tokens per pool block).  T_cap must be a
+ * T_cap := 128.  T_cap must be a
  * multiple of 128 (the logical capacity: T_cap / 128 table entries per sequence).  The
  * README "MHA2MLA" runs ragged LongBench batches; 128-token blocks match the decode tile,
  * so each tile of the attention kernel reads one block.  A table entry outside
@@ -110,10 +110,9 @@ typedef struct {
  *   c_kv      SAME: [B][T_cap][d_c] dtype;  INT4*: [B][T_cap][d_c/2] uint8 codes;
  *             INT2: [B][T_cap][d_c/4] uint8 codes
  *   c_scales  INT4*, INT2: [B][T_cap][d_c/32] fp16;  SAME: must be NULL
- *   k_rope    [B][ceil(T_cap/32)][n_kv][32][2r] dtype (may be NULL when r == 0): the kept
- *             RoPE key dims in blocks of 32 tokens, KV-head-major inside a block, so the
- *             2r dims of one KV head for 32 consecutive tokens are contiguous; element
- *             (b, t, g, j) sits at ((b*ceil(T_cap/32) + t/32)*n_kv + g)*32*2r + (t%32)*2r + j
+ *   k_rope    [B][T_cap][n_kv][2r] dtype (may be NULL when r == 0): the kept RoPE key
+ *             dims, one row of n_kv*2r values per token (token-major, like c_kv); element
+ *             (b, t, g, j) sits at ((b*T_cap + t)*n_kv + g)*2r + j
  *   c_resid   INT4_G32_R128: [B][128][d_c] dtype, the residual ring; otherwise NULL
  *   resid_pos INT4_G32_R128: [B][128] int32, the position each ring slot holds; set every
  *             entry to -1 before a sequence's first append (and again when a sequence

@@ -48,8 +48,8 @@ class LatentCache:
             self.c_resid = torch.zeros(B, W, cfg.d_c, dtype=dt, device=device)
             self.resid_pos = torch.full((B, W), -1, dtype=torch.int32, device=device)
         R = cfg.n_kv_heads * 2 * cfg.r_pairs
-        # blocked layout [B][ceil(T_cap/32)][n_kv][32][2r] (see mla_cache_t; pool blocks when paged)
-        self.k_rope = torch.zeros(rows, (cap + 31) // 32, cfg.n_kv_heads, 32, 2 * cfg.r_pairs, dtype=dt,
+        # token-major layout [B][T_cap][n_kv][2r] (see mla_cache_t; pool blocks when paged)
+        self.k_rope = torch.zeros(rows, cap, cfg.n_kv_heads, 2 * cfg.r_pairs, dtype=dt,
                                   device=device) if R > 0 else None
         self.struct = _lib.cache_struct(self.c_kv, self.c_scales, self.k_rope, B, T_cap, self.c_resid,
                                         self.resid_pos, self.block_table, self.n_blocks)
@@ -106,20 +106,13 @@ class LatentCache:
         if self.resid_pos is not None:
             self.resid_pos[b].fill_(-1)
 
-    def _kr_index(self, b: int, t0: int, t1: int):
-        pb, pt = self._loc(b, t0, t1)
-        dev = self.k_rope.device
-        return pb.to(dev), (pt // 32).to(dev), (pt % 32).to(dev)
-
     def k_rope_tokens(self, b: int, t0: int, t1: int) -> torch.Tensor:
         """RoPE key dims of tokens [t0, t1) of sequence b, as [t1-t0][n_kv][2r] (a copy)."""
-        pb, blk, row = self._kr_index(b, t0, t1)
-        return self.k_rope.permute(0, 1, 3, 2, 4)[pb, blk, row]
+        return self._rows(self.k_rope, b, t0, t1)
 
     def set_k_rope_tokens(self, b: int, t0: int, values: torch.Tensor) -> None:
         """Write [n][n_kv][2r] RoPE key dims as tokens [t0, t0+n) of sequence b."""
-        pb, blk, row = self._kr_index(b, t0, t0 + values.shape[0])
-        self.k_rope.permute(0, 1, 3, 2, 4)[pb, blk, row] = values.to(self.k_rope.device, self.k_rope.dtype)
+        self._set_rows(self.k_rope, b, t0, values)
 
     def nbytes_used(self, seq_lens) -> int:
         per_tok = _lib.mla_cache_bytes_per_token(self.cfg)

@@ -190,8 +190,8 @@ __device__ __forceinline__ MlaLoc tc_loc(const TcArgs& a, int b, int t) {
 // carry no code of the others.
 template <int QB, bool RESID, bool PAGED, int R2>
 __global__ void __launch_bounds__(384, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
-                 const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ TcArgs a) {
+decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_q,
+                 const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ TcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (sbase_u32 - smem_u32(smem_raw));
@@ -238,6 +238,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_c);
     tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_kr);
   }
   const uint32_t tmem_cols = (O_COL + a.NO * dc) <= 256 ? 256u : 512u;
   if (warp == 1) {
@@ -271,10 +272,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
         const MlaLoc lc = tc_loc<PAGED>(a, ti.b, ti.t);
         const size_t row = (size_t)lc.pb * lc.cap + lc.pt;
         const uint8_t* cp = reinterpret_cast<const uint8_t*>(a.cache.c_kv) + row * a.c_row;
-        const uint8_t* kp = a.kr_base + mla_kr_offset(lc.pb, lc.pt, 0, 0, lc.cap, R / R2, R2) * 2;
+        const uint8_t* kp = a.kr_base + row * a.kr_row;
         const uint8_t* sp = INT4 ? reinterpret_cast<const uint8_t*>(a.scales) + row * (dc / 16) : nullptr;
         const uint32_t cbytes = (uint32_t)nvalid * a.c_row;
-        const uint32_t kbytes = (uint32_t)((nvalid + 31) / 32) * (uint32_t)(R / R2) * 32u * R2 * 2u;
+        const uint32_t kbytes = (uint32_t)nvalid * a.kr_row;
         const uint32_t sbytes = INT4 ? (uint32_t)nvalid * (dc / 16) : 0u;
         if (a.pf_mode == 2) {   // bulk prefetches (sizes rounded down to 16 bytes: a hint)
           if (lane == 0) {
@@ -546,33 +547,34 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
       return wwait(bars.grp(i), ph & 1);
     };
     const int G = kH / (R / R2);         // query heads per KV head
-    // RoPE keys: in the blocked cache layout a tile's keys (4 blocks of [n_kv][32][2r]) are
-    // one contiguous range, brought into the shared stage by a single bulk copy.  Each warp
-    // moves its part (block q, the KV heads of its 16 heads: lane t reads token t, so the
-    // reads are conflict-free) into registers as soon as the copy lands and releases the
-    // stage; the eighth warp to release it issues the copy of the tile after.  The
-    // registers hold tile n+1's keys while tile n is processed, so the copy of tile n+2
-    // has a whole tile period to land.
-    const int n_kv = R / R2;
-    const uint32_t kr_blk = (uint32_t)n_kv * 32u * R2 * 2u;   // bytes per 32-token block
+    // RoPE keys: a tile's keys (128 token rows of n_kv*2r values) come into the shared stage
+    // as 64-column boxes with the 128-byte swizzle: row t of a box holds 8 KV heads' 2r = 8
+    // dims, the 16-byte chunk of head g at chunk (g % 8) ^ (t % 8), so a warp whose lane t
+    // reads "KV head g of token t" hits 8 different chunks per 8 rows (conflict-free).  Each
+    // warp moves its part (its 32 tokens, the KV heads of its 16 heads) into registers as
+    // soon as the copy lands and releases the stage; the eighth warp to release it issues
+    // the copy of the tile after.  The registers hold tile n+1's keys while tile n is
+    // processed, so the copy of tile n+2 has a whole tile period to land.
+    const int n_kbox = R / 64;   // 64-column boxes per tile (8 KV heads of 2r = 8 each)
     uint4 kr[kHh];
     auto issue_kr = [&](const TileIter& ti) {   // one thread
       if (!ti.valid()) return;
-      const int nblk = min(4, (ti.t1 - ti.t + 31) / 32);
       const MlaLoc lc = tc_loc<PAGED>(a, ti.b, ti.t);
-      const uint8_t* src = a.kr_base + mla_kr_offset(lc.pb, lc.pt, 0, 0, lc.cap, n_kv, R2) * 2;
+      const int row = lc.pb * lc.cap + lc.pt;
       fence_proxy_async_smem();
-      mbar_expect_tx(bars.kr_full(), nblk * kr_blk);
-      for (int k = 0; k < nblk; ++k)   // one copy per 32-token block: they proceed in parallel
-        bulk_load(sbase_u32 + a.off_kr + k * kr_blk, src + (size_t)k * kr_blk, kr_blk, bars.kr_full());
+      mbar_expect_tx(bars.kr_full(), (uint32_t)n_kbox * kBox);
+      for (int k = 0; k < n_kbox; ++k)
+        tma_load_2d(sbase_u32 + a.off_kr + k * kBox, &tm_kr, bars.kr_full(), k * 64, row);
       misc->kr_issued += 1;
     };
     auto fetch_kr = [&](int k, const TileIter& ti_after) -> bool {   // tile k's keys -> kr
       if (!wwait(bars.kr_full(), k & 1)) return false;
-      const uint8_t* blk = sbase + a.off_kr + q * kr_blk + lane * 16;
+      const uint8_t* rowp = sbase + a.off_kr + tr * 128;
 #pragma unroll
-      for (int h = 0; h < kHh; ++h)
-        kr[h] = *reinterpret_cast<const uint4*>(blk + (size_t)((kHh * hh + h) / G) * 32 * 16);
+      for (int h = 0; h < kHh; ++h) {
+        const int g = (kHh * hh + h) / G;
+        kr[h] = *reinterpret_cast<const uint4*>(rowp + (g >> 3) * kBox + (((g & 7) ^ (tr & 7)) << 4));
+      }
       __syncwarp();
       if (lane == 0) {
         __threadfence_block();
@@ -847,7 +849,7 @@ static TcLayout tc_layout(int dc, int R, int r2, bool int4, int qbits) {
   auto size = [&](int nc, int nraw, int np) {
     uint32_t s = nc * c_stage + q_bytes + np * kPtBytes + kr_bytes;
     s += int4 ? ((nraw * raw_stage + 1023) & ~1023u) : 0;
-    s += qr_bytes + 8 * (2 * nc + 2 * nraw + kFixedBars) + sizeof(Misc) + 64;
+    s += qr_bytes + 8 * (2 * nc + 2 * nraw + kFixedBars) + sizeof(Misc) + 64 + 1024;
     return s;
   };
   int nc = 2, np = 1, nraw = int4 ? 2 : 0;
@@ -867,7 +869,7 @@ static TcLayout tc_layout(int dc, int R, int r2, bool int4, int qbits) {
   L.off_q = o; o += q_bytes;
   L.off_raw = o; o += int4 ? ((nraw * raw_stage + 1023) & ~1023u) : 0;
   L.off_qr = o; o += qr_bytes;
-  o = (o + 127) & ~127u;
+  o = (o + 1023) & ~1023u;   // swizzled TMA boxes
   L.off_kr = o; o += kr_bytes;
   o = (o + 15) & ~15u;
   L.off_bar = o; o += 8 * (2 * nc + 2 * nraw + kFixedBars);
@@ -923,6 +925,9 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
                       CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map_2d(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qlat, dc, (uint64_t)B * kH, (uint64_t)dc * 2, 64, kH,
                     CU_TENSOR_MAP_SWIZZLE_128B);
+  CUtensorMap tm_kr;
+  ok &= make_map_2d(&tm_kr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, c.k_rope, R, rows, (uint64_t)R * 2, 64, kTile,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
   const TcLayout L = tc_layout(dc, R, 2 * cfg.r_pairs, int4, qbits);
   TcArgs a;
@@ -954,7 +959,7 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
   if (e != cudaSuccess) return e;
   // the optional profiling events bracket the launch alone, after all host-side set-up
   if ((e = mla_profile_event(p, kProfAttention, false, s)) != cudaSuccess) return e;
-  e = mla_launch_kernel(kern, dim3(G), dim3(384), L.total, s, p.opt_pdl, tm_c, tm_q, a);
+  e = mla_launch_kernel(kern, dim3(G), dim3(384), L.total, s, p.opt_pdl, tm_c, tm_q, tm_kr, a);
   if (e != cudaSuccess) return e;
   if ((e = mla_profile_event(p, kProfAttention, true, s)) != cudaSuccess) return e;
   return cudaSuccess;

@@ -8,11 +8,10 @@
 
 #include "mla_api.h"
 
-// Element offset of RoPE key dim j of KV head g, token t of sequence b, in the blocked
-// k_rope layout [B][ceil(T_cap/32)][n_kv][32][2r].
+// Element offset of RoPE key dim j of KV head g, token t of sequence b, in the token-major
+// k_rope layout [B][T_cap][n_kv][2r] (one row of n_kv*2r values per token, like c_kv).
 inline __host__ __device__ size_t mla_kr_offset(int b, int t, int g, int j, int T_cap, int n_kv, int r2) {
-  const size_t blocks = (size_t)(T_cap + 31) / 32;
-  return (((size_t)b * blocks + (size_t)(t >> 5)) * n_kv + g) * 32u * r2 + (size_t)(t & 31) * r2 + j;
+  return (((size_t)b * T_cap + (size_t)t) * n_kv + g) * r2 + j;
 }
 
 // Storage location of token t of sequence b: (row-space sequence pb, token pt, capacity cap).

@@ -166,8 +166,7 @@ def test_binding_constants_match_the_header(mla):
 def test_cache_accessors_follow_the_documented_layout(mla):
     """LatentCache's token accessors (used by the parity tests to read and write the cache)
     against the layout mla_cache_t documents, on CPU tensors: contiguous rows [b][t], paged
-    rows [block_table[b][t/128]][t%128], RoPE keys at
-    ((pb*ceil(cap/32) + pt/32)*n_kv + g)*32*2r + (pt%32)*2r + j."""
+    rows [block_table[b][t/128]][t%128], RoPE keys token-major at ((pb*cap + pt)*n_kv + g)*2r + j."""
     from mha_mla_latent_b200.cache import LatentCache
     import torch
     cfg = mla.make_config(256, 8, 4, 32, 2, 64, cache="int4_g32", resid=128)
@@ -196,7 +195,7 @@ def test_cache_accessors_follow_the_documented_layout(mla):
             np.testing.assert_array_equal(flat_c[pb * cap + pt], codes[i].numpy())
             for g in range(n_kv):
                 for j in range(r2):
-                    off = ((pb * ((cap + 31) // 32) + pt // 32) * n_kv + g) * 32 * r2 + (pt % 32) * r2 + j
+                    off = ((pb * cap + pt) * n_kv + g) * r2 + j
                     assert flat_kr[off] == float(kr[i, g, j].to(torch.bfloat16))
     # per-query views alias a sequence's table row and keep the pool (no residual window:
     # its ring belongs to a sequence row)
