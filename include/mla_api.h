@@ -156,7 +156,7 @@ enum {
                                  run out (after MLA_OPT_WAIT_LIMIT_US) and the call reports
                                  MLA_DEVERR_TIMEOUT.  Nothing faults; later calls with the
                                  option cleared run normally. */
-  MLA_OPT_PROFILE_KERNELS = 8, /* value: address of a host array of eight cudaEvent_t (0 =
+  MLA_OPT_PROFILE_KERNELS = 8  /* value: address of a host array of eight cudaEvent_t (0 =
                                  off); each call records [2k] just before and [2k+1] just
                                  after its kernel k on the call's stream: k = 0 the append
                                  kernel (mla_append), 1 the query absorption, 2 the split-K
@@ -164,11 +164,6 @@ enum {
                                  kernels stop their launches from overlapping, so each
                                  interval times its kernel alone.  Overrides
                                  MLA_OPT_PROFILE_EVENTS while set. */
-  MLA_OPT_L2_PREFETCH = 7     /* L2 prefetch lookahead of the tensor-core kernel: the low 8
-                                 bits give how many tiles ahead of its shared-memory copies
-                                 it asks L2 for cache bytes (0 = off, at most 16; default 2);
-                                 bits 8.. select the form when non-zero: 1 line prefetches,
-                                 2 bulk prefetches (default 1). */
 };
 
 MLA_API const char* mla_status_string(mla_status_t s);
@@ -257,6 +252,27 @@ MLA_API size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B);
 MLA_API mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
                         const void* q, int32_t B, void* out, void* workspace, size_t ws_bytes,
                         void* stream);
+
+/* Many queries per sequence, causally: the newest Q tokens of each sequence (a chunk of a
+ * long document being prefilled, or drafted tokens to verify) attend over the cache in one
+ * call.  seq_lens[b] counts all of sequence b's cached tokens, the chunk's own included
+ * (append them first); query i (0 <= i < Q) of sequence b sits at position
+ * p = seq_lens[b] - Q + i, is rotated there, and attends over tokens [0, p].  Per query this
+ * is exactly mla_decode with length p + 1.  The queries of a sequence share every cache tile
+ * they read: blocks of 4 queries x 32 heads are scored against each tile together on the
+ * tensor cores.  Notes §方法详解/整体框架 and §关键设计 (absorbed latent scores plus the
+ * separate RoPE term); the README "MHA2MLA" evaluates long documents (LongBench).
+ *   seq_lens  device [B] int32, Q <= L <= T_cap
+ *   q         device [B][Q][H][d_h] dtype, unrotated, original dim order
+ *   out       device [B][Q][H][d_h] dtype, per-head attention output (before W_o)
+ *   workspace device, >= mla_decode_chunk_workspace_bytes(plan, B, Q) bytes
+ * Q == 1 is mla_decode.  For Q > 1 this build needs bf16, a bf16 latent cache, 32 query
+ * heads, d_c in {64, 128, 256} and r = 4 (MLA_ERR_UNSUPPORTED otherwise; one mla_decode per
+ * query through per-query views of a paged cache covers the other shapes). */
+MLA_API size_t mla_decode_chunk_workspace_bytes(const mla_plan_t* plan, int32_t B, int32_t Q);
+MLA_API mla_status_t mla_decode_chunk(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
+                                      const void* q, int32_t B, int32_t Q, void* out, void* workspace,
+                                      size_t ws_bytes, void* stream);
 
 /* One serving-loop decode step in a single call: the append of every sequence's new
  * token, then the decode of every sequence's new query.  Token b (row b of x) is the

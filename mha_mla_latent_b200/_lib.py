@@ -20,7 +20,7 @@ MLA_F32, MLA_BF16 = 0, 1
 MLA_CACHE_SAME, MLA_CACHE_INT4_G32, MLA_CACHE_INT4_G32_R128, MLA_CACHE_INT2_G32 = 0, 1, 2, 3
 MLA_RESID_WINDOW = 128
 MLA_OPT_DECODE_KERNEL, MLA_OPT_DECODE_SPLITS, MLA_OPT_PROFILE_EVENTS, MLA_OPT_OVERLAP_LAUNCH = 1, 2, 3, 4
-MLA_OPT_WAIT_LIMIT_US, MLA_OPT_TEST_SKIP_COPY, MLA_OPT_L2_PREFETCH, MLA_OPT_PROFILE_KERNELS = 5, 6, 7, 8
+MLA_OPT_WAIT_LIMIT_US, MLA_OPT_TEST_SKIP_COPY, MLA_OPT_PROFILE_KERNELS = 5, 6, 8
 MLA_DEVERR_SEQ_LEN, MLA_DEVERR_APPEND_SLOT, MLA_DEVERR_TIMEOUT, MLA_DEVERR_BLOCK = 1, 2, 4, 8
 MLA_BLOCK_TOKENS = 128
 
@@ -28,7 +28,8 @@ EXPORTED = (
     "mla_status_string", "mla_version", "mla_cache_bytes_per_token", "mla_select_pairs",
     "mla_plan_create", "mla_plan_destroy", "mla_plan_set_option", "mla_append",
     "mla_decode_workspace_bytes", "mla_decode", "mla_device_error", "mla_decode_noalloc",
-    "mla_fixed_pairs", "mla_decode_step", "mla_decode_step_host",
+    "mla_fixed_pairs", "mla_decode_step", "mla_decode_step_host", "mla_decode_chunk",
+    "mla_decode_chunk_workspace_bytes",
 )
 MLA_PAIRS_FULL, MLA_PAIRS_HIGH, MLA_PAIRS_UNIFORM, MLA_PAIRS_LOW = 0, 1, 2, 5
 MLA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -76,6 +77,8 @@ def _load():
         "mla_device_error": (i32, [vp, ctypes.POINTER(i32)]),
         "mla_decode_noalloc": (i32, [vp, cachep, vp, vp, i32, vp, vp]),
         "mla_decode_step": (i32, [vp, cachep, vp, vp, vp, i32, vp, vp, sz, vp]),
+        "mla_decode_chunk": (i32, [vp, cachep, vp, vp, i32, i32, vp, vp, sz, vp]),
+        "mla_decode_chunk_workspace_bytes": (sz, [vp, i32, i32]),
         "mla_decode_step_host": (i32, [vp, cachep, vp, vp, vp, i32, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
@@ -229,6 +232,20 @@ def mla_decode(plan: Plan, cache: MlaCache, seq_lens, q, out, workspace, stream=
                          _ptr(out), _ptr(workspace), ws_bytes, _stream(stream))
     if check:
         _check(st, "mla_decode")
+    return st
+
+
+def mla_decode_chunk_workspace_bytes(plan: Plan, B: int, Q: int) -> int:
+    return int(_lib.mla_decode_chunk_workspace_bytes(plan.handle, int(B), int(Q)))
+
+
+def mla_decode_chunk(plan: Plan, cache: MlaCache, seq_lens, q, out, workspace, stream=None, check=True):
+    """Causal attention of each sequence's newest Q tokens: q and out are [B][Q][H][d_h]."""
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = _lib.mla_decode_chunk(plan.handle, ctypes.byref(cache), _ptr(seq_lens), _ptr(q), int(q.shape[0]),
+                               int(q.shape[1]), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream))
+    if check:
+        _check(st, "mla_decode_chunk")
     return st
 
 

@@ -1,0 +1,539 @@
+// Many queries per sequence (a chunk of new tokens: chunked prefill, drafted tokens to
+// verify) on the 5th-generation tensor cores: every query attends causally over its
+// sequence's latent cache, and the queries of a sequence share each cache tile they read.
+//
+// Paper notes "MHA2MLA" (ACL 2025), §关键设计 and §方法详解/整体框架: the converted layer
+// scores all heads against the one shared latent (W_uk absorbed into each query), adds the
+// separately computed partial-RoPE term, and takes the probability-weighted latent through
+// W_uv; a chunk of a long document's tokens reads the same latent prefix with every query.
+//
+// A unit of work is (sequence b, block of 4 consecutive queries) = 128 rows (query j,
+// head h), row = 32 j + h.  The units' tokens (up to the block's last query) are laid end
+// to end and split among the CTAs like the decode's split-K schedule, in tiles of 64
+// tokens.  Per tile:
+//     S[row][t]   = sum_c Qlat[row][c] * C[t][c]              MMA1  M = 128 rows, N = 64 tokens
+//     S[row][t]  += sum_j Qrope[row][j] * KR[t][g(h)][j]       CUDA cores (fp32), one row per thread
+//     O[row][d]  += sum_t P[row][t] * C[t][d]                  MMA2  M = 128, N = d_c, K = 64
+// with the causal mask t <= position of the row's query.  The transposed orientation gives
+// each softmax thread a whole row: its running max and sum are thread-local.  MMA2 reads
+// the C tile already in shared memory as an MN-major operand, so each cache byte is read
+// into the SM once per unit.
+//
+// Warp roles (8 warps): warp 0 producer (TMA: the unit's Q_lat rows, C and RoPE-key tiles
+// into a ring of stages), warp 1 TMEM owner and single-thread
+// MMA issuer, warps 4-7 softmax (warp 4 + j owns the rows of query j: TMEM lane quarter j).
+// Every wait is bounded; a timeout sets MLA_DEVERR_TIMEOUT, drains and releases TMEM.
+#include <cuda.h>
+
+#include "decode_common.cuh"
+#include "sm100.cuh"
+
+namespace mla {
+namespace chunk {
+
+using namespace sm100;
+
+constexpr int kCT = 64;              // tokens per tile
+constexpr int kRows = 128;           // rows per unit: 4 queries x 32 heads
+constexpr int kQB = 4;               // queries per unit
+constexpr int kHeads = 32;
+constexpr uint32_t kQBox = 16384;    // Q_lat box: 128 rows x 128 B
+constexpr uint32_t kTBox = 8192;     // cache box: 64 rows x 128 B
+constexpr uint32_t kPBytes = 16384;  // P: 128 rows x 64 tokens bf16
+constexpr float kTau = 8.0f;         // lazy-rescale threshold, log2 units
+constexpr uint32_t kSCol = 0, kOCol = 128;
+
+struct ChunkArgs {
+  int q_chunk, nqb, d_c, R, P, T_cap;
+  Sched sched;
+  const int32_t* seq_lens;
+  const float* qrope;      // [B*Q][32][2r], rotated at each query's position, scaled
+  float* opart;            // [P][128][d_c]
+  float* mlpart;           // [128][P][2]
+  mla_cache_t cache;
+  int32_t* err;
+  uint64_t wait_ns;
+  int NC;
+  uint32_t off_q, off_stage, off_p, off_bar, off_misc, stage_bytes;
+};
+
+struct Bars {
+  uint32_t base;
+  int NC;
+  __device__ uint32_t at(int i) const { return base + 8u * (uint32_t)i; }
+  __device__ uint32_t c_full(int s) const { return at(s); }
+  __device__ uint32_t c_empty(int s) const { return at(NC + s); }
+  __device__ uint32_t s_full(int i) const { return at(2 * NC + i); }
+  __device__ uint32_t s_empty(int i) const { return at(2 * NC + 2 + i); }
+  __device__ uint32_t p_full(int i) const { return at(2 * NC + 4 + i); }
+  __device__ uint32_t p_empty(int i) const { return at(2 * NC + 6 + i); }
+  __device__ uint32_t o_full() const { return at(2 * NC + 8); }
+  __device__ uint32_t o_empty() const { return at(2 * NC + 9); }
+  __device__ uint32_t q_full() const { return at(2 * NC + 10); }
+  __device__ uint32_t q_empty() const { return at(2 * NC + 11); }
+  __device__ uint32_t mma_done() const { return at(2 * NC + 12); }
+};
+constexpr int kFixedBars = 13;
+
+struct Misc {
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct TileIter {
+  const Sched* s;
+  int pc, pc_end;
+  int v, t0, t1;
+  int t;
+  __device__ void init(const Sched* sc, int w) {
+    s = sc;
+    pc = sc->worker_first[w];
+    pc_end = sc->worker_first[w + 1];
+    t = 0;
+    if (pc < pc_end) load();
+  }
+  __device__ void load() { v = s->piece_b[pc]; t0 = s->piece_t0[pc]; t1 = s->piece_t1[pc]; t = t0; }
+  __device__ bool valid() const { return pc < pc_end; }
+  __device__ bool first_of_piece() const { return t == t0; }
+  __device__ bool last_of_piece() const { return t + kCT >= t1; }
+  __device__ void next() {
+    t += kCT;
+    if (t >= t1) { ++pc; if (pc < pc_end) load(); }
+  }
+};
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+__device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+template <bool PAGED>
+__device__ __forceinline__ MlaLoc chunk_loc(const ChunkArgs& a, int b, int t) {
+  if (!PAGED) return MlaLoc{b, t, a.T_cap};
+  return mla_loc(a.cache, b, t, a.err);
+}
+
+template <bool PAGED>
+__global__ void __launch_bounds__(256, 1)
+chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_kr,
+                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ ChunkArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t sbase_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (sbase_u32 - smem_u32(smem_raw));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int dc = a.d_c, R = a.R;
+  const int n_cbox = dc / 64, n_kbox = R / 64;
+  Bars bars{sbase_u32 + a.off_bar, a.NC};
+  Misc* misc = reinterpret_cast<Misc*>(sbase + a.off_misc);
+  volatile int* abort_flag = &misc->abort_flag;
+  const uint64_t lim = a.wait_ns;
+
+  if (threadIdx.x == 0) {
+    misc->abort_flag = 0;
+    for (int s = 0; s < a.NC; ++s) { mbar_init(bars.c_full(s), 1); mbar_init(bars.c_empty(s), 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bars.s_full(i), 1);
+      mbar_init(bars.s_empty(i), 4);
+      mbar_init(bars.p_full(i), 4);
+      mbar_init(bars.p_empty(i), 1);
+    }
+    mbar_init(bars.o_full(), 1);
+    mbar_init(bars.o_empty(), 4);
+    mbar_init(bars.q_full(), 1);
+    mbar_init(bars.q_empty(), 1);
+    mbar_init(bars.mma_done(), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_c);
+    tma_prefetch_desc(&tm_kr);
+    tma_prefetch_desc(&tm_q);
+  }
+  constexpr uint32_t kTmemCols = 512;   // S 2 x 64 columns, O d_c <= 256 columns
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&misc->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();   // schedule, absorbed queries and the cache come from earlier kernels
+  pdl_trigger();
+  const uint32_t tmem = misc->tmem_base;
+  const int w = blockIdx.x;
+  auto qrow0 = [&](int v) {   // first Q_lat row of unit v: query (v % nqb) * 4 of sequence v / nqb
+    return ((v / a.nqb) * a.q_chunk + (v % a.nqb) * kQB) * kHeads;
+  };
+
+  if (warp == 0) {
+    // ============================================================ TMA producer
+    TileIter it;
+    it.init(&a.sched, w);
+    int n = 0, u = 0, q_loads = 0, last = -1;
+    bool ok = true;
+    while (ok && it.valid()) {
+      if (it.first_of_piece()) {
+        if (u > 0) ok = __all_sync(0xffffffffu, mbar_wait(bars.q_empty(), (u - 1) & 1, abort_flag, lim));
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_expect_tx(bars.q_full(), (uint32_t)n_cbox * kQBox);
+          for (int kb = 0; kb < n_cbox; ++kb)
+            tma_load_2d(sbase_u32 + a.off_q + kb * kQBox, &tm_q, bars.q_full(), kb * 64, qrow0(it.v));
+        }
+        ++q_loads;
+      }
+      const int cs = n % a.NC;
+      if (n >= a.NC) ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag, lim));
+      if (!ok) break;
+      if (lane == 0) {
+        const MlaLoc lc = chunk_loc<PAGED>(a, it.v / a.nqb, it.t);   // a 64-token tile lies in one block
+        const int row = lc.pb * lc.cap + lc.pt;
+        const uint32_t st = sbase_u32 + a.off_stage + cs * a.stage_bytes;
+        mbar_expect_tx(bars.c_full(cs), (uint32_t)(n_cbox + n_kbox) * kTBox);
+        for (int kb = 0; kb < n_cbox; ++kb) tma_load_2d(st + kb * kTBox, &tm_c, bars.c_full(cs), kb * 64, row);
+        for (int kb = 0; kb < n_kbox; ++kb)
+          tma_load_2d(st + (n_cbox + kb) * kTBox, &tm_kr, bars.c_full(cs), kb * 64, row);
+      }
+      last = n;
+      if (it.last_of_piece()) ++u;
+      it.next();
+      ++n;
+    }
+    if (lane == 0) {   // drain: every issued copy lands before the CTA exits
+      volatile int never = 0;
+      if (q_loads > 0) mbar_wait(bars.q_full(), (q_loads - 1) & 1, &never, lim);
+      for (int s = 0; s < a.NC; ++s) {
+        const int k = last - ((last - s) % a.NC + a.NC) % a.NC;
+        if (last >= 0 && k >= 0) mbar_wait(bars.c_full(s), (k / a.NC) & 1, &never, lim);
+      }
+    }
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc1 = idesc_bf16_f32(kRows, kCT, false, false);   // S[row][t]
+      const uint32_t idesc2 = idesc_bf16_f32(kRows, dc, false, true);     // O[row][d]
+      TileIter it;
+      it.init(&a.sched, w);
+      int n = 0, u = 0;
+      bool ok = true;
+      int pend_n = -1, pend_u = 0;
+      bool pend_first = false, pend_last = false;
+      auto do_mma2 = [&](int pn, int pu, bool first, bool lastp) -> bool {
+        const int pb = pn & 1, cs = pn % a.NC;
+        if (!mbar_wait(bars.p_full(pb), (pn >> 1) & 1, abort_flag, lim)) return false;
+        if (first && pu > 0)
+          if (!mbar_wait(bars.o_empty(), (pu - 1) & 1, abort_flag, lim)) return false;
+        tc_fence_after();
+        const uint32_t c0 = sbase_u32 + a.off_stage + cs * a.stage_bytes;
+        const uint32_t p0 = sbase_u32 + a.off_p + pb * kPBytes;
+#pragma unroll
+        for (int kk = 0; kk < kCT / 16; ++kk) {
+          const uint64_t ad = smem_desc(p0 + kk * 32, 16, 1024, kLayoutSW128);
+          const uint64_t bd = smem_desc(c0 + kk * 2048, kTBox, 1024, kLayoutSW128);
+          tc_mma_bf16(tmem + kOCol, ad, bd, idesc2, (first && kk == 0) ? 0u : 1u);
+        }
+        tc_commit(bars.p_empty(pb));
+        tc_commit(bars.c_empty(cs));
+        if (lastp) tc_commit(bars.o_full());
+        return true;
+      };
+      while (ok && it.valid()) {
+        const int sb = n & 1, cs = n % a.NC;
+        const bool first = it.first_of_piece();
+        {
+          const uint64_t t_start = globaltimer();
+          while (true) {
+            if (pend_n >= 0 && mbar_test(bars.p_full(pend_n & 1), (pend_n >> 1) & 1)) {
+              ok = do_mma2(pend_n, pend_u, pend_first, pend_last);
+              pend_n = -1;
+              if (!ok) break;
+              continue;
+            }
+            if ((n < 2 || mbar_test(bars.s_empty(sb), ((n >> 1) - 1) & 1)) &&
+                (!first || mbar_test(bars.q_full(), u & 1)) && mbar_test(bars.c_full(cs), (n / a.NC) & 1))
+              break;
+            if (*abort_flag || globaltimer() - t_start > lim) {
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+          }
+        }
+        if (!ok) break;
+        tc_fence_after();
+        {  // MMA1: S = Q_lat C^T
+          const uint32_t c0 = sbase_u32 + a.off_stage + cs * a.stage_bytes;
+          for (int kk = 0; kk < dc / 16; ++kk) {
+            const uint64_t ad = smem_desc(sbase_u32 + a.off_q + (kk >> 2) * kQBox + (kk & 3) * 32, 16, 1024,
+                                          kLayoutSW128);
+            const uint64_t bd = smem_desc(c0 + (kk >> 2) * kTBox + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+            tc_mma_bf16(tmem + kSCol + sb * kCT, ad, bd, idesc1, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bars.s_full(sb));
+          if (it.last_of_piece()) tc_commit(bars.q_empty());
+        }
+        if (pend_n >= 0) {
+          ok = do_mma2(pend_n, pend_u, pend_first, pend_last);
+          if (!ok) break;
+        }
+        pend_n = n; pend_u = u; pend_first = first; pend_last = it.last_of_piece();
+        if (it.last_of_piece()) ++u;
+        it.next();
+        ++n;
+      }
+      if (ok && pend_n >= 0) do_mma2(pend_n, pend_u, pend_first, pend_last);
+      tc_commit(bars.mma_done());
+      volatile int never = 0;
+      mbar_wait(bars.mma_done(), 0, &never, lim);
+    }
+  } else if (warp >= 4) {
+    // ============================================================ softmax + epilogue
+    const int q = warp - 4;                  // TMEM lane quarter = query j of the unit
+    const int r = 32 * q + lane;             // this thread's row: query q, head lane
+    const int n_kv = R / 8;
+    const int g = lane / (kHeads / n_kv);    // KV head of this row's head
+    TileIter it;
+    it.init(&a.sched, w);
+    int n = 0, u = 0;
+    bool ok = true;
+    float m = -INFINITY, l = 0.f;
+    float qr[8];
+    int p_row = -1;                          // position of this row's query (-1: past the chunk)
+    auto wwait = [&](uint32_t bar, int parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, lim));
+    };
+    while (ok && it.valid()) {
+      const bool first = it.first_of_piece();
+      const int pc = it.pc;
+      if (first) {
+        const int bseq = it.v / a.nqb, i = (it.v % a.nqb) * kQB + q;
+        p_row = -1;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) qr[j] = 0.f;
+        if (i < a.q_chunk) {
+          p_row = __ldg(a.seq_lens + bseq) - a.q_chunk + i;
+          const float4* src = reinterpret_cast<const float4*>(a.qrope + (((size_t)bseq * a.q_chunk + i) * kHeads + lane) * 8);
+          const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
+          qr[0] = x0.x; qr[1] = x0.y; qr[2] = x0.z; qr[3] = x0.w;
+          qr[4] = x1.x; qr[5] = x1.y; qr[6] = x1.z; qr[7] = x1.w;
+        }
+        m = -INFINITY;
+        l = 0.f;
+      }
+      const int sb = n & 1, pb = n & 1, cs = n % a.NC;
+      ok = wwait(bars.s_full(sb), (n >> 1) & 1);
+      if (ok) ok = wwait(bars.c_full(cs), (n / a.NC) & 1);   // the RoPE keys of this tile
+      if (!ok) break;
+      tc_fence_after();
+      float s[kCT];
+      {
+        uint32_t raw[16];
+#pragma unroll
+        for (int k = 0; k < kCT / 16; ++k) {
+          tmem_ld16(taddr(tmem, 32 * q, kSCol + sb * kCT + 16 * k), raw);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) s[16 * k + e] = u2f(raw[e]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.s_empty(sb));
+      // RoPE score against the tile's keys: row t of the swizzled stage, KV head g's chunk
+      const uint8_t* krb = sbase + a.off_stage + cs * a.stage_bytes + (n_cbox + (g >> 3)) * kTBox;
+      const int lim_t = min(it.t1, p_row + 1) - it.t;   // tokens [0, lim_t) of the tile count
+      float mx = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < kCT; ++t) {
+        const uint4 kw = *reinterpret_cast<const uint4*>(krb + t * 128 + (((g & 7) ^ (t & 7)) << 4));
+        float v = s[t] + qr[0] * bf16lo(kw.x) + qr[1] * bf16hi(kw.x) + qr[2] * bf16lo(kw.y) + qr[3] * bf16hi(kw.y) +
+                  qr[4] * bf16lo(kw.z) + qr[5] * bf16hi(kw.z) + qr[6] * bf16lo(kw.w) + qr[7] * bf16hi(kw.w);
+        v = t < lim_t ? v : -INFINITY;
+        s[t] = v;
+        mx = fmaxf(mx, v);
+      }
+      if (mx > m + kTau) {   // raise the running max (lazily), rescale what O holds
+        const float al = exp2f(m - mx);   // m = -inf: 0
+        if (!first) {
+          // O holds the piece's tiles before this one: wait for MMA2(n-1), then rescale the row
+          const int pn = n - 1;
+          if (!wwait(bars.p_empty(pn & 1), (pn >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          for (int cc = 0; cc < dc / 16; ++cc) {
+            const uint32_t ta = taddr(tmem, 32 * q, kOCol + 16 * cc);
+            uint32_t o[16];
+            tmem_ld16(ta, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = f2u(u2f(o[k]) * al);
+            tmem_st16(ta, o);
+          }
+          tmem_wait_st();
+        }
+        l *= al;
+        m = mx;
+      }
+      uint32_t pk[kCT / 2];
+#pragma unroll
+      for (int t = 0; t < kCT; t += 2) {
+        const float p0 = t < lim_t ? exp2f(s[t] - m) : 0.f;
+        const float p1 = t + 1 < lim_t ? exp2f(s[t + 1] - m) : 0.f;
+        l += p0 + p1;
+        pk[t / 2] = pack_bf16x2(p0, p1);
+      }
+      if (n >= 2) {
+        ok = wwait(bars.p_empty(pb), ((n >> 1) - 1) & 1);
+        if (!ok) break;
+      }
+      {  // P row r: 64 tokens = 128 B, 16-byte chunk c at (c ^ (r % 8))
+        uint8_t* prow = sbase + a.off_p + pb * kPBytes + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.p_full(pb));
+
+      if (it.last_of_piece()) {
+        // ---------------- piece epilogue: this row's partial (m, l, O)
+        a.mlpart[((size_t)r * a.P + pc) * 2] = m;
+        a.mlpart[((size_t)r * a.P + pc) * 2 + 1] = l;
+        ok = wwait(bars.o_full(), u & 1);
+        if (!ok) break;
+        tc_fence_after();
+        float* dst = a.opart + ((size_t)pc * kRows + r) * dc;
+        for (int c0 = 0; c0 < dc; c0 += 32) {
+          uint32_t o[2][16];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) tmem_ld16(taddr(tmem, 32 * q, kOCol + c0 + 16 * k), o[k]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+              *reinterpret_cast<float4*>(dst + c0 + 16 * k + e) =
+                  make_float4(u2f(o[k][e]), u2f(o[k][e + 1]), u2f(o[k][e + 2]), u2f(o[k][e + 3]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.o_empty());
+        ++u;
+      }
+      it.next();
+      ++n;
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && misc->abort_flag) raise_error(a.err, MLA_DEVERR_TIMEOUT);
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map with 64-column (128-byte) boxes and the 128-byte swizzle.
+static bool map_bf16_sw128(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {cols, rows};
+  cuuint64_t gstride[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct ChunkLayoutSmem {
+  int NC;
+  uint32_t off_q, off_stage, off_p, off_bar, off_misc, stage_bytes, total;
+};
+
+static ChunkLayoutSmem chunk_smem(int dc, int R) {
+  const uint32_t budget = 232448 - 1024;
+  ChunkLayoutSmem L{};
+  L.stage_bytes = (uint32_t)(dc / 64 + R / 64) * kTBox;
+  const uint32_t q_bytes = (uint32_t)(dc / 64) * kQBox;
+  auto size = [&](int nc) { return q_bytes + nc * L.stage_bytes + 2 * kPBytes + 8 * (2 * nc + kFixedBars) + 256; };
+  int nc = 2;
+  while (nc < 6 && size(nc + 1) <= budget) ++nc;
+  L.NC = nc;
+  uint32_t o = 0;
+  L.off_q = o; o += q_bytes;
+  L.off_stage = o; o += nc * L.stage_bytes;
+  L.off_p = o; o += 2 * kPBytes;
+  L.off_bar = o; o += 8 * (2 * nc + kFixedBars);
+  o = (o + 15) & ~15u;
+  L.off_misc = o; o += sizeof(Misc);
+  L.total = o + 1024;
+  return L;
+}
+
+}  // namespace chunk
+}  // namespace mla
+
+// Shapes the chunk kernel covers: bf16 latent (no quantised cache), 32 query heads, d_c in
+// {64, 128, 256}, r = 4 kept pairs per KV head.
+bool mla_chunk_capable(const mla_plan& p) {
+  const mla_config_t& cfg = p.cfg;
+  if (cfg.dtype != MLA_BF16 || cfg.cache_kind != MLA_CACHE_SAME || cfg.n_heads != mla::chunk::kHeads) return false;
+  if (cfg.d_c % 64 != 0 || cfg.d_c > 256 || 2 * cfg.r_pairs != 8 || p.R % 64 != 0) return false;
+  return mla::chunk::chunk_smem(cfg.d_c, p.R).total <= 232448;
+}
+
+cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B, int Q,
+                                const Sched& sched, const void* qlat, const float* qrope, float* opart,
+                                float* mlpart, int P, int G, cudaStream_t s) {
+  using namespace mla::chunk;
+  const mla_config_t& cfg = p.cfg;
+  const int dc = cfg.d_c, R = p.R;
+  const uint64_t rows = mla_cache_rows(c);
+  CUtensorMap tm_c, tm_kr, tm_q;
+  bool ok = map_bf16_sw128(&tm_c, c.c_kv, dc, rows, kCT) && map_bf16_sw128(&tm_kr, c.k_rope, R, rows, kCT) &&
+            map_bf16_sw128(&tm_q, qlat, dc, (uint64_t)B * Q * kHeads, kRows);
+  if (!ok) return cudaErrorInvalidValue;
+  const ChunkLayoutSmem L = chunk_smem(dc, R);
+  ChunkArgs a;
+  a.q_chunk = Q; a.nqb = (Q + kQB - 1) / kQB; a.d_c = dc; a.R = R; a.P = P; a.T_cap = c.T_cap;
+  a.sched = sched; a.seq_lens = seq_lens; a.qrope = qrope; a.opart = opart; a.mlpart = mlpart;
+  a.cache = c; a.err = p.err;
+  a.wait_ns = (uint64_t)p.opt_wait_us * 1000u;
+  a.NC = L.NC;
+  a.off_q = L.off_q; a.off_stage = L.off_stage; a.off_p = L.off_p; a.off_bar = L.off_bar; a.off_misc = L.off_misc;
+  a.stage_bytes = L.stage_bytes;
+  auto kern = c.block_table ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+  if (e != cudaSuccess) return e;
+  if ((e = mla_profile_event(p, kProfAttention, false, s)) != cudaSuccess) return e;
+  e = mla_launch_kernel(kern, dim3(G), dim3(256), L.total, s, p.opt_pdl, tm_c, tm_kr, tm_q, a);
+  if (e != cudaSuccess) return e;
+  return mla_profile_event(p, kProfAttention, true, s);
+}

@@ -37,6 +37,9 @@ struct AbsorbArgs {
   int sched_ints;             // shared memory of the schedule CTA, in ints
   float sm_scale;             // softmax scale of the scores (1/sqrt(d_h) unless the config sets one)
   int vec_ok;                 // q and W_uk^T rows allow 16-byte loads
+  // many queries per sequence: query rows s = b * q_chunk + i sit at position
+  // seq_lens[b] - q_chunk + i; the schedule runs over units of q_block queries (1, 1: decode)
+  int q_chunk, q_block;
 };
 
 constexpr int kAbsRows = 8;    // (b, h) rows per CTA: one per warp in the product
@@ -55,8 +58,9 @@ __device__ __forceinline__ void absorb_body(const AbsorbArgs& a, int blk_id, flo
   const int rows_total = a.B * G;
   const int n_rb = (rows_total + kAbsRows - 1) / kAbsRows;
   if (blk_id == 0) {  // the split-K schedule
-    build_schedule(a.seq_lens, a.B, a.T_cap, a.tile, a.G, a.sched, a.err, reinterpret_cast<int32_t*>(sm),
-                   a.sched_ints);
+    const int nunits = a.q_chunk > 1 ? (a.B / a.q_chunk) * ((a.q_chunk + a.q_block - 1) / a.q_block) : a.B;
+    build_schedule(a.seq_lens, nunits, a.T_cap, a.tile, a.G, a.sched, a.err, reinterpret_cast<int32_t*>(sm),
+                   a.sched_ints, a.q_chunk, a.q_block);
     return;
   }
   const int blk = blk_id - 1;
@@ -97,7 +101,11 @@ __device__ __forceinline__ void absorb_body(const AbsorbArgs& a, int blk_id, flo
     const int row = row0 + r;
     return q + ((size_t)(row / G) * a.H + g * G + row % G) * dh;
   });
-  const int rp_pos = rope_item ? __ldg(a.seq_lens + (row0 + tid / a.r) / G) : 0;
+  int rp_pos = 0;   // length up to and including the query row's token (its position + 1)
+  if (rope_item) {
+    const int sq = (row0 + tid / a.r) / G;
+    rp_pos = __ldg(a.seq_lens + sq / a.q_chunk) - (a.q_chunk - 1 - sq % a.q_chunk);
+  }
   __syncthreads();
   for (int i = tid; i < kAbsRows * dn; i += 256) s_qn[(i / dn) * dnp + i % dn] = s_q[(i / dn) * dh + s_idx[i % dn]];
   // RoPE query part: rotate the kept pairs at position L-1 (angle in double), scale
@@ -301,7 +309,21 @@ struct CombineArgs {
   int P;              // piece capacity of the partial arrays [H][P]
   int ncols;          // output columns per CTA: 64, or 32 when the latent is wide
   int vec_ok;         // W_uv rows allow 16-byte loads
+  // Many queries per sequence: the merged units are (sequence, block of q_block queries)
+  // with H = q_block * heads rows each; row h of unit v is query (v % nqb) * q_block +
+  // h / heads of sequence v / nqb, head h % heads (W_uv group (h % heads) / G).  Decode:
+  // q_chunk = q_block = 1, heads = H.
+  int q_chunk, q_block, heads;
 };
+
+// Output row (query row x head) of merged row h of unit v, or -1 past the chunk's last query.
+__device__ __forceinline__ long long combine_out_row(const CombineArgs& a, int v, int h) {
+  if (a.q_chunk <= 1) return (long long)v * a.H + h;
+  const int nqb = (a.q_chunk + a.q_block - 1) / a.q_block;
+  const int i = (v % nqb) * a.q_block + h / a.heads;
+  if (i >= a.q_chunk) return -1;
+  return ((long long)(v / nqb) * a.q_chunk + i) * a.heads + h % a.heads;
+}
 
 constexpr int kCmbRows = 8;    // (b, h) rows per CTA, one warp each
 
@@ -311,7 +333,7 @@ constexpr int kCmbRows = 8;    // (b, h) rows per CTA, one warp each
 // into shared memory (all of a batch of pieces' loads in flight together), and then
 // out[row][d] = sum_c O_lat[row][c] W_uv[g][c][d] with lane l on columns 2l, 2l+1.
 template <typename T>
-__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+__global__ void __launch_bounds__(256, 1) combine_kernel(CombineArgs a) {
   extern __shared__ __align__(16) float sm[];
   const int G = a.H / a.n_kv;
   const int rows_total = a.B * G;
@@ -330,7 +352,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   float* s_w = sm;                       // f32 [d_c][NCOL], or bf16 [d_c][WLD] for the MMA form
   float* s_o = s_w + dc * NCOL;          // [kCmbRows][d_c]
   __nv_bfloat16* s_a = reinterpret_cast<__nv_bfloat16*>(s_o + kCmbRows * dc);   // [16][ALD]
-  const T* W = (const T*)a.W_uv + (size_t)g * dc * a.dh;
+  const T* W = (const T*)a.W_uv + (size_t)(g % (a.heads / G)) * dc * a.dh;
   const int ncol = min(NCOL, a.dh - d0);
   if (mma) {
     __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(s_w);
@@ -441,8 +463,9 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
       wmma16::mma_16816(acc[1], af, bf[2], bf[3]);
     }
     const int r = lane >> 2, row = row0 + r;
-    if (row < rows_total) {
-      T* out = (T*)a.out + ((size_t)(row / G) * a.H + g * G + row % G) * a.dh + d0 + 16 * warp + 2 * (lane & 3);
+    const long long orow = row < rows_total ? combine_out_row(a, row / G, g * G + row % G) : -1;
+    if (orow >= 0) {
+      T* out = (T*)a.out + (size_t)orow * a.dh + d0 + 16 * warp + 2 * (lane & 3);
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         __nv_bfloat162 v = __floats2bfloat162_rn(acc[j][0], acc[j][1]);
@@ -465,8 +488,9 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
     acc0 += x.x * w0.x + x.y * w1.x + x.z * w2.x + x.w * w3.x;
     acc1 += x.x * w0.y + x.y * w1.y + x.z * w2.y + x.w * w3.y;
   }
-  if (row < rows_total && d < a.dh) {
-    T* out = (T*)a.out + ((size_t)(row / G) * a.H + g * G + row % G) * a.dh + d;
+  const long long orow = row < rows_total ? combine_out_row(a, row / G, g * G + row % G) : -1;
+  if (orow >= 0 && d < a.dh) {
+    T* out = (T*)a.out + (size_t)orow * a.dh + d;
     out[0] = from_f32<T>(acc0);
     if (d + 1 < a.dh) out[1] = from_f32<T>(acc1);
   }
@@ -488,6 +512,8 @@ void absorb_setup(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_le
   aa->qrope = (float*)(base + L.off_qrope);
   aa->sched = mla_sched_view(L, ws, B); aa->tile = L.tile; aa->G = L.G; aa->err = p.err;
   aa->sm_scale = cfg.softmax_scale > 0.0f ? cfg.softmax_scale : (float)(1.0 / sqrt((double)cfg.head_dim));
+  aa->q_chunk = 1;
+  aa->q_block = 1;
   {
     const int vecn = 16 / (int)sizeof(T);   // elements per 16-byte load
     aa->vec_ok = ((uintptr_t)q % 16 == 0) && cfg.d_c % vecn == 0 && cfg.head_dim % vecn == 0;
@@ -500,6 +526,33 @@ void absorb_setup(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_le
   *smem = std::min<size_t>(std::max(smem_work, sched_ints * sizeof(int32_t)), std::max<size_t>(smem_work, 160 * 1024));
   aa->sched_ints = (int)(*smem / sizeof(int32_t));
   *nblocks = cfg.n_kv_heads * n_rb * n_cc + 1;
+}
+
+// The split merge with W_uv over `units` merged units of H rows in n_kv row groups (decode:
+// sequences, heads, KV heads; many queries per sequence: (sequence, query block) units of
+// q_block * heads rows).
+template <typename T>
+cudaError_t launch_combine(const mla_plan& p, int units, int H, int n_kv, int q_chunk, int q_block, void* out,
+                           void* ws, const DecodeLayout& L, const Sched& sched, cudaStream_t s) {
+  const mla_config_t& cfg = p.cfg;
+  char* base = (char*)ws;
+  CombineArgs ca;
+  ca.B = units; ca.H = H; ca.n_kv = n_kv; ca.d_c = cfg.d_c; ca.dh = cfg.head_dim;
+  ca.opart = (const float*)(base + L.off_opart); ca.mlpart = (const float*)(base + L.off_mlpart);
+  ca.sched = sched; ca.W_uv = p.W_uv; ca.out = out; ca.P = L.P;
+  ca.ncols = (size_t)cfg.d_c * (64 + kCmbRows) * sizeof(float) <= 160 * 1024 ? 64 : 32;
+  ca.vec_ok = cfg.head_dim % (16 / (int)sizeof(T)) == 0;
+  ca.q_chunk = q_chunk; ca.q_block = q_block; ca.heads = cfg.n_heads;
+  const size_t smem_c = (size_t)cfg.d_c * (ca.ncols + kCmbRows) * sizeof(float) +
+                        (size_t)16 * (cfg.d_c + 8) * sizeof(__nv_bfloat16);   // + the MMA form's A tile
+  const int G = H / n_kv;
+  const int n_rbc = (units * G + kCmbRows - 1) / kCmbRows, n_dc = (cfg.head_dim + ca.ncols - 1) / ca.ncols;
+  cudaError_t e = cudaFuncSetAttribute(combine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
+  if (e != cudaSuccess) return e;
+  if ((e = mla_profile_event(p, kProfCombine, false, s)) != cudaSuccess) return e;
+  e = mla_launch_kernel(combine_kernel<T>, dim3(n_kv * n_rbc * n_dc), dim3(256), smem_c, s, p.opt_pdl, ca);
+  if (e != cudaSuccess) return e;
+  return mla_profile_event(p, kProfCombine, true, s);
 }
 
 // Split-K attention over the latent cache, then the split merge with W_uv.
@@ -533,23 +586,7 @@ cudaError_t launch_attention_combine(const mla_plan& p, const mla_cache_t& c, co
                              (float*)(base + L.off_opart), (float*)(base + L.off_mlpart), L.P, L.G, s);
     if (e != cudaSuccess) return e;
   }
-  // merge the splits and apply W_uv
-  CombineArgs ca;
-  ca.B = B; ca.H = H; ca.n_kv = cfg.n_kv_heads; ca.d_c = cfg.d_c; ca.dh = cfg.head_dim;
-  ca.opart = (const float*)(base + L.off_opart); ca.mlpart = (const float*)(base + L.off_mlpart);
-  ca.sched = sched; ca.W_uv = p.W_uv; ca.out = out; ca.P = L.P;
-  ca.ncols = (size_t)cfg.d_c * (64 + kCmbRows) * sizeof(float) <= 160 * 1024 ? 64 : 32;
-  ca.vec_ok = cfg.head_dim % (16 / (int)sizeof(T)) == 0;
-  const size_t smem_c = (size_t)cfg.d_c * (ca.ncols + kCmbRows) * sizeof(float) +
-                        (size_t)16 * (cfg.d_c + 8) * sizeof(__nv_bfloat16);   // + the MMA form's A tile
-  const int G = H / cfg.n_kv_heads;
-  const int n_rbc = (B * G + kCmbRows - 1) / kCmbRows, n_dc = (cfg.head_dim + ca.ncols - 1) / ca.ncols;
-  e = cudaFuncSetAttribute(combine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
-  if (e != cudaSuccess) return e;
-  if ((e = mla_profile_event(p, kProfCombine, false, s)) != cudaSuccess) return e;
-  e = mla_launch_kernel(combine_kernel<T>, dim3(cfg.n_kv_heads * n_rbc * n_dc), dim3(256), smem_c, s, p.opt_pdl, ca);
-  if (e != cudaSuccess) return e;
-  return mla_profile_event(p, kProfCombine, true, s);
+  return launch_combine<T>(p, B, H, cfg.n_kv_heads, 1, 1, out, ws, L, sched, s);
 }
 
 template <typename T, bool INT4>
@@ -624,6 +661,34 @@ cudaError_t launch_step_t(const mla_plan& p, const mla_cache_t& c, const int32_t
   return launch_attention_combine<bf16, INT4>(p, c, seq_lens, B, out, ws, L, sp.abs, s);
 }
 
+// Many queries per sequence: absorption of every query (each rotated at its own position)
+// with the schedule over (sequence, block of 4 queries) units, the chunk attention kernel,
+// and the merge of the units' 128 rows.
+cudaError_t launch_chunk(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, const void* q, int B,
+                         int Q, void* out, void* ws, const DecodeLayout& L, cudaStream_t s) {
+  using bf16 = __nv_bfloat16;
+  const mla_config_t& cfg = p.cfg;
+  constexpr int kQB = 4;
+  AbsorbArgs aa;
+  size_t smem_abs;
+  int nblk;
+  absorb_setup<bf16>(p, c, seq_lens, q, B * Q, ws, L, &aa, &smem_abs, &nblk);
+  aa.q_chunk = Q;
+  aa.q_block = kQB;
+  cudaError_t e = cudaFuncSetAttribute(absorb_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_abs);
+  if (e != cudaSuccess) return e;
+  if ((e = mla_profile_event(p, kProfAbsorb, false, s)) != cudaSuccess) return e;
+  e = mla_launch_kernel(absorb_kernel<bf16>, dim3(nblk), dim3(256), smem_abs, s, p.opt_pdl, aa);
+  if (e != cudaSuccess) return e;
+  if ((e = mla_profile_event(p, kProfAbsorb, true, s)) != cudaSuccess) return e;
+  char* base = (char*)ws;
+  const int units = B * ((Q + kQB - 1) / kQB);
+  e = mla_launch_chunk_tc(p, c, seq_lens, B, Q, aa.sched, base + L.off_qlat, (const float*)(base + L.off_qrope),
+                          (float*)(base + L.off_opart), (float*)(base + L.off_mlpart), L.P, L.G, s);
+  if (e != cudaSuccess) return e;
+  return launch_combine<bf16>(p, units, kQB * cfg.n_heads, kQB * cfg.n_kv_heads, Q, kQB, out, ws, L, aa.sched, s);
+}
+
 }  // namespace mla
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -657,6 +722,40 @@ DecodeLayout mla_decode_layout(const mla_plan& p, int B, int kernel) {
   L.off_mlpart = take(sizeof(float) * (size_t)L.P * H * 2);
   L.total = o;
   return L;
+}
+
+DecodeLayout mla_chunk_layout(const mla_plan& p, int B, int Q) {
+  const mla_config_t& cfg = p.cfg;
+  DecodeLayout L;
+  L.kernel = 3;
+  L.tile = 64;
+  L.G = p.opt_splits > 0 ? p.opt_splits : p.num_sms;
+  const int units = B * ((Q + 3) / 4), rows = 4 * cfg.n_heads;
+  L.P = units + L.G;
+  L.K = cfg.d_c + p.R;
+  const size_t nq = (size_t)B * Q * cfg.n_heads;   // query rows (query x head)
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o = align256(o + bytes); return r; };
+  L.off_seq_tile0 = take(sizeof(int32_t) * units);
+  L.off_seq_ntiles = take(sizeof(int32_t) * units);
+  L.off_seq_ne = take(sizeof(int32_t) * (units + 1));
+  L.off_seq_first = take(sizeof(int32_t) * units);
+  L.off_seq_np = take(sizeof(int32_t) * units);
+  L.off_worker_first = take(sizeof(int32_t) * (L.G + 1));
+  L.off_piece_b = take(sizeof(int32_t) * L.P);
+  L.off_piece_t0 = take(sizeof(int32_t) * L.P);
+  L.off_piece_t1 = take(sizeof(int32_t) * L.P);
+  L.off_qlat = take(sizeof(uint16_t) * nq * cfg.d_c);
+  L.off_qrope = take(sizeof(float) * nq * 2 * cfg.r_pairs + 4);
+  L.off_opart = take(sizeof(float) * (size_t)L.P * rows * cfg.d_c);
+  L.off_mlpart = take(sizeof(float) * (size_t)L.P * rows * 2);
+  L.total = o;
+  return L;
+}
+
+cudaError_t mla_launch_chunk(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, const void* q,
+                             int B, int Q, void* out, void* ws, const DecodeLayout& L, cudaStream_t s) {
+  return mla::launch_chunk(p, c, seq_lens, q, B, Q, out, ws, L, s);
 }
 
 Sched mla_sched_view(const DecodeLayout& L, void* ws, int B) {

@@ -45,9 +45,20 @@ __device__ inline int block_exscan(int v, int* total, int* s_warp) {
 // be read by the previous call).  When `scratch` (shared memory, `scratch_ints` ints) can
 // hold all of it, the schedule is built there and copied out once, coalesced; otherwise
 // it is built in the workspace directly.
+// Many queries per sequence (q_chunk > 1): the schedule runs over units v = (sequence b =
+// v / nqb, block k = v % nqb of q_block consecutive queries) and unit v's length is the
+// last position of its block + 1: L_b - q_chunk + min(q_chunk, (k + 1) q_block) tokens,
+// L_b = seq_lens[b] counting the chunk's own tokens.  B is then the number of units.
+__device__ __forceinline__ int unit_len(const int32_t* __restrict__ seq_lens, int v, int q_chunk, int q_block) {
+  if (q_chunk <= 1) return __ldg(seq_lens + v);
+  const int nqb = (q_chunk + q_block - 1) / q_block, k = v % nqb;
+  const int L = __ldg(seq_lens + v / nqb);
+  return L < q_chunk ? -1 : L - q_chunk + min(q_chunk, (k + 1) * q_block);
+}
+
 __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int B, int T_cap,
                                       int tile, int G, Sched out, int32_t* err, int32_t* scratch,
-                                      int scratch_ints) {
+                                      int scratch_ints, int q_chunk = 1, int q_block = 1) {
   __shared__ int s_warp[32];
   const int tid = threadIdx.x, nt = blockDim.x;
   const int Pcap = B + G;
@@ -75,7 +86,7 @@ __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int 
     const int b = base + tid;
     int nti = 0;
     if (b < B) {
-      int L = __ldg(seq_lens + b);
+      int L = unit_len(seq_lens, b, q_chunk, q_block);
       if (L < 0 || L > T_cap) { raise_error(err, MLA_DEVERR_SEQ_LEN); L = 0; }
       nti = (L + tile - 1) / tile;
       s.seq_ntiles[b] = nti;
@@ -136,7 +147,7 @@ __device__ inline void build_schedule(const int32_t* __restrict__ seq_lens, int 
     while (t < c1) {
       long long e = (long long)s.seq_tile0[b] + s.seq_ntiles[b];
       if (e > c1) e = c1;
-      int L = seq_len ? seq_len[b] : __ldg(seq_lens + b);
+      int L = seq_len ? seq_len[b] : unit_len(seq_lens, b, q_chunk, q_block);
       if (L < 0 || L > T_cap) L = 0;
       s.piece_b[pidx] = b;
       s.piece_t0[pidx] = (int)((t - s.seq_tile0[b]) * tile);

@@ -62,7 +62,6 @@ struct TcArgs {
   uint32_t c_row, kr_row;
   int32_t* err;
   uint64_t wait_ns;       // bound of every pipeline wait
-  int pf_dist, pf_mode;   // L2 prefetch: tiles ahead of the copies (0 = off); 1 lines, 2 bulk
   int skip_tile;          // testing only: 1-based tile whose latent copy is left out (0 = none)
   int NC, NRAW, NP, NO;  // ring depths; P^T and O buffers
   uint32_t off_c, off_q, off_p, off_raw, off_qr, off_bar, off_misc;
@@ -261,94 +260,59 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant
     setmaxnreg_dec<56>();
     if (warp == 0) {
       // ============================================================ TMA producer
-      // Lane 0 issues the copies; the whole warp walks the schedule a.pf_dist tiles ahead
-      // and asks L2 to fetch those tiles' cache bytes (latent rows, int4 scales, RoPE-key
-      // blocks), so HBM keeps streaming while the shared-memory stages are all busy.
-      TileIter it, pf;
-      it.init(&a.sched, w);
-      pf = it;
-      auto prefetch_tile = [&](const TileIter& ti) {
-        const int nvalid = min(kTile, ti.t1 - ti.t);
-        const MlaLoc lc = tc_loc<PAGED>(a, ti.b, ti.t);
-        const size_t row = (size_t)lc.pb * lc.cap + lc.pt;
-        const uint8_t* cp = reinterpret_cast<const uint8_t*>(a.cache.c_kv) + row * a.c_row;
-        const uint8_t* kp = a.kr_base + row * a.kr_row;
-        const uint8_t* sp = INT4 ? reinterpret_cast<const uint8_t*>(a.scales) + row * (dc / 16) : nullptr;
-        const uint32_t cbytes = (uint32_t)nvalid * a.c_row;
-        const uint32_t kbytes = (uint32_t)nvalid * a.kr_row;
-        const uint32_t sbytes = INT4 ? (uint32_t)nvalid * (dc / 16) : 0u;
-        if (a.pf_mode == 2) {   // bulk prefetches (sizes rounded down to 16 bytes: a hint)
-          if (lane == 0) {
-            prefetch_l2(cp, cbytes & ~15u);
-            prefetch_l2(kp, kbytes & ~15u);
-            if (INT4 && sbytes >= 16) prefetch_l2(sp, sbytes & ~15u);
-          }
-        } else {                // one 128-byte line per lane and instruction
-          for (uint32_t o = lane * 128u; o < cbytes; o += 32u * 128u) prefetch_l2_line(cp + o);
-          for (uint32_t o = lane * 128u; o < kbytes; o += 32u * 128u) prefetch_l2_line(kp + o);
-          if (INT4)
-            for (uint32_t o = lane * 128u; o < sbytes; o += 32u * 128u) prefetch_l2_line(sp + o);
-        }
-      };
-      if (a.pf_dist > 0) {   // tiles 1 .. pf_dist ahead of the first copy
-        pf.next();
-        for (int k = 0; k < a.pf_dist && pf.valid(); ++k) { prefetch_tile(pf); pf.next(); }
-      }
-      int n = 0, u = 0, q_loads = 0;
-      int last_c = -1, last_raw = -1, skipped = -1;
-      bool ok = true;
-      while (ok && it.valid()) {
-        if (a.pf_dist > 0 && pf.valid()) { prefetch_tile(pf); pf.next(); }
-        if (it.first_of_piece()) {
-          if (u > 0) ok = __all_sync(0xffffffffu, mbar_wait(bars.q_empty(), (u - 1) & 1, abort_flag, lim));
-          if (!ok) break;
-          if (lane == 0) {
+      if (lane == 0) {
+        TileIter it;
+        it.init(&a.sched, w);
+        int n = 0, u = 0, q_loads = 0;
+        int last = -1, skipped = -1;
+        bool ok = true;
+        while (ok && it.valid()) {
+          if (it.first_of_piece()) {
+            if (u > 0) ok = mbar_wait(bars.q_empty(), (u - 1) & 1, abort_flag, lim);
+            if (!ok) break;
             mbar_expect_tx(bars.q_full(), (uint32_t)n_cbox * kQBox);
             for (int kb = 0; kb < n_cbox; ++kb)
               tma_load_2d(qbox(kb), &tm_q, bars.q_full(), kb * 64, it.b * a.H);
+            ++q_loads;
           }
-          ++q_loads;
+          const MlaLoc lc = tc_loc<PAGED>(a, it.b, it.t);   // a tile is one paged block
+          const int row = lc.pb * lc.cap + lc.pt;
+          // testing hook (off unless set): leave this tile's latent copy out, so the waits
+          // on it run out and the kernel reports MLA_DEVERR_TIMEOUT
+          const bool skip = (n + 1 == a.skip_tile);
+          if (!INT4) {
+            const int cs = n % a.NC;
+            if (n >= a.NC) ok = mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag, lim);
+            if (!ok) break;
+            if (!skip) {
+              mbar_expect_tx(bars.c_full(cs), c_stage);
+              for (int cb = 0; cb < n_cbox; ++cb)
+                tma_load_2d(sbase_u32 + a.off_c + cs * c_stage + cb * kBox, &tm_c, bars.c_full(cs), cb * 64, row);
+            }
+          } else {
+            const int rs = n % a.NRAW;
+            if (n >= a.NRAW) ok = mbar_wait(bars.raw_empty(rs), ((n / a.NRAW) - 1) & 1, abort_flag, lim);
+            if (!ok) break;
+            const int nvalid = min(kTile, it.t1 - it.t);
+            const uint32_t sbytes = (uint32_t)((((nvalid + 1) & ~1) * (dc / 16) + 15) & ~15);
+            if (!skip) {
+              mbar_expect_tx(bars.raw_full(rs), raw_codes + sbytes);
+              tma_load_2d(sbase_u32 + a.off_raw + rs * raw_stage, &tm_c, bars.raw_full(rs), 0, row);
+              bulk_load(sbase_u32 + a.off_raw + rs * raw_stage + raw_codes, a.scales + (size_t)row * (dc / 32),
+                        sbytes, bars.raw_full(rs));
+            }
+          }
+          last = n;
+          if (skip) skipped = n;
+          if (it.last_of_piece()) ++u;
+          it.next();
+          ++n;
         }
-        const MlaLoc lc = tc_loc<PAGED>(a, it.b, it.t);   // a tile is one paged block
-        const int row = lc.pb * lc.cap + lc.pt;
-        // testing hook (off unless set): leave this tile's latent copy out, so the waits
-        // on it run out and the kernel reports MLA_DEVERR_TIMEOUT
-        const bool skip = (n + 1 == a.skip_tile);
-        if (!INT4) {
-          const int cs = n % a.NC;
-          if (n >= a.NC) ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag, lim));
-          if (!ok) break;
-          if (lane == 0 && !skip) {
-            mbar_expect_tx(bars.c_full(cs), c_stage);
-            for (int cb = 0; cb < n_cbox; ++cb)
-              tma_load_2d(sbase_u32 + a.off_c + cs * c_stage + cb * kBox, &tm_c, bars.c_full(cs), cb * 64, row);
-          }
-          last_c = n;
-        } else {
-          const int rs = n % a.NRAW;
-          if (n >= a.NRAW) ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_empty(rs), ((n / a.NRAW) - 1) & 1, abort_flag, lim));
-          if (!ok) break;
-          const int nvalid = min(kTile, it.t1 - it.t);
-          const uint32_t sbytes = (uint32_t)((((nvalid + 1) & ~1) * (dc / 16) + 15) & ~15);
-          if (lane == 0 && !skip) {
-            mbar_expect_tx(bars.raw_full(rs), raw_codes + sbytes);
-            tma_load_2d(sbase_u32 + a.off_raw + rs * raw_stage, &tm_c, bars.raw_full(rs), 0, row);
-            bulk_load(sbase_u32 + a.off_raw + rs * raw_stage + raw_codes, a.scales + (size_t)row * (dc / 32), sbytes,
-                      bars.raw_full(rs));
-          }
-          last_raw = n;
-        }
-        if (skip) skipped = n;
-        if (it.last_of_piece()) ++u;
-        it.next();
-        ++n;
-      }
-      // drain: every issued copy must land before the CTA can exit (a skipped copy's
-      // stage waits for the copy before it instead)
-      if (lane == 0) {
+        // drain: every issued copy must land before the CTA can exit (a skipped copy's
+        // stage waits for the copy before it instead)
         volatile int never = 0;
         if (q_loads > 0) mbar_wait(bars.q_full(), (q_loads - 1) & 1, &never, lim);
-        const int NS = INT4 ? a.NRAW : a.NC, last = INT4 ? last_raw : last_c;
+        const int NS = INT4 ? a.NRAW : a.NC;
         for (int s = 0; s < NS; ++s) {
           int k = last - ((last - s) % NS + NS) % NS;
           if (k == skipped) k -= NS;
@@ -942,8 +906,6 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
   a.c_row = int4 ? (uint32_t)code_row : (uint32_t)dc * 2;
   a.kr_row = (uint32_t)R * 2;
   a.wait_ns = (uint64_t)p.opt_wait_us * 1000u;
-  a.pf_dist = p.opt_pf_dist;
-  a.pf_mode = p.opt_pf_mode;
   a.skip_tile = p.opt_skip_tile;
   a.NC = L.NC; a.NRAW = L.NRAW; a.NP = L.NP; a.NO = L.NO;
   a.off_c = L.off_c; a.off_q = L.off_q; a.off_p = L.off_p; a.off_raw = L.off_raw;

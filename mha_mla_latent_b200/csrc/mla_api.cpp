@@ -254,11 +254,7 @@ mla_status_t mla_plan_set_option(mla_plan_t* plan, int32_t option, int64_t value
       if (value < 0 || value > (1 << 20)) return MLA_ERR_INVALID_ARG;
       plan->opt_skip_tile = (int)value;
       return MLA_OK;
-    case MLA_OPT_L2_PREFETCH:
-      if (value < 0 || (value & 0xFF) > 16 || (value >> 8) > 2) return MLA_ERR_INVALID_ARG;
-      plan->opt_pf_dist = (int)(value & 0xFF);
-      if ((value >> 8) != 0) plan->opt_pf_mode = (int)(value >> 8);
-      return MLA_OK;
+
   }
   return MLA_ERR_INVALID_ARG;
 }
@@ -331,6 +327,28 @@ mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache, const 
   if (ws_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
   return cuda_status(mla_launch_decode(*plan, *cache, seq_lens, q, B, out, workspace, L,
                                        (cudaStream_t)stream));
+}
+
+size_t mla_decode_chunk_workspace_bytes(const mla_plan_t* plan, int32_t B, int32_t Q) {
+  if (!plan || B <= 0 || Q <= 0) return 0;
+  if (Q == 1) return mla_decode_workspace_bytes(plan, B);
+  return mla_chunk_layout(*plan, B, Q).total;
+}
+
+mla_status_t mla_decode_chunk(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
+                              const void* q, int32_t B, int32_t Q, void* out, void* workspace, size_t ws_bytes,
+                              void* stream) {
+  if (!plan || !seq_lens || !q || !out || !workspace || B <= 0 || Q <= 0) return MLA_ERR_INVALID_ARG;
+  if (Q == 1) return mla_decode(plan, cache, seq_lens, q, B, out, workspace, ws_bytes, stream);
+  mla_status_t st = mla_validate_cache(plan->cfg, cache);
+  if (st != MLA_OK) return st;
+  if (B > cache->B || (long long)Q > cache->T_cap) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace) || ((uintptr_t)seq_lens & 3))
+    return MLA_ERR_ALIGNMENT;
+  if (!mla_chunk_capable(*plan) || plan->opt_kernel == 1) return MLA_ERR_UNSUPPORTED;
+  DecodeLayout L = mla_chunk_layout(*plan, B, Q);
+  if (ws_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  return cuda_status(mla_launch_chunk(*plan, *cache, seq_lens, q, B, Q, out, workspace, L, (cudaStream_t)stream));
 }
 
 mla_status_t mla_decode_step(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,

@@ -78,7 +78,6 @@ struct mla_plan {
   int opt_pdl = 1;                            // programmatic dependent launch
   int64_t opt_wait_us = 1000000;              // bound of each pipeline wait (tensor-core kernel)
   int opt_skip_tile = 0;                      // testing: leave out one latent copy per CTA
-  int opt_pf_dist = 2, opt_pf_mode = 1;       // L2 prefetch lookahead (tiles) and form
 };
 
 // Launches a kernel, with programmatic stream serialization when `pdl` is set (the kernel
@@ -156,6 +155,14 @@ cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const 
                                  const void* qlat, const float* qrope, float* opart, float* mlpart, int P, int G,
                                  cudaStream_t s);
 Sched mla_sched_view(const DecodeLayout& L, void* ws, int B);
+// Many queries per sequence: workspace layout, the chunk kernel's shape limits and launches.
+DecodeLayout mla_chunk_layout(const mla_plan& p, int B, int Q);
+bool mla_chunk_capable(const mla_plan& p);
+cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B, int Q,
+                                const Sched& sched, const void* qlat, const float* qrope, float* opart,
+                                float* mlpart, int P, int G, cudaStream_t s);
+cudaError_t mla_launch_chunk(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, const void* q,
+                             int B, int Q, void* out, void* ws, const DecodeLayout& L, cudaStream_t s);
 
 cudaError_t mla_launch_select_pairs(const mla_config_t& cfg, const void* q, const void* k, int T,
                                     int32_t* pair_idx, float* contrib, cudaStream_t s);

@@ -500,5 +500,6 @@ def test_decode_softmax_scale(idx):
         ref = O.decode_unabsorbed(case.q[b], cc["c"], cc["kr"], case.conv["W_uk"], case.conv["W_uv"],
                                   case.conv["pair_idx"], case.theta, scale=scale)
         assert_close(got[b], ref, wl.dtype, f"{wl.name} scale seq {b}")
-        assert not np.allclose(ref, case.reference(b), rtol=1e-3)
+        if case.lens[b] > 1:   # one token: its value whatever the scale
+            assert not np.allclose(ref, case.reference(b), rtol=1e-3)
     plan.close()
