@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--kernel", type=int, default=0, help="decode kernel: 0 auto, 1 CUDA-core, 2 tcgen05")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--separate-calls", action="store_true",
+                    help="time the step as mla_append + mla_decode instead of one mla_decode_step")
     ap.add_argument("--no-per-workload", dest="per_workload", action="store_false",
                     help="measure only --workload (default: also the ragged and int4 workloads at N=1)")
     return ap.parse_args()
@@ -67,7 +69,7 @@ def wl_config(wl, lens):
             "latent_cache": ("int4 g32 + fp16 scales" + (f", {wl.resid}-token bf16 residual window" if wl.resid else "")
                              if wl.cache == "int4_g32" else
                              "int2 g32 + fp16 scales" if wl.cache == "int2_g32" else wl.dtype),
-            "step": "mla_append(B new tokens) + mla_decode(B queries)"}
+            "step": "mla_decode_step: append of the B new tokens + decode of the B queries"}
 
 
 # ------------------------------------------------------------------ oracle (CPU) timing
@@ -253,7 +255,7 @@ class Bench:
     """One workload set up on one GPU: the converted plan, cache replicas that together
     exceed twice the L2, the step's inputs, and the measurements of one step."""
 
-    def __init__(self, name, dev, kernel=0):
+    def __init__(self, name, dev, kernel=0, fused=True):
         import torch
         import mha_mla_latent_b200 as mla
         from mha_mla_latent_b200.cache import LatentCache, workspace
@@ -261,6 +263,7 @@ class Bench:
         from workloads import generate as gen
 
         self.mla, self.torch = mla, torch
+        self.fused = fused
         wl = self.wl = workload(name)
         self.dev = dev
         cfg = self.cfg = mla.config_from_workload(wl)
@@ -327,13 +330,18 @@ class Bench:
         torch.cuda.synchronize()
         assert mla.mla_device_error(plan) == 0
         self.tokens = int(np.sum(lens))
-        # append, absorb(+schedule), split-K attention, combine(+W_uv); + the ring-slot claim
-        self.launches_per_step = 4 + (1 if wl.resid else 0)
+        # fused step: append + absorb(+schedule) in one kernel, split-K attention, combine(+W_uv);
+        # separate calls: append (+ the ring-slot claim), absorb, attention, combine
+        self.launches_per_step = 3 if fused else 4 + (1 if wl.resid else 0)
 
     def step(self, i):
         c = self.caches[i % self.n_rep].struct
-        self.mla.mla_append(self.plan, self.xd, self.seq_idx, self.pos, c, stream=self.stream)
-        self.mla.mla_decode(self.plan, c, self.seq_lens, self.q, self.out, self.ws, stream=self.stream)
+        if self.fused:   # one call: append of the B new tokens + decode of the B queries
+            self.mla.mla_decode_step(self.plan, c, self.seq_lens, self.xd, self.q, self.out, self.ws,
+                                     stream=self.stream)
+        else:
+            self.mla.mla_append(self.plan, self.xd, self.seq_idx, self.pos, c, stream=self.stream)
+            self.mla.mla_decode(self.plan, c, self.seq_lens, self.q, self.out, self.ws, stream=self.stream)
 
     def timed_steps(self, K, world=1, sampler=None):
         """ms per step over K steps (device time, CUDA events on the launching stream), the
@@ -385,8 +393,10 @@ class Bench:
         torch.cuda.synchronize()
         mla.mla_plan_set_option(self.plan, mla.MLA_OPT_PROFILE_KERNELS, 0)
         names = ("append", "absorb", "attention", "combine")
+        if self.fused:   # the append runs inside the first kernel with the absorption
+            names = (None, "append+absorb", "attention", "combine")
         return {n: statistics.mean(ev[i][2 * k].elapsed_time(ev[i][2 * k + 1]) for i in range(K))
-                for k, n in enumerate(names)}
+                for k, n in enumerate(names) if n}
 
     def decode_only_ms(self, K):
         torch = self.torch
@@ -401,9 +411,11 @@ class Bench:
         return s2.elapsed_time(e2) / K
 
     def e2e(self, E):
-        """The same step end to end through the public API with host buffers: pinned host
-        x and q copied in and the output read back inside the timed region, every step."""
+        """The same step end to end through one C-ABI call with host buffers
+        (mla_decode_step_host): pinned host sequence lengths, x and q copied in and the
+        output copied back inside the timed region, every step."""
         torch = self.torch
+        lh = self.seq_lens.cpu().pin_memory()
         xh = self.xd.cpu().pin_memory()
         qh = self.q.cpu().pin_memory()
         oh = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
@@ -411,14 +423,12 @@ class Bench:
         s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s3.record(self.stream)
         for i in range(E):
-            self.xd.copy_(xh, non_blocking=True)
-            self.q.copy_(qh, non_blocking=True)
-            self.step(i)
-            oh.copy_(self.out, non_blocking=True)
+            self.mla.mla_decode_step_host(self.plan, self.caches[i % self.n_rep].struct, lh, xh, qh, oh, self.ws,
+                                          stream=self.stream)
         e3.record(self.stream)
         torch.cuda.synchronize()
-        h2d = self.xd.numel() * self.xd.element_size() + self.q.numel() * self.q.element_size()
-        d2h = self.out.numel() * self.out.element_size()
+        h2d = sum(t.numel() * t.element_size() for t in (lh, xh, qh))
+        d2h = oh.numel() * oh.element_size()
         return s3.elapsed_time(e3) / E, h2d, d2h
 
     def roofline(self, attention_ms, workload_name):
@@ -463,7 +473,7 @@ def run_ours(args):
     build.build()
 
     dev = torch.device("cuda", local)
-    bn = Bench(args.workload, dev, args.kernel)
+    bn = Bench(args.workload, dev, args.kernel, fused=not args.separate_calls)
     wl, K = bn.wl, args.steps
     for i in range(args.warmup):
         bn.step(i)
@@ -509,7 +519,7 @@ def run_ours(args):
         for name in PER_WORKLOADS:
             if name == args.workload:
                 continue
-            b2 = Bench(name, dev, args.kernel)
+            b2 = Bench(name, dev, args.kernel, fused=not args.separate_calls)
             Kw = max(20, min(K, 500))
             for i in range(args.warmup):
                 b2.step(i)

@@ -23,40 +23,44 @@ namespace mla {
 struct AbsorbArgs {
   const void* q;              // [B][H][d_h]
   const int32_t* seq_lens;
-  int B, T_cap, H, n_kv, dh, r, d_c, dn;
-  const void* W_ukT;          // [n_kv][dn][d_c]
-  const int32_t* nope_idx;    // [n_kv][dn]
+  int B, T_cap, H, n_kv, dh, r, d_c;
+  const void* W_ukF;          // [n_kv][d_h][d_c]: W_uk^T on the NoPE dims, zero rows on the kept pairs
   const int32_t* rope_pair;   // [n_kv][r]
   const double* theta;
   float* qlat;                // f32 [B][H][d_c]        (CUDA-core kernel), or null
-  __nv_bfloat16* qlat16;      // bf16 [B][H][d_c]       (tcgen05 kernel), or null
+  __nv_bfloat16* qlat16;      // bf16 [B][H][d_c]       (tcgen05 kernels), or null
   float* qrope;               // f32 [B][H][2r]
   Sched sched;
   int tile, G;
   int32_t* err;
   int sched_ints;             // shared memory of the schedule CTA, in ints
   float sm_scale;             // softmax scale of the scores (1/sqrt(d_h) unless the config sets one)
-  int vec_ok;                 // q and W_uk^T rows allow 16-byte loads
+  int vec_ok;                 // q and W rows allow 16-byte loads
+  int mma;                    // product as bf16 warp MMAs (32 rows per CTA), else CUDA cores (8 rows)
   // many queries per sequence: query rows s = b * q_chunk + i sit at position
   // seq_lens[b] - q_chunk + i; the schedule runs over units of q_block queries (1, 1: decode)
   int q_chunk, q_block;
 };
 
-constexpr int kAbsRows = 8;    // (b, h) rows per CTA: one per warp in the product
-constexpr int kAbsCols = 64;   // latent columns per CTA: two per lane
+constexpr int kAbsRows = 8;       // (b, h) rows per CTA, CUDA-core form: one per warp
+constexpr int kAbsRowsMma = 32;   // rows per CTA, warp-MMA form: two m16 tiles
+constexpr int kAbsCols = 64;      // latent columns per CTA
 
 // Block `blk` of the absorption grid: block 0 builds the split-K schedule (dispatched
-// first), blocks 1 .. n_kv * (row blocks) * (column chunks) compute q_lat.  A CTA stages
-// what comes from the plan (its W_uk^T slice, the NoPE index table, the RoPE pair table
-// and frequencies) before the dependency wait and the caller's queries and sequence lengths
-// after it, then q_lat[row][c] = scale * sum_j q[row][nope_j] * W_uk^T[g][j][c] with warp r
-// owning row r and lane l columns 2l, 2l+1 of the chunk.  `sm` is the CTA's dynamic shared
-// memory.
+// first), blocks 1 .. n_kv * (row blocks) * (column chunks) compute
+//     q_lat[row][c] = scale * sum_d q[row][d] * W_ukF[g][d][c]
+// for a block of (b, h) rows of KV head g and 64 latent columns.  W_ukF carries W_uk^T on
+// the NoPE dims and zero rows on the kept pairs' dims, so the unrotated query is used as it
+// is (no NoPE gather).  The kept pairs of the first column chunk's rows are rotated at the
+// query's position (angle in double) and scaled into q_rope.  What comes from the plan
+// (W_ukF slice, pair table, frequencies) is staged before the dependency wait, the
+// caller's queries and lengths after it.  `sm` is the CTA's dynamic shared memory.
 template <typename T>
 __device__ __forceinline__ void absorb_body(const AbsorbArgs& a, int blk_id, float* sm) {
   const int G = a.H / a.n_kv;
   const int rows_total = a.B * G;
-  const int n_rb = (rows_total + kAbsRows - 1) / kAbsRows;
+  const int RPC = a.mma ? kAbsRowsMma : kAbsRows;
+  const int n_rb = (rows_total + RPC - 1) / RPC;
   if (blk_id == 0) {  // the split-K schedule
     const int nunits = a.q_chunk > 1 ? (a.B / a.q_chunk) * ((a.q_chunk + a.q_block - 1) / a.q_block) : a.B;
     build_schedule(a.seq_lens, nunits, a.T_cap, a.tile, a.G, a.sched, a.err, reinterpret_cast<int32_t*>(sm),
@@ -67,65 +71,115 @@ __device__ __forceinline__ void absorb_body(const AbsorbArgs& a, int blk_id, flo
   const int g = blk % a.n_kv;
   const int rb = (blk / a.n_kv) % n_rb;
   const int cc = blk / (a.n_kv * n_rb);
-  const int row0 = rb * kAbsRows, c0 = cc * kAbsCols;
+  const int row0 = rb * RPC, c0 = cc * kAbsCols;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int dn = a.dn, dh = a.dh, dnp = (dn + 3) & ~3;
-  float* s_w = sm;                              // [dn][kAbsCols]
-  float* s_q = s_w + dn * kAbsCols;             // [kAbsRows][dh] raw query rows
-  float* s_qn = s_q + kAbsRows * dh;            // [kAbsRows][dnp] NoPE dims, gathered
-  int* s_idx = reinterpret_cast<int*>(s_qn + kAbsRows * dnp);   // [dn]
+  const int dh = a.dh;
   const T* q = (const T*)a.q;
-  const T* W = (const T*)a.W_ukT + (size_t)g * dn * a.d_c;
-  // ---- plan data: W slice, NoPE indices, RoPE pair frequencies
-  const int ncol = min(kAbsCols, a.d_c - c0);
-  if (ncol < kAbsCols)
-    for (int i = tid; i < dn * kAbsCols; i += 256) s_w[i] = 0.f;   // columns past d_c
-  stage_rows_f32<T>(s_w, kAbsCols, dn, ncol, a.vec_ok && ncol == kAbsCols,
-                    [&](int j) { return W + (size_t)j * a.d_c + c0; });
-  for (int j = tid; j < dn; j += 256) s_idx[j] = __ldg(a.nope_idx + g * dn + j);
+  const T* W = (const T*)a.W_ukF + (size_t)g * dh * a.d_c;
   const float scale = kLog2e * a.sm_scale;
-  const int nrope = (cc == 0) ? kAbsRows * a.r : 0;
-  int rp_k = 0;
-  double rp_th = 0.0;
-  const bool rope_item = tid < nrope && row0 + tid / max(a.r, 1) < rows_total;
-  if (rope_item) {
-    rp_k = __ldg(a.rope_pair + g * a.r + tid % a.r);
-    rp_th = __ldg(a.theta + rp_k);
-  }
-  // ---- the caller's queries and lengths; the outputs are read by the attention kernel of
-  // the previous call until it has finished
-  pdl_wait();
-  pdl_trigger();
-  const int nrow = min(kAbsRows, rows_total - row0);
-  stage_rows_f32<T>(s_q, dh, nrow, dh, a.vec_ok, [&](int r) {
+  const int nrow = min(RPC, rows_total - row0);
+  auto q_row = [&](int r) {   // query row r of this CTA
     const int row = row0 + r;
     return q + ((size_t)(row / G) * a.H + g * G + row % G) * dh;
-  });
-  int rp_pos = 0;   // length up to and including the query row's token (its position + 1)
-  if (rope_item) {
-    const int sq = (row0 + tid / a.r) / G;
-    rp_pos = __ldg(a.seq_lens + sq / a.q_chunk) - (a.q_chunk - 1 - sq % a.q_chunk);
+  };
+  auto out_index = [&](int row, int c) { return ((size_t)(row / G) * a.H + g * G + row % G) * a.d_c + c; };
+  // RoPE query part (first column chunk): rotate the kept pairs at the query's position
+  // (angle in double), scale.  qv(r, d) reads element d of staged row r.
+  auto rope = [&](auto qv) {
+    if (cc != 0) return;
+    for (int item = tid; item < nrow * a.r; item += blockDim.x) {
+      const int r = item / a.r, jr = item % a.r, row = row0 + r;
+      const int k = __ldg(a.rope_pair + g * a.r + jr);
+      const int sq = row / G;
+      const int L = __ldg(a.seq_lens + sq / a.q_chunk) - (a.q_chunk - 1 - sq % a.q_chunk);
+      const int p = (L >= 1 && L <= a.T_cap) ? L - 1 : 0;
+      const double x0 = qv(r, 2 * k), x1 = qv(r, 2 * k + 1);
+      double sn, cs;
+      sincos((double)p * __ldg(a.theta + k), &sn, &cs);
+      const size_t o = ((size_t)sq * a.H + g * G + row % G) * 2 * a.r + 2 * jr;
+      a.qrope[o] = (float)((x0 * cs - x1 * sn) * (double)scale);
+      a.qrope[o + 1] = (float)((x0 * sn + x1 * cs) * (double)scale);
+    }
+  };
+
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    if (a.mma) {
+      // ---- warp-MMA form: Qs [32][KP+8] and Ws [KP][64+8] bf16 tiles (16-byte padded rows,
+      // conflict-free ldmatrix), staged with 16-byte asynchronous copies (zero-filled past
+      // the matrix edges); warps 0-3 each take 16 columns x 32 rows, K = d_h
+      using bf16 = __nv_bfloat16;
+      const int KP = (dh + 15) & ~15, QLD = KP + 8;
+      constexpr int WLD = kAbsCols + 8;
+      bf16* Ws = reinterpret_cast<bf16*>(sm);   // [KP][WLD]
+      bf16* Qs = Ws + KP * WLD;                 // [32][QLD]
+      for (int v = tid; v < KP * (kAbsCols / 8); v += blockDim.x) {
+        const int d = v / (kAbsCols / 8), part = v % (kAbsCols / 8), c = c0 + part * 8;
+        const bool ok = d < dh && c + 8 <= a.d_c;
+        sm100::cp_async16(wmma16::smem_addr(Ws + d * WLD + part * 8),
+                          ok ? (const void*)(W + (size_t)d * a.d_c + c) : a.W_ukF, ok ? 16u : 0u);
+      }
+      sm100::cp_async_commit();
+      pdl_wait();
+      pdl_trigger();
+      for (int v = tid; v < kAbsRowsMma * (KP / 8); v += blockDim.x) {
+        const int r = v / (KP / 8), ch = v % (KP / 8);
+        const bool ok = r < nrow && ch * 8 + 8 <= dh;
+        sm100::cp_async16(wmma16::smem_addr(Qs + r * QLD + ch * 8), ok ? (const void*)(q_row(r) + ch * 8) : a.q,
+                          ok ? 16u : 0u);
+      }
+      sm100::cp_async_commit();
+      sm100::cp_async_wait_all();
+      __syncthreads();
+      rope([&](int r, int d) { return (double)__bfloat162float(Qs[r * QLD + d]); });
+      if (warp < 4) {
+        float acc[2][2][4] = {};
+        for (int k0 = 0; k0 < KP; k0 += 16) {
+          uint32_t af[2][4], bfr[4];
+          wmma16::load_a(af[0], Qs, QLD, 0, k0, lane);
+          wmma16::load_a(af[1], Qs, QLD, 16, k0, lane);
+          wmma16::load_b2(bfr, Ws, WLD, k0, 16 * warp, lane);
+#pragma unroll
+          for (int m = 0; m < 2; ++m) {
+            wmma16::mma_16816(acc[m][0], af[m], bfr[0], bfr[1]);
+            wmma16::mma_16816(acc[m][1], af[m], bfr[2], bfr[3]);
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) {
+              const int r = 16 * m + (lane >> 2) + 8 * hlf, c = c0 + 16 * warp + 8 * nt + 2 * (lane & 3);
+              if (r >= nrow || c >= a.d_c) continue;
+              const float v0 = acc[m][nt][2 * hlf] * scale, v1 = acc[m][nt][2 * hlf + 1] * scale;
+              const size_t o = out_index(row0 + r, c);
+              if (a.qlat16) *reinterpret_cast<__nv_bfloat162*>(a.qlat16 + o) = __floats2bfloat162_rn(v0, v1);
+              if (a.qlat) *reinterpret_cast<float2*>(a.qlat + o) = make_float2(v0, v1);
+            }
+      }
+      return;
+    }
   }
+  // ---- CUDA-core form: W slice and query rows as float in shared memory; warp r takes
+  // row r, lane l columns 2l, 2l+1 of the chunk
+  float* s_w = sm;                              // [dh][kAbsCols]
+  float* s_q = s_w + dh * kAbsCols;             // [kAbsRows][dh]
+  const int ncol = min(kAbsCols, a.d_c - c0);
+  if (ncol < kAbsCols)
+    for (int i = tid; i < dh * kAbsCols; i += blockDim.x) s_w[i] = 0.f;   // columns past d_c
+  stage_rows_f32<T>(s_w, kAbsCols, dh, ncol, a.vec_ok && ncol == kAbsCols,
+                    [&](int j) { return W + (size_t)j * a.d_c + c0; });
+  pdl_wait();
+  pdl_trigger();
+  stage_rows_f32<T>(s_q, dh, nrow, dh, a.vec_ok, q_row);
   __syncthreads();
-  for (int i = tid; i < kAbsRows * dn; i += 256) s_qn[(i / dn) * dnp + i % dn] = s_q[(i / dn) * dh + s_idx[i % dn]];
-  // RoPE query part: rotate the kept pairs at position L-1 (angle in double), scale
-  float ro0 = 0.f, ro1 = 0.f;
-  if (rope_item) {
-    const int r = tid / a.r;
-    const int p = (rp_pos >= 1 && rp_pos <= a.T_cap) ? rp_pos - 1 : 0;
-    const double x0 = s_q[r * dh + 2 * rp_k], x1 = s_q[r * dh + 2 * rp_k + 1];
-    double sn, cs;
-    sincos((double)p * rp_th, &sn, &cs);
-    ro0 = (float)((x0 * cs - x1 * sn) * (double)scale);
-    ro1 = (float)((x0 * sn + x1 * cs) * (double)scale);
-  }
-  __syncthreads();
-  // ---- product: warp r -> row r, lane l -> columns 2l, 2l+1 of the chunk
+  rope([&](int r, int d) { return (double)s_q[r * dh + d]; });
   const int r = warp, row = row0 + r, c = c0 + 2 * lane;
-  const float* qn = s_qn + r * dnp;
+  const float* qn = s_q + r * dh;
   float acc0 = 0.f, acc1 = 0.f;
   int j = 0;
-  for (; j + 4 <= dn; j += 4) {
+  for (; j + 4 <= dh; j += 4) {
     const float4 x = *reinterpret_cast<const float4*>(qn + j);
     const float2 w0 = *reinterpret_cast<const float2*>(s_w + (j + 0) * kAbsCols + 2 * lane);
     const float2 w1 = *reinterpret_cast<const float2*>(s_w + (j + 1) * kAbsCols + 2 * lane);
@@ -134,19 +188,13 @@ __device__ __forceinline__ void absorb_body(const AbsorbArgs& a, int blk_id, flo
     acc0 += x.x * w0.x + x.y * w1.x + x.z * w2.x + x.w * w3.x;
     acc1 += x.x * w0.y + x.y * w1.y + x.z * w2.y + x.w * w3.y;
   }
-  for (; j < dn; ++j) {
+  for (; j < dh; ++j) {
     const float2 w = *reinterpret_cast<const float2*>(s_w + j * kAbsCols + 2 * lane);
     acc0 += qn[j] * w.x;
     acc1 += qn[j] * w.y;
   }
-  if (rope_item) {
-    const int rr = tid / a.r, jr = tid % a.r, rrow = row0 + rr;
-    const size_t o = ((size_t)(rrow / G) * a.H + g * G + rrow % G) * 2 * a.r + 2 * jr;
-    a.qrope[o] = ro0;
-    a.qrope[o + 1] = ro1;
-  }
-  if (row < rows_total && c < a.d_c) {
-    const size_t o = ((size_t)(row / G) * a.H + g * G + row % G) * a.d_c + c;
+  if (r < nrow && c < a.d_c) {
+    const size_t o = out_index(row, c);
     if (a.qlat) {
       a.qlat[o] = acc0 * scale;
       if (c + 1 < a.d_c) a.qlat[o + 1] = acc1 * scale;
@@ -505,7 +553,7 @@ void absorb_setup(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_le
   char* base = (char*)ws;
   aa->q = q; aa->seq_lens = seq_lens; aa->B = B; aa->T_cap = c.T_cap; aa->H = H;
   aa->n_kv = cfg.n_kv_heads; aa->dh = cfg.head_dim; aa->r = cfg.r_pairs; aa->d_c = cfg.d_c;
-  aa->dn = p.dn; aa->W_ukT = p.W_ukT; aa->nope_idx = p.nope_idx;
+  aa->W_ukF = p.W_ukF;
   aa->rope_pair = p.rope_pair; aa->theta = p.theta;
   aa->qlat = L.kernel == 1 ? (float*)(base + L.off_qlat) : nullptr;
   aa->qlat16 = L.kernel == 2 ? (__nv_bfloat16*)(base + L.off_qlat) : nullptr;
@@ -518,10 +566,13 @@ void absorb_setup(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_le
     const int vecn = 16 / (int)sizeof(T);   // elements per 16-byte load
     aa->vec_ok = ((uintptr_t)q % 16 == 0) && cfg.d_c % vecn == 0 && cfg.head_dim % vecn == 0;
   }
-  const int n_rb = (B * G + kAbsRows - 1) / kAbsRows, n_cc = (cfg.d_c + kAbsCols - 1) / kAbsCols;
-  const int dnp = (p.dn + 3) & ~3;
-  const size_t smem_work = sizeof(float) * ((size_t)p.dn * kAbsCols + (size_t)kAbsRows * cfg.head_dim +
-                                            (size_t)kAbsRows * dnp + p.dn);
+  aa->mma = std::is_same<T, __nv_bfloat16>::value && aa->vec_ok && cfg.d_c % 8 == 0 && cfg.head_dim % 8 == 0;
+  const int RPC = aa->mma ? kAbsRowsMma : kAbsRows;
+  const int n_rb = (B * G + RPC - 1) / RPC, n_cc = (cfg.d_c + kAbsCols - 1) / kAbsCols;
+  const int KP = (cfg.head_dim + 15) & ~15;
+  const size_t smem_work =
+      aa->mma ? sizeof(__nv_bfloat16) * ((size_t)KP * (kAbsCols + 8) + (size_t)kAbsRowsMma * (KP + 8))
+              : sizeof(float) * ((size_t)cfg.head_dim * kAbsCols + (size_t)kAbsRows * cfg.head_dim);
   const size_t sched_ints = (size_t)9 * B + 4 * L.G + 2;
   *smem = std::min<size_t>(std::max(smem_work, sched_ints * sizeof(int32_t)), std::max<size_t>(smem_work, 160 * 1024));
   aa->sched_ints = (int)(*smem / sizeof(int32_t));

@@ -67,8 +67,7 @@ bool dev_alloc_copy(void** dst, const void* src, size_t bytes) {
 
 void free_plan(mla_plan* p) {
   if (!p) return;
-  void* bufs[] = {p->W_app, p->W_ukT, p->W_uv, p->nope_idx, p->rope_pair, p->theta, p->err, p->app_part,
-                  p->app_ticket};
+  void* bufs[] = {p->W_app, p->W_ukF, p->W_uv, p->rope_pair, p->theta, p->err, p->app_part, p->app_ticket};
   for (void* b : bufs)
     if (b) cudaFree(b);
   delete p;
@@ -184,28 +183,29 @@ mla_status_t mla_plan_create(const mla_config_t* cfg, const void* W_dkv, const v
                  (const unsigned char*)W_k + ((size_t)i * nkv * dh + src_col) * eb, eb);
         }
   }
-  // W_uk transposed per head: [g][j][c]
-  std::vector<unsigned char> ukT((size_t)nkv * std::max(p->dn, 1) * dc * eb, 0);
-  for (int g = 0; g < nkv; ++g)
-    for (int c = 0; c < dc; ++c)
-      for (int j = 0; j < p->dn; ++j)
-        memcpy(&ukT[(((size_t)g * p->dn + j) * dc + c) * eb],
-               (const unsigned char*)W_uk + (((size_t)g * dc + c) * p->dn + j) * eb, eb);
-  std::vector<int32_t> nope((size_t)nkv * std::max(p->dn, 1), 0), rp((size_t)nkv * std::max(r, 1), 0);
+  // W_uk transposed per head onto the full head dims: [g][d][c] = W_uk[g][c][j] where d is
+  // the j-th NoPE dim of KV head g; the rows of the kept pairs' dims stay zero, so an
+  // unrotated query can be multiplied as it is
+  std::vector<unsigned char> ukF((size_t)nkv * dh * dc * eb, 0);
+  std::vector<int32_t> rp((size_t)nkv * std::max(r, 1), 0);
   for (int g = 0; g < nkv; ++g) {
     std::vector<char> kept(dh / 2, 0);
     for (int j = 0; j < r; ++j) { kept[pair_idx[g * r + j]] = 1; rp[g * r + j] = pair_idx[g * r + j]; }
-    int n = 0;
-    for (int i = 0; i < dh; ++i)
-      if (!kept[i / 2]) nope[(size_t)g * p->dn + (n++)] = i;
+    int j = 0;
+    for (int d = 0; d < dh; ++d) {
+      if (kept[d / 2]) continue;
+      for (int c = 0; c < dc; ++c)
+        memcpy(&ukF[(((size_t)g * dh + d) * dc + c) * eb],
+               (const unsigned char*)W_uk + (((size_t)g * dc + c) * p->dn + j) * eb, eb);
+      ++j;
+    }
   }
   std::vector<double> theta(dh / 2);
   for (int k = 0; k < dh / 2; ++k) theta[k] = pow(cfg->rope_base, -2.0 * k / dh);
 
   bool ok = dev_alloc_copy(&p->W_app, app.data(), app.size()) &&
-            dev_alloc_copy(&p->W_ukT, ukT.data(), ukT.size()) &&
+            dev_alloc_copy(&p->W_ukF, ukF.data(), ukF.size()) &&
             dev_alloc_copy(&p->W_uv, W_uv, (size_t)nkv * dc * dh * eb) &&
-            dev_alloc_copy((void**)&p->nope_idx, nope.data(), nope.size() * sizeof(int32_t)) &&
             dev_alloc_copy((void**)&p->rope_pair, rp.data(), rp.size() * sizeof(int32_t)) &&
             dev_alloc_copy((void**)&p->theta, theta.data(), theta.size() * sizeof(double)) &&
             cudaMalloc((void**)&p->err, sizeof(int32_t)) == cudaSuccess &&

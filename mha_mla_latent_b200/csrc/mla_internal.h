@@ -62,9 +62,8 @@ struct mla_plan {
   int ncols = 0;   // d_c + R     (columns of the packed append weight)
   // plan-owned device memory
   void* W_app = nullptr;       // [d][ncols] dtype: [W_dkv | W_krope]
-  void* W_ukT = nullptr;       // [n_kv][dn][d_c] dtype (W_uk transposed per head)
+  void* W_ukF = nullptr;       // [n_kv][d_h][d_c] dtype: W_uk^T on the NoPE dims, zero rows on the kept pairs
   void* W_uv = nullptr;        // [n_kv][d_c][d_h] dtype
-  int32_t* nope_idx = nullptr;   // [n_kv][dn]  NoPE dims, ascending
   int32_t* rope_pair = nullptr;  // [n_kv][r]   kept pair indices, ascending
   double* theta = nullptr;       // [d_h/2]     RoPE frequencies
   int32_t* err = nullptr;        // device error word (MLA_DEVERR_* bits)
