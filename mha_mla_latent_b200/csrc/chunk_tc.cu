@@ -45,6 +45,8 @@ constexpr uint32_t kSCol = 0, kOCol = 128;
 
 struct ChunkArgs {
   int q_chunk, nqb, d_c, R, P, T_cap;
+  const __half* scales;    // quantised cache: [rows][d_c/32] fp16 group scales
+  uint32_t code_row;       // quantised cache: code bytes per token
   Sched sched;
   const int32_t* seq_lens;
   const float* qrope;      // [B*Q][32][2r], rotated at each query's position, scaled
@@ -53,8 +55,8 @@ struct ChunkArgs {
   mla_cache_t cache;
   int32_t* err;
   uint64_t wait_ns;
-  int NC;
-  uint32_t off_q, off_stage, off_p, off_bar, off_misc, stage_bytes;
+  int NC, NRAW;
+  uint32_t off_q, off_stage, off_p, off_bar, off_misc, stage_bytes, off_raw, raw_stage;
 };
 
 struct Bars {
@@ -72,6 +74,9 @@ struct Bars {
   __device__ uint32_t q_full() const { return at(2 * NC + 10); }
   __device__ uint32_t q_empty() const { return at(2 * NC + 11); }
   __device__ uint32_t mma_done() const { return at(2 * NC + 12); }
+  __device__ uint32_t raw_full(int s) const { return at(2 * NC + 13 + s); }
+  __device__ uint32_t raw_empty(int s) const { return at(2 * NC + 13 + NRAW + s); }
+  int NRAW;
 };
 constexpr int kFixedBars = 13;
 
@@ -117,24 +122,29 @@ __device__ __forceinline__ MlaLoc chunk_loc(const ChunkArgs& a, int b, int t) {
   return mla_loc(a.cache, b, t, a.err);
 }
 
-template <bool PAGED>
+// QB: code width of a quantised latent cache (4 or 2), whose rows warps 2-3 dequantise into
+// the stage's latent boxes; 0 for a bf16 latent loaded by TMA.
+template <int QB, bool PAGED>
 __global__ void __launch_bounds__(256, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_kr,
                 const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ ChunkArgs a) {
+  constexpr bool QUANT = QB != 0;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (sbase_u32 - smem_u32(smem_raw));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int dc = a.d_c, R = a.R;
   const int n_cbox = dc / 64, n_kbox = R / 64;
-  Bars bars{sbase_u32 + a.off_bar, a.NC};
+  Bars bars{sbase_u32 + a.off_bar, a.NC, a.NRAW};
   Misc* misc = reinterpret_cast<Misc*>(sbase + a.off_misc);
   volatile int* abort_flag = &misc->abort_flag;
   const uint64_t lim = a.wait_ns;
 
   if (threadIdx.x == 0) {
     misc->abort_flag = 0;
-    for (int s = 0; s < a.NC; ++s) { mbar_init(bars.c_full(s), 1); mbar_init(bars.c_empty(s), 1); }
+    // a stage is full after its TMA bytes (and, for a quantised cache, both dequantising warps)
+    for (int s = 0; s < a.NC; ++s) { mbar_init(bars.c_full(s), QUANT ? 3 : 1); mbar_init(bars.c_empty(s), 1); }
+    for (int s = 0; s < a.NRAW; ++s) { mbar_init(bars.raw_full(s), 1); mbar_init(bars.raw_empty(s), 2); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars.s_full(i), 1);
       mbar_init(bars.s_empty(i), 4);
@@ -186,17 +196,29 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
         }
         ++q_loads;
       }
-      const int cs = n % a.NC;
+      const int cs = n % a.NC, rs = QUANT ? n % a.NRAW : 0;
       if (n >= a.NC) ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag, lim));
+      if (ok && QUANT && n >= a.NRAW)
+        ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_empty(rs), ((n / a.NRAW) - 1) & 1, abort_flag, lim));
       if (!ok) break;
       if (lane == 0) {
         const MlaLoc lc = chunk_loc<PAGED>(a, it.v / a.nqb, it.t);   // a 64-token tile lies in one block
         const int row = lc.pb * lc.cap + lc.pt;
         const uint32_t st = sbase_u32 + a.off_stage + cs * a.stage_bytes;
-        mbar_expect_tx(bars.c_full(cs), (uint32_t)(n_cbox + n_kbox) * kTBox);
-        for (int kb = 0; kb < n_cbox; ++kb) tma_load_2d(st + kb * kTBox, &tm_c, bars.c_full(cs), kb * 64, row);
+        mbar_expect_tx(bars.c_full(cs), (uint32_t)((QUANT ? 0 : n_cbox) + n_kbox) * kTBox);
+        if (!QUANT)
+          for (int kb = 0; kb < n_cbox; ++kb) tma_load_2d(st + kb * kTBox, &tm_c, bars.c_full(cs), kb * 64, row);
         for (int kb = 0; kb < n_kbox; ++kb)
           tma_load_2d(st + (n_cbox + kb) * kTBox, &tm_kr, bars.c_full(cs), kb * 64, row);
+        if (QUANT) {   // codes (one box of 64 rows) and the rows' scales into the raw ring
+          const int nvalid = min(kCT, it.t1 - it.t);
+          const uint32_t codes = (uint32_t)kCT * a.code_row;
+          const uint32_t sbytes = (uint32_t)((((nvalid + 1) & ~1) * (dc / 16) + 15) & ~15);
+          const uint32_t rb = sbase_u32 + a.off_raw + rs * a.raw_stage;
+          mbar_expect_tx(bars.raw_full(rs), codes + sbytes);
+          tma_load_2d(rb, &tm_c, bars.raw_full(rs), 0, row);
+          bulk_load(rb + codes, a.scales + (size_t)row * (dc / 32), sbytes, bars.raw_full(rs));
+        }
       }
       last = n;
       if (it.last_of_piece()) ++u;
@@ -209,6 +231,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
       for (int s = 0; s < a.NC; ++s) {
         const int k = last - ((last - s) % a.NC + a.NC) % a.NC;
         if (last >= 0 && k >= 0) mbar_wait(bars.c_full(s), (k / a.NC) & 1, &never, lim);
+      }
+      for (int s = 0; QUANT && s < a.NRAW; ++s) {
+        const int k = last - ((last - s) % a.NRAW + a.NRAW) % a.NRAW;
+        if (last >= 0 && k >= 0) mbar_wait(bars.raw_full(s), (k / a.NRAW) & 1, &never, lim);
       }
     }
   } else if (warp == 1) {
@@ -289,6 +315,75 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
       tc_commit(bars.mma_done());
       volatile int never = 0;
       mbar_wait(bars.mma_done(), 0, &never, lim);
+    }
+  } else if (QUANT && warp >= 2 && warp < 4) {
+    // ============================================================ dequantisation
+    // thread = token row of the tile: codes * scale -> bf16 into the stage's swizzled latent
+    // boxes; rows past the unit's last token are zeroed (MMA2 multiplies them by P = 0)
+    const int tok = threadIdx.x - 64;   // 0..63
+    TileIter it;
+    it.init(&a.sched, w);
+    int n = 0;
+    bool ok = true;
+    while (ok && it.valid()) {
+      const int rs = n % a.NRAW, cs = n % a.NC;
+      ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_full(rs), (n / a.NRAW) & 1, abort_flag, lim));
+      if (ok && n >= a.NC)
+        ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag, lim));
+      if (!ok) break;
+      const int nvalid = min(kCT, it.t1 - it.t);
+      const uint8_t* raw = sbase + a.off_raw + rs * a.raw_stage;
+      uint8_t* C = sbase + a.off_stage + cs * a.stage_bytes + tok * 128;
+      if (tok < nvalid) {
+        const __half* sc = reinterpret_cast<const __half*>(raw + kCT * a.code_row) + tok * (dc / 32);
+        const uint8_t* codes = raw + tok * a.code_row;
+        for (int half = 0; half < dc / 64; ++half) {
+          const float s0 = __half2float(sc[half * 2]), s1 = __half2float(sc[half * 2 + 1]);
+          if (QB == 4) {   // two's-complement nibbles, element 2i in the low nibble of byte i
+            const uint4 c0 = *reinterpret_cast<const uint4*>(codes + half * 32);
+            const uint4 c1 = *reinterpret_cast<const uint4*>(codes + half * 32 + 16);
+            const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              const float sv = ch < 4 ? s0 : s1;
+              uint32_t o[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t byte = (words[ch] >> (8 * j)) & 0xFFu;
+                o[j] = pack_bf16x2((float)nib_to_int(byte & 15u) * sv, (float)nib_to_int(byte >> 4) * sv);
+              }
+              *reinterpret_cast<uint4*>(C + half * kTBox + ((ch ^ (tok & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          } else {         // two's-complement 2-bit fields, element 4i+k in bits 2k..2k+1 of byte i
+            const uint4 c0 = *reinterpret_cast<const uint4*>(codes + half * 16);
+            const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              const uint32_t bits = (words[ch >> 1] >> (16 * (ch & 1))) & 0xFFFFu;
+              const float sv = ch < 4 ? s0 : s1;
+              uint32_t o[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int f0 = (int)((bits >> (4 * j)) & 3u), f1 = (int)((bits >> (4 * j + 2)) & 3u);
+                o[j] = pack_bf16x2((float)(f0 >= 2 ? f0 - 4 : f0) * sv, (float)(f1 >= 2 ? f1 - 4 : f1) * sv);
+              }
+              *reinterpret_cast<uint4*>(C + half * kTBox + ((ch ^ (tok & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
+        }
+      } else {
+        for (int half = 0; half < dc / 64; ++half)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(C + half * kTBox + ch * 16) = make_uint4(0, 0, 0, 0);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bars.raw_empty(rs));
+        mbar_arrive(bars.c_full(cs));
+      }
+      it.next();
+      ++n;
     }
   } else if (warp >= 4) {
     // ============================================================ softmax + epilogue
@@ -385,6 +480,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
         l += p0 + p1;
         pk[t / 2] = pack_bf16x2(p0, p1);
       }
+      if (!QUANT && it.t1 - it.t < kCT) {
+        // latent rows past the unit's last token (stale cache rows, possibly not finite):
+        // zeroed before MMA2 multiplies them by P = 0
+        const int nvalid = it.t1 - it.t;
+        uint8_t* C = sbase + a.off_stage + cs * a.stage_bytes;
+        const int nchunk = (kCT - nvalid) * 8 * n_cbox;   // 16-byte chunks
+        for (int i = r; i < nchunk; i += kRows) {
+          const int box = i / ((kCT - nvalid) * 8), rem = i % ((kCT - nvalid) * 8);
+          *reinterpret_cast<uint4*>(C + box * kTBox + (nvalid + rem / 8) * 128 + (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
+        }
+      }
       if (n >= 2) {
         ok = wwait(bars.p_empty(pb), ((n >> 1) - 1) & 1);
         if (!ok) break;
@@ -473,24 +579,30 @@ static bool map_bf16_sw128(CUtensorMap* m, const void* base, uint64_t cols, uint
 }
 
 struct ChunkLayoutSmem {
-  int NC;
-  uint32_t off_q, off_stage, off_p, off_bar, off_misc, stage_bytes, total;
+  int NC, NRAW;
+  uint32_t off_q, off_stage, off_p, off_raw, off_bar, off_misc, stage_bytes, raw_stage, total;
 };
 
-static ChunkLayoutSmem chunk_smem(int dc, int R) {
+static ChunkLayoutSmem chunk_smem(int dc, int R, int qbits) {
   const uint32_t budget = 232448 - 1024;
   ChunkLayoutSmem L{};
   L.stage_bytes = (uint32_t)(dc / 64 + R / 64) * kTBox;
+  L.raw_stage = qbits ? (((uint32_t)kCT * (dc * qbits / 8) + (uint32_t)kCT * (dc / 16)) + 127) & ~127u : 0;
+  const int nraw = qbits ? 3 : 0;
   const uint32_t q_bytes = (uint32_t)(dc / 64) * kQBox;
-  auto size = [&](int nc) { return q_bytes + nc * L.stage_bytes + 2 * kPBytes + 8 * (2 * nc + kFixedBars) + 256; };
+  auto size = [&](int nc) {
+    return q_bytes + nc * L.stage_bytes + 2 * kPBytes + nraw * L.raw_stage + 8 * (2 * nc + 2 * nraw + kFixedBars) + 256;
+  };
   int nc = 2;
   while (nc < 6 && size(nc + 1) <= budget) ++nc;
   L.NC = nc;
+  L.NRAW = nraw;
   uint32_t o = 0;
   L.off_q = o; o += q_bytes;
   L.off_stage = o; o += nc * L.stage_bytes;
   L.off_p = o; o += 2 * kPBytes;
-  L.off_bar = o; o += 8 * (2 * nc + kFixedBars);
+  L.off_raw = o; o += nraw * L.raw_stage;
+  L.off_bar = o; o += 8 * (2 * nc + 2 * nraw + kFixedBars);
   o = (o + 15) & ~15u;
   L.off_misc = o; o += sizeof(Misc);
   L.total = o + 1024;
@@ -500,13 +612,24 @@ static ChunkLayoutSmem chunk_smem(int dc, int R) {
 }  // namespace chunk
 }  // namespace mla
 
-// Shapes the chunk kernel covers: bf16 latent (no quantised cache), 32 query heads, d_c in
-// {64, 128, 256}, r = 4 kept pairs per KV head.
+// Shapes the chunk kernel covers: bf16, 32 query heads, d_c in {64, 128, 256}, r = 4 kept
+// pairs per KV head, KV heads a multiple of 8; a bf16, int4 or 2-bit latent cache without
+// the residual window (the window depends on each query's own length, so a tile's latent
+// rows would differ between the queries that share it).
 bool mla_chunk_capable(const mla_plan& p) {
   const mla_config_t& cfg = p.cfg;
-  if (cfg.dtype != MLA_BF16 || cfg.cache_kind != MLA_CACHE_SAME || cfg.n_heads != mla::chunk::kHeads) return false;
+  if (cfg.dtype != MLA_BF16 || cfg.n_heads != mla::chunk::kHeads) return false;
+  if (cfg.cache_kind == MLA_CACHE_INT4_G32_R128) return false;
   if (cfg.d_c % 64 != 0 || cfg.d_c > 256 || 2 * cfg.r_pairs != 8 || p.R % 64 != 0) return false;
-  return mla::chunk::chunk_smem(cfg.d_c, p.R).total <= 232448;
+  const int qbits = mla_kind_quant(cfg.cache_kind) ? mla_quant_bits(cfg.cache_kind) : 0;
+  return mla::chunk::chunk_smem(cfg.d_c, p.R, qbits).total <= 232448;
+}
+
+// The scale rows of a quantised cache are fetched with 1-D bulk copies, which need an even
+// capacity.
+bool mla_chunk_supported(const mla_plan& p, const mla_cache_t& c) {
+  if (!mla_chunk_capable(p)) return false;
+  return !(mla_kind_quant(p.cfg.cache_kind) && c.T_cap % 2 != 0);
 }
 
 cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B, int Q,
@@ -515,21 +638,38 @@ cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const i
   using namespace mla::chunk;
   const mla_config_t& cfg = p.cfg;
   const int dc = cfg.d_c, R = p.R;
+  const int qbits = mla_kind_quant(cfg.cache_kind) ? mla_quant_bits(cfg.cache_kind) : 0;
+  const uint32_t code_row = (uint32_t)(dc * qbits / 8);
   const uint64_t rows = mla_cache_rows(c);
   CUtensorMap tm_c, tm_kr, tm_q;
-  bool ok = map_bf16_sw128(&tm_c, c.c_kv, dc, rows, kCT) && map_bf16_sw128(&tm_kr, c.k_rope, R, rows, kCT) &&
-            map_bf16_sw128(&tm_q, qlat, dc, (uint64_t)B * Q * kHeads, kRows);
+  bool ok = map_bf16_sw128(&tm_kr, c.k_rope, R, rows, kCT) && map_bf16_sw128(&tm_q, qlat, dc, (uint64_t)B * Q * kHeads, kRows);
+  if (qbits) {   // code rows, one 64-row box per tile, no swizzle
+    EncodeTiledFn fn = encode_fn();
+    cuuint64_t gdim[2] = {code_row, rows};
+    cuuint64_t gstride[1] = {code_row};
+    cuuint32_t box[2] = {code_row, (cuuint32_t)kCT};
+    cuuint32_t es[2] = {1, 1};
+    ok = ok && fn && fn(&tm_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, c.c_kv, gdim, gstride, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  } else {
+    ok = ok && map_bf16_sw128(&tm_c, c.c_kv, dc, rows, kCT);
+  }
   if (!ok) return cudaErrorInvalidValue;
-  const ChunkLayoutSmem L = chunk_smem(dc, R);
+  const ChunkLayoutSmem L = chunk_smem(dc, R, qbits);
   ChunkArgs a;
   a.q_chunk = Q; a.nqb = (Q + kQB - 1) / kQB; a.d_c = dc; a.R = R; a.P = P; a.T_cap = c.T_cap;
+  a.scales = (const __half*)c.c_scales; a.code_row = code_row;
   a.sched = sched; a.seq_lens = seq_lens; a.qrope = qrope; a.opart = opart; a.mlpart = mlpart;
   a.cache = c; a.err = p.err;
   a.wait_ns = (uint64_t)p.opt_wait_us * 1000u;
-  a.NC = L.NC;
+  a.NC = L.NC; a.NRAW = L.NRAW;
   a.off_q = L.off_q; a.off_stage = L.off_stage; a.off_p = L.off_p; a.off_bar = L.off_bar; a.off_misc = L.off_misc;
-  a.stage_bytes = L.stage_bytes;
-  auto kern = c.block_table ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;
+  a.stage_bytes = L.stage_bytes; a.off_raw = L.off_raw; a.raw_stage = L.raw_stage;
+  const bool paged = c.block_table != nullptr;
+  auto kern = qbits == 4 ? (paged ? chunk_tc_kernel<4, true> : chunk_tc_kernel<4, false>)
+              : qbits == 2 ? (paged ? chunk_tc_kernel<2, true> : chunk_tc_kernel<2, false>)
+                           : (paged ? chunk_tc_kernel<0, true> : chunk_tc_kernel<0, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
   if ((e = mla_profile_event(p, kProfAttention, false, s)) != cudaSuccess) return e;

@@ -345,7 +345,7 @@ mla_status_t mla_decode_chunk(const mla_plan_t* plan, const mla_cache_t* cache, 
   if (B > cache->B || (long long)Q > cache->T_cap) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace) || ((uintptr_t)seq_lens & 3))
     return MLA_ERR_ALIGNMENT;
-  if (!mla_chunk_capable(*plan) || plan->opt_kernel == 1) return MLA_ERR_UNSUPPORTED;
+  if (!mla_chunk_supported(*plan, *cache) || plan->opt_kernel == 1) return MLA_ERR_UNSUPPORTED;
   DecodeLayout L = mla_chunk_layout(*plan, B, Q);
   if (ws_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
   return cuda_status(mla_launch_chunk(*plan, *cache, seq_lens, q, B, Q, out, workspace, L, (cudaStream_t)stream));

@@ -157,6 +157,7 @@ Sched mla_sched_view(const DecodeLayout& L, void* ws, int B);
 // Many queries per sequence: workspace layout, the chunk kernel's shape limits and launches.
 DecodeLayout mla_chunk_layout(const mla_plan& p, int B, int Q);
 bool mla_chunk_capable(const mla_plan& p);
+bool mla_chunk_supported(const mla_plan& p, const mla_cache_t& c);
 cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B, int Q,
                                 const Sched& sched, const void* qlat, const float* qrope, float* opart,
                                 float* mlpart, int P, int G, cudaStream_t s);

@@ -5,7 +5,8 @@ rotated there and attends over tokens [0, L - Q + i].  The oracle decodes every 
 its own (float64, the unabsorbed definition) over its causal prefix; the chunk kernel's
 outputs must match within the parity tolerances.  Chunk sizes cover a partial query block
 (Q = 2), several blocks whose positions straddle 64-token tiles (Q = 12) and a long chunk
-(Q = 64); lengths are not tile multiples; contiguous and paged caches.
+(Q = 64); lengths are not tile multiples; contiguous and paged caches; bf16, int4 and
+2-bit latents.
 """
 
 import numpy as np
@@ -19,7 +20,9 @@ from workloads import PARITY_WORKLOADS, generate as gen
 pytestmark = pytest.mark.gpu
 
 WLS = [PARITY_WORKLOADS[2].with_(name="llama_dc256_chunk", fixed_lens=(1000, 333, 130)),
-       PARITY_WORKLOADS[3].with_(name="llama_dc64_chunk", batch=3, fixed_lens=(2500, 129, 77))]
+       PARITY_WORKLOADS[3].with_(name="llama_dc64_chunk", batch=3, fixed_lens=(2500, 129, 77)),
+       PARITY_WORKLOADS[4].with_(name="llama_int4_chunk", fixed_lens=(700, 200, 77)),
+       PARITY_WORKLOADS[7].with_(name="llama_int2_chunk", fixed_lens=(700, 130, 65))]
 _CASES = {}
 
 
