@@ -555,8 +555,9 @@ void absorb_setup(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_le
   aa->n_kv = cfg.n_kv_heads; aa->dh = cfg.head_dim; aa->r = cfg.r_pairs; aa->d_c = cfg.d_c;
   aa->W_ukF = p.W_ukF;
   aa->rope_pair = p.rope_pair; aa->theta = p.theta;
+  // f32 absorbed queries for the CUDA-core kernel, bf16 for the tensor-core kernels
   aa->qlat = L.kernel == 1 ? (float*)(base + L.off_qlat) : nullptr;
-  aa->qlat16 = L.kernel == 2 ? (__nv_bfloat16*)(base + L.off_qlat) : nullptr;
+  aa->qlat16 = L.kernel != 1 ? (__nv_bfloat16*)(base + L.off_qlat) : nullptr;
   aa->qrope = (float*)(base + L.off_qrope);
   aa->sched = mla_sched_view(L, ws, B); aa->tile = L.tile; aa->G = L.G; aa->err = p.err;
   aa->sm_scale = cfg.softmax_scale > 0.0f ? cfg.softmax_scale : (float)(1.0 / sqrt((double)cfg.head_dim));

@@ -120,7 +120,7 @@ inline cudaError_t mla_profile_event(const mla_plan& p, MlaProfKernel k, bool af
 
 // Decode workspace layout (byte offsets from the workspace base).
 struct DecodeLayout {
-  int kernel = 1;          // 1 CUDA-core, 2 tcgen05
+  int kernel = 1;          // 1 CUDA-core, 2 tcgen05 decode, 3 tcgen05 query chunks
   int tile = 32;           // tokens per schedule tile
   int G = 0;               // workers (CTAs of the split-K kernel)
   int P = 0;               // max pieces = B + G
