@@ -134,7 +134,9 @@ typedef struct mla_plan mla_plan_t;   /* opaque, created by mla_plan_create */
 
 /* Options for mla_plan_set_option. */
 enum {
-  MLA_OPT_DECODE_KERNEL = 1,  /* 0 auto, 1 CUDA-core split-K kernel, 2 tcgen05 kernel */
+  MLA_OPT_DECODE_KERNEL = 1,  /* 0 auto, 1 CUDA-core split-K kernel, 2 tcgen05 kernel with a
+                                 token per softmax thread, 3 tcgen05 kernel with a head per
+                                 softmax thread (the query-chunk kernel's form, one query) */
   MLA_OPT_DECODE_SPLITS = 2,  /* 0 auto (SM count based); n > 0: split the context
                                  tiles into n contiguous worker ranges */
   MLA_OPT_PROFILE_EVENTS = 3, /* value: address of a host array of two cudaEvent_t; each

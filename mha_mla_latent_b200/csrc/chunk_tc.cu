@@ -34,13 +34,19 @@ namespace chunk {
 using namespace sm100;
 
 constexpr int kCT = 64;              // tokens per tile
-constexpr int kRows = 128;           // rows per unit: 4 queries x 32 heads
-constexpr int kQB = 4;               // queries per unit
 constexpr int kHeads = 32;
-constexpr uint32_t kQBox = 16384;    // Q_lat box: 128 rows x 128 B
 constexpr uint32_t kTBox = 8192;     // cache box: 64 rows x 128 B
-constexpr uint32_t kPBytes = 16384;  // P: 128 rows x 64 tokens bf16
 constexpr float kTau = 8.0f;         // lazy-rescale threshold, log2 units
+// Rows per unit: 128 = 4 queries x 32 heads (many queries per sequence, MMA M = 128), or
+// 32 = the 32 heads of one query (decode, MMA M = 64: rows 32..63 of the A operands read
+// the next 4 KB of shared memory, whose values only reach output rows nobody reads).
+template <int ROWS> struct Geo {
+  static constexpr int M = ROWS == 32 ? 64 : 128;   // MMA M
+  static constexpr int QPER = ROWS / 32;             // queries per unit
+  static constexpr int SW = ROWS == 32 ? 2 : 4;      // softmax warps (TMEM lane quarters used)
+  static constexpr uint32_t QBOX = ROWS * 128u;      // Q_lat box: ROWS rows x 128 B
+  static constexpr uint32_t PBYTES = ROWS * 128u;    // P buffer: ROWS rows x 64 tokens bf16
+};
 constexpr uint32_t kSCol = 0, kOCol = 128;
 
 struct ChunkArgs {
@@ -122,13 +128,18 @@ __device__ __forceinline__ MlaLoc chunk_loc(const ChunkArgs& a, int b, int t) {
   return mla_loc(a.cache, b, t, a.err);
 }
 
-// QB: code width of a quantised latent cache (4 or 2), whose rows warps 2-3 dequantise into
-// the stage's latent boxes; 0 for a bf16 latent loaded by TMA.
-template <int QB, bool PAGED>
+// ROWS: rows per unit (see Geo); QB: code width of a quantised latent cache (4 or 2),
+// whose rows warps 2-3 dequantise into the stage's latent boxes, 0 for a bf16 latent loaded
+// by TMA; RESID: the int4 cache's residual window (decode only: the window follows the one
+// query's length); PAGED: cache addressed through a block table.
+template <int ROWS, int QB, bool RESID, bool PAGED>
 __global__ void __launch_bounds__(256, 1)
-chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_kr,
-                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ ChunkArgs a) {
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_kr,
+               const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ ChunkArgs a) {
   constexpr bool QUANT = QB != 0;
+  using GG = Geo<ROWS>;
+  constexpr int kRows = ROWS, kQB = GG::QPER, kSW = GG::SW;
+  constexpr uint32_t kQBox = GG::QBOX, kPBytes = GG::PBYTES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (sbase_u32 - smem_u32(smem_raw));
@@ -147,12 +158,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
     for (int s = 0; s < a.NRAW; ++s) { mbar_init(bars.raw_full(s), 1); mbar_init(bars.raw_empty(s), 2); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars.s_full(i), 1);
-      mbar_init(bars.s_empty(i), 4);
-      mbar_init(bars.p_full(i), 4);
+      mbar_init(bars.s_empty(i), kSW);
+      mbar_init(bars.p_full(i), kSW);
       mbar_init(bars.p_empty(i), 1);
     }
     mbar_init(bars.o_full(), 1);
-    mbar_init(bars.o_empty(), 4);
+    mbar_init(bars.o_empty(), kSW);
     mbar_init(bars.q_full(), 1);
     mbar_init(bars.q_empty(), 1);
     mbar_init(bars.mma_done(), 1);
@@ -240,8 +251,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
   } else if (warp == 1) {
     // ============================================================ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc1 = idesc_bf16_f32(kRows, kCT, false, false);   // S[row][t]
-      const uint32_t idesc2 = idesc_bf16_f32(kRows, dc, false, true);     // O[row][d]
+      const uint32_t idesc1 = idesc_bf16_f32(GG::M, kCT, false, false);   // S[row][t]
+      const uint32_t idesc2 = idesc_bf16_f32(GG::M, dc, false, true);     // O[row][d]
       TileIter it;
       it.init(&a.sched, w);
       int n = 0, u = 0;
@@ -325,8 +336,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
     it.init(&a.sched, w);
     int n = 0;
     bool ok = true;
+    int lo_v = -1, lo = INT_MAX;   // residual window (decode): tokens from lo on may sit in the ring
     while (ok && it.valid()) {
       const int rs = n % a.NRAW, cs = n % a.NC;
+      if (RESID && it.v != lo_v) {   // once per sequence, ahead of the stage wait
+        lo_v = it.v;
+        lo = __ldg(a.seq_lens + it.v) - MLA_RESID_WINDOW;
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_full(rs), (n / a.NRAW) & 1, abort_flag, lim));
       if (ok && n >= a.NC)
         ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag, lim));
@@ -334,7 +350,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
       const int nvalid = min(kCT, it.t1 - it.t);
       const uint8_t* raw = sbase + a.off_raw + rs * a.raw_stage;
       uint8_t* C = sbase + a.off_stage + cs * a.stage_bytes + tok * 128;
-      if (tok < nvalid) {
+      const int tp = it.t + tok;
+      const size_t rslot = (size_t)it.v * MLA_RESID_WINDOW + (tp & (MLA_RESID_WINDOW - 1));
+      if (RESID && tok < nvalid && tp >= lo && __ldg(a.cache.resid_pos + rslot) == tp) {
+        // one of the window's tokens: its unquantised row from the ring
+        const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.cache.c_resid) +
+                                                          rslot * dc);
+        for (int half = 0; half < dc / 64; ++half)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4*>(C + half * kTBox + ((ch ^ (tok & 7)) << 4)) = __ldg(src + half * 8 + ch);
+      } else if (tok < nvalid) {
         const __half* sc = reinterpret_cast<const __half*>(raw + kCT * a.code_row) + tok * (dc / 32);
         const uint8_t* codes = raw + tok * a.code_row;
         for (int half = 0; half < dc / 64; ++half) {
@@ -385,12 +411,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
       it.next();
       ++n;
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 4 + kSW) {
     // ============================================================ softmax + epilogue
-    const int q = warp - 4;                  // TMEM lane quarter = query j of the unit
-    const int r = 32 * q + lane;             // this thread's row: query q, head lane
+    // M = 128: warp 4 + q reads TMEM lane quarter q = rows 32q .. 32q+31 (query q of the
+    // unit).  M = 64: rows 16q .. 16q+15 sit in lanes 0..15 of quarter q; lanes 16..31 of
+    // the warp shadow them (they run the same code for the warp-wide instructions and
+    // store nothing).
+    const int q = warp - 4;
+    const bool live = ROWS == 128 || lane < 16;
+    const int r = ROWS == 128 ? 32 * q + lane : 16 * q + (lane & 15);   // this thread's row
+    const int hd = r % kHeads;               // its head; its query is r / 32 of the unit
     const int n_kv = R / 8;
-    const int g = lane / (kHeads / n_kv);    // KV head of this row's head
+    const int g = hd / (kHeads / n_kv);      // KV head of this row's head
     TileIter it;
     it.init(&a.sched, w);
     int n = 0, u = 0;
@@ -405,13 +437,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
       const bool first = it.first_of_piece();
       const int pc = it.pc;
       if (first) {
-        const int bseq = it.v / a.nqb, i = (it.v % a.nqb) * kQB + q;
+        const int bseq = it.v / a.nqb, i = (it.v % a.nqb) * kQB + r / kHeads;
         p_row = -1;
 #pragma unroll
         for (int j = 0; j < 8; ++j) qr[j] = 0.f;
-        if (i < a.q_chunk) {
+        if (live && i < a.q_chunk) {
           p_row = __ldg(a.seq_lens + bseq) - a.q_chunk + i;
-          const float4* src = reinterpret_cast<const float4*>(a.qrope + (((size_t)bseq * a.q_chunk + i) * kHeads + lane) * 8);
+          const float4* src = reinterpret_cast<const float4*>(a.qrope + (((size_t)bseq * a.q_chunk + i) * kHeads + hd) * 8);
           const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
           qr[0] = x0.x; qr[1] = x0.y; qr[2] = x0.z; qr[3] = x0.w;
           qr[4] = x1.x; qr[5] = x1.y; qr[6] = x1.z; qr[7] = x1.w;
@@ -486,7 +518,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
         const int nvalid = it.t1 - it.t;
         uint8_t* C = sbase + a.off_stage + cs * a.stage_bytes;
         const int nchunk = (kCT - nvalid) * 8 * n_cbox;   // 16-byte chunks
-        for (int i = r; i < nchunk; i += kRows) {
+        for (int i = r; live && i < nchunk; i += kRows) {
           const int box = i / ((kCT - nvalid) * 8), rem = i % ((kCT - nvalid) * 8);
           *reinterpret_cast<uint4*>(C + box * kTBox + (nvalid + rem / 8) * 128 + (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
         }
@@ -495,7 +527,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
         ok = wwait(bars.p_empty(pb), ((n >> 1) - 1) & 1);
         if (!ok) break;
       }
-      {  // P row r: 64 tokens = 128 B, 16-byte chunk c at (c ^ (r % 8))
+      if (live) {  // P row r: 64 tokens = 128 B, 16-byte chunk c at (c ^ (r % 8))
         uint8_t* prow = sbase + a.off_p + pb * kPBytes + r * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
@@ -509,8 +541,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
 
       if (it.last_of_piece()) {
         // ---------------- piece epilogue: this row's partial (m, l, O)
-        a.mlpart[((size_t)r * a.P + pc) * 2] = m;
-        a.mlpart[((size_t)r * a.P + pc) * 2 + 1] = l;
+        if (live) {
+          a.mlpart[((size_t)r * a.P + pc) * 2] = m;
+          a.mlpart[((size_t)r * a.P + pc) * 2 + 1] = l;
+        }
         ok = wwait(bars.o_full(), u & 1);
         if (!ok) break;
         tc_fence_after();
@@ -520,6 +554,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant_
 #pragma unroll
           for (int k = 0; k < 2; ++k) tmem_ld16(taddr(tmem, 32 * q, kOCol + c0 + 16 * k), o[k]);
           tmem_wait_ld();
+          if (!live) continue;
 #pragma unroll
           for (int k = 0; k < 2; ++k)
 #pragma unroll
@@ -583,15 +618,19 @@ struct ChunkLayoutSmem {
   uint32_t off_q, off_stage, off_p, off_raw, off_bar, off_misc, stage_bytes, raw_stage, total;
 };
 
-static ChunkLayoutSmem chunk_smem(int dc, int R, int qbits) {
+// Shared memory: [Q_lat boxes][P buffers][stages][raw ring][barriers][misc].  With M = 64
+// the A operands' rows 32..63 read the 4 KB after each 32-row box: Q's last box runs into
+// P0, P1 into stage 0, all inside the allocation.
+static ChunkLayoutSmem chunk_smem(int dc, int R, int qbits, int rows) {
   const uint32_t budget = 232448 - 1024;
   ChunkLayoutSmem L{};
   L.stage_bytes = (uint32_t)(dc / 64 + R / 64) * kTBox;
   L.raw_stage = qbits ? (((uint32_t)kCT * (dc * qbits / 8) + (uint32_t)kCT * (dc / 16)) + 127) & ~127u : 0;
   const int nraw = qbits ? 3 : 0;
-  const uint32_t q_bytes = (uint32_t)(dc / 64) * kQBox;
+  const uint32_t box = (uint32_t)rows * 128u;
+  const uint32_t q_bytes = (uint32_t)(dc / 64) * box;
   auto size = [&](int nc) {
-    return q_bytes + nc * L.stage_bytes + 2 * kPBytes + nraw * L.raw_stage + 8 * (2 * nc + 2 * nraw + kFixedBars) + 256;
+    return q_bytes + nc * L.stage_bytes + 2 * box + nraw * L.raw_stage + 8 * (2 * nc + 2 * nraw + kFixedBars) + 256;
   };
   int nc = 2;
   while (nc < 6 && size(nc + 1) <= budget) ++nc;
@@ -599,8 +638,8 @@ static ChunkLayoutSmem chunk_smem(int dc, int R, int qbits) {
   L.NRAW = nraw;
   uint32_t o = 0;
   L.off_q = o; o += q_bytes;
+  L.off_p = o; o += 2 * box;
   L.off_stage = o; o += nc * L.stage_bytes;
-  L.off_p = o; o += 2 * kPBytes;
   L.off_raw = o; o += nraw * L.raw_stage;
   L.off_bar = o; o += 8 * (2 * nc + 2 * nraw + kFixedBars);
   o = (o + 15) & ~15u;
@@ -622,7 +661,17 @@ bool mla_chunk_capable(const mla_plan& p) {
   if (cfg.cache_kind == MLA_CACHE_INT4_G32_R128) return false;
   if (cfg.d_c % 64 != 0 || cfg.d_c > 256 || 2 * cfg.r_pairs != 8 || p.R % 64 != 0) return false;
   const int qbits = mla_kind_quant(cfg.cache_kind) ? mla_quant_bits(cfg.cache_kind) : 0;
-  return mla::chunk::chunk_smem(cfg.d_c, p.R, qbits).total <= 232448;
+  return mla::chunk::chunk_smem(cfg.d_c, p.R, qbits, 128).total <= 232448;
+}
+
+// The decode form of the same kernel (32 rows per sequence, MMA M = 64): the chunk kernel's
+// shapes, with the residual window too (one query per sequence).
+bool mla_decode_t_capable(const mla_plan& p) {
+  const mla_config_t& cfg = p.cfg;
+  if (cfg.dtype != MLA_BF16 || cfg.n_heads != mla::chunk::kHeads) return false;
+  if (cfg.d_c % 64 != 0 || cfg.d_c > 256 || 2 * cfg.r_pairs != 8 || p.R % 64 != 0) return false;
+  const int qbits = mla_kind_quant(cfg.cache_kind) ? mla_quant_bits(cfg.cache_kind) : 0;
+  return mla::chunk::chunk_smem(cfg.d_c, p.R, qbits, 32).total <= 232448;
 }
 
 // The scale rows of a quantised cache are fetched with 1-D bulk copies, which need an even
@@ -634,18 +683,19 @@ bool mla_chunk_supported(const mla_plan& p, const mla_cache_t& c) {
 
 cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B, int Q,
                                 const Sched& sched, const void* qlat, const float* qrope, float* opart,
-                                float* mlpart, int P, int G, cudaStream_t s) {
+                                float* mlpart, int P, int G, cudaStream_t s, int rows) {
   using namespace mla::chunk;
   const mla_config_t& cfg = p.cfg;
   const int dc = cfg.d_c, R = p.R;
   const int qbits = mla_kind_quant(cfg.cache_kind) ? mla_quant_bits(cfg.cache_kind) : 0;
   const uint32_t code_row = (uint32_t)(dc * qbits / 8);
-  const uint64_t rows = mla_cache_rows(c);
+  const uint64_t crows = mla_cache_rows(c);
   CUtensorMap tm_c, tm_kr, tm_q;
-  bool ok = map_bf16_sw128(&tm_kr, c.k_rope, R, rows, kCT) && map_bf16_sw128(&tm_q, qlat, dc, (uint64_t)B * Q * kHeads, kRows);
+  bool ok = map_bf16_sw128(&tm_kr, c.k_rope, R, crows, kCT) &&
+            map_bf16_sw128(&tm_q, qlat, dc, (uint64_t)B * Q * kHeads, (uint32_t)rows);
   if (qbits) {   // code rows, one 64-row box per tile, no swizzle
     EncodeTiledFn fn = encode_fn();
-    cuuint64_t gdim[2] = {code_row, rows};
+    cuuint64_t gdim[2] = {code_row, crows};
     cuuint64_t gstride[1] = {code_row};
     cuuint32_t box[2] = {code_row, (cuuint32_t)kCT};
     cuuint32_t es[2] = {1, 1};
@@ -653,12 +703,12 @@ cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const i
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   } else {
-    ok = ok && map_bf16_sw128(&tm_c, c.c_kv, dc, rows, kCT);
+    ok = ok && map_bf16_sw128(&tm_c, c.c_kv, dc, crows, kCT);
   }
   if (!ok) return cudaErrorInvalidValue;
-  const ChunkLayoutSmem L = chunk_smem(dc, R, qbits);
+  const ChunkLayoutSmem L = chunk_smem(dc, R, qbits, rows);
   ChunkArgs a;
-  a.q_chunk = Q; a.nqb = (Q + kQB - 1) / kQB; a.d_c = dc; a.R = R; a.P = P; a.T_cap = c.T_cap;
+  a.q_chunk = Q; a.nqb = (Q + rows / 32 - 1) / (rows / 32); a.d_c = dc; a.R = R; a.P = P; a.T_cap = c.T_cap;
   a.scales = (const __half*)c.c_scales; a.code_row = code_row;
   a.sched = sched; a.seq_lens = seq_lens; a.qrope = qrope; a.opart = opart; a.mlpart = mlpart;
   a.cache = c; a.err = p.err;
@@ -666,10 +716,17 @@ cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const i
   a.NC = L.NC; a.NRAW = L.NRAW;
   a.off_q = L.off_q; a.off_stage = L.off_stage; a.off_p = L.off_p; a.off_bar = L.off_bar; a.off_misc = L.off_misc;
   a.stage_bytes = L.stage_bytes; a.off_raw = L.off_raw; a.raw_stage = L.raw_stage;
-  const bool paged = c.block_table != nullptr;
-  auto kern = qbits == 4 ? (paged ? chunk_tc_kernel<4, true> : chunk_tc_kernel<4, false>)
-              : qbits == 2 ? (paged ? chunk_tc_kernel<2, true> : chunk_tc_kernel<2, false>)
-                           : (paged ? chunk_tc_kernel<0, true> : chunk_tc_kernel<0, false>);
+  const bool paged = c.block_table != nullptr, resid = qbits == 4 && c.c_resid != nullptr;
+  decltype(&attn_tc_kernel<128, 0, false, false>) kern;
+  if (rows == 128)
+    kern = qbits == 4 ? (paged ? attn_tc_kernel<128, 4, false, true> : attn_tc_kernel<128, 4, false, false>)
+           : qbits == 2 ? (paged ? attn_tc_kernel<128, 2, false, true> : attn_tc_kernel<128, 2, false, false>)
+                        : (paged ? attn_tc_kernel<128, 0, false, true> : attn_tc_kernel<128, 0, false, false>);
+  else
+    kern = qbits == 4 ? (resid ? (paged ? attn_tc_kernel<32, 4, true, true> : attn_tc_kernel<32, 4, true, false>)
+                               : (paged ? attn_tc_kernel<32, 4, false, true> : attn_tc_kernel<32, 4, false, false>))
+           : qbits == 2 ? (paged ? attn_tc_kernel<32, 2, false, true> : attn_tc_kernel<32, 2, false, false>)
+                        : (paged ? attn_tc_kernel<32, 0, false, true> : attn_tc_kernel<32, 0, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
   if ((e = mla_profile_event(p, kProfAttention, false, s)) != cudaSuccess) return e;

@@ -633,6 +633,10 @@ cudaError_t launch_attention_combine(const mla_plan& p, const mla_cache_t& c, co
     e = mla_launch_kernel(decode_simt_kernel<T, INT4>, dim3(L.G), dim3(256), smem, s, p.opt_pdl, da);
     if (e != cudaSuccess) return e;
     if ((e = mla_profile_event(p, kProfAttention, true, s)) != cudaSuccess) return e;
+  } else if (L.kernel == 4) {
+    e = mla_launch_chunk_tc(p, c, seq_lens, B, 1, sched, base + L.off_qlat, (const float*)(base + L.off_qrope),
+                            (float*)(base + L.off_opart), (float*)(base + L.off_mlpart), L.P, L.G, s, 32);
+    if (e != cudaSuccess) return e;
   } else {
     e = mla_launch_decode_tc(p, c, seq_lens, B, sched, base + L.off_qlat, (const float*)(base + L.off_qrope),
                              (float*)(base + L.off_opart), (float*)(base + L.off_mlpart), L.P, L.G, s);
@@ -736,7 +740,7 @@ cudaError_t launch_chunk(const mla_plan& p, const mla_cache_t& c, const int32_t*
   char* base = (char*)ws;
   const int units = B * ((Q + kQB - 1) / kQB);
   e = mla_launch_chunk_tc(p, c, seq_lens, B, Q, aa.sched, base + L.off_qlat, (const float*)(base + L.off_qrope),
-                          (float*)(base + L.off_opart), (float*)(base + L.off_mlpart), L.P, L.G, s);
+                          (float*)(base + L.off_opart), (float*)(base + L.off_mlpart), L.P, L.G, s, 128);
   if (e != cudaSuccess) return e;
   return launch_combine<bf16>(p, units, kQB * cfg.n_heads, kQB * cfg.n_kv_heads, Q, kQB, out, ws, L, aa.sched, s);
 }
@@ -749,7 +753,7 @@ DecodeLayout mla_decode_layout(const mla_plan& p, int B, int kernel) {
   const mla_config_t& cfg = p.cfg;
   DecodeLayout L;
   L.kernel = kernel;
-  L.tile = kernel == 2 ? 128 : mla::kSimtTile;
+  L.tile = kernel == 2 ? 128 : kernel == 4 ? 64 : mla::kSimtTile;
   L.G = p.opt_splits > 0 ? p.opt_splits : (kernel == 2 ? p.num_sms : 2 * p.num_sms);
   L.P = B + L.G;
   L.K = cfg.d_c + p.R;

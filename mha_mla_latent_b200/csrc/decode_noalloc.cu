@@ -62,9 +62,8 @@ extern "C" mla_status_t mla_decode_noalloc(const mla_plan_t* plan, const mla_cac
   if (!scratch) return MLA_ERR_CUDA;
 
   int kernel = 1;
-  if (plan->opt_kernel != 1 && mla_tc_kind_ok(cfg) && mla_tc_supported(*plan, *cache)) kernel = 2;
-  if (plan->opt_kernel == 2 && kernel != 2) return MLA_ERR_UNSUPPORTED;
-  if (kernel == 1 && (size_t)cfg.n_heads * cfg.d_c > 8192) return MLA_ERR_UNSUPPORTED;
+  const mla_status_t pk = mla_pick_decode_kernel(*plan, *cache, &kernel);
+  if (pk != MLA_OK) return pk;
   const DecodeLayout L = mla_decode_layout(*plan, B, kernel);
   if (L.total > kNoAllocScratchBytes) return MLA_ERR_WORKSPACE_TOO_SMALL;
   const cudaError_t e =

@@ -75,6 +75,22 @@ void free_plan(mla_plan* p) {
 
 }  // namespace
 
+// The decode kernel a call runs: the tensor-core kernel where the plan, cache and options
+// allow it, else the CUDA-core kernel.  MLA_OK, or the status that refuses the call.
+mla_status_t mla_pick_decode_kernel(const mla_plan& p, const mla_cache_t& c, int* kernel) {
+  *kernel = 1;
+  if (p.opt_kernel == 3) {   // the head-row tensor-core form
+    const bool even = !(mla_kind_quant(p.cfg.cache_kind) && c.T_cap % 2 != 0);
+    if (!mla_decode_t_capable(p) || !even) return MLA_ERR_UNSUPPORTED;
+    *kernel = 4;
+    return MLA_OK;
+  }
+  if (p.opt_kernel != 1 && mla_tc_kind_ok(p.cfg) && mla_tc_supported(p, c)) *kernel = 2;
+  if (p.opt_kernel == 2 && *kernel != 2) return MLA_ERR_UNSUPPORTED;
+  if (*kernel == 1 && (size_t)p.cfg.n_heads * p.cfg.d_c > 8192) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
 extern "C" {
 
 const char* mla_status_string(mla_status_t s) {
@@ -229,7 +245,7 @@ mla_status_t mla_plan_set_option(mla_plan_t* plan, int32_t option, int64_t value
   if (!plan) return MLA_ERR_INVALID_ARG;
   switch (option) {
     case MLA_OPT_DECODE_KERNEL:
-      if (value < 0 || value > 2) return MLA_ERR_INVALID_ARG;
+      if (value < 0 || value > 3) return MLA_ERR_INVALID_ARG;
       plan->opt_kernel = (int)value;
       return MLA_OK;
     case MLA_OPT_DECODE_SPLITS:
@@ -293,14 +309,8 @@ HostStage host_stage(const mla_plan& p, int B, size_t base) {
   return h;
 }
 
-// The decode kernel a call runs: the tensor-core kernel where the plan, cache and options
-// allow it, else the CUDA-core kernel.  MLA_OK, or the status that refuses the call.
 mla_status_t pick_kernel(const mla_plan& p, const mla_cache_t& c, int* kernel) {
-  *kernel = 1;
-  if (p.opt_kernel != 1 && mla_tc_kind_ok(p.cfg) && mla_tc_supported(p, c)) *kernel = 2;
-  if (p.opt_kernel == 2 && *kernel != 2) return MLA_ERR_UNSUPPORTED;
-  if (*kernel == 1 && (size_t)p.cfg.n_heads * p.cfg.d_c > 8192) return MLA_ERR_UNSUPPORTED;
-  return MLA_OK;
+  return mla_pick_decode_kernel(p, c, kernel);
 }
 
 }  // namespace
@@ -309,6 +319,7 @@ size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B) {
   if (!plan || B <= 0) return 0;
   size_t n = mla_decode_layout(*plan, B, 1).total;
   if (mla_tc_kind_ok(plan->cfg) && mla_tc_capable(*plan)) n = std::max(n, mla_decode_layout(*plan, B, 2).total);
+  if (mla_decode_t_capable(*plan)) n = std::max(n, mla_decode_layout(*plan, B, 4).total);
   return host_stage(*plan, B, n).total;
 }
 

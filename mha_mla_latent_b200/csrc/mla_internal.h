@@ -120,7 +120,8 @@ inline cudaError_t mla_profile_event(const mla_plan& p, MlaProfKernel k, bool af
 
 // Decode workspace layout (byte offsets from the workspace base).
 struct DecodeLayout {
-  int kernel = 1;          // 1 CUDA-core, 2 tcgen05 decode, 3 tcgen05 query chunks
+  int kernel = 1;          // 1 CUDA-core, 2 tcgen05 decode (token rows), 3 tcgen05 query
+                           // chunks, 4 tcgen05 decode (head rows: the chunk kernel's form)
   int tile = 32;           // tokens per schedule tile
   int G = 0;               // workers (CTAs of the split-K kernel)
   int P = 0;               // max pieces = B + G
@@ -158,9 +159,13 @@ Sched mla_sched_view(const DecodeLayout& L, void* ws, int B);
 DecodeLayout mla_chunk_layout(const mla_plan& p, int B, int Q);
 bool mla_chunk_capable(const mla_plan& p);
 bool mla_chunk_supported(const mla_plan& p, const mla_cache_t& c);
+// rows = 128: units of 4 queries x 32 heads (query chunks); rows = 32: one query's heads (decode)
 cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B, int Q,
                                 const Sched& sched, const void* qlat, const float* qrope, float* opart,
-                                float* mlpart, int P, int G, cudaStream_t s);
+                                float* mlpart, int P, int G, cudaStream_t s, int rows);
+bool mla_decode_t_capable(const mla_plan& p);
+// The decode kernel a call runs (layout kernel id 1, 2 or 4), or the status refusing the call.
+mla_status_t mla_pick_decode_kernel(const mla_plan& p, const mla_cache_t& c, int* kernel);
 cudaError_t mla_launch_chunk(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, const void* q,
                              int B, int Q, void* out, void* ws, const DecodeLayout& L, cudaStream_t s);
 

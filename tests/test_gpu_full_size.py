@@ -30,14 +30,19 @@ def _sampled(wl, lens):
     return sorted({0, wl.batch - 1, b_long, b_short})
 
 
+@pytest.mark.parametrize("kernel", [0, 3], ids=["auto", "head_rows"])
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_sampled_parity(name):
+def test_full_size_sampled_parity(name, kernel):
     wl = get(name)
+    if kernel == 3 and wl.n_heads != 32:
+        pytest.skip("the head-row tensor-core kernel takes 32 heads")
     lens = gen.seq_lens(wl)
     seqs = _sampled(wl, lens)
     case = OracleCase(wl, seqs=seqs)
     cfg = mla.config_from_workload(wl)
     plan = mla.mla_plan_create(cfg, **plan_inputs(case))
+    if kernel:
+        mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, kernel)
     T_cap = int(lens.max())
     T_cap += T_cap % 2
     dev = "cuda"

@@ -229,13 +229,14 @@ def test_append_quant_codes_bit_exact_on_exact_latents(wl):
 
 
 # --------------------------------------------------------------------------- a1-a8
-@pytest.mark.parametrize("kernel", [0, 1, 2])
+@pytest.mark.parametrize("kernel", [0, 1, 2, 3])
 @pytest.mark.parametrize("wl", PARITY_WORKLOADS, ids=IDS)
 def test_decode_parity(wl, kernel):
-    """kernel 0: the plan's choice; 1: CUDA-core split-K; 2: tcgen05 (bf16, 32 heads)."""
+    """kernel 0: the plan's choice; 1: CUDA-core split-K; 2: tcgen05, a token per softmax
+    thread; 3: tcgen05, a head per softmax thread (both: bf16, 32 heads)."""
     case = case_for(wl)
     cfg, plan = make_plan(case, kernel=kernel)
-    if kernel == 2 and (wl.dtype == "f32" or wl.n_heads != 32):
+    if kernel >= 2 and (wl.dtype == "f32" or wl.n_heads != 32):
         with pytest.raises(mla.MlaError) as ei:
             run_decode(case, plan, cfg)
         assert ei.value.status == mla.MLA_ERR_UNSUPPORTED
@@ -246,12 +247,13 @@ def test_decode_parity(wl, kernel):
         assert_close(got[b], case.reference(b), wl.dtype, f"decode seq {b} (L={case.lens[b]})")
 
 
+@pytest.mark.parametrize("kernel", [0, 3])
 @pytest.mark.parametrize("wl", PARITY_WORKLOADS[2:4], ids=IDS[2:4])
-def test_decode_split_invariance(wl):
+def test_decode_split_invariance(wl, kernel):
     case = case_for(wl)
     outs = []
     for splits in (1, 2, 7, 0):
-        cfg, plan = make_plan(case, splits=splits)
+        cfg, plan = make_plan(case, kernel=kernel, splits=splits)
         outs.append(run_decode(case, plan, cfg))
     for o in outs[1:]:
         np.testing.assert_allclose(o, outs[0], rtol=0, atol=2e-2 if wl.dtype == "bf16" else 1e-6)
@@ -411,12 +413,12 @@ def test_paged_append_matches_contiguous(wl):
             assert torch.equal(flat.c_resid[b], paged.c_resid[b])
 
 
-@pytest.mark.parametrize("kernel", [1, 2])
+@pytest.mark.parametrize("kernel", [1, 2, 3])
 @pytest.mark.parametrize("wl", PAGED, ids=[w.name for w in PAGED])
 def test_paged_decode_parity(wl, kernel):
     """Decode over a paged cache (shuffled blocks) equals the decode over the contiguous
     cache bit for bit, and the oracle within tolerance."""
-    if kernel == 2 and (wl.dtype == "f32" or wl.n_heads != 32):
+    if kernel >= 2 and (wl.dtype == "f32" or wl.n_heads != 32):
         pytest.skip("outside the tensor-core kernel (fp32 or H != 32)")
     case = case_for(wl)
     cfg, plan = make_plan(case, kernel=kernel)
@@ -436,7 +438,7 @@ def test_paged_block_outside_pool_is_flagged():
     wl = PARITY_WORKLOADS[2]
     case = case_for(wl)
     lens = [int(L) for L in case.lens]
-    for kernel in (1, 2):
+    for kernel in (1, 2, 3):
         cfg, plan = make_plan(case, kernel=kernel)
         paged = _paged_cache(cfg, wl.batch, lens, seed=9)
         upload_oracle_cache(case, paged, paged.T_cap)
