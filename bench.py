@@ -43,7 +43,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama2_7b_bf16")
-    ap.add_argument("--kernel", type=int, default=0, help="decode kernel: 0 auto, 1 CUDA-core, 2 tcgen05")
+    ap.add_argument("--kernel", type=int, default=0,
+                    help="decode kernel: 0 auto, 1 CUDA-core, 2 tcgen05 (token rows), 3 tcgen05 (head rows)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--separate-calls", action="store_true",
@@ -210,10 +211,11 @@ def measured_traffic(workload_name, kernel_used):
     """DRAM bytes (read + write) per launch of the tensor-core attention kernel, from the
     committed ncu summary, when that summary was taken on this workload and on the current
     kernel code (else None: the counters no longer describe the kernel)."""
-    if kernel_used != 2:
+    files = {2: ("decode_tc_traffic.txt", "decode_tc.cu"), 3: ("attn_tc_traffic.txt", "chunk_tc.cu")}
+    if kernel_used not in files:
         return None
-    path = os.path.join(ROOT, "profiles", "decode_tc_traffic.txt")
-    src = os.path.join(ROOT, "mha_mla_latent_b200", "csrc", "decode_tc.cu")
+    path = os.path.join(ROOT, "profiles", files[kernel_used][0])
+    src = os.path.join(ROOT, "mha_mla_latent_b200", "csrc", files[kernel_used][1])
     try:
         kv = {}
         with open(path) as f:
@@ -434,8 +436,9 @@ class Bench:
     def roofline(self, attention_ms, workload_name):
         peak, peak_src = measured_peak_hbm()
         achieved = self.cache_bytes / (attention_ms * 1e-3) / 1e9
-        kernel_name = ("tcgen05 split-K latent attention (decode_tc_kernel)" if self.kernel_used == 2
-                       else "CUDA-core split-K latent attention (decode_simt_kernel)")
+        kernel_name = {2: "tcgen05 split-K latent attention, a token per softmax thread (decode_tc_kernel)",
+                       3: "tcgen05 split-K latent attention, a head per softmax thread (attn_tc_kernel<32>)"}.get(
+                           self.kernel_used, "CUDA-core split-K latent attention (decode_simt_kernel)")
         return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": measured_traffic(workload_name, self.kernel_used), "kernel": kernel_name,
                 "bytes_per_launch": self.cache_bytes, "avg_launch_ms": attention_ms, "peak_source": peak_src}

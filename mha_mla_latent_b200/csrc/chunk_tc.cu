@@ -417,9 +417,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
     // unit).  M = 64: rows 16q .. 16q+15 sit in lanes 0..15 of quarter q; lanes 16..31 of
     // the warp shadow them (they run the same code for the warp-wide instructions and
     // store nothing).
+    // With M = 64 the shadow lanes take the second half of each tile's tokens of their
+    // row (the scores come over by a shuffle), so both halves of a warp work.
     const int q = warp - 4;
     const bool live = ROWS == 128 || lane < 16;
     const int r = ROWS == 128 ? 32 * q + lane : 16 * q + (lane & 15);   // this thread's row
+    constexpr int TPL = ROWS == 32 ? kCT / 2 : kCT;                      // tokens per lane
+    const int tbase = (ROWS == 32 && lane >= 16) ? kCT / 2 : 0;          // its first token
     const int hd = r % kHeads;               // its head; its query is r / 32 of the unit
     const int n_kv = R / 8;
     const int g = hd / (kHeads / n_kv);      // KV head of this row's head
@@ -470,19 +474,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.s_empty(sb));
-      // RoPE score against the tile's keys: row t of the swizzled stage, KV head g's chunk
+      if (ROWS == 32) {   // the shadow lane takes tokens 32..63 of its row
+#pragma unroll
+        for (int t = 0; t < kCT / 2; ++t) {
+          const float hi = __shfl_xor_sync(0xffffffffu, s[kCT / 2 + t], 16);
+          if (lane >= 16) s[t] = hi;
+        }
+      }
+      // RoPE score against the tile's keys: row tt of the swizzled stage, KV head g's chunk
       const uint8_t* krb = sbase + a.off_stage + cs * a.stage_bytes + (n_cbox + (g >> 3)) * kTBox;
       const int lim_t = min(it.t1, p_row + 1) - it.t;   // tokens [0, lim_t) of the tile count
       float mx = -INFINITY;
 #pragma unroll
-      for (int t = 0; t < kCT; ++t) {
-        const uint4 kw = *reinterpret_cast<const uint4*>(krb + t * 128 + (((g & 7) ^ (t & 7)) << 4));
+      for (int t = 0; t < TPL; ++t) {
+        const int tt = tbase + t;
+        const uint4 kw = *reinterpret_cast<const uint4*>(krb + tt * 128 + (((g & 7) ^ (tt & 7)) << 4));
         float v = s[t] + qr[0] * bf16lo(kw.x) + qr[1] * bf16hi(kw.x) + qr[2] * bf16lo(kw.y) + qr[3] * bf16hi(kw.y) +
                   qr[4] * bf16lo(kw.z) + qr[5] * bf16hi(kw.z) + qr[6] * bf16lo(kw.w) + qr[7] * bf16hi(kw.w);
-        v = t < lim_t ? v : -INFINITY;
+        v = tt < lim_t ? v : -INFINITY;
         s[t] = v;
         mx = fmaxf(mx, v);
       }
+      if (ROWS == 32) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       if (mx > m + kTau) {   // raise the running max (lazily), rescale what O holds
         const float al = exp2f(m - mx);   // m = -inf: 0
         if (!first) {
@@ -504,11 +517,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         l *= al;
         m = mx;
       }
-      uint32_t pk[kCT / 2];
+      uint32_t pk[TPL / 2];
 #pragma unroll
-      for (int t = 0; t < kCT; t += 2) {
-        const float p0 = t < lim_t ? exp2f(s[t] - m) : 0.f;
-        const float p1 = t + 1 < lim_t ? exp2f(s[t + 1] - m) : 0.f;
+      for (int t = 0; t < TPL; t += 2) {   // l: this lane's tokens (the pair adds up at the end)
+        const float p0 = tbase + t < lim_t ? exp2f(s[t] - m) : 0.f;
+        const float p1 = tbase + t + 1 < lim_t ? exp2f(s[t + 1] - m) : 0.f;
         l += p0 + p1;
         pk[t / 2] = pack_bf16x2(p0, p1);
       }
@@ -527,12 +540,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         ok = wwait(bars.p_empty(pb), ((n >> 1) - 1) & 1);
         if (!ok) break;
       }
-      if (live) {  // P row r: 64 tokens = 128 B, 16-byte chunk c at (c ^ (r % 8))
+      {  // P row r: 64 tokens = 128 B, 16-byte chunk c at (c ^ (r % 8)); each lane its tokens
         uint8_t* prow = sbase + a.off_p + pb * kPBytes + r * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+        for (int c = 0; c < TPL / 8; ++c) {
+          const int cc = tbase / 8 + c;
+          *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -541,6 +556,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
 
       if (it.last_of_piece()) {
         // ---------------- piece epilogue: this row's partial (m, l, O)
+        if (ROWS == 32) l += __shfl_xor_sync(0xffffffffu, l, 16);   // the two token halves
         if (live) {
           a.mlpart[((size_t)r * a.P + pc) * 2] = m;
           a.mlpart[((size_t)r * a.P + pc) * 2 + 1] = l;
