@@ -66,8 +66,8 @@ __device__ void append_epilogue(const AppendArgs& a, const float* tile, int tok0
       const int rc = col - a.d_c;
       const int g = rc / (2 * a.r), j = (rc % (2 * a.r)) / 2;
       const int kpair = a.rope_pair[g * a.r + j];
-      double sn, cs;
-      sincos((double)p * a.theta[kpair], &sn, &cs);
+      float sn, cs;
+      rope_sincos(p, a.theta[kpair], &sn, &cs);
       T* dst = (T*)c.k_rope + mla_kr_offset(lc.pb, lc.pt, g, rc % (2 * a.r), lc.cap, a.R / (2 * a.r), 2 * a.r);
       dst[0] = from_f64<T>((double)v0 * cs - (double)v1 * sn);
       dst[1] = from_f64<T>((double)v0 * sn + (double)v1 * cs);

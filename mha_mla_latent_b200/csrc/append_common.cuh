@@ -167,8 +167,8 @@ __device__ __forceinline__ void append_small_finish(const AppendSmallArgs& sa, f
       }
     } else {
       const int rc = col - a.d_c;
-      double sn, cs;
-      sincos((double)p * s_theta[cp], &sn, &cs);
+      float sn, cs;
+      rope_sincos(p, s_theta[cp], &sn, &cs);
       T* dst = (T*)c.k_rope + mla_kr_offset(lc.pb, lc.pt, rc / (2 * a.r), rc % (2 * a.r), lc.cap, n_kv, 2 * a.r);
       dst[0] = from_f64<T>((double)v0 * cs - (double)v1 * sn);
       dst[1] = from_f64<T>((double)v0 * sn + (double)v1 * cs);

@@ -94,4 +94,17 @@ __device__ __forceinline__ int nib_to_int(uint32_t n) { return (int)((n ^ 8u) & 
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// sin and cos of the RoPE angle p * theta.  The angle is formed and reduced to [-pi, pi] in
+// float64 by Cody and Waite's two-constant reduction (2 pi = hi + lo, hi with 31 significant
+// bits so that k * hi is exact for |k| < 2^20, i.e. angles below ~6.5e6 rad), and the
+// float32 sincos of the reduced angle follows: about 3e-7 absolute error, far below the
+// rounding of the bf16 / f32 values it rotates.
+__device__ __forceinline__ void rope_sincos(int p, double theta, float* s, float* c) {
+  const double a = (double)p * theta;
+  const double k = rint(a * 0.15915494309189535);   // 1 / (2 pi)
+  double r = fma(-k, 6.2831853069365025, a);        // hi part of 2 pi
+  r = fma(-k, 2.430840202602477e-10, r);            // lo part
+  sincosf((float)r, s, c);
+}
+
 }  // namespace mla

@@ -94,8 +94,8 @@ __device__ __forceinline__ void absorb_body(const AbsorbArgs& a, int blk_id, flo
       const int L = __ldg(a.seq_lens + sq / a.q_chunk) - (a.q_chunk - 1 - sq % a.q_chunk);
       const int p = (L >= 1 && L <= a.T_cap) ? L - 1 : 0;
       const double x0 = qv(r, 2 * k), x1 = qv(r, 2 * k + 1);
-      double sn, cs;
-      sincos((double)p * __ldg(a.theta + k), &sn, &cs);
+      float sn, cs;
+      rope_sincos(p, __ldg(a.theta + k), &sn, &cs);
       const size_t o = ((size_t)sq * a.H + g * G + row % G) * 2 * a.r + 2 * jr;
       a.qrope[o] = (float)((x0 * cs - x1 * sn) * (double)scale);
       a.qrope[o + 1] = (float)((x0 * sn + x1 * cs) * (double)scale);
@@ -674,7 +674,7 @@ struct StepPreArgs {
 };
 
 template <bool INT4>
-__global__ void __launch_bounds__(256) step_pre_kernel(StepPreArgs sp) {
+__global__ void __launch_bounds__(256, 1) step_pre_kernel(StepPreArgs sp) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int b = blockIdx.x;
   if (b < sp.n_abs) {
