@@ -37,12 +37,12 @@ constexpr int kCT = 64;              // tokens per tile
 constexpr int kHeads = 32;
 constexpr uint32_t kTBox = 8192;     // cache box: 64 rows x 128 B
 constexpr float kTau = 8.0f;         // lazy-rescale threshold, log2 units
-// Rows per unit: 128 = 4 queries x 32 heads (many queries per sequence, MMA M = 128), or
-// 32 = the 32 heads of one query (decode, MMA M = 64: rows 32..63 of the A operands read
-// the next 4 KB of shared memory, whose values only reach output rows nobody reads).
+// Row capacity of a unit: 128 (MMA M = 128: a block of queries x heads, or the heads of one
+// query when there are more than 32), or 32 (MMA M = 64: the heads of one query, at most
+// 32; rows 32..63 of the A operands read the next 4 KB of shared memory, whose values only
+// reach output rows nobody reads).  A unit holds qper queries x H heads = rows <= ROWS.
 template <int ROWS> struct Geo {
   static constexpr int M = ROWS == 32 ? 64 : 128;   // MMA M
-  static constexpr int QPER = ROWS / 32;             // queries per unit
   static constexpr int SW = ROWS == 32 ? 2 : 4;      // softmax warps (TMEM lane quarters used)
   static constexpr uint32_t QBOX = ROWS * 128u;      // Q_lat box: ROWS rows x 128 B
   static constexpr uint32_t PBYTES = ROWS * 128u;    // P buffer: ROWS rows x 64 tokens bf16
@@ -51,6 +51,8 @@ constexpr uint32_t kSCol = 0, kOCol = 128;
 
 struct ChunkArgs {
   int q_chunk, nqb, d_c, R, P, T_cap;
+  int H, qper, rows;       // heads, queries per unit, rows per unit (qper * H <= the kernel's ROWS)
+  int dcp;                 // d_c rounded up to 64: the TMA boxes zero-fill the columns past d_c
   const __half* scales;    // quantised cache: [rows][d_c/32] fp16 group scales
   uint32_t code_row;       // quantised cache: code bytes per token
   Sched sched;
@@ -138,14 +140,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ ChunkArgs a) {
   constexpr bool QUANT = QB != 0;
   using GG = Geo<ROWS>;
-  constexpr int kRows = ROWS, kQB = GG::QPER, kSW = GG::SW;
+  constexpr int kSW = GG::SW;
   constexpr uint32_t kQBox = GG::QBOX, kPBytes = GG::PBYTES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t sbase_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (sbase_u32 - smem_u32(smem_raw));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int dc = a.d_c, R = a.R;
-  const int n_cbox = dc / 64, n_kbox = R / 64;
+  const int dc = a.d_c, R = a.R, dcp = a.dcp;
+  const int n_cbox = dcp / 64, n_kbox = (R + 63) / 64;
   Bars bars{sbase_u32 + a.off_bar, a.NC, a.NRAW};
   Misc* misc = reinterpret_cast<Misc*>(sbase + a.off_misc);
   volatile int* abort_flag = &misc->abort_flag;
@@ -186,8 +188,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
   pdl_trigger();
   const uint32_t tmem = misc->tmem_base;
   const int w = blockIdx.x;
-  auto qrow0 = [&](int v) {   // first Q_lat row of unit v: query (v % nqb) * 4 of sequence v / nqb
-    return ((v / a.nqb) * a.q_chunk + (v % a.nqb) * kQB) * kHeads;
+  auto qrow0 = [&](int v) {   // first Q_lat row of unit v: query (v % nqb) * qper of sequence v / nqb
+    return ((v / a.nqb) * a.q_chunk + (v % a.nqb) * a.qper) * a.H;
   };
 
   if (warp == 0) {
@@ -221,14 +223,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
           for (int kb = 0; kb < n_cbox; ++kb) tma_load_2d(st + kb * kTBox, &tm_c, bars.c_full(cs), kb * 64, row);
         for (int kb = 0; kb < n_kbox; ++kb)
           tma_load_2d(st + (n_cbox + kb) * kTBox, &tm_kr, bars.c_full(cs), kb * 64, row);
-        if (QUANT) {   // codes (one box of 64 rows) and the rows' scales into the raw ring
-          const int nvalid = min(kCT, it.t1 - it.t);
-          const uint32_t codes = (uint32_t)kCT * a.code_row;
-          const uint32_t sbytes = (uint32_t)((((nvalid + 1) & ~1) * (dc / 16) + 15) & ~15);
+        if (QUANT) {   // codes (one box of 64 rows) into the raw ring; the dequantising
+                       // warps read the rows' scales themselves
           const uint32_t rb = sbase_u32 + a.off_raw + rs * a.raw_stage;
-          mbar_expect_tx(bars.raw_full(rs), codes + sbytes);
+          mbar_expect_tx(bars.raw_full(rs), (uint32_t)kCT * a.code_row);
           tma_load_2d(rb, &tm_c, bars.raw_full(rs), 0, row);
-          bulk_load(rb + codes, a.scales + (size_t)row * (dc / 32), sbytes, bars.raw_full(rs));
         }
       }
       last = n;
@@ -252,7 +251,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
     // ============================================================ MMA issuer
     if (lane == 0) {
       const uint32_t idesc1 = idesc_bf16_f32(GG::M, kCT, false, false);   // S[row][t]
-      const uint32_t idesc2 = idesc_bf16_f32(GG::M, dc, false, true);     // O[row][d]
+      const uint32_t idesc2 = idesc_bf16_f32(GG::M, dcp, false, true);    // O[row][d]
       TileIter it;
       it.init(&a.sched, w);
       int n = 0, u = 0;
@@ -304,7 +303,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         tc_fence_after();
         {  // MMA1: S = Q_lat C^T
           const uint32_t c0 = sbase_u32 + a.off_stage + cs * a.stage_bytes;
-          for (int kk = 0; kk < dc / 16; ++kk) {
+          for (int kk = 0; kk < dcp / 16; ++kk) {
             const uint64_t ad = smem_desc(sbase_u32 + a.off_q + (kk >> 2) * kQBox + (kk & 3) * 32, 16, 1024,
                                           kLayoutSW128);
             const uint64_t bd = smem_desc(c0 + (kk >> 2) * kTBox + (kk & 3) * 32, 16, 1024, kLayoutSW128);
@@ -343,6 +342,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         lo_v = it.v;
         lo = __ldg(a.seq_lens + it.v) - MLA_RESID_WINDOW;
       }
+      // this token's group scales (up to 8), loaded ahead of the stage wait
+      __half scl[8];
+      {
+        const MlaLoc lc = chunk_loc<PAGED>(a, it.v / a.nqb, it.t);
+        const __half* sp = a.scales + ((size_t)lc.pb * lc.cap + lc.pt + tok) * (dc / 32);
+        const bool in = tok < it.t1 - it.t;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) scl[j] = (in && j < dc / 32) ? __ldg(sp + j) : __float2half(0.f);
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_full(rs), (n / a.NRAW) & 1, abort_flag, lim));
       if (ok && n >= a.NC)
         ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag, lim));
@@ -352,56 +360,54 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
       uint8_t* C = sbase + a.off_stage + cs * a.stage_bytes + tok * 128;
       const int tp = it.t + tok;
       const size_t rslot = (size_t)it.v * MLA_RESID_WINDOW + (tp & (MLA_RESID_WINDOW - 1));
+      // latent value j of the row goes to box j / 64, 16-byte chunk (j % 64) / 8 (swizzled)
+      auto put = [&](int chunk, uint4 v) {
+        *reinterpret_cast<uint4*>(C + (chunk >> 3) * kTBox + (((chunk & 7) ^ (tok & 7)) << 4)) = v;
+      };
       if (RESID && tok < nvalid && tp >= lo && __ldg(a.cache.resid_pos + rslot) == tp) {
         // one of the window's tokens: its unquantised row from the ring
         const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.cache.c_resid) +
                                                           rslot * dc);
-        for (int half = 0; half < dc / 64; ++half)
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch)
-            *reinterpret_cast<uint4*>(C + half * kTBox + ((ch ^ (tok & 7)) << 4)) = __ldg(src + half * 8 + ch);
+        for (int j = 0; j < dc / 8; ++j) put(j, __ldg(src + j));
       } else if (tok < nvalid) {
-        const __half* sc = reinterpret_cast<const __half*>(raw + kCT * a.code_row) + tok * (dc / 32);
         const uint8_t* codes = raw + tok * a.code_row;
-        for (int half = 0; half < dc / 64; ++half) {
-          const float s0 = __half2float(sc[half * 2]), s1 = __half2float(sc[half * 2 + 1]);
-          if (QB == 4) {   // two's-complement nibbles, element 2i in the low nibble of byte i
-            const uint4 c0 = *reinterpret_cast<const uint4*>(codes + half * 32);
-            const uint4 c1 = *reinterpret_cast<const uint4*>(codes + half * 32 + 16);
-            const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              const float sv = ch < 4 ? s0 : s1;
+        for (int grp = 0; grp < 8; ++grp) {   // 32 values, one scale
+          if (grp >= dc / 32) break;
+          const float sv = __half2float(scl[grp]);
+          if (QB == 4) {   // two's-complement nibbles, element 2i in the low nibble of byte i
+            const uint4 cw = *reinterpret_cast<const uint4*>(codes + grp * 16);
+            const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
               uint32_t o[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 const uint32_t byte = (words[ch] >> (8 * j)) & 0xFFu;
                 o[j] = pack_bf16x2((float)nib_to_int(byte & 15u) * sv, (float)nib_to_int(byte >> 4) * sv);
               }
-              *reinterpret_cast<uint4*>(C + half * kTBox + ((ch ^ (tok & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+              put(grp * 4 + ch, make_uint4(o[0], o[1], o[2], o[3]));
             }
           } else {         // two's-complement 2-bit fields, element 4i+k in bits 2k..2k+1 of byte i
-            const uint4 c0 = *reinterpret_cast<const uint4*>(codes + half * 16);
-            const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
+            const uint2 cw = *reinterpret_cast<const uint2*>(codes + grp * 8);
+            const uint32_t words[2] = {cw.x, cw.y};
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
+            for (int ch = 0; ch < 4; ++ch) {
               const uint32_t bits = (words[ch >> 1] >> (16 * (ch & 1))) & 0xFFFFu;
-              const float sv = ch < 4 ? s0 : s1;
               uint32_t o[4];
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 const int f0 = (int)((bits >> (4 * j)) & 3u), f1 = (int)((bits >> (4 * j + 2)) & 3u);
                 o[j] = pack_bf16x2((float)(f0 >= 2 ? f0 - 4 : f0) * sv, (float)(f1 >= 2 ? f1 - 4 : f1) * sv);
               }
-              *reinterpret_cast<uint4*>(C + half * kTBox + ((ch ^ (tok & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+              put(grp * 4 + ch, make_uint4(o[0], o[1], o[2], o[3]));
             }
           }
         }
       } else {
-        for (int half = 0; half < dc / 64; ++half)
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(C + half * kTBox + ch * 16) = make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < dc / 8; ++j) put(j, make_uint4(0, 0, 0, 0));
       }
+      for (int j = dc / 8; j < dcp / 8; ++j) put(j, make_uint4(0, 0, 0, 0));   // padding columns
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -424,9 +430,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
     const int r = ROWS == 128 ? 32 * q + lane : 16 * q + (lane & 15);   // this thread's row
     constexpr int TPL = ROWS == 32 ? kCT / 2 : kCT;                      // tokens per lane
     const int tbase = (ROWS == 32 && lane >= 16) ? kCT / 2 : 0;          // its first token
-    const int hd = r % kHeads;               // its head; its query is r / 32 of the unit
+    const bool valid_row = live && r < a.rows;
+    const int hd = r % a.H;                  // its head; its query is r / H of the unit
     const int n_kv = R / 8;
-    const int g = hd / (kHeads / n_kv);      // KV head of this row's head
+    const int g = hd / (a.H / n_kv);         // KV head of this row's head
     TileIter it;
     it.init(&a.sched, w);
     int n = 0, u = 0;
@@ -441,13 +448,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
       const bool first = it.first_of_piece();
       const int pc = it.pc;
       if (first) {
-        const int bseq = it.v / a.nqb, i = (it.v % a.nqb) * kQB + r / kHeads;
+        const int bseq = it.v / a.nqb, i = (it.v % a.nqb) * a.qper + r / a.H;
         p_row = -1;
 #pragma unroll
         for (int j = 0; j < 8; ++j) qr[j] = 0.f;
-        if (live && i < a.q_chunk) {
+        if (r < a.rows && i < a.q_chunk) {
           p_row = __ldg(a.seq_lens + bseq) - a.q_chunk + i;
-          const float4* src = reinterpret_cast<const float4*>(a.qrope + (((size_t)bseq * a.q_chunk + i) * kHeads + hd) * 8);
+          const float4* src = reinterpret_cast<const float4*>(a.qrope + (((size_t)bseq * a.q_chunk + i) * a.H + hd) * 8);
           const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
           qr[0] = x0.x; qr[1] = x0.y; qr[2] = x0.z; qr[3] = x0.w;
           qr[4] = x1.x; qr[5] = x1.y; qr[6] = x1.z; qr[7] = x1.w;
@@ -503,7 +510,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
           const int pn = n - 1;
           if (!wwait(bars.p_empty(pn & 1), (pn >> 1) & 1)) { ok = false; break; }
           tc_fence_after();
-          for (int cc = 0; cc < dc / 16; ++cc) {
+          for (int cc = 0; cc < dcp / 16; ++cc) {
             const uint32_t ta = taddr(tmem, 32 * q, kOCol + 16 * cc);
             uint32_t o[16];
             tmem_ld16(ta, o);
@@ -531,7 +538,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         const int nvalid = it.t1 - it.t;
         uint8_t* C = sbase + a.off_stage + cs * a.stage_bytes;
         const int nchunk = (kCT - nvalid) * 8 * n_cbox;   // 16-byte chunks
-        for (int i = r; live && i < nchunk; i += kRows) {
+        for (int i = r; live && i < nchunk; i += ROWS) {
           const int box = i / ((kCT - nvalid) * 8), rem = i % ((kCT - nvalid) * 8);
           *reinterpret_cast<uint4*>(C + box * kTBox + (nvalid + rem / 8) * 128 + (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
         }
@@ -557,20 +564,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
       if (it.last_of_piece()) {
         // ---------------- piece epilogue: this row's partial (m, l, O)
         if (ROWS == 32) l += __shfl_xor_sync(0xffffffffu, l, 16);   // the two token halves
-        if (live) {
+        if (valid_row) {
           a.mlpart[((size_t)r * a.P + pc) * 2] = m;
           a.mlpart[((size_t)r * a.P + pc) * 2 + 1] = l;
         }
         ok = wwait(bars.o_full(), u & 1);
         if (!ok) break;
         tc_fence_after();
-        float* dst = a.opart + ((size_t)pc * kRows + r) * dc;
+        float* dst = a.opart + ((size_t)pc * a.rows + (valid_row ? r : 0)) * dc;
         for (int c0 = 0; c0 < dc; c0 += 32) {
           uint32_t o[2][16];
 #pragma unroll
           for (int k = 0; k < 2; ++k) tmem_ld16(taddr(tmem, 32 * q, kOCol + c0 + 16 * k), o[k]);
           tmem_wait_ld();
-          if (!live) continue;
+          if (!valid_row) continue;
 #pragma unroll
           for (int k = 0; k < 2; ++k)
 #pragma unroll
@@ -639,12 +646,13 @@ struct ChunkLayoutSmem {
 // P0, P1 into stage 0, all inside the allocation.
 static ChunkLayoutSmem chunk_smem(int dc, int R, int qbits, int rows) {
   const uint32_t budget = 232448 - 1024;
+  const int dcp = (dc + 63) / 64 * 64;
   ChunkLayoutSmem L{};
-  L.stage_bytes = (uint32_t)(dc / 64 + R / 64) * kTBox;
-  L.raw_stage = qbits ? (((uint32_t)kCT * (dc * qbits / 8) + (uint32_t)kCT * (dc / 16)) + 127) & ~127u : 0;
+  L.stage_bytes = (uint32_t)(dcp / 64 + (R + 63) / 64) * kTBox;
+  L.raw_stage = qbits ? (((uint32_t)kCT * (dc * qbits / 8)) + 127) & ~127u : 0;
   const int nraw = qbits ? 3 : 0;
   const uint32_t box = (uint32_t)rows * 128u;
-  const uint32_t q_bytes = (uint32_t)(dc / 64) * box;
+  const uint32_t q_bytes = (uint32_t)(dcp / 64) * box;
   auto size = [&](int nc) {
     return q_bytes + nc * L.stage_bytes + 2 * box + nraw * L.raw_stage + 8 * (2 * nc + 2 * nraw + kFixedBars) + 256;
   };
@@ -667,34 +675,39 @@ static ChunkLayoutSmem chunk_smem(int dc, int R, int qbits, int rows) {
 }  // namespace chunk
 }  // namespace mla
 
-// Shapes the chunk kernel covers: bf16, 32 query heads, d_c in {64, 128, 256}, r = 4 kept
-// pairs per KV head, KV heads a multiple of 8; a bf16, int4 or 2-bit latent cache without
-// the residual window (the window depends on each query's own length, so a tile's latent
-// rows would differ between the queries that share it).
+// Shapes the kernel covers: bf16 with r = 4 kept pairs per KV head (2r = 8 RoPE dims, one
+// 16-byte chunk per KV head), d_c a multiple of 32 up to 256 (the TMA boxes zero-fill a
+// latent narrower than a multiple of 64), RoPE keys up to 256 dims, heads up to 128; the
+// quantised caches with whole 16-byte code rows.
+static bool attn_shape_ok(const mla_plan& p, int rows_cap) {
+  const mla_config_t& cfg = p.cfg;
+  if (cfg.dtype != MLA_BF16 || 2 * cfg.r_pairs != 8 || p.R > 256 || p.R % 8 != 0) return false;
+  if (cfg.d_c % 32 != 0 || cfg.d_c > 256 || cfg.n_heads > 128) return false;
+  const bool quant = mla_kind_quant(cfg.cache_kind);
+  const int qbits = quant ? mla_quant_bits(cfg.cache_kind) : 0;
+  if (quant && (cfg.d_c * qbits / 8) % 16 != 0) return false;
+  return mla::chunk::chunk_smem(cfg.d_c, p.R, qbits, rows_cap).total <= 232448;
+}
+
+// Any cache view the validation accepts (the dequantising warps read scales with plain loads).
+static bool attn_cache_ok(const mla_plan&, const mla_cache_t&) { return true; }
+
+// Many queries per sequence: units of 128 / H queries x H heads (M = 128), without the
+// residual window (it depends on each query's own length, so a tile's latent rows would
+// differ between the queries that share it).
 bool mla_chunk_capable(const mla_plan& p) {
-  const mla_config_t& cfg = p.cfg;
-  if (cfg.dtype != MLA_BF16 || cfg.n_heads != mla::chunk::kHeads) return false;
-  if (cfg.cache_kind == MLA_CACHE_INT4_G32_R128) return false;
-  if (cfg.d_c % 64 != 0 || cfg.d_c > 256 || 2 * cfg.r_pairs != 8 || p.R % 64 != 0) return false;
-  const int qbits = mla_kind_quant(cfg.cache_kind) ? mla_quant_bits(cfg.cache_kind) : 0;
-  return mla::chunk::chunk_smem(cfg.d_c, p.R, qbits, 128).total <= 232448;
+  return p.cfg.cache_kind != MLA_CACHE_INT4_G32_R128 && attn_shape_ok(p, 128);
 }
 
-// The decode form of the same kernel (32 rows per sequence, MMA M = 64): the chunk kernel's
-// shapes, with the residual window too (one query per sequence).
-bool mla_decode_t_capable(const mla_plan& p) {
-  const mla_config_t& cfg = p.cfg;
-  if (cfg.dtype != MLA_BF16 || cfg.n_heads != mla::chunk::kHeads) return false;
-  if (cfg.d_c % 64 != 0 || cfg.d_c > 256 || 2 * cfg.r_pairs != 8 || p.R % 64 != 0) return false;
-  const int qbits = mla_kind_quant(cfg.cache_kind) ? mla_quant_bits(cfg.cache_kind) : 0;
-  return mla::chunk::chunk_smem(cfg.d_c, p.R, qbits, 32).total <= 232448;
-}
-
-// The scale rows of a quantised cache are fetched with 1-D bulk copies, which need an even
-// capacity.
 bool mla_chunk_supported(const mla_plan& p, const mla_cache_t& c) {
-  if (!mla_chunk_capable(p)) return false;
-  return !(mla_kind_quant(p.cfg.cache_kind) && c.T_cap % 2 != 0);
+  return mla_chunk_capable(p) && attn_cache_ok(p, c);
+}
+
+// The decode form (one query per unit: M = 64 for up to 32 heads, else M = 128).
+bool mla_decode_t_capable(const mla_plan& p) { return attn_shape_ok(p, p.cfg.n_heads <= 32 ? 32 : 128); }
+
+bool mla_decode_t_supported(const mla_plan& p, const mla_cache_t& c) {
+  return mla_decode_t_capable(p) && attn_cache_ok(p, c);
 }
 
 cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B, int Q,
@@ -702,13 +715,14 @@ cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const i
                                 float* mlpart, int P, int G, cudaStream_t s, int rows) {
   using namespace mla::chunk;
   const mla_config_t& cfg = p.cfg;
-  const int dc = cfg.d_c, R = p.R;
+  const int dc = cfg.d_c, R = p.R, H = cfg.n_heads;
   const int qbits = mla_kind_quant(cfg.cache_kind) ? mla_quant_bits(cfg.cache_kind) : 0;
+  const int qper = rows == 128 ? (Q > 1 ? 128 / H : 1) : 1;   // queries per unit
   const uint32_t code_row = (uint32_t)(dc * qbits / 8);
   const uint64_t crows = mla_cache_rows(c);
   CUtensorMap tm_c, tm_kr, tm_q;
   bool ok = map_bf16_sw128(&tm_kr, c.k_rope, R, crows, kCT) &&
-            map_bf16_sw128(&tm_q, qlat, dc, (uint64_t)B * Q * kHeads, (uint32_t)rows);
+            map_bf16_sw128(&tm_q, qlat, dc, (uint64_t)B * Q * H, (uint32_t)rows);
   if (qbits) {   // code rows, one 64-row box per tile, no swizzle
     EncodeTiledFn fn = encode_fn();
     cuuint64_t gdim[2] = {code_row, crows};
@@ -724,7 +738,8 @@ cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const i
   if (!ok) return cudaErrorInvalidValue;
   const ChunkLayoutSmem L = chunk_smem(dc, R, qbits, rows);
   ChunkArgs a;
-  a.q_chunk = Q; a.nqb = (Q + rows / 32 - 1) / (rows / 32); a.d_c = dc; a.R = R; a.P = P; a.T_cap = c.T_cap;
+  a.q_chunk = Q; a.nqb = (Q + qper - 1) / qper; a.d_c = dc; a.R = R; a.P = P; a.T_cap = c.T_cap;
+  a.H = H; a.qper = qper; a.rows = qper * H; a.dcp = (dc + 63) / 64 * 64;
   a.scales = (const __half*)c.c_scales; a.code_row = code_row;
   a.sched = sched; a.seq_lens = seq_lens; a.qrope = qrope; a.opart = opart; a.mlpart = mlpart;
   a.cache = c; a.err = p.err;

@@ -635,7 +635,8 @@ cudaError_t launch_attention_combine(const mla_plan& p, const mla_cache_t& c, co
     if ((e = mla_profile_event(p, kProfAttention, true, s)) != cudaSuccess) return e;
   } else if (L.kernel == 4) {
     e = mla_launch_chunk_tc(p, c, seq_lens, B, 1, sched, base + L.off_qlat, (const float*)(base + L.off_qrope),
-                            (float*)(base + L.off_opart), (float*)(base + L.off_mlpart), L.P, L.G, s, 32);
+                            (float*)(base + L.off_opart), (float*)(base + L.off_mlpart), L.P, L.G, s,
+                            H <= 32 ? 32 : 128);
     if (e != cudaSuccess) return e;
   } else {
     e = mla_launch_decode_tc(p, c, seq_lens, B, sched, base + L.off_qlat, (const float*)(base + L.off_qrope),
@@ -724,7 +725,7 @@ cudaError_t launch_chunk(const mla_plan& p, const mla_cache_t& c, const int32_t*
                          int Q, void* out, void* ws, const DecodeLayout& L, cudaStream_t s) {
   using bf16 = __nv_bfloat16;
   const mla_config_t& cfg = p.cfg;
-  constexpr int kQB = 4;
+  const int kQB = 128 / cfg.n_heads;   // queries per unit: a unit holds up to 128 (query, head) rows
   AbsorbArgs aa;
   size_t smem_abs;
   int nblk;
@@ -786,7 +787,8 @@ DecodeLayout mla_chunk_layout(const mla_plan& p, int B, int Q) {
   L.kernel = 3;
   L.tile = 64;
   L.G = p.opt_splits > 0 ? p.opt_splits : p.num_sms;
-  const int units = B * ((Q + 3) / 4), rows = 4 * cfg.n_heads;
+  const int qper = 128 / cfg.n_heads;   // queries per unit (see launch_chunk)
+  const int units = B * ((Q + qper - 1) / qper), rows = qper * cfg.n_heads;
   L.P = units + L.G;
   L.K = cfg.d_c + p.R;
   const size_t nq = (size_t)B * Q * cfg.n_heads;   // query rows (query x head)

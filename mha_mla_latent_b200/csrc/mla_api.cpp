@@ -80,8 +80,7 @@ void free_plan(mla_plan* p) {
 mla_status_t mla_pick_decode_kernel(const mla_plan& p, const mla_cache_t& c, int* kernel) {
   *kernel = 1;
   if (p.opt_kernel == 3) {   // the head-row tensor-core form
-    const bool even = !(mla_kind_quant(p.cfg.cache_kind) && c.T_cap % 2 != 0);
-    if (!mla_decode_t_capable(p) || !even) return MLA_ERR_UNSUPPORTED;
+    if (!mla_decode_t_supported(p, c)) return MLA_ERR_UNSUPPORTED;
     *kernel = 4;
     return MLA_OK;
   }

@@ -164,6 +164,7 @@ cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const i
                                 const Sched& sched, const void* qlat, const float* qrope, float* opart,
                                 float* mlpart, int P, int G, cudaStream_t s, int rows);
 bool mla_decode_t_capable(const mla_plan& p);
+bool mla_decode_t_supported(const mla_plan& p, const mla_cache_t& c);
 // The decode kernel a call runs (layout kernel id 1, 2 or 4), or the status refusing the call.
 mla_status_t mla_pick_decode_kernel(const mla_plan& p, const mla_cache_t& c, int* kernel);
 cudaError_t mla_launch_chunk(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, const void* q,
