@@ -7,10 +7,11 @@
 // separately computed partial-RoPE term, and takes the probability-weighted latent through
 // W_uv; a chunk of a long document's tokens reads the same latent prefix with every query.
 //
-// A unit of work is (sequence b, block of 4 consecutive queries) = 128 rows (query j,
-// head h), row = 32 j + h.  The units' tokens (up to the block's last query) are laid end
-// to end and split among the CTAs like the decode's split-K schedule, in tiles of 64
-// tokens.  Per tile:
+// A unit of work is (sequence b, block of qper = floor(128 / H) consecutive queries):
+// qper * H rows (query j, head h), row = H j + h; a single decode query with more than 32
+// heads is a unit of H rows, one with at most 32 heads a unit of the MMA's M = 64 form.
+// The units' tokens (up to the block's last query) are laid end to end and split among the
+// CTAs like the decode's split-K schedule, in tiles of 64 tokens.  Per tile:
 //     S[row][t]   = sum_c Qlat[row][c] * C[t][c]              MMA1  M = 128 rows, N = 64 tokens
 //     S[row][t]  += sum_j Qrope[row][j] * KR[t][g(h)][j]       CUDA cores (fp32), one row per thread
 //     O[row][d]  += sum_t P[row][t] * C[t][d]                  MMA2  M = 128, N = d_c, K = 64
@@ -21,7 +22,8 @@
 //
 // Warp roles (8 warps): warp 0 producer (TMA: the unit's Q_lat rows, C and RoPE-key tiles
 // into a ring of stages), warp 1 TMEM owner and single-thread
-// MMA issuer, warps 4-7 softmax (warp 4 + j owns the rows of query j: TMEM lane quarter j).
+// MMA issuer, warps 2-3 dequantisers of a quantised cache, warps 4-7 softmax (warp 4 + k
+// owns TMEM lane quarter k).
 // Every wait is bounded; a timeout sets MLA_DEVERR_TIMEOUT, drains and releases TMEM.
 #include <cuda.h>
 
@@ -34,7 +36,6 @@ namespace chunk {
 using namespace sm100;
 
 constexpr int kCT = 64;              // tokens per tile
-constexpr int kHeads = 32;
 constexpr uint32_t kTBox = 8192;     // cache box: 64 rows x 128 B
 constexpr float kTau = 8.0f;         // lazy-rescale threshold, log2 units
 // Row capacity of a unit: 128 (MMA M = 128: a block of queries x heads, or the heads of one
@@ -57,9 +58,9 @@ struct ChunkArgs {
   uint32_t code_row;       // quantised cache: code bytes per token
   Sched sched;
   const int32_t* seq_lens;
-  const float* qrope;      // [B*Q][32][2r], rotated at each query's position, scaled
-  float* opart;            // [P][128][d_c]
-  float* mlpart;           // [128][P][2]
+  const float* qrope;      // [B*Q][H][2r], rotated at each query's position, scaled
+  float* opart;            // [P][rows][d_c]
+  float* mlpart;           // [rows][P][2]
   mla_cache_t cache;
   int32_t* err;
   uint64_t wait_ns;
@@ -503,10 +504,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         mx = fmaxf(mx, v);
       }
       if (ROWS == 32) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      if (mx > m + kTau) {   // raise the running max (lazily), rescale what O holds
-        const float al = exp2f(m - mx);   // m = -inf: 0
+      // Raise the running max lazily: a row rescales when its max grew by more than kTau.
+      // Rows decide on their own, but the TMEM loads and stores (and the wait before them)
+      // are warp-collective, so the warp takes the branch when any of its rows needs it and
+      // the other rows multiply by 1.
+      const bool raise = mx > m + kTau;
+      if (__any_sync(0xffffffffu, raise)) {
+        const float al = raise ? exp2f(m - mx) : 1.f;   // m = -inf: 0
         if (!first) {
-          // O holds the piece's tiles before this one: wait for MMA2(n-1), then rescale the row
+          // O holds the piece's tiles before this one: wait for MMA2(n-1), then rescale
           const int pn = n - 1;
           if (!wwait(bars.p_empty(pn & 1), (pn >> 1) & 1)) { ok = false; break; }
           tc_fence_after();
@@ -521,8 +527,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
           }
           tmem_wait_st();
         }
-        l *= al;
-        m = mx;
+        if (raise) {
+          l *= al;
+          m = mx;
+        }
       }
       uint32_t pk[TPL / 2];
 #pragma unroll

@@ -755,7 +755,8 @@ DecodeLayout mla_decode_layout(const mla_plan& p, int B, int kernel) {
   DecodeLayout L;
   L.kernel = kernel;
   L.tile = kernel == 2 ? 128 : kernel == 4 ? 64 : mla::kSimtTile;
-  L.G = p.opt_splits > 0 ? p.opt_splits : (kernel == 2 ? p.num_sms : 2 * p.num_sms);
+  // the tensor-core kernels hold one CTA per SM (one wave); the CUDA-core kernel two
+  L.G = p.opt_splits > 0 ? p.opt_splits : (kernel == 2 || kernel == 4 ? p.num_sms : 2 * p.num_sms);
   L.P = B + L.G;
   L.K = cfg.d_c + p.R;
   const int H = cfg.n_heads;

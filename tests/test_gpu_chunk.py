@@ -6,7 +6,7 @@ its own (float64, the unabsorbed definition) over its causal prefix; the chunk k
 outputs must match within the parity tolerances.  Chunk sizes cover a partial query block
 (Q = 2), several blocks whose positions straddle 64-token tiles (Q = 12) and a long chunk
 (Q = 64); lengths are not tile multiples; contiguous and paged caches; bf16, int4 and
-2-bit latents.
+2-bit latents; 32 heads (four queries per 128-row unit) and 9 GQA heads (fourteen).
 """
 
 import os
@@ -24,7 +24,8 @@ pytestmark = pytest.mark.gpu
 WLS = [PARITY_WORKLOADS[2].with_(name="llama_dc256_chunk", fixed_lens=(1000, 333, 130)),
        PARITY_WORKLOADS[3].with_(name="llama_dc64_chunk", batch=3, fixed_lens=(2500, 129, 77)),
        PARITY_WORKLOADS[4].with_(name="llama_int4_chunk", fixed_lens=(700, 200, 77)),
-       PARITY_WORKLOADS[7].with_(name="llama_int2_chunk", fixed_lens=(700, 130, 65))]
+       PARITY_WORKLOADS[7].with_(name="llama_int2_chunk", fixed_lens=(700, 130, 65)),
+       PARITY_WORKLOADS[1].with_(name="smollm_gqa_chunk", fixed_lens=(300, 100, 70))]
 _CASES = {}
 
 

@@ -31,6 +31,24 @@ def case_for(wl):
     return _CASES[wl.name]
 
 
+def tc_kernel_ok(wl, kernel):
+    """Kernel 2 (a token per softmax thread) takes bf16 with 32 heads; kernel 3 (a head per
+    softmax thread) takes bf16 with up to 128 heads, GQA included, and up to 256 RoPE
+    key columns."""
+    if kernel == 2:
+        return wl.dtype == "bf16" and wl.n_heads == 32
+    if kernel == 3:
+        return wl.dtype == "bf16" and wl.n_heads <= 128 and wl.n_kv_heads * 2 * wl.r_pairs <= 256
+    return True
+
+
+# 64 query heads: two per KV head (256 RoPE key columns), and eight per KV head over an int4 cache
+WIDE_WORKLOADS = [PARITY_WORKLOADS[2].with_(name="h64_gqa2_dc128_small", n_heads=64, n_kv_heads=32, head_dim=64,
+                                            d_c=128, fixed_lens=(900, 1, 200)),
+                  PARITY_WORKLOADS[4].with_(name="h64_gqa8_int4_small", n_heads=64, n_kv_heads=8, head_dim=64,
+                                            d_c=128, fixed_lens=(513, 64, 2))]
+
+
 def make_plan(case, kernel=0, splits=0):
     cfg = mla.config_from_workload(case.wl)
     plan = mla.mla_plan_create(cfg, **plan_inputs(case))
@@ -233,14 +251,26 @@ def test_append_quant_codes_bit_exact_on_exact_latents(wl):
 @pytest.mark.parametrize("wl", PARITY_WORKLOADS, ids=IDS)
 def test_decode_parity(wl, kernel):
     """kernel 0: the plan's choice; 1: CUDA-core split-K; 2: tcgen05, a token per softmax
-    thread; 3: tcgen05, a head per softmax thread (both: bf16, 32 heads)."""
+    thread (bf16, 32 heads); 3: tcgen05, a head per softmax thread (bf16, up to 128 heads)."""
     case = case_for(wl)
     cfg, plan = make_plan(case, kernel=kernel)
-    if kernel >= 2 and (wl.dtype == "f32" or wl.n_heads != 32):
+    if not tc_kernel_ok(wl, kernel):
         with pytest.raises(mla.MlaError) as ei:
             run_decode(case, plan, cfg)
         assert ei.value.status == mla.MLA_ERR_UNSUPPORTED
-        pytest.skip("outside the tensor-core kernel (fp32 or H != 32)")
+        pytest.skip("outside this tensor-core kernel")
+    got = run_decode(case, plan, cfg)
+    assert mla.mla_device_error(plan) == 0
+    for b in case.seqs:
+        assert_close(got[b], case.reference(b), wl.dtype, f"decode seq {b} (L={case.lens[b]})")
+
+
+@pytest.mark.parametrize("kernel", [0, 1, 3])
+@pytest.mark.parametrize("wl", WIDE_WORKLOADS, ids=[w.name for w in WIDE_WORKLOADS])
+def test_decode_parity_wide_heads(wl, kernel):
+    """64 query heads: kernel 3 fills all 128 MMA rows with one query's heads."""
+    case = case_for(wl)
+    cfg, plan = make_plan(case, kernel=kernel)
     got = run_decode(case, plan, cfg)
     assert mla.mla_device_error(plan) == 0
     for b in case.seqs:
@@ -418,8 +448,8 @@ def test_paged_append_matches_contiguous(wl):
 def test_paged_decode_parity(wl, kernel):
     """Decode over a paged cache (shuffled blocks) equals the decode over the contiguous
     cache bit for bit, and the oracle within tolerance."""
-    if kernel >= 2 and (wl.dtype == "f32" or wl.n_heads != 32):
-        pytest.skip("outside the tensor-core kernel (fp32 or H != 32)")
+    if not tc_kernel_ok(wl, kernel):
+        pytest.skip("outside this tensor-core kernel")
     case = case_for(wl)
     cfg, plan = make_plan(case, kernel=kernel)
     lens = [int(L) for L in case.lens]
