@@ -42,11 +42,20 @@ constexpr float kTau = 8.0f;         // lazy-rescale threshold, log2 units
 // query when there are more than 32), or 32 (MMA M = 64: the heads of one query, at most
 // 32; rows 32..63 of the A operands read the next 4 KB of shared memory, whose values only
 // reach output rows nobody reads).  A unit holds qper queries x H heads = rows <= ROWS.
+// Warps (a warp reads TMEM lane quarter warp % 4 and issues on scheduler warp % 4).
+// 128 rows: the softmax warp of quarter q is warp 4 + q; producer 0, MMA issuer 1,
+// dequantisers 2 and 3.  32 rows: only quarters 0 and 1 hold rows (16 each), so warps 0, 1,
+// 4 and 5 are the softmax warps, two per quarter, each taking half of every tile's tokens;
+// the producer and the issuer sit on warps 2 and 3 and the dequantisers on 6 and 7, off the
+// softmax warps' schedulers.
 template <int ROWS> struct Geo {
   static constexpr int M = ROWS == 32 ? 64 : 128;   // MMA M
-  static constexpr int SW = ROWS == 32 ? 2 : 4;      // softmax warps (TMEM lane quarters used)
+  static constexpr int SW = 4;                       // softmax warps
   static constexpr uint32_t QBOX = ROWS * 128u;      // Q_lat box: ROWS rows x 128 B
   static constexpr uint32_t PBYTES = ROWS * 128u;    // P buffer: ROWS rows x 64 tokens bf16
+  static constexpr int PROD = ROWS == 32 ? 2 : 0;    // TMA producer warp
+  static constexpr int MMA = ROWS == 32 ? 3 : 1;     // TMEM owner and MMA issuer warp
+  static constexpr int DQ = ROWS == 32 ? 6 : 2;      // first of the two dequantising warps
 };
 constexpr uint32_t kSCol = 0, kOCol = 128;
 
@@ -54,6 +63,7 @@ struct ChunkArgs {
   int q_chunk, nqb, d_c, R, P, T_cap;
   int H, qper, rows;       // heads, queries per unit, rows per unit (qper * H <= the kernel's ROWS)
   int dcp;                 // d_c rounded up to 64: the TMA boxes zero-fill the columns past d_c
+  int rtc;                 // RoPE scores on the tensor cores (block-diagonal query rows in MMA1)
   const __half* scales;    // quantised cache: [rows][d_c/32] fp16 group scales
   uint32_t code_row;       // quantised cache: code bytes per token
   Sched sched;
@@ -64,30 +74,38 @@ struct ChunkArgs {
   mla_cache_t cache;
   int32_t* err;
   uint64_t wait_ns;
-  int NC, NRAW;
-  uint32_t off_q, off_stage, off_p, off_bar, off_misc, stage_bytes, off_raw, raw_stage;
+  int NC, NK, NRAW;        // latent stages, RoPE-key stages, code stages
+  uint32_t off_q, off_ar, off_p, off_c, off_k, off_raw, off_bar, off_misc;
+  uint32_t c_stage, k_stage, raw_stage;
 };
 
 struct Bars {
   uint32_t base;
-  int NC;
+  int NC, NK, NRAW;
   __device__ uint32_t at(int i) const { return base + 8u * (uint32_t)i; }
   __device__ uint32_t c_full(int s) const { return at(s); }
   __device__ uint32_t c_empty(int s) const { return at(NC + s); }
-  __device__ uint32_t s_full(int i) const { return at(2 * NC + i); }
-  __device__ uint32_t s_empty(int i) const { return at(2 * NC + 2 + i); }
-  __device__ uint32_t p_full(int i) const { return at(2 * NC + 4 + i); }
-  __device__ uint32_t p_empty(int i) const { return at(2 * NC + 6 + i); }
-  __device__ uint32_t o_full() const { return at(2 * NC + 8); }
-  __device__ uint32_t o_empty() const { return at(2 * NC + 9); }
-  __device__ uint32_t q_full() const { return at(2 * NC + 10); }
-  __device__ uint32_t q_empty() const { return at(2 * NC + 11); }
-  __device__ uint32_t mma_done() const { return at(2 * NC + 12); }
-  __device__ uint32_t raw_full(int s) const { return at(2 * NC + 13 + s); }
-  __device__ uint32_t raw_empty(int s) const { return at(2 * NC + 13 + NRAW + s); }
-  int NRAW;
+  __device__ uint32_t k_full(int s) const { return at(2 * NC + s); }
+  __device__ uint32_t k_empty(int s) const { return at(2 * NC + NK + s); }
+  __device__ uint32_t raw_full(int s) const { return at(2 * NC + 2 * NK + s); }
+  __device__ uint32_t raw_empty(int s) const { return at(2 * NC + 2 * NK + NRAW + s); }
+  __device__ uint32_t fixed(int i) const { return at(2 * NC + 2 * NK + 2 * NRAW + i); }
+  __device__ uint32_t s_full(int i) const { return fixed(i); }
+  __device__ uint32_t s_empty(int i) const { return fixed(2 + i); }
+  __device__ uint32_t p_full(int i) const { return fixed(4 + i); }
+  __device__ uint32_t p_empty(int i) const { return fixed(6 + i); }
+  __device__ uint32_t o_full() const { return fixed(8); }
+  __device__ uint32_t o_empty() const { return fixed(9); }
+  __device__ uint32_t q_full() const { return fixed(10); }
+  __device__ uint32_t q_empty() const { return fixed(11); }
+  __device__ uint32_t mma_done() const { return fixed(12); }
+  // 32-row units: the two softmax warps of a lane quarter exchange row maxima every tile
+  // (by tile parity) and row sums every piece
+  __device__ uint32_t x_max(int par, int q) const { return fixed(13 + 2 * par + q); }
+  __device__ uint32_t x_sum(int q) const { return fixed(17 + q); }
 };
-constexpr int kFixedBars = 13;
+constexpr int kFixedBars = 19;
+constexpr uint32_t kXchgBytes = 768;   // row maxima [2 parities][2 quarters][2 halves][16], sums [2][2][16]
 
 struct Misc {
   uint32_t tmem_base;
@@ -131,10 +149,17 @@ __device__ __forceinline__ MlaLoc chunk_loc(const ChunkArgs& a, int b, int t) {
   return mla_loc(a.cache, b, t, a.err);
 }
 
+// Byte offset of 16-byte chunk `c` of row `r` in a 128-byte-swizzled box of 128-byte rows.
+__device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)r * 128u + (uint32_t)(((c ^ r) & 7) << 4); }
+
 // ROWS: rows per unit (see Geo); QB: code width of a quantised latent cache (4 or 2),
-// whose rows warps 2-3 dequantise into the stage's latent boxes, 0 for a bf16 latent loaded
-// by TMA; RESID: the int4 cache's residual window (decode only: the window follows the one
-// query's length); PAGED: cache addressed through a block table.
+// whose rows warps 2-3 dequantise into the latent ring, 0 for a bf16 latent loaded by TMA;
+// RESID: the int4 cache's residual window (decode only: the window follows the one query's
+// length); PAGED: cache addressed through a block table.
+//
+// Rings: the latent tile of tile n sits in stage n % NC until MMA2(n) has read it; its RoPE
+// keys in stage n % NK, released after MMA1(n) when the RoPE scores run on the tensor cores
+// (a.rtc), else after MMA2(n) (the softmax warps read them).
 template <int ROWS, int QB, bool RESID, bool PAGED>
 __global__ void __launch_bounds__(256, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_kr,
@@ -148,16 +173,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
   uint8_t* sbase = smem_raw + (sbase_u32 - smem_u32(smem_raw));
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int dc = a.d_c, R = a.R, dcp = a.dcp;
+  const bool rtc = a.rtc != 0;
   const int n_cbox = dcp / 64, n_kbox = (R + 63) / 64;
-  Bars bars{sbase_u32 + a.off_bar, a.NC, a.NRAW};
+  const int kr16 = (R + 15) / 16;   // RoPE K chunks of MMA1 (the boxes zero-fill past R)
+  Bars bars{sbase_u32 + a.off_bar, a.NC, a.NK, a.NRAW};
   Misc* misc = reinterpret_cast<Misc*>(sbase + a.off_misc);
   volatile int* abort_flag = &misc->abort_flag;
   const uint64_t lim = a.wait_ns;
 
   if (threadIdx.x == 0) {
     misc->abort_flag = 0;
-    // a stage is full after its TMA bytes (and, for a quantised cache, both dequantising warps)
-    for (int s = 0; s < a.NC; ++s) { mbar_init(bars.c_full(s), QUANT ? 3 : 1); mbar_init(bars.c_empty(s), 1); }
+    // latent stage: its TMA bytes, or both dequantising warps; RoPE-key stage: its TMA bytes
+    for (int s = 0; s < a.NC; ++s) { mbar_init(bars.c_full(s), QUANT ? 2 : 1); mbar_init(bars.c_empty(s), 1); }
+    for (int s = 0; s < a.NK; ++s) { mbar_init(bars.k_full(s), 1); mbar_init(bars.k_empty(s), 1); }
     for (int s = 0; s < a.NRAW; ++s) { mbar_init(bars.raw_full(s), 1); mbar_init(bars.raw_empty(s), 2); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars.s_full(i), 1);
@@ -167,18 +195,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
     }
     mbar_init(bars.o_full(), 1);
     mbar_init(bars.o_empty(), kSW);
-    mbar_init(bars.q_full(), 1);
+    mbar_init(bars.q_full(), rtc ? 1 + kSW : 1);   // Q_lat bytes (+ the softmax warps' RoPE rows)
     mbar_init(bars.q_empty(), 1);
     mbar_init(bars.mma_done(), 1);
+    for (int i = 0; i < 4; ++i) mbar_init(bars.x_max(i >> 1, i & 1), 2);
+    for (int i = 0; i < 2; ++i) mbar_init(bars.x_sum(i), 2);
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (rtc) {   // block-diagonal RoPE query rows: zero once, each piece rewrites one chunk per row
+    uint4* ar = reinterpret_cast<uint4*>(sbase + a.off_ar);
+    for (int i = threadIdx.x; i < n_kbox * (int)kQBox / 16; i += blockDim.x) ar[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
+  if (warp == GG::PROD && lane == 0) {
     tma_prefetch_desc(&tm_c);
     tma_prefetch_desc(&tm_kr);
     tma_prefetch_desc(&tm_q);
   }
   constexpr uint32_t kTmemCols = 512;   // S 2 x 64 columns, O d_c <= 256 columns
-  if (warp == 1) {
+  if (warp == GG::MMA) {
     tmem_alloc(smem_u32(&misc->tmem_base), kTmemCols);
     tmem_relinquish();
   }
@@ -193,62 +228,64 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
     return ((v / a.nqb) * a.q_chunk + (v % a.nqb) * a.qper) * a.H;
   };
 
-  if (warp == 0) {
-    // ============================================================ TMA producer
-    TileIter it;
-    it.init(&a.sched, w);
-    int n = 0, u = 0, q_loads = 0, last = -1;
-    bool ok = true;
-    while (ok && it.valid()) {
-      if (it.first_of_piece()) {
-        if (u > 0) ok = __all_sync(0xffffffffu, mbar_wait(bars.q_empty(), (u - 1) & 1, abort_flag, lim));
-        if (!ok) break;
-        if (lane == 0) {
+  if (warp == GG::PROD) {
+    // ============================================================ TMA producer (lane 0)
+    if (lane == 0) {
+      TileIter it;
+      it.init(&a.sched, w);
+      int n = 0, u = 0, q_loads = 0, last = -1;
+      bool ok = true;
+      while (ok && it.valid()) {
+        if (it.first_of_piece()) {
+          if (u > 0 && !mbar_wait(bars.q_empty(), (u - 1) & 1, abort_flag, lim)) { ok = false; break; }
           mbar_expect_tx(bars.q_full(), (uint32_t)n_cbox * kQBox);
           for (int kb = 0; kb < n_cbox; ++kb)
             tma_load_2d(sbase_u32 + a.off_q + kb * kQBox, &tm_q, bars.q_full(), kb * 64, qrow0(it.v));
+          ++q_loads;
         }
-        ++q_loads;
-      }
-      const int cs = n % a.NC, rs = QUANT ? n % a.NRAW : 0;
-      if (n >= a.NC) ok = __all_sync(0xffffffffu, mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag, lim));
-      if (ok && QUANT && n >= a.NRAW)
-        ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_empty(rs), ((n / a.NRAW) - 1) & 1, abort_flag, lim));
-      if (!ok) break;
-      if (lane == 0) {
+        const int cs = n % a.NC, ks = n % a.NK, rs = QUANT ? n % a.NRAW : 0;
         const MlaLoc lc = chunk_loc<PAGED>(a, it.v / a.nqb, it.t);   // a 64-token tile lies in one block
         const int row = lc.pb * lc.cap + lc.pt;
-        const uint32_t st = sbase_u32 + a.off_stage + cs * a.stage_bytes;
-        mbar_expect_tx(bars.c_full(cs), (uint32_t)((QUANT ? 0 : n_cbox) + n_kbox) * kTBox);
-        if (!QUANT)
+        if (!QUANT) {   // latent boxes
+          if (n >= a.NC && !mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag, lim)) { ok = false; break; }
+          const uint32_t st = sbase_u32 + a.off_c + cs * a.c_stage;
+          mbar_expect_tx(bars.c_full(cs), (uint32_t)n_cbox * kTBox);
           for (int kb = 0; kb < n_cbox; ++kb) tma_load_2d(st + kb * kTBox, &tm_c, bars.c_full(cs), kb * 64, row);
-        for (int kb = 0; kb < n_kbox; ++kb)
-          tma_load_2d(st + (n_cbox + kb) * kTBox, &tm_kr, bars.c_full(cs), kb * 64, row);
-        if (QUANT) {   // codes (one box of 64 rows) into the raw ring; the dequantising
-                       // warps read the rows' scales themselves
+        } else {        // code rows (one box of 64 rows) into the raw ring
+          if (n >= a.NRAW && !mbar_wait(bars.raw_empty(rs), ((n / a.NRAW) - 1) & 1, abort_flag, lim)) {
+            ok = false;
+            break;
+          }
           const uint32_t rb = sbase_u32 + a.off_raw + rs * a.raw_stage;
           mbar_expect_tx(bars.raw_full(rs), (uint32_t)kCT * a.code_row);
           tma_load_2d(rb, &tm_c, bars.raw_full(rs), 0, row);
         }
+        {   // RoPE-key boxes
+          if (n >= a.NK && !mbar_wait(bars.k_empty(ks), ((n / a.NK) - 1) & 1, abort_flag, lim)) { ok = false; break; }
+          const uint32_t st = sbase_u32 + a.off_k + ks * a.k_stage;
+          mbar_expect_tx(bars.k_full(ks), (uint32_t)n_kbox * kTBox);
+          for (int kb = 0; kb < n_kbox; ++kb) tma_load_2d(st + kb * kTBox, &tm_kr, bars.k_full(ks), kb * 64, row);
+        }
+        last = n;
+        if (it.last_of_piece()) ++u;
+        it.next();
+        ++n;
       }
-      last = n;
-      if (it.last_of_piece()) ++u;
-      it.next();
-      ++n;
-    }
-    if (lane == 0) {   // drain: every issued copy lands before the CTA exits
+      // drain: every issued copy lands before the CTA exits (a copy that was not issued
+      // because its wait gave up leaves its barrier one phase behind: skipped by `last`)
       volatile int never = 0;
       if (q_loads > 0) mbar_wait(bars.q_full(), (q_loads - 1) & 1, &never, lim);
-      for (int s = 0; s < a.NC; ++s) {
-        const int k = last - ((last - s) % a.NC + a.NC) % a.NC;
-        if (last >= 0 && k >= 0) mbar_wait(bars.c_full(s), (k / a.NC) & 1, &never, lim);
-      }
-      for (int s = 0; QUANT && s < a.NRAW; ++s) {
-        const int k = last - ((last - s) % a.NRAW + a.NRAW) % a.NRAW;
-        if (last >= 0 && k >= 0) mbar_wait(bars.raw_full(s), (k / a.NRAW) & 1, &never, lim);
-      }
+      auto drain = [&](int NS, auto bar) {
+        for (int s = 0; s < NS; ++s) {
+          const int k = last - ((last - s) % NS + NS) % NS;
+          if (last >= 0 && k >= 0) mbar_wait(bar(s), (k / NS) & 1, &never, lim);
+        }
+      };
+      if (!QUANT) drain(a.NC, [&](int s) { return bars.c_full(s); });
+      else drain(a.NRAW, [&](int s) { return bars.raw_full(s); });
+      drain(a.NK, [&](int s) { return bars.k_full(s); });
     }
-  } else if (warp == 1) {
+  } else if (warp == GG::MMA) {
     // ============================================================ MMA issuer
     if (lane == 0) {
       const uint32_t idesc1 = idesc_bf16_f32(GG::M, kCT, false, false);   // S[row][t]
@@ -265,7 +302,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         if (first && pu > 0)
           if (!mbar_wait(bars.o_empty(), (pu - 1) & 1, abort_flag, lim)) return false;
         tc_fence_after();
-        const uint32_t c0 = sbase_u32 + a.off_stage + cs * a.stage_bytes;
+        const uint32_t c0 = sbase_u32 + a.off_c + cs * a.c_stage;
         const uint32_t p0 = sbase_u32 + a.off_p + pb * kPBytes;
 #pragma unroll
         for (int kk = 0; kk < kCT / 16; ++kk) {
@@ -275,11 +312,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         }
         tc_commit(bars.p_empty(pb));
         tc_commit(bars.c_empty(cs));
+        if (!rtc) tc_commit(bars.k_empty(pn % a.NK));   // the softmax warps have read the keys
         if (lastp) tc_commit(bars.o_full());
         return true;
       };
       while (ok && it.valid()) {
-        const int sb = n & 1, cs = n % a.NC;
+        const int sb = n & 1, cs = n % a.NC, ks = n % a.NK;
         const bool first = it.first_of_piece();
         {
           const uint64_t t_start = globaltimer();
@@ -291,24 +329,37 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
               continue;
             }
             if ((n < 2 || mbar_test(bars.s_empty(sb), ((n >> 1) - 1) & 1)) &&
-                (!first || mbar_test(bars.q_full(), u & 1)) && mbar_test(bars.c_full(cs), (n / a.NC) & 1))
+                (!first || mbar_test(bars.q_full(), u & 1)) && mbar_test(bars.c_full(cs), (n / a.NC) & 1) &&
+                mbar_test(bars.k_full(ks), (n / a.NK) & 1))
               break;
             if (*abort_flag || globaltimer() - t_start > lim) {
               *abort_flag = 1;
               ok = false;
               break;
             }
+            __nanosleep(32);   // leave the scheduler's issue slots to the other warps
           }
         }
         if (!ok) break;
         tc_fence_after();
-        {  // MMA1: S = Q_lat C^T
-          const uint32_t c0 = sbase_u32 + a.off_stage + cs * a.stage_bytes;
+        {  // MMA1: S = Q_lat C^T (+ Q_rope KR^T)
+          const uint32_t c0 = sbase_u32 + a.off_c + cs * a.c_stage;
+          const uint32_t d = tmem + kSCol + sb * kCT;
           for (int kk = 0; kk < dcp / 16; ++kk) {
             const uint64_t ad = smem_desc(sbase_u32 + a.off_q + (kk >> 2) * kQBox + (kk & 3) * 32, 16, 1024,
                                           kLayoutSW128);
             const uint64_t bd = smem_desc(c0 + (kk >> 2) * kTBox + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-            tc_mma_bf16(tmem + kSCol + sb * kCT, ad, bd, idesc1, kk > 0 ? 1u : 0u);
+            tc_mma_bf16(d, ad, bd, idesc1, kk > 0 ? 1u : 0u);
+          }
+          if (rtc) {
+            const uint32_t k0 = sbase_u32 + a.off_k + ks * a.k_stage;
+            for (int kk = 0; kk < kr16; ++kk) {
+              const uint64_t ad = smem_desc(sbase_u32 + a.off_ar + (kk >> 2) * kQBox + (kk & 3) * 32, 16, 1024,
+                                            kLayoutSW128);
+              const uint64_t bd = smem_desc(k0 + (kk >> 2) * kTBox + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+              tc_mma_bf16(d, ad, bd, idesc1, 1u);
+            }
+            tc_commit(bars.k_empty(ks));
           }
           tc_commit(bars.s_full(sb));
           if (it.last_of_piece()) tc_commit(bars.q_empty());
@@ -327,11 +378,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
       volatile int never = 0;
       mbar_wait(bars.mma_done(), 0, &never, lim);
     }
-  } else if (QUANT && warp >= 2 && warp < 4) {
+  } else if (QUANT && warp >= GG::DQ && warp < GG::DQ + 2) {
     // ============================================================ dequantisation
-    // thread = token row of the tile: codes * scale -> bf16 into the stage's swizzled latent
+    // thread = token row of the tile: codes * scale -> bf16 into the latent stage's swizzled
     // boxes; rows past the unit's last token are zeroed (MMA2 multiplies them by P = 0)
-    const int tok = threadIdx.x - 64;   // 0..63
+    const int tok = threadIdx.x - 32 * GG::DQ;   // 0..63
     TileIter it;
     it.init(&a.sched, w);
     int n = 0;
@@ -358,12 +409,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
       if (!ok) break;
       const int nvalid = min(kCT, it.t1 - it.t);
       const uint8_t* raw = sbase + a.off_raw + rs * a.raw_stage;
-      uint8_t* C = sbase + a.off_stage + cs * a.stage_bytes + tok * 128;
+      uint8_t* C = sbase + a.off_c + cs * a.c_stage;
       const int tp = it.t + tok;
       const size_t rslot = (size_t)it.v * MLA_RESID_WINDOW + (tp & (MLA_RESID_WINDOW - 1));
       // latent value j of the row goes to box j / 64, 16-byte chunk (j % 64) / 8 (swizzled)
       auto put = [&](int chunk, uint4 v) {
-        *reinterpret_cast<uint4*>(C + (chunk >> 3) * kTBox + (((chunk & 7) ^ (tok & 7)) << 4)) = v;
+        *reinterpret_cast<uint4*>(C + (chunk >> 3) * kTBox + sw128(tok, chunk)) = v;
       };
       if (RESID && tok < nvalid && tp >= lo && __ldg(a.cache.resid_pos + rslot) == tp) {
         // one of the window's tokens: its unquantised row from the ring
@@ -418,20 +469,196 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
       it.next();
       ++n;
     }
-  } else if (warp >= 4 && warp < 4 + kSW) {
-    // ============================================================ softmax + epilogue
-    // M = 128: warp 4 + q reads TMEM lane quarter q = rows 32q .. 32q+31 (query q of the
-    // unit).  M = 64: rows 16q .. 16q+15 sit in lanes 0..15 of quarter q; lanes 16..31 of
-    // the warp shadow them (they run the same code for the warp-wide instructions and
-    // store nothing).
-    // With M = 64 the shadow lanes take the second half of each tile's tokens of their
-    // row (the scores come over by a shuffle), so both halves of a warp work.
+  } else if (ROWS == 32 && (warp & 2) == 0) {
+    // ============================================================ softmax + epilogue, 32 rows
+    // Rows 16q .. 16q+15 sit in TMEM lanes 0..15 of quarter q = warp & 1 (M = 64).  Four
+    // threads share a row: warp half = warp >> 2 and lane half hb = lane >> 4 take tokens
+    // 32 hb + 16 half + [0, 16) of each tile (one 16x32bx2 TMEM load).  The row's running
+    // max is common to the four (a shuffle, then an exchange with the other warp of the
+    // quarter through shared memory); each keeps its own partial sum.
+    const int q = warp & 1, half = warp >> 2, hb = lane >> 4;
+    const int r = 16 * q + (lane & 15);
+    const int tb = 32 * hb + 16 * half;          // this thread's first token of a tile
+    const int sidx = 64 * half + 32 * q + lane;  // 0..127 over the four warps
+    const bool valid_row = r < a.rows;
+    const int hd = r % a.H;
+    const int n_kv = R / 8;
+    const int g = hd / (a.H / n_kv);
+    float* xmax = reinterpret_cast<float*>(sbase + a.off_misc + 16);   // [2][2][2][16]
+    float* xsum = xmax + 128;                                           // [2][2][16]
+    TileIter it;
+    it.init(&a.sched, w);
+    int n = 0, u = 0;
+    bool ok = true;
+    float m = -INFINITY, l = 0.f;
+    float qr[8];
+    int p_row = -1;
+    auto wwait = [&](uint32_t bar, int parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, lim));
+    };
+    while (ok && it.valid()) {
+      const bool first = it.first_of_piece();
+      const int pc = it.pc;
+      if (first) {
+        const int bseq = it.v / a.nqb, i = (it.v % a.nqb) * a.qper + r / a.H;
+        p_row = -1;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) qr[j] = 0.f;
+        if (r < a.rows && i < a.q_chunk) {
+          p_row = __ldg(a.seq_lens + bseq) - a.q_chunk + i;
+          const float4* src = reinterpret_cast<const float4*>(a.qrope + (((size_t)bseq * a.q_chunk + i) * a.H + hd) * 8);
+          const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
+          qr[0] = x0.x; qr[1] = x0.y; qr[2] = x0.z; qr[3] = x0.w;
+          qr[4] = x1.x; qr[5] = x1.y; qr[6] = x1.z; qr[7] = x1.w;
+        }
+        m = -INFINITY;
+        l = 0.f;
+      }
+      const int sb = n & 1, pb = n & 1, ks = n % a.NK;
+      ok = wwait(bars.s_full(sb), (n >> 1) & 1);
+      if (ok) ok = wwait(bars.k_full(ks), (n / a.NK) & 1);   // the RoPE keys of this tile
+      if (!ok) break;
+      tc_fence_after();
+      float s[16];
+      {
+        uint32_t raw[16];
+        tmem_ld16x2<32>(taddr(tmem, 32 * q, kSCol + sb * kCT + 16 * half), raw);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          asm volatile("" : "+r"(raw[e]));   // the values exist only after the wait
+          s[e] = u2f(raw[e]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.s_empty(sb));
+      // RoPE score against the tile's keys: row tt of the swizzled key stage, KV head g's chunk
+      const uint8_t* krb = sbase + a.off_k + ks * a.k_stage + (g >> 3) * kTBox;
+      const int lim_t = min(it.t1, p_row + 1) - it.t;   // tokens [0, lim_t) of the tile count
+      float mx = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const int tt = tb + t;
+        const uint4 kw = *reinterpret_cast<const uint4*>(krb + sw128(tt, g));
+        float v = s[t] + qr[0] * bf16lo(kw.x) + qr[1] * bf16hi(kw.x) + qr[2] * bf16lo(kw.y) + qr[3] * bf16hi(kw.y) +
+                  qr[4] * bf16lo(kw.z) + qr[5] * bf16hi(kw.z) + qr[6] * bf16lo(kw.w) + qr[7] * bf16hi(kw.w);
+        v = tt < lim_t ? v : -INFINITY;
+        s[t] = v;
+        mx = fmaxf(mx, v);
+      }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      {   // the other warp of this quarter holds the row's other 32 tokens
+        float* xm = xmax + (((n & 1) * 2 + q) * 2) * 16;
+        if (lane < 16) xm[half * 16 + lane] = mx;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.x_max(n & 1, q));
+        if (!wwait(bars.x_max(n & 1, q), (n >> 1) & 1)) { ok = false; break; }
+        mx = fmaxf(mx, xm[(1 - half) * 16 + (lane & 15)]);
+      }
+      // Raise the running max lazily (the four threads of a row decide alike): the TMEM
+      // loads and stores are warp-collective, so the warp rescales when any row needs it.
+      // Each warp rescales its half of O's columns; lanes 16-31 touch lanes M = 64 leaves unused.
+      const bool raise = mx > m + kTau;
+      if (__any_sync(0xffffffffu, raise)) {
+        const float al = raise ? exp2f(m - mx) : 1.f;   // m = -inf: 0
+        if (!first) {
+          const int pn = n - 1;
+          if (!wwait(bars.p_empty(pn & 1), (pn >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          for (int cc = 0; cc < dcp / 32; ++cc) {
+            const uint32_t ta = taddr(tmem, 32 * q, kOCol + half * (dcp / 2) + 16 * cc);
+            uint32_t o[16];
+            tmem_ld16(ta, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = f2u(u2f(o[k]) * al);
+            tmem_st16(ta, o);
+          }
+          tmem_wait_st();
+        }
+        if (raise) {
+          l *= al;
+          m = mx;
+        }
+      }
+      uint32_t pk[8];
+      const float mb = m == -INFINITY ? 0.f : m;   // masked scores are -inf: 2^(-inf) = 0
+#pragma unroll
+      for (int t = 0; t < 16; t += 2) {
+        const float p0 = ex2_approx(s[t] - mb), p1 = ex2_approx(s[t + 1] - mb);
+        l += p0 + p1;
+        pk[t / 2] = pack_bf16x2(p0, p1);
+      }
+      if (!QUANT && it.t1 - it.t < kCT) {
+        // latent rows past the unit's last token (stale cache rows, possibly not finite):
+        // zeroed before MMA2 multiplies them by P = 0 (MMA1 has read the stage: S is full)
+        const int nvalid = it.t1 - it.t;
+        uint8_t* C = sbase + a.off_c + (n % a.NC) * a.c_stage;
+        const int nchunk = (kCT - nvalid) * 8 * n_cbox;   // 16-byte chunks
+        for (int i = sidx; i < nchunk; i += 128) {
+          const int box = i / ((kCT - nvalid) * 8), rem = i % ((kCT - nvalid) * 8);
+          *reinterpret_cast<uint4*>(C + box * kTBox + (nvalid + rem / 8) * 128 + (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      if (n >= 2) {
+        ok = wwait(bars.p_empty(pb), ((n >> 1) - 1) & 1);
+        if (!ok) break;
+      }
+      {  // P row r, this thread's 16 tokens: chunks tb / 8 and tb / 8 + 1
+        uint8_t* prow = sbase + a.off_p + pb * kPBytes;
+        *reinterpret_cast<uint4*>(prow + sw128(r, tb / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(prow + sw128(r, tb / 8 + 1)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.p_full(pb));
+
+      if (it.last_of_piece()) {
+        // ---------------- piece epilogue: the row's partial (m, l, O)
+        float lr = l + __shfl_xor_sync(0xffffffffu, l, 16);
+        {
+          float* xs = xsum + (q * 2) * 16;
+          if (lane < 16) xs[half * 16 + lane] = lr;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bars.x_sum(q));
+          if (!wwait(bars.x_sum(q), u & 1)) { ok = false; break; }
+          lr += xs[(1 - half) * 16 + (lane & 15)];
+        }
+        if (valid_row && half == 0 && hb == 0) {
+          a.mlpart[((size_t)r * a.P + pc) * 2] = m;
+          a.mlpart[((size_t)r * a.P + pc) * 2 + 1] = lr;
+        }
+        ok = wwait(bars.o_full(), u & 1);
+        if (!ok) break;
+        tc_fence_after();
+        // this warp's half of the columns; lanes 16-31 read lanes M = 64 leaves unused
+        float* dst = a.opart + ((size_t)pc * a.rows + (valid_row ? r : 0)) * dc;
+        for (int c0 = half * (dc / 2); c0 < (half + 1) * (dc / 2); c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(taddr(tmem, 32 * q, kOCol + c0), o);
+          tmem_wait_ld();
+          if (!valid_row || hb) continue;
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<float4*>(dst + c0 + e) = make_float4(u2f(o[e]), u2f(o[e + 1]), u2f(o[e + 2]), u2f(o[e + 3]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.o_empty());
+        ++u;
+      }
+      it.next();
+      ++n;
+    }
+  } else if (ROWS == 128 && warp >= 4) {
+    // ============================================================ softmax + epilogue, 128 rows
+    // Warp 4 + q reads TMEM lane quarter q = rows 32q .. 32q+31, a row per thread.
     const int q = warp - 4;
-    const bool live = ROWS == 128 || lane < 16;
-    const int r = ROWS == 128 ? 32 * q + lane : 16 * q + (lane & 15);   // this thread's row
-    constexpr int TPL = ROWS == 32 ? kCT / 2 : kCT;                      // tokens per lane
-    const int tbase = (ROWS == 32 && lane >= 16) ? kCT / 2 : 0;          // its first token
-    const bool valid_row = live && r < a.rows;
+    const int r = 32 * q + lane;   // this thread's row
+    constexpr int TPL = kCT;       // tokens per thread
+    const bool valid_row = r < a.rows;
     const int hd = r % a.H;                  // its head; its query is r / H of the unit
     const int n_kv = R / 8;
     const int g = hd / (a.H / n_kv);         // KV head of this row's head
@@ -460,50 +687,65 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
           qr[0] = x0.x; qr[1] = x0.y; qr[2] = x0.z; qr[3] = x0.w;
           qr[4] = x1.x; qr[5] = x1.y; qr[6] = x1.z; qr[7] = x1.w;
         }
+        if (rtc) {
+          // this row's RoPE query (bf16) into its KV head's 16-byte chunk of the block-diagonal
+          // operand, once MMA1 of the previous piece has read it
+          if (u > 0 && !wwait(bars.q_empty(), (u - 1) & 1)) { ok = false; break; }
+          if (valid_row)
+            *reinterpret_cast<uint4*>(sbase + a.off_ar + (g >> 3) * kQBox + sw128(r, g & 7)) =
+                make_uint4(pack_bf16x2(qr[0], qr[1]), pack_bf16x2(qr[2], qr[3]), pack_bf16x2(qr[4], qr[5]),
+                           pack_bf16x2(qr[6], qr[7]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bars.q_full());
+        }
         m = -INFINITY;
         l = 0.f;
       }
-      const int sb = n & 1, pb = n & 1, cs = n % a.NC;
+      const int sb = n & 1, pb = n & 1, ks = n % a.NK;
       ok = wwait(bars.s_full(sb), (n >> 1) & 1);
-      if (ok) ok = wwait(bars.c_full(cs), (n / a.NC) & 1);   // the RoPE keys of this tile
+      if (ok && !rtc) ok = wwait(bars.k_full(ks), (n / a.NK) & 1);   // the RoPE keys of this tile
       if (!ok) break;
       tc_fence_after();
       float s[kCT];
       {
-        uint32_t raw[16];
+        uint32_t raw[kCT];
 #pragma unroll
-        for (int k = 0; k < kCT / 16; ++k) {
-          tmem_ld16(taddr(tmem, 32 * q, kSCol + sb * kCT + 16 * k), raw);
-          tmem_wait_ld();
+        for (int k = 0; k < kCT / 16; ++k)
+          tmem_ld16(taddr(tmem, 32 * q, kSCol + sb * kCT + 16 * k), *reinterpret_cast<uint32_t(*)[16]>(raw + 16 * k));
+        tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) s[16 * k + e] = u2f(raw[e]);
+        for (int e = 0; e < kCT; ++e) {
+          asm volatile("" : "+r"(raw[e]));   // the values exist only after the wait
+          s[e] = u2f(raw[e]);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.s_empty(sb));
-      if (ROWS == 32) {   // the shadow lane takes tokens 32..63 of its row
-#pragma unroll
-        for (int t = 0; t < kCT / 2; ++t) {
-          const float hi = __shfl_xor_sync(0xffffffffu, s[kCT / 2 + t], 16);
-          if (lane >= 16) s[t] = hi;
-        }
-      }
-      // RoPE score against the tile's keys: row tt of the swizzled stage, KV head g's chunk
-      const uint8_t* krb = sbase + a.off_stage + cs * a.stage_bytes + (n_cbox + (g >> 3)) * kTBox;
       const int lim_t = min(it.t1, p_row + 1) - it.t;   // tokens [0, lim_t) of the tile count
       float mx = -INFINITY;
+      if (rtc) {
 #pragma unroll
-      for (int t = 0; t < TPL; ++t) {
-        const int tt = tbase + t;
-        const uint4 kw = *reinterpret_cast<const uint4*>(krb + tt * 128 + (((g & 7) ^ (tt & 7)) << 4));
-        float v = s[t] + qr[0] * bf16lo(kw.x) + qr[1] * bf16hi(kw.x) + qr[2] * bf16lo(kw.y) + qr[3] * bf16hi(kw.y) +
-                  qr[4] * bf16lo(kw.z) + qr[5] * bf16hi(kw.z) + qr[6] * bf16lo(kw.w) + qr[7] * bf16hi(kw.w);
-        v = tt < lim_t ? v : -INFINITY;
-        s[t] = v;
-        mx = fmaxf(mx, v);
+        for (int t = 0; t < TPL; ++t) {
+          const float v = t < lim_t ? s[t] : -INFINITY;
+          s[t] = v;
+          mx = fmaxf(mx, v);
+        }
+      } else {
+        // RoPE score against the tile's keys: row tt of the swizzled stage, KV head g's chunk
+        const uint8_t* krb = sbase + a.off_k + ks * a.k_stage + (g >> 3) * kTBox;
+#pragma unroll
+        for (int t = 0; t < TPL; ++t) {
+          const int tt = t;
+          const uint4 kw = *reinterpret_cast<const uint4*>(krb + sw128(tt, g));
+          float v = s[t] + qr[0] * bf16lo(kw.x) + qr[1] * bf16hi(kw.x) + qr[2] * bf16lo(kw.y) + qr[3] * bf16hi(kw.y) +
+                    qr[4] * bf16lo(kw.z) + qr[5] * bf16hi(kw.z) + qr[6] * bf16lo(kw.w) + qr[7] * bf16hi(kw.w);
+          v = tt < lim_t ? v : -INFINITY;
+          s[t] = v;
+          mx = fmaxf(mx, v);
+        }
       }
-      if (ROWS == 32) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       // Raise the running max lazily: a row rescales when its max grew by more than kTau.
       // Rows decide on their own, but the TMEM loads and stores (and the wait before them)
       // are warp-collective, so the warp takes the branch when any of its rows needs it and
@@ -533,20 +775,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         }
       }
       uint32_t pk[TPL / 2];
+      const float mb = m == -INFINITY ? 0.f : m;   // masked scores are -inf: 2^(-inf) = 0
 #pragma unroll
-      for (int t = 0; t < TPL; t += 2) {   // l: this lane's tokens (the pair adds up at the end)
-        const float p0 = tbase + t < lim_t ? exp2f(s[t] - m) : 0.f;
-        const float p1 = tbase + t + 1 < lim_t ? exp2f(s[t + 1] - m) : 0.f;
+      for (int t = 0; t < TPL; t += 2) {
+        const float p0 = ex2_approx(s[t] - mb), p1 = ex2_approx(s[t + 1] - mb);
         l += p0 + p1;
         pk[t / 2] = pack_bf16x2(p0, p1);
       }
       if (!QUANT && it.t1 - it.t < kCT) {
         // latent rows past the unit's last token (stale cache rows, possibly not finite):
-        // zeroed before MMA2 multiplies them by P = 0
+        // zeroed before MMA2 multiplies them by P = 0 (MMA1 has read the stage: S is full)
         const int nvalid = it.t1 - it.t;
-        uint8_t* C = sbase + a.off_stage + cs * a.stage_bytes;
+        uint8_t* C = sbase + a.off_c + (n % a.NC) * a.c_stage;
         const int nchunk = (kCT - nvalid) * 8 * n_cbox;   // 16-byte chunks
-        for (int i = r; live && i < nchunk; i += ROWS) {
+        for (int i = r; i < nchunk; i += ROWS) {
           const int box = i / ((kCT - nvalid) * 8), rem = i % ((kCT - nvalid) * 8);
           *reinterpret_cast<uint4*>(C + box * kTBox + (nvalid + rem / 8) * 128 + (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
         }
@@ -555,14 +797,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         ok = wwait(bars.p_empty(pb), ((n >> 1) - 1) & 1);
         if (!ok) break;
       }
-      {  // P row r: 64 tokens = 128 B, 16-byte chunk c at (c ^ (r % 8)); each lane its tokens
-        uint8_t* prow = sbase + a.off_p + pb * kPBytes + r * 128;
+      {  // P row r: 64 tokens = 128 B, 16-byte chunk c at (c ^ (r % 8))
+        uint8_t* prow = sbase + a.off_p + pb * kPBytes;
 #pragma unroll
-        for (int c = 0; c < TPL / 8; ++c) {
-          const int cc = tbase / 8 + c;
-          *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
+        for (int c = 0; c < TPL / 8; ++c)
+          *reinterpret_cast<uint4*>(prow + sw128(r, c)) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -571,7 +811,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
 
       if (it.last_of_piece()) {
         // ---------------- piece epilogue: this row's partial (m, l, O)
-        if (ROWS == 32) l += __shfl_xor_sync(0xffffffffu, l, 16);   // the two token halves
         if (valid_row) {
           a.mlpart[((size_t)r * a.P + pc) * 2] = m;
           a.mlpart[((size_t)r * a.P + pc) * 2 + 1] = l;
@@ -606,7 +845,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == GG::MMA) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -645,39 +884,68 @@ static bool map_bf16_sw128(CUtensorMap* m, const void* base, uint64_t cols, uint
 }
 
 struct ChunkLayoutSmem {
-  int NC, NRAW;
-  uint32_t off_q, off_stage, off_p, off_raw, off_bar, off_misc, stage_bytes, raw_stage, total;
+  int NC, NK, NRAW;
+  bool rtc;
+  uint32_t off_q, off_ar, off_p, off_c, off_k, off_raw, off_bar, off_misc, c_stage, k_stage, raw_stage, total;
 };
 
-// Shared memory: [Q_lat boxes][P buffers][stages][raw ring][barriers][misc].  With M = 64
-// the A operands' rows 32..63 read the 4 KB after each 32-row box: Q's last box runs into
-// P0, P1 into stage 0, all inside the allocation.
-static ChunkLayoutSmem chunk_smem(int dc, int R, int qbits, int rows) {
+// Shared memory: [Q_lat boxes][RoPE query boxes][P buffers][latent ring][RoPE-key ring]
+// [code ring][barriers][misc].  With M = 64 the A operands' rows 32..63 read the 4 KB after
+// each 32-row box (the next box, P0, or the first latent stage), all inside the allocation.
+// The rings take what is left: with the RoPE scores on the tensor cores the key ring holds a
+// tile only until MMA1 and the latent ring until MMA2, so stages go to the latent ring
+// first; otherwise a tile holds a stage of each until MMA2 and the rings grow together.
+static ChunkLayoutSmem chunk_smem_rtc(int dc, int R, int qbits, int rows, bool rtc) {
   const uint32_t budget = 232448 - 1024;
   const int dcp = (dc + 63) / 64 * 64;
+  const int n_cbox = dcp / 64, n_kbox = (R + 63) / 64;
   ChunkLayoutSmem L{};
-  L.stage_bytes = (uint32_t)(dcp / 64 + (R + 63) / 64) * kTBox;
+  L.rtc = rtc;
+  L.c_stage = (uint32_t)n_cbox * kTBox;
+  L.k_stage = (uint32_t)n_kbox * kTBox;
   L.raw_stage = qbits ? (((uint32_t)kCT * (dc * qbits / 8)) + 127) & ~127u : 0;
-  const int nraw = qbits ? 3 : 0;
+  L.NRAW = qbits ? 3 : 0;
   const uint32_t box = (uint32_t)rows * 128u;
-  const uint32_t q_bytes = (uint32_t)(dcp / 64) * box;
-  auto size = [&](int nc) {
-    return q_bytes + nc * L.stage_bytes + 2 * box + nraw * L.raw_stage + 8 * (2 * nc + 2 * nraw + kFixedBars) + 256;
+  const uint32_t fixed = (uint32_t)(n_cbox + (rtc ? n_kbox : 0)) * box + 2 * box + L.NRAW * L.raw_stage;
+  auto size = [&](int nc, int nk) {
+    return fixed + nc * L.c_stage + nk * L.k_stage + 8 * (2 * nc + 2 * nk + 2 * L.NRAW + kFixedBars) + 16 + kXchgBytes + 256;
   };
-  int nc = 2;
-  while (nc < 6 && size(nc + 1) <= budget) ++nc;
+  int nc = 2, nk = 2;
+  if (!rtc) {   // a tile holds both until MMA2: the rings grow together
+    while (nc < 6 && size(nc + 1, nk + 1) <= budget) { ++nc; ++nk; }
+  } else {
+    while (true) {
+      if (nc <= nk && nc < 6 && size(nc + 1, nk) <= budget) { ++nc; continue; }
+      if (nk < nc && nk < 6 && size(nc, nk + 1) <= budget) { ++nk; continue; }
+      if (nc < 6 && size(nc + 1, nk) <= budget) { ++nc; continue; }
+      break;
+    }
+  }
   L.NC = nc;
-  L.NRAW = nraw;
+  L.NK = nk;
   uint32_t o = 0;
-  L.off_q = o; o += q_bytes;
+  L.off_q = o; o += (uint32_t)n_cbox * box;
+  L.off_ar = o; o += rtc ? (uint32_t)n_kbox * box : 0;
   L.off_p = o; o += 2 * box;
-  L.off_stage = o; o += nc * L.stage_bytes;
-  L.off_raw = o; o += nraw * L.raw_stage;
-  L.off_bar = o; o += 8 * (2 * nc + 2 * nraw + kFixedBars);
+  L.off_c = o; o += nc * L.c_stage;
+  L.off_k = o; o += nk * L.k_stage;
+  L.off_raw = o; o += L.NRAW * L.raw_stage;
+  L.off_bar = o; o += 8 * (2 * nc + 2 * nk + 2 * L.NRAW + kFixedBars);
   o = (o + 15) & ~15u;
-  L.off_misc = o; o += sizeof(Misc);
+  L.off_misc = o; o += 16 + kXchgBytes;
   L.total = o + 1024;
   return L;
+}
+
+// The RoPE scores of a 128-row unit go to the tensor cores (block-diagonal query rows in
+// MMA1) when their operand leaves room for at least three latent and two key stages; else,
+// and always for 32 rows (whose MMA1 would double on mostly zero rows while only two
+// softmax warps share the CUDA-core form), the softmax warps compute them from the key stage.
+static ChunkLayoutSmem chunk_smem(int dc, int R, int qbits, int rows) {
+  if (rows == 32) return chunk_smem_rtc(dc, R, qbits, rows, false);
+  const ChunkLayoutSmem t = chunk_smem_rtc(dc, R, qbits, rows, true);
+  if (t.total <= 232448 && t.NC >= 3 && t.NK >= 2) return t;
+  return chunk_smem_rtc(dc, R, qbits, rows, false);
 }
 
 }  // namespace chunk
@@ -752,9 +1020,11 @@ cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const i
   a.sched = sched; a.seq_lens = seq_lens; a.qrope = qrope; a.opart = opart; a.mlpart = mlpart;
   a.cache = c; a.err = p.err;
   a.wait_ns = (uint64_t)p.opt_wait_us * 1000u;
-  a.NC = L.NC; a.NRAW = L.NRAW;
-  a.off_q = L.off_q; a.off_stage = L.off_stage; a.off_p = L.off_p; a.off_bar = L.off_bar; a.off_misc = L.off_misc;
-  a.stage_bytes = L.stage_bytes; a.off_raw = L.off_raw; a.raw_stage = L.raw_stage;
+  a.rtc = L.rtc ? 1 : 0;
+  a.NC = L.NC; a.NK = L.NK; a.NRAW = L.NRAW;
+  a.off_q = L.off_q; a.off_ar = L.off_ar; a.off_p = L.off_p; a.off_c = L.off_c; a.off_k = L.off_k;
+  a.off_raw = L.off_raw; a.off_bar = L.off_bar; a.off_misc = L.off_misc;
+  a.c_stage = L.c_stage; a.k_stage = L.k_stage; a.raw_stage = L.raw_stage;
   const bool paged = c.block_table != nullptr, resid = qbits == 4 && c.c_resid != nullptr;
   decltype(&attn_tc_kernel<128, 0, false, false>) kern;
   if (rows == 128)
