@@ -320,13 +320,9 @@ class Bench:
         self.ws = workspace(plan, B, dev)
         self.stream = torch.cuda.current_stream(dev)
 
-        # which split-K kernel runs: the tcgen05 kernel where the shape allows it
-        kernel_used = kernel
-        if kernel_used == 0:
-            mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, 2)
-            st = mla.mla_decode(plan, caches[0].struct, self.seq_lens, self.q, self.out, self.ws,
-                                stream=self.stream, check=False)
-            kernel_used = 2 if st == mla.MLA_OK else 1
+        # which split-K attention kernel runs (the library's automatic choice unless forced)
+        mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, kernel)
+        kernel_used = mla.mla_decode_kernel_choice(plan, caches[0].struct)
         self.kernel_used = kernel_used
         mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, kernel_used)
         torch.cuda.synchronize()

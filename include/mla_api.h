@@ -134,9 +134,10 @@ typedef struct mla_plan mla_plan_t;   /* opaque, created by mla_plan_create */
 
 /* Options for mla_plan_set_option. */
 enum {
-  MLA_OPT_DECODE_KERNEL = 1,  /* 0 auto, 1 CUDA-core split-K kernel, 2 tcgen05 kernel with a
-                                 token per softmax thread, 3 tcgen05 kernel with a head per
-                                 softmax thread (the query-chunk kernel's form, one query) */
+  MLA_OPT_DECODE_KERNEL = 1,  /* 0 auto (see mla_decode_kernel_choice), 1 CUDA-core split-K
+                                 kernel, 2 tcgen05 kernel with a token per softmax thread,
+                                 3 tcgen05 kernel with a head per softmax thread (the
+                                 query-chunk kernel's form, one query) */
   MLA_OPT_DECODE_SPLITS = 2,  /* 0 auto (SM count based); n > 0: split the context
                                  tiles into n contiguous worker ranges */
   MLA_OPT_PROFILE_EVENTS = 3, /* value: address of a host array of two cudaEvent_t; each
@@ -239,6 +240,15 @@ MLA_API mla_status_t mla_append(const mla_plan_t* plan, const void* x, const int
  * of B sequences (bytes, 256-aligned; it includes the host variant's staging of the step's
  * inputs and output). */
 MLA_API size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B);
+
+/* The attention kernel mla_decode runs for this plan and cache under the plan's
+ * MLA_OPT_DECODE_KERNEL setting: *kernel = 1 (CUDA cores), 2 (tcgen05, a token per softmax
+ * thread) or 3 (tcgen05, a head per softmax thread), the option's own numbering.  Automatic
+ * choice (option 0): a bf16 latent cache on kernel 3 where its shapes allow, a quantised
+ * one on kernel 2 where its shapes allow, else kernel 3, else kernel 1.  Host only; no
+ * device work.  Returns MLA_ERR_UNSUPPORTED where the forced kernel cannot run the shape,
+ * MLA_ERR_INVALID_ARG for null arguments. */
+MLA_API mla_status_t mla_decode_kernel_choice(const mla_plan_t* plan, const mla_cache_t* cache, int32_t* kernel);
 
 /* One decode step: attention of each sequence's new query over its cached tokens
  * [0, seq_lens[b]).  The query sits at position seq_lens[b]-1 (append it first).

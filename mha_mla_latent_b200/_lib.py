@@ -29,7 +29,7 @@ EXPORTED = (
     "mla_plan_create", "mla_plan_destroy", "mla_plan_set_option", "mla_append",
     "mla_decode_workspace_bytes", "mla_decode", "mla_device_error", "mla_decode_noalloc",
     "mla_fixed_pairs", "mla_decode_step", "mla_decode_step_host", "mla_decode_chunk",
-    "mla_decode_chunk_workspace_bytes",
+    "mla_decode_chunk_workspace_bytes", "mla_decode_kernel_choice",
 )
 MLA_PAIRS_FULL, MLA_PAIRS_HIGH, MLA_PAIRS_UNIFORM, MLA_PAIRS_LOW = 0, 1, 2, 5
 MLA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -73,6 +73,7 @@ def _load():
         "mla_plan_set_option": (i32, [vp, i32, i64]),
         "mla_append": (i32, [vp, vp, vp, vp, i32, cachep, vp]),
         "mla_decode_workspace_bytes": (sz, [vp, i32]),
+        "mla_decode_kernel_choice": (i32, [vp, cachep, ctypes.POINTER(i32)]),
         "mla_decode": (i32, [vp, cachep, vp, vp, i32, vp, vp, sz, vp]),
         "mla_device_error": (i32, [vp, ctypes.POINTER(i32)]),
         "mla_decode_noalloc": (i32, [vp, cachep, vp, vp, i32, vp, vp]),
@@ -224,6 +225,13 @@ def mla_append(plan: Plan, x, seq_idx, pos, cache: MlaCache, stream=None, check=
 
 def mla_decode_workspace_bytes(plan: Plan, B: int) -> int:
     return int(_lib.mla_decode_workspace_bytes(plan.handle, int(B)))
+
+
+def mla_decode_kernel_choice(plan: Plan, cache: MlaCache) -> int:
+    """The attention kernel mla_decode runs (1, 2 or 3, MLA_OPT_DECODE_KERNEL numbering)."""
+    k = ctypes.c_int32(0)
+    _check(_lib.mla_decode_kernel_choice(plan.handle, ctypes.byref(cache), ctypes.byref(k)), "mla_decode_kernel_choice")
+    return int(k.value)
 
 
 def mla_decode(plan: Plan, cache: MlaCache, seq_lens, q, out, workspace, stream=None, check=True):

@@ -143,6 +143,38 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// s + sum_j q[j] k[j] over one KV head's 8 RoPE dims (k: 8 bf16), in pairs of lanes of the
+// packed f32x2 FMA: (even dims, odd dims) accumulate apart and add at the end.
+__device__ __forceinline__ float rope_dot8(float s, const float (&q)[8], uint4 kw) {
+  const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
+  uint64_t acc;
+  {
+    const float2 a0 = make_float2(s, 0.f);
+    acc = *reinterpret_cast<const uint64_t*>(&a0);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 kk = make_float2(bf16lo(w[i]), bf16hi(w[i]));
+    const float2 qq = make_float2(q[2 * i], q[2 * i + 1]);
+    asm("fma.rn.f32x2 %0, %1, %2, %0;"
+        : "+l"(acc)
+        : "l"(*reinterpret_cast<const uint64_t*>(&qq)), "l"(*reinterpret_cast<const uint64_t*>(&kk)));
+  }
+  const float2 r = *reinterpret_cast<const float2*>(&acc);
+  return r.x + r.y;
+}
+
+// Two's-complement 4-bit code (in the low nibble) to float without a conversion
+// instruction: the offset code (n ^ 8) goes into the mantissa of 2^23, whose value then
+// exceeds 2^23 + 8 by exactly the code.
+__device__ __forceinline__ float nib_to_float(uint32_t n) {
+  return __uint_as_float(0x4B000000u | ((n ^ 8u) & 15u)) - 8388616.0f;
+}
+// The same for a 2-bit code (n ^ 2 is the offset code; 2^23 + 2 its zero).
+__device__ __forceinline__ float crumb_to_float(uint32_t n) {
+  return __uint_as_float(0x4B000000u | ((n ^ 2u) & 3u)) - 8388610.0f;
+}
+
 template <bool PAGED>
 __device__ __forceinline__ MlaLoc chunk_loc(const ChunkArgs& a, int b, int t) {
   if (!PAGED) return MlaLoc{b, t, a.T_cap};
@@ -388,20 +420,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
     int n = 0;
     bool ok = true;
     int lo_v = -1, lo = INT_MAX;   // residual window (decode): tokens from lo on may sit in the ring
+    // this token's group scales (up to 8 per token) come from global memory with plain loads,
+    // issued two tiles ahead so their latency hides behind the dequantisation of two tiles
+    auto load_scales = [&](const TileIter& ti, __half (&sc)[8]) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) sc[j] = __float2half(0.f);
+      if (!ti.valid() || tok >= ti.t1 - ti.t) return;
+      const MlaLoc lc = chunk_loc<PAGED>(a, ti.v / a.nqb, ti.t);
+      const __half* sp = a.scales + ((size_t)lc.pb * lc.cap + lc.pt + tok) * (dc / 32);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j < dc / 32) sc[j] = __ldg(sp + j);
+    };
+    TileIter pf = it;
+    __half scl[8], scl1[8], scl2[8];   // tiles n, n + 1, n + 2
+    load_scales(pf, scl);
+    if (pf.valid()) pf.next();
+    load_scales(pf, scl1);
+    if (pf.valid()) pf.next();
+    load_scales(pf, scl2);
     while (ok && it.valid()) {
       const int rs = n % a.NRAW, cs = n % a.NC;
       if (RESID && it.v != lo_v) {   // once per sequence, ahead of the stage wait
         lo_v = it.v;
         lo = __ldg(a.seq_lens + it.v) - MLA_RESID_WINDOW;
-      }
-      // this token's group scales (up to 8), loaded ahead of the stage wait
-      __half scl[8];
-      {
-        const MlaLoc lc = chunk_loc<PAGED>(a, it.v / a.nqb, it.t);
-        const __half* sp = a.scales + ((size_t)lc.pb * lc.cap + lc.pt + tok) * (dc / 32);
-        const bool in = tok < it.t1 - it.t;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) scl[j] = (in && j < dc / 32) ? __ldg(sp + j) : __float2half(0.f);
       }
       ok = __all_sync(0xffffffffu, mbar_wait(bars.raw_full(rs), (n / a.NRAW) & 1, abort_flag, lim));
       if (ok && n >= a.NC)
@@ -436,7 +478,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 const uint32_t byte = (words[ch] >> (8 * j)) & 0xFFu;
-                o[j] = pack_bf16x2((float)nib_to_int(byte & 15u) * sv, (float)nib_to_int(byte >> 4) * sv);
+                o[j] = pack_bf16x2(nib_to_float(byte) * sv, nib_to_float(byte >> 4) * sv);
               }
               put(grp * 4 + ch, make_uint4(o[0], o[1], o[2], o[3]));
             }
@@ -448,10 +490,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
               const uint32_t bits = (words[ch >> 1] >> (16 * (ch & 1))) & 0xFFFFu;
               uint32_t o[4];
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int f0 = (int)((bits >> (4 * j)) & 3u), f1 = (int)((bits >> (4 * j + 2)) & 3u);
-                o[j] = pack_bf16x2((float)(f0 >= 2 ? f0 - 4 : f0) * sv, (float)(f1 >= 2 ? f1 - 4 : f1) * sv);
-              }
+              for (int j = 0; j < 4; ++j)
+                o[j] = pack_bf16x2(crumb_to_float(bits >> (4 * j)) * sv, crumb_to_float(bits >> (4 * j + 2)) * sv);
               put(grp * 4 + ch, make_uint4(o[0], o[1], o[2], o[3]));
             }
           }
@@ -466,6 +506,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         mbar_arrive(bars.raw_empty(rs));
         mbar_arrive(bars.c_full(cs));
       }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { scl[j] = scl1[j]; scl1[j] = scl2[j]; }
+      if (pf.valid()) pf.next();
+      load_scales(pf, scl2);
       it.next();
       ++n;
     }
@@ -537,15 +581,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
       const uint8_t* krb = sbase + a.off_k + ks * a.k_stage + (g >> 3) * kTBox;
       const int lim_t = min(it.t1, p_row + 1) - it.t;   // tokens [0, lim_t) of the tile count
       float mx = -INFINITY;
+      {
+        uint4 kw[16];   // all 16 keys in flight before the first use
 #pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        const int tt = tb + t;
-        const uint4 kw = *reinterpret_cast<const uint4*>(krb + sw128(tt, g));
-        float v = s[t] + qr[0] * bf16lo(kw.x) + qr[1] * bf16hi(kw.x) + qr[2] * bf16lo(kw.y) + qr[3] * bf16hi(kw.y) +
-                  qr[4] * bf16lo(kw.z) + qr[5] * bf16hi(kw.z) + qr[6] * bf16lo(kw.w) + qr[7] * bf16hi(kw.w);
-        v = tt < lim_t ? v : -INFINITY;
-        s[t] = v;
-        mx = fmaxf(mx, v);
+        for (int t = 0; t < 16; ++t) kw[t] = *reinterpret_cast<const uint4*>(krb + sw128(tb + t, g));
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          const int tt = tb + t;
+          float v = rope_dot8(s[t], qr, kw[t]);
+          v = tt < lim_t ? v : -INFINITY;
+          s[t] = v;
+          mx = fmaxf(mx, v);
+        }
       }
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       {   // the other warp of this quarter holds the row's other 32 tokens

@@ -77,15 +77,27 @@ void free_plan(mla_plan* p) {
 
 // The decode kernel a call runs: the tensor-core kernel where the plan, cache and options
 // allow it, else the CUDA-core kernel.  MLA_OK, or the status that refuses the call.
+// Kernel ids of the decode layout: 1 CUDA cores, 2 tcgen05 token rows, 4 tcgen05 head rows.
 mla_status_t mla_pick_decode_kernel(const mla_plan& p, const mla_cache_t& c, int* kernel) {
   *kernel = 1;
-  if (p.opt_kernel == 3) {   // the head-row tensor-core form
-    if (!mla_decode_t_supported(p, c)) return MLA_ERR_UNSUPPORTED;
-    *kernel = 4;
-    return MLA_OK;
+  const bool head_rows = mla_decode_t_supported(p, c);
+  const bool token_rows = mla_tc_kind_ok(p.cfg) && mla_tc_supported(p, c);
+  switch (p.opt_kernel) {
+    case 1: break;
+    case 2:
+      if (!token_rows) return MLA_ERR_UNSUPPORTED;
+      *kernel = 2;
+      break;
+    case 3:
+      if (!head_rows) return MLA_ERR_UNSUPPORTED;
+      *kernel = 4;
+      break;
+    default:   // bf16 latents stream fastest through the head-row kernel, quantised ones
+               // (dequantised in shared memory) through the token-row kernel
+      if (head_rows && (!mla_kind_quant(p.cfg.cache_kind) || !token_rows)) *kernel = 4;
+      else if (token_rows) *kernel = 2;
+      break;
   }
-  if (p.opt_kernel != 1 && mla_tc_kind_ok(p.cfg) && mla_tc_supported(p, c)) *kernel = 2;
-  if (p.opt_kernel == 2 && *kernel != 2) return MLA_ERR_UNSUPPORTED;
   if (*kernel == 1 && (size_t)p.cfg.n_heads * p.cfg.d_c > 8192) return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
 }
@@ -313,6 +325,15 @@ mla_status_t pick_kernel(const mla_plan& p, const mla_cache_t& c, int* kernel) {
 }
 
 }  // namespace
+
+mla_status_t mla_decode_kernel_choice(const mla_plan_t* plan, const mla_cache_t* cache, int32_t* kernel) {
+  if (!plan || !cache || !kernel) return MLA_ERR_INVALID_ARG;
+  int k = 1;
+  const mla_status_t st = mla_pick_decode_kernel(*plan, *cache, &k);
+  if (st != MLA_OK) return st;
+  *kernel = k == 4 ? 3 : k;
+  return MLA_OK;
+}
 
 size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B) {
   if (!plan || B <= 0) return 0;
