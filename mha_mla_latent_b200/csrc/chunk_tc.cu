@@ -217,7 +217,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
     misc->abort_flag = 0;
     // latent stage: its TMA bytes, or both dequantising warps; RoPE-key stage: its TMA bytes
     for (int s = 0; s < a.NC; ++s) { mbar_init(bars.c_full(s), QUANT ? 2 : 1); mbar_init(bars.c_empty(s), 1); }
-    for (int s = 0; s < a.NK; ++s) { mbar_init(bars.k_full(s), 1); mbar_init(bars.k_empty(s), 1); }
+    // a key stage is free after MMA1 (RoPE scores on the tensor cores) or after every
+    // softmax warp has read its keys
+    for (int s = 0; s < a.NK; ++s) { mbar_init(bars.k_full(s), 1); mbar_init(bars.k_empty(s), rtc ? 1 : kSW); }
     for (int s = 0; s < a.NRAW; ++s) { mbar_init(bars.raw_full(s), 1); mbar_init(bars.raw_empty(s), 2); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars.s_full(i), 1);
@@ -263,59 +265,85 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
   if (warp == GG::PROD) {
     // ============================================================ TMA producer (lane 0)
     if (lane == 0) {
-      TileIter it;
-      it.init(&a.sched, w);
-      int n = 0, u = 0, q_loads = 0, last = -1;
+      // Two cursors over the CTA's tiles: the latent (or code) ring with the query boxes, and
+      // the RoPE-key ring, whose stages free up at different times; each copy is issued as
+      // soon as its stage is free.
+      TileIter ic, ik;
+      ic.init(&a.sched, w);
+      ik = ic;
+      int nc = 0, nk = 0, u = 0, q_loads = 0;
       bool ok = true;
-      while (ok && it.valid()) {
-        if (it.first_of_piece()) {
-          if (u > 0 && !mbar_wait(bars.q_empty(), (u - 1) & 1, abort_flag, lim)) { ok = false; break; }
-          mbar_expect_tx(bars.q_full(), (uint32_t)n_cbox * kQBox);
-          for (int kb = 0; kb < n_cbox; ++kb)
-            tma_load_2d(sbase_u32 + a.off_q + kb * kQBox, &tm_q, bars.q_full(), kb * 64, qrow0(it.v));
-          ++q_loads;
+      uint64_t t_idle = globaltimer();
+      while (ic.valid() || ik.valid()) {
+        bool progress = false;
+        if (ic.valid()) {
+          const int cs = nc % a.NC, rs = QUANT ? nc % a.NRAW : 0;
+          const bool q_ok = !ic.first_of_piece() || u == 0 || mbar_test(bars.q_empty(), (u - 1) & 1);
+          const bool slot_ok = QUANT ? (nc < a.NRAW || mbar_test(bars.raw_empty(rs), ((nc / a.NRAW) - 1) & 1))
+                                     : (nc < a.NC || mbar_test(bars.c_empty(cs), ((nc / a.NC) - 1) & 1));
+          if (q_ok && slot_ok) {
+            if (ic.first_of_piece()) {
+              mbar_expect_tx(bars.q_full(), (uint32_t)n_cbox * kQBox);
+              for (int kb = 0; kb < n_cbox; ++kb)
+                tma_load_2d(sbase_u32 + a.off_q + kb * kQBox, &tm_q, bars.q_full(), kb * 64, qrow0(ic.v));
+              ++q_loads;
+            }
+            const MlaLoc lc = chunk_loc<PAGED>(a, ic.v / a.nqb, ic.t);   // a 64-token tile lies in one block
+            const int row = lc.pb * lc.cap + lc.pt;
+            if (!QUANT) {   // latent boxes
+              const uint32_t st = sbase_u32 + a.off_c + cs * a.c_stage;
+              mbar_expect_tx(bars.c_full(cs), (uint32_t)n_cbox * kTBox);
+              for (int kb = 0; kb < n_cbox; ++kb) tma_load_2d(st + kb * kTBox, &tm_c, bars.c_full(cs), kb * 64, row);
+            } else {        // code rows (one box of 64 rows) into the raw ring
+              const uint32_t rb = sbase_u32 + a.off_raw + rs * a.raw_stage;
+              mbar_expect_tx(bars.raw_full(rs), (uint32_t)kCT * a.code_row);
+              tma_load_2d(rb, &tm_c, bars.raw_full(rs), 0, row);
+            }
+            if (ic.last_of_piece()) ++u;
+            ic.next();
+            ++nc;
+            progress = true;
+          }
         }
-        const int cs = n % a.NC, ks = n % a.NK, rs = QUANT ? n % a.NRAW : 0;
-        const MlaLoc lc = chunk_loc<PAGED>(a, it.v / a.nqb, it.t);   // a 64-token tile lies in one block
-        const int row = lc.pb * lc.cap + lc.pt;
-        if (!QUANT) {   // latent boxes
-          if (n >= a.NC && !mbar_wait(bars.c_empty(cs), ((n / a.NC) - 1) & 1, abort_flag, lim)) { ok = false; break; }
-          const uint32_t st = sbase_u32 + a.off_c + cs * a.c_stage;
-          mbar_expect_tx(bars.c_full(cs), (uint32_t)n_cbox * kTBox);
-          for (int kb = 0; kb < n_cbox; ++kb) tma_load_2d(st + kb * kTBox, &tm_c, bars.c_full(cs), kb * 64, row);
-        } else {        // code rows (one box of 64 rows) into the raw ring
-          if (n >= a.NRAW && !mbar_wait(bars.raw_empty(rs), ((n / a.NRAW) - 1) & 1, abort_flag, lim)) {
+        if (ik.valid() && nk < nc) {   // keys never run ahead of their tile's latent copy
+          const int ks = nk % a.NK;
+          if (nk < a.NK || mbar_test(bars.k_empty(ks), ((nk / a.NK) - 1) & 1)) {
+            const MlaLoc lc = chunk_loc<PAGED>(a, ik.v / a.nqb, ik.t);
+            const int row = lc.pb * lc.cap + lc.pt;
+            const uint32_t st = sbase_u32 + a.off_k + ks * a.k_stage;
+            mbar_expect_tx(bars.k_full(ks), (uint32_t)n_kbox * kTBox);
+            for (int kb = 0; kb < n_kbox; ++kb) tma_load_2d(st + kb * kTBox, &tm_kr, bars.k_full(ks), kb * 64, row);
+            ik.next();
+            ++nk;
+            progress = true;
+          }
+        }
+        if (progress) {
+          t_idle = globaltimer();
+        } else {
+          if (*abort_flag || globaltimer() - t_idle > lim) {
+            *abort_flag = 1;
             ok = false;
             break;
           }
-          const uint32_t rb = sbase_u32 + a.off_raw + rs * a.raw_stage;
-          mbar_expect_tx(bars.raw_full(rs), (uint32_t)kCT * a.code_row);
-          tma_load_2d(rb, &tm_c, bars.raw_full(rs), 0, row);
+          __nanosleep(32);
         }
-        {   // RoPE-key boxes
-          if (n >= a.NK && !mbar_wait(bars.k_empty(ks), ((n / a.NK) - 1) & 1, abort_flag, lim)) { ok = false; break; }
-          const uint32_t st = sbase_u32 + a.off_k + ks * a.k_stage;
-          mbar_expect_tx(bars.k_full(ks), (uint32_t)n_kbox * kTBox);
-          for (int kb = 0; kb < n_kbox; ++kb) tma_load_2d(st + kb * kTBox, &tm_kr, bars.k_full(ks), kb * 64, row);
-        }
-        last = n;
-        if (it.last_of_piece()) ++u;
-        it.next();
-        ++n;
       }
-      // drain: every issued copy lands before the CTA exits (a copy that was not issued
-      // because its wait gave up leaves its barrier one phase behind: skipped by `last`)
+      (void)ok;
+      // drain: every issued copy lands before the CTA exits (copies not issued because the
+      // wait gave up are not waited for)
       volatile int never = 0;
       if (q_loads > 0) mbar_wait(bars.q_full(), (q_loads - 1) & 1, &never, lim);
-      auto drain = [&](int NS, auto bar) {
+      auto drain = [&](int NS, int issued, auto bar) {
+        const int last = issued - 1;
         for (int s = 0; s < NS; ++s) {
           const int k = last - ((last - s) % NS + NS) % NS;
           if (last >= 0 && k >= 0) mbar_wait(bar(s), (k / NS) & 1, &never, lim);
         }
       };
-      if (!QUANT) drain(a.NC, [&](int s) { return bars.c_full(s); });
-      else drain(a.NRAW, [&](int s) { return bars.raw_full(s); });
-      drain(a.NK, [&](int s) { return bars.k_full(s); });
+      if (!QUANT) drain(a.NC, nc, [&](int s) { return bars.c_full(s); });
+      else drain(a.NRAW, nc, [&](int s) { return bars.raw_full(s); });
+      drain(a.NK, nk, [&](int s) { return bars.k_full(s); });
     }
   } else if (warp == GG::MMA) {
     // ============================================================ MMA issuer
@@ -344,7 +372,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         }
         tc_commit(bars.p_empty(pb));
         tc_commit(bars.c_empty(cs));
-        if (!rtc) tc_commit(bars.k_empty(pn % a.NK));   // the softmax warps have read the keys
         if (lastp) tc_commit(bars.o_full());
         return true;
       };
@@ -362,7 +389,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
             }
             if ((n < 2 || mbar_test(bars.s_empty(sb), ((n >> 1) - 1) & 1)) &&
                 (!first || mbar_test(bars.q_full(), u & 1)) && mbar_test(bars.c_full(cs), (n / a.NC) & 1) &&
-                mbar_test(bars.k_full(ks), (n / a.NK) & 1))
+                (!rtc || mbar_test(bars.k_full(ks), (n / a.NK) & 1)))   // MMA1 reads keys only with rtc
               break;
             if (*abort_flag || globaltimer() - t_start > lim) {
               *abort_flag = 1;
@@ -465,10 +492,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         for (int j = 0; j < dc / 8; ++j) put(j, __ldg(src + j));
       } else if (tok < nvalid) {
         const uint8_t* codes = raw + tok * a.code_row;
+        float svs[8];
 #pragma unroll
-        for (int grp = 0; grp < 8; ++grp) {   // 32 values, one scale
-          if (grp >= dc / 32) break;
-          const float sv = __half2float(scl[grp]);
+        for (int j = 0; j < 8; ++j) svs[j] = __half2float(scl[j]);
+#pragma unroll 1
+        for (int grp = 0; grp < dc / 32; ++grp) {   // 32 values, one scale (a loop: code size)
+          float sv = svs[0];
+#pragma unroll
+          for (int j = 1; j < 8; ++j) sv = grp == j ? svs[j] : sv;
           if (QB == 4) {   // two's-complement nibbles, element 2i in the low nibble of byte i
             const uint4 cw = *reinterpret_cast<const uint4*>(codes + grp * 16);
             const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
@@ -585,6 +616,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         uint4 kw[16];   // all 16 keys in flight before the first use
 #pragma unroll
         for (int t = 0; t < 16; ++t) kw[t] = *reinterpret_cast<const uint4*>(krb + sw128(tb + t, g));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.k_empty(ks));   // the keys are in registers
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
           const int tt = tb + t;
@@ -786,12 +819,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         for (int t = 0; t < TPL; ++t) {
           const int tt = t;
           const uint4 kw = *reinterpret_cast<const uint4*>(krb + sw128(tt, g));
-          float v = s[t] + qr[0] * bf16lo(kw.x) + qr[1] * bf16hi(kw.x) + qr[2] * bf16lo(kw.y) + qr[3] * bf16hi(kw.y) +
-                    qr[4] * bf16lo(kw.z) + qr[5] * bf16hi(kw.z) + qr[6] * bf16lo(kw.w) + qr[7] * bf16hi(kw.w);
+          float v = rope_dot8(s[t], qr, kw);
           v = tt < lim_t ? v : -INFINITY;
           s[t] = v;
           mx = fmaxf(mx, v);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.k_empty(ks));   // this warp has read its keys
       }
       // Raise the running max lazily: a row rescales when its max grew by more than kTau.
       // Rows decide on their own, but the TMEM loads and stores (and the wait before them)
@@ -939,9 +973,9 @@ struct ChunkLayoutSmem {
 // Shared memory: [Q_lat boxes][RoPE query boxes][P buffers][latent ring][RoPE-key ring]
 // [code ring][barriers][misc].  With M = 64 the A operands' rows 32..63 read the 4 KB after
 // each 32-row box (the next box, P0, or the first latent stage), all inside the allocation.
-// The rings take what is left: with the RoPE scores on the tensor cores the key ring holds a
-// tile only until MMA1 and the latent ring until MMA2, so stages go to the latent ring
-// first; otherwise a tile holds a stage of each until MMA2 and the rings grow together.
+// The rings take what is left.  A key stage is free after MMA1 (RoPE scores on the tensor
+// cores) or once the softmax warps hold its keys in registers, a latent stage only after
+// MMA2, so the latent ring gets up to two stages more than the key ring.
 static ChunkLayoutSmem chunk_smem_rtc(int dc, int R, int qbits, int rows, bool rtc) {
   const uint32_t budget = 232448 - 1024;
   const int dcp = (dc + 63) / 64 * 64;
@@ -958,15 +992,12 @@ static ChunkLayoutSmem chunk_smem_rtc(int dc, int R, int qbits, int rows, bool r
     return fixed + nc * L.c_stage + nk * L.k_stage + 8 * (2 * nc + 2 * nk + 2 * L.NRAW + kFixedBars) + 16 + kXchgBytes + 256;
   };
   int nc = 2, nk = 2;
-  if (!rtc) {   // a tile holds both until MMA2: the rings grow together
-    while (nc < 6 && size(nc + 1, nk + 1) <= budget) { ++nc; ++nk; }
-  } else {
-    while (true) {
-      if (nc <= nk && nc < 6 && size(nc + 1, nk) <= budget) { ++nc; continue; }
-      if (nk < nc && nk < 6 && size(nc, nk + 1) <= budget) { ++nk; continue; }
-      if (nc < 6 && size(nc + 1, nk) <= budget) { ++nc; continue; }
-      break;
-    }
+  while (true) {   // the latent ring up to two stages ahead of the key ring, then alternately
+    const bool want_c = nc < nk + 2;
+    if (want_c && nc < 6 && size(nc + 1, nk) <= budget) { ++nc; continue; }
+    if (nk < nc && nk < 6 && size(nc, nk + 1) <= budget) { ++nk; continue; }
+    if (nc < 6 && size(nc + 1, nk) <= budget) { ++nc; continue; }
+    break;
   }
   L.NC = nc;
   L.NK = nk;
