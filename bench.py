@@ -33,6 +33,7 @@ METRIC = "MLA decode cached tokens/s (batch×ctx per step) and % of B200 HBM pea
 UNIT = "cached tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 PER_WORKLOADS = ("llama2_7b_ragged_bf16", "llama2_7b_int4", "llama2_7b_int4_r128", "llama2_7b_int2")
 
 
@@ -231,6 +232,15 @@ def measured_traffic(workload_name, kernel_used):
         return None
 
 
+def measured_peak_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return FALLBACK_BF16_TFLOPS
+
+
 def measured_peak_hbm():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -396,6 +406,63 @@ class Bench:
         return {n: statistics.mean(ev[i][2 * k].elapsed_time(ev[i][2 * k + 1]) for i in range(K))
                 for k, n in enumerate(names) if n}
 
+    def chunk_line(self, Q, K):
+        """Many queries per sequence (chunked prefill): the newest Q tokens of every sequence
+        attend causally over its cache in one mla_decode_chunk call, the chunk kernel sharing
+        each cache tile among a unit's queries.  Times K calls over the rotated cache
+        replicas (CUDA events on the call's stream), then the attention kernel alone from
+        the library's per-kernel events in a separate loop."""
+        import ctypes
+        torch, mla, wl = self.torch, self.mla, self.wl
+        B, H = wl.batch, wl.n_heads
+        g = torch.Generator(device="cpu").manual_seed(1234)
+        q = (torch.randn(B, Q, H, wl.head_dim, generator=g) * 0.5).to(self.q.dtype).to(self.dev)
+        out = torch.empty_like(q)
+        ws = torch.empty(mla.mla_decode_chunk_workspace_bytes(self.plan, B, Q), dtype=torch.uint8, device=self.dev)
+        call = lambda i: mla.mla_decode_chunk(self.plan, self.caches[i % self.n_rep].struct, self.seq_lens, q, out, ws,
+                                              stream=self.stream)
+        for i in range(3):
+            call(i)
+        torch.cuda.synchronize()
+        s0, e0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(self.stream)
+        for i in range(K):
+            call(i)
+        e0.record(self.stream)
+        torch.cuda.synchronize()
+        call_ms = s0.elapsed_time(e0) / K
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)]
+        handles = [(ctypes.c_void_p * 8)(*[e.cuda_event for e in row]) for row in ev]
+        for row in ev:
+            for e in row:
+                e.record(self.stream)
+        torch.cuda.synchronize()
+        for i in range(K):
+            mla.mla_plan_set_option(self.plan, mla.MLA_OPT_PROFILE_KERNELS, ctypes.addressof(handles[i]))
+            call(i)
+        torch.cuda.synchronize()
+        mla.mla_plan_set_option(self.plan, mla.MLA_OPT_PROFILE_KERNELS, 0)
+        att_ms = statistics.mean(ev[i][4].elapsed_time(ev[i][5]) for i in range(K))
+        assert mla.mla_device_error(self.plan) == 0
+        qper = max(1, 128 // H)
+        units = -(-Q // qper)
+        lens = np.asarray(self.lens, dtype=np.int64)
+        # per query: latent scores and values over d_c, RoPE scores over 2r, for every head
+        flops = 0
+        for L in lens:
+            pos = np.arange(L - Q, L) + 1   # tokens each query sees
+            flops += int(pos.sum()) * H * (4 * wl.d_c + 2 * 2 * wl.r_pairs)
+        per_tok = self.cache_bytes / float(lens.sum())
+        streamed = sum(float(L - Q + min(Q, (k + 1) * qper)) for L in lens for k in range(units)) * per_tok
+        peak_tf = measured_peak_tflops()
+        return {"queries_per_seq": Q, "q_tokens_per_s": B * Q / (call_ms * 1e-3), "call_ms": call_ms,
+                "attention_ms": att_ms, "queries_per_unit": qper,
+                "tensor": {"achieved_tflops": flops / (att_ms * 1e-3) / 1e12, "peak_tflops": peak_tf,
+                           "frac": flops / (att_ms * 1e-3) / 1e12 / peak_tf, "flops": flops},
+                "hbm": {"unique_cache_bytes": self.cache_bytes, "streamed_bytes": streamed,
+                        "streamed_gbs": streamed / (att_ms * 1e-3) / 1e9},
+                "steps": K}
+
     def decode_only_ms(self, K):
         torch = self.torch
         torch.cuda.synchronize()
@@ -433,7 +500,7 @@ class Bench:
         peak, peak_src = measured_peak_hbm()
         achieved = self.cache_bytes / (attention_ms * 1e-3) / 1e9
         kernel_name = {2: "tcgen05 split-K latent attention, a token per softmax thread (decode_tc_kernel)",
-                       3: "tcgen05 split-K latent attention, a head per softmax thread (attn_tc_kernel<32>)"}.get(
+                       3: "tcgen05 split-K latent attention, a head per softmax thread (attn_tc_kernel)"}.get(
                            self.kernel_used, "CUDA-core split-K latent attention (decode_simt_kernel)")
         return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": measured_traffic(workload_name, self.kernel_used), "kernel": kernel_name,
@@ -506,6 +573,11 @@ def run_ours(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = bn.cpu_baseline(20.0)
+    if world == 1 and args.per_workload:
+        try:   # chunked prefill over the same caches: 64 new tokens per sequence
+            line["prefill_chunk"] = bn.chunk_line(64, max(5, min(K, 50)))
+        except Exception as e:   # shapes the chunk kernel does not take
+            line["prefill_chunk"] = {"unavailable": str(e).splitlines()[0][:200]}
     bn.close()
     del bn
     torch.cuda.empty_cache()

@@ -244,10 +244,9 @@ MLA_API size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B);
 /* The attention kernel mla_decode runs for this plan and cache under the plan's
  * MLA_OPT_DECODE_KERNEL setting: *kernel = 1 (CUDA cores), 2 (tcgen05, a token per softmax
  * thread) or 3 (tcgen05, a head per softmax thread), the option's own numbering.  Automatic
- * choice (option 0): a bf16 latent cache on kernel 3 where its shapes allow, a quantised
- * one on kernel 2 where its shapes allow, else kernel 3, else kernel 1.  Host only; no
- * device work.  Returns MLA_ERR_UNSUPPORTED where the forced kernel cannot run the shape,
- * MLA_ERR_INVALID_ARG for null arguments. */
+ * choice (option 0): kernel 3 where its shapes allow, else kernel 2, else kernel 1.  Host
+ * only; no device work.  Returns MLA_ERR_UNSUPPORTED where the forced kernel cannot run the
+ * shape, MLA_ERR_INVALID_ARG for null arguments. */
 MLA_API mla_status_t mla_decode_kernel_choice(const mla_plan_t* plan, const mla_cache_t* cache, int32_t* kernel);
 
 /* One decode step: attention of each sequence's new query over its cached tokens

@@ -92,9 +92,8 @@ mla_status_t mla_pick_decode_kernel(const mla_plan& p, const mla_cache_t& c, int
       if (!head_rows) return MLA_ERR_UNSUPPORTED;
       *kernel = 4;
       break;
-    default:   // bf16 latents stream fastest through the head-row kernel, quantised ones
-               // (dequantised in shared memory) through the token-row kernel
-      if (head_rows && (!mla_kind_quant(p.cfg.cache_kind) || !token_rows)) *kernel = 4;
+    default:   // the head-row kernel where its shapes allow, else the token-row kernel
+      if (head_rows) *kernel = 4;
       else if (token_rows) *kernel = 2;
       break;
   }
