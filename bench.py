@@ -442,7 +442,9 @@ class Bench:
             call(i)
         torch.cuda.synchronize()
         mla.mla_plan_set_option(self.plan, mla.MLA_OPT_PROFILE_KERNELS, 0)
-        att_ms = statistics.mean(ev[i][4].elapsed_time(ev[i][5]) for i in range(K))
+        kt = {n: statistics.mean(ev[i][2 * k].elapsed_time(ev[i][2 * k + 1]) for i in range(K))
+              for k, n in ((1, "absorb"), (2, "attention"), (3, "combine"))}
+        att_ms = kt["attention"]
         assert mla.mla_device_error(self.plan) == 0
         qper = max(1, 128 // H)
         units = -(-Q // qper)
@@ -456,7 +458,7 @@ class Bench:
         streamed = sum(float(L - Q + min(Q, (k + 1) * qper)) for L in lens for k in range(units)) * per_tok
         peak_tf = measured_peak_tflops()
         return {"queries_per_seq": Q, "q_tokens_per_s": B * Q / (call_ms * 1e-3), "call_ms": call_ms,
-                "attention_ms": att_ms, "queries_per_unit": qper,
+                "attention_ms": att_ms, "kernel_ms": kt, "queries_per_unit": qper,
                 "tensor": {"achieved_tflops": flops / (att_ms * 1e-3) / 1e12, "peak_tflops": peak_tf,
                            "frac": flops / (att_ms * 1e-3) / 1e12 / peak_tf, "flops": flops},
                 "hbm": {"unique_cache_bytes": self.cache_bytes, "streamed_bytes": streamed,

@@ -164,6 +164,20 @@ __device__ __forceinline__ float rope_dot8(float s, const float (&q)[8], uint4 k
   return r.x + r.y;
 }
 
+// s + sum_j q[j] k[j] with both factors bf16 (q packed in pairs like the keys) and the
+// products accumulated in f32 by the mixed-precision FMA (no unpacking of the keys).
+__device__ __forceinline__ float rope_dot8_bf16(float s, const uint32_t (&q)[4], uint4 kw) {
+  float acc0 = s, acc1 = 0.f;
+  const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    asm("{\n\t.reg .b16 ql, qh, kl, kh;\n\tmov.b32 {ql, qh}, %2;\n\tmov.b32 {kl, kh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, ql, kl, %0;\n\tfma.rn.f32.bf16 %1, qh, kh, %1;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "r"(q[i]), "r"(w[i]));
+  return acc0 + acc1;
+}
+
 // Two's-complement 4-bit code (in the low nibble) to float without a conversion
 // instruction: the offset code (n ^ 8) goes into the mantissa of 2^23, whose value then
 // exceeds 2^23 + 8 by exactly the code.
@@ -567,6 +581,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
     bool ok = true;
     float m = -INFINITY, l = 0.f;
     float qr[8];
+    uint32_t qb[4];   // the RoPE query rounded to bf16, in pairs
     int p_row = -1;
     auto wwait = [&](uint32_t bar, int parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, lim));
@@ -586,6 +601,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
           qr[0] = x0.x; qr[1] = x0.y; qr[2] = x0.z; qr[3] = x0.w;
           qr[4] = x1.x; qr[5] = x1.y; qr[6] = x1.z; qr[7] = x1.w;
         }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) qb[j] = pack_bf16x2(qr[2 * j], qr[2 * j + 1]);
         m = -INFINITY;
         l = 0.f;
       }
@@ -621,7 +638,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
           const int tt = tb + t;
-          float v = rope_dot8(s[t], qr, kw[t]);
+          float v = rope_dot8_bf16(s[t], qb, kw[t]);
           v = tt < lim_t ? v : -INFINITY;
           s[t] = v;
           mx = fmaxf(mx, v);
