@@ -409,10 +409,9 @@ class Bench:
     def chunk_line(self, Q, K):
         """Many queries per sequence (chunked prefill): the newest Q tokens of every sequence
         attend causally over its cache in one mla_decode_chunk call, the chunk kernel sharing
-        each cache tile among a unit's queries.  Times K calls over the rotated cache
-        replicas (CUDA events on the call's stream), then the attention kernel alone from
-        the library's per-kernel events in a separate loop."""
-        import ctypes
+        each cache tile among a unit's queries.  Times K whole calls (absorption, attention,
+        merge) over the rotated cache replicas with CUDA events on the call's stream; the
+        rates below are per whole call."""
         torch, mla, wl = self.torch, self.mla, self.wl
         B, H = wl.batch, wl.n_heads
         g = torch.Generator(device="cpu").manual_seed(1234)
@@ -431,20 +430,6 @@ class Bench:
         e0.record(self.stream)
         torch.cuda.synchronize()
         call_ms = s0.elapsed_time(e0) / K
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(K)]
-        handles = [(ctypes.c_void_p * 8)(*[e.cuda_event for e in row]) for row in ev]
-        for row in ev:
-            for e in row:
-                e.record(self.stream)
-        torch.cuda.synchronize()
-        for i in range(K):
-            mla.mla_plan_set_option(self.plan, mla.MLA_OPT_PROFILE_KERNELS, ctypes.addressof(handles[i]))
-            call(i)
-        torch.cuda.synchronize()
-        mla.mla_plan_set_option(self.plan, mla.MLA_OPT_PROFILE_KERNELS, 0)
-        kt = {n: statistics.mean(ev[i][2 * k].elapsed_time(ev[i][2 * k + 1]) for i in range(K))
-              for k, n in ((1, "absorb"), (2, "attention"), (3, "combine"))}
-        att_ms = kt["attention"]
         assert mla.mla_device_error(self.plan) == 0
         qper = max(1, 128 // H)
         units = -(-Q // qper)
@@ -458,11 +443,12 @@ class Bench:
         streamed = sum(float(L - Q + min(Q, (k + 1) * qper)) for L in lens for k in range(units)) * per_tok
         peak_tf = measured_peak_tflops()
         return {"queries_per_seq": Q, "q_tokens_per_s": B * Q / (call_ms * 1e-3), "call_ms": call_ms,
-                "attention_ms": att_ms, "kernel_ms": kt, "queries_per_unit": qper,
-                "tensor": {"achieved_tflops": flops / (att_ms * 1e-3) / 1e12, "peak_tflops": peak_tf,
-                           "frac": flops / (att_ms * 1e-3) / 1e12 / peak_tf, "flops": flops},
+                "queries_per_unit": qper,
+                "tensor": {"achieved_tflops": flops / (call_ms * 1e-3) / 1e12, "peak_tflops": peak_tf,
+                           "frac": flops / (call_ms * 1e-3) / 1e12 / peak_tf, "flops": flops},
                 "hbm": {"unique_cache_bytes": self.cache_bytes, "streamed_bytes": streamed,
-                        "streamed_gbs": streamed / (att_ms * 1e-3) / 1e9},
+                        "streamed_gbs": streamed / (call_ms * 1e-3) / 1e9,
+                        "frac": streamed / (call_ms * 1e-3) / 1e9 / measured_peak_hbm()[0]},
                 "steps": K}
 
     def decode_only_ms(self, K):

@@ -143,27 +143,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// s + sum_j q[j] k[j] over one KV head's 8 RoPE dims (k: 8 bf16), in pairs of lanes of the
-// packed f32x2 FMA: (even dims, odd dims) accumulate apart and add at the end.
-__device__ __forceinline__ float rope_dot8(float s, const float (&q)[8], uint4 kw) {
-  const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
-  uint64_t acc;
-  {
-    const float2 a0 = make_float2(s, 0.f);
-    acc = *reinterpret_cast<const uint64_t*>(&a0);
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 kk = make_float2(bf16lo(w[i]), bf16hi(w[i]));
-    const float2 qq = make_float2(q[2 * i], q[2 * i + 1]);
-    asm("fma.rn.f32x2 %0, %1, %2, %0;"
-        : "+l"(acc)
-        : "l"(*reinterpret_cast<const uint64_t*>(&qq)), "l"(*reinterpret_cast<const uint64_t*>(&kk)));
-  }
-  const float2 r = *reinterpret_cast<const float2*>(&acc);
-  return r.x + r.y;
-}
-
 // s + sum_j q[j] k[j] with both factors bf16 (q packed in pairs like the keys) and the
 // products accumulated in f32 by the mixed-precision FMA (no unpacking of the keys).
 __device__ __forceinline__ float rope_dot8_bf16(float s, const uint32_t (&q)[4], uint4 kw) {
@@ -765,6 +744,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
     bool ok = true;
     float m = -INFINITY, l = 0.f;
     float qr[8];
+    uint32_t qb[4];   // the RoPE query rounded to bf16, in pairs
     int p_row = -1;                          // position of this row's query (-1: past the chunk)
     auto wwait = [&](uint32_t bar, int parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, lim));
@@ -784,6 +764,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
           qr[0] = x0.x; qr[1] = x0.y; qr[2] = x0.z; qr[3] = x0.w;
           qr[4] = x1.x; qr[5] = x1.y; qr[6] = x1.z; qr[7] = x1.w;
         }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) qb[j] = pack_bf16x2(qr[2 * j], qr[2 * j + 1]);
         if (rtc) {
           // this row's RoPE query (bf16) into its KV head's 16-byte chunk of the block-diagonal
           // operand, once MMA1 of the previous piece has read it
@@ -833,16 +815,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         // RoPE score against the tile's keys: row tt of the swizzled stage, KV head g's chunk
         const uint8_t* krb = sbase + a.off_k + ks * a.k_stage + (g >> 3) * kTBox;
 #pragma unroll
-        for (int t = 0; t < TPL; ++t) {
-          const int tt = t;
-          const uint4 kw = *reinterpret_cast<const uint4*>(krb + sw128(tt, g));
-          float v = rope_dot8(s[t], qr, kw);
-          v = tt < lim_t ? v : -INFINITY;
-          s[t] = v;
-          mx = fmaxf(mx, v);
+        for (int t0 = 0; t0 < TPL; t0 += 16) {   // 16 keys in flight at a time
+          uint4 kw[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) kw[t] = *reinterpret_cast<const uint4*>(krb + sw128(t0 + t, g));
+          if (t0 + 16 == TPL) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.k_empty(ks));   // this warp holds all its keys
+          }
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const int tt = t0 + t;
+            float v = rope_dot8_bf16(s[tt], qb, kw[t]);
+            v = tt < lim_t ? v : -INFINITY;
+            s[tt] = v;
+            mx = fmaxf(mx, v);
+          }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bars.k_empty(ks));   // this warp has read its keys
       }
       // Raise the running max lazily: a row rescales when its max grew by more than kTau.
       // Rows decide on their own, but the TMEM loads and stores (and the wait before them)

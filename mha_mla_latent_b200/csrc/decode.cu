@@ -362,6 +362,7 @@ struct CombineArgs {
   // h / heads of sequence v / nqb, head h % heads (W_uv group (h % heads) / G).  Decode:
   // q_chunk = q_block = 1, heads = H.
   int q_chunk, q_block, heads;
+  int rpw;            // rows per warp: a CTA merges 8 rpw rows against one staged W_uv chunk
 };
 
 // Output row (query row x head) of merged row h of unit v, or -1 past the chunk's last query.
@@ -373,10 +374,12 @@ __device__ __forceinline__ long long combine_out_row(const CombineArgs& a, int v
   return ((long long)(v / nqb) * a.q_chunk + i) * a.heads + h % a.heads;
 }
 
-constexpr int kCmbRows = 8;    // (b, h) rows per CTA, one warp each
+constexpr int kCmbRows = 8;    // warps per CTA; a warp merges rpw rows (b, h)
+constexpr int kCmbMaxRpw = 4;
 
-// grid: n_kv * (row blocks) * (output column chunks).  Before the dependency wait the CTA
-// stages its W_uv[g] column chunk; after it, warp r merges the pieces of row r,
+// grid: n_kv * (row blocks of 8 rpw rows) * (output column chunks).  Before the dependency
+// wait the CTA stages its W_uv[g] column chunk; after it, warp r merges the pieces of rows
+// r, r + 8, ... of its block,
 //     O_lat = sum_j 2^(m_j - M) O_j / sum_j 2^(m_j - M) l_j,
 // into shared memory (all of a batch of pieces' loads in flight together), and then
 // out[row][d] = sum_c O_lat[row][c] W_uv[g][c][d] with lane l on columns 2l, 2l+1.
@@ -385,12 +388,14 @@ __global__ void __launch_bounds__(256, 1) combine_kernel(CombineArgs a) {
   extern __shared__ __align__(16) float sm[];
   const int G = a.H / a.n_kv;
   const int rows_total = a.B * G;
-  const int n_rb = (rows_total + kCmbRows - 1) / kCmbRows;
+  const int RB = kCmbRows * a.rpw;            // rows of this CTA
+  const int RBP = (RB + 15) & ~15;            // padded to whole m16 tiles
+  const int n_rb = (rows_total + RB - 1) / RB;
   const int g = blockIdx.x % a.n_kv;
   const int rb = (blockIdx.x / a.n_kv) % n_rb;
   const int dcb = blockIdx.x / (a.n_kv * n_rb);
   const int NCOL = a.ncols;
-  const int row0 = rb * kCmbRows, d0 = dcb * NCOL;
+  const int row0 = rb * RB, d0 = dcb * NCOL;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int dc = a.d_c;
   // bf16 with whole 16-byte rows: the output product runs as warp MMAs on bf16 tiles
@@ -398,8 +403,8 @@ __global__ void __launch_bounds__(256, 1) combine_kernel(CombineArgs a) {
   constexpr int WLD = 64 + 8;            // bf16 W tile row stride (conflict-free ldmatrix)
   const int ALD = dc + 8;                // bf16 A tile row stride
   float* s_w = sm;                       // f32 [d_c][NCOL], or bf16 [d_c][WLD] for the MMA form
-  float* s_o = s_w + dc * NCOL;          // [kCmbRows][d_c]
-  __nv_bfloat16* s_a = reinterpret_cast<__nv_bfloat16*>(s_o + kCmbRows * dc);   // [16][ALD]
+  float* s_o = s_w + dc * NCOL;          // [RB][d_c]
+  __nv_bfloat16* s_a = reinterpret_cast<__nv_bfloat16*>(s_o + RB * dc);   // [RBP][ALD]
   const T* W = (const T*)a.W_uv + (size_t)(g % (a.heads / G)) * dc * a.dh;
   const int ncol = min(NCOL, a.dh - d0);
   if (mma) {
@@ -416,16 +421,27 @@ __global__ void __launch_bounds__(256, 1) combine_kernel(CombineArgs a) {
   }
   // the schedule was written two kernels back (complete before the attention kernel let
   // this one launch); the partials need the dependency wait
-  int first = 0, np = 0;
-  if (row0 + warp < rows_total) {
-    const int b = (row0 + warp) / G;
-    first = __ldg(a.sched.seq_first + b);
-    np = __ldg(a.sched.seq_np + b);
+  int firsts[kCmbMaxRpw], nps[kCmbMaxRpw];
+#pragma unroll
+  for (int j = 0; j < kCmbMaxRpw; ++j) {
+    firsts[j] = 0;
+    nps[j] = 0;
+    const int row = row0 + warp + kCmbRows * j;
+    if (j < a.rpw && row < rows_total) {
+      const int b = row / G;
+      firsts[j] = __ldg(a.sched.seq_first + b);
+      nps[j] = __ldg(a.sched.seq_np + b);
+    }
   }
   pdl_wait();   // the partials of the attention kernel
   pdl_trigger();
-  {
-    const int r = warp, row = row0 + r;
+#pragma unroll 1
+  for (int j = 0; j < a.rpw; ++j) {
+    int first = firsts[0], np = nps[0];
+#pragma unroll
+    for (int k = 1; k < kCmbMaxRpw; ++k)
+      if (j == k) { first = firsts[k]; np = nps[k]; }
+    const int r = warp + kCmbRows * j, row = row0 + r;
     float* o = s_o + r * dc;
     if (row < rows_total) {
       const int h = g * G + row % G;
@@ -492,39 +508,46 @@ __global__ void __launch_bounds__(256, 1) combine_kernel(CombineArgs a) {
     }
   }
   if (mma) {
-    // A = merged rows as bf16 (rows 8..15 zero), B = W_uv chunk; warps 0-3 take 16 columns each
-    __syncthreads();   // every warp's merged row is in s_o
-    for (int i = tid; i < 16 * dc; i += 256) {
+    // A = merged rows as bf16 (pad rows zero), B = W_uv chunk: 16-row tiles x 16-column
+    // slices, one (tile, slice) pair per warp at a time
+    __syncthreads();   // every warp's merged rows are in s_o
+    for (int i = tid; i < RBP * dc; i += 256) {
       const int r = i / dc, c = i % dc;
-      s_a[r * ALD + c] = __float2bfloat16_rn(r < kCmbRows ? s_o[r * dc + c] : 0.f);
+      s_a[r * ALD + c] = __float2bfloat16_rn(r < RB ? s_o[r * dc + c] : 0.f);
     }
     sm100::cp_async_wait_all();
     __syncthreads();
-    if (warp >= 4) return;
     const __nv_bfloat16* wt = reinterpret_cast<const __nv_bfloat16*>(s_w);
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    for (int k0 = 0; k0 < dc; k0 += 16) {
-      uint32_t af[4], bf[4];
-      wmma16::load_a(af, s_a, ALD, 0, k0, lane);
-      wmma16::load_b2(bf, wt, WLD, k0, 16 * warp, lane);
-      wmma16::mma_16816(acc[0], af, bf[0], bf[1]);
-      wmma16::mma_16816(acc[1], af, bf[2], bf[3]);
-    }
-    const int r = lane >> 2, row = row0 + r;
-    const long long orow = row < rows_total ? combine_out_row(a, row / G, g * G + row % G) : -1;
-    if (orow >= 0) {
-      T* out = (T*)a.out + (size_t)orow * a.dh + d0 + 16 * warp + 2 * (lane & 3);
+    for (int job = warp; job < (RBP / 16) * 4; job += kCmbRows) {
+      const int mt = job >> 2, ns = job & 3;   // row tile, 16-column slice
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      for (int k0 = 0; k0 < dc; k0 += 16) {
+        uint32_t af[4], bf[4];
+        wmma16::load_a(af, s_a, ALD, 16 * mt, k0, lane);
+        wmma16::load_b2(bf, wt, WLD, k0, 16 * ns, lane);
+        wmma16::mma_16816(acc[0], af, bf[0], bf[1]);
+        wmma16::mma_16816(acc[1], af, bf[2], bf[3]);
+      }
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        __nv_bfloat162 v = __floats2bfloat162_rn(acc[j][0], acc[j][1]);
-        *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(out) + 8 * j) = v;
+      for (int hr = 0; hr < 2; ++hr) {   // fragment rows lane / 4 and lane / 4 + 8
+        const int r = 16 * mt + (lane >> 2) + 8 * hr, row = row0 + r;
+        const long long orow = r < RB && row < rows_total ? combine_out_row(a, row / G, g * G + row % G) : -1;
+        if (orow < 0) continue;
+        T* out = (T*)a.out + (size_t)orow * a.dh + d0 + 16 * ns + 2 * (lane & 3);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          __nv_bfloat162 v = __floats2bfloat162_rn(acc[j][2 * hr], acc[j][2 * hr + 1]);
+          *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(out) + 8 * j) = v;
+        }
       }
     }
     return;
   }
   __syncthreads();
-  const int r = warp, row = row0 + r, d = d0 + 2 * lane;
+  const int d = d0 + 2 * lane;
   if (2 * lane >= NCOL) return;
+  for (int j = 0; j < a.rpw; ++j) {
+  const int r = warp + kCmbRows * j, row = row0 + r;
   const float* o = s_o + r * dc;
   float acc0 = 0.f, acc1 = 0.f;
   for (int c = 0; c < dc; c += 4) {
@@ -541,6 +564,7 @@ __global__ void __launch_bounds__(256, 1) combine_kernel(CombineArgs a) {
     T* out = (T*)a.out + (size_t)orow * a.dh + d;
     out[0] = from_f32<T>(acc0);
     if (d + 1 < a.dh) out[1] = from_f32<T>(acc1);
+  }
   }
 }
 
@@ -592,13 +616,16 @@ cudaError_t launch_combine(const mla_plan& p, int units, int H, int n_kv, int q_
   ca.B = units; ca.H = H; ca.n_kv = n_kv; ca.d_c = cfg.d_c; ca.dh = cfg.head_dim;
   ca.opart = (const float*)(base + L.off_opart); ca.mlpart = (const float*)(base + L.off_mlpart);
   ca.sched = sched; ca.W_uv = p.W_uv; ca.out = out; ca.P = L.P;
-  ca.ncols = (size_t)cfg.d_c * (64 + kCmbRows) * sizeof(float) <= 160 * 1024 ? 64 : 32;
+  // many rows per W_uv group (a chunk of queries): more rows per CTA, fewer W stagings
+  const int G = H / n_kv;
+  ca.rpw = units * G >= 64 * kCmbRows ? kCmbMaxRpw : 1;
+  const int RB = kCmbRows * ca.rpw, RBP = (RB + 15) & ~15;
+  ca.ncols = (size_t)cfg.d_c * (64 + RB) * sizeof(float) <= 160 * 1024 ? 64 : 32;
   ca.vec_ok = cfg.head_dim % (16 / (int)sizeof(T)) == 0;
   ca.q_chunk = q_chunk; ca.q_block = q_block; ca.heads = cfg.n_heads;
-  const size_t smem_c = (size_t)cfg.d_c * (ca.ncols + kCmbRows) * sizeof(float) +
-                        (size_t)16 * (cfg.d_c + 8) * sizeof(__nv_bfloat16);   // + the MMA form's A tile
-  const int G = H / n_kv;
-  const int n_rbc = (units * G + kCmbRows - 1) / kCmbRows, n_dc = (cfg.head_dim + ca.ncols - 1) / ca.ncols;
+  const size_t smem_c = (size_t)cfg.d_c * (ca.ncols + RB) * sizeof(float) +
+                        (size_t)RBP * (cfg.d_c + 8) * sizeof(__nv_bfloat16);   // + the MMA form's A tiles
+  const int n_rbc = (units * G + RB - 1) / RB, n_dc = (cfg.head_dim + ca.ncols - 1) / ca.ncols;
   cudaError_t e = cudaFuncSetAttribute(combine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
   if (e != cudaSuccess) return e;
   if ((e = mla_profile_event(p, kProfCombine, false, s)) != cudaSuccess) return e;
