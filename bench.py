@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--separate-calls", action="store_true",
                     help="time the step as mla_append + mla_decode instead of one mla_decode_step")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="print only the chunked-prefill figure (64 queries per sequence) of the workload")
     ap.add_argument("--no-per-workload", dest="per_workload", action="store_false",
                     help="measure only --workload (default: also the ragged and int4 workloads at N=1)")
     return ap.parse_args()
@@ -529,6 +531,12 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     bn = Bench(args.workload, dev, args.kernel, fused=not args.separate_calls)
     wl, K = bn.wl, args.steps
+    if args.prefill_only:
+        if rank == 0:
+            print(json.dumps({"workload": args.workload, "prefill_chunk": bn.chunk_line(64, max(3, min(K, 50)))}),
+                  flush=True)
+        bn.close()
+        return 0
     for i in range(args.warmup):
         bn.step(i)
     torch.cuda.synchronize()

@@ -55,7 +55,20 @@ template <int ROWS> struct Geo {
   static constexpr uint32_t PBYTES = ROWS * 128u;    // P buffer: ROWS rows x 64 tokens bf16
   static constexpr int PROD = ROWS == 32 ? 2 : 0;    // TMA producer warp
   static constexpr int MMA = ROWS == 32 ? 3 : 1;     // TMEM owner and MMA issuer warp
-  static constexpr int DQ = ROWS == 32 ? 6 : 2;      // first of the two dequantising warps
+  static constexpr int DQ = ROWS == 32 ? 6 : 2;      // first dequantising warp
+};
+// A quantised cache with 32-row units runs 12 warps: four dequantising warps (6, 7, 10, 11,
+// on the two schedulers without softmax warps), two threads per token row, each taking
+// every other group of 32 values; warps 8 and 9 idle.  Otherwise 8 warps and two
+// dequantising warps (DQ, DQ + 1), a thread per token row.
+template <int ROWS, int QB> struct Crew {
+  static constexpr bool WIDE = ROWS == 32 && QB != 0;
+  static constexpr int WARPS = WIDE ? 12 : 8;
+  static constexpr int NDQ = WIDE ? 4 : 2;   // dequantising warps
+  __device__ static int dq_index(int warp) {   // 0..NDQ-1, or -1
+    if (WIDE) return warp == 6 ? 0 : warp == 7 ? 1 : warp == 10 ? 2 : warp == 11 ? 3 : -1;
+    return warp == Geo<ROWS>::DQ ? 0 : warp == Geo<ROWS>::DQ + 1 ? 1 : -1;
+  }
 };
 constexpr uint32_t kSCol = 0, kOCol = 128;
 
@@ -186,7 +199,7 @@ __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)r * 1
 // keys in stage n % NK, released after MMA1(n) when the RoPE scores run on the tensor cores
 // (a.rtc), else after MMA2(n) (the softmax warps read them).
 template <int ROWS, int QB, bool RESID, bool PAGED>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(Crew<ROWS, QB>::WARPS * 32, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_kr,
                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ ChunkArgs a) {
   constexpr bool QUANT = QB != 0;
@@ -209,11 +222,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
   if (threadIdx.x == 0) {
     misc->abort_flag = 0;
     // latent stage: its TMA bytes, or both dequantising warps; RoPE-key stage: its TMA bytes
-    for (int s = 0; s < a.NC; ++s) { mbar_init(bars.c_full(s), QUANT ? 2 : 1); mbar_init(bars.c_empty(s), 1); }
+    for (int s = 0; s < a.NC; ++s) {
+      mbar_init(bars.c_full(s), QUANT ? Crew<ROWS, QB>::NDQ : 1);
+      mbar_init(bars.c_empty(s), 1);
+    }
     // a key stage is free after MMA1 (RoPE scores on the tensor cores) or after every
     // softmax warp has read its keys
     for (int s = 0; s < a.NK; ++s) { mbar_init(bars.k_full(s), 1); mbar_init(bars.k_empty(s), rtc ? 1 : kSW); }
-    for (int s = 0; s < a.NRAW; ++s) { mbar_init(bars.raw_full(s), 1); mbar_init(bars.raw_empty(s), 2); }
+    for (int s = 0; s < a.NRAW; ++s) { mbar_init(bars.raw_full(s), 1); mbar_init(bars.raw_empty(s), Crew<ROWS, QB>::NDQ); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars.s_full(i), 1);
       mbar_init(bars.s_empty(i), kSW);
@@ -430,11 +446,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
       volatile int never = 0;
       mbar_wait(bars.mma_done(), 0, &never, lim);
     }
-  } else if (QUANT && warp >= GG::DQ && warp < GG::DQ + 2) {
+  } else if (QUANT && Crew<ROWS, QB>::dq_index(warp) >= 0) {
     // ============================================================ dequantisation
-    // thread = token row of the tile: codes * scale -> bf16 into the latent stage's swizzled
-    // boxes; rows past the unit's last token are zeroed (MMA2 multiplies them by P = 0)
-    const int tok = threadIdx.x - 32 * GG::DQ;   // 0..63
+    // thread = token row of the tile (with four dequantising warps: a token row and the
+    // groups of one parity): codes * scale -> bf16 into the latent stage's swizzled boxes;
+    // rows past the unit's last token are zeroed (MMA2 multiplies them by P = 0)
+    constexpr int NPART = Crew<ROWS, QB>::NDQ / 2;   // threads per token row
+    const int dqt = Crew<ROWS, QB>::dq_index(warp) * 32 + lane;
+    const int tok = dqt & 63, part = dqt >> 6;        // token row, group parity (NPART = 2)
     TileIter it;
     it.init(&a.sched, w);
     int n = 0;
@@ -482,14 +501,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
         // one of the window's tokens: its unquantised row from the ring
         const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.cache.c_resid) +
                                                           rslot * dc);
-        for (int j = 0; j < dc / 8; ++j) put(j, __ldg(src + j));
+        for (int j = part; j < dc / 8; j += NPART) put(j, __ldg(src + j));
       } else if (tok < nvalid) {
         const uint8_t* codes = raw + tok * a.code_row;
         float svs[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) svs[j] = __half2float(scl[j]);
 #pragma unroll 1
-        for (int grp = 0; grp < dc / 32; ++grp) {   // 32 values, one scale (a loop: code size)
+        for (int grp = part; grp < dc / 32; grp += NPART) {   // 32 values, one scale (a loop: code size)
           float sv = svs[0];
 #pragma unroll
           for (int j = 1; j < 8; ++j) sv = grp == j ? svs[j] : sv;
@@ -521,9 +540,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
           }
         }
       } else {
-        for (int j = 0; j < dc / 8; ++j) put(j, make_uint4(0, 0, 0, 0));
+        for (int j = part; j < dc / 8; j += NPART) put(j, make_uint4(0, 0, 0, 0));
       }
-      for (int j = dc / 8; j < dcp / 8; ++j) put(j, make_uint4(0, 0, 0, 0));   // padding columns
+      for (int j = dc / 8 + part; j < dcp / 8; j += NPART) put(j, make_uint4(0, 0, 0, 0));   // padding columns
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -537,7 +556,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__
       it.next();
       ++n;
     }
-  } else if (ROWS == 32 && (warp & 2) == 0) {
+  } else if (ROWS == 32 && (warp & 2) == 0 && warp < 8) {
     // ============================================================ softmax + epilogue, 32 rows
     // Rows 16q .. 16q+15 sit in TMEM lanes 0..15 of quarter q = warp & 1 (M = 64).  Four
     // threads share a row: warp half = warp >> 2 and lane half hb = lane >> 4 take tokens
@@ -1123,7 +1142,8 @@ cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const i
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
   if ((e = mla_profile_event(p, kProfAttention, false, s)) != cudaSuccess) return e;
-  e = mla_launch_kernel(kern, dim3(G), dim3(256), L.total, s, p.opt_pdl, tm_c, tm_kr, tm_q, a);
+  const int threads = rows == 32 && qbits ? Crew<32, 4>::WARPS * 32 : 256;
+  e = mla_launch_kernel(kern, dim3(G), dim3(threads), L.total, s, p.opt_pdl, tm_c, tm_kr, tm_q, a);
   if (e != cudaSuccess) return e;
   return mla_profile_event(p, kProfAttention, true, s);
 }

@@ -384,7 +384,7 @@ constexpr int kCmbMaxRpw = 4;
 // into shared memory (all of a batch of pieces' loads in flight together), and then
 // out[row][d] = sum_c O_lat[row][c] W_uv[g][c][d] with lane l on columns 2l, 2l+1.
 template <typename T>
-__global__ void __launch_bounds__(256, 1) combine_kernel(CombineArgs a) {
+__global__ void __launch_bounds__(256, 2) combine_kernel(CombineArgs a) {
   extern __shared__ __align__(16) float sm[];
   const int G = a.H / a.n_kv;
   const int rows_total = a.B * G;
