@@ -227,7 +227,11 @@ def measured_traffic(workload_name, kernel_used):
                     k, v = line.strip().split("=", 1)
                     kv[k] = v
         sha = code_sha1(src)
-        if kv.get("workload") != workload_name or kv.get("source_sha1") != sha:
+        if kv.get("source_sha1") != sha:
+            return None
+        if "traffic_bytes." + workload_name in kv:   # one capture per workload
+            return int(kv["traffic_bytes." + workload_name])
+        if kv.get("workload") != workload_name:
             return None
         return int(kv["traffic_bytes"])
     except (OSError, KeyError, ValueError):
