@@ -1,6 +1,8 @@
-// Many queries per sequence (a chunk of new tokens: chunked prefill, drafted tokens to
-// verify) on the 5th-generation tensor cores: every query attends causally over its
-// sequence's latent cache, and the queries of a sequence share each cache tile they read.
+// Split-K latent attention on the 5th-generation tensor cores with a (query, head) row per
+// softmax thread: the decode (one query per sequence) and many queries per sequence (a
+// chunk of new tokens: chunked prefill, drafted tokens to verify), where every query
+// attends causally over its sequence's latent cache and the queries of a sequence share
+// each cache tile they read.
 //
 // Paper notes "MHA2MLA" (ACL 2025), §关键设计 and §方法详解/整体框架: the converted layer
 // scores all heads against the one shared latent (W_uk absorbed into each query), adds the
@@ -12,19 +14,19 @@
 // heads is a unit of H rows, one with at most 32 heads a unit of the MMA's M = 64 form.
 // The units' tokens (up to the block's last query) are laid end to end and split among the
 // CTAs like the decode's split-K schedule, in tiles of 64 tokens.  Per tile:
-//     S[row][t]   = sum_c Qlat[row][c] * C[t][c]              MMA1  M = 128 rows, N = 64 tokens
-//     S[row][t]  += sum_j Qrope[row][j] * KR[t][g(h)][j]       CUDA cores (fp32), one row per thread
-//     O[row][d]  += sum_t P[row][t] * C[t][d]                  MMA2  M = 128, N = d_c, K = 64
+//     S[row][t]   = sum_c Qlat[row][c] * C[t][c]              MMA1  M = 64 or 128, N = 64 tokens
+//     S[row][t]  += sum_j Qrope[row][j] * KR[t][g(h)][j]       softmax threads (f32 += bf16 x bf16),
+//                                                              or MMA1 over block-diagonal query rows
+//     O[row][d]  += sum_t P[row][t] * C[t][d]                  MMA2  N = d_c, K = 64
 // with the causal mask t <= position of the row's query.  The transposed orientation gives
-// each softmax thread a whole row: its running max and sum are thread-local.  MMA2 reads
-// the C tile already in shared memory as an MN-major operand, so each cache byte is read
-// into the SM once per unit.
+// each softmax thread a row (or a quarter of a row's tokens): its running max and sum are
+// thread-local.  MMA2 reads the C tile already in shared memory as an MN-major operand, so
+// each cache byte is read into the SM once per unit.
 //
-// Warp roles (8 warps): warp 0 producer (TMA: the unit's Q_lat rows, C and RoPE-key tiles
-// into a ring of stages), warp 1 TMEM owner and single-thread
-// MMA issuer, warps 2-3 dequantisers of a quantised cache, warps 4-7 softmax (warp 4 + k
-// owns TMEM lane quarter k).
-// Every wait is bounded; a timeout sets MLA_DEVERR_TIMEOUT, drains and releases TMEM.
+// Roles: a TMA producer (the unit's Q_lat rows, latent and RoPE-key tiles into two rings),
+// a single-thread MMA issuer that owns TMEM, dequantising warps for a quantised cache, and
+// softmax warps (placement below).  Every wait is bounded; a timeout sets
+// MLA_DEVERR_TIMEOUT, drains the copies in flight and releases TMEM.
 #include <cuda.h>
 
 #include "decode_common.cuh"

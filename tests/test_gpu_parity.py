@@ -535,3 +535,23 @@ def test_decode_softmax_scale(idx):
         if case.lens[b] > 1:   # one token: its value whatever the scale
             assert not np.allclose(ref, case.reference(b), rtol=1e-3)
     plan.close()
+
+
+def test_decode_kernel_choice():
+    """The automatic choice runs the head-row tensor-core kernel wherever its shapes allow
+    (bf16, up to 128 heads, GQA included), the CUDA-core kernel for fp32; forcing a kernel
+    that cannot take the shape is reported."""
+    for wl, want in ((PARITY_WORKLOADS[0], 1), (PARITY_WORKLOADS[1], 3), (PARITY_WORKLOADS[2], 3),
+                     (PARITY_WORKLOADS[4], 3), (PARITY_WORKLOADS[6], 3), (PARITY_WORKLOADS[7], 3)):
+        case = OracleCase(wl, seqs=[])
+        cfg, plan = make_plan(case)
+        cache = LatentCache(cfg, wl.batch, 256, "cuda")
+        assert mla.mla_decode_kernel_choice(plan, cache.struct) == want, wl.name
+        mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, 1)
+        assert mla.mla_decode_kernel_choice(plan, cache.struct) == 1
+        if wl.n_heads != 32 or wl.dtype == "f32":
+            mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, 2)
+            with pytest.raises(mla.MlaError) as ei:
+                mla.mla_decode_kernel_choice(plan, cache.struct)
+            assert ei.value.status == mla.MLA_ERR_UNSUPPORTED
+        plan.close()
