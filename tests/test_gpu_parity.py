@@ -514,15 +514,21 @@ def test_multi_query_causal_decode(wl, kernel):
         assert_close(got[j], ref, wl.dtype, f"query at position {p}")
 
 
-@pytest.mark.parametrize("idx", [2, 4, 1], ids=["bf16_dc256", "int4_dc128", "gqa_cuda_core"])
-def test_decode_softmax_scale(idx):
-    """A config softmax_scale other than 1/sqrt(d_h) scales every score (both kernels)."""
+@pytest.mark.parametrize("kernel", [0, 1, 2])
+@pytest.mark.parametrize("idx", [2, 4, 1], ids=["bf16_dc256", "int4_dc128", "gqa_smollm"])
+def test_decode_softmax_scale(idx, kernel):
+    """A config softmax_scale other than 1/sqrt(d_h) scales every score (every kernel that
+    takes the shape: 0 the automatic choice, 1 CUDA cores, 2 token-row tcgen05)."""
     wl = PARITY_WORKLOADS[idx]
+    if not tc_kernel_ok(wl, kernel):
+        pytest.skip("outside this tensor-core kernel")
     case = case_for(wl)
     scale = 0.6 / np.sqrt(wl.head_dim)
     cfg = mla.make_config(wl.hidden, wl.n_heads, wl.n_kv_heads, wl.head_dim, wl.r_pairs, wl.d_c, wl.rope_base,
                           wl.dtype, wl.cache, wl.resid, softmax_scale=scale)
     plan = mla.mla_plan_create(cfg, **plan_inputs(case))
+    if kernel:
+        mla.mla_plan_set_option(plan, mla.MLA_OPT_DECODE_KERNEL, kernel)
     got = run_decode(case, plan, cfg)
     assert mla.mla_device_error(plan) == 0
     for b in case.seqs:

@@ -17,7 +17,7 @@ from workloads import PARITY_WORKLOADS, generate as gen
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("idx", [2, 4, 1], ids=["bf16_dc256", "int4_dc128", "gqa_cuda_core"])
+@pytest.mark.parametrize("idx", [2, 4, 1], ids=["bf16_dc256", "int4_dc128", "gqa_smollm"])
 def test_noalloc_decode_matches_decode_twice(idx):
     import mha_mla_latent_b200 as mla
     from mha_mla_latent_b200.cache import LatentCache, workspace
