@@ -80,8 +80,10 @@ typedef enum {
  * quantisation stacks on the latent): per token, groups of 32, fp16 scale s = fp16(absmax),
  * codes clamp(round_half_even(c/s), -1, 1) (0 when s == 0), two's-complement 2-bit fields,
  * element 4i+k in bits 2k..2k+1 of byte i; value = code*s.  The quantised caches are
- * decoded by the tensor-core kernel at d_c = 128 (32 heads, r = 4) and by the CUDA-core
- * kernel otherwise. */
+ * decoded on the tensor cores wherever the head-row kernel's shapes allow (dtype bf16,
+ * r = 4, at most 128 query heads and 32 KV heads, d_c a multiple of 32 up to 256 whose
+ * code rows are whole 16-byte chunks: a multiple of 64 at 2 bits) and on the CUDA cores
+ * otherwise. */
 #define MLA_RESID_WINDOW 128
 
 typedef struct {
@@ -269,17 +271,20 @@ MLA_API mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache
  * call.  seq_lens[b] counts all of sequence b's cached tokens, the chunk's own included
  * (append them first); query i (0 <= i < Q) of sequence b sits at position
  * p = seq_lens[b] - Q + i, is rotated there, and attends over tokens [0, p].  Per query this
- * is exactly mla_decode with length p + 1.  The queries of a sequence share every cache tile
- * they read: blocks of 4 queries x 32 heads are scored against each tile together on the
- * tensor cores.  Notes §方法详解/整体框架 and §关键设计 (absorbed latent scores plus the
+ * is exactly mla_decode with length p + 1.  The queries of a sequence share the cache tiles
+ * they read: blocks of floor(128/H) queries x H heads (at most 128 score rows) are scored
+ * against each tile together on the tensor cores, so a block streams its prefix once.  Notes §方法详解/整体框架 and §关键设计 (absorbed latent scores plus the
  * separate RoPE term); the README "MHA2MLA" evaluates long documents (LongBench).
  *   seq_lens  device [B] int32, Q <= L <= T_cap
  *   q         device [B][Q][H][d_h] dtype, unrotated, original dim order
  *   out       device [B][Q][H][d_h] dtype, per-head attention output (before W_o)
  *   workspace device, >= mla_decode_chunk_workspace_bytes(plan, B, Q) bytes
- * Q == 1 is mla_decode.  For Q > 1 this build needs bf16, a bf16 latent cache, 32 query
- * heads, d_c in {64, 128, 256} and r = 4 (MLA_ERR_UNSUPPORTED otherwise; one mla_decode per
- * query through per-query views of a paged cache covers the other shapes). */
+ * Q == 1 is mla_decode.  For Q > 1 this build needs the head-row kernel's shapes (dtype
+ * bf16, r = 4, at most 128 query heads and 32 KV heads, d_c a multiple of 32 up to 256;
+ * bf16, int4 or int2 latent cache, paged or contiguous) and no residual window
+ * (MLA_CACHE_INT4_G32_R128: each query's window depends on its own position).  Otherwise,
+ * and with MLA_OPT_DECODE_KERNEL = 1, it returns MLA_ERR_UNSUPPORTED; one mla_decode per
+ * query through per-query views of a paged cache covers those shapes. */
 MLA_API size_t mla_decode_chunk_workspace_bytes(const mla_plan_t* plan, int32_t B, int32_t Q);
 MLA_API mla_status_t mla_decode_chunk(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
                                       const void* q, int32_t B, int32_t Q, void* out, void* workspace,

@@ -746,8 +746,8 @@ cudaError_t launch_step_t(const mla_plan& p, const mla_cache_t& c, const int32_t
 }
 
 // Many queries per sequence: absorption of every query (each rotated at its own position)
-// with the schedule over (sequence, block of 4 queries) units, the chunk attention kernel,
-// and the merge of the units' 128 rows.
+// with the schedule over (sequence, block of floor(128 / H) queries) units, the chunk
+// attention kernel, and the merge of the units' rows.
 cudaError_t launch_chunk(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, const void* q, int B,
                          int Q, void* out, void* ws, const DecodeLayout& L, cudaStream_t s) {
   using bf16 = __nv_bfloat16;

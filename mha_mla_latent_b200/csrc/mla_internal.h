@@ -159,7 +159,8 @@ Sched mla_sched_view(const DecodeLayout& L, void* ws, int B);
 DecodeLayout mla_chunk_layout(const mla_plan& p, int B, int Q);
 bool mla_chunk_capable(const mla_plan& p);
 bool mla_chunk_supported(const mla_plan& p, const mla_cache_t& c);
-// rows = 128: units of 4 queries x 32 heads (query chunks); rows = 32: one query's heads (decode)
+// rows = 128: units of floor(128 / H) queries x H heads (query chunks, and decode with more
+// than 32 heads); rows = 32: one query's heads (decode with up to 32 heads)
 cudaError_t mla_launch_chunk_tc(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B, int Q,
                                 const Sched& sched, const void* qlat, const float* qrope, float* opart,
                                 float* mlpart, int P, int G, cudaStream_t s, int rows);
