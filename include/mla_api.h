@@ -108,7 +108,9 @@ typedef struct {
  * multiple of 128 (the logical capacity: T_cap / 128 table entries per sequence).  The
  * README "MHA2MLA" runs ragged LongBench batches; 128-token blocks match the decode tile,
  * so each tile of the attention kernel reads one block.  A table entry outside
- * [0, n_blocks) flags MLA_DEVERR_BLOCK and reads or writes block 0 instead.
+ * [0, n_blocks) flags MLA_DEVERR_BLOCK and reads or writes block 0 instead.  The arrays
+ * may hold at most 2^31 - 1 token rows (B * T_cap, or n_blocks * 128 when paged); a larger
+ * view is refused with MLA_ERR_UNSUPPORTED.
  *   c_kv      SAME: [B][T_cap][d_c] dtype;  INT4*: [B][T_cap][d_c/2] uint8 codes;
  *             INT2: [B][T_cap][d_c/4] uint8 codes
  *   c_scales  INT4*, INT2: [B][T_cap][d_c/32] fp16;  SAME: must be NULL

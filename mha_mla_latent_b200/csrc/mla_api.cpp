@@ -47,6 +47,8 @@ mla_status_t mla_validate_cache(const mla_config_t& cfg, const mla_cache_t* c) {
   } else if (c->n_blocks != 0) {
     return MLA_ERR_INVALID_ARG;
   }
+  // The attention kernels name a token row by a signed 32-bit TMA coordinate.
+  if (mla_cache_rows(*c) > (size_t)INT32_MAX) return MLA_ERR_UNSUPPORTED;
   const bool resid = cfg.cache_kind == MLA_CACHE_INT4_G32_R128;
   if (resid != (c->c_resid != nullptr) || resid != (c->resid_pos != nullptr)) return MLA_ERR_INVALID_ARG;
   if (!aligned16(c->c_kv) || (c->c_scales && !aligned16(c->c_scales)) ||

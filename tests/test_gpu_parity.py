@@ -481,6 +481,33 @@ def test_paged_block_outside_pool_is_flagged():
         assert mla.mla_device_error(plan) & mla.MLA_DEVERR_BLOCK
 
 
+def test_cache_view_beyond_32bit_rows_is_refused():
+    """A view of 2^31 token rows (B * T_cap, or n_blocks * 128 when paged) is refused before
+    any launch.  The views describe small real arrays, and every access the calls would make
+    (sequence 0, positions below 128, block 0) stays inside them."""
+    wl = PARITY_WORKLOADS[2]
+    case = case_for(wl)
+    cfg, plan = make_plan(case)
+    small = LatentCache(cfg, 2, 256, "cuda")
+    table = torch.zeros(2, 2, dtype=torch.int32, device="cuda")
+    views = [mla.cache_struct(small.c_kv, None, small.k_rope, 2, 1 << 30),
+             mla.cache_struct(small.c_kv, None, small.k_rope, 2, 256, block_table=table, n_blocks=1 << 24)]
+    x = gen.to_torch(case.x_dec[:1], wl.dtype, "cuda")
+    zero = torch.zeros(1, dtype=torch.int32, device="cuda")
+    seq = torch.full((1,), 5, dtype=torch.int32, device="cuda")
+    q = gen.to_torch(case.q[:1], wl.dtype, "cuda")
+    out = torch.empty_like(q)
+    ws = workspace(plan, 1, "cuda")
+    for view in views:
+        assert mla.mla_append(plan, x, zero, zero, view, check=False) == mla.MLA_ERR_UNSUPPORTED
+        assert mla.mla_decode(plan, view, seq, q, out, ws, check=False) == mla.MLA_ERR_UNSUPPORTED
+        assert mla.mla_decode_step(plan, view, seq, x, q, out, ws, check=False) == mla.MLA_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert mla.mla_device_error(plan) == 0
+    rows = mla.cache_struct(small.c_kv, None, small.k_rope, 2, 256)   # the real view still runs
+    assert mla.mla_append(plan, x, zero, zero, rows, check=False) == mla.MLA_OK
+
+
 # --------------------------------------------------------------------------- many queries per sequence
 @pytest.mark.parametrize("wl,kernel", [(PARITY_WORKLOADS[2], 2), (PARITY_WORKLOADS[2], 1),
                                        (PARITY_WORKLOADS[1], 1), (PARITY_WORKLOADS[4], 2)],
