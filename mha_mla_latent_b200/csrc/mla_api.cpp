@@ -83,7 +83,7 @@ void free_plan(mla_plan* p) {
 mla_status_t mla_pick_decode_kernel(const mla_plan& p, const mla_cache_t& c, int* kernel) {
   *kernel = 1;
   const bool head_rows = mla_decode_t_supported(p, c);
-  const bool token_rows = mla_tc_kind_ok(p.cfg) && mla_tc_supported(p, c);
+  const bool token_rows = mla_tc_supported(p, c);
   switch (p.opt_kernel) {
     case 1: break;
     case 2:
@@ -339,7 +339,7 @@ mla_status_t mla_decode_kernel_choice(const mla_plan_t* plan, const mla_cache_t*
 size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B) {
   if (!plan || B <= 0) return 0;
   size_t n = mla_decode_layout(*plan, B, 1).total;
-  if (mla_tc_kind_ok(plan->cfg) && mla_tc_capable(*plan)) n = std::max(n, mla_decode_layout(*plan, B, 2).total);
+  if (mla_tc_capable(*plan)) n = std::max(n, mla_decode_layout(*plan, B, 2).total);
   if (mla_decode_t_capable(*plan)) n = std::max(n, mla_decode_layout(*plan, B, 4).total);
   return host_stage(*plan, B, n).total;
 }

@@ -148,8 +148,6 @@ struct Sched {
 DecodeLayout mla_decode_layout(const mla_plan& p, int B, int kernel);
 bool mla_tc_supported(const mla_plan& p, const mla_cache_t& c);
 bool mla_tc_capable(const mla_plan& p);   // shape/dtype allow the tensor-core kernel
-// The tensor-core kernel reads bf16, int4 and 2-bit latents.
-inline bool mla_tc_kind_ok(const mla_config_t&) { return true; }
 cudaError_t mla_launch_decode_tc(const mla_plan& p, const mla_cache_t& c, const int32_t* seq_lens, int B,
                                  const Sched& sched,
                                  const void* qlat, const float* qrope, float* opart, float* mlpart, int P, int G,
