@@ -3,7 +3,8 @@
 T1 absorbed == unabsorbed; T2 brute-force top-r; T3 equivalence with plain (partial-)RoPE
 MHA written with loops; T4 Eckart-Young; T6 softmax edge cases; T7 RoPE relative
 property; T8 int4 bounds and hand-derived codes; T9 cache accounting vs printed figures;
-plus hand-derived fixtures under tests/golden/.
+T10 fixed pair sets; T11 residual window; T12 2-bit codes; T13 many queries per sequence
+as rows of causal self-attention; plus hand-derived fixtures under tests/golden/.
 """
 
 import itertools
@@ -508,3 +509,57 @@ def test_T12_int2_error_bound_and_round_trip():
     # 2 bits lose more than 4 on the same latents
     c4, s4 = O.quant_int4_g32(c)
     assert np.linalg.norm(O.dequant_int4_g32(c4, s4) - c32) < np.linalg.norm(deq - c32)
+
+
+# ------------------------------------------------------------------ T13 many queries per sequence
+def _causal_rope_mha(x, W_q, W_k, W_v, H, n_kv, dh, pair_idx, theta):
+    """Causal self-attention of the original layer over a whole sequence as one masked score
+    matrix: token i's query (rotated at i on the kept pairs of its KV head) against every key
+    j <= i (rotated at j), scale 1/sqrt(d_h).  Returns o [L][H][d_h]."""
+    L = x.shape[0]
+    G = H // n_kv
+    q = (x @ W_q).reshape(L, H, dh)
+    k = (x @ W_k).reshape(L, n_kv, dh)
+    v = (x @ W_v).reshape(L, n_kv, dh)
+    pos = np.arange(L, dtype=np.float64)
+    o = np.zeros((L, H, dh))
+    for h in range(H):
+        g = h // G
+        qh, kg = q[:, h].copy(), k[:, g].copy()
+        for kk in pair_idx[g]:
+            ang = pos * theta[kk]
+            cos, sin = np.cos(ang), np.sin(ang)
+            for m in (qh, kg):
+                a, b = m[:, 2 * kk].copy(), m[:, 2 * kk + 1].copy()
+                m[:, 2 * kk], m[:, 2 * kk + 1] = a * cos - b * sin, a * sin + b * cos
+        s = qh @ kg.T / np.sqrt(dh)
+        s[np.triu_indices(L, 1)] = -np.inf          # key j > query i: masked
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        o[:, h] = (p / p.sum(axis=1, keepdims=True)) @ v[:, g]
+    return o
+
+
+@pytest.mark.parametrize("H,n_kv", [(4, 4), (6, 3)])
+def test_T13_chunk_queries_are_rows_of_causal_attention(H, n_kv):
+    """A chunk of the newest Q tokens, each query decoded over its own prefix [0, L-Q+i] and
+    rotated at L-Q+i (the reading the chunk kernel's parity tests use), equals the last Q rows
+    of the original layer's causal self-attention when the latent has full rank."""
+    rng = np.random.default_rng(41)
+    dh, d, L, r, Q = 8, 96, 23, 2, 7
+    W_q, W_k, W_v = _rand_layer(rng, d, H, n_kv, dh)
+    pair_idx = np.stack([np.sort(rng.choice(dh // 2, r, replace=False)) for _ in range(n_kv)])
+    d_c = n_kv * (dh - 2 * r) + n_kv * dh
+    W_dkv, W_uk, W_uv, _ = O.svd_joint(W_k, W_v, pair_idx, d_c, dh)
+    theta = O.rope_theta(dh, 10000.0)
+    x = rng.standard_normal((L, d))
+    c, kr = O.append(x, np.arange(L), W_dkv, O.krope_weights(W_k, pair_idx, dh), pair_idx, theta)
+    ref = _causal_rope_mha(x, W_q, W_k, W_v, H, n_kv, dh, pair_idx, theta)
+    q = (x @ W_q).reshape(L, H, dh)
+    for i in range(Q):
+        p = L - Q + i
+        got = O.decode_unabsorbed(q[p], c[:p + 1], kr[:p + 1], W_uk, W_uv, pair_idx, theta)
+        np.testing.assert_allclose(got, ref[p], rtol=1e-10, atol=1e-11)
+    # the prefix is inclusive: leaving out the query's own token changes the result
+    p = L - 1
+    short = O.decode_unabsorbed(q[p], c[:p], kr[:p], W_uk, W_uv, pair_idx, theta)
+    assert np.abs(short - ref[p]).max() > 1e-3
