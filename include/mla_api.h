@@ -219,7 +219,9 @@ MLA_API mla_status_t mla_fixed_pairs(const mla_config_t* cfg, int32_t strategy, 
  *   W_uk     [n_kv][d_c][d_h-2r] NoPE key up-projection (rows of Sigma V^T)
  *   W_uv     [n_kv][d_c][d_h]    value up-projection
  * Notes §关键设计 (SVDjoint): W_dkv = U_trunc, Sigma V^T split per head.
- * On success *out receives the plan; release it with mla_plan_destroy. */
+ * On success *out receives the plan; release it with mla_plan_destroy.  MLA_ERR_CUDA when
+ * a device call fails or the host or device memory for the packed copies cannot be
+ * allocated; *out is then NULL and nothing is left allocated. */
 MLA_API mla_status_t mla_plan_create(const mla_config_t* cfg, const void* W_dkv, const void* W_k,
                              const int32_t* pair_idx, const void* W_uk, const void* W_uv,
                              mla_plan_t** out);

@@ -169,35 +169,17 @@ mla_status_t mla_select_pairs(const mla_config_t* cfg, const void* q_cal, const 
                                              (cudaStream_t)stream));
 }
 
-mla_status_t mla_plan_create(const mla_config_t* cfg, const void* W_dkv, const void* W_k,
-                             const int32_t* pair_idx, const void* W_uk, const void* W_uv,
-                             mla_plan_t** out) {
-  if (!out) return MLA_ERR_INVALID_ARG;
-  *out = nullptr;
-  mla_status_t st = validate_config(cfg);
-  if (st != MLA_OK) return st;
-  const int d = cfg->hidden, nkv = cfg->n_kv_heads, dh = cfg->head_dim, r = cfg->r_pairs;
-  const int dc = cfg->d_c;
-  if (!W_dkv || !W_uv || (dh - 2 * r > 0 && !W_uk) || (r > 0 && (!W_k || !pair_idx)))
-    return MLA_ERR_INVALID_ARG;
-  for (int g = 0; g < nkv; ++g)
-    for (int j = 0; j < r; ++j) {
-      int k = pair_idx[g * r + j];
-      if (k < 0 || k >= dh / 2) return MLA_ERR_INVALID_ARG;
-      if (j > 0 && k <= pair_idx[g * r + j - 1]) return MLA_ERR_INVALID_ARG;  // strictly ascending
-    }
-  mla_plan* p = new (std::nothrow) mla_plan();
-  if (!p) return MLA_ERR_CUDA;
-  p->cfg = *cfg;
-  p->R = nkv * 2 * r;
-  p->dn = dh - 2 * r;
-  p->ncols = dc + p->R;
-  if (cudaGetDevice(&p->device) != cudaSuccess ||
-      cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess) {
-    free_plan(p);
-    return MLA_ERR_CUDA;
-  }
-  const size_t eb = elem_bytes(*cfg);
+namespace {
+
+// Packs the converted weights on the host and copies them into plan-owned device memory:
+// [W_dkv | W_krope], W_uk spread over the full head dims, W_uv, the pair tables, the
+// frequencies and the append scratch.  False when a device allocation or copy fails; host
+// allocation failures throw std::bad_alloc, which mla_plan_create turns into a status.
+bool pack_and_upload(mla_plan* p, const void* W_dkv, const void* W_k, const int32_t* pair_idx, const void* W_uk,
+                     const void* W_uv) {
+  const int d = p->cfg.hidden, nkv = p->cfg.n_kv_heads, dh = p->cfg.head_dim, r = p->cfg.r_pairs;
+  const int dc = p->cfg.d_c;
+  const size_t eb = elem_bytes(p->cfg);
   // [W_dkv | W_krope]: column block of the selected pairs of each KV head, ascending.
   std::vector<unsigned char> app((size_t)d * p->ncols * eb);
   for (int i = 0; i < d; ++i) {
@@ -220,16 +202,16 @@ mla_status_t mla_plan_create(const mla_config_t* cfg, const void* W_dkv, const v
     std::vector<char> kept(dh / 2, 0);
     for (int j = 0; j < r; ++j) { kept[pair_idx[g * r + j]] = 1; rp[g * r + j] = pair_idx[g * r + j]; }
     int j = 0;
-    for (int d = 0; d < dh; ++d) {
-      if (kept[d / 2]) continue;
+    for (int hd = 0; hd < dh; ++hd) {
+      if (kept[hd / 2]) continue;
       for (int c = 0; c < dc; ++c)
-        memcpy(&ukF[(((size_t)g * dh + d) * dc + c) * eb],
+        memcpy(&ukF[(((size_t)g * dh + hd) * dc + c) * eb],
                (const unsigned char*)W_uk + (((size_t)g * dc + c) * p->dn + j) * eb, eb);
       ++j;
     }
   }
   std::vector<double> theta(dh / 2);
-  for (int k = 0; k < dh / 2; ++k) theta[k] = pow(cfg->rope_base, -2.0 * k / dh);
+  for (int k = 0; k < dh / 2; ++k) theta[k] = pow(p->cfg.rope_base, -2.0 * k / dh);
 
   bool ok = dev_alloc_copy(&p->W_app, app.data(), app.size()) &&
             dev_alloc_copy(&p->W_ukF, ukF.data(), ukF.size()) &&
@@ -243,6 +225,44 @@ mla_status_t mla_plan_create(const mla_config_t* cfg, const void* W_dkv, const v
   ok = ok && cudaMalloc((void**)&p->app_part, app_tiles * 8 * 32 * 32 * sizeof(float)) == cudaSuccess &&
        cudaMalloc((void**)&p->app_ticket, app_tiles * sizeof(int32_t)) == cudaSuccess &&
        cudaMemset(p->app_ticket, 0, app_tiles * sizeof(int32_t)) == cudaSuccess;
+  return ok;
+}
+
+}  // namespace
+
+mla_status_t mla_plan_create(const mla_config_t* cfg, const void* W_dkv, const void* W_k,
+                             const int32_t* pair_idx, const void* W_uk, const void* W_uv,
+                             mla_plan_t** out) {
+  if (!out) return MLA_ERR_INVALID_ARG;
+  *out = nullptr;
+  mla_status_t st = validate_config(cfg);
+  if (st != MLA_OK) return st;
+  const int nkv = cfg->n_kv_heads, dh = cfg->head_dim, r = cfg->r_pairs;
+  if (!W_dkv || !W_uv || (dh - 2 * r > 0 && !W_uk) || (r > 0 && (!W_k || !pair_idx)))
+    return MLA_ERR_INVALID_ARG;
+  for (int g = 0; g < nkv; ++g)
+    for (int j = 0; j < r; ++j) {
+      int k = pair_idx[g * r + j];
+      if (k < 0 || k >= dh / 2) return MLA_ERR_INVALID_ARG;
+      if (j > 0 && k <= pair_idx[g * r + j - 1]) return MLA_ERR_INVALID_ARG;  // strictly ascending
+    }
+  mla_plan* p = new (std::nothrow) mla_plan();
+  if (!p) return MLA_ERR_CUDA;
+  p->cfg = *cfg;
+  p->R = nkv * 2 * r;
+  p->dn = dh - 2 * r;
+  p->ncols = cfg->d_c + p->R;
+  if (cudaGetDevice(&p->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess) {
+    free_plan(p);
+    return MLA_ERR_CUDA;
+  }
+  bool ok = false;
+  try {
+    ok = pack_and_upload(p, W_dkv, W_k, pair_idx, W_uk, W_uv);
+  } catch (const std::exception&) {   // no host memory for the packed copies
+    ok = false;
+  }
   if (!ok) {
     free_plan(p);
     return MLA_ERR_CUDA;
