@@ -173,7 +173,10 @@ enum {
                                  MLA_OPT_PROFILE_EVENTS while set. */
 };
 
+/* A static, NUL-terminated English name of a status ("unknown status" for a value outside
+ * mla_status_t); never NULL, never to be freed. */
 MLA_API const char* mla_status_string(mla_status_t s);
+/* A static string naming this library build and its target (sm_100a); never NULL. */
 MLA_API const char* mla_version(void);
 
 /* Bytes cached per token per layer for this config (c_kv, scales, RoPE dims).
@@ -192,6 +195,14 @@ MLA_API size_t mla_cache_bytes_per_token(const mla_config_t* cfg);
 MLA_API mla_status_t mla_select_pairs(const mla_config_t* cfg, const void* q_cal, const void* k_cal,
                               int32_t T, int32_t* pair_idx, float* contrib, void* stream);
 
+/* Fixed partial-RoPE strategies for mla_fixed_pairs. */
+enum {
+  MLA_PAIRS_HIGH = 1,
+  MLA_PAIRS_UNIFORM = 2,
+  MLA_PAIRS_LOW = 5,
+  MLA_PAIRS_FULL = 0
+};
+
 /* Fixed partial-RoPE pair sets, the alternatives to the 2-norm selection that the README
  * "MHA2MLA" (§Fine-Tuning strategy tables: partial-RoPE versions) lists and the Notes
  * (§消融实验, Partial-RoPE strategy comparison) compare.  With P = d_h/2 pairs, r = r_pairs
@@ -202,12 +213,6 @@ MLA_API mla_status_t mla_select_pairs(const mla_config_t* cfg, const void* q_cal
  *   MLA_PAIRS_FULL     every pair (requires r == P: full RoPE)
  * The same set is used for every KV head.  pair_idx: HOST [n_kv][r] int32, ascending.
  * Returns MLA_ERR_INVALID_ARG for an unknown strategy or r out of range.  No GPU use. */
-enum {
-  MLA_PAIRS_HIGH = 1,
-  MLA_PAIRS_UNIFORM = 2,
-  MLA_PAIRS_LOW = 5,
-  MLA_PAIRS_FULL = 0
-};
 MLA_API mla_status_t mla_fixed_pairs(const mla_config_t* cfg, int32_t strategy, int32_t* pair_idx);
 
 /* Build a plan: validate the config and copy/pack the converted weights into
@@ -225,7 +230,12 @@ MLA_API mla_status_t mla_fixed_pairs(const mla_config_t* cfg, int32_t strategy, 
 MLA_API mla_status_t mla_plan_create(const mla_config_t* cfg, const void* W_dkv, const void* W_k,
                              const int32_t* pair_idx, const void* W_uk, const void* W_uv,
                              mla_plan_t** out);
+/* Release a plan and its device memory (cudaFree, which waits for the device to go idle).
+ * NULL is a no-op.  No work that uses the plan may still be in flight on any stream. */
 MLA_API void mla_plan_destroy(mla_plan_t* plan);
+/* Set one MLA_OPT_* option (the enum above gives each option's values and meaning); it
+ * applies to the calls made after it.  MLA_ERR_INVALID_ARG for a NULL plan, an unknown
+ * option or a value outside the option's range; the plan is then unchanged. */
 MLA_API mla_status_t mla_plan_set_option(mla_plan_t* plan, int32_t option, int64_t value);
 
 /* Append N tokens to the cache.  For token n: c = x[n] W_dkv (float32 accumulation),
@@ -244,7 +254,7 @@ MLA_API mla_status_t mla_append(const mla_plan_t* plan, const void* x, const int
 
 /* Device workspace mla_decode, mla_decode_step and mla_decode_step_host need for a batch
  * of B sequences (bytes, 256-aligned; it includes the host variant's staging of the step's
- * inputs and output). */
+ * inputs and output).  0 for a NULL plan or B <= 0. */
 MLA_API size_t mla_decode_workspace_bytes(const mla_plan_t* plan, int32_t B);
 
 /* The attention kernel mla_decode runs for this plan and cache under the plan's
@@ -270,6 +280,10 @@ MLA_API mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache
                         const void* q, int32_t B, void* out, void* workspace, size_t ws_bytes,
                         void* stream);
 
+/* Device workspace of mla_decode_chunk for B sequences of Q queries (bytes, 256-aligned;
+ * 0 for a NULL plan or B, Q <= 0). */
+MLA_API size_t mla_decode_chunk_workspace_bytes(const mla_plan_t* plan, int32_t B, int32_t Q);
+
 /* Many queries per sequence, causally: the newest Q tokens of each sequence (a chunk of a
  * long document being prefilled, or drafted tokens to verify) attend over the cache in one
  * call.  seq_lens[b] counts all of sequence b's cached tokens, the chunk's own included
@@ -289,7 +303,6 @@ MLA_API mla_status_t mla_decode(const mla_plan_t* plan, const mla_cache_t* cache
  * (MLA_CACHE_INT4_G32_R128: each query's window depends on its own position).  Otherwise,
  * and with MLA_OPT_DECODE_KERNEL = 1, it returns MLA_ERR_UNSUPPORTED; one mla_decode per
  * query through per-query views of a paged cache covers those shapes. */
-MLA_API size_t mla_decode_chunk_workspace_bytes(const mla_plan_t* plan, int32_t B, int32_t Q);
 MLA_API mla_status_t mla_decode_chunk(const mla_plan_t* plan, const mla_cache_t* cache, const int32_t* seq_lens,
                                       const void* q, int32_t B, int32_t Q, void* out, void* workspace,
                                       size_t ws_bytes, void* stream);
@@ -351,15 +364,17 @@ MLA_API mla_status_t mla_decode_noalloc(const mla_plan_t* plan, const mla_cache_
                                         const int32_t* seq_lens, const void* q, int32_t B, void* out,
                                         void* stream);
 
-/* Synchronise the device, read and clear the plan's device error word.
- * *code receives 0 (none) or a bitwise OR of MLA_DEVERR_* values.
- * Returns MLA_OK, or MLA_ERR_CUDA when the synchronisation itself failed. */
+/* Device error bits (the plan's device error word). */
 enum {
   MLA_DEVERR_SEQ_LEN = 1,     /* a seq_lens entry was < 0 or > T_cap (treated as 0) */
   MLA_DEVERR_APPEND_SLOT = 2, /* an append token had seq_idx/pos out of range (skipped) */
   MLA_DEVERR_TIMEOUT = 4,     /* a pipeline wait exceeded its bound (output invalid) */
   MLA_DEVERR_BLOCK = 8        /* a paged cache's block table named a block outside the pool */
 };
+/* Synchronise the device, read and clear the plan's device error word.
+ * *code receives 0 (none) or a bitwise OR of MLA_DEVERR_* values.
+ * Returns MLA_OK, MLA_ERR_INVALID_ARG for a NULL plan or code, or MLA_ERR_CUDA when the
+ * synchronisation itself failed. */
 MLA_API mla_status_t mla_device_error(mla_plan_t* plan, int32_t* code);
 
 #ifdef __cplusplus

@@ -34,6 +34,25 @@ def test_header_declares_the_boundary():
         assert n in names
 
 
+def test_every_entry_point_has_its_own_doc_comment():
+    """Each MLA_API declaration sits right under a comment block that names it or documents
+    it (argument meaning, layout, ownership, errors)."""
+    lines = open(HEADER).read().splitlines()
+    for i, line in enumerate(lines):
+        m = re.match(r"MLA_API\s+[\w\s\*]+?\b(mla_\w+)\s*\(", line)
+        if not m or line.startswith("#"):
+            continue
+        j = i - 1
+        while j >= 0 and lines[j].strip() == "":
+            j -= 1
+        assert lines[j].rstrip().endswith("*/"), f"{m.group(1)}: no doc comment directly above"
+        k = j
+        while k >= 0 and not lines[k].lstrip().startswith("/*"):
+            k -= 1
+        block = " ".join(lines[k:j + 1])
+        assert len(block) > 60, f"{m.group(1)}: doc comment too short"
+
+
 def test_library_exports_every_declared_symbol(mla):
     so = ctypes.CDLL(mla.LIB_PATH)
     for name in declared_functions():
