@@ -79,14 +79,13 @@ PARITY_WORKLOADS = [
                        ctx_range=None, fixed_lens=(2500, 129, 64, 1), t_cal=512),
     WORKLOADS[4].with_(name="llama_int4_small", hidden=512, batch=3, ctx=None,
                        fixed_lens=(700, 65, 1), t_cal=512),
-    # the int4 cache with the 128-token residual window: on the tensor-core kernel (window
-    # across a tile boundary, a window covering the whole sequence, a single token) and on
-    # the CUDA-core kernel (9 heads)
+    # the int4 cache with the 128-token residual window: a window across a tile boundary, a
+    # window covering the whole sequence, a single token; 32 heads and 9 GQA heads
     WORKLOADS[4].with_(name="llama_int4_r128_small", hidden=512, batch=4, ctx=None,
                        fixed_lens=(700, 200, 128, 1), t_cal=512, resid=128),
     WORKLOADS[1].with_(name="smollm_int4_r128_small", cache="int4_g32", batch=3, ctx=None,
                        fixed_lens=(300, 129, 5), t_cal=512, resid=128),
-    # the 2-bit latent cache (CUDA-core kernel)
+    # the 2-bit latent cache
     WORKLOADS[4].with_(name="llama_int2_small", cache="int2_g32", hidden=512, batch=3, ctx=None,
                        fixed_lens=(700, 65, 1), t_cal=512),
 ]
