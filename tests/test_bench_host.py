@@ -2,6 +2,7 @@
 the gate that keeps a stored DRAM-traffic figure only while the kernel code it was
 measured on is unchanged, and the peak figures' fallbacks."""
 
+import json
 import os
 import shutil
 import stat
@@ -125,3 +126,25 @@ def test_peak_fallbacks(monkeypatch, tmp_path):
     gbs, source = bench.measured_peak_hbm()
     assert gbs == 6551.0 and source.startswith("measured")
     assert bench.measured_peak_tflops() == pytest.approx(1600.5)
+
+
+def test_reference_arm_prints_one_contract_line(capsys, monkeypatch):
+    """The reference arm (the float64 oracle on the host cores) prints exactly one JSON line
+    with the bench contract's keys, its own e2e figure and the CPU-baseline description."""
+    monkeypatch.setenv("RANK", "0")
+    args = type("A", (), {"workload": "tiny_f32", "steps": 3, "warmup": 3, "gpus": 1})()
+    assert bench.run_reference(args) == 0
+    out = capsys.readouterr().out.strip().splitlines()
+    assert len(out) == 1
+    line = json.loads(out[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["steps"] == 3 and line["warmup"] == 3
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT and line["higher_is_better"] is True
+    assert line["value"] > 0 and line["ms_per_step"] > 0 and line["vs_baseline"] is None
+    assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["config"]["workload"] == "tiny_f32"
